@@ -1,0 +1,210 @@
+"""CPU fp64 oracle of the Swimba (Switch Mamba) layer -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import
+this module. The library's compute path never calls it, and it shares no code with that path: it
+is written with numpy in float64, step by step in the order the sources give, with no blocking,
+fusion or reordering.
+
+Sources (cited by title and section; the pages give the method in prose only):
+
+[SW]  "Swimba: Switch Mamba Model Scales State Space Models" (arXiv 2603.06938), summaries at
+      gist.science in Spanish (technical summary §2 "Metodología", "Arquitectura de Swimba"),
+      Dutch ("Methodologie", "Kernmechanisme van Swimba") and French ("2. Méthodologie",
+      "Architecture de Swimba"; "Fondements Théoriques", Théorèmes 1-3).
+[MB]  "Mamba y las SSMs: el retorno del estado persistente" (maquinaoraculo.com), sections
+      "SSMs – Modelos de espacios de estados" (h_t = A h_{t-1} + B x_t, y_t = C h_t + D x_t),
+      "Mamba" (selective SSM, Ā = exp(Δ_t A), Figura 2) and "Estado interno puramente lineal".
+
+What [SW] fixes: a router gives per-token mixing weights π_t over the active experts (top-1 or
+top-k); every expert has its own linear projections that produce token-dependent parameter
+streams; the streams are mixed with π_t in parameter space -- injection Σ_e π_{t,e} B^(e)_t X_t,
+readout (Σ_e π_{t,e} C^(e)_t)ᵀ h_t -- and ONE recurrence runs on a single state h_t.
+
+What this library's layer definition adds where the pages are silent (each reading is listed with
+its reason in the design notes of the repository):
+
+* logits_t = x_t · W_r; idx_t = the k largest, in descending order, ties to the lower index;
+  gates π_t = softmax over the k selected logits (so they sum to 1; top-1 gives exactly 1).
+* expert e maps x_t to [dt_low (R) | B (N) | C (N)] = x_t · W_x^e, and dt^e = dt_low · W_dt^e
+  + b_dt^e; the mixed streams are dt_mix = Σ_j π_j dt^{e_j}, B_mix = Σ_j π_j B^{e_j},
+  C_mix = Σ_j π_j C^{e_j} (X_t is the shared input x_t).
+* Δ_t = softplus(dt_mix); the transition A_t[d, n] = Σ_j π_j A^{e_j}[d, n] (a convex mix of
+  per-expert diagonal A; all experts equal gives the shared A of [SW]); ā = exp(Δ_t A_t)
+  as in [MB] "Mamba"; injection Δ_t · B_mix · x_t (the Euler form, not the ZOH B̄ of [MB]).
+* h_t = ā ⊙ h_{t-1} + Δ_t B_mix x_t from h_{-1} = h0 (zeros when absent);
+  y_t = Σ_n C_mix[n] h_t[·, n] + D_skip ⊙ x_t ([MB] "SSMs" output equation with its D term);
+  out_t = y_t ⊙ SiLU(z_t).
+
+Every function below is pinned by the CPU tests (closed forms, brute force, invariants, special
+cases that reduce to a dense selective scan); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "softplus",
+    "silu",
+    "router_logits",
+    "route",
+    "expert_projections",
+    "selective_scan",
+    "layer_forward",
+    "decode_step",
+]
+
+
+def softplus(v):
+    """softplus(v) = log(1 + e^v), written in the overflow-free form max(v,0) + log1p(e^{-|v|})."""
+    v = np.asarray(v, dtype=np.float64)
+    return np.maximum(v, 0.0) + np.log1p(np.exp(-np.abs(v)))
+
+
+def silu(z):
+    """SiLU(z) = z · σ(z) = z / (1 + e^{-z}) (the gate nonlinearity of the Mamba block, [MB])."""
+    z = np.asarray(z, dtype=np.float64)
+    return z / (1.0 + np.exp(-z))
+
+
+def router_logits(x, W_r):
+    """Router scores: logits[..., e] = Σ_d x[..., d] W_r[d, e]  ([SW]: the router computes π_t)."""
+    return np.asarray(x, dtype=np.float64) @ np.asarray(W_r, dtype=np.float64)
+
+
+def route(x, W_r, k):
+    """Top-k routing ([SW] "Routing": weights π_t for the active experts, top-1 or top-k).
+
+    Returns (idx [..., k] int32, gates [..., k] float64, logits [..., E]). idx lists the k largest
+    logits in descending order; equal logits keep the lower expert index first. gates are the
+    softmax of the selected logits, so each row sums to 1.
+    """
+    logits = router_logits(x, W_r)
+    E = logits.shape[-1]
+    if not 1 <= k <= E:
+        raise ValueError("need 1 <= k <= E")
+    order = np.argsort(-logits, axis=-1, kind="stable")[..., :k]
+    sel = np.take_along_axis(logits, order, axis=-1)
+    w = np.exp(sel - sel[..., :1])
+    gates = w / w.sum(axis=-1, keepdims=True)
+    return order.astype(np.int32), gates, logits
+
+
+def expert_projections(x, idx, gates, W_x, W_dt, b_dt, dt_rank, d_state):
+    """Per-expert parameter streams mixed with the gates ([SW] "Generación de Parámetros" and
+    "Mezcla en el Espacio de Parámetros").
+
+    x [T, D]; idx, gates [T, k]; W_x [E, D, R+2N]; W_dt [E, R, D]; b_dt [E, D] (all fp64 values).
+    For slot j of token t with expert e = idx[t, j]:
+        v = x_t · W_x^e = [dt_low | B^j | C^j];   dt^j = dt_low · W_dt^e + b_dt^e.
+    Returns dict with xdbl [T, k, R+2N], dt_j [T, k, D], dt_mix [T, D], B_mix [T, N], C_mix [T, N].
+    """
+    x = np.asarray(x, dtype=np.float64)
+    T, D = x.shape
+    k = idx.shape[1]
+    E = W_x.shape[0]
+    R, N = dt_rank, d_state
+    xdbl = np.zeros((T, k, R + 2 * N))
+    dt_j = np.zeros((T, k, D))
+    for j in range(k):
+        for e in range(E):
+            rows = np.nonzero(idx[:, j] == e)[0]
+            if rows.size == 0:
+                continue
+            v = x[rows] @ W_x[e]
+            xdbl[rows, j] = v
+            dt_j[rows, j] = v[:, :R] @ W_dt[e] + b_dt[e]
+    g = np.asarray(gates, dtype=np.float64)
+    dt_mix = np.einsum("tj,tjd->td", g, dt_j)
+    B_mix = np.einsum("tj,tjn->tn", g, xdbl[:, :, R:R + N])
+    C_mix = np.einsum("tj,tjn->tn", g, xdbl[:, :, R + N:R + 2 * N])
+    return {"xdbl": xdbl, "dt_j": dt_j, "dt_mix": dt_mix, "B_mix": B_mix, "C_mix": C_mix}
+
+
+def selective_scan(x, z, dt_mix, B_mix, C_mix, idx, gates, A, D_skip, h0=None, channels=None):
+    """The single recurrence over the mixed parameters ([SW] one state trajectory; [MB] "Mamba").
+
+    x, z, dt_mix [B, L, D]; B_mix, C_mix [B, L, N]; idx, gates [B, L, k]; A [E, D, N];
+    D_skip [D]; h0 [B, D, N] or None (zeros). ``channels`` optionally restricts the work to a list
+    of channel indices d; the recurrence of every (b, d, n) is independent, so the restricted
+    result equals the corresponding columns of the full one.
+
+    For t = 0 .. L-1 in order:
+        Δ = softplus(dt_mix[:, t]);  A_t = Σ_j gates_j A^{idx_j};  ā = exp(Δ A_t)
+        h = ā ⊙ h + Δ · B_mix[t] · x[t]
+        y[t] = Σ_n C_mix[t, n] h[·, n] + D_skip ⊙ x[t];   out[t] = y[t] ⊙ SiLU(z[t]).
+    Returns (y, out, h_final, delta) with y, out, delta [B, L, D'] and h_final [B, D', N].
+    """
+    x = np.asarray(x, dtype=np.float64)
+    z = np.asarray(z, dtype=np.float64)
+    dt_mix = np.asarray(dt_mix, dtype=np.float64)
+    A = np.asarray(A, dtype=np.float64)
+    D_skip = np.asarray(D_skip, dtype=np.float64)
+    if channels is not None:
+        ch = np.asarray(channels)
+        x, z, dt_mix = x[:, :, ch], z[:, :, ch], dt_mix[:, :, ch]
+        A, D_skip = A[:, ch, :], D_skip[ch]
+        if h0 is not None:
+            h0 = np.asarray(h0)[:, ch, :]
+    Bsz, L, D = x.shape
+    N = A.shape[2]
+    h = np.zeros((Bsz, D, N)) if h0 is None else np.array(h0, dtype=np.float64)
+    y = np.empty((Bsz, L, D))
+    delta = softplus(dt_mix)
+    g = np.asarray(gates, dtype=np.float64)
+    for t in range(L):
+        d_t = delta[:, t, :]  # [B, D]
+        A_t = np.zeros((Bsz, D, N))
+        for j in range(idx.shape[2]):
+            A_t += g[:, t, j, None, None] * A[idx[:, t, j]]
+        a_bar = np.exp(d_t[:, :, None] * A_t)
+        u = d_t[:, :, None] * B_mix[:, t, None, :] * x[:, t, :, None]
+        h = a_bar * h + u
+        y[:, t, :] = np.einsum("bn,bdn->bd", C_mix[:, t, :], h) + D_skip[None, :] * x[:, t, :]
+    out = y * silu(z)
+    return y, out, h, delta
+
+
+def layer_forward(x, z, W, k, h0=None, channels=None):
+    """The Swimba layer: route -> per-expert projections mixed by the gates -> one scan.
+
+    x, z [B, L, D] fp64 values; W: a mapping with fp64 values W_r [D,E], W_x [E,D,R+2N],
+    W_dt [E,R,D], b_dt [E,D], A [E,D,N], D_skip [D]; h0 [B,D,N] or None. Returns a dict with every
+    intermediate: logits, idx, gates, xdbl, dt_mix, B_mix, C_mix, delta, y, out, h_final.
+    ``channels`` restricts the scan (not the routing or the projections) to some channels.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    Bsz, L, D = x.shape
+    E = W["W_r"].shape[1]
+    N = W["A"].shape[2]
+    R = W["W_dt"].shape[1]
+    idx, gates, logits = route(x.reshape(-1, D), W["W_r"], k)
+    proj = expert_projections(x.reshape(-1, D), idx, gates, W["W_x"], W["W_dt"], W["b_dt"], R, N)
+    shp = lambda a: a.reshape(Bsz, L, *a.shape[1:])
+    idx_b, gates_b = shp(idx), shp(gates)
+    dt_mix, B_mix, C_mix = shp(proj["dt_mix"]), shp(proj["B_mix"]), shp(proj["C_mix"])
+    y, out, h_final, delta = selective_scan(
+        x, z, dt_mix, B_mix, C_mix, idx_b, gates_b, W["A"], W["D_skip"], h0=h0, channels=channels
+    )
+    assert E == W["W_x"].shape[0]
+    return {
+        "logits": shp(logits),
+        "idx": idx_b,
+        "gates": gates_b,
+        "xdbl": shp(proj["xdbl"]),
+        "dt_mix": dt_mix,
+        "B_mix": B_mix,
+        "C_mix": C_mix,
+        "delta": delta,
+        "y": y,
+        "out": out,
+        "h_final": h_final,
+    }
+
+
+def decode_step(h, x_t, z_t, W, k, channels=None):
+    """One recurrent decode step: the layer with L = 1 continuing from the cached state h [B,D,N].
+
+    x_t, z_t [B, 1, D]. Returns (out [B, 1, D'], h_new [B, D', N], full intermediates dict).
+    """
+    r = layer_forward(x_t, z_t, W, k, h0=h, channels=channels)
+    return r["out"], r["h_final"], r

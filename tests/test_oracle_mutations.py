@@ -1,0 +1,91 @@
+"""The oracle's pins catch plausible mistakes: each case plants one mistake in a copy of an
+oracle function (on the CPU, by a textual edit of its source), installs it, and checks that at
+least one pin of ``test_oracle_pins`` fails."""
+import inspect
+import textwrap
+
+import pytest
+
+from oracle import swimba_oracle as O
+import tests.test_oracle_pins as P
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+PINS = [
+    P.test_softplus_special_values_and_library,
+    P.test_silu_identities,
+    lambda: P.test_route_brute_force(5, 3),
+    lambda: P.test_route_brute_force(4, 2),
+    P.test_route_top1_gate_is_exactly_one,
+    P.test_projection_unit_vector_selects_weight_row,
+    P.test_projection_brute_force_loops,
+    P.test_mixing_streams_equals_mixing_weights,
+    P.test_zero_dt_projection_leaves_mixed_bias,
+    P.test_scan_closed_form_constant_inputs_scalar_state,
+    lambda: P.test_scan_brute_force_unrolled_sum(5),
+    P.test_identical_experts_reduce_to_dense_scan,
+    P.test_invariants_and_bibo_bound_under_fast_switching,
+    P.test_skip_path_alone_when_injection_or_readout_is_zero,
+    P.test_free_decay_of_the_initial_state,
+    P.test_chunk_split_and_step_by_step_equal_prefill,
+    P.test_gate_placement_out_is_y_times_silu_z,
+]
+
+MUTATIONS = {
+    "skip term dropped": ("selective_scan", " + D_skip[None, :] * x[:, t, :]", ""),
+    "no delta in injection": ("selective_scan", "u = d_t[:, :, None] * B_mix", "u = 1.0 * B_mix"),
+    "no delta in decay": ("selective_scan", "np.exp(d_t[:, :, None] * A_t)", "np.exp(A_t)"),
+    "injection decayed too": ("selective_scan", "h = a_bar * h + u", "h = a_bar * (h + u)"),
+    "readout before update": (
+        "selective_scan",
+        ["h = a_bar * h + u\n", "+ D_skip[None, :] * x[:, t, :]\n"],
+        ["h_next = a_bar * h + u\n", "+ D_skip[None, :] * x[:, t, :]\n        h = h_next\n"],
+    ),
+    "exp instead of softplus": ("selective_scan", "delta = softplus(dt_mix)", "delta = np.exp(dt_mix)"),
+    "gate z not SiLU": ("selective_scan", "out = y * silu(z)", "out = y * z"),
+    "A mixed without gates": ("selective_scan", "g[:, t, j, None, None] * A[idx", "(1.0 / idx.shape[2]) * A[idx"),
+    "h0 ignored": ("selective_scan", "if h0 is None else np.array(h0, dtype=np.float64)", "if True else None"),
+    "sign of A flipped": ("selective_scan", "np.exp(d_t[:, :, None] * A_t)", "np.exp(-d_t[:, :, None] * A_t)"),
+    "ties to the higher index": (
+        "route",
+        'order = np.argsort(-logits, axis=-1, kind="stable")[..., :k]',
+        'order = (E - 1 - np.argsort(-logits[..., ::-1], axis=-1, kind="stable"))[..., :k]',
+    ),
+    "gates not normalised": ("route", "gates = w / w.sum(axis=-1, keepdims=True)", "gates = w"),
+    "ascending order": ("route", "np.argsort(-logits", "np.argsort(logits"),
+    "dt bias dropped": ("expert_projections", "@ W_dt[e] + b_dt[e]", "@ W_dt[e]"),
+    "B and C swapped": (
+        "expert_projections",
+        'np.einsum("tj,tjn->tn", g, xdbl[:, :, R:R + N])',
+        'np.einsum("tj,tjn->tn", g, xdbl[:, :, R + N:R + 2 * N])',
+    ),
+    "wrong expert table": ("expert_projections", "v = x[rows] @ W_x[e]", "v = x[rows] @ W_x[(e + 1) % E]"),
+    "dt from the wrong columns": ("expert_projections", "v[:, :R] @ W_dt[e]", "v[:, N:N + R] @ W_dt[e]"),
+    "softplus without max(v,0)": ("softplus", "np.maximum(v, 0.0) + ", ""),
+    "silu as sigmoid": ("silu", "return z / (1.0 + np.exp(-z))", "return 1.0 / (1.0 + np.exp(-z))"),
+}
+
+
+def _mutant(fn_name, old, new):
+    src = textwrap.dedent(inspect.getsource(getattr(O, fn_name)))
+    olds, news = (old, new) if isinstance(old, list) else ([old], [new])
+    for o, n in zip(olds, news):
+        assert o in src, f"mutation target not found in {fn_name}: {o!r}"
+        src = src.replace(o, n, 1)
+    ns = dict(vars(O))
+    exec(compile(src, f"<mutant {fn_name}>", "exec"), ns)
+    return ns[fn_name]
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(name, monkeypatch):
+    fn_name, old, new = MUTATIONS[name]
+    monkeypatch.setattr(O, fn_name, _mutant(fn_name, old, new))
+    failed = []
+    for pin in PINS:
+        try:
+            pin()
+        except Exception as exc:  # an assertion, or an error the mistake provokes
+            failed.append(exc)
+            break
+    assert failed, f"no pin fails with the planted mistake: {name}"
