@@ -1,0 +1,155 @@
+// C ABI of libswimba: argument validation, workspace layout and kernel dispatch. The layer's
+// steps run in the kernels of route.cu, proj_simt.cu, proj_tc.cu and scan.cu.
+#include <atomic>
+#include <cstring>
+
+#include "common.cuh"
+#include "proj.cuh"
+#include "scan.cuh"
+
+namespace swimba {
+cudaError_t run_route(const void* x, bool io_bf16, const float* W_r, int32_t* idx, float* gates, int64_t T, int D,
+                      int E, int k, cudaStream_t s);
+cudaError_t run_proj_simt(const ProjParams& p, bool io_bf16, bool w_bf16, cudaStream_t s);
+}  // namespace swimba
+
+namespace swimba {
+static std::atomic<uint64_t> g_launches{0};
+void note_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace swimba
+
+using namespace swimba;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+swimba_status check_dims(const swimba_dims* d) {
+  if (d == nullptr) return SWIMBA_ERR_INVALID_ARG;
+  if (d->batch <= 0 || d->seqlen <= 0 || d->d_inner <= 0 || d->d_state <= 0 || d->dt_rank <= 0 ||
+      d->n_experts <= 0 || d->top_k <= 0)
+    return SWIMBA_ERR_INVALID_ARG;
+  if (d->top_k > d->n_experts) return SWIMBA_ERR_INVALID_ARG;
+  if ((d->io_dtype != SWIMBA_F32 && d->io_dtype != SWIMBA_BF16) ||
+      (d->w_dtype != SWIMBA_F32 && d->w_dtype != SWIMBA_BF16))
+    return SWIMBA_ERR_INVALID_ARG;
+  if (d->n_experts > 16 || d->d_state > 16 || d->dt_rank > 256 || (d->d_inner % 8) != 0)
+    return SWIMBA_ERR_UNSUPPORTED;
+  if (d->batch > (1 << 30) || d->seqlen > (int64_t(1) << 40) || d->batch * d->seqlen > (int64_t(1) << 31))
+    return SWIMBA_ERR_UNSUPPORTED;
+  if ((int64_t)d->batch * d->seqlen * d->d_inner > (int64_t(1) << 40)) return SWIMBA_ERR_UNSUPPORTED;
+  return SWIMBA_OK;
+}
+
+swimba_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SWIMBA_OK : SWIMBA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t swimba_workspace_size(const swimba_dims* dims, int op) {
+  if (check_dims(dims) != SWIMBA_OK) return 0;
+  switch (op) {
+    case SWIMBA_OP_ROUTE:
+    case SWIMBA_OP_PROJ:
+    case SWIMBA_OP_SCAN:
+    case SWIMBA_OP_STEP:
+    case SWIMBA_OP_LAYER:
+      return kStatusBytes;
+    default:
+      return 0;
+  }
+}
+
+swimba_status swimba_route(const swimba_dims* dims, const void* x, const float* W_r, int32_t* idx, float* gates,
+                           void* stream) {
+  swimba_status st = check_dims(dims);
+  if (st != SWIMBA_OK) return st;
+  if (!x || !W_r || !idx || !gates) return SWIMBA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(W_r)) return SWIMBA_ERR_ALIGN;
+  const int64_t T = dims->batch * dims->seqlen;
+  return cuda_status(run_route(x, dims->io_dtype == SWIMBA_BF16, W_r, idx, gates, T, dims->d_inner, dims->n_experts,
+                               dims->top_k, static_cast<cudaStream_t>(stream)));
+}
+
+swimba_status swimba_mixed_proj(const swimba_dims* dims, const void* x, const int32_t* idx, const float* gates,
+                                const swimba_weights* w, float* delta, float* B_mix, float* C_mix, void* ws,
+                                size_t ws_bytes, void* stream) {
+  swimba_status st = check_dims(dims);
+  if (st != SWIMBA_OK) return st;
+  if (!x || !idx || !gates || !w || !w->W_x || !w->W_dt || !w->b_dt || !delta || !B_mix || !C_mix)
+    return SWIMBA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(delta) || !aligned16(w->W_x) || !aligned16(w->W_dt)) return SWIMBA_ERR_ALIGN;
+  if (ws == nullptr || ws_bytes < swimba_workspace_size(dims, SWIMBA_OP_PROJ)) return SWIMBA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SWIMBA_ERR_ALIGN;
+  ProjParams p{x,     idx,   gates, w->W_x,       w->W_dt,        w->b_dt,         delta,
+               B_mix, C_mix, dims->batch * dims->seqlen, dims->d_inner, dims->d_state, dims->dt_rank,
+               dims->n_experts, dims->top_k};
+  return cuda_status(run_proj_simt(p, dims->io_dtype == SWIMBA_BF16, dims->w_dtype == SWIMBA_BF16,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+static swimba_status scan_common(const swimba_dims* dims, const void* x, const void* z, const float* delta,
+                                 const float* B_mix, const float* C_mix, const int32_t* idx, const float* gates,
+                                 const swimba_weights* w, const float* h0, void* out, float* h_final, float* y_pre,
+                                 bool step, void* stream) {
+  if (!x || !z || !delta || !B_mix || !C_mix || !idx || !gates || !w || !w->A || !w->D_skip || !out)
+    return SWIMBA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(z) || !aligned16(out) || !aligned16(delta)) return SWIMBA_ERR_ALIGN;
+  if (dims->d_state == 16 && (!aligned16(B_mix) || !aligned16(C_mix))) return SWIMBA_ERR_ALIGN;
+  if ((h0 && !aligned16(h0)) || (h_final && !aligned16(h_final))) return SWIMBA_ERR_ALIGN;
+  ScanParams p{x,   z,       delta, B_mix,          C_mix,          idx,           gates,
+               w->A, w->D_skip, h0,  out,            h_final,        y_pre,         dims->seqlen,
+               (int)dims->batch, dims->d_inner, dims->d_state, dims->n_experts, dims->top_k};
+  return cuda_status(run_scan(p, dims->io_dtype == SWIMBA_BF16, step, static_cast<cudaStream_t>(stream)));
+}
+
+swimba_status swimba_scan_fwd(const swimba_dims* dims, const void* x, const void* z, const float* delta,
+                              const float* B_mix, const float* C_mix, const int32_t* idx, const float* gates,
+                              const swimba_weights* w, const float* h0, void* out, float* h_final, float* y_pre,
+                              void* ws, size_t ws_bytes, void* stream) {
+  swimba_status st = check_dims(dims);
+  if (st != SWIMBA_OK) return st;
+  if (ws == nullptr || ws_bytes < swimba_workspace_size(dims, SWIMBA_OP_SCAN)) return SWIMBA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SWIMBA_ERR_ALIGN;
+  return scan_common(dims, x, z, delta, B_mix, C_mix, idx, gates, w, h0, out, h_final, y_pre, false, stream);
+}
+
+swimba_status swimba_step(const swimba_dims* dims, const void* x, const void* z, const float* delta,
+                          const float* B_mix, const float* C_mix, const int32_t* idx, const float* gates,
+                          const swimba_weights* w, float* h, void* out, void* stream) {
+  swimba_status st = check_dims(dims);
+  if (st != SWIMBA_OK) return st;
+  if (dims->seqlen != 1 || h == nullptr) return SWIMBA_ERR_INVALID_ARG;
+  return scan_common(dims, x, z, delta, B_mix, C_mix, idx, gates, w, h, out, h, nullptr, true, stream);
+}
+
+swimba_status swimba_get_device_status(void* ws, void* stream) {
+  if (ws == nullptr) return SWIMBA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SWIMBA_ERR_CUDA;
+  DeviceStatus host{};
+  if (cudaMemcpy(&host, ws, sizeof(host), cudaMemcpyDeviceToHost) != cudaSuccess) return SWIMBA_ERR_CUDA;
+  if (host.code != 0) {
+    if (cudaMemset(ws, 0, sizeof(DeviceStatus)) != cudaSuccess) return SWIMBA_ERR_CUDA;
+    return static_cast<swimba_status>(host.code);
+  }
+  return SWIMBA_OK;
+}
+
+uint64_t swimba_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* swimba_status_string(swimba_status s) {
+  switch (s) {
+    case SWIMBA_OK: return "ok";
+    case SWIMBA_ERR_INVALID_ARG: return "invalid argument";
+    case SWIMBA_ERR_UNSUPPORTED: return "unsupported shape";
+    case SWIMBA_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case SWIMBA_ERR_WORKSPACE: return "workspace missing or too small";
+    case SWIMBA_ERR_CUDA: return "CUDA runtime error";
+    case SWIMBA_ERR_TIMEOUT: return "bounded device wait gave up";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

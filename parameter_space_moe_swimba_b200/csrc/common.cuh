@@ -1,0 +1,74 @@
+// Shared device helpers of libswimba (sm_100a). No step of the layer lives here: only dtype
+// conversion, the exp2 instruction wrapper and the device status block.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "swimba.h"
+
+namespace swimba {
+
+// The first bytes of every workspace: device-side error reporting (bounded waits that gave up).
+constexpr size_t kStatusBytes = 256;
+struct DeviceStatus {
+  int code;   // 0 or a swimba_status
+  int where;  // kernel-specific location code of the first error
+  int info0;  // kernel-specific detail (e.g. CTA index)
+  int info1;
+};
+
+__device__ __forceinline__ void record_device_error(void* ws, int code, int where, int info0, int info1) {
+  if (ws == nullptr) return;
+  DeviceStatus* s = reinterpret_cast<DeviceStatus*>(ws);
+  if (atomicCAS(&s->code, 0, code) == 0) {
+    s->where = where;
+    s->info0 = info0;
+    s->info1 = info1;
+  }
+}
+
+// Counts every kernel launch of the library (read through swimba_kernel_launches).
+void note_launch(int n = 1);
+
+constexpr float kLog2e = 1.4426950408889634f;  // log2(e)
+
+// 2^x with the MUFU ex2 instruction (flush-to-zero; relative error about 2^-22).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ---- io dtype access -----------------------------------------------------------------------
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ void from_f32(float& dst, float v) { dst = v; }
+__device__ __forceinline__ void from_f32(__nv_bfloat16& dst, float v) { dst = __float2bfloat16_rn(v); }
+
+// Low / high bf16 of a packed 32-bit word, widened exactly.
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Unpack 16 bytes of io values into floats: 8 bf16 or 4 fp32.
+template <typename IO>
+struct Vec16;
+template <>
+struct Vec16<__nv_bfloat16> {
+  static constexpr int n = 8;
+  __device__ __forceinline__ static void unpack(const uint4& v, float* f) {
+    f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+    f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+  }
+};
+template <>
+struct Vec16<float> {
+  static constexpr int n = 4;
+  __device__ __forceinline__ static void unpack(const uint4& v, float* f) {
+    f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+  }
+};
+
+}  // namespace swimba

@@ -1,0 +1,231 @@
+// Fused discretise + selective scan + readout + skip + SiLU gate, and the decode step.
+//
+// Sources: "Swimba: Switch Mamba Model Scales State Space Models" -- one state trajectory and one
+// recurrence whatever the number of experts (§2 "Resultado", Teorema 2); the injection and the
+// readout use the gate-mixed streams. "Mamba y las SSMs: el retorno del estado persistente",
+// "Mamba": selective SSM with Ā = exp(Δ_t A); Figura 2: the state stays on chip while inputs
+// stream from HBM; "Estado interno puramente lineal": the linear state admits a scan.
+//
+// Per token t and channel d (Δ = delta[t, d] already holds softplus(dt_mix)):
+//   A_t[d, n] = Σ_j g_j A^{e_j}[d, n]          (per-expert A tables of this CTA's channels in smem)
+//   h[d, n]  = exp(Δ A_t[d, n]) h[d, n] + Δ B_mix[t, n] x[t, d]
+//   y[t, d]  = Σ_n C_mix[t, n] h[d, n] + D_skip[d] x[t, d];   out = y z σ(z)
+//
+// Thread layout: a CTA owns 32 channels of one sequence; 4 lanes share a channel and hold 4 of
+// its 16 fp32 states each, in registers, for the whole sequence. All lanes of a warp read the
+// same token, so the expert indices are warp-uniform. exp is evaluated as 2^(Δ g_j log2(e) A).
+#include "common.cuh"
+#include "scan.cuh"
+
+namespace swimba {
+
+namespace {
+constexpr int kNS = 4;   // states per thread
+constexpr int kG = 4;    // threads per channel (16 states / kNS)
+constexpr int kDT = 32;  // channels per CTA
+constexpr int kNMax = 16;
+
+__device__ __forceinline__ float silu_gate(float y, float z) { return y * z * (1.f / (1.f + __expf(-z))); }
+
+__device__ __forceinline__ void fill_A_table(float* As, const ScanParams& p, int d0) {
+  const int total = p.E * kDT * kNMax;
+  for (int i = threadIdx.x; i < total; i += blockDim.x) {
+    const int e = i / (kDT * kNMax);
+    const int r = i - e * (kDT * kNMax);
+    const int dd = d0 + r / kNMax;
+    const int n = r % kNMax;
+    As[i] = (dd < p.D && n < p.N) ? __ldg(p.A + ((size_t)e * p.D + dd) * p.N + n) : 0.f;
+  }
+}
+
+// One token of the recurrence for the 4 states (n0 .. n0+3) of channel d held by this thread.
+// Returns the partial readout Σ_{n in thread} C[n] h[n].
+template <int K>
+__device__ __forceinline__ float token_update(float (&h)[kNS], const float* As, int dl, int n0, float dlt, float xv,
+                                              const float (&Bv)[kNS], const float (&Cv)[kNS],
+                                              const int32_t* idx_t, const float* g_t, int k, int E) {
+  float arg[kNS] = {0.f, 0.f, 0.f, 0.f};
+  const int kk = K > 0 ? K : k;
+#pragma unroll
+  for (int j = 0; j < (K > 0 ? K : 16); ++j) {
+    if (K == 0 && j >= kk) break;
+    const int e = min(max(__ldg(idx_t + j), 0), E - 1);  // indices outside [0, E) are clamped
+    const float c = dlt * __ldg(g_t + j) * kLog2e;
+    const float4 a4 = *reinterpret_cast<const float4*>(As + (e * kDT + dl) * kNMax + n0);
+    arg[0] = fmaf(c, a4.x, arg[0]);
+    arg[1] = fmaf(c, a4.y, arg[1]);
+    arg[2] = fmaf(c, a4.z, arg[2]);
+    arg[3] = fmaf(c, a4.w, arg[3]);
+  }
+  const float dx = dlt * xv;
+  float y = 0.f;
+#pragma unroll
+  for (int s = 0; s < kNS; ++s) {
+    const float a = ex2_approx(arg[s]);
+    h[s] = fmaf(a, h[s], dx * Bv[s]);
+    y = fmaf(Cv[s], h[s], y);
+  }
+  return y;
+}
+
+__device__ __forceinline__ void load_bc(const ScanParams& p, size_t tok, int n0, float (&Bv)[kNS], float (&Cv)[kNS]) {
+  if (p.N == kNMax) {
+    const float4 b4 = __ldg(reinterpret_cast<const float4*>(p.B_mix + tok * kNMax + n0));
+    const float4 c4 = __ldg(reinterpret_cast<const float4*>(p.C_mix + tok * kNMax + n0));
+    Bv[0] = b4.x; Bv[1] = b4.y; Bv[2] = b4.z; Bv[3] = b4.w;
+    Cv[0] = c4.x; Cv[1] = c4.y; Cv[2] = c4.z; Cv[3] = c4.w;
+  } else {
+#pragma unroll
+    for (int s = 0; s < kNS; ++s) {
+      const int n = n0 + s;
+      Bv[s] = n < p.N ? __ldg(p.B_mix + tok * p.N + n) : 0.f;
+      Cv[s] = n < p.N ? __ldg(p.C_mix + tok * p.N + n) : 0.f;
+    }
+  }
+}
+}  // namespace
+
+template <typename IO, int K>
+__global__ void __launch_bounds__(128) scan_fwd_kernel(ScanParams p) {
+  extern __shared__ float As[];  // [E][kDT][16]
+  const int tid = threadIdx.x;
+  const int dl = tid / kG, gi = tid % kG;
+  const int d0 = blockIdx.x * kDT;
+  const int d = d0 + dl;
+  const int b = blockIdx.y;
+  const int n0 = gi * kNS;
+  const bool dvalid = d < p.D;
+  const int dc = dvalid ? d : 0;  // clamped channel for loads
+  fill_A_table(As, p, d0);
+  __syncthreads();
+
+  float h[kNS];
+#pragma unroll
+  for (int s = 0; s < kNS; ++s)
+    h[s] = (p.h0 != nullptr && dvalid && n0 + s < p.N) ? p.h0[((size_t)b * p.D + d) * p.N + n0 + s] : 0.f;
+  const float dsk = p.D_skip[dc];
+  const IO* x = reinterpret_cast<const IO*>(p.x);
+  const IO* z = reinterpret_cast<const IO*>(p.z);
+  IO* out = reinterpret_cast<IO*>(p.out);
+
+#pragma unroll 2
+  for (int64_t t = 0; t < p.L; ++t) {
+    const size_t tok = (size_t)b * p.L + t;
+    const float dlt = __ldg(p.delta + tok * p.D + dc);
+    const float xv = to_f32(x[tok * p.D + dc]);
+    const float zv = to_f32(z[tok * p.D + dc]);
+    float Bv[kNS], Cv[kNS];
+    load_bc(p, tok, n0, Bv, Cv);
+    float y = token_update<K>(h, As, dl, n0, dlt, xv, Bv, Cv, p.idx + tok * p.k, p.gates + tok * p.k, p.k, p.E);
+    y += __shfl_xor_sync(0xffffffffu, y, 1);
+    y += __shfl_xor_sync(0xffffffffu, y, 2);
+    if (gi == 0 && dvalid) {
+      y = fmaf(dsk, xv, y);
+      if (p.y_pre != nullptr) p.y_pre[tok * p.D + d] = y;
+      from_f32(out[tok * p.D + d], silu_gate(y, zv));
+    }
+  }
+  if (p.h_final != nullptr && dvalid) {
+#pragma unroll
+    for (int s = 0; s < kNS; ++s)
+      if (n0 + s < p.N) p.h_final[((size_t)b * p.D + d) * p.N + n0 + s] = h[s];
+  }
+}
+
+// Decode step: one token per sequence, state read from and written back to p.h_final (= p.h0).
+// A CTA owns 32 channels and kStepRows sequences, so its A tables are loaded once for them.
+constexpr int kStepRows = 16;
+
+template <typename IO, int K>
+__global__ void __launch_bounds__(128) step_kernel(ScanParams p) {
+  extern __shared__ float As[];
+  const int tid = threadIdx.x;
+  const int dl = tid / kG, gi = tid % kG;
+  const int d0 = blockIdx.x * kDT;
+  const int d = d0 + dl;
+  const int n0 = gi * kNS;
+  const bool dvalid = d < p.D;
+  const int dc = dvalid ? d : 0;
+  fill_A_table(As, p, d0);
+  __syncthreads();
+  const float dsk = p.D_skip[dc];
+  const IO* x = reinterpret_cast<const IO*>(p.x);
+  const IO* z = reinterpret_cast<const IO*>(p.z);
+  IO* out = reinterpret_cast<IO*>(p.out);
+  const int b_end = min(p.B, (int)(blockIdx.y + 1) * kStepRows);
+#pragma unroll 2
+  for (int b = blockIdx.y * kStepRows; b < b_end; ++b) {
+    const size_t tok = (size_t)b;  // seqlen == 1
+    float* hp = p.h_final + ((size_t)b * p.D + dc) * p.N + n0;
+    float h[kNS];
+    if (p.N == kNMax) {
+      const float4 h4 = *reinterpret_cast<const float4*>(hp);
+      h[0] = h4.x; h[1] = h4.y; h[2] = h4.z; h[3] = h4.w;
+    } else {
+#pragma unroll
+      for (int s = 0; s < kNS; ++s) h[s] = (n0 + s < p.N) ? hp[s] : 0.f;
+    }
+    const float dlt = __ldg(p.delta + tok * p.D + dc);
+    const float xv = to_f32(x[tok * p.D + dc]);
+    const float zv = to_f32(z[tok * p.D + dc]);
+    float Bv[kNS], Cv[kNS];
+    load_bc(p, tok, n0, Bv, Cv);
+    float y = token_update<K>(h, As, dl, n0, dlt, xv, Bv, Cv, p.idx + tok * p.k, p.gates + tok * p.k, p.k, p.E);
+    y += __shfl_xor_sync(0xffffffffu, y, 1);
+    y += __shfl_xor_sync(0xffffffffu, y, 2);
+    if (dvalid) {
+      if (p.N == kNMax) {
+        *reinterpret_cast<float4*>(hp) = make_float4(h[0], h[1], h[2], h[3]);
+      } else {
+#pragma unroll
+        for (int s = 0; s < kNS; ++s)
+          if (n0 + s < p.N) hp[s] = h[s];
+      }
+      if (gi == 0) {
+        y = fmaf(dsk, xv, y);
+        if (p.y_pre != nullptr) p.y_pre[tok * p.D + d] = y;
+        from_f32(out[tok * p.D + d], silu_gate(y, zv));
+      }
+    }
+  }
+}
+
+template <typename IO, int K>
+static cudaError_t launch_scan(const ScanParams& p, bool step, cudaStream_t s) {
+  const size_t smem = sizeof(float) * (size_t)p.E * kDT * kNMax;
+  const unsigned gx = (unsigned)((p.D + kDT - 1) / kDT);
+  if (step) {
+    if (smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(step_kernel<IO, K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    dim3 grid(gx, (unsigned)((p.B + kStepRows - 1) / kStepRows));
+    step_kernel<IO, K><<<grid, 128, smem, s>>>(p);
+    note_launch();
+  } else {
+    if (smem > 48 * 1024) {
+      cudaError_t e =
+          cudaFuncSetAttribute(scan_fwd_kernel<IO, K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    dim3 grid(gx, (unsigned)p.B);
+    scan_fwd_kernel<IO, K><<<grid, 128, smem, s>>>(p);
+    note_launch();
+  }
+  return cudaGetLastError();
+}
+
+template <typename IO>
+static cudaError_t scan_dispatch(const ScanParams& p, bool step, cudaStream_t s) {
+  switch (p.k) {
+    case 1: return launch_scan<IO, 1>(p, step, s);
+    case 2: return launch_scan<IO, 2>(p, step, s);
+    default: return launch_scan<IO, 0>(p, step, s);
+  }
+}
+
+cudaError_t run_scan(const ScanParams& p, bool io_bf16, bool step, cudaStream_t s) {
+  return io_bf16 ? scan_dispatch<__nv_bfloat16>(p, step, s) : scan_dispatch<float>(p, step, s);
+}
+
+}  // namespace swimba

@@ -1,0 +1,28 @@
+// Parameters of the scan and decode-step kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace swimba {
+
+struct ScanParams {
+  const void* x;         // [B, L, D] io
+  const void* z;         // [B, L, D] io
+  const float* delta;    // [B, L, D]  softplus(dt_mix)
+  const float* B_mix;    // [B, L, N]
+  const float* C_mix;    // [B, L, N]
+  const int32_t* idx;    // [B, L, k]
+  const float* gates;    // [B, L, k]
+  const float* A;        // [E, D, N]
+  const float* D_skip;   // [D]
+  const float* h0;       // [B, D, N] or null
+  void* out;             // [B, L, D] io
+  float* h_final;        // [B, D, N] or null
+  float* y_pre;          // [B, L, D] or null
+  int64_t L;
+  int B, D, N, E, k;
+};
+
+cudaError_t run_scan(const ScanParams& p, bool io_bf16, bool step, cudaStream_t s);
+
+}  // namespace swimba

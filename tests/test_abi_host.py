@@ -1,0 +1,82 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every function
+include/swimba.h declares, sizes workspaces, and rejects bad arguments before any launch."""
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def S():
+    from parameter_space_moe_swimba_b200 import build
+
+    build.build()
+    from parameter_space_moe_swimba_b200 import swimba
+
+    return swimba
+
+
+def declared_functions():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(swimba_\w+)\s*\(", src))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_function(S):
+    names = declared_functions()
+    assert len(names) >= 7
+    for n in names:
+        assert hasattr(S._lib, n), n
+    assert set(names) == set(S.EXPORTED)
+
+
+def test_status_strings(S):
+    assert S.swimba_status_string(0) == "ok"
+    for code in range(1, 7):
+        assert S.swimba_status_string(code) not in ("ok", "unknown status")
+    assert S.swimba_status_string(99) == "unknown status"
+
+
+def test_workspace_sizes(S):
+    from parameter_space_moe_swimba_b200.configs import CONFIGS
+
+    for cfg in CONFIGS.values():
+        dims = S.make_dims(cfg, seqlen=1 if cfg.decode_steps else None)
+        for op in range(5):
+            assert S.swimba_workspace_size(dims, op) >= 256
+        assert S.swimba_workspace_size(dims, 4) == max(S.swimba_workspace_size(dims, op) for op in range(4))
+    bad = S.make_dims(CONFIGS["tiny_fp32"], top_k=9)
+    assert S.swimba_workspace_size(bad, 4) == 0
+
+
+def test_invalid_arguments_return_before_any_launch(S):
+    from parameter_space_moe_swimba_b200.configs import CONFIGS
+
+    cfg = CONFIGS["tiny_fp32"]
+    dims = S.make_dims(cfg)
+    fake = 1 << 40  # never dereferenced: every case fails validation first
+    w = S.swimba_weights(fake, fake, fake, fake, fake, fake)
+    assert S.swimba_route(dims, None, fake, fake, fake, 0) == 1
+    assert S.swimba_route(S.make_dims(cfg, top_k=5), fake, fake, fake, fake, 0) == 1
+    assert S.swimba_route(S.make_dims(cfg, n_experts=17, top_k=2), fake, fake, fake, fake, 0) == 2
+    assert S.swimba_route(dims, fake + 8, fake, fake, fake, 0) == 3
+    odd = S.make_dims(cfg)
+    odd.d_inner = 12
+    assert S.swimba_route(odd, fake, fake, fake, fake, 0) == 2
+    big_n = S.make_dims(cfg)
+    big_n.d_state = 17
+    assert S.swimba_scan_fwd(big_n, fake, fake, fake, fake, fake, fake, fake, w, None, fake, None, None, fake,
+                             1 << 20, 0) == 2
+    assert S.swimba_mixed_proj(dims, fake, fake, fake, w, fake, fake, fake, fake, 8, 0) == 4
+    assert S.swimba_mixed_proj(dims, fake, fake, fake, w, fake, fake, fake, None, 1 << 20, 0) == 4
+    assert S.swimba_scan_fwd(dims, fake, fake, fake, fake, fake, fake, fake, w, None, None, None, None, fake,
+                             1 << 20, 0) == 1
+    step_dims = S.make_dims(cfg)  # seqlen 128: a decode step needs seqlen 1
+    assert S.swimba_step(step_dims, fake, fake, fake, fake, fake, fake, fake, w, fake, fake, 0) == 1
+    assert S.swimba_get_device_status(None, 0) == 1
