@@ -11,6 +11,9 @@ namespace swimba {
 cudaError_t run_route(const void* x, bool io_bf16, const float* W_r, int32_t* idx, float* gates, int64_t T, int D,
                       int E, int k, cudaStream_t s);
 cudaError_t run_proj_simt(const ProjParams& p, bool io_bf16, bool w_bf16, cudaStream_t s);
+bool proj_tc_supported(const ProjParams& p, bool io_bf16, bool w_bf16);
+size_t proj_tc_workspace(int64_t T, int E, int k, int R);
+cudaError_t run_proj_tc(const ProjParams& p, void* ws, cudaStream_t s);
 }  // namespace swimba
 
 namespace swimba {
@@ -43,6 +46,26 @@ swimba_status check_dims(const swimba_dims* d) {
 
 swimba_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SWIMBA_OK : SWIMBA_ERR_CUDA; }
 
+// Shape-only projection parameters (pointers unset), used to pick the path and size workspaces.
+ProjParams proj_shape(const swimba_dims* d) {
+  ProjParams p{};
+  p.T = d->batch * d->seqlen;
+  p.D = d->d_inner;
+  p.N = d->d_state;
+  p.R = d->dt_rank;
+  p.E = d->n_experts;
+  p.k = d->top_k;
+  return p;
+}
+
+bool use_tc(const swimba_dims* d) {
+  return proj_tc_supported(proj_shape(d), d->io_dtype == SWIMBA_BF16, d->w_dtype == SWIMBA_BF16);
+}
+
+size_t proj_workspace(const swimba_dims* d) {
+  return use_tc(d) ? proj_tc_workspace(d->batch * d->seqlen, d->n_experts, d->top_k, d->dt_rank) : kStatusBytes;
+}
+
 }  // namespace
 
 extern "C" {
@@ -51,11 +74,12 @@ size_t swimba_workspace_size(const swimba_dims* dims, int op) {
   if (check_dims(dims) != SWIMBA_OK) return 0;
   switch (op) {
     case SWIMBA_OP_ROUTE:
-    case SWIMBA_OP_PROJ:
     case SWIMBA_OP_SCAN:
     case SWIMBA_OP_STEP:
-    case SWIMBA_OP_LAYER:
       return kStatusBytes;
+    case SWIMBA_OP_PROJ:
+    case SWIMBA_OP_LAYER:
+      return proj_workspace(dims);
     default:
       return 0;
   }
@@ -85,6 +109,10 @@ swimba_status swimba_mixed_proj(const swimba_dims* dims, const void* x, const in
   ProjParams p{x,     idx,   gates, w->W_x,       w->W_dt,        w->b_dt,         delta,
                B_mix, C_mix, dims->batch * dims->seqlen, dims->d_inner, dims->d_state, dims->dt_rank,
                dims->n_experts, dims->top_k};
+  if (use_tc(dims)) {
+    if (!aligned16(w->b_dt) || !aligned16(B_mix) || !aligned16(C_mix)) return SWIMBA_ERR_ALIGN;
+    return cuda_status(run_proj_tc(p, ws, static_cast<cudaStream_t>(stream)));
+  }
   return cuda_status(run_proj_simt(p, dims->io_dtype == SWIMBA_BF16, dims->w_dtype == SWIMBA_BF16,
                                    static_cast<cudaStream_t>(stream)));
 }

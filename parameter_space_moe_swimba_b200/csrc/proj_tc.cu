@@ -1,1 +1,799 @@
-// placeholder
+// Mixed expert projection on the tcgen05 tensor cores (bf16 x and tables, fp32 accumulation).
+//
+// Source: "Swimba: Switch Mamba Model Scales State Space Models", §2 "Generación de Parámetros" /
+// "Mezcla en el Espacio de Parámetros" (es), "Kernmechanisme van Swimba" (nl): every expert has
+// its own linear projections producing token-dependent streams, and the streams of the active
+// experts are mixed with the router weights before the single recurrence. The pages attribute
+// Swimba's serving overhead to routing and to this "dispersion" of tokens over experts.
+//
+// Design. Tokens are bucketed by the SET of experts they selected (k <= 2: an expert, or an
+// unordered expert pair), so every 128-row tile shares its k weight tables and x is read once:
+//   bucket kernels  group id per token, histogram, offsets + tile list, scatter of token ids.
+//   stage 1         per tile: acc_j = X_tile · W_x^{e_j}  (j < k; TMEM, M=128, N=R+2N, K=D).
+//                   x rows are gathered by TMA (tile::gather4, 64-byte swizzle); W_x boxes are
+//                   MN-major 128-byte-swizzled tiles of the [E, D, R+2N] table as stored.
+//                   Epilogue: B_mix, C_mix = Σ_j g_j (B^j, C^j) -> global; the gated low-rank
+//                   rows  A'[row] = [g_0 dt_low^0 | g_1 dt_low^1]  (bf16) -> workspace.
+//   stage 2         per (tile, 256-column chunk): acc = A'_tile · [W_dt^{e_0}; W_dt^{e_1}]
+//                   (K = k·R), i.e. Σ_j g_j dt_low^j W_dt^{e_j} in one accumulation. Epilogue:
+//                   + Σ_j g_j b_dt^{e_j}, softplus, store delta rows of the tile's tokens.
+// Both GEMM kernels are persistent and warp specialised: warp 0 issues TMA, warp 1 owns TMEM and
+// issues the MMAs, the remaining warps drain TMEM. Every mbarrier wait is bounded (1 s); on a
+// timeout the CTA records SWIMBA_ERR_TIMEOUT in the workspace status block, lets its copies in
+// flight land, frees TMEM and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "proj.cuh"
+#include "sm100.cuh"
+
+namespace swimba {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int BM = 128;        // rows (token slots) per tile
+constexpr int BK1 = 32;        // stage-1 K slice per ring stage (64 bytes of bf16 per row)
+constexpr int kStages1 = 6;
+constexpr int kSlot1 = 32768;  // A 8 KB + up to 6 W_x boxes of 4 KB
+constexpr int NC = 256;        // stage-2 output columns per chunk
+constexpr int kStages2 = 4;
+constexpr int kSlot2 = 32768;  // 4 W_dt boxes of up to 64 rows x 128 B
+constexpr int kApBox = BM * 128;  // one 64-column box of A' (16 KB)
+
+struct TileInfo {
+  int row_begin, rows, e0, e1;
+};
+
+struct TcLayout {
+  size_t group_of, counts, cursor, offsets, num_tiles, tiles, slot_tok, slot_gate, aprime, total;
+  int G, max_tiles, K2, R_pad;
+};
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+TcLayout tc_layout(int64_t T, int E, int K, int R) {
+  TcLayout L{};
+  L.G = K == 1 ? E : E * (E - 1) / 2;
+  L.max_tiles = (int)((T + BM - 1) / BM) + L.G;
+  L.R_pad = (R + 63) / 64 * 64;
+  L.K2 = K * L.R_pad;
+  size_t o = kStatusBytes;
+  L.group_of = o; o = align_up(o + 4 * (size_t)T, 256);
+  L.counts = o; o += 4 * (size_t)L.G;
+  L.cursor = o; o = align_up(o + 4 * (size_t)L.G, 256);
+  L.offsets = o; o = align_up(o + 4 * (size_t)(L.G + 1), 256);
+  L.num_tiles = o; o += 256;
+  L.tiles = o; o = align_up(o + sizeof(TileInfo) * (size_t)L.max_tiles, 256);
+  L.slot_tok = o; o = align_up(o + 4 * (size_t)T, 256);
+  L.slot_gate = o; o = align_up(o + 4 * (size_t)T * K, 1024);
+  L.aprime = o; o += 2 * (size_t)L.max_tiles * BM * L.K2;
+  L.total = align_up(o, 256);
+  return L;
+}
+
+__device__ __forceinline__ int clamp_e(int e, int E) { return min(max(e, 0), E - 1); }
+
+// ---- bucketing -----------------------------------------------------------------------------------
+// Group id of a sorted expert set: k = 1 -> e; k = 2 (a < b) -> a + b(b-1)/2.
+template <int K>
+__global__ void group_count_kernel(const int32_t* idx, int64_t T, int E, int* group_of, int* counts) {
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  int g;
+  if (K == 1) {
+    g = clamp_e(idx[t], E);
+  } else {
+    const int e0 = clamp_e(idx[2 * t], E), e1 = clamp_e(idx[2 * t + 1], E);
+    const int a = min(e0, e1), b = max(e0, e1);
+    g = a + b * (b - 1) / 2;
+  }
+  group_of[t] = g;
+  atomicAdd(&counts[g], 1);
+}
+
+template <int K>
+__global__ void group_scan_kernel(const int* counts, int G, int* offsets, int* num_tiles, TileInfo* tiles) {
+  __shared__ int s_off[160];
+  __shared__ int s_tstart[160];
+  if (threadIdx.x == 0) {
+    int off = 0, nt = 0;
+    for (int g = 0; g < G; ++g) {
+      s_off[g] = off;
+      s_tstart[g] = nt;
+      offsets[g] = off;
+      off += counts[g];
+      nt += (counts[g] + BM - 1) / BM;
+    }
+    s_off[G] = off;
+    s_tstart[G] = nt;
+    offsets[G] = off;
+    *num_tiles = nt;
+  }
+  __syncthreads();
+  const int nt = s_tstart[G];
+  for (int tile = threadIdx.x; tile < nt; tile += blockDim.x) {
+    int lo = 0, hi = G - 1;  // last g with s_tstart[g] <= tile
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) / 2;
+      if (s_tstart[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    const int g = lo;
+    const int i = tile - s_tstart[g];
+    TileInfo ti;
+    ti.row_begin = s_off[g] + i * BM;
+    ti.rows = min(BM, counts[g] - i * BM);
+    if (K == 1) {
+      ti.e0 = g;
+      ti.e1 = g;
+    } else {
+      int b = 1;
+      while ((b + 1) * b / 2 <= g) ++b;
+      ti.e1 = b;
+      ti.e0 = g - b * (b - 1) / 2;
+    }
+    tiles[tile] = ti;
+  }
+}
+
+template <int K>
+__global__ void group_scatter_kernel(const int32_t* idx, const float* gates, int64_t T, int E, const int* group_of,
+                                     const int* offsets, int* cursor, int* slot_tok, float* slot_gate) {
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  const int g = group_of[t];
+  const int pos = offsets[g] + atomicAdd(&cursor[g], 1);
+  slot_tok[pos] = (int)t;
+  if (K == 1) {
+    slot_gate[pos] = gates[t];
+  } else {
+    const int e0 = clamp_e(idx[2 * t], E), e1 = clamp_e(idx[2 * t + 1], E);
+    const float g0 = gates[2 * t], g1 = gates[2 * t + 1];
+    // gates in the group's expert order (ascending expert index)
+    slot_gate[2 * pos] = e0 <= e1 ? g0 : g1;
+    slot_gate[2 * pos + 1] = e0 <= e1 ? g1 : g0;
+  }
+}
+
+// ---- stage 1 ---------------------------------------------------------------------------------------
+struct Stage1Params {
+  int D, W, R, N, R_pad, K2, nbw;  // nbw: 64-column W_x boxes per expert
+  const int* num_tiles;
+  const TileInfo* tiles;
+  const int* slot_tok;
+  const float* slot_gate;
+  __nv_bfloat16* aprime;
+  float* B_mix;
+  float* C_mix;
+  void* status;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+  const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+  return l | (h << 16);
+}
+
+// After a failed wait: let the producer's copies in flight land (bounded, ignoring the abort flag).
+__device__ void drain_ring(uint64_t* full, int stages, int stage, uint32_t phase, int issued) {
+  for (int i = 0; i < min(issued, stages); ++i) {
+    int s = stage - 1 - i;
+    uint32_t ph = phase;
+    if (s < 0) {
+      s += stages;
+      ph ^= 1u;
+    }
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(&full[s], ph) && globaltimer_ns() - t0 < kWaitLimitNs) {
+    }
+  }
+}
+
+// Commit to a fresh barrier and wait (bounded) until every MMA this thread issued has completed,
+// so that TMEM can be released.
+__device__ __forceinline__ void wait_all_mma(uint64_t* done) {
+  mma_commit(done);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(done, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+  }
+}
+
+template <int K>
+__global__ void __launch_bounds__(192, 1)
+    proj_stage1_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wx,
+                       const Stage1Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages1 * kSlot1);
+  uint64_t* empty = full + kStages1;
+  uint64_t* acc_full = empty + kStages1;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* done = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages1; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 4);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_x);
+    prefetch_tmap(&tm_wx);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int num_tiles = *p.num_tiles;
+  const int ksteps = p.D / BK1;
+  const uint32_t slot_bytes = 8192u + (uint32_t)(K * p.nbw) * 4096u;
+
+  if (warp == 0) {
+    // ---------------- producer ----------------
+    int stage = 0, issued = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const TileInfo ti = p.tiles[tile];
+      int rr[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) rr[i] = p.slot_tok[ti.row_begin + min(4 * lane + i, ti.rows - 1)];
+      const int ej[2] = {ti.e0, ti.e1};
+      for (int ks = 0; ks < ksteps; ++ks) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t* slot = ring + stage * kSlot1;
+        if (lane == 0) mbar_arrive_expect_tx(&full[stage], slot_bytes);
+        __syncwarp();
+        tma_gather4(slot + lane * 256, &tm_x, &full[stage], ks * BK1, rr[0], rr[1], rr[2], rr[3]);
+        if (lane < K * p.nbw) {
+          const int j = lane / p.nbw, nb = lane - j * p.nbw;
+          tma_load_3d(slot + 8192 + lane * 4096, &tm_wx, &full[stage], nb * 64, ks * BK1, ej[j]);
+        }
+        ++issued;
+        if (++stage == kStages1) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) record_device_error(p.status, SWIMBA_ERR_TIMEOUT, 11, blockIdx.x, 0);
+      drain_ring(full, kStages1, stage, phase, issued);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(BM, p.W, /*b_mn_major=*/true);
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int ks = 0; ks < ksteps; ++ks) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t base = smem_u32(ring + stage * kSlot1);
+#pragma unroll
+          for (int kk = 0; kk < BK1 / 16; ++kk) {
+            const uint64_t adesc = smem_desc(base + kk * 32, 16, 512, kLayoutSW64);
+#pragma unroll
+            for (int j = 0; j < K; ++j) {
+              const uint64_t bdesc = smem_desc(base + 8192 + j * p.nbw * 4096 + kk * 16 * 128, 4096, 1024, kLayoutSW128);
+              mma_bf16(tmem + j * 256, adesc, bdesc, idesc, (ks | kk) != 0);
+            }
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == kStages1) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(acc_full);
+        acc_phase ^= 1u;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_device_error(p.status, SWIMBA_ERR_TIMEOUT, 12, blockIdx.x, 0);
+      }
+      wait_all_mma(done);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue: one TMEM lane (= tile row) per thread ----------------
+    const int q = warp & 3;
+    const int row = 32 * q + lane;
+    const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const TileInfo ti = p.tiles[tile];
+      if (!mbar_wait(acc_full, acc_phase, abort_flag)) {
+        *abort_flag = 1;
+        if (lane == 0) record_device_error(p.status, SWIMBA_ERR_TIMEOUT, 13, blockIdx.x, tile);
+        break;
+      }
+      acc_phase ^= 1u;
+      tc_fence_after();
+      const bool valid = row < ti.rows;
+      const int pos = ti.row_begin + min(row, ti.rows - 1);
+      const int t = p.slot_tok[pos];
+      float g[K];
+#pragma unroll
+      for (int j = 0; j < K; ++j) g[j] = p.slot_gate[pos * K + j];
+      uint4* arow = reinterpret_cast<uint4*>(p.aprime + ((size_t)tile * BM + row) * p.K2);
+      float v[16];
+#pragma unroll
+      for (int j = 0; j < K; ++j) {
+        for (int c = 0; c < p.R; c += 16) {
+          tmem_ld16(tl + j * 256 + c, v);
+          uint4 lo, hi;
+          lo.x = pack_bf16x2(g[j] * v[0], g[j] * v[1]);
+          lo.y = pack_bf16x2(g[j] * v[2], g[j] * v[3]);
+          lo.z = pack_bf16x2(g[j] * v[4], g[j] * v[5]);
+          lo.w = pack_bf16x2(g[j] * v[6], g[j] * v[7]);
+          hi.x = pack_bf16x2(g[j] * v[8], g[j] * v[9]);
+          hi.y = pack_bf16x2(g[j] * v[10], g[j] * v[11]);
+          hi.z = pack_bf16x2(g[j] * v[12], g[j] * v[13]);
+          hi.w = pack_bf16x2(g[j] * v[14], g[j] * v[15]);
+          arow[(j * p.R_pad + c) / 8] = lo;
+          arow[(j * p.R_pad + c) / 8 + 1] = hi;
+        }
+        for (int c = p.R; c < p.R_pad; c += 8) arow[(j * p.R_pad + c) / 8] = make_uint4(0, 0, 0, 0);
+      }
+      float bs[16], cs[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) bs[i] = cs[i] = 0.f;
+#pragma unroll
+      for (int j = 0; j < K; ++j) {
+        tmem_ld16(tl + j * 256 + p.R, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) bs[i] = fmaf(g[j], v[i], bs[i]);
+        tmem_ld16(tl + j * 256 + p.R + 16, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) cs[i] = fmaf(g[j], v[i], cs[i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      if (valid) {
+        float4* bo = reinterpret_cast<float4*>(p.B_mix + (size_t)t * 16);
+        float4* co = reinterpret_cast<float4*>(p.C_mix + (size_t)t * 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          bo[i] = make_float4(bs[4 * i], bs[4 * i + 1], bs[4 * i + 2], bs[4 * i + 3]);
+          co[i] = make_float4(cs[4 * i], cs[4 * i + 1], cs[4 * i + 2], cs[4 * i + 3]);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---- stage 2 ---------------------------------------------------------------------------------------
+struct Stage2Params {
+  int D, R, R_pad, K2, RS;  // RS: W_dt rows per ring stage (min(R, 64))
+  const int* num_tiles;
+  const TileInfo* tiles;
+  const int* slot_tok;
+  const float* slot_gate;
+  const float* b_dt;  // [E, D]
+  float* delta;
+  void* status;
+};
+
+// softplus(v) = max(v, 0) + log1p(e^{-|v|}): e^{-|v|} with the ex2 instruction; log1p(e) by its
+// series e - e^2/2 + e^3/3 below e = 2^-6 (truncation < e^4/4), else as ln(1 + e) with the lg2
+// instruction (1 + e >= 1.0156, so the relative error stays near 1e-5 at worst).
+__device__ __forceinline__ float softplus_fast(float v) {
+  const float e = ex2_approx(-fabsf(v) * kLog2e);
+  float l;
+  if (e < 0.015625f) {
+    l = e * fmaf(e, fmaf(e, 0.33333334f, -0.5f), 1.f);
+  } else {
+    float lg;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(1.f + e));
+    l = lg * 0.69314718f;
+  }
+  return fmaxf(v, 0.f) + l;
+}
+
+template <int K>
+__global__ void __launch_bounds__(320, 1)
+    proj_stage2_kernel(const __grid_constant__ CUtensorMap tm_ap, const __grid_constant__ CUtensorMap tm_wdt,
+                       const Stage2Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int nbox_ap = p.K2 / 64;
+  uint8_t* ap = smem;                                // [K2/64][128 rows][128 B]
+  uint8_t* ring = smem + nbox_ap * kApBox;           // [kStages2][kSlot2]
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + kStages2 * kSlot2);
+  uint64_t* empty = full + kStages2;
+  uint64_t* ap_full = empty + kStages2;
+  uint64_t* ap_empty = ap_full + 1;
+  uint64_t* acc_full = ap_empty + 1;   // [2]
+  uint64_t* acc_empty = acc_full + 2;  // [2]
+  uint64_t* done = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages2; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(ap_full, 1);
+    mbar_init(ap_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 8);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_ap);
+    prefetch_tmap(&tm_wdt);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int num_tiles = *p.num_tiles;
+  const int nchunks = (p.D + NC - 1) / NC;
+  const long long total = (long long)num_tiles * nchunks;
+  const long long item_begin = total * blockIdx.x / gridDim.x;
+  const long long item_end = total * (blockIdx.x + 1) / gridDim.x;
+  const int rs_steps = p.R / p.RS;
+
+  if (warp == 0) {
+    // ---------------- producer ----------------
+    int stage = 0, issued = 0, cur_tile = -1;
+    uint32_t phase = 0, ap_phase = 0;
+    int ej[2] = {0, 0};
+    bool ok = true;
+    for (long long item = item_begin; item < item_end && ok; ++item) {
+      const int tile = (int)(item / nchunks);
+      const int c = (int)(item - (long long)tile * nchunks);
+      if (tile != cur_tile) {
+        if (!mbar_wait(ap_empty, ap_phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(ap_full, (uint32_t)(nbox_ap * kApBox));
+          for (int kb = 0; kb < nbox_ap; ++kb) tma_load_2d(ap + kb * kApBox, &tm_ap, ap_full, kb * 64, tile * BM);
+        }
+        ap_phase ^= 1u;
+        cur_tile = tile;
+        const TileInfo ti = p.tiles[tile];
+        ej[0] = ti.e0;
+        ej[1] = ti.e1;
+      }
+      for (int j = 0; j < K && ok; ++j) {
+        for (int rs = 0; rs < rs_steps; ++rs) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* slot = ring + stage * kSlot2;
+          if (lane == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)(4 * p.RS * 128));
+          __syncwarp();
+          if (lane < 4) tma_load_3d(slot + lane * p.RS * 128, &tm_wdt, &full[stage], c * NC + lane * 64, rs * p.RS, ej[j]);
+          ++issued;
+          if (++stage == kStages2) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) record_device_error(p.status, SWIMBA_ERR_TIMEOUT, 21, blockIdx.x, 0);
+      drain_ring(full, kStages2, stage, phase, issued);
+      if (cur_tile >= 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(ap_full, ap_phase ^ 1u) && globaltimer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(BM, NC, /*b_mn_major=*/true);
+      const uint32_t ap_base = smem_u32(ap);
+      int stage = 0, cur_tile = -1, buf = 0;
+      uint32_t phase = 0, ap_phase = 0;
+      uint32_t acc_phase[2] = {0, 0};
+      bool ok = true;
+      for (long long item = item_begin; item < item_end && ok; ++item) {
+        const int tile = (int)(item / nchunks);
+        if (tile != cur_tile) {
+          if (cur_tile >= 0) mma_commit(ap_empty);
+          if (!mbar_wait(ap_full, ap_phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          ap_phase ^= 1u;
+          cur_tile = tile;
+        }
+        if (!mbar_wait(&acc_empty[buf], acc_phase[buf] ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        acc_phase[buf] ^= 1u;
+        tc_fence_after();
+        bool first = true;
+        for (int j = 0; j < K && ok; ++j) {
+          for (int rs = 0; rs < rs_steps; ++rs) {
+            if (!mbar_wait(&full[stage], phase, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sbase = smem_u32(ring + stage * kSlot2);
+            for (int kk = 0; kk < p.RS / 16; ++kk) {
+              const int kg = j * p.R_pad + rs * p.RS + kk * 16;  // K offset inside A'
+              const uint64_t adesc = smem_desc(ap_base + (kg >> 6) * kApBox + (kg & 63) * 2, 16, 1024, kLayoutSW128);
+              const uint64_t bdesc = smem_desc(sbase + kk * 16 * 128, p.RS * 128, 1024, kLayoutSW128);
+              mma_bf16(tmem + buf * NC, adesc, bdesc, idesc, first ? 0u : 1u);
+              first = false;
+            }
+            mma_commit(&empty[stage]);
+            if (++stage == kStages2) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[buf]);
+        buf ^= 1;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_device_error(p.status, SWIMBA_ERR_TIMEOUT, 22, blockIdx.x, 0);
+      }
+      wait_all_mma(done);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue: 8 warps, two per TMEM lane quarter ----------------
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;  // 0: chunk columns [0,128), 1: [128,256)
+    const int row = 32 * q + lane;
+    const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
+    int cur_tile = -1, buf = 0;
+    uint32_t acc_phase[2] = {0, 0};
+    bool valid = false;
+    int t = 0, e[2] = {0, 0};
+    float g[K];
+#pragma unroll
+    for (int j = 0; j < K; ++j) g[j] = 0.f;
+    for (long long item = item_begin; item < item_end; ++item) {
+      const int tile = (int)(item / nchunks);
+      const int c = (int)(item - (long long)tile * nchunks);
+      if (tile != cur_tile) {
+        const TileInfo ti = p.tiles[tile];
+        valid = row < ti.rows;
+        const int pos = ti.row_begin + min(row, ti.rows - 1);
+        t = p.slot_tok[pos];
+#pragma unroll
+        for (int j = 0; j < K; ++j) g[j] = p.slot_gate[pos * K + j];
+        e[0] = ti.e0;
+        e[1] = ti.e1;
+        cur_tile = tile;
+      }
+      if (!mbar_wait(&acc_full[buf], acc_phase[buf], abort_flag)) {
+        *abort_flag = 1;
+        if (lane == 0) record_device_error(p.status, SWIMBA_ERR_TIMEOUT, 23, blockIdx.x, (int)item);
+        break;
+      }
+      acc_phase[buf] ^= 1u;
+      tc_fence_after();
+      for (int cc = 0; cc < 4; ++cc) {
+        const int col = half * 128 + cc * 32;
+        float v[32];
+        tmem_ld32(tl + buf * NC + col, v);
+        if (cc == 3) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        }
+        const int d0 = c * NC + col;
+        if (d0 < p.D) {
+          float bias[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) bias[i] = 0.f;
+#pragma unroll
+          for (int j = 0; j < K; ++j) {
+            const float4* bp = reinterpret_cast<const float4*>(p.b_dt + (size_t)e[j] * p.D + d0);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 b4 = __ldg(bp + i);
+              bias[4 * i + 0] = fmaf(g[j], b4.x, bias[4 * i + 0]);
+              bias[4 * i + 1] = fmaf(g[j], b4.y, bias[4 * i + 1]);
+              bias[4 * i + 2] = fmaf(g[j], b4.z, bias[4 * i + 2]);
+              bias[4 * i + 3] = fmaf(g[j], b4.w, bias[4 * i + 3]);
+            }
+          }
+          if (valid) {
+            float4* out = reinterpret_cast<float4*>(p.delta + (size_t)t * p.D + d0);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              out[i] = make_float4(softplus_fast(v[4 * i + 0] + bias[4 * i + 0]),
+                                   softplus_fast(v[4 * i + 1] + bias[4 * i + 1]),
+                                   softplus_fast(v[4 * i + 2] + bias[4 * i + 2]),
+                                   softplus_fast(v[4 * i + 3] + bias[4 * i + 3]));
+            }
+          }
+        }
+      }
+      buf ^= 1;
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---- host side -------------------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
+            const cuuint32_t* box, CUtensorMapSwizzle swz) {
+  auto fn = get_encode();
+  if (!fn) return false;
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims, strides_bytes, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+template <int K>
+cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s) {
+  const TcLayout L = tc_layout(p.T, p.E, K, p.R);
+  int* group_of = reinterpret_cast<int*>(ws + L.group_of);
+  int* counts = reinterpret_cast<int*>(ws + L.counts);
+  int* cursor = reinterpret_cast<int*>(ws + L.cursor);
+  int* offsets = reinterpret_cast<int*>(ws + L.offsets);
+  int* num_tiles = reinterpret_cast<int*>(ws + L.num_tiles);
+  TileInfo* tiles = reinterpret_cast<TileInfo*>(ws + L.tiles);
+  int* slot_tok = reinterpret_cast<int*>(ws + L.slot_tok);
+  float* slot_gate = reinterpret_cast<float*>(ws + L.slot_gate);
+  __nv_bfloat16* aprime = reinterpret_cast<__nv_bfloat16*>(ws + L.aprime);
+
+  cudaError_t e = cudaMemsetAsync(counts, 0, 8 * (size_t)L.G, s);  // counts and cursor
+  if (e != cudaSuccess) return e;
+  const unsigned tb = (unsigned)((p.T + 255) / 256);
+  group_count_kernel<K><<<tb, 256, 0, s>>>(p.idx, p.T, p.E, group_of, counts);
+  group_scan_kernel<K><<<1, 256, 0, s>>>(counts, L.G, offsets, num_tiles, tiles);
+  group_scatter_kernel<K><<<tb, 256, 0, s>>>(p.idx, p.gates, p.T, p.E, group_of, offsets, cursor, slot_tok, slot_gate);
+  note_launch(3);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  const int W = p.R + 2 * p.N;
+  const int nbw = (W + 63) / 64;
+  CUtensorMap tm_x, tm_wx, tm_ap, tm_wdt;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)p.D, (cuuint64_t)p.T};
+    cuuint64_t str[1] = {(cuuint64_t)p.D * 2};
+    cuuint32_t box[2] = {BK1, 1};
+    if (!encode(&tm_x, p.x, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B)) return cudaErrorInvalidValue;
+  }
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)W, (cuuint64_t)p.D, (cuuint64_t)p.E};
+    cuuint64_t str[2] = {(cuuint64_t)W * 2, (cuuint64_t)W * p.D * 2};
+    cuuint32_t box[3] = {64, BK1, 1};
+    if (!encode(&tm_wx, p.W_x, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
+  }
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)L.K2, (cuuint64_t)L.max_tiles * BM};
+    cuuint64_t str[1] = {(cuuint64_t)L.K2 * 2};
+    cuuint32_t box[2] = {64, BM};
+    if (!encode(&tm_ap, aprime, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
+  }
+  const int RS = p.R < 64 ? p.R : 64;
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)p.D, (cuuint64_t)p.R, (cuuint64_t)p.E};
+    cuuint64_t str[2] = {(cuuint64_t)p.D * 2, (cuuint64_t)p.R * p.D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)RS, 1};
+    if (!encode(&tm_wdt, p.W_dt, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
+  }
+
+  const int sms = num_sms();
+  Stage1Params s1{p.D, W, p.R, p.N, L.R_pad, L.K2, nbw, num_tiles, tiles, slot_tok, slot_gate, aprime,
+                  p.B_mix, p.C_mix, ws};
+  const size_t smem1 = 1024 + (size_t)kStages1 * kSlot1 + 256;
+  e = cudaFuncSetAttribute(proj_stage1_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+  if (e != cudaSuccess) return e;
+  proj_stage1_kernel<K><<<(unsigned)std::min(L.max_tiles, sms), 192, smem1, s>>>(tm_x, tm_wx, s1);
+  note_launch();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  Stage2Params s2{p.D, p.R, L.R_pad, L.K2, RS, num_tiles, tiles, slot_tok, slot_gate, p.b_dt, p.delta, ws};
+  const size_t smem2 = 1024 + (size_t)(L.K2 / 64) * kApBox + (size_t)kStages2 * kSlot2 + 256;
+  e = cudaFuncSetAttribute(proj_stage2_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
+  if (e != cudaSuccess) return e;
+  proj_stage2_kernel<K><<<(unsigned)sms, 320, smem2, s>>>(tm_ap, tm_wdt, s2);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// The tensor-core path covers bf16 activations and tables, k <= 2, N = 16, R a multiple of 16 with
+// R <= 64 or R in {128}, R + 2N <= 192 (<= 256 for k = 1), and D a multiple of 64.
+bool proj_tc_supported(const ProjParams& p, bool io_bf16, bool w_bf16) {
+  const int W = p.R + 2 * p.N;
+  if (!io_bf16 || !w_bf16) return false;
+  if (p.k < 1 || p.k > 2 || p.N != 16) return false;
+  if (p.R % 16 != 0 || !(p.R <= 64 || p.R == 128)) return false;
+  if (W % 16 != 0 || W > (p.k == 2 ? 192 : 256)) return false;
+  if (p.D % 64 != 0 || p.T < 1 || p.T > (int64_t(1) << 30)) return false;
+  return true;
+}
+
+size_t proj_tc_workspace(int64_t T, int E, int k, int R) { return tc_layout(T, E, k, R).total; }
+
+cudaError_t run_proj_tc(const ProjParams& p, void* ws, cudaStream_t s) {
+  uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+  return p.k == 1 ? run_tc<1>(p, w, s) : run_tc<2>(p, w, s);
+}
+
+}  // namespace swimba
