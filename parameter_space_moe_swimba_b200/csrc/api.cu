@@ -1,5 +1,6 @@
 // C ABI of libswimba: argument validation, workspace layout and kernel dispatch. The layer's
 // steps run in the kernels of route.cu, proj_simt.cu, proj_tc.cu and scan.cu.
+#include <algorithm>
 #include <atomic>
 #include <cstring>
 
@@ -66,6 +67,16 @@ size_t proj_workspace(const swimba_dims* d) {
   return use_tc(d) ? proj_tc_workspace(d->batch * d->seqlen, d->n_experts, d->top_k, d->dt_rank) : kStatusBytes;
 }
 
+ScanPlan scan_plan(const swimba_dims* d) {
+  return scan_fast_plan(d->batch, d->seqlen, d->d_inner, d->d_state, d->n_experts, d->top_k,
+                        d->io_dtype == SWIMBA_BF16);
+}
+
+size_t scan_workspace(const swimba_dims* d) {
+  const ScanPlan pl = scan_plan(d);
+  return kStatusBytes + (pl.fast ? pl.ws_bytes : 0);
+}
+
 }  // namespace
 
 extern "C" {
@@ -74,12 +85,14 @@ size_t swimba_workspace_size(const swimba_dims* dims, int op) {
   if (check_dims(dims) != SWIMBA_OK) return 0;
   switch (op) {
     case SWIMBA_OP_ROUTE:
-    case SWIMBA_OP_SCAN:
     case SWIMBA_OP_STEP:
       return kStatusBytes;
+    case SWIMBA_OP_SCAN:
+      return scan_workspace(dims);
     case SWIMBA_OP_PROJ:
-    case SWIMBA_OP_LAYER:
       return proj_workspace(dims);
+    case SWIMBA_OP_LAYER:
+      return std::max(proj_workspace(dims), scan_workspace(dims));
     default:
       return 0;
   }
@@ -120,7 +133,7 @@ swimba_status swimba_mixed_proj(const swimba_dims* dims, const void* x, const in
 static swimba_status scan_common(const swimba_dims* dims, const void* x, const void* z, const float* delta,
                                  const float* B_mix, const float* C_mix, const int32_t* idx, const float* gates,
                                  const swimba_weights* w, const float* h0, void* out, float* h_final, float* y_pre,
-                                 bool step, void* stream) {
+                                 bool step, void* ws, void* stream) {
   if (!x || !z || !delta || !B_mix || !C_mix || !idx || !gates || !w || !w->A || !w->D_skip || !out)
     return SWIMBA_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(z) || !aligned16(out) || !aligned16(delta)) return SWIMBA_ERR_ALIGN;
@@ -129,6 +142,13 @@ static swimba_status scan_common(const swimba_dims* dims, const void* x, const v
   ScanParams p{x,   z,       delta, B_mix,          C_mix,          idx,           gates,
                w->A, w->D_skip, h0,  out,            h_final,        y_pre,         dims->seqlen,
                (int)dims->batch, dims->d_inner, dims->d_state, dims->n_experts, dims->top_k};
+  if (!step) {
+    const ScanPlan pl = scan_plan(dims);
+    if (pl.fast) {
+      uint8_t* seg_ws = reinterpret_cast<uint8_t*>(ws) + kStatusBytes;
+      return cuda_status(run_scan_fast(p, pl, seg_ws, ws, static_cast<cudaStream_t>(stream)));
+    }
+  }
   return cuda_status(run_scan(p, dims->io_dtype == SWIMBA_BF16, step, static_cast<cudaStream_t>(stream)));
 }
 
@@ -140,7 +160,7 @@ swimba_status swimba_scan_fwd(const swimba_dims* dims, const void* x, const void
   if (st != SWIMBA_OK) return st;
   if (ws == nullptr || ws_bytes < swimba_workspace_size(dims, SWIMBA_OP_SCAN)) return SWIMBA_ERR_WORKSPACE;
   if (!aligned16(ws)) return SWIMBA_ERR_ALIGN;
-  return scan_common(dims, x, z, delta, B_mix, C_mix, idx, gates, w, h0, out, h_final, y_pre, false, stream);
+  return scan_common(dims, x, z, delta, B_mix, C_mix, idx, gates, w, h0, out, h_final, y_pre, false, ws, stream);
 }
 
 swimba_status swimba_step(const swimba_dims* dims, const void* x, const void* z, const float* delta,
@@ -149,7 +169,7 @@ swimba_status swimba_step(const swimba_dims* dims, const void* x, const void* z,
   swimba_status st = check_dims(dims);
   if (st != SWIMBA_OK) return st;
   if (dims->seqlen != 1 || h == nullptr) return SWIMBA_ERR_INVALID_ARG;
-  return scan_common(dims, x, z, delta, B_mix, C_mix, idx, gates, w, h, out, h, nullptr, true, stream);
+  return scan_common(dims, x, z, delta, B_mix, C_mix, idx, gates, w, h, out, h, nullptr, true, nullptr, stream);
 }
 
 swimba_status swimba_get_device_status(void* ws, void* stream) {

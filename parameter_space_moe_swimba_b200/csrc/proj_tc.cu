@@ -13,9 +13,11 @@
 //                   x rows are gathered by TMA (tile::gather4, 64-byte swizzle); W_x boxes are
 //                   MN-major 128-byte-swizzled tiles of the [E, D, R+2N] table as stored.
 //                   Epilogue: B_mix, C_mix = Σ_j g_j (B^j, C^j) -> global; the gated low-rank
-//                   rows  A'[row] = [g_0 dt_low^0 | g_1 dt_low^1]  (bf16) -> workspace.
-//   stage 2         per (tile, 256-column chunk): acc = A'_tile · [W_dt^{e_0}; W_dt^{e_1}]
-//                   (K = k·R), i.e. Σ_j g_j dt_low^j W_dt^{e_j} in one accumulation. Epilogue:
+//                   rows g_j dt_low^j, split into bf16 hi + lo parts (hi = bf16(v), lo =
+//                   bf16(v - hi)), -> workspace as A'[row] = [hi_0 | hi_1 | lo_0 | lo_1].
+//   stage 2         per (tile, 256-column chunk): acc = Σ_j (hi_j + lo_j) · W_dt^{e_j}
+//                   (each W_dt box feeds two MMAs), i.e. Σ_j g_j dt_low^j W_dt^{e_j} with the
+//                   low-rank operand carried to about 16 significant bits. Epilogue:
 //                   + Σ_j g_j b_dt^{e_j}, softplus, store delta rows of the tile's tokens.
 // Both GEMM kernels are persistent and warp specialised: warp 0 issues TMA, warp 1 owns TMEM and
 // issues the MMAs, the remaining warps drain TMEM. Every mbarrier wait is bounded (1 s); on a
@@ -40,7 +42,7 @@ constexpr int BK1 = 32;        // stage-1 K slice per ring stage (64 bytes of bf
 constexpr int kStages1 = 6;
 constexpr int kSlot1 = 32768;  // A 8 KB + up to 6 W_x boxes of 4 KB
 constexpr int NC = 256;        // stage-2 output columns per chunk
-constexpr int kStages2 = 4;
+constexpr int kStages2 = 3;
 constexpr int kSlot2 = 32768;  // 4 W_dt boxes of up to 64 rows x 128 B
 constexpr int kApBox = BM * 128;  // one 64-column box of A' (16 KB)
 
@@ -60,7 +62,7 @@ TcLayout tc_layout(int64_t T, int E, int K, int R) {
   L.G = K == 1 ? E : E * (E - 1) / 2;
   L.max_tiles = (int)((T + BM - 1) / BM) + L.G;
   L.R_pad = (R + 63) / 64 * 64;
-  L.K2 = K * L.R_pad;
+  L.K2 = 2 * K * L.R_pad;  // [hi_0 .. hi_{k-1} | lo_0 .. lo_{k-1}], each R_pad wide
   size_t o = kStatusBytes;
   L.group_of = o; o = align_up(o + 4 * (size_t)T, 256);
   L.counts = o; o += 4 * (size_t)L.G;
@@ -171,10 +173,13 @@ struct Stage1Params {
   void* status;
 };
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
-  const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
-  return l | (h << 16);
+// Two floats a, b as packed bf16 pairs: hi = (bf16(a), bf16(b)), lo = the bf16 of the remainders.
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat16 ha = __float2bfloat16_rn(a), hb = __float2bfloat16_rn(b);
+  const __nv_bfloat16 la = __float2bfloat16_rn(a - __bfloat162float(ha));
+  const __nv_bfloat16 lb = __float2bfloat16_rn(b - __bfloat162float(hb));
+  hi = (uint32_t)__bfloat16_as_ushort(ha) | ((uint32_t)__bfloat16_as_ushort(hb) << 16);
+  lo = (uint32_t)__bfloat16_as_ushort(la) | ((uint32_t)__bfloat16_as_ushort(lb) << 16);
 }
 
 // After a failed wait: let the producer's copies in flight land (bounded, ignoring the abort flag).
@@ -352,19 +357,19 @@ __global__ void __launch_bounds__(192, 1)
       for (int j = 0; j < K; ++j) {
         for (int c = 0; c < p.R; c += 16) {
           tmem_ld16(tl + j * 256 + c, v);
-          uint4 lo, hi;
-          lo.x = pack_bf16x2(g[j] * v[0], g[j] * v[1]);
-          lo.y = pack_bf16x2(g[j] * v[2], g[j] * v[3]);
-          lo.z = pack_bf16x2(g[j] * v[4], g[j] * v[5]);
-          lo.w = pack_bf16x2(g[j] * v[6], g[j] * v[7]);
-          hi.x = pack_bf16x2(g[j] * v[8], g[j] * v[9]);
-          hi.y = pack_bf16x2(g[j] * v[10], g[j] * v[11]);
-          hi.z = pack_bf16x2(g[j] * v[12], g[j] * v[13]);
-          hi.w = pack_bf16x2(g[j] * v[14], g[j] * v[15]);
-          arow[(j * p.R_pad + c) / 8] = lo;
-          arow[(j * p.R_pad + c) / 8 + 1] = hi;
+          uint32_t hw[8], lw[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) split_bf16x2(g[j] * v[2 * i], g[j] * v[2 * i + 1], hw[i], lw[i]);
+          const int ohi = (j * p.R_pad + c) / 8, olo = ((K + j) * p.R_pad + c) / 8;
+          arow[ohi] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          arow[ohi + 1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+          arow[olo] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          arow[olo + 1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
         }
-        for (int c = p.R; c < p.R_pad; c += 8) arow[(j * p.R_pad + c) / 8] = make_uint4(0, 0, 0, 0);
+        for (int c = p.R; c < p.R_pad; c += 8) {
+          arow[(j * p.R_pad + c) / 8] = make_uint4(0, 0, 0, 0);
+          arow[((K + j) * p.R_pad + c) / 8] = make_uint4(0, 0, 0, 0);
+        }
       }
       float bs[16], cs[16];
 #pragma unroll
@@ -568,11 +573,15 @@ __global__ void __launch_bounds__(320, 1)
             tc_fence_after();
             const uint32_t sbase = smem_u32(ring + stage * kSlot2);
             for (int kk = 0; kk < p.RS / 16; ++kk) {
-              const int kg = j * p.R_pad + rs * p.RS + kk * 16;  // K offset inside A'
-              const uint64_t adesc = smem_desc(ap_base + (kg >> 6) * kApBox + (kg & 63) * 2, 16, 1024, kLayoutSW128);
               const uint64_t bdesc = smem_desc(sbase + kk * 16 * 128, p.RS * 128, 1024, kLayoutSW128);
-              mma_bf16(tmem + buf * NC, adesc, bdesc, idesc, first ? 0u : 1u);
-              first = false;
+#pragma unroll
+              for (int part = 0; part < 2; ++part) {  // hi, then lo
+                const int kg = (part * K + j) * p.R_pad + rs * p.RS + kk * 16;  // K offset inside A'
+                const uint64_t adesc =
+                    smem_desc(ap_base + (kg >> 6) * kApBox + (kg & 63) * 2, 16, 1024, kLayoutSW128);
+                mma_bf16(tmem + buf * NC, adesc, bdesc, idesc, first ? 0u : 1u);
+                first = false;
+              }
             }
             mma_commit(&empty[stage]);
             if (++stage == kStages2) {

@@ -4,10 +4,13 @@
 // (es) / "Kernmechanisme van Swimba" (nl): a router gives each token mixing weights π_t over the
 // active experts (top-1 or top-k).
 //
-// Layout: one warp routes TOK consecutive tokens. Lanes stride over the channel dimension in
+// Layout (global-memory variant, used when W_r does not fit in shared memory): one warp routes TOK
+// consecutive tokens. Lanes stride over the channel dimension in
 // 16-byte chunks of x (8 bf16 or 4 fp32), so every x load is a coalesced 128-bit load and x is
 // read from HBM exactly once. The TOK x E partial sums of every lane are combined with a
 // butterfly of warp shuffles; then lane tt selects the experts of token t0+tt.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace swimba {
@@ -20,6 +23,40 @@ struct RouteParams {
   int64_t T;
   int D, E, k;
 };
+
+// top-k of one token's logits l[0..E): repeatedly take the largest remaining logit; a strict
+// comparison in ascending expert order keeps the lower index on ties. gates = softmax of the
+// selected logits (exp relative to the largest, so the first gate's weight is exactly 1).
+template <int EP>
+__device__ __forceinline__ void select_topk(const float (&l)[EP], int E, int k, int32_t* idx, float* gates) {
+  unsigned taken = 0u;
+  float wsel[16];
+  float top = 0.f, sum = 0.f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    wsel[j] = 0.f;
+    if (j < k) {
+      int bi = -1;
+      float best = 0.f;
+#pragma unroll
+      for (int e = 0; e < EP; ++e) {
+        const bool ok = (e < E) && !((taken >> e) & 1u);
+        if (ok && (bi < 0 || l[e] > best)) {
+          best = l[e];
+          bi = e;
+        }
+      }
+      taken |= 1u << bi;
+      if (j == 0) top = best;
+      wsel[j] = expf(best - top);
+      sum += wsel[j];
+      idx[j] = bi;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j)
+    if (j < k) gates[j] = wsel[j] / sum;
+}
 
 template <typename IO, int EP, int TOK>
 __global__ void __launch_bounds__(128) route_kernel(RouteParams p) {
@@ -78,46 +115,99 @@ __global__ void __launch_bounds__(128) route_kernel(RouteParams p) {
     }
 
 #pragma unroll
-  for (int tt = 0; tt < TOK; ++tt) {
-    const int64_t t = t0 + tt;
-    if (lane != tt || t >= p.T) continue;
-    // top-k: repeatedly take the largest remaining logit; a strict comparison in ascending
-    // expert order keeps the lower index on ties.
-    unsigned taken = 0u;
-    float wsel[16];
-    float top = 0.f, sum = 0.f;
+  for (int tt = 0; tt < TOK; ++tt)
+    if (lane == tt && t0 + tt < p.T) select_topk<EP>(acc[tt], E, p.k, p.idx + (t0 + tt) * p.k, p.gates + (t0 + tt) * p.k);
+}
+
+template <typename IO, int EP, int TOK>
+__global__ void __launch_bounds__(512, 1) route_smem_kernel(RouteParams p) {
+  extern __shared__ float2 Wp[];  // [EP/2][V][C]
+  constexpr int V = Vec16<IO>::n;
+  const int C = p.D / V;
+  const int E = p.E;
+  for (int q = threadIdx.x; q < (EP / 2) * p.D; q += blockDim.x) {
+    const int ep = q / p.D, d = q - ep * p.D;
+    const int e0 = 2 * ep, e1 = 2 * ep + 1;
+    const float w0 = e0 < E ? p.W_r[(size_t)d * E + e0] : 0.f;
+    const float w1 = e1 < E ? p.W_r[(size_t)d * E + e1] : 0.f;
+    Wp[((size_t)ep * V + (d % V)) * C + d / V] = make_float2(w0, w1);
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  const IO* x = reinterpret_cast<const IO*>(p.x);
+  for (int64_t grp = (int64_t)blockIdx.x * nwarps + (threadIdx.x >> 5); grp * TOK < p.T; grp += (int64_t)gridDim.x * nwarps) {
+    const int64_t t0 = grp * TOK;
+    float2 acc[TOK][EP / 2];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      wsel[j] = 0.f;
-      if (j < p.k) {
-        int bi = -1;
-        float best = 0.f;
+    for (int tt = 0; tt < TOK; ++tt)
 #pragma unroll
-        for (int e = 0; e < EP; ++e) {
-          const bool ok = (e < E) && !((taken >> e) & 1u);
-          if (ok && (bi < 0 || acc[tt][e] > best)) {
-            best = acc[tt][e];
-            bi = e;
-          }
+      for (int e = 0; e < EP / 2; ++e) acc[tt][e] = make_float2(0.f, 0.f);
+    for (int c = lane; c < C; c += 32) {
+      uint4 xv[TOK];
+#pragma unroll
+      for (int tt = 0; tt < TOK; ++tt) {
+        xv[tt] = make_uint4(0, 0, 0, 0);
+        if (t0 + tt < p.T) xv[tt] = __ldcs(reinterpret_cast<const uint4*>(x + (t0 + tt) * p.D) + c);
+      }
+#pragma unroll
+      for (int i = 0; i < V; ++i) {
+        float2 w[EP / 2];
+#pragma unroll
+        for (int e = 0; e < EP / 2; ++e) w[e] = Wp[((size_t)e * V + i) * C + c];
+#pragma unroll
+        for (int tt = 0; tt < TOK; ++tt) {
+          float xf[V];
+          Vec16<IO>::unpack(xv[tt], xf);
+          const float2 xx = make_float2(xf[i], xf[i]);
+#pragma unroll
+          for (int e = 0; e < EP / 2; ++e) acc[tt][e] = __ffma2_rn(xx, w[e], acc[tt][e]);
         }
-        taken |= 1u << bi;
-        if (j == 0) top = best;
-        wsel[j] = expf(best - top);
-        sum += wsel[j];
-        p.idx[t * p.k + j] = bi;
       }
     }
+    float a[TOK][EP];
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
-      if (j < p.k) p.gates[t * p.k + j] = wsel[j] / sum;
+    for (int tt = 0; tt < TOK; ++tt)
+#pragma unroll
+      for (int e = 0; e < EP / 2; ++e) {
+        a[tt][2 * e] = acc[tt][e].x;
+        a[tt][2 * e + 1] = acc[tt][e].y;
+      }
+#pragma unroll
+    for (int tt = 0; tt < TOK; ++tt)
+#pragma unroll
+      for (int e = 0; e < EP; ++e) {
+        float v = a[tt][e];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        a[tt][e] = v;
+      }
+#pragma unroll
+    for (int tt = 0; tt < TOK; ++tt)
+      if (lane == tt && t0 + tt < p.T) select_topk<EP>(a[tt], E, p.k, p.idx + (t0 + tt) * p.k, p.gates + (t0 + tt) * p.k);
   }
 }
 
 template <typename IO, int EP, int TOK>
 static cudaError_t launch_route(const RouteParams& p, cudaStream_t s) {
-  const int64_t warps = (p.T + TOK - 1) / TOK;
-  const int64_t blocks = (warps + 3) / 4;
-  route_kernel<IO, EP, TOK><<<(unsigned)blocks, 128, 0, s>>>(p);
+  constexpr int V = Vec16<IO>::n;
+  const size_t smem = sizeof(float2) * (EP / 2) * (size_t)p.D;
+  (void)V;
+  if (smem <= 160 * 1024) {
+    cudaError_t e =
+        cudaFuncSetAttribute(route_smem_kernel<IO, EP, TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t groups = (p.T + TOK - 1) / TOK;
+    const int64_t blocks = std::min<int64_t>(sms, (groups + 15) / 16);
+    route_smem_kernel<IO, EP, TOK><<<(unsigned)blocks, 512, smem, s>>>(p);
+  } else {
+    const int64_t warps = (p.T + TOK - 1) / TOK;
+    const int64_t blocks = (warps + 3) / 4;
+    route_kernel<IO, EP, TOK><<<(unsigned)blocks, 128, 0, s>>>(p);
+  }
   note_launch();
   return cudaGetLastError();
 }

@@ -25,4 +25,15 @@ struct ScanParams {
 
 cudaError_t run_scan(const ScanParams& p, bool io_bf16, bool step, cudaStream_t s);
 
+// Fast path plan: whether it applies, how many sequence segments, their length (a multiple of the
+// 16-token chunk) and the workspace the segment carries need.
+struct ScanPlan {
+  bool fast;
+  int S;
+  int64_t Lseg;
+  size_t ws_bytes;
+};
+ScanPlan scan_fast_plan(int64_t B, int64_t L, int D, int N, int E, int k, bool io_bf16);
+cudaError_t run_scan_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s);
+
 }  // namespace swimba

@@ -1,0 +1,544 @@
+// Selective scan over the mixed parameters, B200 fast path (bf16 x/z/out, N = 16, k <= 2, E <= 16).
+//
+// Sources: "Swimba: Switch Mamba Model Scales State Space Models" -- one state trajectory and ONE
+// recurrence whatever the number of experts (§2 "Resultado"; Teorema 2: the recurrence cost does
+// not grow with E); "Mamba y las SSMs: el retorno del estado persistente", "Mamba" (Ā = exp(Δ_t A);
+// Figura 2: the state stays on chip, inputs stream from HBM) and "Estado interno puramente lineal"
+// (the linear state admits a scan, used here to split long sequences into segments).
+//
+// Work unit = one warp = CPW channels of one sequence segment; G = 16/NS lanes share a channel and
+// hold NS of its 16 fp32 states in registers. The per-expert transition rows A^e[d, n0..n0+NS)
+// (pre-multiplied by log2 e) also live in registers: every lane of a warp reads the same token, so
+// the selected experts are warp-uniform and a switch on the expert index picks the registers.
+// Per token and state:  arg = Σ_j (Δ g_j) A^{e_j};  ā = 2^arg;  h = ā h + (Δ x) B;  y += C h.
+// The G lanes of a channel then reduce-scatter their partial readouts so that each lane finishes
+// one token: y += D_skip x, out = y z σ(z) (σ via tanh.approx for bf16 outputs).
+//
+// Each warp streams its inputs through its own 3-stage shared-memory ring filled by TMA (x, z, Δ
+// tiles of [16 tokens x CPW channels] and B_mix, C_mix rows of 16 tokens) plus the tokens' expert
+// indices and gates written by the warp's lanes one chunk ahead. Units are spread evenly over one
+// persistent CTA per SM (up to 14 warps each), so no SM gets a whole extra sequence.
+//
+// Segments (when B*D alone cannot fill the GPU): pass 1 computes, per segment, the end state from
+// zero and log2 of the decay product Σ_t Δ_t A_t; a carry pass chains them into each segment's
+// start state; the main pass then runs every segment from its true start state.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "scan.cuh"
+#include "sm100.cuh"
+
+namespace swimba {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int LC = 16;        // tokens per chunk
+constexpr int kStages = 3;    // ring depth per warp
+constexpr int kMaxWarps = 14; // warps per CTA (registers: 14 * 32 * 144 <= 65536)
+
+template <int NS>
+struct Geom {
+  static constexpr int G = 16 / NS;    // lanes per channel
+  static constexpr int CPW = 32 / G;   // channels per warp
+};
+
+// Byte offsets inside one ring stage of one warp.
+template <int NS>
+struct Stage {
+  static constexpr int CPW = Geom<NS>::CPW;
+  static constexpr int X = 0;                      // bf16 [LC][CPW]
+  static constexpr int Z = X + LC * CPW * 2;       // bf16 [LC][CPW]
+  static constexpr int DL = Z + LC * CPW * 2;      // f32  [LC][CPW]
+  static constexpr int B = DL + LC * CPW * 4;      // f32  [LC][16]
+  static constexpr int C = B + LC * 16 * 4;        // f32  [LC][16]
+  static constexpr int META = C + LC * 16 * 4;     // int4 [LC] {e0, e1, g0, g1}
+  static constexpr int BYTES = META + LC * 16;
+  static_assert(X % 128 == 0 && Z % 128 == 0 && DL % 128 == 0 && B % 128 == 0 && C % 128 == 0 && META % 128 == 0,
+                "TMA destinations must be 128-byte aligned");
+  static_assert(BYTES % 128 == 0, "stage size");
+};
+
+// 2^x on the FMA pipe for x <= 0: x = j + f with j = round(x) (the 1.5*2^23 shifter), f in
+// [-1/2, 1/2]; 2^f by a degree-5 polynomial fitted for minimax relative error on that interval
+// (fit_exp2_poly.py beside this file: float32 Horner error 2.4e-7, the size of ex2.approx's);
+// the exponent j is added to the result's exponent field. Inputs below -125 are clamped (result
+// 2^-125 instead of a flushed 0, which no decay product here can tell apart).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  const float2 lo = make_float2(-125.f, -125.f);
+  x = make_float2(fmaxf(x.x, lo.x), fmaxf(x.y, lo.y));
+  const float2 shifter = make_float2(12582912.f, 12582912.f);
+  const float2 t = __fadd2_rn(x, shifter);
+  const float2 j = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __fadd2_rn(x, make_float2(-j.x, -j.y));
+  float2 p = make_float2(0x1.5c08e6p-10f, 0x1.5c08e6p-10f);
+  p = __ffma2_rn(p, f, make_float2(0x1.3d0c52p-7f, 0x1.3d0c52p-7f));
+  p = __ffma2_rn(p, f, make_float2(0x1.c6b6e4p-5f, 0x1.c6b6e4p-5f));
+  p = __ffma2_rn(p, f, make_float2(0x1.ebf918p-3f, 0x1.ebf918p-3f));
+  p = __ffma2_rn(p, f, make_float2(0x1.62e428p-1f, 0x1.62e428p-1f));
+  p = __ffma2_rn(p, f, make_float2(0x1.000002p+0f, 0x1.000002p+0f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// arg (+)= c * A[e]  for a warp-uniform expert e (registers selected by a switch).
+template <int E, int NH, bool FIRST>
+__device__ __forceinline__ void expert_term(int e, float c, const float2 (&A)[E][NH], float2 (&arg)[NH]) {
+  const float2 cc = make_float2(c, c);
+#define SWIMBA_EXPERT_CASE(i)                                                  \
+  case i:                                                                      \
+    if constexpr (i < E) {                                                     \
+      _Pragma("unroll") for (int s = 0; s < NH; ++s) arg[s] =                  \
+          FIRST ? __fmul2_rn(cc, A[i][s]) : __ffma2_rn(cc, A[i][s], arg[s]);   \
+    }                                                                          \
+    break;
+  switch (e) {
+    SWIMBA_EXPERT_CASE(0) SWIMBA_EXPERT_CASE(1) SWIMBA_EXPERT_CASE(2) SWIMBA_EXPERT_CASE(3)
+    SWIMBA_EXPERT_CASE(4) SWIMBA_EXPERT_CASE(5) SWIMBA_EXPERT_CASE(6) SWIMBA_EXPERT_CASE(7)
+    SWIMBA_EXPERT_CASE(8) SWIMBA_EXPERT_CASE(9) SWIMBA_EXPERT_CASE(10) SWIMBA_EXPERT_CASE(11)
+    SWIMBA_EXPERT_CASE(12) SWIMBA_EXPERT_CASE(13) SWIMBA_EXPERT_CASE(14) SWIMBA_EXPERT_CASE(15)
+    default:
+      break;
+  }
+#undef SWIMBA_EXPERT_CASE
+}
+
+struct FastParams {
+  const int32_t* idx;
+  const float* gates;
+  const float* A;       // [E, D, 16]
+  const float* D_skip;  // [D]
+  const float* h0;      // [B, D, 16] or null (start state of segment 0)
+  const float* h_seg;   // [B, S, D, 16] start state of every segment (segmented main pass) or null
+  __nv_bfloat16* out;   // [B, L, D]
+  float* y_pre;         // [B, L, D] or null
+  float* h_final;       // [B, D, 16] or null
+  float* agg_h;         // pass 1: [B, S, D, 16] end state from zero
+  float* agg_logp;      // pass 1: [B, S, D, 16] log2 of the decay product
+  void* status;
+  int64_t L, Lseg;
+  int B, D, E, k, S;
+  int seg_count;        // segments this pass visits (S, or S - 1 for pass 1)
+  int units;            // B * seg_count * (D / CPW)
+};
+
+// AGG = true: pass 1 (segments 0 .. S-2 only; no readout, no output).
+template <int E, int K, int NS, int NPOLY, bool AGG>
+__global__ void __maxnreg__(144)
+    scan_fast_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
+                     const __grid_constant__ CUtensorMap tm_dl, const __grid_constant__ CUtensorMap tm_b,
+                     const __grid_constant__ CUtensorMap tm_c, const FastParams p) {
+  constexpr int G = Geom<NS>::G;
+  constexpr int CPW = Geom<NS>::CPW;
+  constexpr int NH = NS / 2;
+  using St = Stage<NS>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  uint8_t* ring = smem + (size_t)warp * kStages * St::BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)nwarps * kStages * St::BYTES) + warp * kStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(
+      reinterpret_cast<uint64_t*>(smem + (size_t)nwarps * kStages * St::BYTES) + nwarps * kStages);
+
+  if (lane == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+    fence_mbar_init();
+    if (warp == 0) {
+      *abort_flag = 0;
+      prefetch_tmap(&tm_x);
+      prefetch_tmap(&tm_dl);
+      prefetch_tmap(&tm_b);
+      if (!AGG) {
+        prefetch_tmap(&tm_z);
+        prefetch_tmap(&tm_c);
+      }
+    }
+  }
+  __syncthreads();
+
+  const int cl = lane / G;  // channel within the warp
+  const int gi = lane % G;  // state group
+  const int n0 = gi * NS;
+  const int ntiles = p.D / CPW;
+  const int u_begin = (int)((int64_t)p.units * blockIdx.x / gridDim.x);
+  const int u_end = (int)((int64_t)p.units * (blockIdx.x + 1) / gridDim.x);
+  uint32_t phase_bits = 0;  // one parity bit per stage
+  constexpr uint32_t tx_bytes = AGG ? (LC * CPW * 2 + LC * CPW * 4 + LC * 16 * 4)
+                                    : (2 * LC * CPW * 2 + LC * CPW * 4 + 2 * LC * 16 * 4);
+
+  for (int u = u_begin + warp; u < u_end; u += nwarps) {
+    const int tile = u % ntiles;
+    const int bs = u / ntiles;  // b * seg_count + seg
+    const int seg = bs % p.seg_count;
+    const int b = bs / p.seg_count;
+    const int d = tile * CPW + cl;
+    const int64_t t_begin = (int64_t)seg * p.Lseg;
+    const int64_t t_end = std::min<int64_t>(p.L, t_begin + p.Lseg);
+    const int nchunks = (int)((t_end - t_begin + LC - 1) / LC);
+
+    // per-expert transition rows of this lane's states, times log2(e)
+    float2 A[E][NH];
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+#pragma unroll
+      for (int s = 0; s < NH; ++s) {
+        if (e < p.E) {
+          const float2 a = *reinterpret_cast<const float2*>(p.A + ((size_t)e * p.D + d) * 16 + n0 + 2 * s);
+          A[e][s] = make_float2(a.x * kLog2e, a.y * kLog2e);
+        } else {
+          A[e][s] = make_float2(0.f, 0.f);
+        }
+      }
+    float2 h[NH];
+    const float* hs = AGG ? nullptr
+                          : (p.h_seg != nullptr ? p.h_seg + (((size_t)b * p.S + seg) * p.D + d) * 16
+                                                : (p.h0 != nullptr && seg == 0 ? p.h0 + ((size_t)b * p.D + d) * 16 : nullptr));
+#pragma unroll
+    for (int s = 0; s < NH; ++s) h[s] = hs ? *reinterpret_cast<const float2*>(hs + n0 + 2 * s) : make_float2(0.f, 0.f);
+    float2 lsum[NH];
+#pragma unroll
+    for (int s = 0; s < NH; ++s) lsum[s] = make_float2(0.f, 0.f);
+    const float dsk = AGG ? 0.f : p.D_skip[d];
+
+    // meta of one chunk: lane t (< LC) holds token t's {e0, e1, g0, g1}
+    auto load_meta = [&](int c) -> int4 {
+      int4 m = make_int4(0, 0, 0, 0);
+      const int64_t t = t_begin + (int64_t)c * LC + lane;
+      if (lane < LC && c < nchunks && t < t_end) {
+        const size_t tok = (size_t)b * p.L + t;
+        m.x = min(max(p.idx[tok * K], 0), p.E - 1);
+        m.z = __float_as_int(p.gates[tok * K]);
+        if (K == 2) {
+          m.y = min(max(p.idx[tok * K + 1], 0), p.E - 1);
+          m.w = __float_as_int(p.gates[tok * K + 1]);
+        }
+      }
+      return m;
+    };
+    // fill stage (c % kStages) with chunk c: meta from registers, the rest by TMA
+    auto issue = [&](int c, int4 meta) {
+      uint8_t* st = ring + (c % kStages) * St::BYTES;
+      if (lane < LC) reinterpret_cast<int4*>(st + St::META)[lane] = meta;
+      __syncwarp();
+      if (lane == 0) {
+        fence_proxy_async_smem();
+        uint64_t* bar = &full[c % kStages];
+        mbar_arrive_expect_tx(bar, tx_bytes);
+        const int t0 = (int)(t_begin + (int64_t)c * LC);
+        tma_load_3d(st + St::X, &tm_x, bar, tile * CPW, t0, b);
+        tma_load_3d(st + St::DL, &tm_dl, bar, tile * CPW, t0, b);
+        tma_load_3d(st + St::B, &tm_b, bar, 0, t0, b);
+        if (!AGG) {
+          tma_load_3d(st + St::Z, &tm_z, bar, tile * CPW, t0, b);
+          tma_load_3d(st + St::C, &tm_c, bar, 0, t0, b);
+        }
+      }
+    };
+
+    int4 meta_next = load_meta(0);
+    const int pre = nchunks < kStages ? nchunks : kStages;
+    for (int c = 0; c < pre; ++c) {
+      const int4 m = meta_next;
+      meta_next = load_meta(c + 1);
+      issue(c, m);
+    }
+    bool ok = true;
+    int issued = pre;
+    for (int c = 0; c < nchunks; ++c) {
+      const int sidx = c % kStages;
+      if (!mbar_wait(&full[sidx], (phase_bits >> sidx) & 1u, abort_flag)) {
+        ok = false;
+        break;
+      }
+      phase_bits ^= 1u << sidx;
+      const uint8_t* st = ring + sidx * St::BYTES;
+      const int4* meta = reinterpret_cast<const int4*>(st + St::META);
+      const __nv_bfloat16* xs = reinterpret_cast<const __nv_bfloat16*>(st + St::X);
+      const __nv_bfloat16* zs = reinterpret_cast<const __nv_bfloat16*>(st + St::Z);
+      const float* ds = reinterpret_cast<const float*>(st + St::DL);
+      const float4* bsm = reinterpret_cast<const float4*>(st + St::B);
+      const float4* csm = reinterpret_cast<const float4*>(st + St::C);
+      const int64_t t0 = t_begin + (int64_t)c * LC;
+#pragma unroll 1
+      for (int tt = 0; tt < LC; tt += G) {
+        float yp[G];
+#pragma unroll
+        for (int uu = 0; uu < G; ++uu) {
+          const int t = tt + uu;
+          const int4 m = meta[t];
+          const float dlt = ds[t * CPW + cl];
+          const float xv = __bfloat162float(xs[t * CPW + cl]);
+          float2 arg[NH];
+          expert_term<E, NH, true>(m.x, dlt * __int_as_float(m.z), A, arg);
+          if (K == 2) expert_term<E, NH, false>(m.y, dlt * __int_as_float(m.w), A, arg);
+          float2 a[NH];
+#pragma unroll
+          for (int s = 0; s < NH; ++s) {
+            if (s >= NH - NPOLY / 2) {
+              a[s] = exp2_poly2(arg[s]);
+            } else {
+              a[s] = make_float2(ex2_approx(arg[s].x), ex2_approx(arg[s].y));
+            }
+          }
+          const float dx = dlt * xv;
+          const float2 dxx = make_float2(dx, dx);
+          float2 bv[NH];
+#pragma unroll
+          for (int q = 0; q < NS / 4; ++q) {
+            const float4 b4 = bsm[t * 4 + gi * (NS / 4) + q];
+            bv[2 * q] = make_float2(b4.x, b4.y);
+            bv[2 * q + 1] = make_float2(b4.z, b4.w);
+          }
+#pragma unroll
+          for (int s = 0; s < NH; ++s) h[s] = __ffma2_rn(a[s], h[s], __fmul2_rn(dxx, bv[s]));
+          if (AGG) {
+#pragma unroll
+            for (int s = 0; s < NH; ++s) lsum[s] = __fadd2_rn(lsum[s], arg[s]);
+          } else {
+            float2 y2 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int q = 0; q < NS / 4; ++q) {
+              const float4 c4 = csm[t * 4 + gi * (NS / 4) + q];
+              y2 = __ffma2_rn(make_float2(c4.x, c4.y), h[2 * q], y2);
+              y2 = __ffma2_rn(make_float2(c4.z, c4.w), h[2 * q + 1], y2);
+            }
+            yp[uu] = y2.x + y2.y;
+          }
+        }
+        if (!AGG) {
+          // reduce-scatter the partial readouts over the G lanes of the channel: lane gi ends
+          // with the full y of token tt + gi
+          float ysum;
+          if (G == 2) {
+            const float send = gi == 0 ? yp[1 % G] : yp[0];
+            const float keep = gi == 0 ? yp[0] : yp[1 % G];
+            ysum = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+          } else {
+            const bool lo = gi < 2;
+            const float s0 = lo ? yp[2 % G] : yp[0], s1 = lo ? yp[3 % G] : yp[1 % G];
+            const float k0 = (lo ? yp[0] : yp[2 % G]) + __shfl_xor_sync(0xffffffffu, s0, 2);
+            const float k1 = (lo ? yp[1 % G] : yp[3 % G]) + __shfl_xor_sync(0xffffffffu, s1, 2);
+            const bool odd = gi & 1;
+            ysum = (odd ? k1 : k0) + __shfl_xor_sync(0xffffffffu, odd ? k0 : k1, 1);
+          }
+          const int t = tt + gi;
+          if (t0 + t < t_end) {
+            const float xv = __bfloat162float(xs[t * CPW + cl]);
+            const float zv = __bfloat162float(zs[t * CPW + cl]);
+            const float y = fmaf(dsk, xv, ysum);
+            const size_t o = ((size_t)b * p.L + t0 + t) * p.D + d;
+            if (p.y_pre != nullptr) p.y_pre[o] = y;
+            const float sig = fmaf(0.5f, tanh_approx(0.5f * zv), 0.5f);
+            p.out[o] = __float2bfloat16_rn(y * zv * sig);
+          }
+        }
+      }
+      __syncwarp();
+      if (c + kStages < nchunks) {
+        const int4 m = meta_next;
+        meta_next = load_meta(c + kStages + 1);
+        issue(c + kStages, m);
+        ++issued;
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) record_device_error(p.status, SWIMBA_ERR_TIMEOUT, 31, blockIdx.x, u);
+      // let this warp's copies in flight land before the CTA exits (bounded, ignores the flag)
+      for (int c = issued - kStages; c < issued; ++c) {
+        if (c < 0) continue;
+        const int sidx = c % kStages;
+        const uint64_t w0 = globaltimer_ns();
+        while (!mbar_try_wait(&full[sidx], (phase_bits >> sidx) & 1u) && globaltimer_ns() - w0 < kWaitLimitNs) {
+        }
+        phase_bits ^= 1u << sidx;
+      }
+      break;
+    }
+    // stage parity must restart at a known state for the next unit: every issued stage was
+    // consumed, so the parity bits already describe the next phases.
+    if (AGG) {
+      const size_t o = (((size_t)b * p.S + seg) * p.D + d) * 16 + n0;
+#pragma unroll
+      for (int s = 0; s < NH; ++s) {
+        *reinterpret_cast<float2*>(p.agg_h + o + 2 * s) = h[s];
+        *reinterpret_cast<float2*>(p.agg_logp + o + 2 * s) = lsum[s];
+      }
+    } else if (p.h_final != nullptr && seg == p.S - 1) {
+      const size_t o = ((size_t)b * p.D + d) * 16 + n0;
+#pragma unroll
+      for (int s = 0; s < NH; ++s) *reinterpret_cast<float2*>(p.h_final + o + 2 * s) = h[s];
+    }
+  }
+}
+
+// Chain the segments: Hin[s] = start state of segment s; Hin[s+1] = 2^{logp[s]} Hin[s] + h_end[s].
+__global__ void scan_carry_kernel(const float* h0, const float* agg_h, const float* agg_logp, float* h_seg, int B,
+                                  int S, int D) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // over (b, d, n)
+  if (i >= (int64_t)B * D * 16) return;
+  const int n = (int)(i % 16);
+  const int d = (int)((i / 16) % D);
+  const int b = (int)(i / (16 * (int64_t)D));
+  float H = h0 != nullptr ? h0[((size_t)b * D + d) * 16 + n] : 0.f;
+  for (int s = 0; s < S; ++s) {
+    const size_t o = (((size_t)b * S + s) * D + d) * 16 + n;
+    h_seg[o] = H;
+    if (s + 1 < S) H = fmaf(ex2_approx(agg_logp[o]), H, agg_h[o]);
+  }
+}
+
+// ---- host ------------------------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+// 3-D map over a [B, L, inner] row-major tensor, box {box_inner, LC, 1}.
+bool map3(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int64_t inner, int64_t L, int64_t B,
+          int box_inner) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)L, (cuuint64_t)B};
+  cuuint64_t str[2] = {(cuuint64_t)(inner * esize), (cuuint64_t)(inner * L * esize)};
+  cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)LC, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, dt, 3, const_cast<void*>(base), dims, str, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+int device_sms() {
+  int dev = 0, n = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+constexpr int kNPoly = 0;  // states per lane whose exp2 runs on the FMA pipe (even, <= NS)
+
+int ns_for(int E) { return E <= 8 ? 8 : 4; }
+
+}  // namespace
+
+// ---- segment plan and workspace ---------------------------------------------------------------------
+ScanPlan scan_fast_plan(int64_t B, int64_t L, int D, int N, int E, int k, bool io_bf16) {
+  ScanPlan pl{};
+  pl.fast = io_bf16 && N == 16 && (k == 1 || k == 2) && E >= 1 && E <= 16;
+  if (!pl.fast) return pl;
+  const int NS = ns_for(E);
+  const int CPW = 32 / (16 / NS);
+  if (D % CPW != 0 || B * L > (int64_t(1) << 31)) {
+    pl.fast = false;
+    return pl;
+  }
+  const int64_t base_units = B * (D / CPW);
+  const int64_t target = (int64_t)device_sms() * 12;
+  int64_t S = 1;
+  if (base_units < target) S = std::min<int64_t>((target + base_units - 1) / base_units, (L + LC - 1) / LC);
+  int64_t Lseg = (L + S - 1) / S;
+  Lseg = (Lseg + LC - 1) / LC * LC;
+  S = (L + Lseg - 1) / Lseg;
+  pl.S = (int)S;
+  pl.Lseg = Lseg;
+  pl.ws_bytes = S > 1 ? (size_t)3 * B * S * D * 16 * sizeof(float) : 0;
+  return pl;
+}
+
+template <int E, int K, int NS>
+static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s) {
+  constexpr int CPW = Geom<NS>::CPW;
+  CUtensorMap tx, tz, td, tb, tc;
+  if (!map3(&tx, sp.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.D, sp.L, sp.B, CPW) ||
+      !map3(&tz, sp.z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.D, sp.L, sp.B, CPW) ||
+      !map3(&td, sp.delta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, sp.D, sp.L, sp.B, CPW) ||
+      !map3(&tb, sp.B_mix, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 16, sp.L, sp.B, 16) ||
+      !map3(&tc, sp.C_mix, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 16, sp.L, sp.B, 16))
+    return cudaErrorInvalidValue;
+  FastParams p{};
+  p.idx = sp.idx;
+  p.gates = sp.gates;
+  p.A = sp.A;
+  p.D_skip = sp.D_skip;
+  p.h0 = sp.h0;
+  p.out = reinterpret_cast<__nv_bfloat16*>(sp.out);
+  p.y_pre = sp.y_pre;
+  p.h_final = sp.h_final;
+  p.status = status;
+  p.L = sp.L;
+  p.Lseg = pl.Lseg;
+  p.B = sp.B;
+  p.D = sp.D;
+  p.E = sp.E;
+  p.k = sp.k;
+  p.S = pl.S;
+  p.seg_count = pl.S;
+  p.units = sp.B * pl.S * (sp.D / CPW);
+  const int sms = device_sms();
+  auto shape = [&](int units, int& ctas, int& warps) {
+    ctas = std::max(1, std::min(sms, units));
+    warps = std::min(kMaxWarps, (units + ctas - 1) / ctas);
+  };
+  int ctas, warps;
+  const size_t smem_per_warp = (size_t)kStages * Stage<NS>::BYTES + (size_t)kStages * 8;
+  const size_t smem = 128 + (size_t)kMaxWarps * smem_per_warp + 16;
+  cudaError_t e;
+  if (pl.S > 1) {
+    float* agg_h = reinterpret_cast<float*>(seg_ws);
+    float* agg_logp = agg_h + (size_t)sp.B * pl.S * sp.D * 16;
+    float* h_seg = agg_logp + (size_t)sp.B * pl.S * sp.D * 16;
+    FastParams a = p;
+    a.agg_h = agg_h;
+    a.agg_logp = agg_logp;
+    a.h0 = nullptr;
+    a.seg_count = pl.S - 1;  // the last segment needs no aggregate
+    a.units = sp.B * (pl.S - 1) * (sp.D / CPW);
+    auto kagg = scan_fast_kernel<E, K, NS, kNPoly, true>;
+    if ((e = cudaFuncSetAttribute(kagg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+      return e;
+    shape(a.units, ctas, warps);
+    kagg<<<ctas, warps * 32, 128 + warps * smem_per_warp + 16, s>>>(tx, tz, td, tb, tc, a);
+    const int64_t n = (int64_t)sp.B * sp.D * 16;
+    scan_carry_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(sp.h0, agg_h, agg_logp, h_seg, sp.B, pl.S, sp.D);
+    note_launch(2);
+    p.h_seg = h_seg;
+  }
+  auto kmain = scan_fast_kernel<E, K, NS, kNPoly, false>;
+  if ((e = cudaFuncSetAttribute(kmain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+    return e;
+  shape(p.units, ctas, warps);
+  kmain<<<ctas, warps * 32, 128 + warps * smem_per_warp + 16, s>>>(tx, tz, td, tb, tc, p);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <int K>
+static cudaError_t fast_by_E(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s) {
+  if (sp.E <= 2) return launch_fast<2, K, 8>(sp, pl, seg_ws, status, s);
+  if (sp.E <= 4) return launch_fast<4, K, 8>(sp, pl, seg_ws, status, s);
+  if (sp.E <= 8) return launch_fast<8, K, 8>(sp, pl, seg_ws, status, s);
+  return launch_fast<16, K, 4>(sp, pl, seg_ws, status, s);
+}
+
+cudaError_t run_scan_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s) {
+  return sp.k == 1 ? fast_by_E<1>(sp, pl, seg_ws, status, s) : fast_by_E<2>(sp, pl, seg_ws, status, s);
+}
+
+}  // namespace swimba
