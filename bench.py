@@ -180,6 +180,22 @@ class GpuLayer:
             ev[3].record(s)
 
 
+def max_over_ranks(value: float, dist, device) -> float:
+    """The max of a per-rank number over all ranks (the job's time is its slowest rank's)."""
+    if dist is None:
+        return float(value)
+    import torch
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Units all ranks processed, divided by the slowest rank's time (weak scaling)."""
+    return units_per_rank_step * steps * world / (max_ms / 1e3)
+
+
 def timed_steps(torch, layer, steps, warmup, dist=None):
     for _ in range(warmup):
         layer.step()
@@ -344,12 +360,8 @@ def main():
     clk = clocks.stop()
     S.check(S.swimba_get_device_status(layer.buf.ws, layer.stream), "device status")
 
-    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
-    tokens = cfg.tokens * args.steps * world
-    value = tokens / (max_ms / 1e3)
+    max_ms = max_over_ranks(total_ms, dist, device)
+    value = whole_job_rate(cfg.tokens, args.steps, world, max_ms)
 
     # switch overhead against the E=1 dense layer of the same shape (same inputs)
     dense = None
@@ -365,10 +377,7 @@ def main():
     e2e = None
     if not args.no_e2e:
         e_ms, h2d, d2h = e2e_steps(torch, S, layer, args.steps, args.warmup, x_host, z_host)
-        et = torch.tensor([e_ms], dtype=torch.float64, device=device)
-        if dist is not None:
-            dist.all_reduce(et, op=dist.ReduceOp.MAX)
-        e2e = {"value": cfg.tokens * args.steps * world / (float(et.item()) / 1e3), "unit": UNIT,
+        e2e = {"value": whole_job_rate(cfg.tokens, args.steps, world, max_over_ranks(e_ms, dist, device)), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     scan_bytes = scan_bytes_per_token(cfg) * cfg.tokens + 4 * cfg.batch * cfg.d_inner * cfg.d_state

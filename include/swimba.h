@@ -135,6 +135,9 @@ swimba_status swimba_get_device_status(void *ws, void *stream);
 /* Static description of a status code. */
 const char *swimba_status_string(swimba_status s);
 
+/* Name and description of the last CUDA error this thread's calls turned into SWIMBA_ERR_CUDA. */
+const char *swimba_last_error_string(void);
+
 /* Number of kernels this library has launched in this process (all devices, all streams). */
 uint64_t swimba_kernel_launches(void);
 

@@ -2,6 +2,7 @@
 // steps run in the kernels of route.cu, proj_simt.cu, proj_tc.cu and scan.cu.
 #include <algorithm>
 #include <atomic>
+#include <cstdio>
 #include <cstring>
 
 #include "common.cuh"
@@ -45,7 +46,13 @@ swimba_status check_dims(const swimba_dims* d) {
   return SWIMBA_OK;
 }
 
-swimba_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SWIMBA_OK : SWIMBA_ERR_CUDA; }
+thread_local char g_last_error[256] = "no error";
+
+swimba_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SWIMBA_OK;
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+  return SWIMBA_ERR_CUDA;
+}
 
 // Shape-only projection parameters (pointers unset), used to pick the path and size workspaces.
 ProjParams proj_shape(const swimba_dims* d) {
@@ -184,6 +191,8 @@ swimba_status swimba_get_device_status(void* ws, void* stream) {
   }
   return SWIMBA_OK;
 }
+
+const char* swimba_last_error_string(void) { return g_last_error; }
 
 uint64_t swimba_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 

@@ -38,7 +38,7 @@ namespace {
 
 constexpr int LC = 16;        // tokens per chunk
 constexpr int kStages = 3;    // ring depth per warp
-constexpr int kMaxWarps = 14; // warps per CTA (registers: 14 * 32 * 144 <= 65536)
+constexpr int kMaxWarps = 16; // warps per CTA (registers: 16 * 32 * 128 = 65536)
 
 template <int NS>
 struct Geom {
@@ -133,7 +133,7 @@ struct FastParams {
 
 // AGG = true: pass 1 (segments 0 .. S-2 only; no readout, no output).
 template <int E, int K, int NS, int NPOLY, bool AGG>
-__global__ void __maxnreg__(144)
+__global__ void __launch_bounds__(kMaxWarps * 32, 1)
     scan_fast_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
                      const __grid_constant__ CUtensorMap tm_dl, const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_c, const FastParams p) {
@@ -492,9 +492,16 @@ static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* s
   p.seg_count = pl.S;
   p.units = sp.B * pl.S * (sp.D / CPW);
   const int sms = device_sms();
-  auto shape = [&](int units, int& ctas, int& warps) {
+  // block size: the kernel's register use decides how many warps a CTA may hold
+  auto shape = [&](const void* fn, int units, int& ctas, int& warps) -> cudaError_t {
+    cudaFuncAttributes fa;
+    cudaError_t err = cudaFuncGetAttributes(&fa, fn);
+    if (err != cudaSuccess) return err;
+    const int wmax = std::max(1, std::min(kMaxWarps, fa.maxThreadsPerBlock / 32));
     ctas = std::max(1, std::min(sms, units));
-    warps = std::min(kMaxWarps, (units + ctas - 1) / ctas);
+    warps = std::min(wmax, (units + ctas - 1) / ctas);
+    if ((int64_t)ctas * warps < units) ctas = std::min<int64_t>((units + warps - 1) / warps, 65535);
+    return cudaSuccess;
   };
   int ctas, warps;
   const size_t smem_per_warp = (size_t)kStages * Stage<NS>::BYTES + (size_t)kStages * 8;
@@ -513,7 +520,7 @@ static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* s
     auto kagg = scan_fast_kernel<E, K, NS, kNPoly, true>;
     if ((e = cudaFuncSetAttribute(kagg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
       return e;
-    shape(a.units, ctas, warps);
+    if ((e = shape((const void*)kagg, a.units, ctas, warps)) != cudaSuccess) return e;
     kagg<<<ctas, warps * 32, 128 + warps * smem_per_warp + 16, s>>>(tx, tz, td, tb, tc, a);
     const int64_t n = (int64_t)sp.B * sp.D * 16;
     scan_carry_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(sp.h0, agg_h, agg_logp, h_seg, sp.B, pl.S, sp.D);
@@ -523,7 +530,7 @@ static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* s
   auto kmain = scan_fast_kernel<E, K, NS, kNPoly, false>;
   if ((e = cudaFuncSetAttribute(kmain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
     return e;
-  shape(p.units, ctas, warps);
+  if ((e = shape((const void*)kmain, p.units, ctas, warps)) != cudaSuccess) return e;
   kmain<<<ctas, warps * 32, 128 + warps * smem_per_warp + 16, s>>>(tx, tz, td, tb, tc, p);
   note_launch();
   return cudaGetLastError();

@@ -48,6 +48,7 @@ EXPORTED = [
     "swimba_get_device_status",
     "swimba_status_string",
     "swimba_kernel_launches",
+    "swimba_last_error_string",
 ]
 
 
@@ -87,6 +88,8 @@ _lib.swimba_get_device_status.argtypes = [_P, _P]
 _lib.swimba_get_device_status.restype = ctypes.c_int
 _lib.swimba_status_string.argtypes = [ctypes.c_int]
 _lib.swimba_status_string.restype = ctypes.c_char_p
+_lib.swimba_last_error_string.argtypes = []
+_lib.swimba_last_error_string.restype = ctypes.c_char_p
 _lib.swimba_kernel_launches.argtypes = []
 _lib.swimba_kernel_launches.restype = ctypes.c_uint64
 
@@ -94,7 +97,8 @@ _lib.swimba_kernel_launches.restype = ctypes.c_uint64
 class SwimbaError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {STATUS.get(status, status)} ({swimba_status_string(status)})")
+        detail = f"; {swimba_last_error_string()}" if status == 5 else ""
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({swimba_status_string(status)}{detail})")
 
 
 def _ptr(t) -> int | None:
@@ -124,6 +128,10 @@ def check(status: int, where: str = "swimba") -> None:
 
 def swimba_status_string(status: int) -> str:
     return _lib.swimba_status_string(int(status)).decode()
+
+
+def swimba_last_error_string() -> str:
+    return _lib.swimba_last_error_string().decode()
 
 
 def swimba_kernel_launches() -> int:
