@@ -6,10 +6,12 @@
 // Figura 2: the state stays on chip, inputs stream from HBM) and "Estado interno puramente lineal"
 // (the linear state admits a scan, used here to split long sequences into segments).
 //
-// Work unit = one warp = CPW channels of one sequence segment; G = 16/NS lanes share a channel and
-// hold NS of its 16 fp32 states in registers. The per-expert transition rows A^e[d, n0..n0+NS)
-// (pre-multiplied by log2 e) also live in registers: every lane of a warp reads the same token, so
-// the selected experts are warp-uniform and a switch on the expert index picks the registers.
+// Work unit = one warp = 16 channels of one sequence segment; 2 lanes share a channel and hold 8 of
+// its 16 fp32 states in registers. The per-expert transition rows A^e[d, n0..n0+8) (pre-multiplied
+// by log2 e) live in tensor memory: each warp owns 128 TMEM columns of its lane quarter and keeps
+// expert e's 8 values of every lane at columns 8e..8e+7. Every lane of a warp reads the same token,
+// so the selected expert is warp-uniform and one tcgen05.ld.32x32b.x8 at column 8e fetches it:
+// a dynamically indexed, branch-free lookup that costs no registers and no shared memory.
 // Per token and state:  arg = Σ_j (Δ g_j) A^{e_j};  ā = 2^arg;  h = ā h + (Δ x) B;  y += C h.
 // The G lanes of a channel then reduce-scatter their partial readouts so that each lane finishes
 // one token: y += D_skip x, out = y z σ(z) (σ via tanh.approx for bf16 outputs).
@@ -38,7 +40,8 @@ namespace {
 
 constexpr int LC = 16;        // tokens per chunk
 constexpr int kStages = 3;    // ring depth per warp
-constexpr int kMaxWarps = 16; // warps per CTA (registers: 16 * 32 * 128 = 65536)
+constexpr int kMaxWarps = 16; // warps per CTA (registers: 16 * 32 * 128 = 65536; TMEM: 4 per lane quarter)
+constexpr int kNS = 8;        // states per lane (2 lanes per channel, 16 channels per warp)
 
 template <int NS>
 struct Geom {
@@ -90,28 +93,6 @@ __device__ __forceinline__ float tanh_approx(float x) {
   return y;
 }
 
-// arg (+)= c * A[e]  for a warp-uniform expert e (registers selected by a switch).
-template <int E, int NH, bool FIRST>
-__device__ __forceinline__ void expert_term(int e, float c, const float2 (&A)[E][NH], float2 (&arg)[NH]) {
-  const float2 cc = make_float2(c, c);
-#define SWIMBA_EXPERT_CASE(i)                                                  \
-  case i:                                                                      \
-    if constexpr (i < E) {                                                     \
-      _Pragma("unroll") for (int s = 0; s < NH; ++s) arg[s] =                  \
-          FIRST ? __fmul2_rn(cc, A[i][s]) : __ffma2_rn(cc, A[i][s], arg[s]);   \
-    }                                                                          \
-    break;
-  switch (e) {
-    SWIMBA_EXPERT_CASE(0) SWIMBA_EXPERT_CASE(1) SWIMBA_EXPERT_CASE(2) SWIMBA_EXPERT_CASE(3)
-    SWIMBA_EXPERT_CASE(4) SWIMBA_EXPERT_CASE(5) SWIMBA_EXPERT_CASE(6) SWIMBA_EXPERT_CASE(7)
-    SWIMBA_EXPERT_CASE(8) SWIMBA_EXPERT_CASE(9) SWIMBA_EXPERT_CASE(10) SWIMBA_EXPERT_CASE(11)
-    SWIMBA_EXPERT_CASE(12) SWIMBA_EXPERT_CASE(13) SWIMBA_EXPERT_CASE(14) SWIMBA_EXPERT_CASE(15)
-    default:
-      break;
-  }
-#undef SWIMBA_EXPERT_CASE
-}
-
 struct FastParams {
   const int32_t* idx;
   const float* gates;
@@ -132,11 +113,12 @@ struct FastParams {
 };
 
 // AGG = true: pass 1 (segments 0 .. S-2 only; no readout, no output).
-template <int E, int K, int NS, int NPOLY, bool AGG>
+template <int K, int NPOLY, bool AGG>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1)
     scan_fast_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
                      const __grid_constant__ CUtensorMap tm_dl, const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_c, const FastParams p) {
+  constexpr int NS = kNS;
   constexpr int G = Geom<NS>::G;
   constexpr int CPW = Geom<NS>::CPW;
   constexpr int NH = NS / 2;
@@ -146,9 +128,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwarps = blockDim.x >> 5;
   uint8_t* ring = smem + (size_t)warp * kStages * St::BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)nwarps * kStages * St::BYTES) + warp * kStages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(
-      reinterpret_cast<uint64_t*>(smem + (size_t)nwarps * kStages * St::BYTES) + nwarps * kStages);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)nwarps * kStages * St::BYTES);
+  uint64_t* full = bars + warp * kStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + nwarps * kStages);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + nwarps * kStages) + 1;
 
   if (lane == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
@@ -164,7 +147,14 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       }
     }
   }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
   __syncthreads();
+  tc_fence_after();
+  // this warp's TMEM window: its lane quarter, 128 columns
+  const uint32_t tbase = *tmem_slot + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(warp >> 2) * 128u;
 
   const int cl = lane / G;  // channel within the warp
   const int gi = lane % G;  // state group
@@ -186,19 +176,18 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
     const int64_t t_end = std::min<int64_t>(p.L, t_begin + p.Lseg);
     const int nchunks = (int)((t_end - t_begin + LC - 1) / LC);
 
-    // per-expert transition rows of this lane's states, times log2(e)
-    float2 A[E][NH];
-#pragma unroll
-    for (int e = 0; e < E; ++e)
-#pragma unroll
-      for (int s = 0; s < NH; ++s) {
-        if (e < p.E) {
-          const float2 a = *reinterpret_cast<const float2*>(p.A + ((size_t)e * p.D + d) * 16 + n0 + 2 * s);
-          A[e][s] = make_float2(a.x * kLog2e, a.y * kLog2e);
-        } else {
-          A[e][s] = make_float2(0.f, 0.f);
-        }
-      }
+    // per-expert transition rows of this lane's states, times log2(e), into TMEM columns 8e..8e+7
+    for (int e = 0; e < p.E; ++e) {
+      const float4* src = reinterpret_cast<const float4*>(p.A + ((size_t)e * p.D + d) * 16 + n0);
+      const float4 a0 = __ldg(src), a1 = __ldg(src + 1);
+      const uint32_t r[8] = {__float_as_uint(a0.x * kLog2e), __float_as_uint(a0.y * kLog2e),
+                             __float_as_uint(a0.z * kLog2e), __float_as_uint(a0.w * kLog2e),
+                             __float_as_uint(a1.x * kLog2e), __float_as_uint(a1.y * kLog2e),
+                             __float_as_uint(a1.z * kLog2e), __float_as_uint(a1.w * kLog2e)};
+      tmem_st8(tbase + (uint32_t)e * NS, r);
+    }
+    tmem_wait_st();
+
     float2 h[NH];
     const float* hs = AGG ? nullptr
                           : (p.h_seg != nullptr ? p.h_seg + (((size_t)b * p.S + seg) * p.D + d) * 16
@@ -271,16 +260,36 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       const int64_t t0 = t_begin + (int64_t)c * LC;
 #pragma unroll 1
       for (int tt = 0; tt < LC; tt += G) {
+        // the selected experts' A rows of the G tokens, from TMEM
+        int4 m[G];
+        uint32_t a0r[G][8], a1r[G][8];
+#pragma unroll
+        for (int uu = 0; uu < G; ++uu) {
+          m[uu] = meta[tt + uu];
+          tmem_ld8_nowait(tbase + (uint32_t)m[uu].x * NS, a0r[uu]);
+          if (K == 2) tmem_ld8_nowait(tbase + (uint32_t)m[uu].y * NS, a1r[uu]);
+        }
+        tmem_wait_ld();
         float yp[G];
 #pragma unroll
         for (int uu = 0; uu < G; ++uu) {
           const int t = tt + uu;
-          const int4 m = meta[t];
           const float dlt = ds[t * CPW + cl];
           const float xv = __bfloat162float(xs[t * CPW + cl]);
+          const float c0 = dlt * __int_as_float(m[uu].z);
+          const float2 cc0 = make_float2(c0, c0);
           float2 arg[NH];
-          expert_term<E, NH, true>(m.x, dlt * __int_as_float(m.z), A, arg);
-          if (K == 2) expert_term<E, NH, false>(m.y, dlt * __int_as_float(m.w), A, arg);
+#pragma unroll
+          for (int s = 0; s < NH; ++s)
+            arg[s] = __fmul2_rn(cc0, make_float2(__uint_as_float(a0r[uu][2 * s]), __uint_as_float(a0r[uu][2 * s + 1])));
+          if (K == 2) {
+            const float c1 = dlt * __int_as_float(m[uu].w);
+            const float2 cc1 = make_float2(c1, c1);
+#pragma unroll
+            for (int s = 0; s < NH; ++s)
+              arg[s] = __ffma2_rn(cc1, make_float2(__uint_as_float(a1r[uu][2 * s]), __uint_as_float(a1r[uu][2 * s + 1])),
+                                  arg[s]);
+          }
           float2 a[NH];
 #pragma unroll
           for (int s = 0; s < NH; ++s) {
@@ -305,32 +314,22 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
 #pragma unroll
             for (int s = 0; s < NH; ++s) lsum[s] = __fadd2_rn(lsum[s], arg[s]);
           } else {
-            float2 y2 = make_float2(0.f, 0.f);
+            float2 y2a = make_float2(0.f, 0.f), y2b = make_float2(0.f, 0.f);
 #pragma unroll
             for (int q = 0; q < NS / 4; ++q) {
               const float4 c4 = csm[t * 4 + gi * (NS / 4) + q];
-              y2 = __ffma2_rn(make_float2(c4.x, c4.y), h[2 * q], y2);
-              y2 = __ffma2_rn(make_float2(c4.z, c4.w), h[2 * q + 1], y2);
+              y2a = __ffma2_rn(make_float2(c4.x, c4.y), h[2 * q], y2a);
+              y2b = __ffma2_rn(make_float2(c4.z, c4.w), h[2 * q + 1], y2b);
             }
-            yp[uu] = y2.x + y2.y;
+            yp[uu] = (y2a.x + y2b.x) + (y2a.y + y2b.y);
           }
         }
         if (!AGG) {
-          // reduce-scatter the partial readouts over the G lanes of the channel: lane gi ends
-          // with the full y of token tt + gi
-          float ysum;
-          if (G == 2) {
-            const float send = gi == 0 ? yp[1 % G] : yp[0];
-            const float keep = gi == 0 ? yp[0] : yp[1 % G];
-            ysum = keep + __shfl_xor_sync(0xffffffffu, send, 1);
-          } else {
-            const bool lo = gi < 2;
-            const float s0 = lo ? yp[2 % G] : yp[0], s1 = lo ? yp[3 % G] : yp[1 % G];
-            const float k0 = (lo ? yp[0] : yp[2 % G]) + __shfl_xor_sync(0xffffffffu, s0, 2);
-            const float k1 = (lo ? yp[1 % G] : yp[3 % G]) + __shfl_xor_sync(0xffffffffu, s1, 2);
-            const bool odd = gi & 1;
-            ysum = (odd ? k1 : k0) + __shfl_xor_sync(0xffffffffu, odd ? k0 : k1, 1);
-          }
+          // the two lanes of a channel swap half of their partial readouts: lane gi ends with the
+          // full y of token tt + gi
+          const float send = gi == 0 ? yp[1] : yp[0];
+          const float keep = gi == 0 ? yp[0] : yp[1];
+          const float ysum = keep + __shfl_xor_sync(0xffffffffu, send, 1);
           const int t = tt + gi;
           if (t0 + t < t_end) {
             const float xv = __bfloat162float(xs[t * CPW + cl]);
@@ -345,9 +344,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       }
       __syncwarp();
       if (c + kStages < nchunks) {
-        const int4 m = meta_next;
+        const int4 mm = meta_next;
         meta_next = load_meta(c + kStages + 1);
-        issue(c + kStages, m);
+        issue(c + kStages, mm);
         ++issued;
       }
     }
@@ -365,8 +364,6 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       }
       break;
     }
-    // stage parity must restart at a known state for the next unit: every issued stage was
-    // consumed, so the parity bits already describe the next phases.
     if (AGG) {
       const size_t o = (((size_t)b * p.S + seg) * p.D + d) * 16 + n0;
 #pragma unroll
@@ -379,6 +376,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
 #pragma unroll
       for (int s = 0; s < NH; ++s) *reinterpret_cast<float2*>(p.h_final + o + 2 * s) = h[s];
     }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(*tmem_slot, 512);
   }
 }
 
@@ -434,8 +436,6 @@ int device_sms() {
 
 constexpr int kNPoly = 0;  // states per lane whose exp2 runs on the FMA pipe (even, <= NS)
 
-int ns_for(int E) { return E <= 8 ? 8 : 4; }
-
 }  // namespace
 
 // ---- segment plan and workspace ---------------------------------------------------------------------
@@ -443,8 +443,7 @@ ScanPlan scan_fast_plan(int64_t B, int64_t L, int D, int N, int E, int k, bool i
   ScanPlan pl{};
   pl.fast = io_bf16 && N == 16 && (k == 1 || k == 2) && E >= 1 && E <= 16;
   if (!pl.fast) return pl;
-  const int NS = ns_for(E);
-  const int CPW = 32 / (16 / NS);
+  const int CPW = Geom<kNS>::CPW;
   if (D % CPW != 0 || B * L > (int64_t(1) << 31)) {
     pl.fast = false;
     return pl;
@@ -462,8 +461,9 @@ ScanPlan scan_fast_plan(int64_t B, int64_t L, int D, int N, int E, int k, bool i
   return pl;
 }
 
-template <int E, int K, int NS>
+template <int K>
 static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s) {
+  constexpr int NS = kNS;
   constexpr int CPW = Geom<NS>::CPW;
   CUtensorMap tx, tz, td, tb, tc;
   if (!map3(&tx, sp.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.D, sp.L, sp.B, CPW) ||
@@ -505,7 +505,7 @@ static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* s
   };
   int ctas, warps;
   const size_t smem_per_warp = (size_t)kStages * Stage<NS>::BYTES + (size_t)kStages * 8;
-  const size_t smem = 128 + (size_t)kMaxWarps * smem_per_warp + 16;
+  const size_t smem = 128 + (size_t)kMaxWarps * smem_per_warp + 32;
   cudaError_t e;
   if (pl.S > 1) {
     float* agg_h = reinterpret_cast<float*>(seg_ws);
@@ -517,35 +517,27 @@ static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* s
     a.h0 = nullptr;
     a.seg_count = pl.S - 1;  // the last segment needs no aggregate
     a.units = sp.B * (pl.S - 1) * (sp.D / CPW);
-    auto kagg = scan_fast_kernel<E, K, NS, kNPoly, true>;
+    auto kagg = scan_fast_kernel<K, kNPoly, true>;
     if ((e = cudaFuncSetAttribute(kagg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
       return e;
     if ((e = shape((const void*)kagg, a.units, ctas, warps)) != cudaSuccess) return e;
-    kagg<<<ctas, warps * 32, 128 + warps * smem_per_warp + 16, s>>>(tx, tz, td, tb, tc, a);
+    kagg<<<ctas, warps * 32, 128 + warps * smem_per_warp + 32, s>>>(tx, tz, td, tb, tc, a);
     const int64_t n = (int64_t)sp.B * sp.D * 16;
     scan_carry_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(sp.h0, agg_h, agg_logp, h_seg, sp.B, pl.S, sp.D);
     note_launch(2);
     p.h_seg = h_seg;
   }
-  auto kmain = scan_fast_kernel<E, K, NS, kNPoly, false>;
+  auto kmain = scan_fast_kernel<K, kNPoly, false>;
   if ((e = cudaFuncSetAttribute(kmain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
     return e;
   if ((e = shape((const void*)kmain, p.units, ctas, warps)) != cudaSuccess) return e;
-  kmain<<<ctas, warps * 32, 128 + warps * smem_per_warp + 16, s>>>(tx, tz, td, tb, tc, p);
+  kmain<<<ctas, warps * 32, 128 + warps * smem_per_warp + 32, s>>>(tx, tz, td, tb, tc, p);
   note_launch();
   return cudaGetLastError();
 }
 
-template <int K>
-static cudaError_t fast_by_E(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s) {
-  if (sp.E <= 2) return launch_fast<2, K, 8>(sp, pl, seg_ws, status, s);
-  if (sp.E <= 4) return launch_fast<4, K, 8>(sp, pl, seg_ws, status, s);
-  if (sp.E <= 8) return launch_fast<8, K, 8>(sp, pl, seg_ws, status, s);
-  return launch_fast<16, K, 4>(sp, pl, seg_ws, status, s);
-}
-
 cudaError_t run_scan_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s) {
-  return sp.k == 1 ? fast_by_E<1>(sp, pl, seg_ws, status, s) : fast_by_E<2>(sp, pl, seg_ws, status, s);
+  return sp.k == 1 ? launch_fast<1>(sp, pl, seg_ws, status, s) : launch_fast<2>(sp, pl, seg_ws, status, s);
 }
 
 }  // namespace swimba
