@@ -6,20 +6,23 @@
 // Figura 2: the state stays on chip, inputs stream from HBM) and "Estado interno puramente lineal"
 // (the linear state admits a scan, used here to split long sequences into segments).
 //
-// Work unit = one warp = 16 channels of one sequence segment; 2 lanes share a channel and hold 8 of
-// its 16 fp32 states in registers. The per-expert transition rows A^e[d, n0..n0+8) (pre-multiplied
-// by log2 e) live in tensor memory: each warp owns 128 TMEM columns of its lane quarter and keeps
-// expert e's 8 values of every lane at columns 8e..8e+7. Every lane of a warp reads the same token,
-// so the selected expert is warp-uniform and one tcgen05.ld.32x32b.x8 at column 8e fetches it:
-// a dynamically indexed, branch-free lookup that costs no registers and no shared memory.
+// Work unit = one warp = 32 channels of one sequence segment. Lane l holds the channel pair
+// (2*(l>>1), 2*(l>>1)+1) of the warp and the 8 states (l&1)*8 .. +7 of both channels, 16 fp32 states
+// in registers; the two lanes of a pair together hold all 16 states of the two channels. So every
+// B_mix / C_mix value a lane loads serves two channels, and one shuffle finishes the readout.
+// The per-expert transition rows (pre-multiplied by log2 e) live in tensor memory: each warp owns
+// E*16 TMEM columns of its lane quarter and keeps expert e's 16 values of every lane at columns
+// 16e..16e+15. Every lane of a warp reads the same token, so the selected expert is warp-uniform
+// and one tcgen05.ld.32x32b.x16 at column 16e fetches it: a dynamically indexed, branch-free lookup
+// that costs no registers and no shared-memory bandwidth.
 // Per token and state:  arg = Σ_j (Δ g_j) A^{e_j};  ā = 2^arg;  h = ā h + (Δ x) B;  y += C h.
-// The G lanes of a channel then reduce-scatter their partial readouts so that each lane finishes
-// one token: y += D_skip x, out = y z σ(z) (σ via tanh.approx for bf16 outputs).
+// The two lanes of a pair swap one partial readout so that each finishes one channel's token:
+// y += D_skip x, out = y z σ(z) (σ via tanh.approx for bf16 outputs).
 //
 // Each warp streams its inputs through its own 3-stage shared-memory ring filled by TMA (x, z, Δ
-// tiles of [16 tokens x CPW channels] and B_mix, C_mix rows of 16 tokens) plus the tokens' expert
+// tiles of [16 tokens x 32 channels] and B_mix, C_mix rows of 16 tokens) plus the tokens' expert
 // indices and gates written by the warp's lanes one chunk ahead. Units are spread evenly over one
-// persistent CTA per SM (up to 14 warps each), so no SM gets a whole extra sequence.
+// persistent CTA per SM, so no SM gets a whole extra sequence.
 //
 // Segments (when B*D alone cannot fill the GPU): pass 1 computes, per segment, the end state from
 // zero and log2 of the decay product Σ_t Δ_t A_t; a carry pass chains them into each segment's
@@ -38,25 +41,17 @@ using namespace sm100;
 
 namespace {
 
-constexpr int LC = 16;        // tokens per chunk
-constexpr int kStages = 3;    // ring depth per warp
-constexpr int kMaxWarps = 16; // warps per CTA (registers: 16 * 32 * 128 = 65536; TMEM: 4 per lane quarter)
-constexpr int kNS = 8;        // states per lane (2 lanes per channel, 16 channels per warp)
-
-template <int NS>
-struct Geom {
-  static constexpr int G = 16 / NS;    // lanes per channel
-  static constexpr int CPW = 32 / G;   // channels per warp
-};
+constexpr int LC = 16;          // tokens per chunk
+constexpr int kStages = 3;      // ring depth per warp
+constexpr int kCPW = 32;        // channels per warp
+constexpr int kMaxWarps = 8;    // warps per CTA (registers: up to 255 per thread)
 
 // Byte offsets inside one ring stage of one warp.
-template <int NS>
 struct Stage {
-  static constexpr int CPW = Geom<NS>::CPW;
-  static constexpr int X = 0;                      // bf16 [LC][CPW]
-  static constexpr int Z = X + LC * CPW * 2;       // bf16 [LC][CPW]
-  static constexpr int DL = Z + LC * CPW * 2;      // f32  [LC][CPW]
-  static constexpr int B = DL + LC * CPW * 4;      // f32  [LC][16]
+  static constexpr int X = 0;                      // bf16 [LC][32]
+  static constexpr int Z = X + LC * kCPW * 2;      // bf16 [LC][32]
+  static constexpr int DL = Z + LC * kCPW * 2;     // f32  [LC][32]
+  static constexpr int B = DL + LC * kCPW * 4;     // f32  [LC][16]
   static constexpr int C = B + LC * 16 * 4;        // f32  [LC][16]
   static constexpr int META = C + LC * 16 * 4;     // int4 [LC] {e0, e1, g0, g1}
   static constexpr int BYTES = META + LC * 16;
@@ -64,6 +59,9 @@ struct Stage {
                 "TMA destinations must be 128-byte aligned");
   static_assert(BYTES % 128 == 0, "stage size");
 };
+
+// TMEM columns one warp needs (16 per expert) and how many warps share a lane quarter's 512.
+__host__ __device__ constexpr int tmem_cols_per_warp(int E) { return ((E * 16 + 31) / 32) * 32; }
 
 // 2^x on the FMA pipe for x <= 0: x = j + f with j = round(x) (the 1.5*2^23 shifter), f in
 // [-1/2, 1/2]; 2^f by a degree-5 polynomial fitted for minimax relative error on that interval
@@ -118,11 +116,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
     scan_fast_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
                      const __grid_constant__ CUtensorMap tm_dl, const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_c, const FastParams p) {
-  constexpr int NS = kNS;
-  constexpr int G = Geom<NS>::G;
-  constexpr int CPW = Geom<NS>::CPW;
-  constexpr int NH = NS / 2;
-  using St = Stage<NS>;
+  using St = Stage;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -153,51 +147,63 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
   }
   __syncthreads();
   tc_fence_after();
-  // this warp's TMEM window: its lane quarter, 128 columns
-  const uint32_t tbase = *tmem_slot + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(warp >> 2) * 128u;
+  // this warp's TMEM window: its lane quarter, tmem_cols_per_warp(E) columns
+  const uint32_t tbase = *tmem_slot + ((uint32_t)(32 * (warp & 3)) << 16) +
+                         (uint32_t)(warp >> 2) * (uint32_t)tmem_cols_per_warp(p.E);
 
-  const int cl = lane / G;  // channel within the warp
-  const int gi = lane % G;  // state group
-  const int n0 = gi * NS;
-  const int ntiles = p.D / CPW;
+  const int cp = lane >> 1;   // channel pair: channels 2cp, 2cp+1 of the warp's 32
+  const int gi = lane & 1;    // state group: states 8gi .. 8gi+7
+  const int n0 = gi * 8;
+  const int ntiles = p.D / kCPW;
   const int u_begin = (int)((int64_t)p.units * blockIdx.x / gridDim.x);
   const int u_end = (int)((int64_t)p.units * (blockIdx.x + 1) / gridDim.x);
   uint32_t phase_bits = 0;  // one parity bit per stage
-  constexpr uint32_t tx_bytes = AGG ? (LC * CPW * 2 + LC * CPW * 4 + LC * 16 * 4)
-                                    : (2 * LC * CPW * 2 + LC * CPW * 4 + 2 * LC * 16 * 4);
+  constexpr uint32_t tx_bytes = AGG ? (LC * kCPW * 2 + LC * kCPW * 4 + LC * 16 * 4)
+                                    : (2 * LC * kCPW * 2 + LC * kCPW * 4 + 2 * LC * 16 * 4);
 
   for (int u = u_begin + warp; u < u_end; u += nwarps) {
     const int tile = u % ntiles;
     const int bs = u / ntiles;  // b * seg_count + seg
     const int seg = bs % p.seg_count;
     const int b = bs / p.seg_count;
-    const int d = tile * CPW + cl;
+    const int dA = tile * kCPW + 2 * cp;  // this lane's channels dA, dA + 1
     const int64_t t_begin = (int64_t)seg * p.Lseg;
     const int64_t t_end = std::min<int64_t>(p.L, t_begin + p.Lseg);
     const int nchunks = (int)((t_end - t_begin + LC - 1) / LC);
 
-    // per-expert transition rows of this lane's states, times log2(e), into TMEM columns 8e..8e+7
+    // per-expert transition rows of this lane's 2 x 8 states, times log2(e), into TMEM 16e..16e+15
     for (int e = 0; e < p.E; ++e) {
-      const float4* src = reinterpret_cast<const float4*>(p.A + ((size_t)e * p.D + d) * 16 + n0);
-      const float4 a0 = __ldg(src), a1 = __ldg(src + 1);
-      const uint32_t r[8] = {__float_as_uint(a0.x * kLog2e), __float_as_uint(a0.y * kLog2e),
-                             __float_as_uint(a0.z * kLog2e), __float_as_uint(a0.w * kLog2e),
-                             __float_as_uint(a1.x * kLog2e), __float_as_uint(a1.y * kLog2e),
-                             __float_as_uint(a1.z * kLog2e), __float_as_uint(a1.w * kLog2e)};
-      tmem_st8(tbase + (uint32_t)e * NS, r);
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        const float4* src = reinterpret_cast<const float4*>(p.A + ((size_t)e * p.D + dA + ch) * 16 + n0);
+        const float4 a0 = __ldg(src), a1 = __ldg(src + 1);
+        const uint32_t r[8] = {__float_as_uint(a0.x * kLog2e), __float_as_uint(a0.y * kLog2e),
+                               __float_as_uint(a0.z * kLog2e), __float_as_uint(a0.w * kLog2e),
+                               __float_as_uint(a1.x * kLog2e), __float_as_uint(a1.y * kLog2e),
+                               __float_as_uint(a1.z * kLog2e), __float_as_uint(a1.w * kLog2e)};
+        tmem_st8(tbase + (uint32_t)e * 16u + (uint32_t)ch * 8u, r);
+      }
     }
     tmem_wait_st();
 
-    float2 h[NH];
-    const float* hs = AGG ? nullptr
-                          : (p.h_seg != nullptr ? p.h_seg + (((size_t)b * p.S + seg) * p.D + d) * 16
-                                                : (p.h0 != nullptr && seg == 0 ? p.h0 + ((size_t)b * p.D + d) * 16 : nullptr));
+    float2 h[2][4];  // [channel][state pair]
 #pragma unroll
-    for (int s = 0; s < NH; ++s) h[s] = hs ? *reinterpret_cast<const float2*>(hs + n0 + 2 * s) : make_float2(0.f, 0.f);
-    float2 lsum[NH];
+    for (int ch = 0; ch < 2; ++ch) {
+      const float* hs = AGG ? nullptr
+                            : (p.h_seg != nullptr ? p.h_seg + (((size_t)b * p.S + seg) * p.D + dA + ch) * 16
+                                                  : (p.h0 != nullptr && seg == 0 ? p.h0 + ((size_t)b * p.D + dA + ch) * 16
+                                                                                 : nullptr));
 #pragma unroll
-    for (int s = 0; s < NH; ++s) lsum[s] = make_float2(0.f, 0.f);
-    const float dsk = AGG ? 0.f : p.D_skip[d];
+      for (int s = 0; s < 4; ++s)
+        h[ch][s] = hs ? *reinterpret_cast<const float2*>(hs + n0 + 2 * s) : make_float2(0.f, 0.f);
+    }
+    float2 lsum[2][4];
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+      for (int s = 0; s < 4; ++s) lsum[ch][s] = make_float2(0.f, 0.f);
+    const int dmine = dA + gi;  // the channel whose outputs this lane writes
+    const float dsk = AGG ? 0.f : p.D_skip[dmine];
 
     // meta of one chunk: lane t (< LC) holds token t's {e0, e1, g0, g1}
     auto load_meta = [&](int c) -> int4 {
@@ -224,11 +230,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
         uint64_t* bar = &full[c % kStages];
         mbar_arrive_expect_tx(bar, tx_bytes);
         const int t0 = (int)(t_begin + (int64_t)c * LC);
-        tma_load_3d(st + St::X, &tm_x, bar, tile * CPW, t0, b);
-        tma_load_3d(st + St::DL, &tm_dl, bar, tile * CPW, t0, b);
+        tma_load_3d(st + St::X, &tm_x, bar, tile * kCPW, t0, b);
+        tma_load_3d(st + St::DL, &tm_dl, bar, tile * kCPW, t0, b);
         tma_load_3d(st + St::B, &tm_b, bar, 0, t0, b);
         if (!AGG) {
-          tma_load_3d(st + St::Z, &tm_z, bar, tile * CPW, t0, b);
+          tma_load_3d(st + St::Z, &tm_z, bar, tile * kCPW, t0, b);
           tma_load_3d(st + St::C, &tm_c, bar, 0, t0, b);
         }
       }
@@ -252,93 +258,111 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       phase_bits ^= 1u << sidx;
       const uint8_t* st = ring + sidx * St::BYTES;
       const int4* meta = reinterpret_cast<const int4*>(st + St::META);
-      const __nv_bfloat16* xs = reinterpret_cast<const __nv_bfloat16*>(st + St::X);
+      const __nv_bfloat162* xs2 = reinterpret_cast<const __nv_bfloat162*>(st + St::X);
       const __nv_bfloat16* zs = reinterpret_cast<const __nv_bfloat16*>(st + St::Z);
-      const float* ds = reinterpret_cast<const float*>(st + St::DL);
+      const float2* ds2 = reinterpret_cast<const float2*>(st + St::DL);
       const float4* bsm = reinterpret_cast<const float4*>(st + St::B);
       const float4* csm = reinterpret_cast<const float4*>(st + St::C);
       const int64_t t0 = t_begin + (int64_t)c * LC;
+      const bool full_chunk = t0 + LC <= t_end;
+      __nv_bfloat16* outp = AGG ? nullptr : p.out + ((size_t)b * p.L + t0) * p.D + dmine;
+      float* ypp = (AGG || p.y_pre == nullptr) ? nullptr : p.y_pre + ((size_t)b * p.L + t0) * p.D + dmine;
 #pragma unroll 1
-      for (int tt = 0; tt < LC; tt += G) {
-        // the selected experts' A rows of the G tokens, from TMEM
-        int4 m[G];
-        uint32_t a0r[G][8], a1r[G][8];
+      for (int t = 0; t < LC; t += 2) {
+        // loads of both tokens first: the selected experts' A rows (TMEM), Δ, x, B, C (smem)
+        int4 m[2];
+        uint32_t ar[2][2][16];  // [token][expert slot][16 values]
+        float2 dl[2], xv[2];
+        float2 bv[2][4], cv[2][4];
 #pragma unroll
-        for (int uu = 0; uu < G; ++uu) {
-          m[uu] = meta[tt + uu];
-          tmem_ld8_nowait(tbase + (uint32_t)m[uu].x * NS, a0r[uu]);
-          if (K == 2) tmem_ld8_nowait(tbase + (uint32_t)m[uu].y * NS, a1r[uu]);
+        for (int u = 0; u < 2; ++u) {
+          m[u] = meta[t + u];
+          tmem_ld16_nowait(tbase + (uint32_t)m[u].x * 16u, ar[u][0]);
+          if (K == 2) tmem_ld16_nowait(tbase + (uint32_t)m[u].y * 16u, ar[u][1]);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          dl[u] = ds2[(t + u) * (kCPW / 2) + cp];
+          xv[u] = __bfloat1622float2(xs2[(t + u) * (kCPW / 2) + cp]);
+          const float4 bq0 = bsm[(t + u) * 4 + 2 * gi], bq1 = bsm[(t + u) * 4 + 2 * gi + 1];
+          bv[u][0] = make_float2(bq0.x, bq0.y);
+          bv[u][1] = make_float2(bq0.z, bq0.w);
+          bv[u][2] = make_float2(bq1.x, bq1.y);
+          bv[u][3] = make_float2(bq1.z, bq1.w);
+          if (!AGG) {
+            const float4 cq0 = csm[(t + u) * 4 + 2 * gi], cq1 = csm[(t + u) * 4 + 2 * gi + 1];
+            cv[u][0] = make_float2(cq0.x, cq0.y);
+            cv[u][1] = make_float2(cq0.z, cq0.w);
+            cv[u][2] = make_float2(cq1.x, cq1.y);
+            cv[u][3] = make_float2(cq1.z, cq1.w);
+          }
         }
         tmem_wait_ld();
-        float yp[G];
+        // decay factors of both tokens (independent of the state)
+        float2 a[2][2][4];  // [token][channel][state pair]
+        float2 arg[2][2][4];
 #pragma unroll
-        for (int uu = 0; uu < G; ++uu) {
-          const int t = tt + uu;
-          const float dlt = ds[t * CPW + cl];
-          const float xv = __bfloat162float(xs[t * CPW + cl]);
-          const float c0 = dlt * __int_as_float(m[uu].z);
-          const float2 cc0 = make_float2(c0, c0);
-          float2 arg[NH];
+        for (int u = 0; u < 2; ++u)
 #pragma unroll
-          for (int s = 0; s < NH; ++s)
-            arg[s] = __fmul2_rn(cc0, make_float2(__uint_as_float(a0r[uu][2 * s]), __uint_as_float(a0r[uu][2 * s + 1])));
-          if (K == 2) {
-            const float c1 = dlt * __int_as_float(m[uu].w);
-            const float2 cc1 = make_float2(c1, c1);
+          for (int ch = 0; ch < 2; ++ch) {
+            const float dlt = ch == 0 ? dl[u].x : dl[u].y;
+            const float c0 = dlt * __int_as_float(m[u].z);
+            const float c1 = dlt * __int_as_float(m[u].w);
 #pragma unroll
-            for (int s = 0; s < NH; ++s)
-              arg[s] = __ffma2_rn(cc1, make_float2(__uint_as_float(a1r[uu][2 * s]), __uint_as_float(a1r[uu][2 * s + 1])),
-                                  arg[s]);
+            for (int s = 0; s < 4; ++s) {
+              const float2 a0 = make_float2(__uint_as_float(ar[u][0][ch * 8 + 2 * s]), __uint_as_float(ar[u][0][ch * 8 + 2 * s + 1]));
+              arg[u][ch][s] = __fmul2_rn(make_float2(c0, c0), a0);
+              if (K == 2) {
+                const float2 a1 =
+                    make_float2(__uint_as_float(ar[u][1][ch * 8 + 2 * s]), __uint_as_float(ar[u][1][ch * 8 + 2 * s + 1]));
+                arg[u][ch][s] = __ffma2_rn(make_float2(c1, c1), a1, arg[u][ch][s]);
+              }
+              if (s >= 4 - NPOLY / 2) {
+                a[u][ch][s] = exp2_poly2(arg[u][ch][s]);
+              } else {
+                a[u][ch][s] = make_float2(ex2_approx(arg[u][ch][s].x), ex2_approx(arg[u][ch][s].y));
+              }
+            }
           }
-          float2 a[NH];
+        // the recurrence, token t then t+1
+        float ysum[2];
 #pragma unroll
-          for (int s = 0; s < NH; ++s) {
-            if (s >= NH - NPOLY / 2) {
-              a[s] = exp2_poly2(arg[s]);
+        for (int u = 0; u < 2; ++u) {
+          float ych[2];
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            const float dx = (ch == 0 ? dl[u].x : dl[u].y) * (ch == 0 ? xv[u].x : xv[u].y);
+            const float2 dxx = make_float2(dx, dx);
+#pragma unroll
+            for (int s = 0; s < 4; ++s) h[ch][s] = __ffma2_rn(a[u][ch][s], h[ch][s], __fmul2_rn(dxx, bv[u][s]));
+            if (AGG) {
+#pragma unroll
+              for (int s = 0; s < 4; ++s) lsum[ch][s] = __fadd2_rn(lsum[ch][s], arg[u][ch][s]);
             } else {
-              a[s] = make_float2(ex2_approx(arg[s].x), ex2_approx(arg[s].y));
+              const float2 ya = __ffma2_rn(cv[u][1], h[ch][1], __fmul2_rn(cv[u][0], h[ch][0]));
+              const float2 yb = __ffma2_rn(cv[u][3], h[ch][3], __fmul2_rn(cv[u][2], h[ch][2]));
+              ych[ch] = (ya.x + yb.x) + (ya.y + yb.y);
             }
           }
-          const float dx = dlt * xv;
-          const float2 dxx = make_float2(dx, dx);
-          float2 bv[NH];
-#pragma unroll
-          for (int q = 0; q < NS / 4; ++q) {
-            const float4 b4 = bsm[t * 4 + gi * (NS / 4) + q];
-            bv[2 * q] = make_float2(b4.x, b4.y);
-            bv[2 * q + 1] = make_float2(b4.z, b4.w);
-          }
-#pragma unroll
-          for (int s = 0; s < NH; ++s) h[s] = __ffma2_rn(a[s], h[s], __fmul2_rn(dxx, bv[s]));
-          if (AGG) {
-#pragma unroll
-            for (int s = 0; s < NH; ++s) lsum[s] = __fadd2_rn(lsum[s], arg[s]);
-          } else {
-            float2 y2a = make_float2(0.f, 0.f), y2b = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int q = 0; q < NS / 4; ++q) {
-              const float4 c4 = csm[t * 4 + gi * (NS / 4) + q];
-              y2a = __ffma2_rn(make_float2(c4.x, c4.y), h[2 * q], y2a);
-              y2b = __ffma2_rn(make_float2(c4.z, c4.w), h[2 * q + 1], y2b);
-            }
-            yp[uu] = (y2a.x + y2b.x) + (y2a.y + y2b.y);
+          if (!AGG) {
+            // lanes 2cp (states 0-7) and 2cp+1 (states 8-15) swap one partial: lane gi finishes
+            // channel dA + gi
+            const float send = gi == 0 ? ych[1] : ych[0];
+            const float keep = gi == 0 ? ych[0] : ych[1];
+            ysum[u] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
           }
         }
         if (!AGG) {
-          // the two lanes of a channel swap half of their partial readouts: lane gi ends with the
-          // full y of token tt + gi
-          const float send = gi == 0 ? yp[1] : yp[0];
-          const float keep = gi == 0 ? yp[0] : yp[1];
-          const float ysum = keep + __shfl_xor_sync(0xffffffffu, send, 1);
-          const int t = tt + gi;
-          if (t0 + t < t_end) {
-            const float xv = __bfloat162float(xs[t * CPW + cl]);
-            const float zv = __bfloat162float(zs[t * CPW + cl]);
-            const float y = fmaf(dsk, xv, ysum);
-            const size_t o = ((size_t)b * p.L + t0 + t) * p.D + d;
-            if (p.y_pre != nullptr) p.y_pre[o] = y;
-            const float sig = fmaf(0.5f, tanh_approx(0.5f * zv), 0.5f);
-            p.out[o] = __float2bfloat16_rn(y * zv * sig);
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            if (full_chunk || t0 + t + u < t_end) {
+              const float xm = gi == 0 ? xv[u].x : xv[u].y;
+              const float zv = __bfloat162float(zs[(t + u) * kCPW + 2 * cp + gi]);
+              const float y = fmaf(dsk, xm, ysum[u]);
+              if (ypp != nullptr) ypp[(size_t)(t + u) * p.D] = y;
+              const float sig = fmaf(0.5f, tanh_approx(0.5f * zv), 0.5f);
+              outp[(size_t)(t + u) * p.D] = __float2bfloat16_rn(y * zv * sig);
+            }
           }
         }
       }
@@ -364,17 +388,20 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       }
       break;
     }
-    if (AGG) {
-      const size_t o = (((size_t)b * p.S + seg) * p.D + d) * 16 + n0;
 #pragma unroll
-      for (int s = 0; s < NH; ++s) {
-        *reinterpret_cast<float2*>(p.agg_h + o + 2 * s) = h[s];
-        *reinterpret_cast<float2*>(p.agg_logp + o + 2 * s) = lsum[s];
+    for (int ch = 0; ch < 2; ++ch) {
+      if (AGG) {
+        const size_t o = (((size_t)b * p.S + seg) * p.D + dA + ch) * 16 + n0;
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          *reinterpret_cast<float2*>(p.agg_h + o + 2 * s) = h[ch][s];
+          *reinterpret_cast<float2*>(p.agg_logp + o + 2 * s) = lsum[ch][s];
+        }
+      } else if (p.h_final != nullptr && seg == p.S - 1) {
+        const size_t o = ((size_t)b * p.D + dA + ch) * 16 + n0;
+#pragma unroll
+        for (int s = 0; s < 4; ++s) *reinterpret_cast<float2*>(p.h_final + o + 2 * s) = h[ch][s];
       }
-    } else if (p.h_final != nullptr && seg == p.S - 1) {
-      const size_t o = ((size_t)b * p.D + d) * 16 + n0;
-#pragma unroll
-      for (int s = 0; s < NH; ++s) *reinterpret_cast<float2*>(p.h_final + o + 2 * s) = h[s];
     }
   }
   __syncthreads();
@@ -434,7 +461,7 @@ int device_sms() {
   return n;
 }
 
-constexpr int kNPoly = 0;  // states per lane whose exp2 runs on the FMA pipe (even, <= NS)
+constexpr int kNPoly = 0;  // states per lane and channel whose exp2 runs on the FMA pipe (even, <= 8)
 
 }  // namespace
 
@@ -443,13 +470,13 @@ ScanPlan scan_fast_plan(int64_t B, int64_t L, int D, int N, int E, int k, bool i
   ScanPlan pl{};
   pl.fast = io_bf16 && N == 16 && (k == 1 || k == 2) && E >= 1 && E <= 16;
   if (!pl.fast) return pl;
-  const int CPW = Geom<kNS>::CPW;
+  const int CPW = kCPW;
   if (D % CPW != 0 || B * L > (int64_t(1) << 31)) {
     pl.fast = false;
     return pl;
   }
   const int64_t base_units = B * (D / CPW);
-  const int64_t target = (int64_t)device_sms() * 12;
+  const int64_t target = (int64_t)device_sms() * 6;  // at least 6 warps (3072 channels) per SM
   int64_t S = 1;
   if (base_units < target) S = std::min<int64_t>((target + base_units - 1) / base_units, (L + LC - 1) / LC);
   int64_t Lseg = (L + S - 1) / S;
@@ -463,8 +490,7 @@ ScanPlan scan_fast_plan(int64_t B, int64_t L, int D, int N, int E, int k, bool i
 
 template <int K>
 static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s) {
-  constexpr int NS = kNS;
-  constexpr int CPW = Geom<NS>::CPW;
+  constexpr int CPW = kCPW;
   CUtensorMap tx, tz, td, tb, tc;
   if (!map3(&tx, sp.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.D, sp.L, sp.B, CPW) ||
       !map3(&tz, sp.z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.D, sp.L, sp.B, CPW) ||
@@ -497,14 +523,15 @@ static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* s
     cudaFuncAttributes fa;
     cudaError_t err = cudaFuncGetAttributes(&fa, fn);
     if (err != cudaSuccess) return err;
-    const int wmax = std::max(1, std::min(kMaxWarps, fa.maxThreadsPerBlock / 32));
+    const int per_quarter = 512 / tmem_cols_per_warp(sp.E);  // warps that fit one lane quarter's TMEM
+    const int wmax = std::max(1, std::min({kMaxWarps, fa.maxThreadsPerBlock / 32, 4 * per_quarter}));
     ctas = std::max(1, std::min(sms, units));
     warps = std::min(wmax, (units + ctas - 1) / ctas);
     if ((int64_t)ctas * warps < units) ctas = std::min<int64_t>((units + warps - 1) / warps, 65535);
     return cudaSuccess;
   };
   int ctas, warps;
-  const size_t smem_per_warp = (size_t)kStages * Stage<NS>::BYTES + (size_t)kStages * 8;
+  const size_t smem_per_warp = (size_t)kStages * Stage::BYTES + (size_t)kStages * 8;
   const size_t smem = 128 + (size_t)kMaxWarps * smem_per_warp + 32;
   cudaError_t e;
   if (pl.S > 1) {
