@@ -121,6 +121,25 @@ swimba_status swimba_scan_fwd(const swimba_dims *dims, const void *x, const void
                               const float *h0, void *out, float *h_final, float *y_pre, void *ws,
                               size_t ws_bytes, void *stream);
 
+/* swimba_scan_fwd without a caller workspace, for callers that cannot allocate device memory: a
+ * plugin inside a framework that owns all device memory and gives it no allocator, or a
+ * latency-critical loop that must not call cudaMalloc (which can synchronise the device). The pages
+ * have no counterpart of this; it is a deployment convenience.
+ *   Arguments as swimba_scan_fwd, minus ws / ws_bytes. The scratch is a fixed 8 MiB array inside the
+ *   library (every GPU that loads the library holds it until the process exits). Shapes whose
+ *   scratch would exceed it return SWIMBA_ERR_WORKSPACE (swimba_last_error_string says how much was
+ *   needed); nothing is allocated or freed.
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress, once per
+ *   device, with that device current); make that first call before any stream capture.
+ *   Every call shares the one array and overwrites what the last call left there; calls that may
+ *   overlap on the GPU (other streams, other threads) race and must not be issued. Device-side
+ *   status of this variant is cleared at every call and is not reported. */
+swimba_status swimba_scan_fwd_noalloc(const swimba_dims *dims, const void *x, const void *z,
+                                      const float *delta, const float *B_mix, const float *C_mix,
+                                      const int32_t *idx, const float *gates, const swimba_weights *w,
+                                      const float *h0, void *out, float *h_final, float *y_pre,
+                                      void *stream);
+
 /* One decode step (dims->seqlen must be 1): the scan for a single token per sequence, continuing
  * from and overwriting the cached state h [B, D, N] fp32. Other arguments as swimba_scan_fwd. */
 swimba_status swimba_step(const swimba_dims *dims, const void *x, const void *z, const float *delta,

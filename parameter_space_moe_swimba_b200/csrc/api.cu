@@ -170,6 +170,26 @@ swimba_status swimba_scan_fwd(const swimba_dims* dims, const void* x, const void
   return scan_common(dims, x, z, delta, B_mix, C_mix, idx, gates, w, h0, out, h_final, y_pre, false, ws, stream);
 }
 
+swimba_status swimba_scan_fwd_noalloc(const swimba_dims* dims, const void* x, const void* z, const float* delta,
+                                      const float* B_mix, const float* C_mix, const int32_t* idx, const float* gates,
+                                      const swimba_weights* w, const float* h0, void* out, float* h_final,
+                                      float* y_pre, void* stream) {
+  swimba_status st = check_dims(dims);
+  if (st != SWIMBA_OK) return st;
+  const size_t need = scan_workspace(dims);
+  if (need > kScanNoAllocScratchBytes) {
+    snprintf(g_last_error, sizeof(g_last_error), "swimba_scan_fwd_noalloc: needs %zu bytes of scratch, the fixed "
+             "array holds %zu", need, kScanNoAllocScratchBytes);
+    return SWIMBA_ERR_WORKSPACE;
+  }
+  void* scratch = nullptr;
+  if (cuda_status(scan_noalloc_scratch(&scratch)) != SWIMBA_OK) return SWIMBA_ERR_CUDA;
+  // the status block must start at zero; the segment carries are written before they are read
+  if (cuda_status(cudaMemsetAsync(scratch, 0, kStatusBytes, static_cast<cudaStream_t>(stream))) != SWIMBA_OK)
+    return SWIMBA_ERR_CUDA;
+  return scan_common(dims, x, z, delta, B_mix, C_mix, idx, gates, w, h0, out, h_final, y_pre, false, scratch, stream);
+}
+
 swimba_status swimba_step(const swimba_dims* dims, const void* x, const void* z, const float* delta,
                           const float* B_mix, const float* C_mix, const int32_t* idx, const float* gates,
                           const swimba_weights* w, float* h, void* out, void* stream) {

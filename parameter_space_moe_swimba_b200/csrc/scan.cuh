@@ -36,4 +36,8 @@ struct ScanPlan {
 ScanPlan scan_fast_plan(int64_t B, int64_t L, int D, int N, int E, int k, bool io_bf16);
 cudaError_t run_scan_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s);
 
+// Fixed device scratch used by swimba_scan_fwd_noalloc (status block + segment carries).
+constexpr size_t kScanNoAllocScratchBytes = size_t(8) << 20;
+cudaError_t scan_noalloc_scratch(void** addr);
+
 }  // namespace swimba

@@ -31,6 +31,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "scan.cuh"
 #include "sm100.cuh"
@@ -565,6 +566,38 @@ static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* s
 
 cudaError_t run_scan_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s) {
   return sp.k == 1 ? launch_fast<1>(sp, pl, seg_ws, status, s) : launch_fast<2>(sp, pl, seg_ws, status, s);
+}
+
+// ---- scratch for callers that cannot allocate device memory ----------------------------------------
+// Some callers of the scan have no way to hand the library a workspace: a plugin inside a host
+// framework that owns every byte of device memory and exposes no allocator to it, or a latency-
+// critical loop where a cudaMalloc (which can synchronise the device) is not acceptable. For them
+// swimba_scan_fwd_noalloc uses this fixed array instead of a caller workspace. It lives in the
+// library's module, so every GPU that loads the library holds it until the process exits.
+static __device__ __align__(256) unsigned char g_scan_noalloc_scratch[kScanNoAllocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[256] = {};
+}  // namespace
+
+// Device address of the fixed scratch on the current device. In host code the array's name is only
+// a host-side stand-in, so the address comes from cudaGetSymbolAddress, once per device, with that
+// device current, and is cached.
+cudaError_t scan_noalloc_scratch(void** addr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 256) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_scan_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_addr[dev] = ptr;
+  }
+  *addr = g_noalloc_addr[dev];
+  return cudaSuccess;
 }
 
 }  // namespace swimba

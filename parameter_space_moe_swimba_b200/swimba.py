@@ -44,6 +44,7 @@ EXPORTED = [
     "swimba_route",
     "swimba_mixed_proj",
     "swimba_scan_fwd",
+    "swimba_scan_fwd_noalloc",
     "swimba_step",
     "swimba_get_device_status",
     "swimba_status_string",
@@ -81,6 +82,9 @@ _lib.swimba_mixed_proj.restype = ctypes.c_int
 _lib.swimba_scan_fwd.argtypes = [ctypes.POINTER(swimba_dims), _P, _P, _P, _P, _P, _P, _P,
                                  ctypes.POINTER(swimba_weights), _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.swimba_scan_fwd.restype = ctypes.c_int
+_lib.swimba_scan_fwd_noalloc.argtypes = [ctypes.POINTER(swimba_dims), _P, _P, _P, _P, _P, _P, _P,
+                                         ctypes.POINTER(swimba_weights), _P, _P, _P, _P, _P]
+_lib.swimba_scan_fwd_noalloc.restype = ctypes.c_int
 _lib.swimba_step.argtypes = [ctypes.POINTER(swimba_dims), _P, _P, _P, _P, _P, _P, _P,
                              ctypes.POINTER(swimba_weights), _P, _P, _P]
 _lib.swimba_step.restype = ctypes.c_int
@@ -156,6 +160,13 @@ def swimba_scan_fwd(dims, x, z, delta, B_mix, C_mix, idx, gates, weights, h0, ou
     return _lib.swimba_scan_fwd(ctypes.byref(dims), _ptr(x), _ptr(z), _ptr(delta), _ptr(B_mix), _ptr(C_mix),
                                 _ptr(idx), _ptr(gates), ctypes.byref(weights), _ptr(h0), _ptr(out), _ptr(h_final),
                                 _ptr(y_pre), _ptr(ws), int(ws_bytes), _stream(stream))
+
+
+def swimba_scan_fwd_noalloc(dims, x, z, delta, B_mix, C_mix, idx, gates, weights, h0, out, h_final, y_pre,
+                            stream=None) -> int:
+    return _lib.swimba_scan_fwd_noalloc(ctypes.byref(dims), _ptr(x), _ptr(z), _ptr(delta), _ptr(B_mix), _ptr(C_mix),
+                                        _ptr(idx), _ptr(gates), ctypes.byref(weights), _ptr(h0), _ptr(out),
+                                        _ptr(h_final), _ptr(y_pre), _stream(stream))
 
 
 def swimba_step(dims, x, z, delta, B_mix, C_mix, idx, gates, weights, h, out, stream=None) -> int:
