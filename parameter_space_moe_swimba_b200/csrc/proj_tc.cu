@@ -10,7 +10,7 @@
 // unordered expert pair), so every 128-row tile shares its k weight tables and x is read once:
 //   bucket kernels  group id per token, histogram, offsets + tile list, scatter of token ids.
 //   stage 1         per tile: acc_j = X_tile · W_x^{e_j}  (j < k; TMEM, M=128, N=R+2N, K=D).
-//                   x rows are gathered by TMA (tile::gather4, 64-byte swizzle); W_x boxes are
+//                   x rows are gathered by TMA (tile::gather4, 128-byte swizzle); W_x boxes are
 //                   MN-major 128-byte-swizzled tiles of the [E, D, R+2N] table as stored.
 //                   Epilogue: B_mix, C_mix = Σ_j g_j (B^j, C^j) -> global; the gated low-rank
 //                   rows g_j dt_low^j, split into bf16 hi + lo parts (hi = bf16(v), lo =
@@ -38,9 +38,9 @@ using namespace sm100;
 namespace {
 
 constexpr int BM = 128;        // rows (token slots) per tile
-constexpr int BK1 = 32;        // stage-1 K slice per ring stage (64 bytes of bf16 per row)
-constexpr int kStages1 = 6;
-constexpr int kSlot1 = 32768;  // A 8 KB + up to 6 W_x boxes of 4 KB
+constexpr int BK1 = 64;        // stage-1 K slice per ring stage (128 bytes of bf16 per row)
+constexpr int kStages1 = 3;
+constexpr int kSlot1 = 65536;  // A 16 KB + up to 6 W_x boxes of 8 KB
 constexpr int NC = 256;        // stage-2 output columns per chunk
 constexpr int kStages2 = 3;
 constexpr int kSlot2 = 32768;  // 4 W_dt boxes of up to 64 rows x 128 B
@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
   const int num_tiles = *p.num_tiles;
   const int ksteps = p.D / BK1;
-  const uint32_t slot_bytes = 8192u + (uint32_t)(K * p.nbw) * 4096u;
+  const uint32_t slot_bytes = 16384u + (uint32_t)(K * p.nbw) * 8192u;
 
   if (warp == 0) {
     // ---------------- producer ----------------
@@ -267,10 +267,10 @@ __global__ void __launch_bounds__(192, 1)
         uint8_t* slot = ring + stage * kSlot1;
         if (lane == 0) mbar_arrive_expect_tx(&full[stage], slot_bytes);
         __syncwarp();
-        tma_gather4(slot + lane * 256, &tm_x, &full[stage], ks * BK1, rr[0], rr[1], rr[2], rr[3]);
+        tma_gather4(slot + lane * 512, &tm_x, &full[stage], ks * BK1, rr[0], rr[1], rr[2], rr[3]);
         if (lane < K * p.nbw) {
           const int j = lane / p.nbw, nb = lane - j * p.nbw;
-          tma_load_3d(slot + 8192 + lane * 4096, &tm_wx, &full[stage], nb * 64, ks * BK1, ej[j]);
+          tma_load_3d(slot + 16384 + lane * 8192, &tm_wx, &full[stage], nb * 64, ks * BK1, ej[j]);
         }
         ++issued;
         if (++stage == kStages1) {
@@ -306,10 +306,11 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t base = smem_u32(ring + stage * kSlot1);
 #pragma unroll
           for (int kk = 0; kk < BK1 / 16; ++kk) {
-            const uint64_t adesc = smem_desc(base + kk * 32, 16, 512, kLayoutSW64);
+            const uint64_t adesc = smem_desc(base + kk * 32, 16, 1024, kLayoutSW128);
 #pragma unroll
             for (int j = 0; j < K; ++j) {
-              const uint64_t bdesc = smem_desc(base + 8192 + j * p.nbw * 4096 + kk * 16 * 128, 4096, 1024, kLayoutSW128);
+              const uint64_t bdesc =
+                  smem_desc(base + 16384 + j * p.nbw * 8192 + kk * 16 * 128, 8192, 1024, kLayoutSW128);
               mma_bf16(tmem + j * 256, adesc, bdesc, idesc, (ks | kk) != 0);
             }
           }
@@ -603,27 +604,35 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else {
     // ---------------- epilogue: 8 warps, two per TMEM lane quarter ----------------
+    // Each warp drains 128 of the chunk's 256 columns for the 32 rows of its lane quarter, as two
+    // 16-row halves read with the 16x256b shape: four consecutive threads hold eight consecutive
+    // columns of one row, so every warp-wide store writes whole 32-byte sectors of 8 rows.
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;  // 0: chunk columns [0,128), 1: [128,256)
-    const int row = 32 * q + lane;
-    const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
+    const int t0 = lane & 3, t1 = lane >> 2;
     int cur_tile = -1, buf = 0;
     uint32_t acc_phase[2] = {0, 0};
-    bool valid = false;
-    int t = 0, e[2] = {0, 0};
-    float g[K];
-#pragma unroll
-    for (int j = 0; j < K; ++j) g[j] = 0.f;
+    // the 4 rows of this thread: 32q + 16dh + t1 + 8r  (dh, r in {0, 1})
+    bool valid[2][2] = {{false, false}, {false, false}};
+    int tok[2][2] = {{0, 0}, {0, 0}};
+    float g[2][2][K];
+    int e[2] = {0, 0};
     for (long long item = item_begin; item < item_end; ++item) {
       const int tile = (int)(item / nchunks);
       const int c = (int)(item - (long long)tile * nchunks);
       if (tile != cur_tile) {
         const TileInfo ti = p.tiles[tile];
-        valid = row < ti.rows;
-        const int pos = ti.row_begin + min(row, ti.rows - 1);
-        t = p.slot_tok[pos];
 #pragma unroll
-        for (int j = 0; j < K; ++j) g[j] = p.slot_gate[pos * K + j];
+        for (int dh = 0; dh < 2; ++dh)
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int row = 32 * q + 16 * dh + t1 + 8 * r;
+            valid[dh][r] = row < ti.rows;
+            const int pos = ti.row_begin + min(row, ti.rows - 1);
+            tok[dh][r] = p.slot_tok[pos];
+#pragma unroll
+            for (int j = 0; j < K; ++j) g[dh][r][j] = p.slot_gate[pos * K + j];
+          }
         e[0] = ti.e0;
         e[1] = ti.e1;
         cur_tile = tile;
@@ -635,40 +644,38 @@ __global__ void __launch_bounds__(320, 1)
       }
       acc_phase[buf] ^= 1u;
       tc_fence_after();
-      for (int cc = 0; cc < 4; ++cc) {
-        const int col = half * 128 + cc * 32;
-        float v[32];
-        tmem_ld32(tl + buf * NC + col, v);
-        if (cc == 3) {
+      const int dcol = c * NC + half * 128 + 2 * t0;  // column of r[0]; r[4k] is at dcol + 8k
+#pragma unroll
+      for (int dh = 0; dh < 2; ++dh) {
+        uint32_t v[64];
+        tmem_ld_16x256b_x16_nowait(tmem + ((uint32_t)(32 * q + 16 * dh) << 16) + buf * NC + half * 128, v);
+        tmem_wait_ld();
+        if (dh == 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
-        const int d0 = c * NC + col;
-        if (d0 < p.D) {
-          float bias[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) bias[i] = 0.f;
+        for (int k = 0; k < 16; ++k) {
+          const int d = dcol + 8 * k;
+          if (d < p.D) {
+            float2 bmix[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // per row r
 #pragma unroll
-          for (int j = 0; j < K; ++j) {
-            const float4* bp = reinterpret_cast<const float4*>(p.b_dt + (size_t)e[j] * p.D + d0);
+            for (int j = 0; j < K; ++j) {
+              const float2 bj = __ldg(reinterpret_cast<const float2*>(p.b_dt + (size_t)e[j] * p.D + d));
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float4 b4 = __ldg(bp + i);
-              bias[4 * i + 0] = fmaf(g[j], b4.x, bias[4 * i + 0]);
-              bias[4 * i + 1] = fmaf(g[j], b4.y, bias[4 * i + 1]);
-              bias[4 * i + 2] = fmaf(g[j], b4.z, bias[4 * i + 2]);
-              bias[4 * i + 3] = fmaf(g[j], b4.w, bias[4 * i + 3]);
+              for (int r = 0; r < 2; ++r) {
+                bmix[r].x = fmaf(g[dh][r][j], bj.x, bmix[r].x);
+                bmix[r].y = fmaf(g[dh][r][j], bj.y, bmix[r].y);
+              }
             }
-          }
-          if (valid) {
-            float4* out = reinterpret_cast<float4*>(p.delta + (size_t)t * p.D + d0);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              out[i] = make_float4(softplus_fast(v[4 * i + 0] + bias[4 * i + 0]),
-                                   softplus_fast(v[4 * i + 1] + bias[4 * i + 1]),
-                                   softplus_fast(v[4 * i + 2] + bias[4 * i + 2]),
-                                   softplus_fast(v[4 * i + 3] + bias[4 * i + 3]));
+            for (int r = 0; r < 2; ++r) {
+              if (valid[dh][r]) {
+                const float2 o = make_float2(softplus_fast(__uint_as_float(v[4 * k + 2 * r]) + bmix[r].x),
+                                             softplus_fast(__uint_as_float(v[4 * k + 2 * r + 1]) + bmix[r].y));
+                *reinterpret_cast<float2*>(p.delta + (size_t)tok[dh][r] * p.D + d) = o;
+              }
             }
           }
         }
@@ -743,7 +750,7 @@ cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s) {
     cuuint64_t dims[2] = {(cuuint64_t)p.D, (cuuint64_t)p.T};
     cuuint64_t str[1] = {(cuuint64_t)p.D * 2};
     cuuint32_t box[2] = {BK1, 1};
-    if (!encode(&tm_x, p.x, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B)) return cudaErrorInvalidValue;
+    if (!encode(&tm_x, p.x, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
   }
   {
     cuuint64_t dims[3] = {(cuuint64_t)W, (cuuint64_t)p.D, (cuuint64_t)p.E};

@@ -143,13 +143,24 @@ __global__ void __launch_bounds__(512, 1) route_smem_kernel(RouteParams p) {
     for (int tt = 0; tt < TOK; ++tt)
 #pragma unroll
       for (int e = 0; e < EP / 2; ++e) acc[tt][e] = make_float2(0.f, 0.f);
+    // x chunks of the next iteration are loaded while the current one is accumulated
+    uint4 xn[TOK];
+#pragma unroll
+    for (int tt = 0; tt < TOK; ++tt) {
+      xn[tt] = make_uint4(0, 0, 0, 0);
+      if (lane < C && t0 + tt < p.T) xn[tt] = __ldcs(reinterpret_cast<const uint4*>(x + (t0 + tt) * p.D) + lane);
+    }
     for (int c = lane; c < C; c += 32) {
       uint4 xv[TOK];
 #pragma unroll
       for (int tt = 0; tt < TOK; ++tt) {
-        xv[tt] = make_uint4(0, 0, 0, 0);
-        if (t0 + tt < p.T) xv[tt] = __ldcs(reinterpret_cast<const uint4*>(x + (t0 + tt) * p.D) + c);
+        xv[tt] = xn[tt];
+        xn[tt] = make_uint4(0, 0, 0, 0);
+        if (c + 32 < C && t0 + tt < p.T) xn[tt] = __ldcs(reinterpret_cast<const uint4*>(x + (t0 + tt) * p.D) + c + 32);
       }
+      float xf[TOK][V];
+#pragma unroll
+      for (int tt = 0; tt < TOK; ++tt) Vec16<IO>::unpack(xv[tt], xf[tt]);
 #pragma unroll
       for (int i = 0; i < V; ++i) {
         float2 w[EP / 2];
@@ -157,9 +168,7 @@ __global__ void __launch_bounds__(512, 1) route_smem_kernel(RouteParams p) {
         for (int e = 0; e < EP / 2; ++e) w[e] = Wp[((size_t)e * V + i) * C + c];
 #pragma unroll
         for (int tt = 0; tt < TOK; ++tt) {
-          float xf[V];
-          Vec16<IO>::unpack(xv[tt], xf);
-          const float2 xx = make_float2(xf[i], xf[i]);
+          const float2 xx = make_float2(xf[tt][i], xf[tt][i]);
 #pragma unroll
           for (int e = 0; e < EP / 2; ++e) acc[tt][e] = __ffma2_rn(xx, w[e], acc[tt][e]);
         }
@@ -214,9 +223,9 @@ static cudaError_t launch_route(const RouteParams& p, cudaStream_t s) {
 
 template <typename IO>
 static cudaError_t route_dispatch(const RouteParams& p, cudaStream_t s) {
-  if (p.E <= 4) return launch_route<IO, 4, 8>(p, s);
-  if (p.E <= 8) return launch_route<IO, 8, 8>(p, s);
-  return launch_route<IO, 16, 4>(p, s);
+  if (p.E <= 4) return launch_route<IO, 4, 4>(p, s);
+  if (p.E <= 8) return launch_route<IO, 8, 4>(p, s);
+  return launch_route<IO, 16, 2>(p, s);
 }
 
 cudaError_t run_route(const void* x, bool io_bf16, const float* W_r, int32_t* idx, float* gates, int64_t T,
