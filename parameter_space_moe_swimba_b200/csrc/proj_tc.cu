@@ -434,7 +434,7 @@ __device__ __forceinline__ float softplus_fast(float v) {
 }
 
 template <int K>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __maxnreg__(168)
     proj_stage2_kernel(const __grid_constant__ CUtensorMap tm_ap, const __grid_constant__ CUtensorMap tm_wdt,
                        const Stage2Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -637,6 +637,17 @@ __global__ void __launch_bounds__(320, 1)
         e[1] = ti.e1;
         cur_tile = tile;
       }
+      const int dcol = c * NC + half * 128 + 2 * t0;  // column of r[0]; r[4k] is at dcol + 8k
+      // this thread's bias values for the chunk, loaded before the accumulator wait hides them
+      float2 bias[K][16];
+#pragma unroll
+      for (int j = 0; j < K; ++j)
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int d = dcol + 8 * k;
+          bias[j][k] = d < p.D ? __ldg(reinterpret_cast<const float2*>(p.b_dt + (size_t)e[j] * p.D + d))
+                               : make_float2(0.f, 0.f);
+        }
       if (!mbar_wait(&acc_full[buf], acc_phase[buf], abort_flag)) {
         *abort_flag = 1;
         if (lane == 0) record_device_error(p.status, SWIMBA_ERR_TIMEOUT, 23, blockIdx.x, (int)item);
@@ -644,37 +655,36 @@ __global__ void __launch_bounds__(320, 1)
       }
       acc_phase[buf] ^= 1u;
       tc_fence_after();
-      const int dcol = c * NC + half * 128 + 2 * t0;  // column of r[0]; r[4k] is at dcol + 8k
 #pragma unroll
       for (int dh = 0; dh < 2; ++dh) {
-        uint32_t v[64];
-        tmem_ld_16x256b_x16_nowait(tmem + ((uint32_t)(32 * q + 16 * dh) << 16) + buf * NC + half * 128, v);
-        tmem_wait_ld();
-        if (dh == 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[buf]);
-        }
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int d = dcol + 8 * k;
-          if (d < p.D) {
-            float2 bmix[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // per row r
+        for (int kh = 0; kh < 2; ++kh) {
+          uint32_t v[32];
+          tmem_ld_16x256b_x8_nowait(tmem + ((uint32_t)(32 * q + 16 * dh) << 16) + buf * NC + half * 128 + kh * 64, v);
+          tmem_wait_ld();
+          if (dh == 1 && kh == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+          }
 #pragma unroll
-            for (int j = 0; j < K; ++j) {
-              const float2 bj = __ldg(reinterpret_cast<const float2*>(p.b_dt + (size_t)e[j] * p.D + d));
+          for (int kk = 0; kk < 8; ++kk) {
+            const int k = kh * 8 + kk;
+            const int d = dcol + 8 * k;
+            if (d < p.D) {
 #pragma unroll
               for (int r = 0; r < 2; ++r) {
-                bmix[r].x = fmaf(g[dh][r][j], bj.x, bmix[r].x);
-                bmix[r].y = fmaf(g[dh][r][j], bj.y, bmix[r].y);
-              }
-            }
+                float2 bmix = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-              if (valid[dh][r]) {
-                const float2 o = make_float2(softplus_fast(__uint_as_float(v[4 * k + 2 * r]) + bmix[r].x),
-                                             softplus_fast(__uint_as_float(v[4 * k + 2 * r + 1]) + bmix[r].y));
-                *reinterpret_cast<float2*>(p.delta + (size_t)tok[dh][r] * p.D + d) = o;
+                for (int j = 0; j < K; ++j) {
+                  bmix.x = fmaf(g[dh][r][j], bias[j][k].x, bmix.x);
+                  bmix.y = fmaf(g[dh][r][j], bias[j][k].y, bmix.y);
+                }
+                if (valid[dh][r]) {
+                  const float2 o = make_float2(softplus_fast(__uint_as_float(v[4 * kk + 2 * r]) + bmix.x),
+                                               softplus_fast(__uint_as_float(v[4 * kk + 2 * r + 1]) + bmix.y));
+                  *reinterpret_cast<float2*>(p.delta + (size_t)tok[dh][r] * p.D + d) = o;
+                }
               }
             }
           }

@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       const bool full_chunk = t0 + LC <= t_end;
       __nv_bfloat16* outp = AGG ? nullptr : p.out + ((size_t)b * p.L + t0) * p.D + dmine;
       float* ypp = (AGG || p.y_pre == nullptr) ? nullptr : p.y_pre + ((size_t)b * p.L + t0) * p.D + dmine;
-#pragma unroll 1
+#pragma unroll 2
       for (int t = 0; t < LC; t += 2) {
         // loads of both tokens first: the selected experts' A rows (TMEM), Δ, x, B, C (smem)
         int4 m[2];
