@@ -42,10 +42,11 @@ UNIT = "tokens/s"
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="swimba", choices=["swimba", "reference"])
     ap.add_argument("--workload", default="mamba1p4b_like")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
@@ -108,17 +109,37 @@ class ClockSampler:
         self.path = None
 
     def start(self):
+        """Start sampling every 50 ms and wait (at most 3 s) until the first sample is written."""
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
                  "-i", str(self.gpu_index)], stdout=self.f, stderr=subprocess.DEVNULL)
+            t0 = time.time()
+            while self.mark() == 0 and time.time() - t0 < 3.0:
+                time.sleep(0.02)
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def _rows(self):
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and line.endswith("\n"):
+                    rows.append(parts)
+        return rows
+
+    def mark(self):
+        """Number of complete samples so far (brackets the timed region)."""
+        if self.proc is None:
+            return 0
+        return len(self._rows())
+
+    def stop(self, begin=0, end=None):
+        """Summarise the samples taken between the marks ``begin`` and ``end`` (all if none fall there)."""
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -127,13 +148,10 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.f.close()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
+        rows = self._rows()
         os.unlink(self.path)
+        inside = rows[begin:end]
+        rows = inside if inside else rows
         if not rows:
             return None
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
@@ -329,6 +347,8 @@ def config_block(cfg):
 def main():
     args = parse()
     cfg = CONFIGS[args.workload]
+    if args.batch > 0:
+        cfg = cfg.with_(batch=args.batch)
     if args.impl == "reference":
         return run_reference(args, cfg)
 
@@ -356,8 +376,9 @@ def main():
 
     clocks = ClockSampler(torch.cuda.current_device())
     clocks.start()
+    m0 = clocks.mark()
     total_ms, per_kernel, launches = timed_steps(torch, layer, args.steps, args.warmup, dist)
-    clk = clocks.stop()
+    clk = clocks.stop(m0, clocks.mark())
     S.check(S.swimba_get_device_status(layer.buf.ws, layer.stream), "device status")
 
     max_ms = max_over_ranks(total_ms, dist, device)

@@ -44,15 +44,27 @@ namespace {
 
 constexpr int LC = 16;          // tokens per chunk
 constexpr int kStages = 3;      // ring depth per warp
-constexpr int kCPW = 32;        // channels per warp
-constexpr int kMaxWarps = 8;    // warps per CTA (registers: up to 255 per thread)
+
+// Lane geometry, by G = lanes per channel pair (2 or 4): each lane holds NS = 16 / G states of two
+// channels; a warp covers CPW = 64 / G channels; a CTA holds up to 8 (G = 2, up to 255 registers a
+// thread) or 16 (G = 4, up to 128) warps.
+template <int G>
+struct Geo {
+  static_assert(G == 2 || G == 4, "2 or 4 lanes per channel pair");
+  static constexpr int NS = 16 / G;        // states per lane and channel
+  static constexpr int NP = NS / 2;        // float2 pairs per lane and channel
+  static constexpr int CPW = 64 / G;       // channels per warp
+  static constexpr int ACOLS = 2 * NS;     // TMEM columns per expert (both channels of a lane)
+  static constexpr int MAXW = 4 * G;       // warps per CTA
+};
 
 // Byte offsets inside one ring stage of one warp.
+template <int CPW>
 struct Stage {
-  static constexpr int X = 0;                      // bf16 [LC][32]
-  static constexpr int Z = X + LC * kCPW * 2;      // bf16 [LC][32]
-  static constexpr int DL = Z + LC * kCPW * 2;     // f32  [LC][32]
-  static constexpr int B = DL + LC * kCPW * 4;     // f32  [LC][16]
+  static constexpr int X = 0;                      // bf16 [LC][CPW]
+  static constexpr int Z = X + LC * CPW * 2;       // bf16 [LC][CPW]
+  static constexpr int DL = Z + LC * CPW * 2;      // f32  [LC][CPW]
+  static constexpr int B = DL + LC * CPW * 4;      // f32  [LC][16]
   static constexpr int C = B + LC * 16 * 4;        // f32  [LC][16]
   static constexpr int META = C + LC * 16 * 4;     // int4 [LC] {e0, e1, g0, g1}
   static constexpr int BYTES = META + LC * 16;
@@ -61,8 +73,15 @@ struct Stage {
   static_assert(BYTES % 128 == 0, "stage size");
 };
 
-// TMEM columns one warp needs (16 per expert) and how many warps share a lane quarter's 512.
-__host__ __device__ constexpr int tmem_cols_per_warp(int E) { return ((E * 16 + 31) / 32) * 32; }
+// TMEM columns one warp needs (ACOLS per expert, rounded up to the 32-column allocation granule).
+__host__ __device__ constexpr int tmem_cols_per_warp(int E, int acols) { return ((E * acols + 31) / 32) * 32; }
+
+// n consecutive TMEM columns of this thread's lane, without waiting (n = 8 or 16).
+template <int NCOL>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NCOL]) {
+  if constexpr (NCOL == 16) tmem_ld16_nowait(taddr, r);
+  else tmem_ld8_nowait(taddr, r);
+}
 
 // 2^x on the FMA pipe for x <= 0: x = j + f with j = round(x) (the 1.5*2^23 shifter), f in
 // [-1/2, 1/2]; 2^f by a degree-5 polynomial fitted for minimax relative error on that interval
@@ -112,12 +131,13 @@ struct FastParams {
 };
 
 // AGG = true: pass 1 (segments 0 .. S-2 only; no readout, no output).
-template <int K, int NPOLY, bool AGG>
-__global__ void __launch_bounds__(kMaxWarps * 32, 1)
+template <int K, int NPOLY, bool AGG, int G>
+__global__ void __launch_bounds__(Geo<G>::MAXW * 32, 1)
     scan_fast_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
                      const __grid_constant__ CUtensorMap tm_dl, const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_c, const FastParams p) {
-  using St = Stage;
+  constexpr int NS = Geo<G>::NS, NP = Geo<G>::NP, CPW = Geo<G>::CPW, ACOLS = Geo<G>::ACOLS;
+  using St = Stage<CPW>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -148,46 +168,59 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
   }
   __syncthreads();
   tc_fence_after();
-  // this warp's TMEM window: its lane quarter, tmem_cols_per_warp(E) columns
+  // this warp's TMEM window: its lane quarter, tmem_cols_per_warp(E, ACOLS) columns
   const uint32_t tbase = *tmem_slot + ((uint32_t)(32 * (warp & 3)) << 16) +
-                         (uint32_t)(warp >> 2) * (uint32_t)tmem_cols_per_warp(p.E);
+                         (uint32_t)(warp >> 2) * (uint32_t)tmem_cols_per_warp(p.E, ACOLS);
 
-  const int cp = lane >> 1;   // channel pair: channels 2cp, 2cp+1 of the warp's 32
-  const int gi = lane & 1;    // state group: states 8gi .. 8gi+7
-  const int n0 = gi * 8;
-  const int ntiles = p.D / kCPW;
+  const int cp = lane / G;    // channel pair: channels 2cp, 2cp+1 of the warp's CPW
+  const int gi = lane % G;    // state group: states NS*gi .. NS*gi+NS-1
+  const int n0 = gi * NS;
+  // the output this lane finishes: G = 2, channel gi of both tokens of a pair; G = 4, channel
+  // gi & 1 of token gi >> 1 of the pair
+  const int och = G == 2 ? gi : (gi & 1);
+  const int ou = G == 2 ? 0 : (gi >> 1);
+  const int ntiles = p.D / CPW;
   const int u_begin = (int)((int64_t)p.units * blockIdx.x / gridDim.x);
   const int u_end = (int)((int64_t)p.units * (blockIdx.x + 1) / gridDim.x);
   uint32_t phase_bits = 0;  // one parity bit per stage
-  constexpr uint32_t tx_bytes = AGG ? (LC * kCPW * 2 + LC * kCPW * 4 + LC * 16 * 4)
-                                    : (2 * LC * kCPW * 2 + LC * kCPW * 4 + 2 * LC * 16 * 4);
+  constexpr uint32_t tx_bytes = AGG ? (LC * CPW * 2 + LC * CPW * 4 + LC * 16 * 4)
+                                    : (2 * LC * CPW * 2 + LC * CPW * 4 + 2 * LC * 16 * 4);
 
   for (int u = u_begin + warp; u < u_end; u += nwarps) {
     const int tile = u % ntiles;
     const int bs = u / ntiles;  // b * seg_count + seg
     const int seg = bs % p.seg_count;
     const int b = bs / p.seg_count;
-    const int dA = tile * kCPW + 2 * cp;  // this lane's channels dA, dA + 1
+    const int dA = tile * CPW + 2 * cp;  // this lane's channels dA, dA + 1
     const int64_t t_begin = (int64_t)seg * p.Lseg;
     const int64_t t_end = std::min<int64_t>(p.L, t_begin + p.Lseg);
     const int nchunks = (int)((t_end - t_begin + LC - 1) / LC);
 
-    // per-expert transition rows of this lane's 2 x 8 states, times log2(e), into TMEM 16e..16e+15
+    // per-expert transition rows of this lane's 2 x NS states, times log2(e), into TMEM
+    // columns ACOLS*e + NS*ch + s
     for (int e = 0; e < p.E; ++e) {
+      uint32_t r[ACOLS];
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
         const float4* src = reinterpret_cast<const float4*>(p.A + ((size_t)e * p.D + dA + ch) * 16 + n0);
-        const float4 a0 = __ldg(src), a1 = __ldg(src + 1);
-        const uint32_t r[8] = {__float_as_uint(a0.x * kLog2e), __float_as_uint(a0.y * kLog2e),
-                               __float_as_uint(a0.z * kLog2e), __float_as_uint(a0.w * kLog2e),
-                               __float_as_uint(a1.x * kLog2e), __float_as_uint(a1.y * kLog2e),
-                               __float_as_uint(a1.z * kLog2e), __float_as_uint(a1.w * kLog2e)};
-        tmem_st8(tbase + (uint32_t)e * 16u + (uint32_t)ch * 8u, r);
+#pragma unroll
+        for (int q = 0; q < NS / 4; ++q) {
+          const float4 a4 = __ldg(src + q);
+          r[ch * NS + 4 * q + 0] = __float_as_uint(a4.x * kLog2e);
+          r[ch * NS + 4 * q + 1] = __float_as_uint(a4.y * kLog2e);
+          r[ch * NS + 4 * q + 2] = __float_as_uint(a4.z * kLog2e);
+          r[ch * NS + 4 * q + 3] = __float_as_uint(a4.w * kLog2e);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < ACOLS / 8; ++q) {
+        const uint32_t (&r8)[8] = *reinterpret_cast<const uint32_t(*)[8]>(r + 8 * q);
+        tmem_st8(tbase + (uint32_t)(e * ACOLS + 8 * q), r8);
       }
     }
     tmem_wait_st();
 
-    float2 h[2][4];  // [channel][state pair]
+    float2 h[2][NP];  // [channel][state pair]
 #pragma unroll
     for (int ch = 0; ch < 2; ++ch) {
       const float* hs = AGG ? nullptr
@@ -195,15 +228,15 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
                                                   : (p.h0 != nullptr && seg == 0 ? p.h0 + ((size_t)b * p.D + dA + ch) * 16
                                                                                  : nullptr));
 #pragma unroll
-      for (int s = 0; s < 4; ++s)
+      for (int s = 0; s < NP; ++s)
         h[ch][s] = hs ? *reinterpret_cast<const float2*>(hs + n0 + 2 * s) : make_float2(0.f, 0.f);
     }
-    float2 lsum[2][4];
+    float2 lsum[2][NP];
 #pragma unroll
     for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
-      for (int s = 0; s < 4; ++s) lsum[ch][s] = make_float2(0.f, 0.f);
-    const int dmine = dA + gi;  // the channel whose outputs this lane writes
+      for (int s = 0; s < NP; ++s) lsum[ch][s] = make_float2(0.f, 0.f);
+    const int dmine = dA + och;  // the channel whose outputs this lane writes
     const float dsk = AGG ? 0.f : p.D_skip[dmine];
 
     // meta of one chunk: lane t (< LC) holds token t's {e0, e1, g0, g1}
@@ -231,11 +264,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
         uint64_t* bar = &full[c % kStages];
         mbar_arrive_expect_tx(bar, tx_bytes);
         const int t0 = (int)(t_begin + (int64_t)c * LC);
-        tma_load_3d(st + St::X, &tm_x, bar, tile * kCPW, t0, b);
-        tma_load_3d(st + St::DL, &tm_dl, bar, tile * kCPW, t0, b);
+        tma_load_3d(st + St::X, &tm_x, bar, tile * CPW, t0, b);
+        tma_load_3d(st + St::DL, &tm_dl, bar, tile * CPW, t0, b);
         tma_load_3d(st + St::B, &tm_b, bar, 0, t0, b);
         if (!AGG) {
-          tma_load_3d(st + St::Z, &tm_z, bar, tile * kCPW, t0, b);
+          tma_load_3d(st + St::Z, &tm_z, bar, tile * CPW, t0, b);
           tma_load_3d(st + St::C, &tm_c, bar, 0, t0, b);
         }
       }
@@ -268,40 +301,43 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       const bool full_chunk = t0 + LC <= t_end;
       __nv_bfloat16* outp = AGG ? nullptr : p.out + ((size_t)b * p.L + t0) * p.D + dmine;
       float* ypp = (AGG || p.y_pre == nullptr) ? nullptr : p.y_pre + ((size_t)b * p.L + t0) * p.D + dmine;
-#pragma unroll 2
+      // pass over the chunk's tokens: the recurrence only; readout partials are kept in registers
+      // and the reduction, skip term, gate and stores follow for the whole chunk, off the
+      // recurrence's dependency chain
+      float ypart[LC][2];  // [token][channel]
+#pragma unroll
       for (int t = 0; t < LC; t += 2) {
         // loads of both tokens first: the selected experts' A rows (TMEM), Δ, x, B, C (smem)
         int4 m[2];
-        uint32_t ar[2][2][16];  // [token][expert slot][16 values]
+        uint32_t ar[2][2][ACOLS];  // [token][expert slot][columns]
         float2 dl[2], xv[2];
-        float2 bv[2][4], cv[2][4];
+        float2 bv[2][NP], cv[2][NP];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           m[u] = meta[t + u];
-          tmem_ld16_nowait(tbase + (uint32_t)m[u].x * 16u, ar[u][0]);
-          if (K == 2) tmem_ld16_nowait(tbase + (uint32_t)m[u].y * 16u, ar[u][1]);
+          tmem_ld_cols<ACOLS>(tbase + (uint32_t)(m[u].x * ACOLS), ar[u][0]);
+          if (K == 2) tmem_ld_cols<ACOLS>(tbase + (uint32_t)(m[u].y * ACOLS), ar[u][1]);
         }
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-          dl[u] = ds2[(t + u) * (kCPW / 2) + cp];
-          xv[u] = __bfloat1622float2(xs2[(t + u) * (kCPW / 2) + cp]);
-          const float4 bq0 = bsm[(t + u) * 4 + 2 * gi], bq1 = bsm[(t + u) * 4 + 2 * gi + 1];
-          bv[u][0] = make_float2(bq0.x, bq0.y);
-          bv[u][1] = make_float2(bq0.z, bq0.w);
-          bv[u][2] = make_float2(bq1.x, bq1.y);
-          bv[u][3] = make_float2(bq1.z, bq1.w);
-          if (!AGG) {
-            const float4 cq0 = csm[(t + u) * 4 + 2 * gi], cq1 = csm[(t + u) * 4 + 2 * gi + 1];
-            cv[u][0] = make_float2(cq0.x, cq0.y);
-            cv[u][1] = make_float2(cq0.z, cq0.w);
-            cv[u][2] = make_float2(cq1.x, cq1.y);
-            cv[u][3] = make_float2(cq1.z, cq1.w);
+          dl[u] = ds2[(t + u) * (CPW / 2) + cp];
+          xv[u] = __bfloat1622float2(xs2[(t + u) * (CPW / 2) + cp]);
+#pragma unroll
+          for (int q = 0; q < NS / 4; ++q) {
+            const float4 bq = bsm[(t + u) * 4 + gi * (NS / 4) + q];
+            bv[u][2 * q] = make_float2(bq.x, bq.y);
+            bv[u][2 * q + 1] = make_float2(bq.z, bq.w);
+            if (!AGG) {
+              const float4 cq = csm[(t + u) * 4 + gi * (NS / 4) + q];
+              cv[u][2 * q] = make_float2(cq.x, cq.y);
+              cv[u][2 * q + 1] = make_float2(cq.z, cq.w);
+            }
           }
         }
         tmem_wait_ld();
         // decay factors of both tokens (independent of the state)
-        float2 a[2][2][4];  // [token][channel][state pair]
-        float2 arg[2][2][4];
+        float2 a[2][2][NP];  // [token][channel][state pair]
+        float2 arg[2][2][NP];
 #pragma unroll
         for (int u = 0; u < 2; ++u)
 #pragma unroll
@@ -310,59 +346,87 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
             const float c0 = dlt * __int_as_float(m[u].z);
             const float c1 = dlt * __int_as_float(m[u].w);
 #pragma unroll
-            for (int s = 0; s < 4; ++s) {
-              const float2 a0 = make_float2(__uint_as_float(ar[u][0][ch * 8 + 2 * s]), __uint_as_float(ar[u][0][ch * 8 + 2 * s + 1]));
+            for (int s = 0; s < NP; ++s) {
+              const float2 a0 = make_float2(__uint_as_float(ar[u][0][ch * NS + 2 * s]), __uint_as_float(ar[u][0][ch * NS + 2 * s + 1]));
               arg[u][ch][s] = __fmul2_rn(make_float2(c0, c0), a0);
               if (K == 2) {
                 const float2 a1 =
-                    make_float2(__uint_as_float(ar[u][1][ch * 8 + 2 * s]), __uint_as_float(ar[u][1][ch * 8 + 2 * s + 1]));
+                    make_float2(__uint_as_float(ar[u][1][ch * NS + 2 * s]), __uint_as_float(ar[u][1][ch * NS + 2 * s + 1]));
                 arg[u][ch][s] = __ffma2_rn(make_float2(c1, c1), a1, arg[u][ch][s]);
               }
-              if (s >= 4 - NPOLY / 2) {
+              if (s >= NP - NPOLY / 2) {
                 a[u][ch][s] = exp2_poly2(arg[u][ch][s]);
               } else {
                 a[u][ch][s] = make_float2(ex2_approx(arg[u][ch][s].x), ex2_approx(arg[u][ch][s].y));
               }
             }
           }
-        // the recurrence, token t then t+1
-        float ysum[2];
+        // the recurrence, token t then t+1; this lane's partial readouts go to ypart
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-          float ych[2];
 #pragma unroll
           for (int ch = 0; ch < 2; ++ch) {
             const float dx = (ch == 0 ? dl[u].x : dl[u].y) * (ch == 0 ? xv[u].x : xv[u].y);
             const float2 dxx = make_float2(dx, dx);
 #pragma unroll
-            for (int s = 0; s < 4; ++s) h[ch][s] = __ffma2_rn(a[u][ch][s], h[ch][s], __fmul2_rn(dxx, bv[u][s]));
+            for (int s = 0; s < NP; ++s) h[ch][s] = __ffma2_rn(a[u][ch][s], h[ch][s], __fmul2_rn(dxx, bv[u][s]));
             if (AGG) {
 #pragma unroll
-              for (int s = 0; s < 4; ++s) lsum[ch][s] = __fadd2_rn(lsum[ch][s], arg[u][ch][s]);
+              for (int s = 0; s < NP; ++s) lsum[ch][s] = __fadd2_rn(lsum[ch][s], arg[u][ch][s]);
             } else {
-              const float2 ya = __ffma2_rn(cv[u][1], h[ch][1], __fmul2_rn(cv[u][0], h[ch][0]));
-              const float2 yb = __ffma2_rn(cv[u][3], h[ch][3], __fmul2_rn(cv[u][2], h[ch][2]));
-              ych[ch] = (ya.x + yb.x) + (ya.y + yb.y);
+              // two independent accumulation chains (even and odd state pairs)
+              float2 ya = __fmul2_rn(cv[u][0], h[ch][0]);
+              float2 yb = __fmul2_rn(cv[u][1], h[ch][1]);
+#pragma unroll
+              for (int s = 2; s < NP; s += 2) {
+                ya = __ffma2_rn(cv[u][s], h[ch][s], ya);
+                yb = __ffma2_rn(cv[u][s + 1], h[ch][s + 1], yb);
+              }
+              ypart[t + u][ch] = (ya.x + yb.x) + (ya.y + yb.y);
             }
           }
-          if (!AGG) {
-            // lanes 2cp (states 0-7) and 2cp+1 (states 8-15) swap one partial: lane gi finishes
-            // channel dA + gi
-            const float send = gi == 0 ? ych[1] : ych[0];
-            const float keep = gi == 0 ? ych[0] : ych[1];
-            ysum[u] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
-          }
         }
-        if (!AGG) {
+      }
+      if (!AGG) {
+        const __nv_bfloat16* xs = reinterpret_cast<const __nv_bfloat16*>(st + St::X);
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            if (full_chunk || t0 + t + u < t_end) {
-              const float xm = gi == 0 ? xv[u].x : xv[u].y;
-              const float zv = __bfloat162float(zs[(t + u) * kCPW + 2 * cp + gi]);
-              const float y = fmaf(dsk, xm, ysum[u]);
-              if (ypp != nullptr) ypp[(size_t)(t + u) * p.D] = y;
+        for (int t = 0; t < LC; t += 2) {
+          // reduce the partial readouts over the G lanes of the channel pair, scattering them so
+          // that each lane finishes its own (token, channel) outputs
+          float ysum[2];
+          if (G == 2) {
+            // lanes 2cp (states 0-7) and 2cp+1 (states 8-15) swap one partial per token
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const float send = gi == 0 ? ypart[t + u][1] : ypart[t + u][0];
+              const float keep = gi == 0 ? ypart[t + u][0] : ypart[t + u][1];
+              ysum[u] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+            }
+          } else {
+            // step 1 (lanes gi, gi ^ 2): keep token ou, send the other token's two channels
+            float r2[2];
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+              const float send = ou == 0 ? ypart[t + 1][ch] : ypart[t][ch];
+              const float keep = ou == 0 ? ypart[t][ch] : ypart[t + 1][ch];
+              r2[ch] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+            }
+            // step 2 (lanes gi, gi ^ 1): keep channel och, send the other
+            const float send = och == 0 ? r2[1] : r2[0];
+            const float keep = och == 0 ? r2[0] : r2[1];
+            ysum[0] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+            ysum[1] = 0.f;
+          }
+#pragma unroll
+          for (int o = 0; o < (G == 2 ? 2 : 1); ++o) {
+            const int uu = G == 2 ? o : ou;
+            if (full_chunk || t0 + t + uu < t_end) {
+              const float xm = __bfloat162float(xs[(t + uu) * CPW + 2 * cp + och]);
+              const float zv = __bfloat162float(zs[(t + uu) * CPW + 2 * cp + och]);
+              const float y = fmaf(dsk, xm, ysum[o]);
+              if (ypp != nullptr) ypp[(size_t)(t + uu) * p.D] = y;
               const float sig = fmaf(0.5f, tanh_approx(0.5f * zv), 0.5f);
-              outp[(size_t)(t + u) * p.D] = __float2bfloat16_rn(y * zv * sig);
+              outp[(size_t)(t + uu) * p.D] = __float2bfloat16_rn(y * zv * sig);
             }
           }
         }
@@ -394,14 +458,14 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       if (AGG) {
         const size_t o = (((size_t)b * p.S + seg) * p.D + dA + ch) * 16 + n0;
 #pragma unroll
-        for (int s = 0; s < 4; ++s) {
+        for (int s = 0; s < NP; ++s) {
           *reinterpret_cast<float2*>(p.agg_h + o + 2 * s) = h[ch][s];
           *reinterpret_cast<float2*>(p.agg_logp + o + 2 * s) = lsum[ch][s];
         }
       } else if (p.h_final != nullptr && seg == p.S - 1) {
         const size_t o = ((size_t)b * p.D + dA + ch) * 16 + n0;
 #pragma unroll
-        for (int s = 0; s < 4; ++s) *reinterpret_cast<float2*>(p.h_final + o + 2 * s) = h[ch][s];
+        for (int s = 0; s < NP; ++s) *reinterpret_cast<float2*>(p.h_final + o + 2 * s) = h[ch][s];
       }
     }
   }
@@ -462,7 +526,11 @@ int device_sms() {
   return n;
 }
 
-constexpr int kNPoly = 0;  // states per lane and channel whose exp2 runs on the FMA pipe (even, <= 8)
+constexpr int kNPoly = 0;  // states per lane and channel whose exp2 runs on the FMA pipe (even, <= NS)
+#ifndef SWIMBA_SCAN_G
+#define SWIMBA_SCAN_G 2
+#endif
+constexpr int kLanesPerPair = SWIMBA_SCAN_G;  // lanes per channel pair of the launched kernels
 
 }  // namespace
 
@@ -471,13 +539,14 @@ ScanPlan scan_fast_plan(int64_t B, int64_t L, int D, int N, int E, int k, bool i
   ScanPlan pl{};
   pl.fast = io_bf16 && N == 16 && (k == 1 || k == 2) && E >= 1 && E <= 16;
   if (!pl.fast) return pl;
-  const int CPW = kCPW;
+  pl.g = kLanesPerPair;
+  const int CPW = 64 / pl.g;
   if (D % CPW != 0 || B * L > (int64_t(1) << 31)) {
     pl.fast = false;
     return pl;
   }
   const int64_t base_units = B * (D / CPW);
-  const int64_t target = (int64_t)device_sms() * 6;  // at least 6 warps (3072 channels) per SM
+  const int64_t target = (int64_t)device_sms() * 3 * pl.g;  // warps per SM: 6 (G = 2) or 12 (G = 4)
   int64_t S = 1;
   if (base_units < target) S = std::min<int64_t>((target + base_units - 1) / base_units, (L + LC - 1) / LC);
   int64_t Lseg = (L + S - 1) / S;
@@ -489,9 +558,10 @@ ScanPlan scan_fast_plan(int64_t B, int64_t L, int D, int N, int E, int k, bool i
   return pl;
 }
 
-template <int K>
+template <int K, int G>
 static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s) {
-  constexpr int CPW = kCPW;
+  constexpr int CPW = Geo<G>::CPW, MAXW = Geo<G>::MAXW;
+  using St = Stage<CPW>;
   CUtensorMap tx, tz, td, tb, tc;
   if (!map3(&tx, sp.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.D, sp.L, sp.B, CPW) ||
       !map3(&tz, sp.z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.D, sp.L, sp.B, CPW) ||
@@ -524,16 +594,17 @@ static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* s
     cudaFuncAttributes fa;
     cudaError_t err = cudaFuncGetAttributes(&fa, fn);
     if (err != cudaSuccess) return err;
-    const int per_quarter = 512 / tmem_cols_per_warp(sp.E);  // warps that fit one lane quarter's TMEM
-    const int wmax = std::max(1, std::min({kMaxWarps, fa.maxThreadsPerBlock / 32, 4 * per_quarter}));
+    // warps that fit one lane quarter's 512 TMEM columns
+    const int per_quarter = 512 / tmem_cols_per_warp(sp.E, Geo<G>::ACOLS);
+    const int wmax = std::max(1, std::min({MAXW, fa.maxThreadsPerBlock / 32, 4 * per_quarter}));
     ctas = std::max(1, std::min(sms, units));
     warps = std::min(wmax, (units + ctas - 1) / ctas);
     if ((int64_t)ctas * warps < units) ctas = std::min<int64_t>((units + warps - 1) / warps, 65535);
     return cudaSuccess;
   };
   int ctas, warps;
-  const size_t smem_per_warp = (size_t)kStages * Stage::BYTES + (size_t)kStages * 8;
-  const size_t smem = 128 + (size_t)kMaxWarps * smem_per_warp + 32;
+  const size_t smem_per_warp = (size_t)kStages * St::BYTES + (size_t)kStages * 8;
+  const size_t smem = 128 + (size_t)MAXW * smem_per_warp + 32;
   cudaError_t e;
   if (pl.S > 1) {
     float* agg_h = reinterpret_cast<float*>(seg_ws);
@@ -545,7 +616,7 @@ static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* s
     a.h0 = nullptr;
     a.seg_count = pl.S - 1;  // the last segment needs no aggregate
     a.units = sp.B * (pl.S - 1) * (sp.D / CPW);
-    auto kagg = scan_fast_kernel<K, kNPoly, true>;
+    auto kagg = scan_fast_kernel<K, kNPoly, true, G>;
     if ((e = cudaFuncSetAttribute(kagg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
       return e;
     if ((e = shape((const void*)kagg, a.units, ctas, warps)) != cudaSuccess) return e;
@@ -555,7 +626,7 @@ static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* s
     note_launch(2);
     p.h_seg = h_seg;
   }
-  auto kmain = scan_fast_kernel<K, kNPoly, false>;
+  auto kmain = scan_fast_kernel<K, kNPoly, false, G>;
   if ((e = cudaFuncSetAttribute(kmain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
     return e;
   if ((e = shape((const void*)kmain, p.units, ctas, warps)) != cudaSuccess) return e;
@@ -565,7 +636,8 @@ static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* s
 }
 
 cudaError_t run_scan_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s) {
-  return sp.k == 1 ? launch_fast<1>(sp, pl, seg_ws, status, s) : launch_fast<2>(sp, pl, seg_ws, status, s);
+  if (pl.g == 2) return sp.k == 1 ? launch_fast<1, 2>(sp, pl, seg_ws, status, s) : launch_fast<2, 2>(sp, pl, seg_ws, status, s);
+  return sp.k == 1 ? launch_fast<1, 4>(sp, pl, seg_ws, status, s) : launch_fast<2, 4>(sp, pl, seg_ws, status, s);
 }
 
 // ---- scratch for callers that cannot allocate device memory ----------------------------------------
