@@ -26,8 +26,9 @@
  *     the device (a bounded wait that gave up) are written to the status block at the start of
  *     the workspace and returned by swimba_get_device_status.
  *   - Requirements: 1 <= k <= E <= 16; 1 <= N <= 16; D % 8 == 0; 1 <= R <= 256;
- *     x, z, out, delta, W_x, W_dt and the workspace 16-byte aligned. Anything else returns
- *     SWIMBA_ERR_UNSUPPORTED / SWIMBA_ERR_ALIGN; there is no fallback path.
+ *     every tensor pointer (x, z, out, delta, B_mix, C_mix, h0, h_final, y_pre, the weight
+ *     tables) and the workspace 16-byte aligned. Anything else returns SWIMBA_ERR_UNSUPPORTED /
+ *     SWIMBA_ERR_ALIGN; there is no host-side fallback path.
  *   - One workspace must not be used by two calls that may run concurrently.
  */
 #ifndef SWIMBA_H
@@ -89,6 +90,10 @@ size_t swimba_workspace_size(const swimba_dims *dims, int op);
 
 /* Router (the pages' π_t): logits = x W_r accumulated in fp32; idx = the k largest in descending
  * order, equal logits to the lower expert index; gates = softmax of the k selected logits.
+ * bf16 x with D a multiple of 64 and E in {4, 8, 12, 16} runs on the tensor cores (W_r split
+ * exactly into three bf16 parts, fp32 accumulation); other shapes on the SIMT cores. A token whose
+ * routing gave up after a bounded device-side wait (a device error, not expected in operation)
+ * gets idx = -1 and gate 0; the later calls clamp such indices.
  *   x     [B, L, D] io_dtype          (in)
  *   W_r   [D, E] fp32                 (in)
  *   idx   [B, L, k] int32             (out)

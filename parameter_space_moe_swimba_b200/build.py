@@ -17,7 +17,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libswimba.so")
-SOURCES = ["api.cu", "route.cu", "proj_simt.cu", "proj_tc.cu", "scan.cu", "scan_fast.cu"]
+SOURCES = ["api.cu", "route.cu", "route_tc.cu", "proj_simt.cu", "proj_tc.cu", "scan.cu", "scan_fast.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr"]
 

@@ -145,7 +145,9 @@ static swimba_status scan_common(const swimba_dims* dims, const void* x, const v
     return SWIMBA_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(z) || !aligned16(out) || !aligned16(delta)) return SWIMBA_ERR_ALIGN;
   if (dims->d_state == 16 && (!aligned16(B_mix) || !aligned16(C_mix))) return SWIMBA_ERR_ALIGN;
-  if ((h0 && !aligned16(h0)) || (h_final && !aligned16(h_final))) return SWIMBA_ERR_ALIGN;
+  if ((h0 && !aligned16(h0)) || (h_final && !aligned16(h_final)) || (y_pre && !aligned16(y_pre)))
+    return SWIMBA_ERR_ALIGN;
+  if (!aligned16(w->A) || !aligned16(w->D_skip)) return SWIMBA_ERR_ALIGN;
   ScanParams p{x,   z,       delta, B_mix,          C_mix,          idx,           gates,
                w->A, w->D_skip, h0,  out,            h_final,        y_pre,         dims->seqlen,
                (int)dims->batch, dims->d_inner, dims->d_state, dims->n_experts, dims->top_k};

@@ -417,20 +417,21 @@ struct Stage2Params {
   void* status;
 };
 
-// softplus(v) = max(v, 0) + log1p(e^{-|v|}): e^{-|v|} with the ex2 instruction; log1p(e) by its
-// series e - e^2/2 + e^3/3 below e = 2^-6 (truncation < e^4/4), else as ln(1 + e) with the lg2
-// instruction (1 + e >= 1.0156, so the relative error stays near 1e-5 at worst).
+// softplus(v) = max(v, 0) + log1p(e) with e = e^{-|v|} in (0, 1] from the ex2 instruction, and
+// log1p(e) = e q(e), q a degree-7 minimax fit of log1p(e) / e on [0, 1] (fit_log1p_poly.py beside
+// this file; float32 Horner error 3.7e-7 relative). No branch and one special-function
+// instruction, so the 32 values of one TMEM load interleave freely.
 __device__ __forceinline__ float softplus_fast(float v) {
   const float e = ex2_approx(-fabsf(v) * kLog2e);
-  float l;
-  if (e < 0.015625f) {
-    l = e * fmaf(e, fmaf(e, 0.33333334f, -0.5f), 1.f);
-  } else {
-    float lg;
-    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(1.f + e));
-    l = lg * 0.69314718f;
-  }
-  return fmaxf(v, 0.f) + l;
+  float q = -0x1.17d012p-7f;
+  q = fmaf(q, e, 0x1.692eaap-5f);
+  q = fmaf(q, e, -0x1.b91076p-4f);
+  q = fmaf(q, e, 0x1.6b6c2cp-3f);
+  q = fmaf(q, e, -0x1.f5aac6p-3f);
+  q = fmaf(q, e, 0x1.54bdacp-2f);
+  q = fmaf(q, e, -0x1.fff932p-2f);
+  q = fmaf(q, e, 0x1.fffffap-1f);
+  return fmaxf(v, 0.f) + e * q;
 }
 
 template <int K>

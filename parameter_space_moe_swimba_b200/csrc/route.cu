@@ -11,52 +11,9 @@
 // butterfly of warp shuffles; then lane tt selects the experts of token t0+tt.
 #include <algorithm>
 
-#include "common.cuh"
+#include "route.cuh"
 
 namespace swimba {
-
-struct RouteParams {
-  const void* x;
-  const float* W_r;
-  int32_t* idx;
-  float* gates;
-  int64_t T;
-  int D, E, k;
-};
-
-// top-k of one token's logits l[0..E): repeatedly take the largest remaining logit; a strict
-// comparison in ascending expert order keeps the lower index on ties. gates = softmax of the
-// selected logits (exp relative to the largest, so the first gate's weight is exactly 1).
-template <int EP>
-__device__ __forceinline__ void select_topk(const float (&l)[EP], int E, int k, int32_t* idx, float* gates) {
-  unsigned taken = 0u;
-  float wsel[16];
-  float top = 0.f, sum = 0.f;
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    wsel[j] = 0.f;
-    if (j < k) {
-      int bi = -1;
-      float best = 0.f;
-#pragma unroll
-      for (int e = 0; e < EP; ++e) {
-        const bool ok = (e < E) && !((taken >> e) & 1u);
-        if (ok && (bi < 0 || l[e] > best)) {
-          best = l[e];
-          bi = e;
-        }
-      }
-      taken |= 1u << bi;
-      if (j == 0) top = best;
-      wsel[j] = expf(best - top);
-      sum += wsel[j];
-      idx[j] = bi;
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < 16; ++j)
-    if (j < k) gates[j] = wsel[j] / sum;
-}
 
 template <typename IO, int EP, int TOK>
 __global__ void __launch_bounds__(128) route_kernel(RouteParams p) {
@@ -231,6 +188,7 @@ static cudaError_t route_dispatch(const RouteParams& p, cudaStream_t s) {
 cudaError_t run_route(const void* x, bool io_bf16, const float* W_r, int32_t* idx, float* gates, int64_t T,
                       int D, int E, int k, cudaStream_t s) {
   RouteParams p{x, W_r, idx, gates, T, D, E, k};
+  if (route_tc_supported(io_bf16, D, E, k)) return run_route_tc(p, s);
   return io_bf16 ? route_dispatch<__nv_bfloat16>(p, s) : route_dispatch<float>(p, s);
 }
 

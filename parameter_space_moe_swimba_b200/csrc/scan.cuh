@@ -29,7 +29,6 @@ cudaError_t run_scan(const ScanParams& p, bool io_bf16, bool step, cudaStream_t 
 // 16-token chunk) and the workspace the segment carries need.
 struct ScanPlan {
   bool fast;
-  int g;  // fast path: lanes per channel pair (2 or 4)
   int S;
   int64_t Lseg;
   size_t ws_bytes;

@@ -9,15 +9,20 @@
 // Work unit = one warp = 32 channels of one sequence segment. Lane l holds the channel pair
 // (2*(l>>1), 2*(l>>1)+1) of the warp and the 8 states (l&1)*8 .. +7 of both channels, 16 fp32 states
 // in registers; the two lanes of a pair together hold all 16 states of the two channels. So every
-// B_mix / C_mix value a lane loads serves two channels, and one shuffle finishes the readout.
+// B_mix / C_mix value a lane loads serves two channels.
 // The per-expert transition rows (pre-multiplied by log2 e) live in tensor memory: each warp owns
 // E*16 TMEM columns of its lane quarter and keeps expert e's 16 values of every lane at columns
 // 16e..16e+15. Every lane of a warp reads the same token, so the selected expert is warp-uniform
 // and one tcgen05.ld.32x32b.x16 at column 16e fetches it: a dynamically indexed, branch-free lookup
 // that costs no registers and no shared-memory bandwidth.
 // Per token and state:  arg = Σ_j (Δ g_j) A^{e_j};  ā = 2^arg;  h = ā h + (Δ x) B;  y += C h.
-// The two lanes of a pair swap one partial readout so that each finishes one channel's token:
-// y += D_skip x, out = y z σ(z) (σ via tanh.approx for bf16 outputs).
+//
+// A chunk of 16 tokens runs in two passes. The recurrence pass keeps only the state chain: each
+// lane leaves its two partial readouts per token in shared memory. The readout pass then works on
+// the whole chunk at once, with a different lane layout: lane l takes token l/2 and 16 channels,
+// adds the two state halves' partials, the skip term D_skip x and the gate z σ(z) (σ via
+// tanh.approx) with packed f32x2 arithmetic and 16-byte shared-memory loads, and writes 16 bf16
+// outputs; one TMA store per chunk moves the [16 x 32] output tile to HBM (it clips rows past L).
 //
 // Each warp streams its inputs through its own 3-stage shared-memory ring filled by TMA (x, z, Δ
 // tiles of [16 tokens x 32 channels] and B_mix, C_mix rows of 16 tokens) plus the tokens' expert
@@ -44,27 +49,19 @@ namespace {
 
 constexpr int LC = 16;          // tokens per chunk
 constexpr int kStages = 3;      // ring depth per warp
-
-// Lane geometry, by G = lanes per channel pair (2 or 4): each lane holds NS = 16 / G states of two
-// channels; a warp covers CPW = 64 / G channels; a CTA holds up to 8 (G = 2, up to 255 registers a
-// thread) or 16 (G = 4, up to 128) warps.
-template <int G>
-struct Geo {
-  static_assert(G == 2 || G == 4, "2 or 4 lanes per channel pair");
-  static constexpr int NS = 16 / G;        // states per lane and channel
-  static constexpr int NP = NS / 2;        // float2 pairs per lane and channel
-  static constexpr int CPW = 64 / G;       // channels per warp
-  static constexpr int ACOLS = 2 * NS;     // TMEM columns per expert (both channels of a lane)
-  static constexpr int MAXW = 4 * G;       // warps per CTA
-};
+constexpr int kCPW = 32;        // channels per warp
+constexpr int kNS = 8;          // states per lane and channel
+constexpr int kNP = kNS / 2;    // float2 state pairs per lane and channel
+constexpr int kACols = 16;      // TMEM columns per expert (both channels of a lane)
+constexpr int kMaxWarps = 8;    // warps per CTA (registers: up to 255 per thread)
+constexpr int kPRow = kCPW + 4; // floats per row of the partial-readout buffer (padded)
 
 // Byte offsets inside one ring stage of one warp.
-template <int CPW>
 struct Stage {
-  static constexpr int X = 0;                      // bf16 [LC][CPW]
-  static constexpr int Z = X + LC * CPW * 2;       // bf16 [LC][CPW]
-  static constexpr int DL = Z + LC * CPW * 2;      // f32  [LC][CPW]
-  static constexpr int B = DL + LC * CPW * 4;      // f32  [LC][16]
+  static constexpr int X = 0;                      // bf16 [LC][32]
+  static constexpr int Z = X + LC * kCPW * 2;      // bf16 [LC][32]
+  static constexpr int DL = Z + LC * kCPW * 2;     // f32  [LC][32]
+  static constexpr int B = DL + LC * kCPW * 4;     // f32  [LC][16]
   static constexpr int C = B + LC * 16 * 4;        // f32  [LC][16]
   static constexpr int META = C + LC * 16 * 4;     // int4 [LC] {e0, e1, g0, g1}
   static constexpr int BYTES = META + LC * 16;
@@ -73,15 +70,18 @@ struct Stage {
   static_assert(BYTES % 128 == 0, "stage size");
 };
 
-// TMEM columns one warp needs (ACOLS per expert, rounded up to the 32-column allocation granule).
-__host__ __device__ constexpr int tmem_cols_per_warp(int E, int acols) { return ((E * acols + 31) / 32) * 32; }
+// Per-warp readout area (after the ring): partial readouts, two output tiles (the TMA store of
+// one may still be reading while the next is written), the warp's D_skip values.
+struct Epi {
+  static constexpr int P = 0;                              // f32 [LC][2 state halves][kPRow]
+  static constexpr int O = P + LC * 2 * kPRow * 4;         // bf16 [2][LC][32]
+  static constexpr int DS = O + 2 * LC * kCPW * 2;         // f32 [32]
+  static constexpr int BYTES = DS + kCPW * 4;
+  static_assert(O % 128 == 0 && DS % 16 == 0 && BYTES % 128 == 0, "readout area layout");
+};
 
-// n consecutive TMEM columns of this thread's lane, without waiting (n = 8 or 16).
-template <int NCOL>
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NCOL]) {
-  if constexpr (NCOL == 16) tmem_ld16_nowait(taddr, r);
-  else tmem_ld8_nowait(taddr, r);
-}
+// TMEM columns one warp needs (16 per expert, rounded up to the 32-column allocation granule).
+__host__ __device__ constexpr int tmem_cols_per_warp(int E) { return ((E * kACols + 31) / 32) * 32; }
 
 // 2^x on the FMA pipe for x <= 0: x = j + f with j = round(x) (the 1.5*2^23 shifter), f in
 // [-1/2, 1/2]; 2^f by a degree-5 polynomial fitted for minimax relative error on that interval
@@ -111,6 +111,19 @@ __device__ __forceinline__ float tanh_approx(float x) {
   return y;
 }
 
+// 8 bf16 (one 16-byte word) as 4 float2 pairs.
+__device__ __forceinline__ void bf16x8_to_float2(const uint4 q, float2 (&f)[4]) {
+  f[0] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
+  f[1] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
+  f[2] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.z));
+  f[3] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.w));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float2 v) {
+  const __nv_bfloat162 b = __float22bfloat162_rn(v);
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+
 struct FastParams {
   const int32_t* idx;
   const float* gates;
@@ -118,7 +131,6 @@ struct FastParams {
   const float* D_skip;  // [D]
   const float* h0;      // [B, D, 16] or null (start state of segment 0)
   const float* h_seg;   // [B, S, D, 16] start state of every segment (segmented main pass) or null
-  __nv_bfloat16* out;   // [B, L, D]
   float* y_pre;         // [B, L, D] or null
   float* h_final;       // [B, D, 16] or null
   float* agg_h;         // pass 1: [B, S, D, 16] end state from zero
@@ -127,26 +139,30 @@ struct FastParams {
   int64_t L, Lseg;
   int B, D, E, k, S;
   int seg_count;        // segments this pass visits (S, or S - 1 for pass 1)
-  int units;            // B * seg_count * (D / CPW)
+  int units;            // B * seg_count * (D / 32)
 };
 
 // AGG = true: pass 1 (segments 0 .. S-2 only; no readout, no output).
-template <int K, int NPOLY, bool AGG, int G>
-__global__ void __launch_bounds__(Geo<G>::MAXW * 32, 1)
+template <int K, int NPOLY, bool AGG>
+__global__ void __launch_bounds__(kMaxWarps * 32, 1)
     scan_fast_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
                      const __grid_constant__ CUtensorMap tm_dl, const __grid_constant__ CUtensorMap tm_b,
-                     const __grid_constant__ CUtensorMap tm_c, const FastParams p) {
-  constexpr int NS = Geo<G>::NS, NP = Geo<G>::NP, CPW = Geo<G>::CPW, ACOLS = Geo<G>::ACOLS;
-  using St = Stage<CPW>;
+                     const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_o,
+                     const FastParams p) {
+  constexpr int NS = kNS, NP = kNP, CPW = kCPW, ACOLS = kACols;
+  using St = Stage;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwarps = blockDim.x >> 5;
   uint8_t* ring = smem + (size_t)warp * kStages * St::BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)nwarps * kStages * St::BYTES);
+  uint8_t* epi = smem + (size_t)nwarps * kStages * St::BYTES + (size_t)warp * Epi::BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)nwarps * (kStages * St::BYTES + Epi::BYTES));
   uint64_t* full = bars + warp * kStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + nwarps * kStages);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + nwarps * kStages) + 1;
+  float* psm = reinterpret_cast<float*>(epi + Epi::P);
+  const float* dsm = reinterpret_cast<const float*>(epi + Epi::DS);
 
   if (lane == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
@@ -159,6 +175,7 @@ __global__ void __launch_bounds__(Geo<G>::MAXW * 32, 1)
       if (!AGG) {
         prefetch_tmap(&tm_z);
         prefetch_tmap(&tm_c);
+        prefetch_tmap(&tm_o);
       }
     }
   }
@@ -168,21 +185,20 @@ __global__ void __launch_bounds__(Geo<G>::MAXW * 32, 1)
   }
   __syncthreads();
   tc_fence_after();
-  // this warp's TMEM window: its lane quarter, tmem_cols_per_warp(E, ACOLS) columns
+  // this warp's TMEM window: its lane quarter, tmem_cols_per_warp(E) columns
   const uint32_t tbase = *tmem_slot + ((uint32_t)(32 * (warp & 3)) << 16) +
-                         (uint32_t)(warp >> 2) * (uint32_t)tmem_cols_per_warp(p.E, ACOLS);
+                         (uint32_t)(warp >> 2) * (uint32_t)tmem_cols_per_warp(p.E);
 
-  const int cp = lane / G;    // channel pair: channels 2cp, 2cp+1 of the warp's CPW
-  const int gi = lane % G;    // state group: states NS*gi .. NS*gi+NS-1
+  const int cp = lane >> 1;   // recurrence pass: channel pair 2cp, 2cp+1 of the warp's 32
+  const int gi = lane & 1;    //                  state group: states 8gi .. 8gi+7
   const int n0 = gi * NS;
-  // the output this lane finishes: G = 2, channel gi of both tokens of a pair; G = 4, channel
-  // gi & 1 of token gi >> 1 of the pair
-  const int och = G == 2 ? gi : (gi & 1);
-  const int ou = G == 2 ? 0 : (gi >> 1);
+  const int tl = lane >> 1;   // readout pass: token tl of the chunk,
+  const int c0 = (lane & 1) * 16;  //           channels c0 .. c0+15 of the warp's 32
   const int ntiles = p.D / CPW;
   const int u_begin = (int)((int64_t)p.units * blockIdx.x / gridDim.x);
   const int u_end = (int)((int64_t)p.units * (blockIdx.x + 1) / gridDim.x);
   uint32_t phase_bits = 0;  // one parity bit per stage
+  int ochunk = 0;           // output tiles written by this warp (selects the double buffer)
   constexpr uint32_t tx_bytes = AGG ? (LC * CPW * 2 + LC * CPW * 4 + LC * 16 * 4)
                                     : (2 * LC * CPW * 2 + LC * CPW * 4 + 2 * LC * 16 * 4);
 
@@ -196,29 +212,22 @@ __global__ void __launch_bounds__(Geo<G>::MAXW * 32, 1)
     const int64_t t_end = std::min<int64_t>(p.L, t_begin + p.Lseg);
     const int nchunks = (int)((t_end - t_begin + LC - 1) / LC);
 
-    // per-expert transition rows of this lane's 2 x NS states, times log2(e), into TMEM
-    // columns ACOLS*e + NS*ch + s
+    // per-expert transition rows of this lane's 2 x 8 states, times log2(e), into TMEM
+    // columns 16e + 8ch + s
     for (int e = 0; e < p.E; ++e) {
-      uint32_t r[ACOLS];
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
         const float4* src = reinterpret_cast<const float4*>(p.A + ((size_t)e * p.D + dA + ch) * 16 + n0);
-#pragma unroll
-        for (int q = 0; q < NS / 4; ++q) {
-          const float4 a4 = __ldg(src + q);
-          r[ch * NS + 4 * q + 0] = __float_as_uint(a4.x * kLog2e);
-          r[ch * NS + 4 * q + 1] = __float_as_uint(a4.y * kLog2e);
-          r[ch * NS + 4 * q + 2] = __float_as_uint(a4.z * kLog2e);
-          r[ch * NS + 4 * q + 3] = __float_as_uint(a4.w * kLog2e);
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < ACOLS / 8; ++q) {
-        const uint32_t (&r8)[8] = *reinterpret_cast<const uint32_t(*)[8]>(r + 8 * q);
-        tmem_st8(tbase + (uint32_t)(e * ACOLS + 8 * q), r8);
+        const float4 a0 = __ldg(src), a1 = __ldg(src + 1);
+        const uint32_t r[8] = {__float_as_uint(a0.x * kLog2e), __float_as_uint(a0.y * kLog2e),
+                               __float_as_uint(a0.z * kLog2e), __float_as_uint(a0.w * kLog2e),
+                               __float_as_uint(a1.x * kLog2e), __float_as_uint(a1.y * kLog2e),
+                               __float_as_uint(a1.z * kLog2e), __float_as_uint(a1.w * kLog2e)};
+        tmem_st8(tbase + (uint32_t)(e * ACOLS + 8 * ch), r);
       }
     }
     tmem_wait_st();
+    if (!AGG) reinterpret_cast<float*>(epi + Epi::DS)[lane] = p.D_skip[tile * CPW + lane];
 
     float2 h[2][NP];  // [channel][state pair]
 #pragma unroll
@@ -236,8 +245,6 @@ __global__ void __launch_bounds__(Geo<G>::MAXW * 32, 1)
     for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
       for (int s = 0; s < NP; ++s) lsum[ch][s] = make_float2(0.f, 0.f);
-    const int dmine = dA + och;  // the channel whose outputs this lane writes
-    const float dsk = AGG ? 0.f : p.D_skip[dmine];
 
     // meta of one chunk: lane t (< LC) holds token t's {e0, e1, g0, g1}
     auto load_meta = [&](int c) -> int4 {
@@ -293,19 +300,13 @@ __global__ void __launch_bounds__(Geo<G>::MAXW * 32, 1)
       const uint8_t* st = ring + sidx * St::BYTES;
       const int4* meta = reinterpret_cast<const int4*>(st + St::META);
       const __nv_bfloat162* xs2 = reinterpret_cast<const __nv_bfloat162*>(st + St::X);
-      const __nv_bfloat16* zs = reinterpret_cast<const __nv_bfloat16*>(st + St::Z);
       const float2* ds2 = reinterpret_cast<const float2*>(st + St::DL);
       const float4* bsm = reinterpret_cast<const float4*>(st + St::B);
       const float4* csm = reinterpret_cast<const float4*>(st + St::C);
       const int64_t t0 = t_begin + (int64_t)c * LC;
-      const bool full_chunk = t0 + LC <= t_end;
-      __nv_bfloat16* outp = AGG ? nullptr : p.out + ((size_t)b * p.L + t0) * p.D + dmine;
-      float* ypp = (AGG || p.y_pre == nullptr) ? nullptr : p.y_pre + ((size_t)b * p.L + t0) * p.D + dmine;
-      // pass over the chunk's tokens: the recurrence only; readout partials are kept in registers
-      // and the reduction, skip term, gate and stores follow for the whole chunk, off the
-      // recurrence's dependency chain
-      float ypart[LC][2];  // [token][channel]
-#pragma unroll
+
+      // ---- recurrence pass: the state chain only; partial readouts go to shared memory ----
+#pragma unroll 2
       for (int t = 0; t < LC; t += 2) {
         // loads of both tokens first: the selected experts' A rows (TMEM), Δ, x, B, C (smem)
         int4 m[2];
@@ -313,24 +314,24 @@ __global__ void __launch_bounds__(Geo<G>::MAXW * 32, 1)
         float2 dl[2], xv[2];
         float2 bv[2][NP], cv[2][NP];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          m[u] = meta[t + u];
-          tmem_ld_cols<ACOLS>(tbase + (uint32_t)(m[u].x * ACOLS), ar[u][0]);
-          if (K == 2) tmem_ld_cols<ACOLS>(tbase + (uint32_t)(m[u].y * ACOLS), ar[u][1]);
+        for (int u2 = 0; u2 < 2; ++u2) {
+          m[u2] = meta[t + u2];
+          tmem_ld16_nowait(tbase + (uint32_t)(m[u2].x * ACOLS), ar[u2][0]);
+          if (K == 2) tmem_ld16_nowait(tbase + (uint32_t)(m[u2].y * ACOLS), ar[u2][1]);
         }
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          dl[u] = ds2[(t + u) * (CPW / 2) + cp];
-          xv[u] = __bfloat1622float2(xs2[(t + u) * (CPW / 2) + cp]);
+        for (int u2 = 0; u2 < 2; ++u2) {
+          dl[u2] = ds2[(t + u2) * (CPW / 2) + cp];
+          xv[u2] = __bfloat1622float2(xs2[(t + u2) * (CPW / 2) + cp]);
 #pragma unroll
-          for (int q = 0; q < NS / 4; ++q) {
-            const float4 bq = bsm[(t + u) * 4 + gi * (NS / 4) + q];
-            bv[u][2 * q] = make_float2(bq.x, bq.y);
-            bv[u][2 * q + 1] = make_float2(bq.z, bq.w);
+          for (int q = 0; q < 2; ++q) {
+            const float4 bq = bsm[(t + u2) * 4 + gi * 2 + q];
+            bv[u2][2 * q] = make_float2(bq.x, bq.y);
+            bv[u2][2 * q + 1] = make_float2(bq.z, bq.w);
             if (!AGG) {
-              const float4 cq = csm[(t + u) * 4 + gi * (NS / 4) + q];
-              cv[u][2 * q] = make_float2(cq.x, cq.y);
-              cv[u][2 * q + 1] = make_float2(cq.z, cq.w);
+              const float4 cq = csm[(t + u2) * 4 + gi * 2 + q];
+              cv[u2][2 * q] = make_float2(cq.x, cq.y);
+              cv[u2][2 * q + 1] = make_float2(cq.z, cq.w);
             }
           }
         }
@@ -339,97 +340,109 @@ __global__ void __launch_bounds__(Geo<G>::MAXW * 32, 1)
         float2 a[2][2][NP];  // [token][channel][state pair]
         float2 arg[2][2][NP];
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
+        for (int u2 = 0; u2 < 2; ++u2)
 #pragma unroll
           for (int ch = 0; ch < 2; ++ch) {
-            const float dlt = ch == 0 ? dl[u].x : dl[u].y;
-            const float c0 = dlt * __int_as_float(m[u].z);
-            const float c1 = dlt * __int_as_float(m[u].w);
+            const float dlt = ch == 0 ? dl[u2].x : dl[u2].y;
+            const float g0 = dlt * __int_as_float(m[u2].z);
+            const float g1 = dlt * __int_as_float(m[u2].w);
 #pragma unroll
             for (int s = 0; s < NP; ++s) {
-              const float2 a0 = make_float2(__uint_as_float(ar[u][0][ch * NS + 2 * s]), __uint_as_float(ar[u][0][ch * NS + 2 * s + 1]));
-              arg[u][ch][s] = __fmul2_rn(make_float2(c0, c0), a0);
+              const float2 a0 = make_float2(__uint_as_float(ar[u2][0][ch * NS + 2 * s]), __uint_as_float(ar[u2][0][ch * NS + 2 * s + 1]));
+              arg[u2][ch][s] = __fmul2_rn(make_float2(g0, g0), a0);
               if (K == 2) {
                 const float2 a1 =
-                    make_float2(__uint_as_float(ar[u][1][ch * NS + 2 * s]), __uint_as_float(ar[u][1][ch * NS + 2 * s + 1]));
-                arg[u][ch][s] = __ffma2_rn(make_float2(c1, c1), a1, arg[u][ch][s]);
+                    make_float2(__uint_as_float(ar[u2][1][ch * NS + 2 * s]), __uint_as_float(ar[u2][1][ch * NS + 2 * s + 1]));
+                arg[u2][ch][s] = __ffma2_rn(make_float2(g1, g1), a1, arg[u2][ch][s]);
               }
               if (s >= NP - NPOLY / 2) {
-                a[u][ch][s] = exp2_poly2(arg[u][ch][s]);
+                a[u2][ch][s] = exp2_poly2(arg[u2][ch][s]);
               } else {
-                a[u][ch][s] = make_float2(ex2_approx(arg[u][ch][s].x), ex2_approx(arg[u][ch][s].y));
+                a[u2][ch][s] = make_float2(ex2_approx(arg[u2][ch][s].x), ex2_approx(arg[u2][ch][s].y));
               }
             }
           }
-        // the recurrence, token t then t+1; this lane's partial readouts go to ypart
+        // the recurrence, token t then t+1
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u2 = 0; u2 < 2; ++u2) {
+          float yc[2];
 #pragma unroll
           for (int ch = 0; ch < 2; ++ch) {
-            const float dx = (ch == 0 ? dl[u].x : dl[u].y) * (ch == 0 ? xv[u].x : xv[u].y);
+            const float dx = (ch == 0 ? dl[u2].x : dl[u2].y) * (ch == 0 ? xv[u2].x : xv[u2].y);
             const float2 dxx = make_float2(dx, dx);
 #pragma unroll
-            for (int s = 0; s < NP; ++s) h[ch][s] = __ffma2_rn(a[u][ch][s], h[ch][s], __fmul2_rn(dxx, bv[u][s]));
+            for (int s = 0; s < NP; ++s) h[ch][s] = __ffma2_rn(a[u2][ch][s], h[ch][s], __fmul2_rn(dxx, bv[u2][s]));
             if (AGG) {
 #pragma unroll
-              for (int s = 0; s < NP; ++s) lsum[ch][s] = __fadd2_rn(lsum[ch][s], arg[u][ch][s]);
+              for (int s = 0; s < NP; ++s) lsum[ch][s] = __fadd2_rn(lsum[ch][s], arg[u2][ch][s]);
             } else {
               // two independent accumulation chains (even and odd state pairs)
-              float2 ya = __fmul2_rn(cv[u][0], h[ch][0]);
-              float2 yb = __fmul2_rn(cv[u][1], h[ch][1]);
+              float2 ya = __fmul2_rn(cv[u2][0], h[ch][0]);
+              float2 yb = __fmul2_rn(cv[u2][1], h[ch][1]);
 #pragma unroll
               for (int s = 2; s < NP; s += 2) {
-                ya = __ffma2_rn(cv[u][s], h[ch][s], ya);
-                yb = __ffma2_rn(cv[u][s + 1], h[ch][s + 1], yb);
+                ya = __ffma2_rn(cv[u2][s], h[ch][s], ya);
+                yb = __ffma2_rn(cv[u2][s + 1], h[ch][s + 1], yb);
               }
-              ypart[t + u][ch] = (ya.x + yb.x) + (ya.y + yb.y);
+              yc[ch] = (ya.x + yb.x) + (ya.y + yb.y);
             }
           }
+          if (!AGG) *reinterpret_cast<float2*>(psm + ((t + u2) * 2 + gi) * kPRow + 2 * cp) = make_float2(yc[0], yc[1]);
         }
       }
+
+      // ---- readout pass: lane = (token tl, channels c0..c0+15) ----
       if (!AGG) {
-        const __nv_bfloat16* xs = reinterpret_cast<const __nv_bfloat16*>(st + St::X);
+        __syncwarp();
+        const float4* p0 = reinterpret_cast<const float4*>(psm + (tl * 2 + 0) * kPRow + c0);
+        const float4* p1 = reinterpret_cast<const float4*>(psm + (tl * 2 + 1) * kPRow + c0);
+        const uint4* xq = reinterpret_cast<const uint4*>(st + St::X + (tl * CPW + c0) * 2);
+        const uint4* zq = reinterpret_cast<const uint4*>(st + St::Z + (tl * CPW + c0) * 2);
+        const float4* dq = reinterpret_cast<const float4*>(dsm + c0);
+        uint32_t packed[8];
 #pragma unroll
-        for (int t = 0; t < LC; t += 2) {
-          // reduce the partial readouts over the G lanes of the channel pair, scattering them so
-          // that each lane finishes its own (token, channel) outputs
-          float ysum[2];
-          if (G == 2) {
-            // lanes 2cp (states 0-7) and 2cp+1 (states 8-15) swap one partial per token
+        for (int hq = 0; hq < 2; ++hq) {  // 8 channels at a time
+          float2 xf[4], zf[4];
+          bf16x8_to_float2(xq[hq], xf);
+          bf16x8_to_float2(zq[hq], zf);
+          float2 yv[4], dk[4];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const float send = gi == 0 ? ypart[t + u][1] : ypart[t + u][0];
-              const float keep = gi == 0 ? ypart[t + u][0] : ypart[t + u][1];
-              ysum[u] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
-            }
-          } else {
-            // step 1 (lanes gi, gi ^ 2): keep token ou, send the other token's two channels
-            float r2[2];
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-              const float send = ou == 0 ? ypart[t + 1][ch] : ypart[t][ch];
-              const float keep = ou == 0 ? ypart[t][ch] : ypart[t + 1][ch];
-              r2[ch] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-            }
-            // step 2 (lanes gi, gi ^ 1): keep channel och, send the other
-            const float send = och == 0 ? r2[1] : r2[0];
-            const float keep = och == 0 ? r2[0] : r2[1];
-            ysum[0] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
-            ysum[1] = 0.f;
+          for (int i = 0; i < 2; ++i) {
+            const float4 a4 = p0[2 * hq + i], b4 = p1[2 * hq + i], d4 = dq[2 * hq + i];
+            yv[2 * i] = __fadd2_rn(make_float2(a4.x, a4.y), make_float2(b4.x, b4.y));
+            yv[2 * i + 1] = __fadd2_rn(make_float2(a4.z, a4.w), make_float2(b4.z, b4.w));
+            dk[2 * i] = make_float2(d4.x, d4.y);
+            dk[2 * i + 1] = make_float2(d4.z, d4.w);
           }
 #pragma unroll
-          for (int o = 0; o < (G == 2 ? 2 : 1); ++o) {
-            const int uu = G == 2 ? o : ou;
-            if (full_chunk || t0 + t + uu < t_end) {
-              const float xm = __bfloat162float(xs[(t + uu) * CPW + 2 * cp + och]);
-              const float zv = __bfloat162float(zs[(t + uu) * CPW + 2 * cp + och]);
-              const float y = fmaf(dsk, xm, ysum[o]);
-              if (ypp != nullptr) ypp[(size_t)(t + uu) * p.D] = y;
-              const float sig = fmaf(0.5f, tanh_approx(0.5f * zv), 0.5f);
-              outp[(size_t)(t + uu) * p.D] = __float2bfloat16_rn(y * zv * sig);
-            }
+          for (int i = 0; i < 4; ++i) {
+            const float2 y = __ffma2_rn(dk[i], xf[i], yv[i]);  // y + D_skip x
+            yv[i] = y;
+            const float2 hz = __fmul2_rn(zf[i], make_float2(0.5f, 0.5f));
+            const float2 th = make_float2(tanh_approx(hz.x), tanh_approx(hz.y));
+            const float2 sig = __ffma2_rn(th, make_float2(0.5f, 0.5f), make_float2(0.5f, 0.5f));
+            packed[4 * hq + i] = pack_bf16x2(__fmul2_rn(__fmul2_rn(y, zf[i]), sig));
+          }
+          if (p.y_pre != nullptr && t0 + tl < t_end) {
+            float4* yp = reinterpret_cast<float4*>(p.y_pre + ((size_t)b * p.L + t0 + tl) * p.D + tile * CPW + c0 + 8 * hq);
+            yp[0] = make_float4(yv[0].x, yv[0].y, yv[1].x, yv[1].y);
+            yp[1] = make_float4(yv[2].x, yv[2].y, yv[3].x, yv[3].y);
           }
         }
+        // the previous TMA store from this output buffer must have finished reading it
+        uint8_t* obuf = epi + Epi::O + (ochunk & 1) * (LC * CPW * 2);
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        uint4* od = reinterpret_cast<uint4*>(obuf + (tl * CPW + c0) * 2);
+        od[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        od[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tm_o, obuf, tile * CPW, (int)t0, b);
+          bulk_commit();
+        }
+        ++ochunk;
       }
       __syncwarp();
       if (c + kStages < nchunks) {
@@ -468,7 +481,10 @@ __global__ void __launch_bounds__(Geo<G>::MAXW * 32, 1)
         for (int s = 0; s < NP; ++s) *reinterpret_cast<float2*>(p.h_final + o + 2 * s) = h[ch][s];
       }
     }
+    __syncwarp();
   }
+  // the output stores must have read their shared-memory tiles before the CTA's memory goes away
+  if (!AGG && lane == 0) bulk_wait<0>();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
@@ -526,11 +542,7 @@ int device_sms() {
   return n;
 }
 
-constexpr int kNPoly = 0;  // states per lane and channel whose exp2 runs on the FMA pipe (even, <= NS)
-#ifndef SWIMBA_SCAN_G
-#define SWIMBA_SCAN_G 2
-#endif
-constexpr int kLanesPerPair = SWIMBA_SCAN_G;  // lanes per channel pair of the launched kernels
+constexpr int kNPoly = 0;  // states per lane and channel whose exp2 runs on the FMA pipe (even, <= 8)
 
 }  // namespace
 
@@ -539,14 +551,12 @@ ScanPlan scan_fast_plan(int64_t B, int64_t L, int D, int N, int E, int k, bool i
   ScanPlan pl{};
   pl.fast = io_bf16 && N == 16 && (k == 1 || k == 2) && E >= 1 && E <= 16;
   if (!pl.fast) return pl;
-  pl.g = kLanesPerPair;
-  const int CPW = 64 / pl.g;
-  if (D % CPW != 0 || B * L > (int64_t(1) << 31)) {
+  if (D % kCPW != 0 || B * L > (int64_t(1) << 31)) {
     pl.fast = false;
     return pl;
   }
-  const int64_t base_units = B * (D / CPW);
-  const int64_t target = (int64_t)device_sms() * 3 * pl.g;  // warps per SM: 6 (G = 2) or 12 (G = 4)
+  const int64_t base_units = B * (D / kCPW);
+  const int64_t target = (int64_t)device_sms() * 6;  // at least 6 warps (192 channels) per SM
   int64_t S = 1;
   if (base_units < target) S = std::min<int64_t>((target + base_units - 1) / base_units, (L + LC - 1) / LC);
   int64_t Lseg = (L + S - 1) / S;
@@ -558,16 +568,16 @@ ScanPlan scan_fast_plan(int64_t B, int64_t L, int D, int N, int E, int k, bool i
   return pl;
 }
 
-template <int K, int G>
+template <int K>
 static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s) {
-  constexpr int CPW = Geo<G>::CPW, MAXW = Geo<G>::MAXW;
-  using St = Stage<CPW>;
-  CUtensorMap tx, tz, td, tb, tc;
+  constexpr int CPW = kCPW;
+  CUtensorMap tx, tz, td, tb, tc, to;
   if (!map3(&tx, sp.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.D, sp.L, sp.B, CPW) ||
       !map3(&tz, sp.z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.D, sp.L, sp.B, CPW) ||
       !map3(&td, sp.delta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, sp.D, sp.L, sp.B, CPW) ||
       !map3(&tb, sp.B_mix, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 16, sp.L, sp.B, 16) ||
-      !map3(&tc, sp.C_mix, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 16, sp.L, sp.B, 16))
+      !map3(&tc, sp.C_mix, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 16, sp.L, sp.B, 16) ||
+      !map3(&to, sp.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.D, sp.L, sp.B, CPW))
     return cudaErrorInvalidValue;
   FastParams p{};
   p.idx = sp.idx;
@@ -575,7 +585,6 @@ static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* s
   p.A = sp.A;
   p.D_skip = sp.D_skip;
   p.h0 = sp.h0;
-  p.out = reinterpret_cast<__nv_bfloat16*>(sp.out);
   p.y_pre = sp.y_pre;
   p.h_final = sp.h_final;
   p.status = status;
@@ -594,17 +603,16 @@ static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* s
     cudaFuncAttributes fa;
     cudaError_t err = cudaFuncGetAttributes(&fa, fn);
     if (err != cudaSuccess) return err;
-    // warps that fit one lane quarter's 512 TMEM columns
-    const int per_quarter = 512 / tmem_cols_per_warp(sp.E, Geo<G>::ACOLS);
-    const int wmax = std::max(1, std::min({MAXW, fa.maxThreadsPerBlock / 32, 4 * per_quarter}));
+    const int per_quarter = 512 / tmem_cols_per_warp(sp.E);  // warps that fit one lane quarter's TMEM
+    const int wmax = std::max(1, std::min({kMaxWarps, fa.maxThreadsPerBlock / 32, 4 * per_quarter}));
     ctas = std::max(1, std::min(sms, units));
     warps = std::min(wmax, (units + ctas - 1) / ctas);
     if ((int64_t)ctas * warps < units) ctas = std::min<int64_t>((units + warps - 1) / warps, 65535);
     return cudaSuccess;
   };
   int ctas, warps;
-  const size_t smem_per_warp = (size_t)kStages * St::BYTES + (size_t)kStages * 8;
-  const size_t smem = 128 + (size_t)MAXW * smem_per_warp + 32;
+  const size_t smem_per_warp = (size_t)kStages * Stage::BYTES + Epi::BYTES + (size_t)kStages * 8;
+  const size_t smem = 128 + (size_t)kMaxWarps * smem_per_warp + 32;
   cudaError_t e;
   if (pl.S > 1) {
     float* agg_h = reinterpret_cast<float*>(seg_ws);
@@ -616,28 +624,27 @@ static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* s
     a.h0 = nullptr;
     a.seg_count = pl.S - 1;  // the last segment needs no aggregate
     a.units = sp.B * (pl.S - 1) * (sp.D / CPW);
-    auto kagg = scan_fast_kernel<K, kNPoly, true, G>;
+    auto kagg = scan_fast_kernel<K, kNPoly, true>;
     if ((e = cudaFuncSetAttribute(kagg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
       return e;
     if ((e = shape((const void*)kagg, a.units, ctas, warps)) != cudaSuccess) return e;
-    kagg<<<ctas, warps * 32, 128 + warps * smem_per_warp + 32, s>>>(tx, tz, td, tb, tc, a);
+    kagg<<<ctas, warps * 32, 128 + warps * smem_per_warp + 32, s>>>(tx, tz, td, tb, tc, to, a);
     const int64_t n = (int64_t)sp.B * sp.D * 16;
     scan_carry_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(sp.h0, agg_h, agg_logp, h_seg, sp.B, pl.S, sp.D);
     note_launch(2);
     p.h_seg = h_seg;
   }
-  auto kmain = scan_fast_kernel<K, kNPoly, false, G>;
+  auto kmain = scan_fast_kernel<K, kNPoly, false>;
   if ((e = cudaFuncSetAttribute(kmain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
     return e;
   if ((e = shape((const void*)kmain, p.units, ctas, warps)) != cudaSuccess) return e;
-  kmain<<<ctas, warps * 32, 128 + warps * smem_per_warp + 32, s>>>(tx, tz, td, tb, tc, p);
+  kmain<<<ctas, warps * 32, 128 + warps * smem_per_warp + 32, s>>>(tx, tz, td, tb, tc, to, p);
   note_launch();
   return cudaGetLastError();
 }
 
 cudaError_t run_scan_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s) {
-  if (pl.g == 2) return sp.k == 1 ? launch_fast<1, 2>(sp, pl, seg_ws, status, s) : launch_fast<2, 2>(sp, pl, seg_ws, status, s);
-  return sp.k == 1 ? launch_fast<1, 4>(sp, pl, seg_ws, status, s) : launch_fast<2, 4>(sp, pl, seg_ws, status, s);
+  return sp.k == 1 ? launch_fast<1>(sp, pl, seg_ws, status, s) : launch_fast<2>(sp, pl, seg_ws, status, s);
 }
 
 // ---- scratch for callers that cannot allocate device memory ----------------------------------------
