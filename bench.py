@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--report", action="store_true",
+                    help="per-workload table (one JSON line each): every workload, decode steps, E sweep")
     return ap.parse_args()
 
 
@@ -68,6 +70,32 @@ def load_peaks():
 # ------------------------------------------------------------------------------------------------
 # algorithmic bytes per token (only the k active experts count)
 # ------------------------------------------------------------------------------------------------
+
+def measured_traffic(cfg):
+    """DRAM bytes per scan launch from the committed ncu summary (dram__bytes_read.sum +
+    dram__bytes_write.sum), or None when the summary is for another workload or the scan kernel's
+    source has changed since it was taken."""
+    import hashlib
+
+    if cfg.name != "mamba1p4b_like" or cfg.batch != CONFIGS["mamba1p4b_like"].batch:
+        return None
+    summary = os.path.join(ROOT, "profiles", "scan_fast_mamba1p4b_like.md")
+    src = os.path.join(ROOT, "parameter_space_moe_swimba_b200", "csrc", "scan_fast.cu")
+    try:
+        fields = {}
+        with open(summary) as f:
+            for line in f:
+                k, sep, v = line.strip().partition(": ")
+                if sep and k in ("kernel_source_sha256", "dram_bytes_per_launch"):
+                    fields[k] = v.strip()
+        with open(src, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    if fields.get("kernel_source_sha256") != digest or "dram_bytes_per_launch" not in fields:
+        return None
+    return int(fields["dram_bytes_per_launch"])
+
 
 def io_bytes(cfg):
     return 2 if cfg.io_dtype == "bf16" else 4
@@ -343,9 +371,129 @@ def config_block(cfg):
 
 
 # ------------------------------------------------------------------------------------------------
+# --report: every workload, the decode step and the E sweep (one JSON line each)
+# ------------------------------------------------------------------------------------------------
+
+class L2Flush:
+    """Writes a buffer larger than the 126 MB L2 between timed runs (outside the timed events)."""
+
+    def __init__(self, torch, device):
+        self.buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+
+    def __call__(self):
+        self.buf.zero_()
+
+
+def _median_kernel_ms(torch, run, reps, warmup, flush, nev):
+    for _ in range(warmup):
+        flush()
+        run(None)
+    torch.cuda.synchronize()
+    per = []
+    for _ in range(reps):
+        flush()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(nev)]
+        run(ev)
+        torch.cuda.synchronize()
+        per.append([ev[i].elapsed_time(ev[i + 1]) for i in range(nev - 1)])
+    cols = list(zip(*per))
+    return [statistics.median(c) for c in cols], statistics.median([sum(r) for r in per])
+
+
+def report_workload(torch, S, cfg, peaks, flush, reps, warmup):
+    x, z = synth.draw_activations(cfg)
+    layer = GpuLayer(S, cfg, x, z, "cuda:0")
+    (r_ms, p_ms, s_ms), tot = _median_kernel_ms(torch, layer.step, reps, warmup, flush, 4)
+    T = cfg.tokens
+    scan_bytes = scan_bytes_per_token(cfg) * T + 4 * cfg.batch * cfg.d_inner * cfg.d_state
+    pf = proj_flops_per_token(cfg) * T
+    pb = proj_bytes_per_token(cfg) * T
+    tc_peak = peaks["bf16_tflops"] * 1e12
+    proj_bound_s = max(pf / tc_peak, pb / (peaks["hbm_gbs"] * 1e9))
+    exps = T * cfg.d_inner * cfg.d_state
+    mufu_peak = 16 * 148 * peaks["sm_max_mhz"] * 1e6
+    S.check(S.swimba_get_device_status(layer.buf.ws, layer.stream), "device status")
+    return {
+        "report": "workload", "workload": cfg.name, "tokens": T, "layer_us": 1e3 * tot,
+        "tokens_per_s": T / (tot / 1e3),
+        "route_us": 1e3 * r_ms, "route_gbs": route_bytes_per_token(cfg) * T / (r_ms / 1e3) / 1e9,
+        "proj_us": 1e3 * p_ms, "proj_gbs": pb / (p_ms / 1e3) / 1e9, "proj_tflops": pf / (p_ms / 1e3) / 1e12,
+        "proj_frac_of_tc_peak": pf / (p_ms / 1e3) / tc_peak,
+        "proj_frac_of_min_tc_bw": proj_bound_s / (p_ms / 1e3),
+        "scan_us": 1e3 * s_ms, "scan_gbs": scan_bytes / (s_ms / 1e3) / 1e9,
+        "scan_frac_of_hbm": scan_bytes / (s_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+        "scan_frac_of_mufu": exps / (s_ms / 1e3) / mufu_peak,
+        "median_of": reps, "l2": "flushed (256 MB write) before every run",
+    }
+
+
+def report_decode(torch, S, cfg, peaks, flush, steps):
+    """``steps`` decode steps (route -> mixed_proj -> step) on one cached state, L2 flushed before
+    every step; the same x, z every step (draws of step 0)."""
+    dims = S.make_dims(cfg)
+    w = S.upload_weights(synth.draw_weights(cfg), "cuda:0")
+    ws = w.struct()
+    x, z = synth.draw_step_activations(cfg, 0)
+    xd, zd = S.to_device(x, cfg.io_dtype, "cuda:0"), S.to_device(z, cfg.io_dtype, "cuda:0")
+    h = torch.from_numpy(synth.draw_h0(cfg)).to("cuda:0")
+    buf = S.LayerBuffers(dims, torch.bfloat16, "cuda:0")
+    s = torch.cuda.current_stream()
+
+    def run(ev):
+        if ev is not None:
+            ev[0].record(s)
+        S.check(S.swimba_route(dims, xd, ws.W_r, buf.idx, buf.gates, s), "route")
+        if ev is not None:
+            ev[1].record(s)
+        S.check(S.swimba_mixed_proj(dims, xd, buf.idx, buf.gates, ws, buf.delta, buf.B_mix, buf.C_mix, buf.ws,
+                                    buf.ws.numel(), s), "proj")
+        if ev is not None:
+            ev[2].record(s)
+        S.check(S.swimba_step(dims, xd, zd, buf.delta, buf.B_mix, buf.C_mix, buf.idx, buf.gates, ws, h, buf.out, s),
+                "step")
+        if ev is not None:
+            ev[3].record(s)
+
+    (r_ms, p_ms, st_ms), tot = _median_kernel_ms(torch, run, steps, 3, flush, 4)
+    B, D, N = cfg.batch, cfg.d_inner, cfg.d_state
+    step_bytes = scan_bytes_per_token(cfg) * B + 2 * 4 * B * D * N
+    return {
+        "report": "decode", "workload": cfg.name, "steps": steps, "layer_us_per_step": 1e3 * tot,
+        "route_us": 1e3 * r_ms, "proj_us": 1e3 * p_ms, "step_us": 1e3 * st_ms,
+        "step_gbs": step_bytes / (st_ms / 1e3) / 1e9, "step_frac_of_hbm": step_bytes / (st_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+        "l2": "flushed before every step", "inputs": "x, z of step 0 reused every step; the state evolves",
+    }
+
+
+def run_report(args):
+    import torch
+
+    from parameter_space_moe_swimba_b200 import swimba as S
+
+    torch.cuda.set_device(0)
+    peaks = load_peaks()
+    flush = L2Flush(torch, "cuda:0")
+    reps = 20
+    for name in ["tiny_fp32", "mamba130m_like", "mamba1p4b_like", "long_seq_65536"]:
+        print(json.dumps(report_workload(torch, S, CONFIGS[name], peaks, flush, reps, args.warmup)), flush=True)
+    print(json.dumps(report_decode(torch, S, CONFIGS["decode_b256"], peaks, flush, 1000)), flush=True)
+    # Theorem 2: the recurrence's cost does not grow with E (k = 2 fixed; E = 1 forces k = 1)
+    base = CONFIGS["mamba1p4b_like"]
+    for E in (1, 4, 8, 16):
+        cfg = base.with_(name=f"mamba1p4b_like_E{E}", n_experts=E, top_k=min(2, E))
+        row = report_workload(torch, S, cfg, peaks, flush, reps, args.warmup)
+        row["report"] = "e_sweep"
+        row["n_experts"], row["top_k"] = E, cfg.top_k
+        print(json.dumps(row), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------------
 
 def main():
     args = parse()
+    if args.report:
+        return run_report(args)
     cfg = CONFIGS[args.workload]
     if args.batch > 0:
         cfg = cfg.with_(batch=args.batch)
@@ -404,8 +552,16 @@ def main():
     scan_bytes = scan_bytes_per_token(cfg) * cfg.tokens + 4 * cfg.batch * cfg.d_inner * cfg.d_state
     achieved = scan_bytes / (per_kernel["scan"] / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None, "kernel": "scan_fwd",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": measured_traffic(cfg), "kernel": "scan_fwd",
                 "algorithmic_bytes_per_launch": scan_bytes, "peak_source": peaks["source"]}
+    # the scan's arithmetic bound: one ex2 per (token, channel, state) and one tanh per (token,
+    # channel) on the special-function unit, 16 per clock per SM at the maximum SM clock
+    mufu_ops = cfg.tokens * cfg.d_inner * (cfg.d_state + 1)
+    mufu_peak = 16 * 148 * peaks["sm_max_mhz"] * 1e6
+    mufu_achieved = mufu_ops / (per_kernel["scan"] / 1e3)
+    alu_roofline = {"bound": "alu", "unit": "MUFU ops/s", "achieved": mufu_achieved, "peak": mufu_peak,
+                    "frac": mufu_achieved / mufu_peak, "kernel": "scan_fwd",
+                    "peak_from": "16 MUFU ops per clock per SM x 148 SMs x max SM clock"}
     kernels = {
         "route_us": 1e3 * per_kernel["route"], "proj_us": 1e3 * per_kernel["proj"], "scan_us": 1e3 * per_kernel["scan"],
         "route_gbs": route_bytes_per_token(cfg) * cfg.tokens / (per_kernel["route"] / 1e3) / 1e9,
@@ -428,7 +584,7 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_block(cfg),
-            "roofline": roofline, "kernels": kernels, "switch_vs_dense_e1": dense, "e2e": e2e,
+            "roofline": roofline, "alu_roofline": alu_roofline, "kernels": kernels, "switch_vs_dense_e1": dense, "e2e": e2e,
             "gpu_launches": launches, "clocks": clk, "cpu_baseline": cpu,
             "compute": "bf16 x/W on tensor cores with fp32 accumulation; fp32 state and scan arithmetic",
         }
