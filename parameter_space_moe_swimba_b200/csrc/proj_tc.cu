@@ -39,8 +39,12 @@ namespace {
 
 constexpr int BM = 128;        // rows (token slots) per tile
 constexpr int BK1 = 64;        // stage-1 K slice per ring stage (128 bytes of bf16 per row)
-constexpr int kStages1 = 3;
-constexpr int kSlot1 = 65536;  // A 16 KB + up to 6 W_x boxes of 8 KB
+// Stage 1 keeps two rings: the gathered x rows (A, 16 KB a slot) are the slow, latency-bound
+// loads, so their ring is deeper than the W_x ring (up to 6 boxes of 8 KB a slot, L2-resident).
+constexpr int kStagesA = 5;
+constexpr int kSlotA = 16384;
+constexpr int kStagesW = 3;
+constexpr int kSlotW = 49152;
 constexpr int NC = 256;        // stage-2 output columns per chunk
 constexpr int kStages2 = 3;
 constexpr int kSlot2 = 32768;  // 4 W_dt boxes of up to 64 rows x 128 B
@@ -207,25 +211,33 @@ __device__ __forceinline__ void wait_all_mma(uint64_t* done) {
 }
 
 template <int K>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(224, 1)
     proj_stage1_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wx,
                        const Stage1Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* ring = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages1 * kSlot1);
-  uint64_t* empty = full + kStages1;
-  uint64_t* acc_full = empty + kStages1;
+  uint8_t* ring_a = smem;
+  uint8_t* ring_w = smem + kStagesA * kSlotA;
+  uint64_t* full_a = reinterpret_cast<uint64_t*>(ring_w + kStagesW * kSlotW);
+  uint64_t* empty_a = full_a + kStagesA;
+  uint64_t* full_w = empty_a + kStagesA;
+  uint64_t* empty_w = full_w + kStagesW;
+  uint64_t* acc_full = empty_w + kStagesW;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* done = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+  // warp 0: x-row gathers; warp 1: MMA; warps 2-5: epilogue; warp 6: W_x boxes
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages1; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < kStagesA; ++s) {
+      mbar_init(&full_a[s], 1);
+      mbar_init(&empty_a[s], 1);
+    }
+    for (int s = 0; s < kStagesW; ++s) {
+      mbar_init(&full_w[s], 1);
+      mbar_init(&empty_w[s], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 4);
@@ -246,10 +258,10 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
   const int num_tiles = *p.num_tiles;
   const int ksteps = p.D / BK1;
-  const uint32_t slot_bytes = 16384u + (uint32_t)(K * p.nbw) * 8192u;
+  const uint32_t w_bytes = (uint32_t)(K * p.nbw) * 8192u;
 
   if (warp == 0) {
-    // ---------------- producer ----------------
+    // ---------------- producer of A: 128 gathered x rows per K slice ----------------
     int stage = 0, issued = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -258,22 +270,17 @@ __global__ void __launch_bounds__(192, 1)
       int rr[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) rr[i] = p.slot_tok[ti.row_begin + min(4 * lane + i, ti.rows - 1)];
-      const int ej[2] = {ti.e0, ti.e1};
       for (int ks = 0; ks < ksteps; ++ks) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+        if (!mbar_wait(&empty_a[stage], phase ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
-        uint8_t* slot = ring + stage * kSlot1;
-        if (lane == 0) mbar_arrive_expect_tx(&full[stage], slot_bytes);
+        uint8_t* slot = ring_a + stage * kSlotA;
+        if (lane == 0) mbar_arrive_expect_tx(&full_a[stage], (uint32_t)kSlotA);
         __syncwarp();
-        tma_gather4(slot + lane * 512, &tm_x, &full[stage], ks * BK1, rr[0], rr[1], rr[2], rr[3]);
-        if (lane < K * p.nbw) {
-          const int j = lane / p.nbw, nb = lane - j * p.nbw;
-          tma_load_3d(slot + 16384 + lane * 8192, &tm_wx, &full[stage], nb * 64, ks * BK1, ej[j]);
-        }
+        tma_gather4(slot + lane * 512, &tm_x, &full_a[stage], ks * BK1, rr[0], rr[1], rr[2], rr[3]);
         ++issued;
-        if (++stage == kStages1) {
+        if (++stage == kStagesA) {
           stage = 0;
           phase ^= 1u;
         }
@@ -282,14 +289,46 @@ __global__ void __launch_bounds__(192, 1)
     if (!ok) {
       *abort_flag = 1;
       if (lane == 0) record_device_error(p.status, SWIMBA_ERR_TIMEOUT, 11, blockIdx.x, 0);
-      drain_ring(full, kStages1, stage, phase, issued);
+      drain_ring(full_a, kStagesA, stage, phase, issued);
+    }
+  } else if (warp == 6) {
+    // ---------------- producer of B: the tile's k W_x tables, K slice by K slice ----------------
+    int stage = 0, issued = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const TileInfo ti = p.tiles[tile];
+      const int ej[2] = {ti.e0, ti.e1};
+      for (int ks = 0; ks < ksteps; ++ks) {
+        if (!mbar_wait(&empty_w[stage], phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t* slot = ring_w + stage * kSlotW;
+        if (lane == 0) mbar_arrive_expect_tx(&full_w[stage], w_bytes);
+        __syncwarp();
+        if (lane < K * p.nbw) {
+          const int j = lane / p.nbw, nb = lane - j * p.nbw;
+          tma_load_3d(slot + lane * 8192, &tm_wx, &full_w[stage], nb * 64, ks * BK1, ej[j]);
+        }
+        ++issued;
+        if (++stage == kStagesW) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) record_device_error(p.status, SWIMBA_ERR_TIMEOUT, 14, blockIdx.x, 0);
+      drain_ring(full_w, kStagesW, stage, phase, issued);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(BM, p.W, /*b_mn_major=*/true);
-      int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      int sa = 0, sw = 0;
+      uint32_t pa = 0, pw = 0, acc_phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag)) {
@@ -298,26 +337,31 @@ __global__ void __launch_bounds__(192, 1)
         }
         tc_fence_after();
         for (int ks = 0; ks < ksteps; ++ks) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+          if (!mbar_wait(&full_a[sa], pa, abort_flag) || !mbar_wait(&full_w[sw], pw, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t base = smem_u32(ring + stage * kSlot1);
+          const uint32_t abase = smem_u32(ring_a + sa * kSlotA);
+          const uint32_t wbase = smem_u32(ring_w + sw * kSlotW);
 #pragma unroll
           for (int kk = 0; kk < BK1 / 16; ++kk) {
-            const uint64_t adesc = smem_desc(base + kk * 32, 16, 1024, kLayoutSW128);
+            const uint64_t adesc = smem_desc(abase + kk * 32, 16, 1024, kLayoutSW128);
 #pragma unroll
             for (int j = 0; j < K; ++j) {
-              const uint64_t bdesc =
-                  smem_desc(base + 16384 + j * p.nbw * 8192 + kk * 16 * 128, 8192, 1024, kLayoutSW128);
+              const uint64_t bdesc = smem_desc(wbase + j * p.nbw * 8192 + kk * 16 * 128, 8192, 1024, kLayoutSW128);
               mma_bf16(tmem + j * 256, adesc, bdesc, idesc, (ks | kk) != 0);
             }
           }
-          mma_commit(&empty[stage]);
-          if (++stage == kStages1) {
-            stage = 0;
-            phase ^= 1u;
+          mma_commit(&empty_a[sa]);
+          mma_commit(&empty_w[sw]);
+          if (++sa == kStagesA) {
+            sa = 0;
+            pa ^= 1u;
+          }
+          if (++sw == kStagesW) {
+            sw = 0;
+            pw ^= 1u;
           }
         }
         if (!ok) break;
@@ -435,7 +479,7 @@ __device__ __forceinline__ float softplus_fast(float v) {
 }
 
 template <int K>
-__global__ void __maxnreg__(168)
+__global__ void __launch_bounds__(576, 1)
     proj_stage2_kernel(const __grid_constant__ CUtensorMap tm_ap, const __grid_constant__ CUtensorMap tm_wdt,
                        const Stage2Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -463,7 +507,7 @@ __global__ void __maxnreg__(168)
     mbar_init(ap_empty, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 8);
+      mbar_init(&acc_empty[b], 16);
     }
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -604,12 +648,13 @@ __global__ void __maxnreg__(168)
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue: 8 warps, two per TMEM lane quarter ----------------
-    // Each warp drains 128 of the chunk's 256 columns for the 32 rows of its lane quarter, as two
+    // ---------------- epilogue: 16 warps, four per TMEM lane quarter ----------------
+    // Each warp drains 64 of the chunk's 256 columns for the 32 rows of its lane quarter, as two
     // 16-row halves read with the 16x256b shape: four consecutive threads hold eight consecutive
-    // columns of one row, so every warp-wide store writes whole 32-byte sectors of 8 rows.
+    // columns of one row, so every warp-wide store writes whole 32-byte sectors of 8 rows. Four
+    // warps per scheduler hide the latency of the softplus chains.
     const int q = warp & 3;
-    const int half = (warp - 2) >> 2;  // 0: chunk columns [0,128), 1: [128,256)
+    const int cq = (warp - 2) >> 2;  // chunk columns [64 cq, 64 cq + 64)
     const int t0 = lane & 3, t1 = lane >> 2;
     int cur_tile = -1, buf = 0;
     uint32_t acc_phase[2] = {0, 0};
@@ -638,17 +683,7 @@ __global__ void __maxnreg__(168)
         e[1] = ti.e1;
         cur_tile = tile;
       }
-      const int dcol = c * NC + half * 128 + 2 * t0;  // column of r[0]; r[4k] is at dcol + 8k
-      // this thread's bias values for the chunk, loaded before the accumulator wait hides them
-      float2 bias[K][16];
-#pragma unroll
-      for (int j = 0; j < K; ++j)
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int d = dcol + 8 * k;
-          bias[j][k] = d < p.D ? __ldg(reinterpret_cast<const float2*>(p.b_dt + (size_t)e[j] * p.D + d))
-                               : make_float2(0.f, 0.f);
-        }
+      const int dcol = c * NC + cq * 64 + 2 * t0;  // column of r[0]; r[4k] is at dcol + 8k
       if (!mbar_wait(&acc_full[buf], acc_phase[buf], abort_flag)) {
         *abort_flag = 1;
         if (lane == 0) record_device_error(p.status, SWIMBA_ERR_TIMEOUT, 23, blockIdx.x, (int)item);
@@ -658,34 +693,34 @@ __global__ void __maxnreg__(168)
       tc_fence_after();
 #pragma unroll
       for (int dh = 0; dh < 2; ++dh) {
+        uint32_t v[32];
+        tmem_ld_16x256b_x8_nowait(tmem + ((uint32_t)(32 * q + 16 * dh) << 16) + buf * NC + cq * 64, v);
+        tmem_wait_ld();
+        if (dh == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        }
 #pragma unroll
-        for (int kh = 0; kh < 2; ++kh) {
-          uint32_t v[32];
-          tmem_ld_16x256b_x8_nowait(tmem + ((uint32_t)(32 * q + 16 * dh) << 16) + buf * NC + half * 128 + kh * 64, v);
-          tmem_wait_ld();
-          if (dh == 1 && kh == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[buf]);
-          }
+        for (int k = 0; k < 8; ++k) {
+          const int d = dcol + 8 * k;
+          if (d < p.D) {
+            // the k experts' biases of columns d, d+1 (the 8 rows of a quad share them: L1 hits)
+            float2 bias[K];
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const int k = kh * 8 + kk;
-            const int d = dcol + 8 * k;
-            if (d < p.D) {
+            for (int j = 0; j < K; ++j) bias[j] = __ldg(reinterpret_cast<const float2*>(p.b_dt + (size_t)e[j] * p.D + d));
 #pragma unroll
-              for (int r = 0; r < 2; ++r) {
-                float2 bmix = make_float2(0.f, 0.f);
+            for (int r = 0; r < 2; ++r) {
+              float2 bmix = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int j = 0; j < K; ++j) {
-                  bmix.x = fmaf(g[dh][r][j], bias[j][k].x, bmix.x);
-                  bmix.y = fmaf(g[dh][r][j], bias[j][k].y, bmix.y);
-                }
-                if (valid[dh][r]) {
-                  const float2 o = make_float2(softplus_fast(__uint_as_float(v[4 * kk + 2 * r]) + bmix.x),
-                                               softplus_fast(__uint_as_float(v[4 * kk + 2 * r + 1]) + bmix.y));
-                  *reinterpret_cast<float2*>(p.delta + (size_t)tok[dh][r] * p.D + d) = o;
-                }
+              for (int j = 0; j < K; ++j) {
+                bmix.x = fmaf(g[dh][r][j], bias[j].x, bmix.x);
+                bmix.y = fmaf(g[dh][r][j], bias[j].y, bmix.y);
+              }
+              if (valid[dh][r]) {
+                const float2 o = make_float2(softplus_fast(__uint_as_float(v[4 * k + 2 * r]) + bmix.x),
+                                             softplus_fast(__uint_as_float(v[4 * k + 2 * r + 1]) + bmix.y));
+                *reinterpret_cast<float2*>(p.delta + (size_t)tok[dh][r] * p.D + d) = o;
               }
             }
           }
@@ -786,10 +821,10 @@ cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s) {
   const int sms = num_sms();
   Stage1Params s1{p.D, W, p.R, p.N, L.R_pad, L.K2, nbw, num_tiles, tiles, slot_tok, slot_gate, aprime,
                   p.B_mix, p.C_mix, ws};
-  const size_t smem1 = 1024 + (size_t)kStages1 * kSlot1 + 256;
+  const size_t smem1 = 1024 + (size_t)kStagesA * kSlotA + (size_t)kStagesW * kSlotW + 256;
   e = cudaFuncSetAttribute(proj_stage1_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
   if (e != cudaSuccess) return e;
-  proj_stage1_kernel<K><<<(unsigned)std::min(L.max_tiles, sms), 192, smem1, s>>>(tm_x, tm_wx, s1);
+  proj_stage1_kernel<K><<<(unsigned)std::min(L.max_tiles, sms), 224, smem1, s>>>(tm_x, tm_wx, s1);
   note_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
@@ -797,7 +832,7 @@ cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s) {
   const size_t smem2 = 1024 + (size_t)(L.K2 / 64) * kApBox + (size_t)kStages2 * kSlot2 + 256;
   e = cudaFuncSetAttribute(proj_stage2_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
   if (e != cudaSuccess) return e;
-  proj_stage2_kernel<K><<<(unsigned)sms, 320, smem2, s>>>(tm_ap, tm_wdt, s2);
+  proj_stage2_kernel<K><<<(unsigned)sms, 576, smem2, s>>>(tm_ap, tm_wdt, s2);
   note_launch();
   return cudaGetLastError();
 }

@@ -197,7 +197,13 @@ __global__ void __launch_bounds__(256, 1) route_tc_kernel(const __grid_constant_
     __syncwarp();
   } else if (warp < 4) {
     // ---------------- B slices: W_r rows split into three bf16 parts ----------------
-    const int ci = threadIdx.x - 64;  // the K index within the slice this thread converts
+    // thread (rp, eh): K rows 2rp, 2rp+1 of the slice, experts eh*E/2 .. eh*E/2 + E/2 - 1; the two
+    // rows' parts are packed as bf16x2, one 4-byte store per (expert, part)
+    const int ct = threadIdx.x - 64;
+    const int rp = ct & 31, eh = ct >> 5;
+    const int eh0 = eh * (p.E / 2);
+    const uint32_t cin = (uint32_t)(rp & 3) * 4u;
+    const uint32_t chunk = (uint32_t)(rp >> 2);
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -208,23 +214,30 @@ __global__ void __launch_bounds__(256, 1) route_tc_kernel(const __grid_constant_
           ok = false;
           break;
         }
-        const float* wr = reinterpret_cast<const float*>(wring + stage * kWSlot) + ci * p.E;
+        const float* w0 = reinterpret_cast<const float*>(wring + stage * kWSlot) + (2 * rp) * p.E + eh0;
+        const float* w1 = w0 + p.E;
         uint8_t* bt = bring + stage * kBSlot;
-        const uint32_t cin = (uint32_t)(ci & 7) * 2u;
-        const uint32_t chunk = (uint32_t)(ci >> 3);
 #pragma unroll
-        for (int e = 0; e < EP; ++e) {
-          if (e < p.E) {
-            const float w = wr[e];
-            const __nv_bfloat16 h1 = __float2bfloat16_rn(w);
-            const float r1 = w - __bfloat162float(h1);
-            const __nv_bfloat16 h2 = __float2bfloat16_rn(r1);
-            const __nv_bfloat16 h3 = __float2bfloat16_rn(r1 - __bfloat162float(h2));
-            const __nv_bfloat16 part[3] = {h1, h2, h3};
+        for (int i = 0; i < EP / 2; i += 2) {
+          if (i < p.E / 2) {
+            const float2 a = *reinterpret_cast<const float2*>(w0 + i);  // row 2rp: experts eh0+i, +1
+            const float2 b = *reinterpret_cast<const float2*>(w1 + i);  // row 2rp+1
 #pragma unroll
-            for (int q = 0; q < 3; ++q) {
-              const uint32_t n = (uint32_t)(3 * e + q);
-              *reinterpret_cast<__nv_bfloat16*>(bt + n * 128u + ((chunk ^ (n & 7u)) << 4) + cin) = part[q];
+            for (int u = 0; u < 2; ++u) {
+              const float2 w = u == 0 ? make_float2(a.x, b.x) : make_float2(a.y, b.y);  // (row 2rp, 2rp+1)
+              const __nv_bfloat162 h1 = __float22bfloat162_rn(w);
+              const float2 h1f = __bfloat1622float2(h1);
+              const float2 r1 = __fadd2_rn(w, make_float2(-h1f.x, -h1f.y));
+              const __nv_bfloat162 h2 = __float22bfloat162_rn(r1);
+              const float2 h2f = __bfloat1622float2(h2);
+              const __nv_bfloat162 h3 = __float22bfloat162_rn(__fadd2_rn(r1, make_float2(-h2f.x, -h2f.y)));
+              const __nv_bfloat162 part[3] = {h1, h2, h3};
+              const int e = eh0 + i + u;
+#pragma unroll
+              for (int q = 0; q < 3; ++q) {
+                const uint32_t n = (uint32_t)(3 * e + q);
+                *reinterpret_cast<__nv_bfloat162*>(bt + n * 128u + ((chunk ^ (n & 7u)) << 4) + cin) = part[q];
+              }
             }
           }
         }

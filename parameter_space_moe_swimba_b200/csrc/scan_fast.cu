@@ -124,6 +124,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float2 v) {
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
+// One token's scan inputs as the recurrence pass holds them (lane view: channels 2cp, 2cp+1,
+// states 8gi .. 8gi+7).
+struct TokIn {
+  int4 m;              // {e0, e1, g0, g1}
+  uint32_t ar[2][16];  // A rows of the selected experts (x log2 e), from TMEM
+  float2 dl, xv;       // Δ and x of the two channels
+  float2 bv[4], cv[4]; // B_mix, C_mix of the lane's 8 states
+  float dx[2];         // Δ x per channel
+  float2 arg[2][4];    // Σ_j (Δ g_j) A^{e_j}  [channel][state pair]
+  float2 a[2][4];      // 2^arg
+};
+
 struct FastParams {
   const int32_t* idx;
   const float* gates;
@@ -304,90 +316,88 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       const float4* bsm = reinterpret_cast<const float4*>(st + St::B);
       const float4* csm = reinterpret_cast<const float4*>(st + St::C);
       const int64_t t0 = t_begin + (int64_t)c * LC;
+      // issue token t's loads (TMEM loads are waited for by the caller)
+      auto load_tok = [&](TokIn& q, int t) {
+        q.m = meta[t];
+        tmem_ld16_nowait(tbase + (uint32_t)(q.m.x * ACOLS), q.ar[0]);
+        if (K == 2) tmem_ld16_nowait(tbase + (uint32_t)(q.m.y * ACOLS), q.ar[1]);
+        q.dl = ds2[t * (CPW / 2) + cp];
+        q.xv = __bfloat1622float2(xs2[t * (CPW / 2) + cp]);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const float4 bq = bsm[t * 4 + gi * 2 + i];
+          q.bv[2 * i] = make_float2(bq.x, bq.y);
+          q.bv[2 * i + 1] = make_float2(bq.z, bq.w);
+          if (!AGG) {
+            const float4 cq = csm[t * 4 + gi * 2 + i];
+            q.cv[2 * i] = make_float2(cq.x, cq.y);
+            q.cv[2 * i + 1] = make_float2(cq.z, cq.w);
+          }
+        }
+      };
+      // decay factors of a loaded token (independent of the state)
+      auto decay = [&](TokIn& q) {
+        q.dx[0] = q.dl.x * q.xv.x;
+        q.dx[1] = q.dl.y * q.xv.y;
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          const float dlt = ch == 0 ? q.dl.x : q.dl.y;
+          const float g0 = dlt * __int_as_float(q.m.z);
+          const float g1 = dlt * __int_as_float(q.m.w);
+#pragma unroll
+          for (int s = 0; s < NP; ++s) {
+            const float2 a0 = make_float2(__uint_as_float(q.ar[0][ch * NS + 2 * s]), __uint_as_float(q.ar[0][ch * NS + 2 * s + 1]));
+            q.arg[ch][s] = __fmul2_rn(make_float2(g0, g0), a0);
+            if (K == 2) {
+              const float2 a1 = make_float2(__uint_as_float(q.ar[1][ch * NS + 2 * s]), __uint_as_float(q.ar[1][ch * NS + 2 * s + 1]));
+              q.arg[ch][s] = __ffma2_rn(make_float2(g1, g1), a1, q.arg[ch][s]);
+            }
+            if (s >= NP - NPOLY / 2) {
+              q.a[ch][s] = exp2_poly2(q.arg[ch][s]);
+            } else {
+              q.a[ch][s] = make_float2(ex2_approx(q.arg[ch][s].x), ex2_approx(q.arg[ch][s].y));
+            }
+          }
+        }
+      };
 
       // ---- recurrence pass: the state chain only; partial readouts go to shared memory ----
-#pragma unroll 2
-      for (int t = 0; t < LC; t += 2) {
-        // loads of both tokens first: the selected experts' A rows (TMEM), Δ, x, B, C (smem)
-        int4 m[2];
-        uint32_t ar[2][2][ACOLS];  // [token][expert slot][columns]
-        float2 dl[2], xv[2];
-        float2 bv[2][NP], cv[2][NP];
+      // Software-pipelined by one token: while token t updates the state, token t+1's inputs are
+      // loaded (its A rows from TMEM, Δ, x, B, C from the ring) and its decay factors computed,
+      // so the TMEM and shared-memory latencies and the exponentials of t+1 overlap t's FMAs.
+      TokIn cur, nxt;
+      load_tok(cur, 0);
+      tmem_wait_ld();
+      decay(cur);
 #pragma unroll
-        for (int u2 = 0; u2 < 2; ++u2) {
-          m[u2] = meta[t + u2];
-          tmem_ld16_nowait(tbase + (uint32_t)(m[u2].x * ACOLS), ar[u2][0]);
-          if (K == 2) tmem_ld16_nowait(tbase + (uint32_t)(m[u2].y * ACOLS), ar[u2][1]);
-        }
+      for (int t = 0; t < LC; ++t) {
+        if (t + 1 < LC) load_tok(nxt, t + 1);
+        float yc[2];
 #pragma unroll
-        for (int u2 = 0; u2 < 2; ++u2) {
-          dl[u2] = ds2[(t + u2) * (CPW / 2) + cp];
-          xv[u2] = __bfloat1622float2(xs2[(t + u2) * (CPW / 2) + cp]);
+        for (int ch = 0; ch < 2; ++ch) {
+          const float2 dxx = make_float2(cur.dx[ch], cur.dx[ch]);
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const float4 bq = bsm[(t + u2) * 4 + gi * 2 + q];
-            bv[u2][2 * q] = make_float2(bq.x, bq.y);
-            bv[u2][2 * q + 1] = make_float2(bq.z, bq.w);
-            if (!AGG) {
-              const float4 cq = csm[(t + u2) * 4 + gi * 2 + q];
-              cv[u2][2 * q] = make_float2(cq.x, cq.y);
-              cv[u2][2 * q + 1] = make_float2(cq.z, cq.w);
+          for (int s = 0; s < NP; ++s) h[ch][s] = __ffma2_rn(cur.a[ch][s], h[ch][s], __fmul2_rn(dxx, cur.bv[s]));
+          if (AGG) {
+#pragma unroll
+            for (int s = 0; s < NP; ++s) lsum[ch][s] = __fadd2_rn(lsum[ch][s], cur.arg[ch][s]);
+          } else {
+            // two independent accumulation chains (even and odd state pairs)
+            float2 ya = __fmul2_rn(cur.cv[0], h[ch][0]);
+            float2 yb = __fmul2_rn(cur.cv[1], h[ch][1]);
+#pragma unroll
+            for (int s = 2; s < NP; s += 2) {
+              ya = __ffma2_rn(cur.cv[s], h[ch][s], ya);
+              yb = __ffma2_rn(cur.cv[s + 1], h[ch][s + 1], yb);
             }
+            yc[ch] = (ya.x + yb.x) + (ya.y + yb.y);
           }
         }
-        tmem_wait_ld();
-        // decay factors of both tokens (independent of the state)
-        float2 a[2][2][NP];  // [token][channel][state pair]
-        float2 arg[2][2][NP];
-#pragma unroll
-        for (int u2 = 0; u2 < 2; ++u2)
-#pragma unroll
-          for (int ch = 0; ch < 2; ++ch) {
-            const float dlt = ch == 0 ? dl[u2].x : dl[u2].y;
-            const float g0 = dlt * __int_as_float(m[u2].z);
-            const float g1 = dlt * __int_as_float(m[u2].w);
-#pragma unroll
-            for (int s = 0; s < NP; ++s) {
-              const float2 a0 = make_float2(__uint_as_float(ar[u2][0][ch * NS + 2 * s]), __uint_as_float(ar[u2][0][ch * NS + 2 * s + 1]));
-              arg[u2][ch][s] = __fmul2_rn(make_float2(g0, g0), a0);
-              if (K == 2) {
-                const float2 a1 =
-                    make_float2(__uint_as_float(ar[u2][1][ch * NS + 2 * s]), __uint_as_float(ar[u2][1][ch * NS + 2 * s + 1]));
-                arg[u2][ch][s] = __ffma2_rn(make_float2(g1, g1), a1, arg[u2][ch][s]);
-              }
-              if (s >= NP - NPOLY / 2) {
-                a[u2][ch][s] = exp2_poly2(arg[u2][ch][s]);
-              } else {
-                a[u2][ch][s] = make_float2(ex2_approx(arg[u2][ch][s].x), ex2_approx(arg[u2][ch][s].y));
-              }
-            }
-          }
-        // the recurrence, token t then t+1
-#pragma unroll
-        for (int u2 = 0; u2 < 2; ++u2) {
-          float yc[2];
-#pragma unroll
-          for (int ch = 0; ch < 2; ++ch) {
-            const float dx = (ch == 0 ? dl[u2].x : dl[u2].y) * (ch == 0 ? xv[u2].x : xv[u2].y);
-            const float2 dxx = make_float2(dx, dx);
-#pragma unroll
-            for (int s = 0; s < NP; ++s) h[ch][s] = __ffma2_rn(a[u2][ch][s], h[ch][s], __fmul2_rn(dxx, bv[u2][s]));
-            if (AGG) {
-#pragma unroll
-              for (int s = 0; s < NP; ++s) lsum[ch][s] = __fadd2_rn(lsum[ch][s], arg[u2][ch][s]);
-            } else {
-              // two independent accumulation chains (even and odd state pairs)
-              float2 ya = __fmul2_rn(cv[u2][0], h[ch][0]);
-              float2 yb = __fmul2_rn(cv[u2][1], h[ch][1]);
-#pragma unroll
-              for (int s = 2; s < NP; s += 2) {
-                ya = __ffma2_rn(cv[u2][s], h[ch][s], ya);
-                yb = __ffma2_rn(cv[u2][s + 1], h[ch][s + 1], yb);
-              }
-              yc[ch] = (ya.x + yb.x) + (ya.y + yb.y);
-            }
-          }
-          if (!AGG) *reinterpret_cast<float2*>(psm + ((t + u2) * 2 + gi) * kPRow + 2 * cp) = make_float2(yc[0], yc[1]);
+        if (!AGG) *reinterpret_cast<float2*>(psm + (t * 2 + gi) * kPRow + 2 * cp) = make_float2(yc[0], yc[1]);
+        if (t + 1 < LC) {
+          tmem_wait_ld();
+          decay(nxt);
+          cur = nxt;
         }
       }
 
