@@ -14,7 +14,7 @@ cudaError_t run_route(const void* x, bool io_bf16, const float* W_r, int32_t* id
                       int E, int k, cudaStream_t s);
 cudaError_t run_proj_simt(const ProjParams& p, bool io_bf16, bool w_bf16, cudaStream_t s);
 bool proj_tc_supported(const ProjParams& p, bool io_bf16, bool w_bf16);
-size_t proj_tc_workspace(int64_t T, int E, int k, int R);
+size_t proj_tc_workspace(int64_t T, int E, int k, int R, int D);
 cudaError_t run_proj_tc(const ProjParams& p, void* ws, cudaStream_t s);
 }  // namespace swimba
 
@@ -71,7 +71,7 @@ bool use_tc(const swimba_dims* d) {
 }
 
 size_t proj_workspace(const swimba_dims* d) {
-  return use_tc(d) ? proj_tc_workspace(d->batch * d->seqlen, d->n_experts, d->top_k, d->dt_rank) : kStatusBytes;
+  return use_tc(d) ? proj_tc_workspace(d->batch * d->seqlen, d->n_experts, d->top_k, d->dt_rank, d->d_inner) : kStatusBytes;
 }
 
 ScanPlan scan_plan(const swimba_dims* d) {

@@ -46,8 +46,9 @@ constexpr int kSlotA = 16384;
 constexpr int kStagesW = 3;
 constexpr int kSlotW = 49152;
 constexpr int NC = 256;        // stage-2 output columns per chunk
-constexpr int kStages2 = 3;
-constexpr int kSlot2 = 32768;  // 4 W_dt boxes of up to 64 rows x 128 B
+constexpr int kStages2 = 4;
+constexpr int kSlot2 = 16384;  // 4 W_dt boxes of up to 32 rows x 128 B
+constexpr int kBiasW = 2 * 64 * 4;  // per epilogue warp: the k experts' biases of its 64 columns
 constexpr int kApBox = BM * 128;  // one 64-column box of A' (16 KB)
 
 struct TileInfo {
@@ -55,13 +56,25 @@ struct TileInfo {
 };
 
 struct TcLayout {
-  size_t group_of, counts, cursor, offsets, num_tiles, tiles, slot_tok, slot_gate, aprime, total;
+  size_t group_of, counts, cursor, offsets, num_tiles, tiles, slot_tok, slot_gate, aprime, partial, total;
   int G, max_tiles, K2, R_pad;
+  int split, kper;  // stage-1 K split (1: none) and K slices per split
 };
+
+// Stage-1 K split for few tiles (decode steps, short prompts): each tile's K range is divided
+// among `split` CTAs so that the tiles x splits work items reach about one per SM of a B200;
+// the partial accumulators are summed by stage1_finish_kernel. 1 when the tiles alone fill it.
+inline void stage1_split(int max_tiles, int ksteps, int& split, int& kper) {
+  split = 1;
+  if (max_tiles * 2 <= 148) split = std::min(std::min(8, 148 / std::max(1, max_tiles)), ksteps);
+  split = std::max(split, 1);
+  kper = (ksteps + split - 1) / split;
+  split = (ksteps + kper - 1) / kper;  // no empty split
+}
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-TcLayout tc_layout(int64_t T, int E, int K, int R) {
+TcLayout tc_layout(int64_t T, int E, int K, int R, int D) {
   TcLayout L{};
   L.G = K == 1 ? E : E * (E - 1) / 2;
   L.max_tiles = (int)((T + BM - 1) / BM) + L.G;
@@ -76,7 +89,11 @@ TcLayout tc_layout(int64_t T, int E, int K, int R) {
   L.tiles = o; o = align_up(o + sizeof(TileInfo) * (size_t)L.max_tiles, 256);
   L.slot_tok = o; o = align_up(o + 4 * (size_t)T, 256);
   L.slot_gate = o; o = align_up(o + 4 * (size_t)T * K, 1024);
-  L.aprime = o; o += 2 * (size_t)L.max_tiles * BM * L.K2;
+  L.aprime = o; o = align_up(o + 2 * (size_t)L.max_tiles * BM * L.K2, 256);
+  stage1_split(L.max_tiles, D / BK1, L.split, L.kper);
+  const int W = R + 2 * 16;
+  L.partial = o;
+  if (L.split > 1) o += 4 * (size_t)L.split * L.max_tiles * K * W * BM;
   L.total = align_up(o, 256);
   return L;
 }
@@ -167,6 +184,8 @@ __global__ void group_scatter_kernel(const int32_t* idx, const float* gates, int
 // ---- stage 1 ---------------------------------------------------------------------------------------
 struct Stage1Params {
   int D, W, R, N, R_pad, K2, nbw;  // nbw: 64-column W_x boxes per expert
+  int split, kper;                 // K split (1: the epilogue finishes the tile) and slices per split
+  float* partial;                  // split > 1: [tile * split + s][k * W + c][128 rows] fp32
   const int* num_tiles;
   const TileInfo* tiles;
   const int* slot_tok;
@@ -265,12 +284,14 @@ __global__ void __launch_bounds__(224, 1)
     int stage = 0, issued = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+    for (int it = blockIdx.x; it < num_tiles * p.split && ok; it += gridDim.x) {
+      const int tile = it / p.split, sp = it - tile * p.split;
+      const int kb = sp * p.kper, ke = min(ksteps, kb + p.kper);
       const TileInfo ti = p.tiles[tile];
       int rr[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) rr[i] = p.slot_tok[ti.row_begin + min(4 * lane + i, ti.rows - 1)];
-      for (int ks = 0; ks < ksteps; ++ks) {
+      for (int ks = kb; ks < ke; ++ks) {
         if (!mbar_wait(&empty_a[stage], phase ^ 1u, abort_flag)) {
           ok = false;
           break;
@@ -296,10 +317,12 @@ __global__ void __launch_bounds__(224, 1)
     int stage = 0, issued = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+    for (int it = blockIdx.x; it < num_tiles * p.split && ok; it += gridDim.x) {
+      const int tile = it / p.split, sp = it - tile * p.split;
+      const int kb = sp * p.kper, ke = min(ksteps, kb + p.kper);
       const TileInfo ti = p.tiles[tile];
       const int ej[2] = {ti.e0, ti.e1};
-      for (int ks = 0; ks < ksteps; ++ks) {
+      for (int ks = kb; ks < ke; ++ks) {
         if (!mbar_wait(&empty_w[stage], phase ^ 1u, abort_flag)) {
           ok = false;
           break;
@@ -330,13 +353,15 @@ __global__ void __launch_bounds__(224, 1)
       int sa = 0, sw = 0;
       uint32_t pa = 0, pw = 0, acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int it = blockIdx.x; it < num_tiles * p.split && ok; it += gridDim.x) {
+        const int sp = it % p.split;
+        const int kb = sp * p.kper, ke = min(ksteps, kb + p.kper);
         if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        for (int ks = 0; ks < ksteps; ++ks) {
+        for (int ks = kb; ks < ke; ++ks) {
           if (!mbar_wait(&full_a[sa], pa, abort_flag) || !mbar_wait(&full_w[sw], pw, abort_flag)) {
             ok = false;
             break;
@@ -350,7 +375,7 @@ __global__ void __launch_bounds__(224, 1)
 #pragma unroll
             for (int j = 0; j < K; ++j) {
               const uint64_t bdesc = smem_desc(wbase + j * p.nbw * 8192 + kk * 16 * 128, 8192, 1024, kLayoutSW128);
-              mma_bf16(tmem + j * 256, adesc, bdesc, idesc, (ks | kk) != 0);
+              mma_bf16(tmem + j * 256, adesc, bdesc, idesc, (ks != kb || kk != 0) ? 1u : 0u);
             }
           }
           mma_commit(&empty_a[sa]);
@@ -381,7 +406,8 @@ __global__ void __launch_bounds__(224, 1)
     const int row = 32 * q + lane;
     const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    for (int it = blockIdx.x; it < num_tiles * p.split; it += gridDim.x) {
+      const int tile = it / p.split;
       const TileInfo ti = p.tiles[tile];
       if (!mbar_wait(acc_full, acc_phase, abort_flag)) {
         *abort_flag = 1;
@@ -390,6 +416,23 @@ __global__ void __launch_bounds__(224, 1)
       }
       acc_phase ^= 1u;
       tc_fence_after();
+      if (p.split > 1) {
+        // K split: this item's raw accumulators, column-major (lanes = rows write 128 bytes)
+        float* pp = p.partial + (size_t)it * K * p.W * BM + row;
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < K; ++j)
+          for (int c = 0; c < p.W; c += 16) {
+            tmem_ld16(tl + j * 256 + c, v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (c + i < p.W) pp[(size_t)(j * p.W + c + i) * BM] = v[i];
+          }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
+        continue;
+      }
       const bool valid = row < ti.rows;
       const int pos = ti.row_begin + min(row, ti.rows - 1);
       const int t = p.slot_tok[pos];
@@ -451,7 +494,7 @@ __global__ void __launch_bounds__(224, 1)
 
 // ---- stage 2 ---------------------------------------------------------------------------------------
 struct Stage2Params {
-  int D, R, R_pad, K2, RS;  // RS: W_dt rows per ring stage (min(R, 64))
+  int D, R, R_pad, K2, RS;  // RS: W_dt rows per ring stage (32, or 16 when R is not a multiple of 32)
   const int* num_tiles;
   const TileInfo* tiles;
   const int* slot_tok;
@@ -460,6 +503,73 @@ struct Stage2Params {
   float* delta;
   void* status;
 };
+
+// Finishes a K-split stage 1: sums the splits' partial accumulators (in split order, so the
+// result does not depend on scheduling) and applies the same epilogue as the unsplit kernel:
+// gated dt_low rows as bf16 hi + lo into A', B_mix and C_mix. Block (tile, group), thread = tile
+// row; groups 0 .. k R/8 - 1 are 8 dt_low columns of one expert, the last four are 8 values of
+// B_mix or C_mix. The partial buffer is column-major, so each load instruction of a warp reads
+// 128 consecutive bytes.
+template <int K>
+__global__ void __launch_bounds__(128) stage1_finish_kernel(const Stage1Params p) {
+  const int tile = blockIdx.x;
+  if (tile >= *p.num_tiles) return;
+  const int row = threadIdx.x;
+  const TileInfo ti = p.tiles[tile];
+  const int pos = ti.row_begin + min(row, ti.rows - 1);
+  float g[K];
+#pragma unroll
+  for (int j = 0; j < K; ++j) g[j] = p.slot_gate[pos * K + j];
+  const size_t item_stride = (size_t)K * p.W * BM;
+  const float* base = p.partial + (size_t)tile * p.split * item_stride + row;
+  // Σ over splits of 8 consecutive accumulator columns of expert j starting at c
+  auto sum8 = [&](int j, int c, float (&v)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    for (int sp = 0; sp < p.split; ++sp) {
+      const float* q = base + sp * item_stride + (size_t)(j * p.W + c) * BM;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] += q[(size_t)i * BM];
+    }
+  };
+  const int ng = p.R / 8;  // dt_low groups per expert
+  const int grp = blockIdx.y;
+  if (grp < K * ng) {
+    const int j = grp / ng, c = (grp - j * ng) * 8;
+    float v[8];
+    sum8(j, c, v);
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) split_bf16x2(g[j] * v[2 * i], g[j] * v[2 * i + 1], hw[i], lw[i]);
+    uint4* arow = reinterpret_cast<uint4*>(p.aprime + ((size_t)tile * BM + row) * p.K2);
+    arow[(j * p.R_pad + c) / 8] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    arow[((K + j) * p.R_pad + c) / 8] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    if (c + 8 == p.R) {  // the expert's last group also clears the padding columns
+      for (int cz = p.R; cz < p.R_pad; cz += 8) {
+        arow[(j * p.R_pad + cz) / 8] = make_uint4(0, 0, 0, 0);
+        arow[((K + j) * p.R_pad + cz) / 8] = make_uint4(0, 0, 0, 0);
+      }
+    }
+  } else {
+    const int q = grp - K * ng;      // 0, 1: B_mix n = 0..7, 8..15; 2, 3: C_mix
+    const int which = q >> 1, n0 = (q & 1) * 8;
+    float o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+      float v[8];
+      sum8(j, p.R + 16 * which + n0, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = fmaf(g[j], v[i], o[i]);
+    }
+    if (row < ti.rows) {
+      float4* dst = reinterpret_cast<float4*>((which == 0 ? p.B_mix : p.C_mix) + (size_t)p.slot_tok[pos] * 16 + n0);
+      dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+      dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+    }
+  }
+}
 
 // softplus(v) = max(v, 0) + log1p(e) with e = e^{-|v|} in (0, 1] from the ex2 instruction, and
 // log1p(e) = e q(e), q a degree-7 minimax fit of log1p(e) / e on [0, 1] (fit_log1p_poly.py beside
@@ -487,7 +597,8 @@ __global__ void __launch_bounds__(576, 1)
   const int nbox_ap = p.K2 / 64;
   uint8_t* ap = smem;                                // [K2/64][128 rows][128 B]
   uint8_t* ring = smem + nbox_ap * kApBox;           // [kStages2][kSlot2]
-  uint64_t* full = reinterpret_cast<uint64_t*>(ring + kStages2 * kSlot2);
+  uint8_t* bias_area = ring + kStages2 * kSlot2;     // [16 epilogue warps][kBiasW]
+  uint64_t* full = reinterpret_cast<uint64_t*>(bias_area + 16 * kBiasW);
   uint64_t* empty = full + kStages2;
   uint64_t* ap_full = empty + kStages2;
   uint64_t* ap_empty = ap_full + 1;
@@ -663,6 +774,20 @@ __global__ void __launch_bounds__(576, 1)
     int tok[2][2] = {{0, 0}, {0, 0}};
     float g[2][2][K];
     int e[2] = {0, 0};
+    // The k experts' biases of this warp's 64 columns go through a warp-private shared-memory
+    // buffer, one 16-byte load per lane per item, issued one item ahead.
+    float* bias_w = reinterpret_cast<float*>(bias_area + (warp - 2) * kBiasW);
+    const int bj = lane >> 4, bc4 = (lane & 15) * 4;  // lane's expert slot and first column
+    auto load_bias = [&](long long it) -> float4 {
+      const int tl = (int)(it / nchunks);
+      const int cl = (int)(it - (long long)tl * nchunks);
+      const int col = cl * NC + cq * 64 + bc4;
+      if (bj >= K || col >= p.D) return make_float4(0.f, 0.f, 0.f, 0.f);
+      const TileInfo tn = p.tiles[tl];
+      const int ee = bj == 0 ? tn.e0 : tn.e1;
+      return __ldg(reinterpret_cast<const float4*>(p.b_dt + (size_t)ee * p.D + col));
+    };
+    float4 bq_next = item_begin < item_end ? load_bias(item_begin) : make_float4(0.f, 0.f, 0.f, 0.f);
     for (long long item = item_begin; item < item_end; ++item) {
       const int tile = (int)(item / nchunks);
       const int c = (int)(item - (long long)tile * nchunks);
@@ -684,6 +809,13 @@ __global__ void __launch_bounds__(576, 1)
         cur_tile = tile;
       }
       const int dcol = c * NC + cq * 64 + 2 * t0;  // column of r[0]; r[4k] is at dcol + 8k
+      {
+        const float4 bq = bq_next;
+        if (item + 1 < item_end) bq_next = load_bias(item + 1);
+        __syncwarp();  // the previous item's reads of bias_w are done
+        if (bj < K) *reinterpret_cast<float4*>(bias_w + bj * 64 + bc4) = bq;
+        __syncwarp();
+      }
       if (!mbar_wait(&acc_full[buf], acc_phase[buf], abort_flag)) {
         *abort_flag = 1;
         if (lane == 0) record_device_error(p.status, SWIMBA_ERR_TIMEOUT, 23, blockIdx.x, (int)item);
@@ -705,10 +837,10 @@ __global__ void __launch_bounds__(576, 1)
         for (int k = 0; k < 8; ++k) {
           const int d = dcol + 8 * k;
           if (d < p.D) {
-            // the k experts' biases of columns d, d+1 (the 8 rows of a quad share them: L1 hits)
+            // the k experts' biases of columns d, d+1
             float2 bias[K];
 #pragma unroll
-            for (int j = 0; j < K; ++j) bias[j] = __ldg(reinterpret_cast<const float2*>(p.b_dt + (size_t)e[j] * p.D + d));
+            for (int j = 0; j < K; ++j) bias[j] = *reinterpret_cast<const float2*>(bias_w + j * 64 + 2 * t0 + 8 * k);
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
               float2 bmix = make_float2(0.f, 0.f);
@@ -769,7 +901,7 @@ int num_sms() {
 
 template <int K>
 cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s) {
-  const TcLayout L = tc_layout(p.T, p.E, K, p.R);
+  const TcLayout L = tc_layout(p.T, p.E, K, p.R, p.D);
   int* group_of = reinterpret_cast<int*>(ws + L.group_of);
   int* counts = reinterpret_cast<int*>(ws + L.counts);
   int* cursor = reinterpret_cast<int*>(ws + L.cursor);
@@ -810,7 +942,7 @@ cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s) {
     cuuint32_t box[2] = {64, BM};
     if (!encode(&tm_ap, aprime, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
   }
-  const int RS = p.R < 64 ? p.R : 64;
+  const int RS = p.R % 32 == 0 ? 32 : 16;
   {
     cuuint64_t dims[3] = {(cuuint64_t)p.D, (cuuint64_t)p.R, (cuuint64_t)p.E};
     cuuint64_t str[2] = {(cuuint64_t)p.D * 2, (cuuint64_t)p.R * p.D * 2};
@@ -819,17 +951,23 @@ cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s) {
   }
 
   const int sms = num_sms();
-  Stage1Params s1{p.D, W, p.R, p.N, L.R_pad, L.K2, nbw, num_tiles, tiles, slot_tok, slot_gate, aprime,
-                  p.B_mix, p.C_mix, ws};
+  Stage1Params s1{p.D,     W,       p.R,    p.N,      L.R_pad, L.K2,      nbw,       L.split,
+                  L.kper,  reinterpret_cast<float*>(ws + L.partial), num_tiles, tiles, slot_tok, slot_gate,
+                  aprime,  p.B_mix, p.C_mix, ws};
   const size_t smem1 = 1024 + (size_t)kStagesA * kSlotA + (size_t)kStagesW * kSlotW + 256;
   e = cudaFuncSetAttribute(proj_stage1_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
   if (e != cudaSuccess) return e;
-  proj_stage1_kernel<K><<<(unsigned)std::min(L.max_tiles, sms), 224, smem1, s>>>(tm_x, tm_wx, s1);
+  proj_stage1_kernel<K><<<(unsigned)std::min(L.max_tiles * L.split, sms), 224, smem1, s>>>(tm_x, tm_wx, s1);
   note_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (L.split > 1) {
+    stage1_finish_kernel<K><<<dim3((unsigned)L.max_tiles, (unsigned)(K * p.R / 8 + 4)), 128, 0, s>>>(s1);
+    note_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
 
   Stage2Params s2{p.D, p.R, L.R_pad, L.K2, RS, num_tiles, tiles, slot_tok, slot_gate, p.b_dt, p.delta, ws};
-  const size_t smem2 = 1024 + (size_t)(L.K2 / 64) * kApBox + (size_t)kStages2 * kSlot2 + 256;
+  const size_t smem2 = 1024 + (size_t)(L.K2 / 64) * kApBox + (size_t)kStages2 * kSlot2 + 16 * kBiasW + 256;
   e = cudaFuncSetAttribute(proj_stage2_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
   if (e != cudaSuccess) return e;
   proj_stage2_kernel<K><<<(unsigned)sms, 576, smem2, s>>>(tm_ap, tm_wdt, s2);
@@ -851,7 +989,7 @@ bool proj_tc_supported(const ProjParams& p, bool io_bf16, bool w_bf16) {
   return true;
 }
 
-size_t proj_tc_workspace(int64_t T, int E, int k, int R) { return tc_layout(T, E, k, R).total; }
+size_t proj_tc_workspace(int64_t T, int E, int k, int R, int D) { return tc_layout(T, E, k, R, D).total; }
 
 cudaError_t run_proj_tc(const ProjParams& p, void* ws, cudaStream_t s) {
   uint8_t* w = reinterpret_cast<uint8_t*>(ws);

@@ -154,12 +154,67 @@ __global__ void __launch_bounds__(512, 1) route_smem_kernel(RouteParams p) {
   }
 }
 
+// Few tokens (decode steps, short prompts): one CTA of 128 threads per token, so every SM works
+// even when T is a few hundred. The threads split the channels in 16-byte chunks of x, each
+// accumulates the E partial logits of its chunks (W_r rows from L2), a shuffle butterfly and a
+// shared-memory pass reduce them, and thread 0 selects and normalises the token's experts.
+template <typename IO, int EP>
+__global__ void __launch_bounds__(128) route_small_kernel(RouteParams p) {
+  constexpr int V = Vec16<IO>::n;
+  __shared__ float part[4][EP];
+  const int64_t t = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const IO* x = reinterpret_cast<const IO*>(p.x) + t * p.D;
+  float acc[EP];
+#pragma unroll
+  for (int e = 0; e < EP; ++e) acc[e] = 0.f;
+  const bool vec = (p.E & 3) == 0;  // W_r rows of 16-byte multiples: float4 loads
+  for (int c = threadIdx.x; c < p.D / V; c += 128) {
+    float xf[V];
+    Vec16<IO>::unpack(__ldg(reinterpret_cast<const uint4*>(x) + c), xf);
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      const float* w = p.W_r + (size_t)(c * V + v) * p.E;
+      if (vec) {
+#pragma unroll
+        for (int q = 0; q < EP / 4; ++q)
+          if (4 * q < p.E) {
+            const float4 w4 = __ldg(reinterpret_cast<const float4*>(w) + q);
+            acc[4 * q] = fmaf(xf[v], w4.x, acc[4 * q]);
+            acc[4 * q + 1] = fmaf(xf[v], w4.y, acc[4 * q + 1]);
+            acc[4 * q + 2] = fmaf(xf[v], w4.z, acc[4 * q + 2]);
+            acc[4 * q + 3] = fmaf(xf[v], w4.w, acc[4 * q + 3]);
+          }
+      } else {
+#pragma unroll
+        for (int e = 0; e < EP; ++e)
+          if (e < p.E) acc[e] = fmaf(xf[v], __ldg(w + e), acc[e]);
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < EP; ++e) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+    if (lane == 0) part[warp][e] = acc[e];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float l[EP];
+#pragma unroll
+    for (int e = 0; e < EP; ++e) l[e] = (part[0][e] + part[1][e]) + (part[2][e] + part[3][e]);
+    select_topk<EP>(l, p.E, p.k, p.idx + t * p.k, p.gates + t * p.k);
+  }
+}
+
 template <typename IO, int EP, int TOK>
 static cudaError_t launch_route(const RouteParams& p, cudaStream_t s) {
   constexpr int V = Vec16<IO>::n;
   const size_t smem = sizeof(float2) * (EP / 2) * (size_t)p.D;
   (void)V;
-  if (smem <= 160 * 1024) {
+  if (p.T <= kSmallT) {
+    route_small_kernel<IO, EP><<<(unsigned)p.T, 128, 0, s>>>(p);
+  } else if (smem <= 160 * 1024) {
     cudaError_t e =
         cudaFuncSetAttribute(route_smem_kernel<IO, EP, TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -188,7 +243,7 @@ static cudaError_t route_dispatch(const RouteParams& p, cudaStream_t s) {
 cudaError_t run_route(const void* x, bool io_bf16, const float* W_r, int32_t* idx, float* gates, int64_t T,
                       int D, int E, int k, cudaStream_t s) {
   RouteParams p{x, W_r, idx, gates, T, D, E, k};
-  if (route_tc_supported(io_bf16, D, E, k)) return run_route_tc(p, s);
+  if (T > kSmallT && route_tc_supported(io_bf16, D, E, k)) return run_route_tc(p, s);
   return io_bf16 ? route_dispatch<__nv_bfloat16>(p, s) : route_dispatch<float>(p, s);
 }
 

@@ -133,59 +133,76 @@ __global__ void __launch_bounds__(128) scan_fwd_kernel(ScanParams p) {
 }
 
 // Decode step: one token per sequence, state read from and written back to p.h_final (= p.h0).
-// A CTA owns 32 channels and kStepRows sequences, so its A tables are loaded once for them.
-constexpr int kStepRows = 16;
-
+// The step moves each sequence's state through HBM once (read, then written back), so the kernel
+// is built for memory parallelism: one thread per (sequence, channel, 4 states), no shared-memory
+// staging, every load of the thread issued before any arithmetic. The selected experts' A rows
+// are read straight from the A tables (a few MB, L2-resident across the grid).
 template <typename IO, int K>
 __global__ void __launch_bounds__(128) step_kernel(ScanParams p) {
-  extern __shared__ float As[];
-  const int tid = threadIdx.x;
-  const int dl = tid / kG, gi = tid % kG;
-  const int d0 = blockIdx.x * kDT;
-  const int d = d0 + dl;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // over (b, d, state group)
+  const int gi = (int)(i % kG);
+  const int64_t bd = i / kG;
+  const bool valid = bd < (int64_t)p.B * p.D;
+  const int64_t bdc = valid ? bd : 0;
+  const int d = (int)(bdc % p.D);
+  const size_t tok = (size_t)(bdc / p.D);  // seqlen == 1: token = sequence
   const int n0 = gi * kNS;
-  const bool dvalid = d < p.D;
-  const int dc = dvalid ? d : 0;
-  fill_A_table(As, p, d0);
-  __syncthreads();
-  const float dsk = p.D_skip[dc];
-  const IO* x = reinterpret_cast<const IO*>(p.x);
-  const IO* z = reinterpret_cast<const IO*>(p.z);
-  IO* out = reinterpret_cast<IO*>(p.out);
-  const int b_end = min(p.B, (int)(blockIdx.y + 1) * kStepRows);
-#pragma unroll 2
-  for (int b = blockIdx.y * kStepRows; b < b_end; ++b) {
-    const size_t tok = (size_t)b;  // seqlen == 1
-    float* hp = p.h_final + ((size_t)b * p.D + dc) * p.N + n0;
-    float h[kNS];
+  float* hp = p.h_final + (size_t)bdc * p.N + n0;
+  float h[kNS];
+  if (p.N == kNMax) {
+    const float4 h4 = *reinterpret_cast<const float4*>(hp);
+    h[0] = h4.x; h[1] = h4.y; h[2] = h4.z; h[3] = h4.w;
+  } else {
+#pragma unroll
+    for (int s = 0; s < kNS; ++s) h[s] = (n0 + s < p.N) ? hp[s] : 0.f;
+  }
+  const float dlt = __ldg(p.delta + tok * p.D + d);
+  const float xv = to_f32(reinterpret_cast<const IO*>(p.x)[tok * p.D + d]);
+  const float zv = to_f32(reinterpret_cast<const IO*>(p.z)[tok * p.D + d]);
+  float Bv[kNS], Cv[kNS];
+  load_bc(p, tok, n0, Bv, Cv);
+  // arg = Σ_j (Δ g_j log2 e) A^{e_j}[d, n]
+  float arg[kNS] = {0.f, 0.f, 0.f, 0.f};
+  const int kk = K > 0 ? K : p.k;
+#pragma unroll
+  for (int j = 0; j < (K > 0 ? K : 16); ++j) {
+    if (K == 0 && j >= kk) break;
+    const int e = min(max(__ldg(p.idx + tok * p.k + j), 0), p.E - 1);
+    const float c = dlt * __ldg(p.gates + tok * p.k + j) * kLog2e;
+    const float* ar = p.A + ((size_t)e * p.D + d) * p.N + n0;
+    float a[kNS];
     if (p.N == kNMax) {
-      const float4 h4 = *reinterpret_cast<const float4*>(hp);
-      h[0] = h4.x; h[1] = h4.y; h[2] = h4.z; h[3] = h4.w;
+      const float4 a4 = __ldg(reinterpret_cast<const float4*>(ar));
+      a[0] = a4.x; a[1] = a4.y; a[2] = a4.z; a[3] = a4.w;
     } else {
 #pragma unroll
-      for (int s = 0; s < kNS; ++s) h[s] = (n0 + s < p.N) ? hp[s] : 0.f;
+      for (int s = 0; s < kNS; ++s) a[s] = (n0 + s < p.N) ? __ldg(ar + s) : 0.f;
     }
-    const float dlt = __ldg(p.delta + tok * p.D + dc);
-    const float xv = to_f32(x[tok * p.D + dc]);
-    const float zv = to_f32(z[tok * p.D + dc]);
-    float Bv[kNS], Cv[kNS];
-    load_bc(p, tok, n0, Bv, Cv);
-    float y = token_update<K>(h, As, dl, n0, dlt, xv, Bv, Cv, p.idx + tok * p.k, p.gates + tok * p.k, p.k, p.E);
-    y += __shfl_xor_sync(0xffffffffu, y, 1);
-    y += __shfl_xor_sync(0xffffffffu, y, 2);
-    if (dvalid) {
-      if (p.N == kNMax) {
-        *reinterpret_cast<float4*>(hp) = make_float4(h[0], h[1], h[2], h[3]);
-      } else {
 #pragma unroll
-        for (int s = 0; s < kNS; ++s)
-          if (n0 + s < p.N) hp[s] = h[s];
-      }
-      if (gi == 0) {
-        y = fmaf(dsk, xv, y);
-        if (p.y_pre != nullptr) p.y_pre[tok * p.D + d] = y;
-        from_f32(out[tok * p.D + d], silu_gate(y, zv));
-      }
+    for (int s = 0; s < kNS; ++s) arg[s] = fmaf(c, a[s], arg[s]);
+  }
+  const float dx = dlt * xv;
+  float y = 0.f;
+#pragma unroll
+  for (int s = 0; s < kNS; ++s) {
+    h[s] = fmaf(ex2_approx(arg[s]), h[s], dx * Bv[s]);
+    y = fmaf(Cv[s], h[s], y);
+  }
+  // the 4 state groups of a channel are 4 consecutive lanes
+  y += __shfl_xor_sync(0xffffffffu, y, 1);
+  y += __shfl_xor_sync(0xffffffffu, y, 2);
+  if (valid) {
+    if (p.N == kNMax) {
+      *reinterpret_cast<float4*>(hp) = make_float4(h[0], h[1], h[2], h[3]);
+    } else {
+#pragma unroll
+      for (int s = 0; s < kNS; ++s)
+        if (n0 + s < p.N) hp[s] = h[s];
+    }
+    if (gi == 0) {
+      y = fmaf(p.D_skip[d], xv, y);
+      if (p.y_pre != nullptr) p.y_pre[tok * p.D + d] = y;
+      from_f32(reinterpret_cast<IO*>(p.out)[tok * p.D + d], silu_gate(y, zv));
     }
   }
 }
@@ -195,12 +212,8 @@ static cudaError_t launch_scan(const ScanParams& p, bool step, cudaStream_t s) {
   const size_t smem = sizeof(float) * (size_t)p.E * kDT * kNMax;
   const unsigned gx = (unsigned)((p.D + kDT - 1) / kDT);
   if (step) {
-    if (smem > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(step_kernel<IO, K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-    }
-    dim3 grid(gx, (unsigned)((p.B + kStepRows - 1) / kStepRows));
-    step_kernel<IO, K><<<grid, 128, smem, s>>>(p);
+    const int64_t threads = (int64_t)p.B * p.D * kG;
+    step_kernel<IO, K><<<(unsigned)((threads + 127) / 128), 128, 0, s>>>(p);
     note_launch();
   } else {
     if (smem > 48 * 1024) {

@@ -193,9 +193,13 @@ EDGE = [
     (1, 200, 320, 16, 64, 5, 1, "bf16", "bf16"),   # top-1, D = 256 + 64
     (4, 129, 256, 16, 128, 6, 2, "bf16", "bf16"),  # R = 128, many ragged tiles
     (2, 1000, 128, 16, 32, 3, 2, "bf16", "bf16"),  # several full tiles per expert pair
-    # tensor-core router shapes (bf16 x, D % 64 == 0, E % 4 == 0): E = 12, a ragged last token tile
-    (3, 71, 128, 16, 16, 12, 2, "bf16", "bf16"),
-    (1, 130, 64, 16, 16, 16, 1, "bf16", "bf16"),
+    # tensor-core router shapes (bf16 x, D % 64 == 0, E % 4 == 0, more than 2048 tokens): E = 12
+    # and E = 16, a ragged last token tile
+    (3, 700, 128, 16, 16, 12, 2, "bf16", "bf16"),
+    (1, 2100, 64, 16, 16, 16, 1, "bf16", "bf16"),
+    # the SIMT tile router for more than 2048 tokens (E % 4 != 0; fp32 x)
+    (1, 2100, 96, 16, 8, 6, 3, "bf16", "f32"),
+    (1, 2100, 40, 5, 3, 3, 3, "f32", "f32"),
 ]
 
 
@@ -222,12 +226,12 @@ def test_layer_is_deterministic(S, name):
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 def test_exact_router_ties_go_to_the_lower_index(S, io):
-    """f32: the SIMT router; bf16 (D = 128, E = 8): the tensor-core router, whose tied B columns get
-    bitwise equal partial logits."""
+    """f32, 100 tokens: the one-CTA-per-token router; bf16, 2200 tokens (D = 128, E = 8): the
+    tensor-core router, whose tied B columns get bitwise equal partial logits."""
     if io == "f32":
         cfg = LayerConfig("ties", 2, 50, 64, 16, 4, 6, 2, "f32", "f32", seed=5)
     else:
-        cfg = LayerConfig("ties", 2, 50, 128, 16, 16, 8, 2, "bf16", "bf16", seed=5)
+        cfg = LayerConfig("ties", 2, 1100, 128, 16, 16, 8, 2, "bf16", "bf16", seed=5)
     case = make_case(cfg, condition=False)
     case.w.W_r[:, 3] = case.w.W_r[:, 1]  # experts 1 and 3 always tie (same fp32 sums on both sides)
     case.w.W_r[:, 5] = case.w.W_r[:, 0]
