@@ -352,6 +352,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
               const float2 a1 = make_float2(__uint_as_float(q.ar[1][ch * NS + 2 * s]), __uint_as_float(q.ar[1][ch * NS + 2 * s + 1]));
               q.arg[ch][s] = __ffma2_rn(make_float2(g1, g1), a1, q.arg[ch][s]);
             }
+            if (AGG) lsum[ch][s] = __fadd2_rn(lsum[ch][s], q.arg[ch][s]);  // Σ_t log2 ā_t
             if (s >= NP - NPOLY / 2) {
               q.a[ch][s] = exp2_poly2(q.arg[ch][s]);
             } else {
@@ -369,8 +370,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       load_tok(cur, 0);
       tmem_wait_ld();
       decay(cur);
-#pragma unroll
-      for (int t = 0; t < LC; ++t) {
+      auto token = [&](int t) {
         if (t + 1 < LC) load_tok(nxt, t + 1);
         float yc[2];
 #pragma unroll
@@ -378,10 +378,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
           const float2 dxx = make_float2(cur.dx[ch], cur.dx[ch]);
 #pragma unroll
           for (int s = 0; s < NP; ++s) h[ch][s] = __ffma2_rn(cur.a[ch][s], h[ch][s], __fmul2_rn(dxx, cur.bv[s]));
-          if (AGG) {
-#pragma unroll
-            for (int s = 0; s < NP; ++s) lsum[ch][s] = __fadd2_rn(lsum[ch][s], cur.arg[ch][s]);
-          } else {
+          if (!AGG) {
             // two independent accumulation chains (even and odd state pairs)
             float2 ya = __fmul2_rn(cur.cv[0], h[ch][0]);
             float2 yb = __fmul2_rn(cur.cv[1], h[ch][1]);
@@ -399,7 +396,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
           decay(nxt);
           cur = nxt;
         }
-      }
+      };
+#pragma unroll
+      for (int t = 0; t < LC; ++t) token(t);
 
       // ---- readout pass: lane = (token tl, channels c0..c0+15) ----
       if (!AGG) {
