@@ -778,16 +778,22 @@ __global__ void __launch_bounds__(576, 1)
     // buffer, one 16-byte load per lane per item, issued one item ahead.
     float* bias_w = reinterpret_cast<float*>(bias_area + (warp - 2) * kBiasW);
     const int bj = lane >> 4, bc4 = (lane & 15) * 4;  // lane's expert slot and first column
-    auto load_bias = [&](long long it) -> float4 {
+    // the experts of item `it` come from `known` (the current tile's) unless it starts a new tile
+    auto load_bias = [&](long long it, int known_tile, const int (&known_e)[2]) -> float4 {
       const int tl = (int)(it / nchunks);
       const int cl = (int)(it - (long long)tl * nchunks);
       const int col = cl * NC + cq * 64 + bc4;
       if (bj >= K || col >= p.D) return make_float4(0.f, 0.f, 0.f, 0.f);
-      const TileInfo tn = p.tiles[tl];
-      const int ee = bj == 0 ? tn.e0 : tn.e1;
+      int ee;
+      if (tl == known_tile) {
+        ee = known_e[bj];
+      } else {
+        const TileInfo tn = p.tiles[tl];
+        ee = bj == 0 ? tn.e0 : tn.e1;
+      }
       return __ldg(reinterpret_cast<const float4*>(p.b_dt + (size_t)ee * p.D + col));
     };
-    float4 bq_next = item_begin < item_end ? load_bias(item_begin) : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 bq_next = item_begin < item_end ? load_bias(item_begin, -1, e) : make_float4(0.f, 0.f, 0.f, 0.f);
     for (long long item = item_begin; item < item_end; ++item) {
       const int tile = (int)(item / nchunks);
       const int c = (int)(item - (long long)tile * nchunks);
@@ -811,7 +817,7 @@ __global__ void __launch_bounds__(576, 1)
       const int dcol = c * NC + cq * 64 + 2 * t0;  // column of r[0]; r[4k] is at dcol + 8k
       {
         const float4 bq = bq_next;
-        if (item + 1 < item_end) bq_next = load_bias(item + 1);
+        if (item + 1 < item_end) bq_next = load_bias(item + 1, cur_tile, e);
         __syncwarp();  // the previous item's reads of bias_w are done
         if (bj < K) *reinterpret_cast<float4*>(bias_w + bj * 64 + bc4) = bq;
         __syncwarp();
