@@ -8,9 +8,11 @@
 //
 // Design. Tokens are bucketed by the SET of experts they selected (k <= 2: an expert, or an
 // unordered expert pair), so every 128-row tile shares its k weight tables and x is read once:
-//   bucket kernels  group id per token, histogram, offsets + tile list, scatter of token ids.
+//   bucket kernels  a stable counting sort of the tokens by group: per-block histograms, group
+//                   offsets + tile list, scatter of token ids (ascending inside every group).
 //   stage 1         per tile: acc_j = X_tile · W_x^{e_j}  (j < k; TMEM, M=128, N=R+2N, K=D).
-//                   x rows are gathered by TMA (tile::gather4, 128-byte swizzle); W_x boxes are
+//                   x rows are gathered with cp.async 16-byte copies into the 128-byte-swizzled
+//                   layout (a deep ring of its own); W_x boxes (TMA) are
 //                   MN-major 128-byte-swizzled tiles of the [E, D, R+2N] table as stored.
 //                   Epilogue: B_mix, C_mix = Σ_j g_j (B^j, C^j) -> global; the gated low-rank
 //                   rows g_j dt_low^j, split into bf16 hi + lo parts (hi = bf16(v), lo =
@@ -40,7 +42,7 @@ namespace {
 constexpr int BM = 128;        // rows (token slots) per tile
 constexpr int BK1 = 64;        // stage-1 K slice per ring stage (128 bytes of bf16 per row)
 // Stage 1 keeps two rings: the gathered x rows (A, 16 KB a slot) are the slow, latency-bound
-// loads, so their ring is deeper than the W_x ring (up to 6 boxes of 8 KB a slot, L2-resident).
+// loads, so their ring is deeper than the W_x ring (up to 6 TMA boxes of 8 KB a slot, L2-resident).
 constexpr int kStagesA = 5;
 constexpr int kSlotA = 16384;
 constexpr int kStagesW = 3;
@@ -55,9 +57,12 @@ struct TileInfo {
   int row_begin, rows, e0, e1;
 };
 
+constexpr int kBucketBlock = 256;  // tokens per counting block of the bucketing sort
+constexpr int kMaxGroups = 160;    // E <= 16: at most 120 groups for k = 2
+
 struct TcLayout {
-  size_t group_of, counts, cursor, offsets, num_tiles, tiles, slot_tok, slot_gate, aprime, partial, total;
-  int G, max_tiles, K2, R_pad;
+  size_t group_of, blockhist, blockbase, offsets, num_tiles, tiles, slot_tok, slot_gate, aprime, partial, total;
+  int G, nb, max_tiles, K2, R_pad;
   int split, kper;  // stage-1 K split (1: none) and K slices per split
 };
 
@@ -81,9 +86,10 @@ TcLayout tc_layout(int64_t T, int E, int K, int R, int D) {
   L.R_pad = (R + 63) / 64 * 64;
   L.K2 = 2 * K * L.R_pad;  // [hi_0 .. hi_{k-1} | lo_0 .. lo_{k-1}], each R_pad wide
   size_t o = kStatusBytes;
+  L.nb = (int)((T + kBucketBlock - 1) / kBucketBlock);
   L.group_of = o; o = align_up(o + 4 * (size_t)T, 256);
-  L.counts = o; o += 4 * (size_t)L.G;
-  L.cursor = o; o = align_up(o + 4 * (size_t)L.G, 256);
+  L.blockhist = o; o = align_up(o + 4 * (size_t)L.nb * L.G, 256);
+  L.blockbase = o; o = align_up(o + 4 * (size_t)L.nb * L.G, 256);
   L.offsets = o; o = align_up(o + 4 * (size_t)(L.G + 1), 256);
   L.num_tiles = o; o += 256;
   L.tiles = o; o = align_up(o + sizeof(TileInfo) * (size_t)L.max_tiles, 256);
@@ -101,35 +107,58 @@ TcLayout tc_layout(int64_t T, int E, int K, int R, int D) {
 __device__ __forceinline__ int clamp_e(int e, int E) { return min(max(e, 0), E - 1); }
 
 // ---- bucketing -----------------------------------------------------------------------------------
+// Tokens are bucketed by their expert set with a stable counting sort: inside a group, slots keep
+// ascending token order, so a tile's rows are nearby tokens (the stage-2 Δ stores of a tile stay
+// within a narrow address range) and the slot order does not depend on scheduling.
 // Group id of a sorted expert set: k = 1 -> e; k = 2 (a < b) -> a + b(b-1)/2.
-template <int K>
-__global__ void group_count_kernel(const int32_t* idx, int64_t T, int E, int* group_of, int* counts) {
-  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= T) return;
-  int g;
-  if (K == 1) {
-    g = clamp_e(idx[t], E);
-  } else {
-    const int e0 = clamp_e(idx[2 * t], E), e1 = clamp_e(idx[2 * t + 1], E);
-    const int a = min(e0, e1), b = max(e0, e1);
-    g = a + b * (b - 1) / 2;
-  }
-  group_of[t] = g;
-  atomicAdd(&counts[g], 1);
-}
 
 template <int K>
-__global__ void group_scan_kernel(const int* counts, int G, int* offsets, int* num_tiles, TileInfo* tiles) {
-  __shared__ int s_off[160];
-  __shared__ int s_tstart[160];
+__device__ __forceinline__ int group_id(const int32_t* idx, int64_t t, int E) {
+  if (K == 1) return clamp_e(idx[t], E);
+  const int e0 = clamp_e(idx[2 * t], E), e1 = clamp_e(idx[2 * t + 1], E);
+  const int a = min(e0, e1), b = max(e0, e1);
+  return a + b * (b - 1) / 2;
+}
+
+// Per block of kBucketBlock tokens: the count of every group -> blockhist[block][G].
+template <int K>
+__global__ void __launch_bounds__(kBucketBlock) group_count_kernel(const int32_t* idx, int64_t T, int E, int G,
+                                                                   int* group_of, int* blockhist) {
+  __shared__ int hist[kMaxGroups];
+  for (int g = threadIdx.x; g < G; g += blockDim.x) hist[g] = 0;
+  __syncthreads();
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t < T) {
+    const int g = group_id<K>(idx, t, E);
+    group_of[t] = g;
+    atomicAdd(&hist[g], 1);
+  }
+  __syncthreads();
+  for (int g = threadIdx.x; g < G; g += blockDim.x) blockhist[(size_t)blockIdx.x * G + g] = hist[g];
+}
+
+// One CTA: group sizes and offsets, every block's first slot per group (blockbase, in block
+// order), and the tile list (tiles of up to BM rows, never crossing a group).
+template <int K>
+__global__ void group_scan_kernel(const int* blockhist, int nb, int G, int* offsets, int* blockbase,
+                                  int* num_tiles, TileInfo* tiles) {
+  __shared__ int s_cnt[kMaxGroups];
+  __shared__ int s_off[kMaxGroups + 1];
+  __shared__ int s_tstart[kMaxGroups + 1];
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    int c = 0;
+    for (int bb = 0; bb < nb; ++bb) c += blockhist[(size_t)bb * G + g];
+    s_cnt[g] = c;
+  }
+  __syncthreads();
   if (threadIdx.x == 0) {
     int off = 0, nt = 0;
     for (int g = 0; g < G; ++g) {
       s_off[g] = off;
       s_tstart[g] = nt;
       offsets[g] = off;
-      off += counts[g];
-      nt += (counts[g] + BM - 1) / BM;
+      off += s_cnt[g];
+      nt += (s_cnt[g] + BM - 1) / BM;
     }
     s_off[G] = off;
     s_tstart[G] = nt;
@@ -137,6 +166,13 @@ __global__ void group_scan_kernel(const int* counts, int G, int* offsets, int* n
     *num_tiles = nt;
   }
   __syncthreads();
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    int base = s_off[g];
+    for (int bb = 0; bb < nb; ++bb) {
+      blockbase[(size_t)bb * G + g] = base;
+      base += blockhist[(size_t)bb * G + g];
+    }
+  }
   const int nt = s_tstart[G];
   for (int tile = threadIdx.x; tile < nt; tile += blockDim.x) {
     int lo = 0, hi = G - 1;  // last g with s_tstart[g] <= tile
@@ -148,7 +184,7 @@ __global__ void group_scan_kernel(const int* counts, int G, int* offsets, int* n
     const int i = tile - s_tstart[g];
     TileInfo ti;
     ti.row_begin = s_off[g] + i * BM;
-    ti.rows = min(BM, counts[g] - i * BM);
+    ti.rows = min(BM, s_cnt[g] - i * BM);
     if (K == 1) {
       ti.e0 = g;
       ti.e1 = g;
@@ -162,13 +198,27 @@ __global__ void group_scan_kernel(const int* counts, int G, int* offsets, int* n
   }
 }
 
+// Slot of every token: its block's first slot for its group plus its rank among the block's
+// earlier tokens of the same group (warp match + per-warp counts), i.e. a stable order.
 template <int K>
-__global__ void group_scatter_kernel(const int32_t* idx, const float* gates, int64_t T, int E, const int* group_of,
-                                     const int* offsets, int* cursor, int* slot_tok, float* slot_gate) {
+__global__ void __launch_bounds__(kBucketBlock) group_scatter_kernel(const int32_t* idx, const float* gates, int64_t T,
+                                                                     int E, int G, const int* group_of,
+                                                                     const int* blockbase, int* slot_tok,
+                                                                     float* slot_gate) {
+  __shared__ int warpcnt[kBucketBlock / 32][kMaxGroups];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < (kBucketBlock / 32) * kMaxGroups; i += blockDim.x) (&warpcnt[0][0])[i] = 0;
+  __syncthreads();
   const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= T) return;
-  const int g = group_of[t];
-  const int pos = offsets[g] + atomicAdd(&cursor[g], 1);
+  const bool valid = t < T;
+  const int g = valid ? group_of[t] : -1;
+  const unsigned same = __match_any_sync(0xffffffffu, g);
+  const int lane_rank = __popc(same & ((1u << lane) - 1u));
+  if (valid && lane_rank == 0) warpcnt[warp][g] = __popc(same);
+  __syncthreads();
+  if (!valid) return;
+  int pos = blockbase[(size_t)blockIdx.x * G + g] + lane_rank;
+  for (int w = 0; w < warp; ++w) pos += warpcnt[w][g];
   slot_tok[pos] = (int)t;
   if (K == 1) {
     slot_gate[pos] = gates[t];
@@ -185,6 +235,7 @@ __global__ void group_scatter_kernel(const int32_t* idx, const float* gates, int
 struct Stage1Params {
   int D, W, R, N, R_pad, K2, nbw;  // nbw: 64-column W_x boxes per expert
   int split, kper;                 // K split (1: the epilogue finishes the tile) and slices per split
+  const __nv_bfloat16* x;          // [T, D]
   float* partial;                  // split > 1: [tile * split + s][k * W + c][128 rows] fp32
   const int* num_tiles;
   const TileInfo* tiles;
@@ -231,8 +282,7 @@ __device__ __forceinline__ void wait_all_mma(uint64_t* done) {
 
 template <int K>
 __global__ void __launch_bounds__(224, 1)
-    proj_stage1_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wx,
-                       const Stage1Params p) {
+    proj_stage1_kernel(const __grid_constant__ CUtensorMap tm_wx, const Stage1Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring_a = smem;
@@ -247,7 +297,7 @@ __global__ void __launch_bounds__(224, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  // warp 0: x-row gathers; warp 1: MMA; warps 2-5: epilogue; warp 6: W_x boxes
+  // warp 0: x-row gathers (cp.async); warp 1: MMA; warps 2-5: epilogue; warp 6: W_x boxes (TMA)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStagesA; ++s) {
@@ -265,7 +315,6 @@ __global__ void __launch_bounds__(224, 1)
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tm_x);
     prefetch_tmap(&tm_wx);
   }
   if (warp == 1) {
@@ -281,36 +330,58 @@ __global__ void __launch_bounds__(224, 1)
 
   if (warp == 0) {
     // ---------------- producer of A: 128 gathered x rows per K slice ----------------
-    int stage = 0, issued = 0;
+    // cp.async 16-byte copies (lanes 8i..8i+7 fetch one 128-byte row slice, 4 rows per
+    // instruction) written straight into the 128-byte-swizzled layout the MMA reads. The slot is
+    // handed to the MMA LAG slots later, once this thread's copies into it have landed (wait_group)
+    // and been made visible to the tensor-core proxy (fence). Plain copies keep more rows in flight
+    // than the TMA row gathers did (stage 1: 171 -> ~115 µs on the Mamba-1.4B-like shape).
+    constexpr int LAG = 3;  // < kStagesA
+    int stage = 0, n = 0, retired = 0;
     uint32_t phase = 0;
     bool ok = true;
+    const int ch = lane & 7;
     for (int it = blockIdx.x; it < num_tiles * p.split && ok; it += gridDim.x) {
       const int tile = it / p.split, sp = it - tile * p.split;
       const int kb = sp * p.kper, ke = min(ksteps, kb + p.kper);
       const TileInfo ti = p.tiles[tile];
-      int rr[4];
+      int tokrow[32];  // token of tile row 4i + lane/8
 #pragma unroll
-      for (int i = 0; i < 4; ++i) rr[i] = p.slot_tok[ti.row_begin + min(4 * lane + i, ti.rows - 1)];
+      for (int i = 0; i < 32; ++i) tokrow[i] = p.slot_tok[ti.row_begin + min(4 * i + (lane >> 3), ti.rows - 1)];
       for (int ks = kb; ks < ke; ++ks) {
         if (!mbar_wait(&empty_a[stage], phase ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
-        uint8_t* slot = ring_a + stage * kSlotA;
-        if (lane == 0) mbar_arrive_expect_tx(&full_a[stage], (uint32_t)kSlotA);
-        __syncwarp();
-        tma_gather4(slot + lane * 512, &tm_x, &full_a[stage], ks * BK1, rr[0], rr[1], rr[2], rr[3]);
-        ++issued;
+        const uint32_t sbase = smem_u32(ring_a + stage * kSlotA);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int r = 4 * i + (lane >> 3);
+          const __nv_bfloat16* src = p.x + (size_t)tokrow[i] * p.D + ks * BK1 + ch * 8;
+          cp_async16(sbase + r * 128 + ((ch ^ (r & 7)) << 4), src);
+        }
+        cp_async_commit();
+        ++n;
+        if (n - retired > LAG) {
+          cp_async_wait<LAG>();
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full_a[retired % kStagesA]);
+          ++retired;
+        }
         if (++stage == kStagesA) {
           stage = 0;
           phase ^= 1u;
         }
       }
     }
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    __syncwarp();
+    for (; retired < n; ++retired)
+      if (lane == 0) mbar_arrive(&full_a[retired % kStagesA]);
     if (!ok) {
       *abort_flag = 1;
       if (lane == 0) record_device_error(p.status, SWIMBA_ERR_TIMEOUT, 11, blockIdx.x, 0);
-      drain_ring(full_a, kStagesA, stage, phase, issued);
     }
   } else if (warp == 6) {
     // ---------------- producer of B: the tile's k W_x tables, K slice by K slice ----------------
@@ -909,8 +980,8 @@ template <int K>
 cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s) {
   const TcLayout L = tc_layout(p.T, p.E, K, p.R, p.D);
   int* group_of = reinterpret_cast<int*>(ws + L.group_of);
-  int* counts = reinterpret_cast<int*>(ws + L.counts);
-  int* cursor = reinterpret_cast<int*>(ws + L.cursor);
+  int* blockhist = reinterpret_cast<int*>(ws + L.blockhist);
+  int* blockbase = reinterpret_cast<int*>(ws + L.blockbase);
   int* offsets = reinterpret_cast<int*>(ws + L.offsets);
   int* num_tiles = reinterpret_cast<int*>(ws + L.num_tiles);
   TileInfo* tiles = reinterpret_cast<TileInfo*>(ws + L.tiles);
@@ -918,24 +989,17 @@ cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s) {
   float* slot_gate = reinterpret_cast<float*>(ws + L.slot_gate);
   __nv_bfloat16* aprime = reinterpret_cast<__nv_bfloat16*>(ws + L.aprime);
 
-  cudaError_t e = cudaMemsetAsync(counts, 0, 8 * (size_t)L.G, s);  // counts and cursor
-  if (e != cudaSuccess) return e;
-  const unsigned tb = (unsigned)((p.T + 255) / 256);
-  group_count_kernel<K><<<tb, 256, 0, s>>>(p.idx, p.T, p.E, group_of, counts);
-  group_scan_kernel<K><<<1, 256, 0, s>>>(counts, L.G, offsets, num_tiles, tiles);
-  group_scatter_kernel<K><<<tb, 256, 0, s>>>(p.idx, p.gates, p.T, p.E, group_of, offsets, cursor, slot_tok, slot_gate);
+  cudaError_t e;
+  group_count_kernel<K><<<(unsigned)L.nb, kBucketBlock, 0, s>>>(p.idx, p.T, p.E, L.G, group_of, blockhist);
+  group_scan_kernel<K><<<1, 256, 0, s>>>(blockhist, L.nb, L.G, offsets, blockbase, num_tiles, tiles);
+  group_scatter_kernel<K><<<(unsigned)L.nb, kBucketBlock, 0, s>>>(p.idx, p.gates, p.T, p.E, L.G, group_of, blockbase,
+                                                                   slot_tok, slot_gate);
   note_launch(3);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   const int W = p.R + 2 * p.N;
   const int nbw = (W + 63) / 64;
-  CUtensorMap tm_x, tm_wx, tm_ap, tm_wdt;
-  {
-    cuuint64_t dims[2] = {(cuuint64_t)p.D, (cuuint64_t)p.T};
-    cuuint64_t str[1] = {(cuuint64_t)p.D * 2};
-    cuuint32_t box[2] = {BK1, 1};
-    if (!encode(&tm_x, p.x, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
-  }
+  CUtensorMap tm_wx, tm_ap, tm_wdt;
   {
     cuuint64_t dims[3] = {(cuuint64_t)W, (cuuint64_t)p.D, (cuuint64_t)p.E};
     cuuint64_t str[2] = {(cuuint64_t)W * 2, (cuuint64_t)W * p.D * 2};
@@ -958,12 +1022,12 @@ cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s) {
 
   const int sms = num_sms();
   Stage1Params s1{p.D,     W,       p.R,    p.N,      L.R_pad, L.K2,      nbw,       L.split,
-                  L.kper,  reinterpret_cast<float*>(ws + L.partial), num_tiles, tiles, slot_tok, slot_gate,
-                  aprime,  p.B_mix, p.C_mix, ws};
+                  L.kper,  reinterpret_cast<const __nv_bfloat16*>(p.x), reinterpret_cast<float*>(ws + L.partial),
+                  num_tiles, tiles, slot_tok, slot_gate, aprime, p.B_mix, p.C_mix, ws};
   const size_t smem1 = 1024 + (size_t)kStagesA * kSlotA + (size_t)kStagesW * kSlotW + 256;
   e = cudaFuncSetAttribute(proj_stage1_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
   if (e != cudaSuccess) return e;
-  proj_stage1_kernel<K><<<(unsigned)std::min(L.max_tiles * L.split, sms), 224, smem1, s>>>(tm_x, tm_wx, s1);
+  proj_stage1_kernel<K><<<(unsigned)std::min(L.max_tiles * L.split, sms), 224, smem1, s>>>(tm_wx, s1);
   note_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (L.split > 1) {

@@ -1,6 +1,6 @@
 // Thin wrappers over sm_100a PTX used by the tensor-core kernels: mbarriers with bounded waits,
-// TMA tile / gather4 loads, tcgen05 (TMEM alloc, MMA, commit, loads, fences) and the UMMA shared
-// memory / instruction descriptors. Field layouts follow the PTX ISA (tcgen05 "Shared memory
+// TMA tile loads and stores, cp.async copies, tcgen05 (TMEM alloc, MMA, commit, loads, fences)
+// and the UMMA shared memory / instruction descriptors. Field layouts follow the PTX ISA (tcgen05 "Shared memory
 // descriptor" and "Instruction descriptor" tables).
 #pragma once
 
@@ -72,15 +72,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
-// Four rows (r0..r3) of a 2-D tensor, columns [c0, c0 + box width), into consecutive box rows.
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int r0, int r1,
-                                            int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
-      "%5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-      : "memory");
-}
 // TMA tile store from shared memory (bulk-group completion), and the bulk-group waits.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
   asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
@@ -98,6 +89,17 @@ __device__ __forceinline__ void bulk_wait_read() {
 template <int N>
 __device__ __forceinline__ void bulk_wait() {
   asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// 16-byte asynchronous copy global -> shared (L2 only), its group commit and group wait.
+__device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// at most N committed groups of this thread may still be pending
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
