@@ -156,6 +156,15 @@ swimba_status swimba_step(const swimba_dims *dims, const void *x, const void *z,
  * (SWIMBA_OK or SWIMBA_ERR_TIMEOUT) and clears it. */
 swimba_status swimba_get_device_status(void *ws, void *stream);
 
+/* Runs the library's bounded-wait error path on the device, on purpose: one warp waits on an
+ * mbarrier that nothing completes; after `limit_ns` nanoseconds (1e3 .. 1e9) it gives up and
+ * records SWIMBA_ERR_TIMEOUT in the status block at the start of `ws`, as a stalled pipeline
+ * stage of the other kernels would, then the kernel exits normally. Lets a caller check that a
+ * stalled wait ends with a status (read it with swimba_get_device_status) rather than a hang, and
+ * that the context stays usable. ws: at least 256 bytes of device memory (the status block).
+ * The pages have no counterpart of this call; it exists to test failure reporting. */
+swimba_status swimba_check_wait_timeout(void *ws, size_t ws_bytes, uint64_t limit_ns, void *stream);
+
 /* Static description of a status code. */
 const char *swimba_status_string(swimba_status s);
 

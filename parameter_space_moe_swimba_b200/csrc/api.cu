@@ -8,6 +8,7 @@
 #include "common.cuh"
 #include "proj.cuh"
 #include "scan.cuh"
+#include "sm100.cuh"
 
 namespace swimba {
 cudaError_t run_route(const void* x, bool io_bf16, const float* W_r, int32_t* idx, float* gates, int64_t T, int D,
@@ -85,6 +86,26 @@ size_t scan_workspace(const swimba_dims* d) {
 }
 
 }  // namespace
+
+namespace swimba {
+// One warp waits on an mbarrier that nothing arrives on (its phase 0 never completes) until
+// limit_ns have passed, then records SWIMBA_ERR_TIMEOUT like the pipelines' bounded waits do.
+__global__ void wait_timeout_kernel(void* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    sm100::fence_mbar_init();
+  }
+  __syncwarp();
+  const uint64_t t0 = sm100::globaltimer_ns();
+  while (!sm100::mbar_try_wait(&bar, 0)) {
+    if (sm100::globaltimer_ns() - t0 > limit_ns) {
+      if (threadIdx.x == 0) record_device_error(status, SWIMBA_ERR_TIMEOUT, 90, 0, 0);
+      break;
+    }
+  }
+}
+}  // namespace swimba
 
 extern "C" {
 
@@ -199,6 +220,15 @@ swimba_status swimba_step(const swimba_dims* dims, const void* x, const void* z,
   if (st != SWIMBA_OK) return st;
   if (dims->seqlen != 1 || h == nullptr) return SWIMBA_ERR_INVALID_ARG;
   return scan_common(dims, x, z, delta, B_mix, C_mix, idx, gates, w, h, out, h, nullptr, true, nullptr, stream);
+}
+
+swimba_status swimba_check_wait_timeout(void* ws, size_t ws_bytes, uint64_t limit_ns, void* stream) {
+  if (ws == nullptr || ws_bytes < kStatusBytes) return SWIMBA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SWIMBA_ERR_ALIGN;
+  if (limit_ns < 1000 || limit_ns > 1000000000ull) return SWIMBA_ERR_INVALID_ARG;
+  wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(ws, limit_ns);
+  note_launch();
+  return cuda_status(cudaGetLastError());
 }
 
 swimba_status swimba_get_device_status(void* ws, void* stream) {

@@ -138,17 +138,21 @@ __global__ void __launch_bounds__(kBucketBlock) group_count_kernel(const int32_t
 }
 
 // One CTA: group sizes and offsets, every block's first slot per group (blockbase, in block
-// order), and the tile list (tiles of up to BM rows, never crossing a group).
+// order), and the tile list (tiles of up to BM rows, never crossing a group). A warp per group
+// sums and prefix-sums the group's per-block counts 32 blocks at a time.
 template <int K>
-__global__ void group_scan_kernel(const int* blockhist, int nb, int G, int* offsets, int* blockbase,
-                                  int* num_tiles, TileInfo* tiles) {
+__global__ void __launch_bounds__(256) group_scan_kernel(const int* blockhist, int nb, int G, int* offsets,
+                                                         int* blockbase, int* num_tiles, TileInfo* tiles) {
   __shared__ int s_cnt[kMaxGroups];
   __shared__ int s_off[kMaxGroups + 1];
   __shared__ int s_tstart[kMaxGroups + 1];
-  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  for (int g = warp; g < G; g += nwarps) {
     int c = 0;
-    for (int bb = 0; bb < nb; ++bb) c += blockhist[(size_t)bb * G + g];
-    s_cnt[g] = c;
+    for (int bb = lane; bb < nb; bb += 32) c += blockhist[(size_t)bb * G + g];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    if (lane == 0) s_cnt[g] = c;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -166,11 +170,19 @@ __global__ void group_scan_kernel(const int* blockhist, int nb, int G, int* offs
     *num_tiles = nt;
   }
   __syncthreads();
-  for (int g = threadIdx.x; g < G; g += blockDim.x) {
-    int base = s_off[g];
-    for (int bb = 0; bb < nb; ++bb) {
-      blockbase[(size_t)bb * G + g] = base;
-      base += blockhist[(size_t)bb * G + g];
+  for (int g = warp; g < G; g += nwarps) {
+    int carry = s_off[g];
+    for (int b0 = 0; b0 < nb; b0 += 32) {
+      const int bb = b0 + lane;
+      const int v = bb < nb ? blockhist[(size_t)bb * G + g] : 0;
+      int incl = v;  // inclusive warp scan
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      if (bb < nb) blockbase[(size_t)bb * G + g] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
     }
   }
   const int nt = s_tstart[G];

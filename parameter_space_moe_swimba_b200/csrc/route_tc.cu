@@ -6,9 +6,9 @@
 //
 // The router is a [T x D] x [D x E] product with E <= 16: almost no arithmetic per byte of x, so
 // the kernel's job is to stream x from HBM once at full bandwidth. Tiles of 128 consecutive tokens
-// x 64 channels arrive by TMA (128-byte swizzle) into a 6-stage ring; one thread issues
-// tcgen05.mma (M = 128, N = 3E rounded up to 16, K = 16) into a double-buffered TMEM accumulator,
-// so the dot products cost the SM's issue slots nothing.
+// x 64 channels arrive by TMA (128-byte swizzle) into a 4-stage ring (two CTAs per SM); one thread
+// issues tcgen05.mma (M = 128, N = 3E rounded up to 16, K = 16) into a double-buffered TMEM
+// accumulator, so the dot products cost the SM's issue slots nothing.
 //
 // W_r stays fp32-exact: every weight is split into three bf16 parts w = w1 + w2 + w3 (each part is
 // the bf16 rounding of what the previous ones leave; three 8-bit significands cover fp32's 24);
@@ -34,7 +34,7 @@ namespace {
 
 constexpr int RBM = 128;            // tokens per tile
 constexpr int RBK = 64;             // channels per K slice (128 bytes of bf16)
-constexpr int kRStages = 8;         // ring depth
+constexpr int kRStages = 4;         // ring depth (two CTAs per SM: 8 stages of x per SM)
 constexpr int kXSlot = RBM * RBK * 2;  // 16 KB
 constexpr int kBSlot = 6144;           // 48 B rows of 128 bytes (3E <= 48)
 constexpr int kWSlot = RBK * 16 * 4;   // the slice's W_r rows, fp32 [64][E <= 16]
@@ -72,7 +72,7 @@ __device__ __forceinline__ void wait_all_mma_done(uint64_t* done) {
 }
 
 template <int EP>
-__global__ void __launch_bounds__(256, 1) route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+__global__ void __launch_bounds__(256, 2) route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                                                           const RouteTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -322,7 +322,9 @@ cudaError_t launch_route_tc(const RouteParams& rp, const CUtensorMap& tm, const 
   const size_t smem = 1024 + (size_t)kRStages * (kXSlot + kBSlot + kWSlot) + 512;  // + barriers
   cudaError_t e = cudaFuncSetAttribute(route_tc_kernel<EP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  route_tc_kernel<EP><<<(unsigned)std::min(ntiles, sms), 256, smem, s>>>(tm, tw, p);
+  // two CTAs per SM: two independent tile streams per SM (and every tile in the first wave when
+  // T <= 296 x 128)
+  route_tc_kernel<EP><<<(unsigned)std::min(ntiles, 2 * sms), 256, smem, s>>>(tm, tw, p);
   note_launch();
   return cudaGetLastError();
 }

@@ -47,6 +47,7 @@ EXPORTED = [
     "swimba_scan_fwd_noalloc",
     "swimba_step",
     "swimba_get_device_status",
+    "swimba_check_wait_timeout",
     "swimba_status_string",
     "swimba_kernel_launches",
     "swimba_last_error_string",
@@ -90,6 +91,8 @@ _lib.swimba_step.argtypes = [ctypes.POINTER(swimba_dims), _P, _P, _P, _P, _P, _P
 _lib.swimba_step.restype = ctypes.c_int
 _lib.swimba_get_device_status.argtypes = [_P, _P]
 _lib.swimba_get_device_status.restype = ctypes.c_int
+_lib.swimba_check_wait_timeout.argtypes = [_P, ctypes.c_size_t, ctypes.c_uint64, _P]
+_lib.swimba_check_wait_timeout.restype = ctypes.c_int
 _lib.swimba_status_string.argtypes = [ctypes.c_int]
 _lib.swimba_status_string.restype = ctypes.c_char_p
 _lib.swimba_last_error_string.argtypes = []
@@ -176,6 +179,10 @@ def swimba_step(dims, x, z, delta, B_mix, C_mix, idx, gates, weights, h, out, st
 
 def swimba_get_device_status(ws, stream=None) -> int:
     return _lib.swimba_get_device_status(_ptr(ws), _stream(stream))
+
+
+def swimba_check_wait_timeout(ws, ws_bytes, limit_ns, stream=None) -> int:
+    return _lib.swimba_check_wait_timeout(_ptr(ws), ws_bytes, limit_ns, _stream(stream))
 
 
 # ------------------------------------------------------------------------------------------------

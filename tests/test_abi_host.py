@@ -80,3 +80,8 @@ def test_invalid_arguments_return_before_any_launch(S):
     step_dims = S.make_dims(cfg)  # seqlen 128: a decode step needs seqlen 1
     assert S.swimba_step(step_dims, fake, fake, fake, fake, fake, fake, fake, w, fake, fake, 0) == 1
     assert S.swimba_get_device_status(None, 0) == 1
+    assert S.swimba_check_wait_timeout(None, 256, 10**6, 0) == 4
+    assert S.swimba_check_wait_timeout(fake, 64, 10**6, 0) == 4
+    assert S.swimba_check_wait_timeout(fake + 8, 256, 10**6, 0) == 3
+    assert S.swimba_check_wait_timeout(fake, 256, 10, 0) == 1
+    assert S.swimba_check_wait_timeout(fake, 256, 2 * 10**9, 0) == 1
