@@ -35,8 +35,23 @@ its reason in the design notes of the repository):
   y_t = Σ_n C_mix[n] h_t[·, n] + D_skip ⊙ x_t ([MB] "SSMs" output equation with its D term);
   out_t = y_t ⊙ SiLU(z_t).
 
+The surrounding block (the steps on either side of the layer), from [MB] "Mamba" (Figura 3: a
+linear projection that makes the two branches, a convolution and SiLU on the SSM branch, the
+gated SSM, a linear output projection), [MB] "Estado interno puramente lineal" (output projection
+followed by a residual connection) and [SW] Dutch summary §2 "Architectuur Implementatie" (the
+in-projection of the base block becomes the module that makes the expert-specific parameters; the
+rest of the block is unchanged). Readings where the pages are silent:
+
+* [x_pre | z] = u · W_in with W_in [d_model, 2D]; x = SiLU(causal depthwise conv of x_pre, width W,
+  per-channel taps and bias); the Swimba layer runs on (x, z); o = out · W_out + u, W_out [D, d_model].
+* the convolution looks back W-1 tokens of the same sequence; before the first token it reads the
+  carried conv state [B, W-1, D] (zeros when absent), and the last W-1 inputs are the new state.
+* with bf16 activations, x_pre, z, x, the layer output and o are stored in bf16 (round to nearest
+  even), each once, where the block stores them.
+
 Every function below is pinned by the CPU tests (closed forms, brute force, invariants, special
-cases that reduce to a dense selective scan); none is "parity unpinned".
+cases that reduce to a dense selective scan or to a library convolution); none is "parity
+unpinned".
 """
 from __future__ import annotations
 
@@ -51,6 +66,10 @@ __all__ = [
     "selective_scan",
     "layer_forward",
     "decode_step",
+    "round_bf16",
+    "causal_conv1d",
+    "block_forward",
+    "block_decode_step",
 ]
 
 
@@ -208,3 +227,72 @@ def decode_step(h, x_t, z_t, W, k, channels=None):
     """
     r = layer_forward(x_t, z_t, W, k, h0=h, channels=channels)
     return r["out"], r["h_final"], r
+
+
+# ------------------------------------------------------------------------------------------------
+# The surrounding block
+# ------------------------------------------------------------------------------------------------
+
+def round_bf16(v):
+    """Nearest bfloat16 value (8 significant bits, ties to even) of fp64 values in bf16's normal
+    range or zero: with v = m 2^e, 0.5 <= |m| < 1, the result is rint(m 2^8) 2^(e-8)."""
+    v = np.asarray(v, dtype=np.float64)
+    m, e = np.frexp(v)
+    return np.ldexp(np.rint(m * 256.0), e - 8)
+
+
+def causal_conv1d(x_pre, w, b, state=None):
+    """Depthwise causal convolution over time, then SiLU ([MB] "Mamba", Figura 3: the convolution
+    and the nonlinearity on the SSM branch of the block).
+
+    x_pre [B, L, D]; w [D, W] taps; b [D] bias; state [B, W-1, D] = the W-1 inputs before the
+    first token, oldest first (zeros when None). With p = [state; x_pre] along time:
+        c[t, d] = b[d] + sum_{i=0}^{W-1} w[d, i] p[t + i, d]      (tap W-1 weighs the current token)
+        x[t, d] = SiLU(c[t, d]);   state_out = the last W-1 rows of p.
+    Returns (c, x, state_out).
+    """
+    x_pre = np.asarray(x_pre, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    Bsz, L, D = x_pre.shape
+    W = w.shape[1]
+    if state is None:
+        state = np.zeros((Bsz, W - 1, D))
+    p = np.concatenate([np.asarray(state, dtype=np.float64), x_pre], axis=1)
+    c = np.empty((Bsz, L, D))
+    for t in range(L):
+        acc = np.array(b, dtype=np.float64)[None, :].repeat(Bsz, axis=0)
+        for i in range(W):
+            acc = acc + w[None, :, i] * p[:, t + i, :]
+        c[:, t, :] = acc
+    return c, silu(c), p[:, L:, :].copy()
+
+
+def block_forward(u, BW, k, h0=None, conv_state=None, io="f32"):
+    """The Swimba block: in-projection, convolution + SiLU, the Swimba layer, out-projection and
+    residual (sources in the module header).
+
+    u [B, L, d_model]; BW: W_in [d_model, 2D], conv_w [D, W], conv_b [D], W_out [D, d_model] and
+    the layer's weights (W_r, W_x, W_dt, b_dt, A, D_skip); h0 [B, D, N] or None; conv_state
+    [B, W-1, D] or None; io = "bf16" rounds x_pre, z, x, the layer output and o to bf16 where the
+    block stores them. Returns a dict: x_pre, z, x, the layer's intermediates (layer), o,
+    h_final, conv_state.
+    """
+    store = round_bf16 if io == "bf16" else (lambda a: np.asarray(a, dtype=np.float64))
+    u = np.asarray(u, dtype=np.float64)
+    D = BW["conv_w"].shape[0]
+    xz = u @ np.asarray(BW["W_in"], dtype=np.float64)
+    x_pre, z = store(xz[..., :D]), store(xz[..., D:])
+    _, x, conv_out = causal_conv1d(x_pre, BW["conv_w"], BW["conv_b"], conv_state)
+    x = store(x)
+    layer = layer_forward(x, z, BW, k, h0=h0)
+    y_g = store(layer["out"])
+    o = store(y_g @ np.asarray(BW["W_out"], dtype=np.float64) + u)
+    return {"x_pre": x_pre, "z": z, "x": x, "layer": layer, "o": o, "h_final": layer["h_final"],
+            "conv_state": conv_out}
+
+
+def block_decode_step(u_t, BW, k, h, conv_state, io="f32"):
+    """One decode step of the block (L = 1) from the cached (h, conv_state). Returns
+    (o [B, 1, d_model], h_new, conv_state_new)."""
+    r = block_forward(u_t, BW, k, h0=h, conv_state=conv_state, io=io)
+    return r["o"], r["h_final"], r["conv_state"]

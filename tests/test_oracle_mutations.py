@@ -7,6 +7,7 @@ import textwrap
 import pytest
 
 from oracle import swimba_oracle as O
+import tests.test_oracle_block_pins as BP
 import tests.test_oracle_pins as P
 
 pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
@@ -29,6 +30,19 @@ PINS = [
     P.test_free_decay_of_the_initial_state,
     P.test_chunk_split_and_step_by_step_equal_prefill,
     P.test_gate_placement_out_is_y_times_silu_z,
+    lambda: BP.test_conv1d_matches_library_convolution(4),
+    BP.test_conv1d_impulse_taps_are_identity_and_shift,
+    BP.test_conv1d_zero_state_when_absent,
+    lambda: BP.test_conv1d_state_handoff_equals_whole(2),
+    BP.test_round_bf16_matches_torch,
+    BP.test_block_is_residual_when_W_out_is_zero,
+    BP.test_block_zero_gate_branch_gives_residual,
+    BP.test_block_zero_convolution_gives_residual,
+    BP.test_block_ssm_branch_takes_the_first_half_of_W_in,
+    BP.test_block_is_causal,
+    lambda: BP.test_block_split_and_decode_equal_whole(2),
+    BP.test_block_output_minus_residual_is_linear_in_W_out,
+    BP.test_block_bf16_stores_bf16_values,
 ]
 
 MUTATIONS = {
@@ -63,6 +77,23 @@ MUTATIONS = {
     "dt from the wrong columns": ("expert_projections", "v[:, :R] @ W_dt[e]", "v[:, N:N + R] @ W_dt[e]"),
     "softplus without max(v,0)": ("softplus", "np.maximum(v, 0.0) + ", ""),
     "silu as sigmoid": ("silu", "return z / (1.0 + np.exp(-z))", "return 1.0 / (1.0 + np.exp(-z))"),
+    "conv taps reversed": ("causal_conv1d", "w[None, :, i] * p[:, t + i, :]", "w[None, :, W - 1 - i] * p[:, t + i, :]"),
+    "conv state ignored": ("causal_conv1d", "if state is None:", "if True:"),
+    "conv bias dropped": ("causal_conv1d", "acc = np.array(b, dtype=np.float64)", "acc = 0.0 * np.array(b, dtype=np.float64)"),
+    "conv without SiLU": ("causal_conv1d", "return c, silu(c), p[:, L:, :].copy()", "return c, c, p[:, L:, :].copy()"),
+    "conv state from the first rows": ("causal_conv1d", "p[:, L:, :].copy()", "p[:, :W - 1, :].copy()"),
+    "conv reads one token late": ("causal_conv1d", "p[:, t + i, :]", "p[:, max(t + i - 1, 0), :]"),
+    "x and z halves swapped": (
+        "block_forward",
+        "x_pre, z = store(xz[..., :D]), store(xz[..., D:])",
+        "z, x_pre = store(xz[..., :D]), store(xz[..., D:])",
+    ),
+    "residual dropped": ("block_forward", "@ np.asarray(BW[\"W_out\"], dtype=np.float64) + u)", "@ np.asarray(BW[\"W_out\"], dtype=np.float64))"),
+    "block conv state not carried": ("block_forward", "BW[\"conv_b\"], conv_state)", "BW[\"conv_b\"], None)"),
+    "block h0 not carried": ("block_forward", "layer_forward(x, z, BW, k, h0=h0)", "layer_forward(x, z, BW, k, h0=None)"),
+    "block layer on x_pre": ("block_forward", "layer_forward(x, z, BW, k", "layer_forward(x_pre, z, BW, k"),
+    "bf16 rounding toward zero": ("round_bf16", "np.rint(m * 256.0)", "np.trunc(m * 256.0)"),
+    "bf16 rounding with 7 bits": ("round_bf16", "np.ldexp(np.rint(m * 256.0), e - 8)", "np.ldexp(np.rint(m * 128.0), e - 7)"),
 }
 
 
