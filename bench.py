@@ -465,6 +465,83 @@ def report_decode(torch, S, cfg, peaks, flush, steps):
     }
 
 
+def _device_block(torch, S, cfg, d_model, d_conv, seqlen=None):
+    bw = synth.draw_block_weights(cfg, d_model, d_conv)
+    dims = S.swimba_block_dims(S.make_dims(cfg, seqlen=seqlen), d_model, d_conv)
+    keep = {
+        "lw": S.upload_weights(bw.layer, "cuda:0"),
+        "W_in": S.to_device(bw.W_in, cfg.w_dtype, "cuda:0"),
+        "W_out": S.to_device(bw.W_out, cfg.w_dtype, "cuda:0"),
+        "conv_w": torch.from_numpy(bw.conv_w).to("cuda:0"),
+        "conv_b": torch.from_numpy(bw.conv_b).to("cuda:0"),
+    }
+    w = S.swimba_block_weights(keep["W_in"].data_ptr(), keep["conv_w"].data_ptr(), keep["conv_b"].data_ptr(),
+                               keep["W_out"].data_ptr(), keep["lw"].struct())
+    ws = torch.zeros(S.swimba_block_workspace_size(dims), dtype=torch.uint8, device="cuda:0")
+    return dims, w, ws, keep
+
+
+def report_block(torch, S, cfg, d_model, d_conv, peaks, flush, reps, warmup):
+    """The surrounding block (in-projection, causal conv + SiLU, the layer, out-projection +
+    residual) over whole sequences, and its causal convolution timed alone on the same shape."""
+    dims, w, ws, keep = _device_block(torch, S, cfg, d_model, d_conv)
+    u = S.to_device(synth.draw_block_input(cfg, d_model), cfg.io_dtype, "cuda:0")
+    out = torch.empty_like(u)
+    T, D = cfg.tokens, cfg.d_inner
+    x_pre = torch.randn(cfg.batch, cfg.seqlen, D, device="cuda:0").to(torch.bfloat16)
+    x_conv = torch.empty_like(x_pre)
+    s = torch.cuda.current_stream()
+
+    def run(ev):
+        if ev is not None:
+            ev[0].record(s)
+        S.check(S.swimba_block_fwd(dims, u, w, None, None, out, None, None, ws, ws.numel(), s), "block_fwd")
+        if ev is not None:
+            ev[1].record(s)
+        S.check(S.swimba_conv1d_fwd(dims.layer, d_conv, x_pre, keep["conv_w"], keep["conv_b"], None, x_conv, None, s),
+                "conv1d_fwd")
+        if ev is not None:
+            ev[2].record(s)
+
+    (b_ms, c_ms), _ = _median_kernel_ms(torch, run, reps, warmup, flush, 3)
+    S.check(S.swimba_get_device_status(ws, s), "device status")
+    conv_bytes = 2 * T * D * 2
+    gemm_flops = 2 * T * d_model * 2 * D + 2 * T * D * d_model
+    return {
+        "report": "block", "workload": cfg.name, "d_model": d_model, "d_conv": d_conv, "tokens": T,
+        "block_us": 1e3 * b_ms, "tokens_per_s": T / (b_ms / 1e3),
+        "projection_gemm_gflop": gemm_flops / 1e9,
+        "conv_us": 1e3 * c_ms, "conv_gbs": conv_bytes / (c_ms / 1e3) / 1e9,
+        "conv_frac_of_hbm": conv_bytes / (c_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+        "median_of": reps, "l2": "flushed (256 MB write) before every run",
+    }
+
+
+def report_block_decode(torch, S, cfg, d_model, d_conv, peaks, flush, steps):
+    """``steps`` block decode steps on one cached (h, conv state), L2 flushed before every step."""
+    dims, w, ws, keep = _device_block(torch, S, cfg, d_model, d_conv)
+    u = S.to_device(synth.draw_block_input(cfg.with_(seqlen=1), d_model), cfg.io_dtype, "cuda:0")
+    out = torch.empty_like(u)
+    h = torch.from_numpy(synth.draw_h0(cfg)).to("cuda:0")
+    cs = S.to_device(synth.draw_conv_state(cfg, d_conv), cfg.io_dtype, "cuda:0")
+    s = torch.cuda.current_stream()
+
+    def run(ev):
+        if ev is not None:
+            ev[0].record(s)
+        S.check(S.swimba_block_step(dims, u, w, h, cs, out, ws, ws.numel(), s), "block_step")
+        if ev is not None:
+            ev[1].record(s)
+
+    (b_ms,), _ = _median_kernel_ms(torch, run, steps, 3, flush, 2)
+    S.check(S.swimba_get_device_status(ws, s), "device status")
+    return {
+        "report": "block_decode", "workload": cfg.name, "d_model": d_model, "d_conv": d_conv, "steps": steps,
+        "block_us_per_step": 1e3 * b_ms, "tokens_per_s": cfg.batch / (b_ms / 1e3),
+        "l2": "flushed before every step", "inputs": "u of step 0 reused every step; both states evolve",
+    }
+
+
 def run_report(args):
     import torch
 
@@ -477,6 +554,10 @@ def run_report(args):
     for name in ["tiny_fp32", "mamba130m_like", "mamba1p4b_like", "long_seq_65536"]:
         print(json.dumps(report_workload(torch, S, CONFIGS[name], peaks, flush, reps, args.warmup)), flush=True)
     print(json.dumps(report_decode(torch, S, CONFIGS["decode_b256"], peaks, flush, 1000)), flush=True)
+    # the surrounding block at the Mamba-1.4B-like width (d_model = D / 2, 4 conv taps)
+    print(json.dumps(report_block(torch, S, CONFIGS["mamba1p4b_like"], 2048, 4, peaks, flush, reps, args.warmup)),
+          flush=True)
+    print(json.dumps(report_block_decode(torch, S, CONFIGS["decode_b256"], 2048, 4, peaks, flush, 200)), flush=True)
     # Theorem 2: the recurrence's cost does not grow with E (k = 2 fixed; E = 1 forces k = 1)
     base = CONFIGS["mamba1p4b_like"]
     for E in (1, 4, 8, 16):

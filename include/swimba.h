@@ -152,6 +152,74 @@ swimba_status swimba_step(const swimba_dims *dims, const void *x, const void *z,
                           const float *gates, const swimba_weights *w, float *h, void *out,
                           void *stream);
 
+/* ---- The surrounding block -------------------------------------------------------------------
+ * ("Mamba y las SSMs: el retorno del estado persistente", section "Mamba", Figura 3: a linear
+ * projection makes the two branches, a convolution and SiLU act on the SSM branch, the gated SSM,
+ * a linear output projection; section "Estado interno puramente lineal": output projection and
+ * residual connection. "Swimba: Switch Mamba Model Scales State Space Models", Dutch summary §2
+ * "Architectuur Implementatie": the base block's in-projection becomes the module that makes the
+ * expert-specific parameters, the rest of the block is unchanged.)
+ *
+ *   [x_pre | z] = u W_in;  x = SiLU(c),  c[t,d] = conv_b[d] + sum_{i<W} conv_w[d,i] p[t+i,d],
+ *   p = [conv_state_in ; x_pre] along time (the W-1 inputs before the first token, oldest first);
+ *   the Swimba layer on (x, z) gives out_layer = y * SiLU(z);  o = out_layer W_out + u.
+ *
+ * The in- and out-projections are plain dense GEMMs run by cuBLAS (operands in io_dtype, fp32
+ * accumulation); the first block call of a host thread on a device creates that thread's cuBLAS
+ * handle for the device (cuBLAS allocates its own state then): make it before any stream capture.
+ * With bf16 activations x_pre, z, x, the layer output and o are each rounded to bf16 once. */
+
+typedef struct {
+  swimba_dims layer; /* B, L, D, N, R, E, k and dtypes of the Swimba layer inside the block */
+  int32_t d_model;   /* width of the block's input u and output o; a multiple of 8 */
+  int32_t d_conv;    /* taps W of the causal convolution, 1 .. 8 */
+} swimba_block_dims;
+
+typedef struct {
+  const void *W_in;     /* [d_model, 2D] io_dtype: columns [0, D) make x_pre, [D, 2D) make z */
+  const float *conv_w;  /* [D, d_conv] taps; tap d_conv-1 weighs the current token */
+  const float *conv_b;  /* [D] */
+  const void *W_out;    /* [D, d_model] io_dtype */
+  swimba_weights layer; /* the layer's weights (W_r, W_x, W_dt, b_dt, A, D_skip) */
+} swimba_block_weights;
+
+/* Causal depthwise convolution + SiLU over whole sequences (the block's second step).
+ *   x_pre [B, L, D] io (in); conv_w [D, W] fp32; conv_b [D] fp32;
+ *   conv_state_in  [B, W-1, D] io, the inputs before each sequence's first token, or NULL (zeros);
+ *   x [B, L, D] io (out) = SiLU(c);
+ *   conv_state_out [B, W-1, D] io (out) = the last W-1 rows of [conv_state_in ; x_pre], or NULL.
+ *   conv_state_out must not be the same buffer as conv_state_in (W > 1). Both state pointers are
+ *   ignored when W = 1. Requirements of the layer dims apply (D % 8 == 0, 16-byte alignment). */
+swimba_status swimba_conv1d_fwd(const swimba_dims *dims, int32_t d_conv, const void *x_pre,
+                                const float *conv_w, const float *conv_b, const void *conv_state_in,
+                                void *x, void *conv_state_out, void *stream);
+
+/* One decode token per sequence (dims->seqlen must be 1): x = SiLU(conv) from conv_state
+ * [B, W-1, D] io and x_pre [B, 1, D]; conv_state is shifted by one token in place. */
+swimba_status swimba_conv1d_step(const swimba_dims *dims, int32_t d_conv, const void *x_pre,
+                                 const float *conv_w, const float *conv_b, void *conv_state,
+                                 void *x, void *stream);
+
+/* Bytes of device workspace a block call needs (0 on invalid dims). Its first 256 bytes are the
+ * status block read by swimba_get_device_status; zero the workspace once after allocating it. */
+size_t swimba_block_workspace_size(const swimba_block_dims *bd);
+
+/* The whole block over whole sequences.
+ *   u [B, L, d_model] io (in); h0 [B, D, N] fp32 or NULL (zeros); conv_state_in [B, W-1, D] io or
+ *   NULL (zeros); out [B, L, d_model] io (out; may be u itself); h_final [B, D, N] fp32 or NULL
+ *   (may alias h0); conv_state_out [B, W-1, D] io or NULL (not the same buffer as conv_state_in).
+ *   Requires io_dtype == w_dtype and d_model % 8 == 0 (else SWIMBA_ERR_UNSUPPORTED). */
+swimba_status swimba_block_fwd(const swimba_block_dims *bd, const void *u,
+                               const swimba_block_weights *w, const float *h0,
+                               const void *conv_state_in, void *out, float *h_final,
+                               void *conv_state_out, void *ws, size_t ws_bytes, void *stream);
+
+/* One decode step of the block (bd->layer.seqlen must be 1) from the cached SSM state h
+ * [B, D, N] fp32 and conv state [B, W-1, D] io, both updated in place. */
+swimba_status swimba_block_step(const swimba_block_dims *bd, const void *u,
+                                const swimba_block_weights *w, float *h, void *conv_state,
+                                void *out, void *ws, size_t ws_bytes, void *stream);
+
 /* Synchronises `stream`, returns the device status recorded in the workspace's status block
  * (SWIMBA_OK or SWIMBA_ERR_TIMEOUT) and clears it. */
 swimba_status swimba_get_device_status(void *ws, void *stream);

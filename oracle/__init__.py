@@ -1,5 +1,6 @@
 """fp64 CPU oracle of the Swimba layer -- test infrastructure, never the library's compute path."""
 from .swimba_oracle import (  # noqa: F401
+    block_branches,
     block_decode_step,
     block_forward,
     causal_conv1d,

@@ -13,7 +13,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .swimba_oracle import router_logits
+from .swimba_oracle import block_branches, router_logits
 
 
 def near_tie_mask(logits: np.ndarray, k: int, margin: float) -> np.ndarray:
@@ -49,3 +49,23 @@ def condition_router_margin(x_store, widen, W_r, k, redraw, margin=1e-3, max_att
             else:
                 raise RuntimeError(f"token ({b},{t}) stays within {margin} of a router tie")
     return redrawn
+
+
+def condition_block_router_margin(u_store, widen, BW, k, io, redraw, conv_state=None, margin=2e-3,
+                                  max_rounds=64):
+    """The same conditioning for the Swimba block, whose router sees x = SiLU(conv(u W_in)): while
+    a token (b, t) of x sits near a router tie, its block input row u[b, t] (storage form, modified
+    in place) is redrawn with ``redraw(b, t, attempt)``. A new row changes x at t .. t+W-1, so the
+    check repeats over the whole input until no near tie is left. Returns the rows redrawn."""
+    attempts = {}
+    for _ in range(max_rounds):
+        _, _, x, _ = block_branches(widen(u_store), BW, conv_state, io)
+        logits = router_logits(x, BW["W_r"])
+        ties = np.argwhere(near_tie_mask(logits, k, margin))
+        if ties.size == 0:
+            return sum(attempts.values())
+        for b, t in ties:
+            a = attempts.get((int(b), int(t)), 0)
+            u_store[b, t] = redraw(int(b), int(t), a)
+            attempts[(int(b), int(t))] = a + 1
+    raise RuntimeError(f"block input keeps a token within {margin} of a router tie")

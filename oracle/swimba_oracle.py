@@ -68,6 +68,7 @@ __all__ = [
     "decode_step",
     "round_bf16",
     "causal_conv1d",
+    "block_branches",
     "block_forward",
     "block_decode_step",
 ]
@@ -267,6 +268,21 @@ def causal_conv1d(x_pre, w, b, state=None):
     return c, silu(c), p[:, L:, :].copy()
 
 
+def _store_fn(io):
+    return round_bf16 if io == "bf16" else (lambda a: np.asarray(a, dtype=np.float64))
+
+
+def block_branches(u, BW, conv_state=None, io="f32"):
+    """The block's first two steps: the in-projection [x_pre | z] = u W_in and the convolution
+    x = SiLU(conv(x_pre)), each stored in the io dtype. Returns (x_pre, z, x, conv_state_out)."""
+    store = _store_fn(io)
+    D = BW["conv_w"].shape[0]
+    xz = np.asarray(u, dtype=np.float64) @ np.asarray(BW["W_in"], dtype=np.float64)
+    x_pre, z = store(xz[..., :D]), store(xz[..., D:])
+    _, x, conv_out = causal_conv1d(x_pre, BW["conv_w"], BW["conv_b"], conv_state)
+    return x_pre, z, store(x), conv_out
+
+
 def block_forward(u, BW, k, h0=None, conv_state=None, io="f32"):
     """The Swimba block: in-projection, convolution + SiLU, the Swimba layer, out-projection and
     residual (sources in the module header).
@@ -277,13 +293,9 @@ def block_forward(u, BW, k, h0=None, conv_state=None, io="f32"):
     block stores them. Returns a dict: x_pre, z, x, the layer's intermediates (layer), o,
     h_final, conv_state.
     """
-    store = round_bf16 if io == "bf16" else (lambda a: np.asarray(a, dtype=np.float64))
+    store = _store_fn(io)
     u = np.asarray(u, dtype=np.float64)
-    D = BW["conv_w"].shape[0]
-    xz = u @ np.asarray(BW["W_in"], dtype=np.float64)
-    x_pre, z = store(xz[..., :D]), store(xz[..., D:])
-    _, x, conv_out = causal_conv1d(x_pre, BW["conv_w"], BW["conv_b"], conv_state)
-    x = store(x)
+    x_pre, z, x, conv_out = block_branches(u, BW, conv_state, io)
     layer = layer_forward(x, z, BW, k, h0=h0)
     y_g = store(layer["out"])
     o = store(y_g @ np.asarray(BW["W_out"], dtype=np.float64) + u)

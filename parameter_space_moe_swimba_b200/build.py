@@ -17,7 +17,11 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libswimba.so")
-SOURCES = ["api.cu", "route.cu", "route_tc.cu", "proj_simt.cu", "proj_tc.cu", "scan.cu", "scan_fast.cu"]
+SOURCES = [
+    "api.cu", "route.cu", "route_tc.cu", "proj_simt.cu", "proj_tc.cu", "scan.cu", "scan_fast.cu", "conv.cu",
+    "block.cu",
+]
+LIBS = ["-lcublas"]  # the block's in- and out-projection GEMMs
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr"]
 
@@ -73,7 +77,7 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
     if failed:
         raise RuntimeError(f"nvcc failed for {failed}")
     tmp = LIB + ".tmp"
-    cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", *objs, "-o", tmp]
+    cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", *objs, *LIBS, "-o", tmp]
     if verbose:
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)

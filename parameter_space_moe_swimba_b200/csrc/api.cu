@@ -88,6 +88,11 @@ size_t scan_workspace(const swimba_dims* d) {
 }  // namespace
 
 namespace swimba {
+// Shared with block.cu (the surrounding block's entry points).
+swimba_status api_check_dims(const swimba_dims* d) { return check_dims(d); }
+swimba_status api_cuda_status(cudaError_t e) { return cuda_status(e); }
+void api_set_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+
 // One warp waits on an mbarrier that nothing arrives on (its phase 0 never completes) until
 // limit_ns have passed, then records SWIMBA_ERR_TIMEOUT like the pipelines' bounded waits do.
 __global__ void wait_timeout_kernel(void* status, uint64_t limit_ns) {

@@ -51,6 +51,11 @@ EXPORTED = [
     "swimba_status_string",
     "swimba_kernel_launches",
     "swimba_last_error_string",
+    "swimba_conv1d_fwd",
+    "swimba_conv1d_step",
+    "swimba_block_workspace_size",
+    "swimba_block_fwd",
+    "swimba_block_step",
 ]
 
 
@@ -70,6 +75,14 @@ class swimba_dims(ctypes.Structure):
 
 class swimba_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("W_r", "W_x", "W_dt", "b_dt", "A", "D_skip")]
+
+
+class swimba_block_dims(ctypes.Structure):
+    _fields_ = [("layer", swimba_dims), ("d_model", ctypes.c_int32), ("d_conv", ctypes.c_int32)]
+
+
+class swimba_block_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("W_in", "conv_w", "conv_b", "W_out")] + [("layer", swimba_weights)]
 
 
 _P = ctypes.c_void_p
@@ -99,6 +112,18 @@ _lib.swimba_last_error_string.argtypes = []
 _lib.swimba_last_error_string.restype = ctypes.c_char_p
 _lib.swimba_kernel_launches.argtypes = []
 _lib.swimba_kernel_launches.restype = ctypes.c_uint64
+_lib.swimba_conv1d_fwd.argtypes = [ctypes.POINTER(swimba_dims), ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P]
+_lib.swimba_conv1d_fwd.restype = ctypes.c_int
+_lib.swimba_conv1d_step.argtypes = [ctypes.POINTER(swimba_dims), ctypes.c_int32, _P, _P, _P, _P, _P, _P]
+_lib.swimba_conv1d_step.restype = ctypes.c_int
+_lib.swimba_block_workspace_size.argtypes = [ctypes.POINTER(swimba_block_dims)]
+_lib.swimba_block_workspace_size.restype = ctypes.c_size_t
+_lib.swimba_block_fwd.argtypes = [ctypes.POINTER(swimba_block_dims), _P, ctypes.POINTER(swimba_block_weights), _P, _P,
+                                  _P, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.swimba_block_fwd.restype = ctypes.c_int
+_lib.swimba_block_step.argtypes = [ctypes.POINTER(swimba_block_dims), _P, ctypes.POINTER(swimba_block_weights), _P,
+                                   _P, _P, _P, ctypes.c_size_t, _P]
+_lib.swimba_block_step.restype = ctypes.c_int
 
 
 class SwimbaError(RuntimeError):
@@ -183,6 +208,32 @@ def swimba_get_device_status(ws, stream=None) -> int:
 
 def swimba_check_wait_timeout(ws, ws_bytes, limit_ns, stream=None) -> int:
     return _lib.swimba_check_wait_timeout(_ptr(ws), ws_bytes, limit_ns, _stream(stream))
+
+
+def swimba_conv1d_fwd(dims, d_conv, x_pre, conv_w, conv_b, conv_state_in, x, conv_state_out, stream=None) -> int:
+    return _lib.swimba_conv1d_fwd(ctypes.byref(dims), int(d_conv), _ptr(x_pre), _ptr(conv_w), _ptr(conv_b),
+                                  _ptr(conv_state_in), _ptr(x), _ptr(conv_state_out), _stream(stream))
+
+
+def swimba_conv1d_step(dims, d_conv, x_pre, conv_w, conv_b, conv_state, x, stream=None) -> int:
+    return _lib.swimba_conv1d_step(ctypes.byref(dims), int(d_conv), _ptr(x_pre), _ptr(conv_w), _ptr(conv_b),
+                                   _ptr(conv_state), _ptr(x), _stream(stream))
+
+
+def swimba_block_workspace_size(bdims: swimba_block_dims) -> int:
+    return int(_lib.swimba_block_workspace_size(ctypes.byref(bdims)))
+
+
+def swimba_block_fwd(bdims, u, bweights, h0, conv_state_in, out, h_final, conv_state_out, ws, ws_bytes,
+                     stream=None) -> int:
+    return _lib.swimba_block_fwd(ctypes.byref(bdims), _ptr(u), ctypes.byref(bweights), _ptr(h0), _ptr(conv_state_in),
+                                 _ptr(out), _ptr(h_final), _ptr(conv_state_out), _ptr(ws), int(ws_bytes),
+                                 _stream(stream))
+
+
+def swimba_block_step(bdims, u, bweights, h, conv_state, out, ws, ws_bytes, stream=None) -> int:
+    return _lib.swimba_block_step(ctypes.byref(bdims), _ptr(u), ctypes.byref(bweights), _ptr(h), _ptr(conv_state),
+                                  _ptr(out), _ptr(ws), int(ws_bytes), _stream(stream))
 
 
 # ------------------------------------------------------------------------------------------------

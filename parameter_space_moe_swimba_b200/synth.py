@@ -15,6 +15,10 @@ Initialisation recipe (shared by every workload):
   -logU(0.5, 32) per (e, d, n) ("random").
 * D_skip [D] ~ N(0, 1), fp32.
 * Cached decode state h0 [B, D, N] ~ N(0, 0.1) (variance 0.1), fp32.
+* The surrounding block: u [B, L, d_model] ~ N(0, 1) in the io dtype; W_in [d_model, 2D] ~
+  N(0, 1/d_model) and W_out [D, d_model] ~ N(0, 1/D) in the weight dtype; conv taps [D, W] and
+  conv bias [D] ~ U(-1/sqrt(W), 1/sqrt(W)), fp32; a carried conv state [B, W-1, D] ~ N(0, 1) in
+  the io dtype.
 
 N(m, s2) names the variance. bf16 values are rounded to nearest-even directly from the fp64 draw.
 
@@ -35,6 +39,10 @@ STREAM_ACTIVATIONS = 1
 STREAM_REDRAW = 2
 STREAM_STEP = 3
 STREAM_H0 = 4
+STREAM_BLOCK_WEIGHTS = 5
+STREAM_BLOCK_INPUT = 6
+STREAM_CONV_STATE = 7
+STREAM_BLOCK_REDRAW = 8
 
 _BF16_MIN_NORMAL = 2.0 ** -126
 _BF16_MAX = float.fromhex("0x1.fep127")
@@ -170,3 +178,54 @@ def redraw_x_row(cfg: LayerConfig, b: int, t: int, attempt: int, step: int = -1)
     """
     g = rng(cfg.seed, STREAM_REDRAW, step + 1, b, t, attempt)
     return round_to(g.standard_normal(cfg.d_inner), cfg.io_dtype)
+
+
+# --------------------------------------------------------------------------------------------
+# The surrounding block
+# --------------------------------------------------------------------------------------------
+
+@dataclass
+class BlockWeights:
+    W_in: np.ndarray  # [d_model, 2D] stored w_dtype
+    conv_w: np.ndarray  # [D, W] float32
+    conv_b: np.ndarray  # [D] float32
+    W_out: np.ndarray  # [D, d_model] stored w_dtype
+    layer: LayerWeights
+
+
+def draw_block_weights(cfg: LayerConfig, d_model: int, d_conv: int, a_mode: str = "structured") -> BlockWeights:
+    D = cfg.d_inner
+    g = rng(cfg.seed, STREAM_BLOCK_WEIGHTS, d_model, d_conv)
+    W_in = g.standard_normal((d_model, 2 * D)) * np.sqrt(1.0 / d_model)
+    bound = 1.0 / np.sqrt(d_conv)
+    conv_w = g.uniform(-bound, bound, size=(D, d_conv))
+    conv_b = g.uniform(-bound, bound, size=D)
+    W_out = g.standard_normal((D, d_model)) * np.sqrt(1.0 / D)
+    return BlockWeights(
+        W_in=round_to(W_in, cfg.w_dtype),
+        conv_w=conv_w.astype(np.float32),
+        conv_b=conv_b.astype(np.float32),
+        W_out=round_to(W_out, cfg.w_dtype),
+        layer=draw_weights(cfg, a_mode=a_mode),
+    )
+
+
+def draw_block_input(cfg: LayerConfig, d_model: int, batch_rows=None) -> np.ndarray:
+    """u [B, L, d_model] in storage form; batch row b from stream (seed, 6, b)."""
+    rows = range(cfg.batch) if batch_rows is None else batch_rows
+    u = np.empty((len(rows), cfg.seqlen, d_model), dtype=np.uint16 if cfg.io_dtype == "bf16" else np.float32)
+    for i, b in enumerate(rows):
+        u[i] = round_to(rng(cfg.seed, STREAM_BLOCK_INPUT, b).standard_normal((cfg.seqlen, d_model)), cfg.io_dtype)
+    return u
+
+
+def draw_conv_state(cfg: LayerConfig, d_conv: int) -> np.ndarray:
+    """A carried conv state [B, W-1, D] ~ N(0, 1) in storage form."""
+    g = rng(cfg.seed, STREAM_CONV_STATE, d_conv)
+    return round_to(g.standard_normal((cfg.batch, d_conv - 1, cfg.d_inner)), cfg.io_dtype)
+
+
+def redraw_u_row(cfg: LayerConfig, d_model: int, b: int, t: int, attempt: int) -> np.ndarray:
+    """A fresh block input row [d_model] for token (b, t), from stream (seed, 8, b, t, attempt)."""
+    g = rng(cfg.seed, STREAM_BLOCK_REDRAW, b, t, attempt)
+    return round_to(g.standard_normal(d_model), cfg.io_dtype)

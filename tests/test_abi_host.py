@@ -85,3 +85,46 @@ def test_invalid_arguments_return_before_any_launch(S):
     assert S.swimba_check_wait_timeout(fake + 8, 256, 10**6, 0) == 3
     assert S.swimba_check_wait_timeout(fake, 256, 10, 0) == 1
     assert S.swimba_check_wait_timeout(fake, 256, 2 * 10**9, 0) == 1
+
+
+def test_block_and_conv_arguments_are_checked_before_any_launch(S):
+    from parameter_space_moe_swimba_b200.configs import CONFIGS
+
+    cfg = CONFIGS["mamba1p4b_like"]
+    dims = S.make_dims(cfg)
+    fake = 1 << 40  # never dereferenced
+    bd = S.swimba_block_dims(dims, 2048, 4)
+    n = S.swimba_block_workspace_size(bd)
+    # layer workspace + x_pre, z, x, layer out (bf16) + idx, gates + delta + B_mix, C_mix
+    T, D = cfg.tokens, cfg.d_inner
+    assert n >= S.swimba_workspace_size(dims, 4) + 4 * T * D * 2 + 2 * T * 2 * 4 + T * D * 4 + 2 * T * 16 * 4
+    for bad in (S.swimba_block_dims(dims, 2047, 4), S.swimba_block_dims(dims, 2048, 9),
+                S.swimba_block_dims(dims, 2048, 0), S.swimba_block_dims(dims, 0, 4)):
+        assert S.swimba_block_workspace_size(bad) == 0
+    mixed = S.make_dims(cfg)
+    mixed.io_dtype = 0  # the GEMMs take one operand type
+    assert S.swimba_block_workspace_size(S.swimba_block_dims(mixed, 2048, 4)) == 0
+    lw = S.swimba_weights(fake, fake, fake, fake, fake, fake)
+    w = S.swimba_block_weights(fake, fake, fake, fake, lw)
+    assert S.swimba_block_fwd(bd, fake, w, None, None, fake, None, None, fake, n - 256, 0) == 4
+    assert S.swimba_block_fwd(bd, fake, w, None, None, fake, None, None, None, n, 0) == 4
+    assert S.swimba_block_fwd(bd, None, w, None, None, fake, None, None, fake, n, 0) == 1
+    assert S.swimba_block_fwd(bd, fake + 2, w, None, None, fake, None, None, fake, n, 0) == 3
+    assert S.swimba_block_fwd(S.swimba_block_dims(dims, 2048, 9), fake, w, None, None, fake, None, None, fake, n,
+                              0) == 2
+    nw = S.swimba_block_weights(fake, None, fake, fake, lw)
+    assert S.swimba_block_fwd(bd, fake, nw, None, None, fake, None, None, fake, n, 0) == 1
+    assert S.swimba_block_step(bd, fake, w, fake, fake, fake, fake, n, 0) == 1  # seqlen != 1
+    sd = S.swimba_block_dims(S.make_dims(cfg, seqlen=1), 2048, 4)
+    assert S.swimba_block_step(sd, fake, w, None, fake, fake, fake, n, 0) == 1  # no state
+    assert S.swimba_block_step(sd, fake, w, fake, None, fake, fake, n, 0) == 1  # no conv state
+    # the convolution alone
+    assert S.swimba_conv1d_fwd(dims, 9, fake, fake, fake, None, fake, None, 0) == 2
+    assert S.swimba_conv1d_fwd(dims, 4, None, fake, fake, None, fake, None, 0) == 1
+    assert S.swimba_conv1d_fwd(dims, 4, fake, fake, fake, fake, fake, fake, 0) == 1  # state in == out
+    assert S.swimba_conv1d_fwd(dims, 4, fake + 4, fake, fake, None, fake, None, 0) == 3
+    assert S.swimba_conv1d_fwd(dims, 4, fake, fake, fake, fake + 8, fake, None, 0) == 3
+    assert S.swimba_conv1d_step(dims, 4, fake, fake, fake, fake, fake, 0) == 1  # seqlen != 1
+    step = S.make_dims(cfg, seqlen=1)
+    assert S.swimba_conv1d_step(step, 4, fake, fake, fake, None, fake, 0) == 1
+    assert S.swimba_conv1d_step(step, 4, fake, fake, fake, fake + 2, fake, 0) == 3

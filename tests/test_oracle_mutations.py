@@ -84,12 +84,12 @@ MUTATIONS = {
     "conv state from the first rows": ("causal_conv1d", "p[:, L:, :].copy()", "p[:, :W - 1, :].copy()"),
     "conv reads one token late": ("causal_conv1d", "p[:, t + i, :]", "p[:, max(t + i - 1, 0), :]"),
     "x and z halves swapped": (
-        "block_forward",
+        "block_branches",
         "x_pre, z = store(xz[..., :D]), store(xz[..., D:])",
         "z, x_pre = store(xz[..., :D]), store(xz[..., D:])",
     ),
     "residual dropped": ("block_forward", "@ np.asarray(BW[\"W_out\"], dtype=np.float64) + u)", "@ np.asarray(BW[\"W_out\"], dtype=np.float64))"),
-    "block conv state not carried": ("block_forward", "BW[\"conv_b\"], conv_state)", "BW[\"conv_b\"], None)"),
+    "block conv state not carried": ("block_branches", "BW[\"conv_b\"], conv_state)", "BW[\"conv_b\"], None)"),
     "block h0 not carried": ("block_forward", "layer_forward(x, z, BW, k, h0=h0)", "layer_forward(x, z, BW, k, h0=None)"),
     "block layer on x_pre": ("block_forward", "layer_forward(x, z, BW, k", "layer_forward(x_pre, z, BW, k"),
     "bf16 rounding toward zero": ("round_bf16", "np.rint(m * 256.0)", "np.trunc(m * 256.0)"),
