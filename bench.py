@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--report", action="store_true",
                     help="per-workload table (one JSON line each): every workload, decode steps, E sweep")
+    ap.add_argument("--report-block", action="store_true",
+                    help="only the surrounding block's report lines (with --batch: the prefill line at that batch)")
     return ap.parse_args()
 
 
@@ -542,6 +544,23 @@ def report_block_decode(torch, S, cfg, d_model, d_conv, peaks, flush, steps):
     }
 
 
+def run_report_block(args):
+    import torch
+
+    from parameter_space_moe_swimba_b200 import swimba as S
+
+    torch.cuda.set_device(0)
+    peaks = load_peaks()
+    flush = L2Flush(torch, "cuda:0")
+    cfg = CONFIGS["mamba1p4b_like"]
+    if args.batch:
+        cfg = cfg.with_(batch=args.batch)
+    print(json.dumps(report_block(torch, S, cfg, 2048, 4, peaks, flush, 20, args.warmup)), flush=True)
+    if not args.batch:
+        print(json.dumps(report_block_decode(torch, S, CONFIGS["decode_b256"], 2048, 4, peaks, flush, 200)), flush=True)
+    return 0
+
+
 def run_report(args):
     import torch
 
@@ -575,6 +594,8 @@ def main():
     args = parse()
     if args.report:
         return run_report(args)
+    if args.report_block:
+        return run_report_block(args)
     cfg = CONFIGS[args.workload]
     if args.batch > 0:
         cfg = cfg.with_(batch=args.batch)
