@@ -243,6 +243,110 @@ __global__ void __launch_bounds__(kBucketBlock) group_scatter_kernel(const int32
   }
 }
 
+// The three bucketing kernels above in one CTA, for few tokens (decode steps, short prompts), where
+// their work is a few microseconds of launch and latency each. Same result: group sizes and offsets,
+// the tile list, and the stable slot order (tokens ascending inside every group), taken over
+// chunks of kSmallBucketThreads tokens in order, each chunk ranked with warp matches and per-warp
+// counts and placed after the slots of the earlier chunks.
+constexpr int kSmallBucketThreads = 1024;
+constexpr int kSmallBucketT = 4096;  // tokens up to which the one-CTA kernel is used
+
+template <int K>
+__global__ void __launch_bounds__(kSmallBucketThreads) group_bucket_small_kernel(const int32_t* idx, const float* gates,
+                                                                                 int T, int E, int G, int* offsets,
+                                                                                 int* num_tiles, TileInfo* tiles,
+                                                                                 int* slot_tok, float* slot_gate) {
+  constexpr int kChunks = kSmallBucketT / kSmallBucketThreads;
+  constexpr int kWarps = kSmallBucketThreads / 32;
+  __shared__ int s_cnt[kMaxGroups];
+  __shared__ int s_off[kMaxGroups + 1];
+  __shared__ int s_tstart[kMaxGroups + 1];
+  __shared__ int s_run[kMaxGroups];
+  __shared__ int warpcnt[kWarps][kMaxGroups];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int g = tid; g < G; g += kSmallBucketThreads) s_cnt[g] = 0;
+  __syncthreads();
+  int gs[kChunks];
+#pragma unroll
+  for (int c = 0; c < kChunks; ++c) {
+    const int t = c * kSmallBucketThreads + tid;
+    gs[c] = t < T ? group_id<K>(idx, t, E) : -1;
+    if (gs[c] >= 0) atomicAdd(&s_cnt[gs[c]], 1);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int off = 0, nt = 0;
+    for (int g = 0; g < G; ++g) {
+      s_off[g] = off;
+      s_run[g] = off;
+      s_tstart[g] = nt;
+      offsets[g] = off;
+      off += s_cnt[g];
+      nt += (s_cnt[g] + BM - 1) / BM;
+    }
+    s_off[G] = off;
+    s_tstart[G] = nt;
+    offsets[G] = off;
+    *num_tiles = nt;
+  }
+  __syncthreads();
+  const int nt = s_tstart[G];
+  for (int tile = tid; tile < nt; tile += kSmallBucketThreads) {
+    int lo = 0, hi = G - 1;  // last g with s_tstart[g] <= tile
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) / 2;
+      if (s_tstart[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    const int g = lo;
+    const int i = tile - s_tstart[g];
+    TileInfo ti;
+    ti.row_begin = s_off[g] + i * BM;
+    ti.rows = min(BM, s_cnt[g] - i * BM);
+    if (K == 1) {
+      ti.e0 = g;
+      ti.e1 = g;
+    } else {
+      int b = 1;
+      while ((b + 1) * b / 2 <= g) ++b;
+      ti.e1 = b;
+      ti.e0 = g - b * (b - 1) / 2;
+    }
+    tiles[tile] = ti;
+  }
+#pragma unroll
+  for (int c = 0; c < kChunks; ++c) {
+    if (c * kSmallBucketThreads >= T) break;  // uniform over the CTA
+    for (int g = lane; g < G; g += 32) warpcnt[warp][g] = 0;
+    __syncthreads();
+    const int g = gs[c];
+    const unsigned same = __match_any_sync(0xffffffffu, g);
+    const int lane_rank = __popc(same & ((1u << lane) - 1u));
+    if (g >= 0 && lane_rank == 0) warpcnt[warp][g] = __popc(same);
+    __syncthreads();
+    if (g >= 0) {
+      int pos = s_run[g] + lane_rank;
+      for (int w = 0; w < warp; ++w) pos += warpcnt[w][g];
+      const int t = c * kSmallBucketThreads + tid;
+      slot_tok[pos] = t;
+      if (K == 1) {
+        slot_gate[pos] = gates[t];
+      } else {
+        const int e0 = clamp_e(idx[2 * t], E), e1 = clamp_e(idx[2 * t + 1], E);
+        const float g0 = gates[2 * t], g1 = gates[2 * t + 1];
+        slot_gate[2 * pos] = e0 <= e1 ? g0 : g1;
+        slot_gate[2 * pos + 1] = e0 <= e1 ? g1 : g0;
+      }
+    }
+    __syncthreads();
+    for (int gg = tid; gg < G; gg += kSmallBucketThreads) {
+      int add = 0;
+      for (int w = 0; w < kWarps; ++w) add += warpcnt[w][gg];
+      s_run[gg] += add;
+    }
+    __syncthreads();
+  }
+}
+
 // ---- stage 1 ---------------------------------------------------------------------------------------
 struct Stage1Params {
   int D, W, R, N, R_pad, K2, nbw;  // nbw: 64-column W_x boxes per expert
@@ -617,10 +721,16 @@ __global__ void __launch_bounds__(128) stage1_finish_kernel(const Stage1Params p
   };
   const int ng = p.R / 8;  // dt_low groups per expert
   const int grp = blockIdx.y;
+  const bool live = row < ti.rows;  // rows past the tile's tokens: A' zeros, no B/C output
   if (grp < K * ng) {
     const int j = grp / ng, c = (grp - j * ng) * 8;
     float v[8];
-    sum8(j, c, v);
+    if (live) {
+      sum8(j, c, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    }
     uint32_t hw[4], lw[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) split_bf16x2(g[j] * v[2 * i], g[j] * v[2 * i + 1], hw[i], lw[i]);
@@ -633,7 +743,7 @@ __global__ void __launch_bounds__(128) stage1_finish_kernel(const Stage1Params p
         arow[((K + j) * p.R_pad + cz) / 8] = make_uint4(0, 0, 0, 0);
       }
     }
-  } else {
+  } else if (live) {
     const int q = grp - K * ng;      // 0, 1: B_mix n = 0..7, 8..15; 2, 3: C_mix
     const int which = q >> 1, n0 = (q & 1) * 8;
     float o[8];
@@ -646,11 +756,9 @@ __global__ void __launch_bounds__(128) stage1_finish_kernel(const Stage1Params p
 #pragma unroll
       for (int i = 0; i < 8; ++i) o[i] = fmaf(g[j], v[i], o[i]);
     }
-    if (row < ti.rows) {
-      float4* dst = reinterpret_cast<float4*>((which == 0 ? p.B_mix : p.C_mix) + (size_t)p.slot_tok[pos] * 16 + n0);
-      dst[0] = make_float4(o[0], o[1], o[2], o[3]);
-      dst[1] = make_float4(o[4], o[5], o[6], o[7]);
-    }
+    float4* dst = reinterpret_cast<float4*>((which == 0 ? p.B_mix : p.C_mix) + (size_t)p.slot_tok[pos] * 16 + n0);
+    dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_float4(o[4], o[5], o[6], o[7]);
   }
 }
 
@@ -1002,11 +1110,17 @@ cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s) {
   __nv_bfloat16* aprime = reinterpret_cast<__nv_bfloat16*>(ws + L.aprime);
 
   cudaError_t e;
-  group_count_kernel<K><<<(unsigned)L.nb, kBucketBlock, 0, s>>>(p.idx, p.T, p.E, L.G, group_of, blockhist);
-  group_scan_kernel<K><<<1, 256, 0, s>>>(blockhist, L.nb, L.G, offsets, blockbase, num_tiles, tiles);
-  group_scatter_kernel<K><<<(unsigned)L.nb, kBucketBlock, 0, s>>>(p.idx, p.gates, p.T, p.E, L.G, group_of, blockbase,
-                                                                   slot_tok, slot_gate);
-  note_launch(3);
+  if (p.T <= kSmallBucketT) {
+    group_bucket_small_kernel<K><<<1, kSmallBucketThreads, 0, s>>>(p.idx, p.gates, (int)p.T, p.E, L.G, offsets,
+                                                                    num_tiles, tiles, slot_tok, slot_gate);
+    note_launch();
+  } else {
+    group_count_kernel<K><<<(unsigned)L.nb, kBucketBlock, 0, s>>>(p.idx, p.T, p.E, L.G, group_of, blockhist);
+    group_scan_kernel<K><<<1, 256, 0, s>>>(blockhist, L.nb, L.G, offsets, blockbase, num_tiles, tiles);
+    group_scatter_kernel<K><<<(unsigned)L.nb, kBucketBlock, 0, s>>>(p.idx, p.gates, p.T, p.E, L.G, group_of,
+                                                                     blockbase, slot_tok, slot_gate);
+    note_launch(3);
+  }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   const int W = p.R + 2 * p.N;

@@ -154,14 +154,18 @@ __global__ void __launch_bounds__(512, 1) route_smem_kernel(RouteParams p) {
   }
 }
 
-// Few tokens (decode steps, short prompts): one CTA of 128 threads per token, so every SM works
-// even when T is a few hundred. The threads split the channels in 16-byte chunks of x, each
+// Few tokens (decode steps, short prompts): one CTA of 512 threads per token, so every SM works
+// even when T is a few hundred. The threads split the channels in 16-byte chunks of x (one chunk
+// each at D = 4096 bf16, so a thread's x and W_r loads are all in flight at once), each
 // accumulates the E partial logits of its chunks (W_r rows from L2), a shuffle butterfly and a
 // shared-memory pass reduce them, and thread 0 selects and normalises the token's experts.
+constexpr int kSmallThreads = 512;  // one 16-byte chunk of x per thread at D = 4096 (bf16)
+
 template <typename IO, int EP>
-__global__ void __launch_bounds__(128) route_small_kernel(RouteParams p) {
+__global__ void __launch_bounds__(kSmallThreads) route_small_kernel(RouteParams p) {
   constexpr int V = Vec16<IO>::n;
-  __shared__ float part[4][EP];
+  constexpr int kWarps = kSmallThreads / 32;
+  __shared__ float part[kWarps][EP];
   const int64_t t = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const IO* x = reinterpret_cast<const IO*>(p.x) + t * p.D;
@@ -169,7 +173,7 @@ __global__ void __launch_bounds__(128) route_small_kernel(RouteParams p) {
 #pragma unroll
   for (int e = 0; e < EP; ++e) acc[e] = 0.f;
   const bool vec = (p.E & 3) == 0;  // W_r rows of 16-byte multiples: float4 loads
-  for (int c = threadIdx.x; c < p.D / V; c += 128) {
+  for (int c = threadIdx.x; c < p.D / V; c += kSmallThreads) {
     float xf[V];
     Vec16<IO>::unpack(__ldg(reinterpret_cast<const uint4*>(x) + c), xf);
 #pragma unroll
@@ -202,7 +206,11 @@ __global__ void __launch_bounds__(128) route_small_kernel(RouteParams p) {
   if (threadIdx.x == 0) {
     float l[EP];
 #pragma unroll
-    for (int e = 0; e < EP; ++e) l[e] = (part[0][e] + part[1][e]) + (part[2][e] + part[3][e]);
+    for (int e = 0; e < EP; ++e) {
+      float a = 0.f;
+      for (int w = 0; w < kWarps; ++w) a += part[w][e];
+      l[e] = a;
+    }
     select_topk<EP>(l, p.E, p.k, p.idx + t * p.k, p.gates + t * p.k);
   }
 }
@@ -213,7 +221,7 @@ static cudaError_t launch_route(const RouteParams& p, cudaStream_t s) {
   const size_t smem = sizeof(float2) * (EP / 2) * (size_t)p.D;
   (void)V;
   if (p.T <= kSmallT) {
-    route_small_kernel<IO, EP><<<(unsigned)p.T, 128, 0, s>>>(p);
+    route_small_kernel<IO, EP><<<(unsigned)p.T, kSmallThreads, 0, s>>>(p);
   } else if (smem <= 160 * 1024) {
     cudaError_t e =
         cudaFuncSetAttribute(route_smem_kernel<IO, EP, TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
