@@ -105,10 +105,25 @@ swimba_status gemm_rm(cudaStream_t s, bool bf16, int M, int n, int kd, const voi
   return SWIMBA_OK;
 }
 
+// Every argument a block call hands to the calls it makes, checked before the first launch (the
+// layer's own calls check them again, but by then the in-projection would be queued).
 swimba_status check_weights(const swimba_block_weights* w) {
   if (!w || !w->W_in || !w->conv_w || !w->conv_b || !w->W_out) return SWIMBA_ERR_INVALID_ARG;
+  const swimba_weights& l = w->layer;
+  if (!l.W_r || !l.W_x || !l.W_dt || !l.b_dt || !l.A || !l.D_skip) return SWIMBA_ERR_INVALID_ARG;
   if (!aligned16(w->W_in) || !aligned16(w->W_out) || !aligned16(w->conv_w) || !aligned16(w->conv_b))
     return SWIMBA_ERR_ALIGN;
+  if (!aligned16(l.W_r) || !aligned16(l.W_x) || !aligned16(l.W_dt) || !aligned16(l.b_dt) || !aligned16(l.A) ||
+      !aligned16(l.D_skip))
+    return SWIMBA_ERR_ALIGN;
+  return SWIMBA_OK;
+}
+
+swimba_status check_states(const swimba_block_dims* bd, const float* h0, const float* h_final, const void* cs_in,
+                           const void* cs_out) {
+  if (bd->d_conv > 1 && cs_in != nullptr && cs_in == cs_out) return SWIMBA_ERR_INVALID_ARG;
+  if ((h0 && !aligned16(h0)) || (h_final && !aligned16(h_final))) return SWIMBA_ERR_ALIGN;
+  if (bd->d_conv > 1 && ((cs_in && !aligned16(cs_in)) || (cs_out && !aligned16(cs_out)))) return SWIMBA_ERR_ALIGN;
   return SWIMBA_OK;
 }
 
@@ -180,6 +195,7 @@ swimba_status swimba_block_fwd(const swimba_block_dims* bd, const void* u, const
   if (st != SWIMBA_OK) return st;
   if (!u || !out) return SWIMBA_ERR_INVALID_ARG;
   if ((st = check_weights(w)) != SWIMBA_OK) return st;
+  if ((st = check_states(bd, h0, h_final, conv_state_in, conv_state_out)) != SWIMBA_OK) return st;
   if (!aligned16(u) || !aligned16(out)) return SWIMBA_ERR_ALIGN;
   const BlockLayout l = block_layout(bd);
   if (ws == nullptr || ws_bytes < l.total) return SWIMBA_ERR_WORKSPACE;
@@ -214,6 +230,7 @@ swimba_status swimba_block_step(const swimba_block_dims* bd, const void* u, cons
   if (st != SWIMBA_OK) return st;
   if (bd->layer.seqlen != 1 || !u || !out || !h || (bd->d_conv > 1 && !conv_state)) return SWIMBA_ERR_INVALID_ARG;
   if ((st = check_weights(w)) != SWIMBA_OK) return st;
+  if ((st = check_states(bd, h, nullptr, conv_state, nullptr)) != SWIMBA_OK) return st;
   if (!aligned16(u) || !aligned16(out)) return SWIMBA_ERR_ALIGN;
   const BlockLayout l = block_layout(bd);
   if (ws == nullptr || ws_bytes < l.total) return SWIMBA_ERR_WORKSPACE;

@@ -114,10 +114,20 @@ def test_block_and_conv_arguments_are_checked_before_any_launch(S):
                               0) == 2
     nw = S.swimba_block_weights(fake, None, fake, fake, lw)
     assert S.swimba_block_fwd(bd, fake, nw, None, None, fake, None, None, fake, n, 0) == 1
+    # the layer's and the states' arguments are checked before the in-projection is queued
+    no_A = S.swimba_block_weights(fake, fake, fake, fake, S.swimba_weights(fake, fake, fake, fake, None, fake))
+    assert S.swimba_block_fwd(bd, fake, no_A, None, None, fake, None, None, fake, n, 0) == 1
+    odd_A = S.swimba_block_weights(fake, fake, fake, fake, S.swimba_weights(fake, fake, fake, fake, fake + 4, fake))
+    assert S.swimba_block_fwd(bd, fake, odd_A, None, None, fake, None, None, fake, n, 0) == 3
+    assert S.swimba_block_fwd(bd, fake, w, None, fake, fake, None, fake, fake, n, 0) == 1  # conv state in == out
+    assert S.swimba_block_fwd(bd, fake, w, fake + 4, None, fake, None, None, fake, n, 0) == 3  # h0
+    assert S.swimba_block_fwd(bd, fake, w, None, fake + 8, fake, None, None, fake, n, 0) == 3  # conv state in
     assert S.swimba_block_step(bd, fake, w, fake, fake, fake, fake, n, 0) == 1  # seqlen != 1
     sd = S.swimba_block_dims(S.make_dims(cfg, seqlen=1), 2048, 4)
     assert S.swimba_block_step(sd, fake, w, None, fake, fake, fake, n, 0) == 1  # no state
     assert S.swimba_block_step(sd, fake, w, fake, None, fake, fake, n, 0) == 1  # no conv state
+    assert S.swimba_block_step(sd, fake, w, fake + 4, fake, fake, fake, n, 0) == 3  # h
+    assert S.swimba_block_step(sd, fake, w, fake, fake + 8, fake, fake, n, 0) == 3  # conv state
     # the convolution alone
     assert S.swimba_conv1d_fwd(dims, 9, fake, fake, fake, None, fake, None, 0) == 2
     assert S.swimba_conv1d_fwd(dims, 4, None, fake, fake, None, fake, None, 0) == 1
