@@ -120,3 +120,61 @@ def test_pins_catch_planted_mistake(name, monkeypatch):
             failed.append(exc)
             break
     assert failed, f"no pin fails with the planted mistake: {name}"
+
+
+# ---- the Mamba-2 SSD form (oracle/swimba_ssd_oracle.py) ----------------------------------------
+
+from oracle import swimba_ssd_oracle as SSD  # noqa: E402
+import tests.test_oracle_ssd_pins as SP  # noqa: E402
+
+SSD_PINS = [
+    lambda: SP.test_ssd_brute_force_unrolled_sum(5),
+    SP.test_one_channel_per_head_reduces_to_the_selective_scan,
+    SP.test_identical_experts_equal_one_expert,
+    SP.test_superposition_in_X_and_the_state,
+    SP.test_state_decays_freely_without_input,
+    lambda: SP.test_chunked_form_equals_sequential(4),
+    SP.test_chunked_zero_state_when_absent,
+]
+
+SSD_MUTATIONS = {
+    "decay without delta": ("ssd_scan_sequential", "a = np.exp(delta[t] * A)", "a = np.exp(A)"),
+    "injection without delta": ("ssd_scan_sequential", "S = a[:, None, None] * S + delta[t][:, None, None] * inj",
+                                "S = a[:, None, None] * S + inj"),
+    "injection decayed too": ("ssd_scan_sequential", "S = a[:, None, None] * S + delta[t][:, None, None] * inj",
+                              "S = a[:, None, None] * (S + delta[t][:, None, None] * inj)"),
+    "readout with the first expert's C": ("ssd_scan_sequential", "c_mix = g[t] @ C[t]", "c_mix = C[t, 0]"),
+    "skip on the first expert's X": ("ssd_scan_sequential", 'x_mix = np.einsum("j,jhp->hp", g[t], X[t])',
+                                     "x_mix = X[t, 0]"),
+    "injection ungated": ("ssd_scan_sequential", "inj += g[t, j] * X[t, j]", "inj += X[t, j]"),
+    "chunk mask transposed": ("ssd_scan_chunked", "np.tril(np.ones((n, n)))", "np.triu(np.ones((n, n)))"),
+    "carried state undecayed in the readout": ("ssd_scan_chunked",
+                                               'y_c += np.exp(cum)[:, :, None] * np.einsum("hpn,in->ihp", S, c_mix)',
+                                               'y_c += np.einsum("hpn,in->ihp", S, c_mix)'),
+    "state passed without the tail decay": ("ssd_scan_chunked", "tail = np.exp(cum[-1][None, :] - cum)",
+                                            "tail = np.ones_like(cum)"),
+    "in-chunk term without the gate": ("ssd_scan_chunked", "(cb * (g[c0:c1, j])[None, :])", "(cb * 1.0)"),
+}
+
+
+def _ssd_mutant(fn_name, old, new):
+    src = textwrap.dedent(inspect.getsource(getattr(SSD, fn_name)))
+    assert old in src, f"mutation target not found in {fn_name}: {old!r}"
+    src = src.replace(old, new, 1)
+    ns = dict(vars(SSD))
+    exec(compile(src, f"<mutant {fn_name}>", "exec"), ns)
+    return ns[fn_name]
+
+
+@pytest.mark.parametrize("name", sorted(SSD_MUTATIONS))
+def test_ssd_pins_catch_planted_mistake(name, monkeypatch):
+    fn_name, old, new = SSD_MUTATIONS[name]
+    monkeypatch.setattr(SSD, fn_name, _ssd_mutant(fn_name, old, new))
+    failed = []
+    for pin in SSD_PINS:
+        try:
+            pin()
+        except Exception as exc:
+            failed.append(exc)
+            break
+    assert failed, f"no pin fails with the planted mistake: {name}"
