@@ -192,3 +192,35 @@ def test_block_bf16_stores_bf16_values():
         np.testing.assert_array_equal(O.round_bf16(r[key]), r[key])
     rf = O.block_forward(u, BW, 2, io="f32")
     assert np.abs(r["o"] - rf["o"]).max() < 0.05 * (1 + np.abs(rf["o"]).max())
+
+
+# ------------------------------------------------------------------------------------------
+# the block's seeded inputs
+# ------------------------------------------------------------------------------------------
+
+def test_block_draws_are_reproducible_piecewise_and_follow_the_recipe():
+    from parameter_space_moe_swimba_b200 import synth
+    from parameter_space_moe_swimba_b200.configs import CONFIGS
+
+    cfg = CONFIGS["mamba130m_like"].with_(seqlen=24)
+    dm, W = 256, 4
+    w1, w2 = synth.draw_block_weights(cfg, dm, W), synth.draw_block_weights(cfg, dm, W)
+    np.testing.assert_array_equal(w1.W_in, w2.W_in)
+    np.testing.assert_array_equal(w1.conv_w, w2.conv_w)
+    assert w1.W_in.shape == (dm, 2 * cfg.d_inner) and w1.W_in.dtype == np.uint16
+    assert w1.W_out.shape == (cfg.d_inner, dm) and w1.conv_w.shape == (cfg.d_inner, W)
+    bound = 1.0 / np.sqrt(W)
+    assert np.all(np.abs(w1.conv_w) <= bound) and np.all(np.abs(w1.conv_b) <= bound)
+    # the layer's weights inside the block are the layer's own draw
+    np.testing.assert_array_equal(w1.layer.W_x, synth.draw_weights(cfg).W_x)
+    # scale: W_in ~ N(0, 1/d_model)
+    w_in = synth.widen(w1.W_in, "bf16")
+    assert abs(w_in.std() * np.sqrt(dm) - 1.0) < 0.02
+    u = synth.draw_block_input(cfg, dm)
+    u2 = synth.draw_block_input(cfg, dm, batch_rows=[3])
+    np.testing.assert_array_equal(u[3], u2[0])
+    cs = synth.draw_conv_state(cfg, W)
+    assert cs.shape == (cfg.batch, W - 1, cfg.d_inner) and cs.dtype == np.uint16
+    r1 = synth.redraw_u_row(cfg, dm, 1, 5, 0)
+    np.testing.assert_array_equal(r1, synth.redraw_u_row(cfg, dm, 1, 5, 0))
+    assert not np.array_equal(r1, synth.redraw_u_row(cfg, dm, 1, 5, 1))
