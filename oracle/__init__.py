@@ -1,4 +1,6 @@
-"""fp64 CPU oracle of the Swimba layer -- test infrastructure, never the library's compute path."""
+"""fp64 CPU oracle of the Swimba layer and its surrounding block (``swimba_oracle``) and of the scan
+in the Mamba-2 SSD form (``swimba_ssd_oracle``) -- test infrastructure, never the library's
+compute path."""
 from .swimba_oracle import (  # noqa: F401
     block_branches,
     block_decode_step,
