@@ -66,6 +66,8 @@ __all__ = [
     "selective_scan",
     "layer_forward",
     "decode_step",
+    "scan_summary",
+    "chain_summaries",
     "round_bf16",
     "causal_conv1d",
     "block_branches",
@@ -228,6 +230,50 @@ def decode_step(h, x_t, z_t, W, k, channels=None):
     """
     r = layer_forward(x_t, z_t, W, k, h0=h, channels=channels)
     return r["out"], r["h_final"], r
+
+
+def scan_summary(x, dt_mix, B_mix, idx, gates, A):
+    """What one piece of a sequence hands to the next ([MB] "Estado interno puramente lineal": the
+    state is linear, so the recurrence can be split and recombined).
+
+    Over the given tokens (x, dt_mix [B, L, D]; B_mix [B, L, N]; idx, gates [B, L, k]; A [E, D, N])
+    the state after the last token is linear in the state before the first one:
+        h_end(h_in) = exp(Σ_t Δ_t A_t) ⊙ h_in + h_end(0).
+    Returns (h_zero [B, D, N], log_decay [B, D, N]): the end state of the recurrence started from
+    zero, and Σ_t Δ_t A_t (the natural log of the product of the per-token decays ā_t).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    A = np.asarray(A, dtype=np.float64)
+    Bsz, L, D = x.shape
+    N = A.shape[2]
+    delta = softplus(dt_mix)
+    g = np.asarray(gates, dtype=np.float64)
+    h = np.zeros((Bsz, D, N))
+    log_decay = np.zeros((Bsz, D, N))
+    for t in range(L):
+        d_t = delta[:, t, :]
+        A_t = np.zeros((Bsz, D, N))
+        for j in range(idx.shape[2]):
+            A_t += g[:, t, j, None, None] * A[idx[:, t, j]]
+        log_decay += d_t[:, :, None] * A_t
+        h = np.exp(d_t[:, :, None] * A_t) * h + d_t[:, :, None] * B_mix[:, t, None, :] * x[:, t, :, None]
+    return h, log_decay
+
+
+def chain_summaries(h_zero, log_decay, h0=None):
+    """Start state of every piece of a sequence cut into P consecutive pieces, from the pieces'
+    summaries (``scan_summary``) stacked on a leading axis [P, B, D, N]:
+        H_0 = h0 (zeros when absent);   H_{p+1} = exp(log_decay_p) ⊙ H_p + h_zero_p.
+    Returns H [P + 1, B, D, N]; H[P] is the state after the whole sequence."""
+    h_zero = np.asarray(h_zero, dtype=np.float64)
+    log_decay = np.asarray(log_decay, dtype=np.float64)
+    P = h_zero.shape[0]
+    H = np.zeros((P + 1,) + h_zero.shape[1:])
+    if h0 is not None:
+        H[0] = np.asarray(h0, dtype=np.float64)
+    for p in range(P):
+        H[p + 1] = np.exp(log_decay[p]) * H[p] + h_zero[p]
+    return H
 
 
 # ------------------------------------------------------------------------------------------------

@@ -43,6 +43,9 @@ PINS = [
     lambda: BP.test_block_split_and_decode_equal_whole(2),
     BP.test_block_output_minus_residual_is_linear_in_W_out,
     BP.test_block_bf16_stores_bf16_values,
+    P.test_summary_closed_form_constant_inputs_scalar_state,
+    lambda: P.test_summary_brute_force(3),
+    P.test_chain_of_piece_summaries_gives_the_prefix_states,
 ]
 
 MUTATIONS = {
@@ -92,6 +95,17 @@ MUTATIONS = {
     "block conv state not carried": ("block_branches", "BW[\"conv_b\"], conv_state)", "BW[\"conv_b\"], None)"),
     "block h0 not carried": ("block_forward", "layer_forward(x, z, BW, k, h0=h0)", "layer_forward(x, z, BW, k, h0=None)"),
     "block layer on x_pre": ("block_forward", "layer_forward(x, z, BW, k", "layer_forward(x_pre, z, BW, k"),
+    "summary decay without delta": ("scan_summary", "log_decay += d_t[:, :, None] * A_t", "log_decay += A_t"),
+    "summary injection without delta": ("scan_summary", "h + d_t[:, :, None] * B_mix[:, t, None, :] * x[:, t, :, None]",
+                                        "h + B_mix[:, t, None, :] * x[:, t, :, None]"),
+    "summary injection decayed too": ("scan_summary",
+                                      "h = np.exp(d_t[:, :, None] * A_t) * h + d_t",
+                                      "h = np.exp(d_t[:, :, None] * A_t) * h * 0.5 + d_t"),
+    "chain adds before decaying": ("chain_summaries", "np.exp(log_decay[p]) * H[p] + h_zero[p]",
+                                   "np.exp(log_decay[p]) * (H[p] + h_zero[p])"),
+    "chain ignores h0": ("chain_summaries", "if h0 is not None:", "if False:"),
+    "chain uses the next piece's decay": ("chain_summaries", "np.exp(log_decay[p])",
+                                          "np.exp(log_decay[min(p + 1, P - 1)])"),
     "bf16 rounding toward zero": ("round_bf16", "np.rint(m * 256.0)", "np.trunc(m * 256.0)"),
     "bf16 rounding with 7 bits": ("round_bf16", "np.ldexp(np.rint(m * 256.0), e - 8)", "np.ldexp(np.rint(m * 128.0), e - 7)"),
 }

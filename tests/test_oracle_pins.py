@@ -444,3 +444,83 @@ def test_synthetic_draws_are_reproducible_and_piecewise():
     # dt = softplus(b_dt) in [1e-3, 1e-1]
     dt = O.softplus(w1.b_dt.astype(np.float64))
     assert dt.min() >= 1e-3 * (1 - 1e-6) and dt.max() <= 1e-1 * (1 + 1e-6)
+
+
+# ------------------------------------------------------------------------------------------
+# splitting a sequence into pieces: summaries and their chain
+# ------------------------------------------------------------------------------------------
+
+def _random_scan_inputs(rng, Bsz, L, D, N, E, k):
+    x = rng.standard_normal((Bsz, L, D))
+    dt = rng.normal(-2, 1, (Bsz, L, D))
+    Bm = rng.standard_normal((Bsz, L, N))
+    Cm = rng.standard_normal((Bsz, L, N))
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(Bsz * L)]).reshape(Bsz, L, k).astype(np.int32)
+    g = rng.random((Bsz, L, k))
+    g /= g.sum(-1, keepdims=True)
+    A = -np.exp(rng.uniform(-1, 3, (E, D, N)))
+    return x, dt, Bm, Cm, idx, g, A
+
+
+def test_summary_closed_form_constant_inputs_scalar_state():
+    """N = D = 1, constant Δ, A, B, x over L tokens: h_zero = u (1 - a^L) / (1 - a) and
+    log_decay = L Δ A (a = e^{ΔA}, u = Δ B x)."""
+    L = 5000
+    dt, A, Bv, xv = -1.5, -0.3, 0.7, -1.1
+    delta = math.log1p(math.exp(dt))
+    a, u = math.exp(delta * A), delta * Bv * xv
+    hz, ld = O.scan_summary(np.full((1, L, 1), xv), np.full((1, L, 1), dt), np.full((1, L, 1), Bv),
+                            np.zeros((1, L, 1), np.int32), np.ones((1, L, 1)), np.full((1, 1, 1), A))
+    np.testing.assert_allclose(hz[0, 0, 0], u * (1 - a ** L) / (1 - a), rtol=1e-12)
+    np.testing.assert_allclose(ld[0, 0, 0], L * delta * A, rtol=1e-12)
+
+
+@pytest.mark.parametrize("L", [1, 3, 7])
+def test_summary_brute_force(L):
+    """h_zero = Σ_s (Π_{r=s+1..L-1} a_r) u_s and log_decay = log Π_t a_t, by explicit loops."""
+    rng = np.random.default_rng(200 + L)
+    Bsz, D, N, E, k = 2, 3, 4, 5, 2
+    x, dt, Bm, _, idx, g, A = _random_scan_inputs(rng, Bsz, L, D, N, E, k)
+    hz, ld = O.scan_summary(x, dt, Bm, idx, g, A)
+    for b in range(Bsz):
+        for d in range(D):
+            for n in range(N):
+                a, u = [], []
+                for t in range(L):
+                    dl = math.log1p(math.exp(dt[b, t, d]))
+                    At = sum(g[b, t, j] * A[idx[b, t, j], d, n] for j in range(k))
+                    a.append(math.exp(dl * At))
+                    u.append(dl * Bm[b, t, n] * x[b, t, d])
+                want = sum(math.prod(a[s + 1:]) * u[s] for s in range(L))
+                assert hz[b, d, n] == pytest.approx(want, rel=1e-12, abs=1e-14)
+                assert ld[b, d, n] == pytest.approx(math.log(math.prod(a)), rel=1e-12, abs=1e-14)
+
+
+def test_chain_of_piece_summaries_gives_the_prefix_states():
+    """Cut a random sequence into uneven pieces: the chained start state of piece p equals the
+    state after the first p pieces by the (separately pinned) sequential scan, from h0; and the
+    state after any piece is exp(log_decay) h_in + h_zero (superposition of the linear state)."""
+    rng = np.random.default_rng(7)
+    Bsz, L, D, N, E, k = 2, 29, 3, 4, 5, 2
+    x, dt, Bm, Cm, idx, g, A = _random_scan_inputs(rng, Bsz, L, D, N, E, k)
+    z = rng.standard_normal((Bsz, L, D))
+    Dsk = rng.standard_normal(D)
+    h0 = rng.standard_normal((Bsz, D, N))
+    cuts = [0, 4, 5, 17, 29]
+    pieces = [(cuts[i], cuts[i + 1]) for i in range(len(cuts) - 1)]
+    summ = [O.scan_summary(x[:, a:b], dt[:, a:b], Bm[:, a:b], idx[:, a:b], g[:, a:b], A) for a, b in pieces]
+    H = O.chain_summaries(np.stack([s[0] for s in summ]), np.stack([s[1] for s in summ]), h0=h0)
+    for p, (_, b) in enumerate(pieces):
+        _, _, hT, _ = O.selective_scan(x[:, :b], z[:, :b], dt[:, :b], Bm[:, :b], Cm[:, :b], idx[:, :b], g[:, :b],
+                                       A, Dsk, h0=h0)
+        np.testing.assert_allclose(H[p + 1], hT, rtol=1e-12, atol=1e-13)
+    # each piece run from its chained start state continues the whole sequence
+    h_in = rng.standard_normal((Bsz, D, N))
+    a, b = pieces[2]
+    _, _, hT, _ = O.selective_scan(x[:, a:b], z[:, a:b], dt[:, a:b], Bm[:, a:b], Cm[:, a:b], idx[:, a:b], g[:, a:b],
+                                   A, Dsk, h0=h_in)
+    np.testing.assert_allclose(hT, np.exp(summ[2][1]) * h_in + summ[2][0], rtol=1e-12, atol=1e-13)
+    # no h0: the chain starts from zero
+    H0 = O.chain_summaries(np.stack([s[0] for s in summ]), np.stack([s[1] for s in summ]))
+    assert np.all(H0[0] == 0)
+    np.testing.assert_allclose(H0[1], summ[0][0], rtol=0, atol=0)
