@@ -68,6 +68,7 @@ __all__ = [
     "decode_step",
     "scan_summary",
     "chain_summaries",
+    "separate_ssm_moe",
     "round_bf16",
     "causal_conv1d",
     "block_branches",
@@ -274,6 +275,46 @@ def chain_summaries(h_zero, log_decay, h0=None):
     for p in range(P):
         H[p + 1] = np.exp(log_decay[p]) * H[p] + h_zero[p]
     return H
+
+
+def separate_ssm_moe(x, z, dt_j, B_j, C_j, idx, gates, A, D_skip, h0=None):
+    """The "MoE of separate SSMs" that [SW] sets against Swimba (Spanish summary §2 "Distinción de
+    Diseños", Dutch "Methodologie", French "Distinction des deux designs MoE-SSM"): every expert
+    keeps its own state trajectory and runs its own recurrent update, so the recurrence work grows
+    with the experts; Teorema 2 is the claim that Swimba's single mixed recurrence avoids it.
+
+    Reading (the pages give no equations for it): expert e has its own state h^(e) [B, D, N]; at
+    token t the k active experts e_j = idx[t, j] advance their own states with their own, unmixed
+    streams and their own transition,
+        Δ^j = softplus(dt_j[t, j]);  h^(e_j) = exp(Δ^j A^{e_j}) ⊙ h^(e_j) + Δ^j B_j[t, j] x_t,
+    the states of the experts not chosen at t are left as they are, and the outputs of the active
+    experts are mixed with the gates:
+        y_t = Σ_j g_j C_j[t, j] · h^(e_j) + D_skip ⊙ x_t;   out_t = y_t ⊙ SiLU(z_t).
+
+    x, z [B, L, D]; dt_j [B, L, k, D]; B_j, C_j [B, L, k, N]; idx, gates [B, L, k]; A [E, D, N];
+    D_skip [D]; h0 [E, B, D, N] or None (zeros). Returns (y, out, h [E, B, D, N])."""
+    x = np.asarray(x, dtype=np.float64)
+    z = np.asarray(z, dtype=np.float64)
+    A = np.asarray(A, dtype=np.float64)
+    E = A.shape[0]
+    Bsz, L, D = x.shape
+    N = A.shape[2]
+    k = idx.shape[2]
+    h = np.zeros((E, Bsz, D, N)) if h0 is None else np.array(h0, dtype=np.float64)
+    g = np.asarray(gates, dtype=np.float64)
+    delta = softplus(dt_j)
+    y = np.empty((Bsz, L, D))
+    for t in range(L):
+        y_t = D_skip[None, :] * x[:, t, :]
+        for b in range(Bsz):
+            for j in range(k):
+                e = idx[b, t, j]
+                d_bj = delta[b, t, j]  # [D]
+                h[e, b] = np.exp(d_bj[:, None] * A[e]) * h[e, b] + d_bj[:, None] * B_j[b, t, j][None, :] * x[b, t, :, None]
+                y_t[b] += g[b, t, j] * (h[e, b] @ C_j[b, t, j])
+        y[:, t, :] = y_t
+    out = y * silu(z)
+    return y, out, h
 
 
 # ------------------------------------------------------------------------------------------------

@@ -46,6 +46,9 @@ PINS = [
     P.test_summary_closed_form_constant_inputs_scalar_state,
     lambda: P.test_summary_brute_force(3),
     P.test_chain_of_piece_summaries_gives_the_prefix_states,
+    P.test_separate_moe_one_expert_is_the_selective_scan,
+    lambda: P.test_separate_moe_brute_force(4),
+    P.test_separate_moe_unchosen_expert_keeps_its_state_and_switching_differs_from_one_trajectory,
 ]
 
 MUTATIONS = {
@@ -106,6 +109,12 @@ MUTATIONS = {
     "chain ignores h0": ("chain_summaries", "if h0 is not None:", "if False:"),
     "chain uses the next piece's decay": ("chain_summaries", "np.exp(log_decay[p])",
                                           "np.exp(log_decay[min(p + 1, P - 1)])"),
+    "separate: one shared trajectory": ("separate_ssm_moe", "e = idx[b, t, j]", "e = 0"),
+    "separate: outputs not gated": ("separate_ssm_moe", "y_t[b] += g[b, t, j] * (", "y_t[b] += 1.0 * ("),
+    "separate: first slot's step for every slot": ("separate_ssm_moe", "d_bj = delta[b, t, j]", "d_bj = delta[b, t, 0]"),
+    "separate: skip dropped": ("separate_ssm_moe", "y_t = D_skip[None, :] * x[:, t, :]", "y_t = 0.0 * x[:, t, :]"),
+    "separate: first slot's readout for every slot": ("separate_ssm_moe", "(h[e, b] @ C_j[b, t, j])",
+                                                       "(h[e, b] @ C_j[b, t, 0])"),
     "bf16 rounding toward zero": ("round_bf16", "np.rint(m * 256.0)", "np.trunc(m * 256.0)"),
     "bf16 rounding with 7 bits": ("round_bf16", "np.ldexp(np.rint(m * 256.0), e - 8)", "np.ldexp(np.rint(m * 128.0), e - 7)"),
 }

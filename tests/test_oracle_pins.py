@@ -524,3 +524,81 @@ def test_chain_of_piece_summaries_gives_the_prefix_states():
     H0 = O.chain_summaries(np.stack([s[0] for s in summ]), np.stack([s[1] for s in summ]))
     assert np.all(H0[0] == 0)
     np.testing.assert_allclose(H0[1], summ[0][0], rtol=0, atol=0)
+
+
+# ------------------------------------------------------------------------------------------
+# the "MoE of separate SSMs" (one state trajectory per expert)
+# ------------------------------------------------------------------------------------------
+
+def _separate_inputs(rng, Bsz, L, D, N, E, k):
+    x = rng.standard_normal((Bsz, L, D))
+    z = rng.standard_normal((Bsz, L, D))
+    dt = rng.normal(-2, 1, (Bsz, L, k, D))
+    Bj = rng.standard_normal((Bsz, L, k, N))
+    Cj = rng.standard_normal((Bsz, L, k, N))
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(Bsz * L)]).reshape(Bsz, L, k).astype(np.int32)
+    g = rng.random((Bsz, L, k))
+    g /= g.sum(-1, keepdims=True)
+    A = -np.exp(rng.uniform(-1, 3, (E, D, N)))
+    Dsk = rng.standard_normal(D)
+    h0 = rng.standard_normal((E, Bsz, D, N))
+    return x, z, dt, Bj, Cj, idx, g, A, Dsk, h0
+
+
+def test_separate_moe_one_expert_is_the_selective_scan():
+    """E = 1, k = 1: one trajectory, the unmixed streams are the mixed ones -- the (pinned) scan."""
+    rng = np.random.default_rng(11)
+    x, z, dt, Bj, Cj, idx, g, A, Dsk, h0 = _separate_inputs(rng, 2, 17, 3, 4, 1, 1)
+    y, out, h = O.separate_ssm_moe(x, z, dt, Bj, Cj, idx, g, A, Dsk, h0=h0)
+    y2, out2, hT, _ = O.selective_scan(x, z, dt[:, :, 0], Bj[:, :, 0], Cj[:, :, 0], idx, g, A, Dsk, h0=h0[0])
+    np.testing.assert_allclose(y, y2, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(out, out2, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(h[0], hT, rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("L", [1, 4, 6])
+def test_separate_moe_brute_force(L):
+    """Explicit loops: each expert's state follows only the tokens routed to it; the output mixes
+    the active experts' readouts with the gates and adds the skip term."""
+    rng = np.random.default_rng(300 + L)
+    Bsz, D, N, E, k = 2, 2, 3, 3, 2
+    x, z, dt, Bj, Cj, idx, g, A, Dsk, h0 = _separate_inputs(rng, Bsz, L, D, N, E, k)
+    y, out, h = O.separate_ssm_moe(x, z, dt, Bj, Cj, idx, g, A, Dsk, h0=h0)
+    for b in range(Bsz):
+        for d in range(D):
+            state = {(e, n): h0[e, b, d, n] for e in range(E) for n in range(N)}
+            for t in range(L):
+                want = Dsk[d] * x[b, t, d]
+                for j in range(k):
+                    e = int(idx[b, t, j])
+                    dl = math.log1p(math.exp(dt[b, t, j, d]))
+                    for n in range(N):
+                        state[e, n] = math.exp(dl * A[e, d, n]) * state[e, n] + dl * Bj[b, t, j, n] * x[b, t, d]
+                    want += g[b, t, j] * sum(Cj[b, t, j, n] * state[e, n] for n in range(N))
+                assert y[b, t, d] == pytest.approx(want, rel=1e-12, abs=1e-13)
+                assert out[b, t, d] == pytest.approx(want * z[b, t, d] / (1 + math.exp(-z[b, t, d])), rel=1e-12,
+                                                     abs=1e-13)
+            for e in range(E):
+                for n in range(N):
+                    assert h[e, b, d, n] == pytest.approx(state[e, n], rel=1e-12, abs=1e-13)
+
+
+def test_separate_moe_unchosen_expert_keeps_its_state_and_switching_differs_from_one_trajectory():
+    """An expert never routed to keeps its initial state exactly. With identical experts, constant
+    routing gives the single-trajectory scan; routing that switches between experts does not
+    (the pages' Théorème 4: the compressed and the separate models differ when routing varies)."""
+    rng = np.random.default_rng(12)
+    Bsz, L, D, N, E = 1, 12, 3, 4, 3
+    x, z, dt, Bj, Cj, _, _, A, Dsk, h0 = _separate_inputs(rng, Bsz, L, D, N, E, 1)
+    A[:] = A[0]
+    g = np.ones((Bsz, L, 1))
+    const = np.zeros((Bsz, L, 1), np.int32)
+    y, _, h = O.separate_ssm_moe(x, z, dt, Bj, Cj, const, g, A, Dsk, h0=h0)
+    np.testing.assert_array_equal(h[1], h0[1])
+    np.testing.assert_array_equal(h[2], h0[2])
+    y1, _, _, _ = O.selective_scan(x, z, dt[:, :, 0], Bj[:, :, 0], Cj[:, :, 0], const, g, A, Dsk, h0=h0[0])
+    np.testing.assert_allclose(y, y1, rtol=1e-13, atol=1e-14)
+    switching = (np.arange(L) % 2).reshape(Bsz, L, 1).astype(np.int32)
+    y2, _, _ = O.separate_ssm_moe(x, z, dt, Bj, Cj, switching, g, A, Dsk, h0=np.zeros_like(h0))
+    y3, _, _, _ = O.selective_scan(x, z, dt[:, :, 0], Bj[:, :, 0], Cj[:, :, 0], switching, g, A, Dsk)
+    assert np.max(np.abs(y2 - y3)) > 1e-3
