@@ -143,8 +143,12 @@ def expert_projections(x, idx, gates, W_x, W_dt, b_dt, dt_rank, d_state):
     return {"xdbl": xdbl, "dt_j": dt_j, "dt_mix": dt_mix, "B_mix": B_mix, "C_mix": C_mix}
 
 
-def selective_scan(x, z, dt_mix, B_mix, C_mix, idx, gates, A, D_skip, h0=None, channels=None):
+def selective_scan(x, z, dt_mix, B_mix, C_mix, idx, gates, A, D_skip, h0=None, channels=None, injection="euler"):
     """The single recurrence over the mixed parameters ([SW] one state trajectory; [MB] "Mamba").
+
+    ``injection`` picks the input discretisation: "euler" (the layer's definition, Δ B x) or "zoh",
+    the zero-order hold of [MB] "Mamba" (B̄ = A⁻¹(exp(ΔA) − I) B; with the diagonal mixed transition
+    it is elementwise, (exp(Δ A_t) − 1) / A_t · B_mix · x, written with expm1).
 
     x, z, dt_mix [B, L, D]; B_mix, C_mix [B, L, N]; idx, gates [B, L, k]; A [E, D, N];
     D_skip [D]; h0 [B, D, N] or None (zeros). ``channels`` optionally restricts the work to a list
@@ -180,14 +184,19 @@ def selective_scan(x, z, dt_mix, B_mix, C_mix, idx, gates, A, D_skip, h0=None, c
         for j in range(idx.shape[2]):
             A_t += g[:, t, j, None, None] * A[idx[:, t, j]]
         a_bar = np.exp(d_t[:, :, None] * A_t)
-        u = d_t[:, :, None] * B_mix[:, t, None, :] * x[:, t, :, None]
+        if injection == "zoh":
+            u = np.expm1(d_t[:, :, None] * A_t) / A_t * B_mix[:, t, None, :] * x[:, t, :, None]
+        elif injection == "euler":
+            u = d_t[:, :, None] * B_mix[:, t, None, :] * x[:, t, :, None]
+        else:
+            raise ValueError("injection must be 'euler' or 'zoh'")
         h = a_bar * h + u
         y[:, t, :] = np.einsum("bn,bdn->bd", C_mix[:, t, :], h) + D_skip[None, :] * x[:, t, :]
     out = y * silu(z)
     return y, out, h, delta
 
 
-def layer_forward(x, z, W, k, h0=None, channels=None):
+def layer_forward(x, z, W, k, h0=None, channels=None, injection="euler"):
     """The Swimba layer: route -> per-expert projections mixed by the gates -> one scan.
 
     x, z [B, L, D] fp64 values; W: a mapping with fp64 values W_r [D,E], W_x [E,D,R+2N],
@@ -206,7 +215,8 @@ def layer_forward(x, z, W, k, h0=None, channels=None):
     idx_b, gates_b = shp(idx), shp(gates)
     dt_mix, B_mix, C_mix = shp(proj["dt_mix"]), shp(proj["B_mix"]), shp(proj["C_mix"])
     y, out, h_final, delta = selective_scan(
-        x, z, dt_mix, B_mix, C_mix, idx_b, gates_b, W["A"], W["D_skip"], h0=h0, channels=channels
+        x, z, dt_mix, B_mix, C_mix, idx_b, gates_b, W["A"], W["D_skip"], h0=h0, channels=channels,
+        injection=injection,
     )
     assert E == W["W_x"].shape[0]
     return {

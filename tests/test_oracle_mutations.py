@@ -49,6 +49,8 @@ PINS = [
     P.test_separate_moe_one_expert_is_the_selective_scan,
     lambda: P.test_separate_moe_brute_force(4),
     P.test_separate_moe_unchosen_expert_keeps_its_state_and_switching_differs_from_one_trajectory,
+    P.test_zoh_is_the_exact_solution_for_held_inputs,
+    lambda: P.test_zoh_brute_force_and_small_step_limit(3),
 ]
 
 MUTATIONS = {
@@ -115,6 +117,11 @@ MUTATIONS = {
     "separate: skip dropped": ("separate_ssm_moe", "y_t = D_skip[None, :] * x[:, t, :]", "y_t = 0.0 * x[:, t, :]"),
     "separate: first slot's readout for every slot": ("separate_ssm_moe", "(h[e, b] @ C_j[b, t, j])",
                                                        "(h[e, b] @ C_j[b, t, 0])"),
+    "zoh without the transition's inverse": ("selective_scan", "np.expm1(d_t[:, :, None] * A_t) / A_t",
+                                             "np.expm1(d_t[:, :, None] * A_t)"),
+    "zoh with exp instead of expm1": ("selective_scan", "np.expm1(d_t[:, :, None] * A_t) / A_t",
+                                      "np.exp(d_t[:, :, None] * A_t) / A_t"),
+    "zoh falls back to Euler": ("selective_scan", 'if injection == "zoh":', 'if injection == "never":'),
     "bf16 rounding toward zero": ("round_bf16", "np.rint(m * 256.0)", "np.trunc(m * 256.0)"),
     "bf16 rounding with 7 bits": ("round_bf16", "np.ldexp(np.rint(m * 256.0), e - 8)", "np.ldexp(np.rint(m * 128.0), e - 7)"),
 }

@@ -602,3 +602,55 @@ def test_separate_moe_unchosen_expert_keeps_its_state_and_switching_differs_from
     y2, _, _ = O.separate_ssm_moe(x, z, dt, Bj, Cj, switching, g, A, Dsk, h0=np.zeros_like(h0))
     y3, _, _, _ = O.selective_scan(x, z, dt[:, :, 0], Bj[:, :, 0], Cj[:, :, 0], switching, g, A, Dsk)
     assert np.max(np.abs(y2 - y3)) > 1e-3
+
+
+# ------------------------------------------------------------------------------------------
+# the zero-order-hold injection
+# ------------------------------------------------------------------------------------------
+
+def test_zoh_is_the_exact_solution_for_held_inputs():
+    """With A, B and x held constant and only the step Δ_t varying, the zero-order hold integrates
+    dh/dt = A h + B x exactly: after L steps h = e^{A T} h0 + (e^{A T} - 1) / A · B x, T = Σ Δ_t,
+    however T is split into steps."""
+    rng = np.random.default_rng(21)
+    L = 1000
+    A, Bv, xv, h0 = -0.37, 1.3, -0.8, 0.45
+    dt = rng.normal(-3, 1.5, (1, L, 1))
+    delta = np.log1p(np.exp(dt))
+    T = float(delta.sum())
+    _, _, hT, _ = O.selective_scan(np.full((1, L, 1), xv), np.ones((1, L, 1)), dt, np.full((1, L, 1), Bv),
+                                   np.ones((1, L, 1)), np.zeros((1, L, 1), np.int32), np.ones((1, L, 1)),
+                                   np.full((1, 1, 1), A), np.zeros(1), h0=np.full((1, 1, 1), h0), injection="zoh")
+    want = math.exp(A * T) * h0 + math.expm1(A * T) / A * Bv * xv
+    assert hT[0, 0, 0] == pytest.approx(want, rel=1e-11)
+
+
+@pytest.mark.parametrize("L", [1, 3, 5])
+def test_zoh_brute_force_and_small_step_limit(L):
+    """Unrolled sum with u_t = (e^{Δ A_t} - 1) / A_t B x; and for tiny steps the ZOH injection tends
+    to the Euler one, u_zoh / u_euler = 1 + Δ A_t / 2 + O(Δ²)."""
+    rng = np.random.default_rng(400 + L)
+    Bsz, D, N, E, k = 2, 2, 3, 4, 2
+    x, dt, Bm, Cm, idx, g, A = _random_scan_inputs(rng, Bsz, L, D, N, E, k)
+    z = rng.standard_normal((Bsz, L, D))
+    Dsk = rng.standard_normal(D)
+    h0 = rng.standard_normal((Bsz, D, N))
+    y, _, hT, _ = O.selective_scan(x, z, dt, Bm, Cm, idx, g, A, Dsk, h0=h0, injection="zoh")
+    for b in range(Bsz):
+        for d in range(D):
+            for t in range(L):
+                want = Dsk[d] * x[b, t, d]
+                for n in range(N):
+                    a, u = [], []
+                    for s in range(t + 1):
+                        dl = math.log1p(math.exp(dt[b, s, d]))
+                        At = sum(g[b, s, j] * A[idx[b, s, j], d, n] for j in range(k))
+                        a.append(math.exp(dl * At))
+                        u.append(math.expm1(dl * At) / At * Bm[b, s, n] * x[b, s, d])
+                    h = math.prod(a) * h0[b, d, n] + sum(math.prod(a[s + 1:]) * u[s] for s in range(t + 1))
+                    want += Cm[b, t, n] * h
+                assert y[b, t, d] == pytest.approx(want, rel=1e-11, abs=1e-12)
+    tiny = np.full_like(dt, -16.0)  # Δ = softplus(-16) ~ 1.1e-7
+    _, _, hz, _ = O.selective_scan(x, z, tiny, Bm, Cm, idx, g, A, Dsk, injection="zoh")
+    _, _, he, _ = O.selective_scan(x, z, tiny, Bm, Cm, idx, g, A, Dsk, injection="euler")
+    np.testing.assert_allclose(hz, he, rtol=2e-5, atol=0)
