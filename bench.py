@@ -47,11 +47,14 @@ def parse():
     ap.add_argument("--impl", default="swimba", choices=["swimba", "reference"])
     ap.add_argument("--workload", default="mamba1p4b_like")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling runs)")
+    ap.add_argument("--seqlen", type=int, default=0, help="override the workload's sequence length (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--report", action="store_true",
                     help="per-workload table (one JSON line each): every workload, decode steps, E sweep")
+    ap.add_argument("--report-separate", action="store_true",
+                    help="only the separate-SSM comparison line (Teorema 2)")
     ap.add_argument("--report-block", action="store_true",
                     help="only the surrounding block's report lines (with --batch: the prefill line at that batch)")
     return ap.parse_args()
@@ -74,29 +77,27 @@ def load_peaks():
 # ------------------------------------------------------------------------------------------------
 
 def measured_traffic(cfg):
-    """DRAM bytes per scan launch from the committed ncu summary (dram__bytes_read.sum +
-    dram__bytes_write.sum), or None when the summary is for another workload or the scan kernel's
-    source has changed since it was taken."""
+    """DRAM bytes per scan launch (dram__bytes_read.sum + dram__bytes_write.sum) from the committed
+    ncu figure in profiles/scan_traffic.json, scaled to this workload's tokens when the capture was
+    taken on a shorter sequence of the same shape (the scan's traffic grows with the tokens); None
+    when the figure is for another shape or the scan kernel's source has changed since."""
     import hashlib
 
-    if cfg.name != "mamba1p4b_like" or cfg.batch != CONFIGS["mamba1p4b_like"].batch:
-        return None
-    summary = os.path.join(ROOT, "profiles", "scan_fast_mamba1p4b_like.md")
+    path = os.path.join(ROOT, "profiles", "scan_traffic.json")
     src = os.path.join(ROOT, "parameter_space_moe_swimba_b200", "csrc", "scan_fast.cu")
     try:
-        fields = {}
-        with open(summary) as f:
-            for line in f:
-                k, sep, v = line.strip().partition(": ")
-                if sep and k in ("kernel_source_sha256", "dram_bytes_per_launch"):
-                    fields[k] = v.strip()
+        with open(path) as f:
+            rec = json.load(f)
         with open(src, "rb") as f:
             digest = hashlib.sha256(f.read()).hexdigest()
-    except OSError:
+    except (OSError, ValueError):
         return None
-    if fields.get("kernel_source_sha256") != digest or "dram_bytes_per_launch" not in fields:
+    if rec.get("kernel_source_sha256") != digest:
         return None
-    return int(fields["dram_bytes_per_launch"])
+    shape = {k: getattr(cfg, k) for k in ("batch", "d_inner", "d_state", "n_experts", "top_k", "io_dtype")}
+    if rec.get("shape") != shape:
+        return None
+    return int(rec["dram_bytes_per_launch"] * cfg.seqlen / rec["seqlen"])
 
 
 def io_bytes(cfg):
@@ -313,9 +314,7 @@ def oracle_sample(cfg, tokens):
 
     w = synth.draw_weights(cfg)
     x, z = synth.draw_activations(cfg.with_(seqlen=tokens), batch_rows=[0])
-    W = {"W_r": w.W_r.astype(np.float64), "W_x": synth.widen(w.W_x, cfg.w_dtype),
-         "W_dt": synth.widen(w.W_dt, cfg.w_dtype), "b_dt": w.b_dt.astype(np.float64), "A": w.A.astype(np.float64),
-         "D_skip": w.D_skip.astype(np.float64)}
+    W = _weights64(cfg, w)
     x64, z64 = synth.widen(x, cfg.io_dtype), synth.widen(z, cfg.io_dtype)
 
     def run():
@@ -324,16 +323,73 @@ def oracle_sample(cfg, tokens):
     return run
 
 
-def time_oracle(cfg, tokens, reps=1):
+def _weights64(cfg, w):
+    return {"W_r": w.W_r.astype(np.float64), "W_x": synth.widen(w.W_x, cfg.w_dtype),
+            "W_dt": synth.widen(w.W_dt, cfg.w_dtype), "b_dt": w.b_dt.astype(np.float64), "A": w.A.astype(np.float64),
+            "D_skip": w.D_skip.astype(np.float64)}
+
+
+# Worker side of the parallel oracle: each process draws the weights once, then runs the oracle's
+# layer on one batch row and one block of channels per task (the recurrence of every (row,
+# channel) is independent; the routing and projections of the row are computed by every task, as
+# the oracle does them).
+_ORACLE = {}
+
+
+def _oracle_init(cfg, tokens):
     from threadpoolctl import threadpool_limits
 
-    run = oracle_sample(cfg, tokens)
-    with threadpool_limits(limits=1):
+    _ORACLE["limits"] = threadpool_limits(limits=1)
+    _ORACLE["cfg"] = cfg.with_(seqlen=tokens)
+    _ORACLE["W"] = _weights64(cfg, synth.draw_weights(cfg))
+    _ORACLE["rows"] = {}
+
+
+def _oracle_task(task):
+    from oracle import swimba_oracle as O
+
+    b, lo, hi = task
+    cfg = _ORACLE["cfg"]
+    rows = _ORACLE["rows"]
+    if b not in rows:
+        x, z = synth.draw_activations(cfg, batch_rows=[b])
+        rows[b] = (synth.widen(x, cfg.io_dtype), synth.widen(z, cfg.io_dtype))
+    x64, z64 = rows[b]
+    t0 = time.perf_counter()
+    O.layer_forward(x64, z64, _ORACLE["W"], cfg.top_k, channels=np.arange(lo, hi))
+    return time.perf_counter() - t0
+
+
+class OraclePool:
+    """The fp64 oracle on every host core: a process pool (started with spawn, so it is safe to
+    create after CUDA is initialised) over (batch row, channel block) tasks of one workload."""
+
+    def __init__(self, cfg, tokens, rows):
+        import multiprocessing as mp
+
+        self.cfg, self.tokens, self.rows = cfg, tokens, rows
+        self.cores = os.cpu_count() or 1
+        blocks = max(1, min(cfg.d_inner // 64, -(-self.cores // len(rows))))
+        edges = [round(i * cfg.d_inner / blocks) for i in range(blocks + 1)]
+        self.tasks = [(b, edges[i], edges[i + 1]) for b in rows for i in range(blocks)]
+        self.procs = min(self.cores, len(self.tasks))
+        self.pool = mp.get_context("spawn").Pool(self.procs, initializer=_oracle_init, initargs=(cfg, tokens))
+        self.pool.map(_oracle_task, self.tasks)  # warm-up: every worker has drawn the rows it serves
+
+    def run(self):
+        """Wall seconds of one pass over every task (all rows, all channels)."""
         t0 = time.perf_counter()
-        for _ in range(reps):
-            run()
-        dt = time.perf_counter() - t0
-    return dt / reps
+        self.pool.map(_oracle_task, self.tasks)
+        return time.perf_counter() - t0
+
+    def sample(self):
+        return (f"batch rows {self.rows[0]}..{self.rows[-1]}, first {self.tokens} of {self.cfg.seqlen} tokens, all "
+                f"{self.cfg.d_inner} channels; fp64 numpy oracle, {len(self.tasks)} (row, channel block) tasks on "
+                f"{self.procs} processes")
+
+    def close(self):
+        self.pool.terminate()
+        self.pool.join()
 
 
 def run_reference(args, cfg):
@@ -341,34 +397,33 @@ def run_reference(args, cfg):
     if rank != 0:
         return 0
     tokens = 256
-    run = oracle_sample(cfg, tokens)
-    from threadpoolctl import threadpool_limits
-
-    with threadpool_limits(limits=1):
+    pool = OraclePool(cfg, tokens, list(range(cfg.batch)))
+    try:
         for _ in range(args.warmup):
-            run()
-        t0 = time.perf_counter()
-        for _ in range(args.steps):
-            run()
-        dt = time.perf_counter() - t0
-    value = tokens * args.steps / dt
-    sample = f"batch row 0, first {tokens} of {cfg.seqlen} tokens, all {cfg.d_inner} channels"
+            pool.run()
+        dt = sum(pool.run() for _ in range(args.steps))
+    finally:
+        pool.close()
+    value = tokens * cfg.batch * args.steps / dt
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_block(cfg),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": pool.procs, "kind": "oracle",
+                         "sample": pool.sample()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
     return 0
 
 
-def config_block(cfg):
-    return {"workload": cfg.name, "batch": cfg.batch, "seqlen": cfg.seqlen, "d_inner": cfg.d_inner,
-            "d_state": cfg.d_state, "dt_rank": cfg.dt_rank, "n_experts": cfg.n_experts, "top_k": cfg.top_k,
-            "io_dtype": cfg.io_dtype, "w_dtype": cfg.w_dtype,
+def config_block(cfg, world=1):
+    return {"workload": cfg.name, "batch": cfg.batch, "global_batch": cfg.batch * world, "seqlen": cfg.seqlen,
+            "d_inner": cfg.d_inner, "d_state": cfg.d_state, "dt_rank": cfg.dt_rank, "n_experts": cfg.n_experts,
+            "top_k": cfg.top_k, "io_dtype": cfg.io_dtype, "w_dtype": cfg.w_dtype,
+            "parallelism": f"dp{world}: the global batch of {cfg.batch * world} sequences sharded {cfg.batch} per "
+                           "rank, no data-path collective",
             "l2": "inputs larger than the 126 MB L2 (x, z 268 MB each), no flush between steps"}
 
 
@@ -425,6 +480,50 @@ def report_workload(torch, S, cfg, peaks, flush, reps, warmup):
         "scan_us": 1e3 * s_ms, "scan_gbs": scan_bytes / (s_ms / 1e3) / 1e9,
         "scan_frac_of_hbm": scan_bytes / (s_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
         "scan_frac_of_mufu": exps / (s_ms / 1e3) / mufu_peak,
+        "median_of": reps, "l2": "flushed (256 MB write) before every run",
+    }
+
+
+def report_separate(torch, S, cfg, peaks, flush, reps, warmup):
+    """Teorema 2 measured: the MoE of separate SSMs (one state trajectory per expert, the k active
+    experts' states advanced per token) against Swimba's single mixed recurrence, on the same
+    tokens and routing. Only the two scans are timed; the separate design's per-slot streams are
+    made once beforehand by swimba_separate_proj."""
+    x, z = synth.draw_activations(cfg)
+    layer = GpuLayer(S, cfg, x, z, "cuda:0")
+    layer.step()
+    d, b, w = layer.dims, layer.buf, layer.ws_struct
+    B, L, D, N, k, E = cfg.batch, cfg.seqlen, cfg.d_inner, cfg.d_state, cfg.top_k, cfg.n_experts
+    f32 = dict(dtype=torch.float32, device="cuda:0")
+    dj = torch.empty((B, L, k, D), **f32)
+    bj = torch.empty((B, L, k, N), **f32)
+    cj = torch.empty((B, L, k, N), **f32)
+    S.check(S.swimba_separate_proj(d, layer.x, b.idx, b.gates, w, dj, bj, cj, layer.stream), "separate_proj")
+    out = torch.empty_like(b.out)
+    hf = torch.empty((E, B, D, N), **f32)
+    wsb = S.new_workspace(d, S.SWIMBA_OP_SEPARATE, "cuda:0")
+    s = layer.stream
+
+    def run(ev):
+        if ev is not None:
+            ev[0].record(s)
+        S.check(S.swimba_scan_fwd(d, layer.x, layer.z, b.delta, b.B_mix, b.C_mix, b.idx, b.gates, w, None, b.out,
+                                  b.h_final, None, b.ws, b.ws.numel(), s), "scan")
+        if ev is not None:
+            ev[1].record(s)
+        S.check(S.swimba_separate_scan(d, layer.x, layer.z, dj, bj, cj, b.idx, b.gates, w, None, out, hf, None, wsb,
+                                       wsb.numel(), s), "separate_scan")
+        if ev is not None:
+            ev[2].record(s)
+
+    (sw_ms, sep_ms), _ = _median_kernel_ms(torch, run, reps, warmup, flush, 3)
+    S.check(S.swimba_get_device_status(wsb, s), "device status")
+    T = cfg.tokens
+    return {
+        "report": "separate_ssm_moe", "workload": cfg.name, "tokens": T, "n_experts": E, "top_k": k,
+        "swimba_scan_us": 1e3 * sw_ms, "separate_scan_us": 1e3 * sep_ms, "separate_over_swimba": sep_ms / sw_ms,
+        "exponentials_per_token": {"swimba": D * N, "separate": k * D * N},
+        "state_bytes_per_sequence": {"swimba": 4 * D * N, "separate": 4 * E * D * N},
         "median_of": reps, "l2": "flushed (256 MB write) before every run",
     }
 
@@ -577,6 +676,9 @@ def run_report(args):
     print(json.dumps(report_block(torch, S, CONFIGS["mamba1p4b_like"], 2048, 4, peaks, flush, reps, args.warmup)),
           flush=True)
     print(json.dumps(report_block_decode(torch, S, CONFIGS["decode_b256"], 2048, 4, peaks, flush, 200)), flush=True)
+    # Theorem 2 against the design it is set against: one trajectory per expert
+    print(json.dumps(report_separate(torch, S, CONFIGS["mamba1p4b_like"], peaks, flush, reps, args.warmup)),
+          flush=True)
     # Theorem 2: the recurrence's cost does not grow with E (k = 2 fixed; E = 1 forces k = 1)
     base = CONFIGS["mamba1p4b_like"]
     for E in (1, 4, 8, 16):
@@ -596,9 +698,20 @@ def main():
         return run_report(args)
     if args.report_block:
         return run_report_block(args)
+    if args.report_separate:
+        import torch
+
+        from parameter_space_moe_swimba_b200 import swimba as S
+
+        torch.cuda.set_device(0)
+        print(json.dumps(report_separate(torch, S, CONFIGS[args.workload], load_peaks(), L2Flush(torch, "cuda:0"), 20,
+                                         args.warmup)), flush=True)
+        return 0
     cfg = CONFIGS[args.workload]
     if args.batch > 0:
         cfg = cfg.with_(batch=args.batch)
+    if args.seqlen > 0:
+        cfg = cfg.with_(seqlen=args.seqlen)
     if args.impl == "reference":
         return run_reference(args, cfg)
 
@@ -617,11 +730,19 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     device = f"cuda:{local}"
     torch.cuda.set_device(local)
+    # the CPU baseline's process pool starts (spawned, warmed up) before the timed GPU work
+    cpu_pool = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu_pool = OraclePool(cfg, 1024, list(range(cfg.batch)))
 
     from parameter_space_moe_swimba_b200 import swimba as S
 
     peaks = load_peaks()
-    x_host, z_host = synth.draw_activations(cfg)
+    # this rank's shard of the global batch (world x batch sequences; sequences are independent)
+    from parameter_space_moe_swimba_b200.parallel import batch_shard
+
+    b0, b1 = batch_shard(cfg.batch * world, world, rank)
+    x_host, z_host = synth.draw_activations(cfg, batch_rows=range(b0, b1))
     layer = GpuLayer(S, cfg, x_host, z_host, device)
 
     clocks = ClockSampler(torch.cuda.current_device())
@@ -674,18 +795,17 @@ def main():
     }
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tok = 1024
-        dt = time_oracle(cfg, tok)
-        cpu = {"value": tok / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"batch row 0, first {tok} of {cfg.seqlen} tokens, all {cfg.d_inner} channels "
-                         f"(fp64 numpy, 1 thread)"}
+    if cpu_pool is not None:
+        dt = cpu_pool.run()
+        cpu = {"value": cpu_pool.tokens * len(cpu_pool.rows) / dt, "unit": UNIT, "cores": cpu_pool.procs,
+               "kind": "oracle", "sample": cpu_pool.sample()}
+        cpu_pool.close()
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_block(cfg),
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_block(cfg, world),
             "roofline": roofline, "alu_roofline": alu_roofline, "kernels": kernels, "switch_vs_dense_e1": dense, "e2e": e2e,
             "gpu_launches": launches, "clocks": clk, "cpu_baseline": cpu,
             "compute": "bf16 x/W on tensor cores with fp32 accumulation; fp32 state and scan arithmetic",

@@ -59,7 +59,9 @@ enum {
   SWIMBA_OP_PROJ = 1,
   SWIMBA_OP_SCAN = 2,
   SWIMBA_OP_STEP = 3,
-  SWIMBA_OP_LAYER = 4 /* large enough for every op of the layer */
+  SWIMBA_OP_LAYER = 4,  /* large enough for every op of the layer */
+  SWIMBA_OP_SUMMARY = 5, /* swimba_scan_summary */
+  SWIMBA_OP_SEPARATE = 6 /* swimba_separate_scan */
 };
 
 typedef struct {
@@ -111,7 +113,9 @@ swimba_status swimba_mixed_proj(const swimba_dims *dims, const void *x, const in
                                 const float *gates, const swimba_weights *w, float *delta,
                                 float *B_mix, float *C_mix, void *ws, size_t ws_bytes, void *stream);
 
-/* The fused discretise + scan + readout + skip + gate over the whole sequence.
+/* The scan's contract on delta: it is the step size itself, delta = softplus(dt_mix), as
+ * swimba_mixed_proj writes it (not the pre-softplus dt_mix), and every value must be finite and
+ * >= 0. The fused discretise + scan + readout + skip + gate over the whole sequence.
  *   x, z [B, L, D] io; delta [B, L, D] fp32; B_mix, C_mix [B, L, N] fp32; idx, gates [B, L, k];
  *   weights: A, D_skip used.
  *   h0      [B, D, N] fp32 starting state, or NULL for zeros            (in)
@@ -126,6 +130,18 @@ swimba_status swimba_scan_fwd(const swimba_dims *dims, const void *x, const void
                               const float *h0, void *out, float *h_final, float *y_pre, void *ws,
                               size_t ws_bytes, void *stream);
 
+/* swimba_scan_fwd with the zero-order-hold injection of "Mamba y las SSMs: el retorno del estado
+ * persistente", section "Mamba" (B-bar = A^-1 (exp(delta A) - I) B) in place of the Euler form
+ * delta B x: with the diagonal mixed transition A_t the state update is
+ *   h_t = exp(delta_t A_t) * h_{t-1} + (exp(delta_t A_t) - 1) / A_t * B_mix,t x_t.
+ * Arguments, workspace and outputs as swimba_scan_fwd. Each state element costs one more
+ * special-function operation (a reciprocal) than the Euler scan. */
+swimba_status swimba_scan_fwd_zoh(const swimba_dims *dims, const void *x, const void *z,
+                                  const float *delta, const float *B_mix, const float *C_mix,
+                                  const int32_t *idx, const float *gates, const swimba_weights *w,
+                                  const float *h0, void *out, float *h_final, float *y_pre, void *ws,
+                                  size_t ws_bytes, void *stream);
+
 /* swimba_scan_fwd without a caller workspace, for callers that cannot allocate device memory: a
  * plugin inside a framework that owns all device memory and gives it no allocator, or a
  * latency-critical loop that must not call cudaMalloc (which can synchronise the device). The pages
@@ -137,13 +153,84 @@ swimba_status swimba_scan_fwd(const swimba_dims *dims, const void *x, const void
  *   The first call on a device looks up the array's device address (cudaGetSymbolAddress, once per
  *   device, with that device current); make that first call before any stream capture.
  *   Every call shares the one array and overwrites what the last call left there; calls that may
- *   overlap on the GPU (other streams, other threads) race and must not be issued. Device-side
- *   status of this variant is cleared at every call and is not reported. */
+ *   overlap on the GPU (other streams, other threads) race and must not be issued. The status
+ *   block at the start of the array is cleared at every call; a bounded device-side wait that gave
+ *   up during the call is recorded there and read by swimba_scan_fwd_noalloc_status. */
 swimba_status swimba_scan_fwd_noalloc(const swimba_dims *dims, const void *x, const void *z,
                                       const float *delta, const float *B_mix, const float *C_mix,
                                       const int32_t *idx, const float *gates, const swimba_weights *w,
                                       const float *h0, void *out, float *h_final, float *y_pre,
                                       void *stream);
+
+/* Device status of the last swimba_scan_fwd_noalloc call on the current device: synchronises
+ * `stream`, returns SWIMBA_OK or SWIMBA_ERR_TIMEOUT (a bounded wait that gave up; out, h_final and
+ * y_pre are then incomplete) from the fixed array's status block, and clears it. */
+swimba_status swimba_scan_fwd_noalloc_status(void *stream);
+
+/* Device address of that status block on the current device (NULL if the lookup failed): the
+ * 256-byte block swimba_get_device_status and swimba_check_wait_timeout accept as `ws`. */
+void *swimba_scan_fwd_noalloc_status_block(void);
+
+/* ---- Splitting a long sequence into pieces ---------------------------------------------------
+ * ("Mamba y las SSMs: el retorno del estado persistente", "Estado interno puramente lineal": the
+ * state is linear, so the recurrence can be cut and recombined.) Over a piece of tokens the state
+ * after the piece is exp(sum_t delta_t A_t) * h_in + h_zero, h_zero being the end state when the
+ * piece starts from zero. A sequence cut into P consecutive pieces (e.g. one per GPU) is scanned
+ * by: swimba_scan_summary on every piece, an exchange of the summaries, swimba_scan_chain for the
+ * start states, then swimba_scan_fwd on every piece from its start state (h0).
+ *
+ * Summary of the pieces given as the B sequences of `dims` (each its own piece):
+ *   x [B, L, D] io; delta [B, L, D] fp32; B_mix [B, L, N] fp32; idx, gates [B, L, k]; weights: A.
+ *   h_zero    [B, D, N] fp32 (out) end state of the recurrence started from zero
+ *   log_decay [B, D, N] fp32 (out) sum over the piece's tokens of delta_t A_t (natural log)
+ *   ws: at least swimba_workspace_size(dims, SWIMBA_OP_SUMMARY) bytes. */
+swimba_status swimba_scan_summary(const swimba_dims *dims, const void *x, const float *delta,
+                                  const float *B_mix, const int32_t *idx, const float *gates,
+                                  const swimba_weights *w, float *h_zero, float *log_decay, void *ws,
+                                  size_t ws_bytes, void *stream);
+
+/* Start states of `parts` consecutive pieces from their summaries (dims: batch, d_inner and
+ * d_state are used):
+ *   h_zero, log_decay [parts, B, D, N] fp32 (in), piece 0 first
+ *   h0      [B, D, N] fp32 state before piece 0, or NULL for zeros   (in)
+ *   h_start [parts + 1, B, D, N] fp32 (out): h_start[0] = h0, h_start[p+1] =
+ *           exp(log_decay[p]) * h_start[p] + h_zero[p]; h_start[parts] is the state after the
+ *           whole sequence. */
+swimba_status swimba_scan_chain(const swimba_dims *dims, int32_t parts, const float *h_zero,
+                                const float *log_decay, const float *h0, float *h_start, void *stream);
+
+/* ---- The MoE of separate SSMs (the design Swimba is set against) ----------------------------
+ * ("Swimba: Switch Mamba Model Scales State Space Models", Spanish summary §2 "Distinción de
+ * Diseños", Dutch "Methodologie", French "Distinction des deux designs MoE-SSM"; Teorema 2.) Every
+ * expert keeps its own state trajectory h^(e) [B, D, N] and its own recurrence; at token t the k
+ * active experts advance their states with their own unmixed streams and transition,
+ *   h^(e_j) = exp(delta^j A^{e_j}) * h^(e_j) + delta^j B^j x_t   (delta^j = softplus(dt^j)),
+ * the other experts' states stay as they are, and y_t = sum_j g_j C^j . h^(e_j) + D_skip * x_t,
+ * out_t = y_t * SiLU(z_t). Built as the measured comparison for Teorema 2; the recurrence work
+ * grows with k (Swimba's does not).
+ *
+ * Per-slot streams (SIMT, one CTA per token; weights W_x, W_dt, b_dt):
+ *   delta_j [B, L, k, D] fp32 (out) = softplus(x W_x^{e_j}[:, :R] W_dt^{e_j} + b_dt^{e_j})
+ *   B_j, C_j [B, L, k, N] fp32 (out) = the slot's B and C columns of x W_x^{e_j}, unmixed */
+swimba_status swimba_separate_proj(const swimba_dims *dims, const void *x, const int32_t *idx,
+                                   const float *gates, const swimba_weights *w, float *delta_j,
+                                   float *B_j, float *C_j, void *stream);
+
+/* The separate-SSM scan over whole sequences.
+ *   x, z [B, L, D] io; delta_j [B, L, k, D]; B_j, C_j [B, L, k, N]; idx, gates [B, L, k];
+ *   weights: A, D_skip used.
+ *   h0      [E, B, D, N] fp32 every expert's start state, or NULL for zeros   (in)
+ *   out     [B, L, D] io                                                         (out)
+ *   h_final [E, B, D, N] fp32 every expert's state after the last token, or NULL (out)
+ *   y_pre   [B, L, D] fp32 or NULL                                              (out)
+ *   ws: at least swimba_workspace_size(dims, SWIMBA_OP_SEPARATE) bytes (the status block).
+ * bf16 io with N = 16, k <= 2, E <= 8 and D % 16 == 0 keeps every expert's A rows and state in
+ * tensor memory; other shapes run a per-channel SIMT kernel. */
+swimba_status swimba_separate_scan(const swimba_dims *dims, const void *x, const void *z,
+                                   const float *delta_j, const float *B_j, const float *C_j,
+                                   const int32_t *idx, const float *gates, const swimba_weights *w,
+                                   const float *h0, void *out, float *h_final, float *y_pre, void *ws,
+                                   size_t ws_bytes, void *stream);
 
 /* One decode step (dims->seqlen must be 1): the scan for a single token per sequence, continuing
  * from and overwriting the cached state h [B, D, N] fp32. Other arguments as swimba_scan_fwd. */

@@ -17,6 +17,12 @@ cudaError_t run_proj_simt(const ProjParams& p, bool io_bf16, bool w_bf16, cudaSt
 bool proj_tc_supported(const ProjParams& p, bool io_bf16, bool w_bf16);
 size_t proj_tc_workspace(int64_t T, int E, int k, int R, int D);
 cudaError_t run_proj_tc(const ProjParams& p, void* ws, cudaStream_t s);
+cudaError_t run_separate_proj(const ProjParams& p, bool io_bf16, bool w_bf16, float* dj, float* bj, float* cj,
+                              cudaStream_t s);
+cudaError_t separate_scan_entry(const void* x, const void* z, const float* dj, const float* bj, const float* cj,
+                                const int32_t* idx, const float* gates, const float* A, const float* D_skip,
+                                const float* h0, void* out, float* h_final, float* y_pre, void* status, int64_t L,
+                                int B, int D, int N, int E, int k, bool io_bf16, cudaStream_t s);
 }  // namespace swimba
 
 namespace swimba {
@@ -85,6 +91,11 @@ size_t scan_workspace(const swimba_dims* d) {
   return kStatusBytes + (pl.fast ? pl.ws_bytes : 0);
 }
 
+size_t summary_workspace(const swimba_dims* d) {
+  const ScanPlan pl = scan_plan(d);
+  return kStatusBytes + (pl.fast ? scan_fast_summary_ws(pl, d->batch, d->d_inner) : 0);
+}
+
 }  // namespace
 
 namespace swimba {
@@ -126,6 +137,10 @@ size_t swimba_workspace_size(const swimba_dims* dims, int op) {
       return proj_workspace(dims);
     case SWIMBA_OP_LAYER:
       return std::max(proj_workspace(dims), scan_workspace(dims));
+    case SWIMBA_OP_SUMMARY:
+      return summary_workspace(dims);
+    case SWIMBA_OP_SEPARATE:
+      return kStatusBytes;
     default:
       return 0;
   }
@@ -166,7 +181,7 @@ swimba_status swimba_mixed_proj(const swimba_dims* dims, const void* x, const in
 static swimba_status scan_common(const swimba_dims* dims, const void* x, const void* z, const float* delta,
                                  const float* B_mix, const float* C_mix, const int32_t* idx, const float* gates,
                                  const swimba_weights* w, const float* h0, void* out, float* h_final, float* y_pre,
-                                 bool step, void* ws, void* stream) {
+                                 bool step, void* ws, void* stream, bool zoh = false) {
   if (!x || !z || !delta || !B_mix || !C_mix || !idx || !gates || !w || !w->A || !w->D_skip || !out)
     return SWIMBA_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(z) || !aligned16(out) || !aligned16(delta)) return SWIMBA_ERR_ALIGN;
@@ -177,6 +192,7 @@ static swimba_status scan_common(const swimba_dims* dims, const void* x, const v
   ScanParams p{x,   z,       delta, B_mix,          C_mix,          idx,           gates,
                w->A, w->D_skip, h0,  out,            h_final,        y_pre,         dims->seqlen,
                (int)dims->batch, dims->d_inner, dims->d_state, dims->n_experts, dims->top_k};
+  p.zoh = zoh ? 1 : 0;
   if (!step) {
     const ScanPlan pl = scan_plan(dims);
     if (pl.fast) {
@@ -198,6 +214,18 @@ swimba_status swimba_scan_fwd(const swimba_dims* dims, const void* x, const void
   return scan_common(dims, x, z, delta, B_mix, C_mix, idx, gates, w, h0, out, h_final, y_pre, false, ws, stream);
 }
 
+swimba_status swimba_scan_fwd_zoh(const swimba_dims* dims, const void* x, const void* z, const float* delta,
+                                  const float* B_mix, const float* C_mix, const int32_t* idx, const float* gates,
+                                  const swimba_weights* w, const float* h0, void* out, float* h_final, float* y_pre,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  swimba_status st = check_dims(dims);
+  if (st != SWIMBA_OK) return st;
+  if (ws == nullptr || ws_bytes < swimba_workspace_size(dims, SWIMBA_OP_SCAN)) return SWIMBA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SWIMBA_ERR_ALIGN;
+  return scan_common(dims, x, z, delta, B_mix, C_mix, idx, gates, w, h0, out, h_final, y_pre, false, ws, stream,
+                     true);
+}
+
 swimba_status swimba_scan_fwd_noalloc(const swimba_dims* dims, const void* x, const void* z, const float* delta,
                                       const float* B_mix, const float* C_mix, const int32_t* idx, const float* gates,
                                       const swimba_weights* w, const float* h0, void* out, float* h_final,
@@ -216,6 +244,83 @@ swimba_status swimba_scan_fwd_noalloc(const swimba_dims* dims, const void* x, co
   if (cuda_status(cudaMemsetAsync(scratch, 0, kStatusBytes, static_cast<cudaStream_t>(stream))) != SWIMBA_OK)
     return SWIMBA_ERR_CUDA;
   return scan_common(dims, x, z, delta, B_mix, C_mix, idx, gates, w, h0, out, h_final, y_pre, false, scratch, stream);
+}
+
+swimba_status swimba_scan_fwd_noalloc_status(void* stream) {
+  void* scratch = nullptr;
+  if (cuda_status(scan_noalloc_scratch(&scratch)) != SWIMBA_OK) return SWIMBA_ERR_CUDA;
+  return swimba_get_device_status(scratch, stream);
+}
+
+void* swimba_scan_fwd_noalloc_status_block(void) {
+  void* scratch = nullptr;
+  return scan_noalloc_scratch(&scratch) == cudaSuccess ? scratch : nullptr;
+}
+
+swimba_status swimba_scan_summary(const swimba_dims* dims, const void* x, const float* delta, const float* B_mix,
+                                  const int32_t* idx, const float* gates, const swimba_weights* w, float* h_zero,
+                                  float* log_decay, void* ws, size_t ws_bytes, void* stream) {
+  swimba_status st = check_dims(dims);
+  if (st != SWIMBA_OK) return st;
+  if (!x || !delta || !B_mix || !idx || !gates || !w || !w->A || !h_zero || !log_decay) return SWIMBA_ERR_INVALID_ARG;
+  if (ws == nullptr || ws_bytes < swimba_workspace_size(dims, SWIMBA_OP_SUMMARY)) return SWIMBA_ERR_WORKSPACE;
+  if (!aligned16(ws) || !aligned16(x) || !aligned16(delta) || !aligned16(w->A) || !aligned16(h_zero) ||
+      !aligned16(log_decay))
+    return SWIMBA_ERR_ALIGN;
+  if (dims->d_state == 16 && !aligned16(B_mix)) return SWIMBA_ERR_ALIGN;
+  ScanParams p{x,       nullptr,  delta,   B_mix,  nullptr, idx,          gates,           w->A,
+               nullptr, nullptr,  nullptr, nullptr, nullptr, dims->seqlen, (int)dims->batch, dims->d_inner,
+               dims->d_state, dims->n_experts, dims->top_k};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const ScanPlan pl = scan_plan(dims);
+  if (pl.fast) {
+    uint8_t* seg_ws = reinterpret_cast<uint8_t*>(ws) + kStatusBytes;
+    return cuda_status(run_scan_summary_fast(p, pl, seg_ws, ws, h_zero, log_decay, s));
+  }
+  return cuda_status(run_scan_summary(p, dims->io_dtype == SWIMBA_BF16, h_zero, log_decay, s));
+}
+
+swimba_status swimba_scan_chain(const swimba_dims* dims, int32_t parts, const float* h_zero, const float* log_decay,
+                                const float* h0, float* h_start, void* stream) {
+  if (dims == nullptr || dims->batch <= 0 || dims->d_inner <= 0 || dims->d_state <= 0 || parts <= 0)
+    return SWIMBA_ERR_INVALID_ARG;
+  if (!h_zero || !log_decay || !h_start) return SWIMBA_ERR_INVALID_ARG;
+  const int64_t bdn = dims->batch * (int64_t)dims->d_inner * dims->d_state;
+  if (bdn > (int64_t(1) << 40) || parts > (1 << 20)) return SWIMBA_ERR_UNSUPPORTED;
+  return cuda_status(run_scan_chain(bdn, parts, h_zero, log_decay, h0, h_start, static_cast<cudaStream_t>(stream)));
+}
+
+swimba_status swimba_separate_proj(const swimba_dims* dims, const void* x, const int32_t* idx, const float* gates,
+                                   const swimba_weights* w, float* delta_j, float* B_j, float* C_j, void* stream) {
+  swimba_status st = check_dims(dims);
+  if (st != SWIMBA_OK) return st;
+  if (!x || !idx || !gates || !w || !w->W_x || !w->W_dt || !w->b_dt || !delta_j || !B_j || !C_j)
+    return SWIMBA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(delta_j) || !aligned16(w->W_x) || !aligned16(w->W_dt)) return SWIMBA_ERR_ALIGN;
+  ProjParams p{x,       idx,     gates, w->W_x, w->W_dt, w->b_dt, nullptr, nullptr, nullptr, dims->batch * dims->seqlen,
+               dims->d_inner, dims->d_state, dims->dt_rank, dims->n_experts, dims->top_k};
+  return cuda_status(run_separate_proj(p, dims->io_dtype == SWIMBA_BF16, dims->w_dtype == SWIMBA_BF16, delta_j, B_j,
+                                       C_j, static_cast<cudaStream_t>(stream)));
+}
+
+swimba_status swimba_separate_scan(const swimba_dims* dims, const void* x, const void* z, const float* delta_j,
+                                   const float* B_j, const float* C_j, const int32_t* idx, const float* gates,
+                                   const swimba_weights* w, const float* h0, void* out, float* h_final, float* y_pre,
+                                   void* ws, size_t ws_bytes, void* stream) {
+  swimba_status st = check_dims(dims);
+  if (st != SWIMBA_OK) return st;
+  if (!x || !z || !delta_j || !B_j || !C_j || !idx || !gates || !w || !w->A || !w->D_skip || !out)
+    return SWIMBA_ERR_INVALID_ARG;
+  if (ws == nullptr || ws_bytes < kStatusBytes) return SWIMBA_ERR_WORKSPACE;
+  if (!aligned16(ws) || !aligned16(x) || !aligned16(z) || !aligned16(out) || !aligned16(delta_j) ||
+      !aligned16(B_j) || !aligned16(C_j) || !aligned16(w->A) || !aligned16(w->D_skip))
+    return SWIMBA_ERR_ALIGN;
+  if ((h0 && !aligned16(h0)) || (h_final && !aligned16(h_final)) || (y_pre && !aligned16(y_pre)))
+    return SWIMBA_ERR_ALIGN;
+  return cuda_status(separate_scan_entry(x, z, delta_j, B_j, C_j, idx, gates, w->A, w->D_skip, h0, out, h_final,
+                                         y_pre, ws, dims->seqlen, (int)dims->batch, dims->d_inner, dims->d_state,
+                                         dims->n_experts, dims->top_k, dims->io_dtype == SWIMBA_BF16,
+                                         static_cast<cudaStream_t>(stream)));
 }
 
 swimba_status swimba_step(const swimba_dims* dims, const void* x, const void* z, const float* delta,

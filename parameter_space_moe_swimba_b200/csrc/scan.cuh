@@ -21,6 +21,7 @@ struct ScanParams {
   float* y_pre;          // [B, L, D] or null
   int64_t L;
   int B, D, N, E, k;
+  int zoh = 0;           // 1: zero-order-hold injection instead of Euler's
 };
 
 cudaError_t run_scan(const ScanParams& p, bool io_bf16, bool step, cudaStream_t s);
@@ -35,6 +36,19 @@ struct ScanPlan {
 };
 ScanPlan scan_fast_plan(int64_t B, int64_t L, int D, int N, int E, int k, bool io_bf16);
 cudaError_t run_scan_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s);
+
+// Summary of a whole sequence (the hand-off of one piece of a longer one): h_zero [B, D, N] = the
+// end state from zero, log_decay [B, D, N] = Σ_t Δ_t A_t. The fast path stages per-segment
+// aggregates in scan_fast_summary_ws bytes of workspace; the generic path needs none.
+size_t scan_fast_summary_ws(const ScanPlan& pl, int64_t B, int D);
+cudaError_t run_scan_summary_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, float* h_zero,
+                                  float* log_decay, cudaStream_t s);
+cudaError_t run_scan_summary(const ScanParams& p, bool io_bf16, float* h_zero, float* log_decay, cudaStream_t s);
+
+// Start states of P consecutive pieces from their summaries: h_start[0] = h0 (or zeros),
+// h_start[p+1] = exp(log_decay[p]) h_start[p] + h_zero[p]; arrays [P(+1), B, D, N].
+cudaError_t run_scan_chain(int64_t BDN, int P, const float* h_zero, const float* log_decay, const float* h0,
+                           float* h_start, cudaStream_t s);
 
 // Fixed device scratch used by swimba_scan_fwd_noalloc (status block + segment carries).
 constexpr size_t kScanNoAllocScratchBytes = size_t(8) << 20;

@@ -6,28 +6,35 @@
 // Figura 2: the state stays on chip, inputs stream from HBM) and "Estado interno puramente lineal"
 // (the linear state admits a scan, used here to split long sequences into segments).
 //
-// Work unit = one warp = 32 channels of one sequence segment. Lane l holds the channel pair
-// (2*(l>>1), 2*(l>>1)+1) of the warp and the 8 states (l&1)*8 .. +7 of both channels, 16 fp32 states
-// in registers; the two lanes of a pair together hold all 16 states of the two channels. So every
-// B_mix / C_mix value a lane loads serves two channels.
-// The per-expert transition rows (pre-multiplied by log2 e) live in tensor memory: each warp owns
-// E*16 TMEM columns of its lane quarter and keeps expert e's 16 values of every lane at columns
-// 16e..16e+15. Every lane of a warp reads the same token, so the selected expert is warp-uniform
-// and one tcgen05.ld.32x32b.x16 at column 16e fetches it: a dynamically indexed, branch-free lookup
-// that costs no registers and no shared-memory bandwidth.
 // Per token and state:  arg = Σ_j (Δ g_j) A^{e_j};  ā = 2^arg;  h = ā h + (Δ x) B;  y += C h.
+// At N = 16 every (token, channel) costs 16 exponentials and ~80 FP32 operations against 10 bytes
+// of HBM traffic, so the kernel is bound by the special-function unit and by instruction issue, not
+// by HBM. The design therefore aims at the issue rate: as many resident warps as the SM holds
+// (16, at <= 128 registers), the fewest instructions per state element, and packed f32x2 math.
 //
-// A chunk of 16 tokens runs in two passes. The recurrence pass keeps only the state chain: each
-// lane leaves its two partial readouts per token in shared memory. The readout pass then works on
-// the whole chunk at once, with a different lane layout: lane l takes token l/2 and 16 channels,
-// adds the two state halves' partials, the skip term D_skip x and the gate z σ(z) (σ via
-// tanh.approx) with packed f32x2 arithmetic and 16-byte shared-memory loads, and writes 16 bf16
-// outputs; one TMA store per chunk moves the [16 x 32] output tile to HBM (it clips rows past L).
+// Work unit = one warp = 16 channels of one sequence segment. Lane l holds the channel pair
+// (2*(l>>2), 2*(l>>2)+1) and the 4 states 4*(l&3) .. +3 of both channels: state register s is the
+// float2 (h[c0][s], h[c1][s]), so every packed operation works on the two channels at once and the
+// readout Σ_s C[s] h[s] comes out as the float2 of the two channels' partial sums. B_mix / C_mix
+// loads are one 16-byte broadcast per token (8 lanes share each quarter).
+// The per-expert transition rows (pre-multiplied by log2 e) live in tensor memory: each warp owns a
+// window of its lane quarter, expert e at columns 8e..8e+7 holding (A[c0][s], A[c1][s]) for s = 0..3.
+// Every lane of a warp reads the same token, so the selected expert is warp-uniform and one
+// tcgen05.ld.32x32b.x8 at column 8e fetches the lane's 8 values: a dynamically indexed, branch-free
+// lookup that costs no registers and no shared-memory bandwidth.
 //
-// Each warp streams its inputs through its own 3-stage shared-memory ring filled by TMA (x, z, Δ
-// tiles of [16 tokens x 32 channels] and B_mix, C_mix rows of 16 tokens) plus the tokens' expert
-// indices and gates written by the warp's lanes one chunk ahead. Units are spread evenly over one
-// persistent CTA per SM, so no SM gets a whole extra sequence.
+// A chunk of 16 tokens runs in two passes. The recurrence pass keeps only the state chain; each
+// lane leaves its float2 partial readout per token in shared memory. The readout pass then changes
+// the lane layout: lane l takes token l/2 and 8 channels, adds the four state quarters' partials,
+// the skip term D_skip x and the gate z σ(z) = hz + hz tanh(hz) (hz = z/2), and writes 8 bf16
+// outputs; one TMA store per chunk moves the warp's [16 x 16] output tile to HBM (it clips rows
+// past L).
+//
+// Each warp streams its inputs through its own 2-stage ring filled by TMA (x, z, Δ tiles of
+// [16 tokens x 16 channels], the tokens' B_mix and C_mix rows) plus the tokens' expert columns and
+// gates, which the lanes load one chunk ahead and write into the stage. A chunk's
+// compute takes several microseconds, so one chunk in flight hides the HBM latency. Units are
+// spread evenly over one persistent CTA per SM.
 //
 // Segments (when B*D alone cannot fill the GPU): pass 1 computes, per segment, the end state from
 // zero and log2 of the decay product Σ_t Δ_t A_t; a carry pass chains them into each segment's
@@ -41,68 +48,83 @@
 #include "scan.cuh"
 #include "sm100.cuh"
 
+// Tuning knobs, fixed at build time: the warps per SM the segment plan aims at, the warp count per
+// SM below which a sequence is split into segments, and how many of a lane's 8 exponentials per
+// token run as a polynomial on the FMA pipe instead of the special-function unit.
+#ifndef SWIMBA_SCAN_TARGET_WARPS
+#define SWIMBA_SCAN_TARGET_WARPS 14
+#endif
+#ifndef SWIMBA_SCAN_MIN_WARPS
+#define SWIMBA_SCAN_MIN_WARPS 8
+#endif
+#ifndef SWIMBA_SCAN_NPOLY
+#define SWIMBA_SCAN_NPOLY 0
+#endif
+// 1: with E <= 8 experts, keep the transition rows in registers instead of tensor memory.
+#ifndef SWIMBA_SCAN_AREG
+#define SWIMBA_SCAN_AREG 0
+#endif
+
 namespace swimba {
 
 using namespace sm100;
 
 namespace {
 
-constexpr int LC = 16;          // tokens per chunk
-constexpr int kStages = 3;      // ring depth per warp
-constexpr int kCPW = 32;        // channels per warp
-constexpr int kNS = 8;          // states per lane and channel
-constexpr int kNP = kNS / 2;    // float2 state pairs per lane and channel
-constexpr int kACols = 16;      // TMEM columns per expert (both channels of a lane)
-constexpr int kMaxWarps = 8;    // warps per CTA (registers: up to 255 per thread)
-constexpr int kPRow = kCPW + 4; // floats per row of the partial-readout buffer (padded)
+constexpr int LC = 16;            // tokens per chunk
+constexpr int kStages = 2;        // ring depth per warp
+constexpr int kCPW = 16;          // channels per warp
+constexpr int kSPL = 4;           // states per lane and channel
+constexpr int kMaxWarps = 16;     // warps per CTA (128 registers per thread)
+constexpr int kPRow = 4 * kCPW + 4;  // floats per token row of the partial-readout buffer (padded)
+constexpr int kNPoly = SWIMBA_SCAN_NPOLY;
+static_assert(kNPoly >= 0 && kNPoly <= 8, "exponentials per lane and token");
 
-// Byte offsets inside one ring stage of one warp.
+// Byte offsets inside one ring stage of one warp (TMA destinations, 128-byte aligned).
 struct Stage {
-  static constexpr int X = 0;                      // bf16 [LC][32]
-  static constexpr int Z = X + LC * kCPW * 2;      // bf16 [LC][32]
-  static constexpr int DL = Z + LC * kCPW * 2;     // f32  [LC][32]
-  static constexpr int B = DL + LC * kCPW * 4;     // f32  [LC][16]
-  static constexpr int C = B + LC * 16 * 4;        // f32  [LC][16]
-  static constexpr int META = C + LC * 16 * 4;     // int4 [LC] {e0, e1, g0, g1}
+  static constexpr int X = 0;                    // bf16 [LC][16]
+  static constexpr int Z = X + LC * kCPW * 2;    // bf16 [LC][16]
+  static constexpr int DL = Z + LC * kCPW * 2;   // f32  [LC][16]
+  static constexpr int B = DL + LC * kCPW * 4;   // f32  [LC][16]
+  static constexpr int C = B + LC * 16 * 4;      // f32  [LC][16]
+  static constexpr int META = C + LC * 16 * 4;   // int4 [LC] {TMEM column of e0, of e1, g0, g1}
   static constexpr int BYTES = META + LC * 16;
-  static_assert(X % 128 == 0 && Z % 128 == 0 && DL % 128 == 0 && B % 128 == 0 && C % 128 == 0 && META % 128 == 0,
+  static_assert(X % 128 == 0 && Z % 128 == 0 && DL % 128 == 0 && B % 128 == 0 && C % 128 == 0 && META % 128 == 0 &&
+                    BYTES % 128 == 0,
                 "TMA destinations must be 128-byte aligned");
-  static_assert(BYTES % 128 == 0, "stage size");
 };
 
-// Per-warp readout area (after the ring): partial readouts, two output tiles (the TMA store of
-// one may still be reading while the next is written), the warp's D_skip values.
+// Per-warp area after the rings: partial readouts and two output tiles (the TMA store of one may
+// still be reading while the next is written).
 struct Epi {
-  static constexpr int P = 0;                              // f32 [LC][2 state halves][kPRow]
-  static constexpr int O = P + LC * 2 * kPRow * 4;         // bf16 [2][LC][32]
-  static constexpr int DS = O + 2 * LC * kCPW * 2;         // f32 [32]
-  static constexpr int BYTES = DS + kCPW * 4;
-  static_assert(O % 128 == 0 && DS % 16 == 0 && BYTES % 128 == 0, "readout area layout");
+  static constexpr int P = 0;                        // f32 [LC][kPRow]: [token][state quarter][16 channels]
+  static constexpr int O = P + LC * kPRow * 4;       // bf16 [2][LC][16]
+  static constexpr int BYTES = O + 2 * LC * kCPW * 2;
+  static_assert(O % 128 == 0 && BYTES % 128 == 0, "readout area layout");
 };
 
-// TMEM columns one warp needs (16 per expert, rounded up to the 32-column allocation granule).
-__host__ __device__ constexpr int tmem_cols_per_warp(int E) { return ((E * kACols + 31) / 32) * 32; }
+constexpr int kWarpBytes = kStages * Stage::BYTES + Epi::BYTES;
+
+// TMEM columns one warp needs (8 per expert, rounded up to the 32-column allocation granule).
+__host__ __device__ constexpr int tmem_cols_per_warp(int E) { return ((E * 8 + 31) / 32) * 32; }
 
 // 2^x on the FMA pipe for x <= 0: x = j + f with j = round(x) (the 1.5*2^23 shifter), f in
 // [-1/2, 1/2]; 2^f by a degree-5 polynomial fitted for minimax relative error on that interval
 // (fit_exp2_poly.py beside this file: float32 Horner error 2.4e-7, the size of ex2.approx's);
 // the exponent j is added to the result's exponent field. Inputs below -125 are clamped (result
 // 2^-125 instead of a flushed 0, which no decay product here can tell apart).
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  const float2 lo = make_float2(-125.f, -125.f);
-  x = make_float2(fmaxf(x.x, lo.x), fmaxf(x.y, lo.y));
-  const float2 shifter = make_float2(12582912.f, 12582912.f);
-  const float2 t = __fadd2_rn(x, shifter);
-  const float2 j = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = __fadd2_rn(x, make_float2(-j.x, -j.y));
-  float2 p = make_float2(0x1.5c08e6p-10f, 0x1.5c08e6p-10f);
-  p = __ffma2_rn(p, f, make_float2(0x1.3d0c52p-7f, 0x1.3d0c52p-7f));
-  p = __ffma2_rn(p, f, make_float2(0x1.c6b6e4p-5f, 0x1.c6b6e4p-5f));
-  p = __ffma2_rn(p, f, make_float2(0x1.ebf918p-3f, 0x1.ebf918p-3f));
-  p = __ffma2_rn(p, f, make_float2(0x1.62e428p-1f, 0x1.62e428p-1f));
-  p = __ffma2_rn(p, f, make_float2(0x1.000002p+0f, 0x1.000002p+0f));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = __fadd_rn(x, 12582912.f);
+  const float j = __fadd_rn(t, -12582912.f);
+  const float f = __fadd_rn(x, -j);
+  float p = 0x1.5c08e6p-10f;
+  p = __fmaf_rn(p, f, 0x1.3d0c52p-7f);
+  p = __fmaf_rn(p, f, 0x1.c6b6e4p-5f);
+  p = __fmaf_rn(p, f, 0x1.ebf918p-3f);
+  p = __fmaf_rn(p, f, 0x1.62e428p-1f);
+  p = __fmaf_rn(p, f, 0x1.000002p+0f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ float tanh_approx(float x) {
@@ -113,10 +135,10 @@ __device__ __forceinline__ float tanh_approx(float x) {
 
 // 8 bf16 (one 16-byte word) as 4 float2 pairs.
 __device__ __forceinline__ void bf16x8_to_float2(const uint4 q, float2 (&f)[4]) {
-  f[0] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
-  f[1] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
-  f[2] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.z));
-  f[3] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.w));
+  f[0] = make_float2(bf16lo(q.x), bf16hi(q.x));
+  f[1] = make_float2(bf16lo(q.y), bf16hi(q.y));
+  f[2] = make_float2(bf16lo(q.z), bf16hi(q.z));
+  f[3] = make_float2(bf16lo(q.w), bf16hi(q.w));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float2 v) {
@@ -124,21 +146,47 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float2 v) {
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
-// One token's scan inputs as the recurrence pass holds them (lane view: channels 2cp, 2cp+1,
-// states 8gi .. 8gi+7).
+__device__ __forceinline__ float2 f2(float v) { return make_float2(v, v); }
+
+// arg[s] (+)= dg * A^e[s] for the lane's 4 state pairs, with the E <= 8 experts' rows held in
+// registers: the expert is warp-uniform, so the switch is one uniform indexed branch, and every case
+// reads its own registers (a dynamically indexed register array would live in local memory).
+template <bool ACC>
+__device__ __forceinline__ void mix_areg(const float2 (&ar)[8][4], int e, float2 dg, float2 (&arg)[4]) {
+#define SWIMBA_MIX_CASE(c)                                                                   \
+  case c:                                                                                    \
+    _Pragma("unroll") for (int s = 0; s < 4; ++s) arg[s] =                                    \
+        ACC ? __ffma2_rn(dg, ar[c][s], arg[s]) : __fmul2_rn(dg, ar[c][s]);                     \
+    break;
+  switch (e) {
+    SWIMBA_MIX_CASE(0)
+    SWIMBA_MIX_CASE(1)
+    SWIMBA_MIX_CASE(2)
+    SWIMBA_MIX_CASE(3)
+    SWIMBA_MIX_CASE(4)
+    SWIMBA_MIX_CASE(5)
+    SWIMBA_MIX_CASE(6)
+    default:
+      SWIMBA_MIX_CASE(7)
+  }
+#undef SWIMBA_MIX_CASE
+}
+
+// One token's scan inputs as the recurrence pass holds them (lane view: channels c0, c1 as the two
+// halves of every float2; states 4q .. 4q+3).
 struct TokIn {
-  int4 m;              // {e0, e1, g0, g1}
-  uint32_t ar[2][16];  // A rows of the selected experts (x log2 e), from TMEM
-  float2 dl, xv;       // Δ and x of the two channels
-  float2 bv[4], cv[4]; // B_mix, C_mix of the lane's 8 states
-  float dx[2];         // Δ x per channel
-  float2 arg[2][4];    // Σ_j (Δ g_j) A^{e_j}  [channel][state pair]
-  float2 a[2][4];      // 2^arg
+  int4 m;             // {TMEM column of e0, of e1, g0, g1}
+  uint32_t ar[2][8];  // A rows of the selected experts (x log2 e), from TMEM: (c0, c1) per state
+  float2 dl, xv;      // Δ and x of the two channels
+  float4 bq, cq;      // B_mix, C_mix of the lane's 4 states
+  float2 dx;          // Δ x
+  float2 a[kSPL];     // 2^arg per state, both channels
+  float2 phi[kSPL];   // zero-order-hold factor per state (ZOH only)
 };
 
 struct FastParams {
-  const int32_t* idx;
-  const float* gates;
+  const int32_t* idx;   // [B, L, k]
+  const float* gates;   // [B, L, k]
   const float* A;       // [E, D, 16]
   const float* D_skip;  // [D]
   const float* h0;      // [B, D, 16] or null (start state of segment 0)
@@ -149,32 +197,33 @@ struct FastParams {
   float* agg_logp;      // pass 1: [B, S, D, 16] log2 of the decay product
   void* status;
   int64_t L, Lseg;
-  int B, D, E, k, S;
+  int B, D, E, S;
   int seg_count;        // segments this pass visits (S, or S - 1 for pass 1)
-  int units;            // B * seg_count * (D / 32)
+  int units;            // B * seg_count * (D / 16)
+  int tmem_cols;        // TMEM columns the CTA allocates
 };
 
-// AGG = true: pass 1 (segments 0 .. S-2 only; no readout, no output).
-template <int K, int NPOLY, bool AGG>
+// AGG = true: pass 1 (segments 0 .. S-2 only; no readout, no output). AREG = true: the experts'
+// transition rows in registers (E <= 8) instead of tensor memory. ZOH = true: zero-order-hold
+// injection (φ Δ B x, φ = (ā - 1) / (Δ A_t)) instead of Euler's Δ B x.
+template <int K, int NPOLY, bool AGG, bool AREG, bool ZOH>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1)
     scan_fast_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
                      const __grid_constant__ CUtensorMap tm_dl, const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_o,
                      const FastParams p) {
-  constexpr int NS = kNS, NP = kNP, CPW = kCPW, ACOLS = kACols;
   using St = Stage;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwarps = blockDim.x >> 5;
-  uint8_t* ring = smem + (size_t)warp * kStages * St::BYTES;
-  uint8_t* epi = smem + (size_t)nwarps * kStages * St::BYTES + (size_t)warp * Epi::BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)nwarps * (kStages * St::BYTES + Epi::BYTES));
+  uint8_t* ring = smem + (size_t)warp * kWarpBytes;
+  uint8_t* epi = ring + kStages * St::BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)nwarps * kWarpBytes);
   uint64_t* full = bars + warp * kStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + nwarps * kStages);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + nwarps * kStages) + 1;
   float* psm = reinterpret_cast<float*>(epi + Epi::P);
-  const float* dsm = reinterpret_cast<const float*>(epi + Epi::DS);
 
   if (lane == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
@@ -191,103 +240,132 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       }
     }
   }
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, 512);
+  if (!AREG && warp == 0) {
+    tmem_alloc(tmem_slot, (uint32_t)p.tmem_cols);
     tmem_relinquish();
   }
   __syncthreads();
   tc_fence_after();
   // this warp's TMEM window: its lane quarter, tmem_cols_per_warp(E) columns
-  const uint32_t tbase = *tmem_slot + ((uint32_t)(32 * (warp & 3)) << 16) +
-                         (uint32_t)(warp >> 2) * (uint32_t)tmem_cols_per_warp(p.E);
+  const uint32_t tbase = AREG ? 0u
+                              : *tmem_slot + ((uint32_t)(32 * (warp & 3)) << 16) +
+                                    (uint32_t)(warp >> 2) * (uint32_t)tmem_cols_per_warp(p.E);
+  float2 areg[8][4];  // AREG: the experts' rows (x log2 e), (c0, c1) per state
 
-  const int cp = lane >> 1;   // recurrence pass: channel pair 2cp, 2cp+1 of the warp's 32
-  const int gi = lane & 1;    //                  state group: states 8gi .. 8gi+7
-  const int n0 = gi * NS;
-  const int tl = lane >> 1;   // readout pass: token tl of the chunk,
-  const int c0 = (lane & 1) * 16;  //           channels c0 .. c0+15 of the warp's 32
-  const int ntiles = p.D / CPW;
+  const int cp = lane >> 2;        // recurrence pass: channel pair 2cp, 2cp+1 of the warp's 16
+  const int q = lane & 3;          //                  state quarter: states 4q .. 4q+3
+  const int rt = lane >> 1;        // readout pass: token rt of the chunk,
+  const int rc = (lane & 1) * 8;   //               channels rc .. rc+7 of the warp's 16
+  const int ntiles = p.D / kCPW;
   const int u_begin = (int)((int64_t)p.units * blockIdx.x / gridDim.x);
   const int u_end = (int)((int64_t)p.units * (blockIdx.x + 1) / gridDim.x);
   uint32_t phase_bits = 0;  // one parity bit per stage
   int ochunk = 0;           // output tiles written by this warp (selects the double buffer)
-  constexpr uint32_t tx_bytes = AGG ? (LC * CPW * 2 + LC * CPW * 4 + LC * 16 * 4)
-                                    : (2 * LC * CPW * 2 + LC * CPW * 4 + 2 * LC * 16 * 4);
+  constexpr uint32_t tx_bytes = AGG ? (LC * kCPW * 2 + LC * kCPW * 4 + LC * 16 * 4)
+                                    : (2 * LC * kCPW * 2 + LC * kCPW * 4 + 2 * LC * 16 * 4);
+  const uint32_t emax = (uint32_t)(p.E - 1);
 
   for (int u = u_begin + warp; u < u_end; u += nwarps) {
     const int tile = u % ntiles;
     const int bs = u / ntiles;  // b * seg_count + seg
     const int seg = bs % p.seg_count;
     const int b = bs / p.seg_count;
-    const int dA = tile * CPW + 2 * cp;  // this lane's channels dA, dA + 1
+    const int dA = tile * kCPW + 2 * cp;  // this lane's channels dA, dA + 1
     const int64_t t_begin = (int64_t)seg * p.Lseg;
     const int64_t t_end = std::min<int64_t>(p.L, t_begin + p.Lseg);
     const int nchunks = (int)((t_end - t_begin + LC - 1) / LC);
 
-    // per-expert transition rows of this lane's 2 x 8 states, times log2(e), into TMEM
-    // columns 16e + 8ch + s
-    for (int e = 0; e < p.E; ++e) {
+    // per-expert transition rows of this lane's 2 channels x 4 states, times log2(e), into TMEM
+    // columns 8e + 2s + channel (or into registers)
+    if (AREG) {
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        const float4* src = reinterpret_cast<const float4*>(p.A + ((size_t)e * p.D + dA + ch) * 16 + n0);
-        const float4 a0 = __ldg(src), a1 = __ldg(src + 1);
-        const uint32_t r[8] = {__float_as_uint(a0.x * kLog2e), __float_as_uint(a0.y * kLog2e),
-                               __float_as_uint(a0.z * kLog2e), __float_as_uint(a0.w * kLog2e),
-                               __float_as_uint(a1.x * kLog2e), __float_as_uint(a1.y * kLog2e),
-                               __float_as_uint(a1.z * kLog2e), __float_as_uint(a1.w * kLog2e)};
-        tmem_st8(tbase + (uint32_t)(e * ACOLS + 8 * ch), r);
+      for (int e = 0; e < 8; ++e) {
+        float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+        if (e < p.E) {
+          a0 = __ldg(reinterpret_cast<const float4*>(p.A + ((size_t)e * p.D + dA) * 16 + 4 * q));
+          a1 = __ldg(reinterpret_cast<const float4*>(p.A + ((size_t)e * p.D + dA + 1) * 16 + 4 * q));
+        }
+        areg[e][0] = make_float2(a0.x * kLog2e, a1.x * kLog2e);
+        areg[e][1] = make_float2(a0.y * kLog2e, a1.y * kLog2e);
+        areg[e][2] = make_float2(a0.z * kLog2e, a1.z * kLog2e);
+        areg[e][3] = make_float2(a0.w * kLog2e, a1.w * kLog2e);
       }
     }
-    tmem_wait_st();
-    if (!AGG) reinterpret_cast<float*>(epi + Epi::DS)[lane] = p.D_skip[tile * CPW + lane];
-
-    float2 h[2][NP];  // [channel][state pair]
-#pragma unroll
-    for (int ch = 0; ch < 2; ++ch) {
-      const float* hs = AGG ? nullptr
-                            : (p.h_seg != nullptr ? p.h_seg + (((size_t)b * p.S + seg) * p.D + dA + ch) * 16
-                                                  : (p.h0 != nullptr && seg == 0 ? p.h0 + ((size_t)b * p.D + dA + ch) * 16
-                                                                                 : nullptr));
-#pragma unroll
-      for (int s = 0; s < NP; ++s)
-        h[ch][s] = hs ? *reinterpret_cast<const float2*>(hs + n0 + 2 * s) : make_float2(0.f, 0.f);
+    for (int e = 0; e < (AREG ? 0 : p.E); ++e) {
+      const float4 a0 = __ldg(reinterpret_cast<const float4*>(p.A + ((size_t)e * p.D + dA) * 16 + 4 * q));
+      const float4 a1 = __ldg(reinterpret_cast<const float4*>(p.A + ((size_t)e * p.D + dA + 1) * 16 + 4 * q));
+      const uint32_t r[8] = {__float_as_uint(a0.x * kLog2e), __float_as_uint(a1.x * kLog2e),
+                             __float_as_uint(a0.y * kLog2e), __float_as_uint(a1.y * kLog2e),
+                             __float_as_uint(a0.z * kLog2e), __float_as_uint(a1.z * kLog2e),
+                             __float_as_uint(a0.w * kLog2e), __float_as_uint(a1.w * kLog2e)};
+      tmem_st8(tbase + (uint32_t)(e * 8), r);
     }
-    float2 lsum[2][NP];
-#pragma unroll
-    for (int ch = 0; ch < 2; ++ch)
-#pragma unroll
-      for (int s = 0; s < NP; ++s) lsum[ch][s] = make_float2(0.f, 0.f);
+    if (!AREG) tmem_wait_st();
+    float2 dsk[4];  // readout pass: D_skip of channels rc .. rc+7
+    if (!AGG) {
+      const float4 d0 = __ldg(reinterpret_cast<const float4*>(p.D_skip + tile * kCPW + rc));
+      const float4 d1 = __ldg(reinterpret_cast<const float4*>(p.D_skip + tile * kCPW + rc + 4));
+      dsk[0] = make_float2(d0.x, d0.y);
+      dsk[1] = make_float2(d0.z, d0.w);
+      dsk[2] = make_float2(d1.x, d1.y);
+      dsk[3] = make_float2(d1.z, d1.w);
+    }
 
-    // meta of one chunk: lane t (< LC) holds token t's {e0, e1, g0, g1}
+    // start state: (h[c0][s], h[c1][s])
+    float2 h[kSPL];
+    {
+      const float* hs = nullptr;
+      if (!AGG) {
+        if (p.h_seg != nullptr) hs = p.h_seg + (((size_t)b * p.S + seg) * p.D + dA) * 16;
+        else if (p.h0 != nullptr && seg == 0) hs = p.h0 + ((size_t)b * p.D + dA) * 16;
+      }
+      if (hs != nullptr) {
+        const float4 u0 = *reinterpret_cast<const float4*>(hs + 4 * q);
+        const float4 u1 = *reinterpret_cast<const float4*>(hs + 16 + 4 * q);
+        h[0] = make_float2(u0.x, u1.x);
+        h[1] = make_float2(u0.y, u1.y);
+        h[2] = make_float2(u0.z, u1.z);
+        h[3] = make_float2(u0.w, u1.w);
+      } else {
+#pragma unroll
+        for (int s = 0; s < kSPL; ++s) h[s] = f2(0.f);
+      }
+    }
+    float2 lsum[kSPL];
+#pragma unroll
+    for (int s = 0; s < kSPL; ++s) lsum[s] = f2(0.f);
+
+    // meta of one chunk: lane t (< LC) holds token t's {TMEM column of e0, of e1, g0, g1}; expert
+    // indices outside [0, E) are clamped into the table, tokens past the segment get gate 0
     auto load_meta = [&](int c) -> int4 {
       int4 m = make_int4(0, 0, 0, 0);
       const int64_t t = t_begin + (int64_t)c * LC + lane;
       if (lane < LC && c < nchunks && t < t_end) {
         const size_t tok = (size_t)b * p.L + t;
-        m.x = min(max(p.idx[tok * K], 0), p.E - 1);
-        m.z = __float_as_int(p.gates[tok * K]);
+        m.x = (int)(min((uint32_t)__ldg(p.idx + tok * K), emax) * (AREG ? 1u : 8u));
+        m.z = __float_as_int(__ldg(p.gates + tok * K));
         if (K == 2) {
-          m.y = min(max(p.idx[tok * K + 1], 0), p.E - 1);
-          m.w = __float_as_int(p.gates[tok * K + 1]);
+          m.y = (int)(min((uint32_t)__ldg(p.idx + tok * K + 1), emax) * (AREG ? 1u : 8u));
+          m.w = __float_as_int(__ldg(p.gates + tok * K + 1));
         }
       }
       return m;
     };
     // fill stage (c % kStages) with chunk c: meta from registers, the rest by TMA
-    auto issue = [&](int c, int4 meta) {
+    auto issue = [&](int c, int4 m) {
       uint8_t* st = ring + (c % kStages) * St::BYTES;
-      if (lane < LC) reinterpret_cast<int4*>(st + St::META)[lane] = meta;
+      if (lane < LC) reinterpret_cast<int4*>(st + St::META)[lane] = m;
       __syncwarp();
       if (lane == 0) {
         fence_proxy_async_smem();
         uint64_t* bar = &full[c % kStages];
         mbar_arrive_expect_tx(bar, tx_bytes);
         const int t0 = (int)(t_begin + (int64_t)c * LC);
-        tma_load_3d(st + St::X, &tm_x, bar, tile * CPW, t0, b);
-        tma_load_3d(st + St::DL, &tm_dl, bar, tile * CPW, t0, b);
+        tma_load_3d(st + St::X, &tm_x, bar, tile * kCPW, t0, b);
+        tma_load_3d(st + St::DL, &tm_dl, bar, tile * kCPW, t0, b);
         tma_load_3d(st + St::B, &tm_b, bar, 0, t0, b);
         if (!AGG) {
-          tma_load_3d(st + St::Z, &tm_z, bar, tile * CPW, t0, b);
+          tma_load_3d(st + St::Z, &tm_z, bar, tile * kCPW, t0, b);
           tma_load_3d(st + St::C, &tm_c, bar, 0, t0, b);
         }
       }
@@ -302,153 +380,141 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
     }
     bool ok = true;
     int issued = pre;
+    int failed_chunk = 0;
     for (int c = 0; c < nchunks; ++c) {
       const int sidx = c % kStages;
       if (!mbar_wait(&full[sidx], (phase_bits >> sidx) & 1u, abort_flag)) {
         ok = false;
+        failed_chunk = c;
         break;
       }
       phase_bits ^= 1u << sidx;
       const uint8_t* st = ring + sidx * St::BYTES;
       const int4* meta = reinterpret_cast<const int4*>(st + St::META);
-      const __nv_bfloat162* xs2 = reinterpret_cast<const __nv_bfloat162*>(st + St::X);
+      const uint32_t* xs2 = reinterpret_cast<const uint32_t*>(st + St::X);
       const float2* ds2 = reinterpret_cast<const float2*>(st + St::DL);
       const float4* bsm = reinterpret_cast<const float4*>(st + St::B);
       const float4* csm = reinterpret_cast<const float4*>(st + St::C);
       const int64_t t0 = t_begin + (int64_t)c * LC;
+
       // issue token t's loads (TMEM loads are waited for by the caller)
-      auto load_tok = [&](TokIn& q, int t) {
-        q.m = meta[t];
-        tmem_ld16_nowait(tbase + (uint32_t)(q.m.x * ACOLS), q.ar[0]);
-        if (K == 2) tmem_ld16_nowait(tbase + (uint32_t)(q.m.y * ACOLS), q.ar[1]);
-        q.dl = ds2[t * (CPW / 2) + cp];
-        q.xv = __bfloat1622float2(xs2[t * (CPW / 2) + cp]);
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const float4 bq = bsm[t * 4 + gi * 2 + i];
-          q.bv[2 * i] = make_float2(bq.x, bq.y);
-          q.bv[2 * i + 1] = make_float2(bq.z, bq.w);
-          if (!AGG) {
-            const float4 cq = csm[t * 4 + gi * 2 + i];
-            q.cv[2 * i] = make_float2(cq.x, cq.y);
-            q.cv[2 * i + 1] = make_float2(cq.z, cq.w);
-          }
+      auto load_tok = [&](TokIn& tk, int t) {
+        tk.m = meta[t];
+        if (!AREG) {
+          tmem_ld8_nowait(tbase + (uint32_t)tk.m.x, tk.ar[0]);
+          if (K == 2) tmem_ld8_nowait(tbase + (uint32_t)tk.m.y, tk.ar[1]);
         }
+        tk.dl = ds2[t * (kCPW / 2) + cp];
+        const uint32_t xw = xs2[t * (kCPW / 2) + cp];
+        tk.xv = make_float2(bf16lo(xw), bf16hi(xw));
+        tk.bq = bsm[t * 4 + q];
+        if (!AGG) tk.cq = csm[t * 4 + q];
       };
       // decay factors of a loaded token (independent of the state)
-      auto decay = [&](TokIn& q) {
-        q.dx[0] = q.dl.x * q.xv.x;
-        q.dx[1] = q.dl.y * q.xv.y;
+      auto decay = [&](TokIn& tk) {
+        tk.dx = __fmul2_rn(tk.dl, tk.xv);
+        const float2 dg0 = __fmul2_rn(tk.dl, f2(__int_as_float(tk.m.z)));
+        const float2 dg1 = __fmul2_rn(tk.dl, f2(__int_as_float(tk.m.w)));
+        float2 args[kSPL];
+        if (AREG) {
+          mix_areg<false>(areg, tk.m.x, dg0, args);
+          if (K == 2) mix_areg<true>(areg, tk.m.y, dg1, args);
+        }
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          const float dlt = ch == 0 ? q.dl.x : q.dl.y;
-          const float g0 = dlt * __int_as_float(q.m.z);
-          const float g1 = dlt * __int_as_float(q.m.w);
-#pragma unroll
-          for (int s = 0; s < NP; ++s) {
-            const float2 a0 = make_float2(__uint_as_float(q.ar[0][ch * NS + 2 * s]), __uint_as_float(q.ar[0][ch * NS + 2 * s + 1]));
-            q.arg[ch][s] = __fmul2_rn(make_float2(g0, g0), a0);
-            if (K == 2) {
-              const float2 a1 = make_float2(__uint_as_float(q.ar[1][ch * NS + 2 * s]), __uint_as_float(q.ar[1][ch * NS + 2 * s + 1]));
-              q.arg[ch][s] = __ffma2_rn(make_float2(g1, g1), a1, q.arg[ch][s]);
-            }
-            if (AGG) lsum[ch][s] = __fadd2_rn(lsum[ch][s], q.arg[ch][s]);  // Σ_t log2 ā_t
-            if (s >= NP - NPOLY / 2) {
-              q.a[ch][s] = exp2_poly2(q.arg[ch][s]);
-            } else {
-              q.a[ch][s] = make_float2(ex2_approx(q.arg[ch][s].x), ex2_approx(q.arg[ch][s].y));
-            }
+        for (int s = 0; s < kSPL; ++s) {
+          float2 arg;
+          if (AREG) {
+            arg = args[s];
+          } else {
+            arg = __fmul2_rn(dg0, make_float2(__uint_as_float(tk.ar[0][2 * s]), __uint_as_float(tk.ar[0][2 * s + 1])));
+            if (K == 2)
+              arg = __ffma2_rn(dg1, make_float2(__uint_as_float(tk.ar[1][2 * s]), __uint_as_float(tk.ar[1][2 * s + 1])),
+                               arg);
           }
+          if (AGG) lsum[s] = __fadd2_rn(lsum[s], arg);  // Σ_t log2 ā_t
+          // elements 2s, 2s+1 of the lane's 8; the last NPOLY of them go to the FMA pipe
+          const float ax = (2 * s >= 8 - NPOLY) ? exp2_poly(arg.x) : ex2_approx(arg.x);
+          const float ay = (2 * s + 1 >= 8 - NPOLY) ? exp2_poly(arg.y) : ex2_approx(arg.y);
+          tk.a[s] = make_float2(ax, ay);
+          if (ZOH) tk.phi[s] = make_float2(zoh_phi(arg.x, ax), zoh_phi(arg.y, ay));
         }
       };
 
       // ---- recurrence pass: the state chain only; partial readouts go to shared memory ----
       // Software-pipelined by one token: while token t updates the state, token t+1's inputs are
-      // loaded (its A rows from TMEM, Δ, x, B, C from the ring) and its decay factors computed,
-      // so the TMEM and shared-memory latencies and the exponentials of t+1 overlap t's FMAs.
+      // loaded (its A rows from TMEM, Δ, x, B, C from the ring) and its decay factors computed.
       TokIn cur, nxt;
       load_tok(cur, 0);
-      tmem_wait_ld();
+      if (!AREG) tmem_wait_ld();
       decay(cur);
-      auto token = [&](int t) {
+#pragma unroll
+      for (int t = 0; t < LC; ++t) {
         if (t + 1 < LC) load_tok(nxt, t + 1);
-        float yc[2];
+        const float bsv[4] = {cur.bq.x, cur.bq.y, cur.bq.z, cur.bq.w};
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          const float2 dxx = make_float2(cur.dx[ch], cur.dx[ch]);
-#pragma unroll
-          for (int s = 0; s < NP; ++s) h[ch][s] = __ffma2_rn(cur.a[ch][s], h[ch][s], __fmul2_rn(dxx, cur.bv[s]));
-          if (!AGG) {
-            // two independent accumulation chains (even and odd state pairs)
-            float2 ya = __fmul2_rn(cur.cv[0], h[ch][0]);
-            float2 yb = __fmul2_rn(cur.cv[1], h[ch][1]);
-#pragma unroll
-            for (int s = 2; s < NP; s += 2) {
-              ya = __ffma2_rn(cur.cv[s], h[ch][s], ya);
-              yb = __ffma2_rn(cur.cv[s + 1], h[ch][s + 1], yb);
-            }
-            yc[ch] = (ya.x + yb.x) + (ya.y + yb.y);
-          }
+        for (int s = 0; s < kSPL; ++s) {
+          float2 u = __fmul2_rn(cur.dx, f2(bsv[s]));
+          if (ZOH) u = __fmul2_rn(u, cur.phi[s]);
+          h[s] = __ffma2_rn(cur.a[s], h[s], u);
         }
-        if (!AGG) *reinterpret_cast<float2*>(psm + (t * 2 + gi) * kPRow + 2 * cp) = make_float2(yc[0], yc[1]);
+        if (!AGG) {
+          float2 y = __fmul2_rn(f2(cur.cq.x), h[0]);
+          y = __ffma2_rn(f2(cur.cq.y), h[1], y);
+          y = __ffma2_rn(f2(cur.cq.z), h[2], y);
+          y = __ffma2_rn(f2(cur.cq.w), h[3], y);
+          *reinterpret_cast<float2*>(psm + t * kPRow + q * kCPW + 2 * cp) = y;
+        }
         if (t + 1 < LC) {
-          tmem_wait_ld();
+          if (!AREG) tmem_wait_ld();
           decay(nxt);
           cur = nxt;
         }
-      };
-#pragma unroll
-      for (int t = 0; t < LC; ++t) token(t);
+      }
 
-      // ---- readout pass: lane = (token tl, channels c0..c0+15) ----
+      // ---- readout pass: lane = (token rt, channels rc..rc+7) ----
       if (!AGG) {
         __syncwarp();
-        const float4* p0 = reinterpret_cast<const float4*>(psm + (tl * 2 + 0) * kPRow + c0);
-        const float4* p1 = reinterpret_cast<const float4*>(psm + (tl * 2 + 1) * kPRow + c0);
-        const uint4* xq = reinterpret_cast<const uint4*>(st + St::X + (tl * CPW + c0) * 2);
-        const uint4* zq = reinterpret_cast<const uint4*>(st + St::Z + (tl * CPW + c0) * 2);
-        const float4* dq = reinterpret_cast<const float4*>(dsm + c0);
-        uint32_t packed[8];
+        float2 yv[4];
+        {
+          const float4* pr = reinterpret_cast<const float4*>(psm + rt * kPRow + rc);
+          float4 s0 = pr[0], s1 = pr[1];
 #pragma unroll
-        for (int hq = 0; hq < 2; ++hq) {  // 8 channels at a time
-          float2 xf[4], zf[4];
-          bf16x8_to_float2(xq[hq], xf);
-          bf16x8_to_float2(zq[hq], zf);
-          float2 yv[4], dk[4];
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const float4 a4 = p0[2 * hq + i], b4 = p1[2 * hq + i], d4 = dq[2 * hq + i];
-            yv[2 * i] = __fadd2_rn(make_float2(a4.x, a4.y), make_float2(b4.x, b4.y));
-            yv[2 * i + 1] = __fadd2_rn(make_float2(a4.z, a4.w), make_float2(b4.z, b4.w));
-            dk[2 * i] = make_float2(d4.x, d4.y);
-            dk[2 * i + 1] = make_float2(d4.z, d4.w);
+          for (int qq = 1; qq < 4; ++qq) {
+            const float4 v0 = pr[qq * (kCPW / 4)], v1 = pr[qq * (kCPW / 4) + 1];
+            s0 = make_float4(s0.x + v0.x, s0.y + v0.y, s0.z + v0.z, s0.w + v0.w);
+            s1 = make_float4(s1.x + v1.x, s1.y + v1.y, s1.z + v1.z, s1.w + v1.w);
           }
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 y = __ffma2_rn(dk[i], xf[i], yv[i]);  // y + D_skip x
-            yv[i] = y;
-            const float2 hz = __fmul2_rn(zf[i], make_float2(0.5f, 0.5f));
-            const float2 th = make_float2(tanh_approx(hz.x), tanh_approx(hz.y));
-            const float2 sig = __ffma2_rn(th, make_float2(0.5f, 0.5f), make_float2(0.5f, 0.5f));
-            packed[4 * hq + i] = pack_bf16x2(__fmul2_rn(__fmul2_rn(y, zf[i]), sig));
-          }
-          if (p.y_pre != nullptr && t0 + tl < t_end) {
-            float4* yp = reinterpret_cast<float4*>(p.y_pre + ((size_t)b * p.L + t0 + tl) * p.D + tile * CPW + c0 + 8 * hq);
-            yp[0] = make_float4(yv[0].x, yv[0].y, yv[1].x, yv[1].y);
-            yp[1] = make_float4(yv[2].x, yv[2].y, yv[3].x, yv[3].y);
-          }
+          yv[0] = make_float2(s0.x, s0.y);
+          yv[1] = make_float2(s0.z, s0.w);
+          yv[2] = make_float2(s1.x, s1.y);
+          yv[3] = make_float2(s1.z, s1.w);
         }
-        // the previous TMA store from this output buffer must have finished reading it
-        uint8_t* obuf = epi + Epi::O + (ochunk & 1) * (LC * CPW * 2);
+        float2 xf[4], zf[4];
+        bf16x8_to_float2(*reinterpret_cast<const uint4*>(st + St::X + (rt * kCPW + rc) * 2), xf);
+        bf16x8_to_float2(*reinterpret_cast<const uint4*>(st + St::Z + (rt * kCPW + rc) * 2), zf);
+        uint32_t packed[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          yv[i] = __ffma2_rn(dsk[i], xf[i], yv[i]);  // y + D_skip x
+          const float2 hz = __fmul2_rn(zf[i], f2(0.5f));
+          const float2 th = make_float2(tanh_approx(hz.x), tanh_approx(hz.y));
+          const float2 silu = __ffma2_rn(hz, th, hz);  // z σ(z)
+          packed[i] = pack_bf16x2(__fmul2_rn(yv[i], silu));
+        }
+        if (p.y_pre != nullptr && t0 + rt < t_end) {
+          float4* yp = reinterpret_cast<float4*>(p.y_pre + ((size_t)b * p.L + t0 + rt) * p.D + tile * kCPW + rc);
+          yp[0] = make_float4(yv[0].x, yv[0].y, yv[1].x, yv[1].y);
+          yp[1] = make_float4(yv[2].x, yv[2].y, yv[3].x, yv[3].y);
+        }
+        // the TMA store issued two chunks ago from this output buffer must have read it
+        uint8_t* obuf = epi + Epi::O + (ochunk & 1) * (LC * kCPW * 2);
         if (lane == 0) bulk_wait_read<1>();
         __syncwarp();
-        uint4* od = reinterpret_cast<uint4*>(obuf + (tl * CPW + c0) * 2);
-        od[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-        od[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+        *reinterpret_cast<uint4*>(obuf + (rt * kCPW + rc) * 2) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_3d(&tm_o, obuf, tile * CPW, (int)t0, b);
+          tma_store_3d(&tm_o, obuf, tile * kCPW, (int)t0, b);
           bulk_commit();
         }
         ++ochunk;
@@ -464,9 +530,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
     if (!ok) {
       *abort_flag = 1;
       if (lane == 0) record_device_error(p.status, SWIMBA_ERR_TIMEOUT, 31, blockIdx.x, u);
-      // let this warp's copies in flight land before the CTA exits (bounded, ignores the flag)
-      for (int c = issued - kStages; c < issued; ++c) {
-        if (c < 0) continue;
+      // let the copies this warp still has in flight (chunks failed_chunk .. issued-1) land before
+      // the CTA exits (bounded, ignores the flag)
+      for (int c = failed_chunk; c < issued; ++c) {
         const int sidx = c % kStages;
         const uint64_t w0 = globaltimer_ns();
         while (!mbar_try_wait(&full[sidx], (phase_bits >> sidx) & 1u) && globaltimer_ns() - w0 < kWaitLimitNs) {
@@ -475,29 +541,31 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       }
       break;
     }
-#pragma unroll
-    for (int ch = 0; ch < 2; ++ch) {
-      if (AGG) {
-        const size_t o = (((size_t)b * p.S + seg) * p.D + dA + ch) * 16 + n0;
-#pragma unroll
-        for (int s = 0; s < NP; ++s) {
-          *reinterpret_cast<float2*>(p.agg_h + o + 2 * s) = h[ch][s];
-          *reinterpret_cast<float2*>(p.agg_logp + o + 2 * s) = lsum[ch][s];
-        }
-      } else if (p.h_final != nullptr && seg == p.S - 1) {
-        const size_t o = ((size_t)b * p.D + dA + ch) * 16 + n0;
-#pragma unroll
-        for (int s = 0; s < NP; ++s) *reinterpret_cast<float2*>(p.h_final + o + 2 * s) = h[ch][s];
-      }
+    // end state (segment aggregates in pass 1, h_final after the last segment)
+    float* hout = nullptr;
+    float* lout = nullptr;
+    if (AGG) {
+      hout = p.agg_h + (((size_t)b * p.S + seg) * p.D + dA) * 16;
+      lout = p.agg_logp + (((size_t)b * p.S + seg) * p.D + dA) * 16;
+    } else if (p.h_final != nullptr && seg == p.S - 1) {
+      hout = p.h_final + ((size_t)b * p.D + dA) * 16;
+    }
+    if (hout != nullptr) {
+      *reinterpret_cast<float4*>(hout + 4 * q) = make_float4(h[0].x, h[1].x, h[2].x, h[3].x);
+      *reinterpret_cast<float4*>(hout + 16 + 4 * q) = make_float4(h[0].y, h[1].y, h[2].y, h[3].y);
+    }
+    if (lout != nullptr) {
+      *reinterpret_cast<float4*>(lout + 4 * q) = make_float4(lsum[0].x, lsum[1].x, lsum[2].x, lsum[3].x);
+      *reinterpret_cast<float4*>(lout + 16 + 4 * q) = make_float4(lsum[0].y, lsum[1].y, lsum[2].y, lsum[3].y);
     }
     __syncwarp();
   }
   // the output stores must have read their shared-memory tiles before the CTA's memory goes away
   if (!AGG && lane == 0) bulk_wait<0>();
   __syncthreads();
-  if (warp == 0) {
+  if (!AREG && warp == 0) {
     tc_fence_after();
-    tmem_dealloc(*tmem_slot, 512);
+    tmem_dealloc(*tmem_slot, (uint32_t)p.tmem_cols);
   }
 }
 
@@ -515,6 +583,26 @@ __global__ void scan_carry_kernel(const float* h0, const float* agg_h, const flo
     h_seg[o] = H;
     if (s + 1 < S) H = fmaf(ex2_approx(agg_logp[o]), H, agg_h[o]);
   }
+}
+
+// Summary of a whole sequence from its segments' aggregates: the state after the last segment when
+// the first starts from zero, H = 2^{logp[s]} H + h_end[s] over s, and the total log decay
+// Σ_s logp[s] (log2 units in, natural log out).
+__global__ void summary_combine_kernel(const float* agg_h, const float* agg_logp, float* h_zero, float* log_decay,
+                                       int B, int S, int D) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // over (b, d, n)
+  if (i >= (int64_t)B * D * 16) return;
+  const int n = (int)(i % 16);
+  const int d = (int)((i / 16) % D);
+  const int b = (int)(i / (16 * (int64_t)D));
+  float H = 0.f, lp = 0.f;
+  for (int s = 0; s < S; ++s) {
+    const size_t o = (((size_t)b * S + s) * D + d) * 16 + n;
+    H = fmaf(ex2_approx(agg_logp[o]), H, agg_h[o]);
+    lp += agg_logp[o];
+  }
+  h_zero[i] = H;
+  log_decay[i] = lp * 0.6931471805599453f;  // ln 2
 }
 
 // ---- host ------------------------------------------------------------------------------------------
@@ -551,8 +639,6 @@ int device_sms() {
   return n;
 }
 
-constexpr int kNPoly = 0;  // states per lane and channel whose exp2 runs on the FMA pipe (even, <= 8)
-
 }  // namespace
 
 // ---- segment plan and workspace ---------------------------------------------------------------------
@@ -564,10 +650,14 @@ ScanPlan scan_fast_plan(int64_t B, int64_t L, int D, int N, int E, int k, bool i
     pl.fast = false;
     return pl;
   }
+  const int64_t sms = device_sms();
   const int64_t base_units = B * (D / kCPW);
-  const int64_t target = (int64_t)device_sms() * 6;  // at least 6 warps (192 channels) per SM
   int64_t S = 1;
-  if (base_units < target) S = std::min<int64_t>((target + base_units - 1) / base_units, (L + LC - 1) / LC);
+  if (base_units < sms * SWIMBA_SCAN_MIN_WARPS) {
+    const int64_t target = sms * SWIMBA_SCAN_TARGET_WARPS;
+    S = std::min<int64_t>((target + base_units - 1) / base_units, (L + LC - 1) / LC);
+    S = std::max<int64_t>(S, 1);
+  }
   int64_t Lseg = (L + S - 1) / S;
   Lseg = (Lseg + LC - 1) / LC * LC;
   S = (L + Lseg - 1) / Lseg;
@@ -577,18 +667,40 @@ ScanPlan scan_fast_plan(int64_t B, int64_t L, int D, int N, int E, int k, bool i
   return pl;
 }
 
-template <int K>
-static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s) {
-  constexpr int CPW = kCPW;
+using FastKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                           const CUtensorMap, const CUtensorMap, const FastParams);
+
+template <int K, bool AGG>
+static FastKernel pick_kernel(int E, bool zoh) {
+#if SWIMBA_SCAN_AREG
+  if (E <= 8) return zoh ? scan_fast_kernel<K, kNPoly, AGG, true, true> : scan_fast_kernel<K, kNPoly, AGG, true, false>;
+#endif
+  (void)E;
+  return zoh ? scan_fast_kernel<K, kNPoly, AGG, false, true> : scan_fast_kernel<K, kNPoly, AGG, false, false>;
+}
+
+struct FastLaunch {
   CUtensorMap tx, tz, td, tb, tc, to;
-  if (!map3(&tx, sp.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.D, sp.L, sp.B, CPW) ||
-      !map3(&tz, sp.z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.D, sp.L, sp.B, CPW) ||
-      !map3(&td, sp.delta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, sp.D, sp.L, sp.B, CPW) ||
-      !map3(&tb, sp.B_mix, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 16, sp.L, sp.B, 16) ||
-      !map3(&tc, sp.C_mix, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 16, sp.L, sp.B, 16) ||
-      !map3(&to, sp.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.D, sp.L, sp.B, CPW))
-    return cudaErrorInvalidValue;
-  FastParams p{};
+  FastParams p;
+  int sms, win;
+  bool zoh;
+};
+
+static bool fast_setup(const ScanParams& sp, const ScanPlan& pl, void* status, FastLaunch& f) {
+  if (!map3(&f.tx, sp.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.D, sp.L, sp.B, kCPW) ||
+      !map3(&f.td, sp.delta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, sp.D, sp.L, sp.B, kCPW) ||
+      !map3(&f.tb, sp.B_mix, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 16, sp.L, sp.B, 16))
+    return false;
+  // the summary pass reads no z, C_mix or output: its maps repeat x and B_mix
+  const void* z = sp.z != nullptr ? sp.z : sp.x;
+  const float* C = sp.C_mix != nullptr ? sp.C_mix : sp.B_mix;
+  void* out = sp.out != nullptr ? sp.out : const_cast<void*>(sp.x);
+  if (!map3(&f.tz, z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.D, sp.L, sp.B, kCPW) ||
+      !map3(&f.tc, C, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 16, sp.L, sp.B, 16) ||
+      !map3(&f.to, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.D, sp.L, sp.B, kCPW))
+    return false;
+  FastParams& p = f.p;
+  p = FastParams{};
   p.idx = sp.idx;
   p.gates = sp.gates;
   p.A = sp.A;
@@ -602,58 +714,111 @@ static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* s
   p.B = sp.B;
   p.D = sp.D;
   p.E = sp.E;
-  p.k = sp.k;
   p.S = pl.S;
   p.seg_count = pl.S;
-  p.units = sp.B * pl.S * (sp.D / CPW);
-  const int sms = device_sms();
-  // block size: the kernel's register use decides how many warps a CTA may hold
-  auto shape = [&](const void* fn, int units, int& ctas, int& warps) -> cudaError_t {
-    cudaFuncAttributes fa;
-    cudaError_t err = cudaFuncGetAttributes(&fa, fn);
-    if (err != cudaSuccess) return err;
-    const int per_quarter = 512 / tmem_cols_per_warp(sp.E);  // warps that fit one lane quarter's TMEM
-    const int wmax = std::max(1, std::min({kMaxWarps, fa.maxThreadsPerBlock / 32, 4 * per_quarter}));
-    ctas = std::max(1, std::min(sms, units));
-    warps = std::min(wmax, (units + ctas - 1) / ctas);
-    if ((int64_t)ctas * warps < units) ctas = std::min<int64_t>((units + warps - 1) / warps, 65535);
-    return cudaSuccess;
-  };
+  p.units = sp.B * pl.S * (sp.D / kCPW);
+  f.sms = device_sms();
+  f.win = tmem_cols_per_warp(sp.E);
+  f.zoh = sp.zoh != 0;
+  return true;
+}
+
+// One persistent CTA per SM; the warps per CTA cover the units (at most kMaxWarps, and at most 4
+// windows of `win` TMEM columns per lane quarter); the TMEM allocation covers the CTA's windows.
+static cudaError_t fast_shape(const void* fn, int units, int sms, int win, int& ctas, int& warps, int& cols) {
+  cudaFuncAttributes fa;
+  cudaError_t err = cudaFuncGetAttributes(&fa, fn);
+  if (err != cudaSuccess) return err;
+  const int wmax = std::max(1, std::min({kMaxWarps, fa.maxThreadsPerBlock / 32, 4 * (512 / win)}));
+  ctas = std::max(1, std::min(sms, units));
+  warps = std::min(wmax, (units + ctas - 1) / ctas);
+  if ((int64_t)ctas * warps < units) ctas = (int)std::min<int64_t>((units + warps - 1) / warps, 65535);
+  const int need = ((warps + 3) / 4) * win;
+  cols = 32;
+  while (cols < need) cols *= 2;
+  return cudaSuccess;
+}
+
+static size_t fast_smem(int warps) { return 128 + (size_t)warps * (kWarpBytes + kStages * 8) + 16; }
+
+// Pass 1 over `seg_count` segments (from segment 0): end state from zero and log2 decay sums into
+// agg_h / agg_logp [B, S, D, 16].
+template <int K>
+static cudaError_t launch_agg(FastLaunch& f, int seg_count, float* agg_h, float* agg_logp, cudaStream_t s) {
+  FastParams a = f.p;
+  a.agg_h = agg_h;
+  a.agg_logp = agg_logp;
+  a.h0 = nullptr;
+  a.h_seg = nullptr;
+  a.seg_count = seg_count;
+  a.units = a.B * seg_count * (a.D / kCPW);
+  auto kagg = pick_kernel<K, true>(a.E, f.zoh);
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(kagg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fast_smem(kMaxWarps))) !=
+      cudaSuccess)
+    return e;
   int ctas, warps;
-  const size_t smem_per_warp = (size_t)kStages * Stage::BYTES + Epi::BYTES + (size_t)kStages * 8;
-  const size_t smem = 128 + (size_t)kMaxWarps * smem_per_warp + 32;
+  if ((e = fast_shape((const void*)kagg, a.units, f.sms, f.win, ctas, warps, a.tmem_cols)) != cudaSuccess) return e;
+  kagg<<<ctas, warps * 32, fast_smem(warps), s>>>(f.tx, f.tz, f.td, f.tb, f.tc, f.to, a);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <int K>
+static cudaError_t launch_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s) {
+  FastLaunch f;
+  if (!fast_setup(sp, pl, status, f)) return cudaErrorInvalidValue;
+  FastParams& p = f.p;
   cudaError_t e;
   if (pl.S > 1) {
     float* agg_h = reinterpret_cast<float*>(seg_ws);
     float* agg_logp = agg_h + (size_t)sp.B * pl.S * sp.D * 16;
     float* h_seg = agg_logp + (size_t)sp.B * pl.S * sp.D * 16;
-    FastParams a = p;
-    a.agg_h = agg_h;
-    a.agg_logp = agg_logp;
-    a.h0 = nullptr;
-    a.seg_count = pl.S - 1;  // the last segment needs no aggregate
-    a.units = sp.B * (pl.S - 1) * (sp.D / CPW);
-    auto kagg = scan_fast_kernel<K, kNPoly, true>;
-    if ((e = cudaFuncSetAttribute(kagg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
-      return e;
-    if ((e = shape((const void*)kagg, a.units, ctas, warps)) != cudaSuccess) return e;
-    kagg<<<ctas, warps * 32, 128 + warps * smem_per_warp + 32, s>>>(tx, tz, td, tb, tc, to, a);
+    if ((e = launch_agg<K>(f, pl.S - 1, agg_h, agg_logp, s)) != cudaSuccess) return e;  // the last needs none
     const int64_t n = (int64_t)sp.B * sp.D * 16;
     scan_carry_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(sp.h0, agg_h, agg_logp, h_seg, sp.B, pl.S, sp.D);
-    note_launch(2);
+    note_launch();
     p.h_seg = h_seg;
   }
-  auto kmain = scan_fast_kernel<K, kNPoly, false>;
-  if ((e = cudaFuncSetAttribute(kmain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+  auto kmain = pick_kernel<K, false>(p.E, sp.zoh != 0);
+  if ((e = cudaFuncSetAttribute(kmain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fast_smem(kMaxWarps))) !=
+      cudaSuccess)
     return e;
-  if ((e = shape((const void*)kmain, p.units, ctas, warps)) != cudaSuccess) return e;
-  kmain<<<ctas, warps * 32, 128 + warps * smem_per_warp + 32, s>>>(tx, tz, td, tb, tc, to, p);
+  int ctas, warps;
+  if ((e = fast_shape((const void*)kmain, p.units, f.sms, f.win, ctas, warps, p.tmem_cols)) != cudaSuccess) return e;
+  kmain<<<ctas, warps * 32, fast_smem(warps), s>>>(f.tx, f.tz, f.td, f.tb, f.tc, f.to, p);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <int K>
+static cudaError_t launch_summary(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status,
+                                  float* h_zero, float* log_decay, cudaStream_t s) {
+  FastLaunch f;
+  if (!fast_setup(sp, pl, status, f)) return cudaErrorInvalidValue;
+  float* agg_h = reinterpret_cast<float*>(seg_ws);
+  float* agg_logp = agg_h + (size_t)sp.B * pl.S * sp.D * 16;
+  cudaError_t e;
+  if ((e = launch_agg<K>(f, pl.S, agg_h, agg_logp, s)) != cudaSuccess) return e;
+  const int64_t n = (int64_t)sp.B * sp.D * 16;
+  summary_combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(agg_h, agg_logp, h_zero, log_decay, sp.B, pl.S,
+                                                                       sp.D);
   note_launch();
   return cudaGetLastError();
 }
 
 cudaError_t run_scan_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s) {
   return sp.k == 1 ? launch_fast<1>(sp, pl, seg_ws, status, s) : launch_fast<2>(sp, pl, seg_ws, status, s);
+}
+
+size_t scan_fast_summary_ws(const ScanPlan& pl, int64_t B, int D) {
+  return (size_t)2 * B * pl.S * D * 16 * sizeof(float);
+}
+
+cudaError_t run_scan_summary_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, float* h_zero,
+                                  float* log_decay, cudaStream_t s) {
+  return sp.k == 1 ? launch_summary<1>(sp, pl, seg_ws, status, h_zero, log_decay, s)
+                   : launch_summary<2>(sp, pl, seg_ws, status, h_zero, log_decay, s);
 }
 
 // ---- scratch for callers that cannot allocate device memory ----------------------------------------
@@ -664,27 +829,15 @@ cudaError_t run_scan_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws
 // library's module, so every GPU that loads the library holds it until the process exits.
 static __device__ __align__(256) unsigned char g_scan_noalloc_scratch[kScanNoAllocScratchBytes];
 
-namespace {
-std::mutex g_noalloc_mu;
-void* g_noalloc_addr[256] = {};
-}  // namespace
-
 // Device address of the fixed scratch on the current device. In host code the array's name is only
-// a host-side stand-in, so the address comes from cudaGetSymbolAddress, once per device, with that
-// device current, and is cached.
+// a host-side stand-in, so the address comes from cudaGetSymbolAddress with the device current. It
+// is looked up on every call (cheap once the module is loaded), so a context that was reset and
+// re-created never sees a stale address.
 cudaError_t scan_noalloc_scratch(void** addr) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* ptr = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&ptr, g_scan_noalloc_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 256) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_addr[dev] == nullptr) {
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_scan_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_noalloc_addr[dev] = ptr;
-  }
-  *addr = g_noalloc_addr[dev];
+  *addr = ptr;
   return cudaSuccess;
 }
 

@@ -26,7 +26,8 @@ import torch  # noqa: E402  (after the library check so a missing build is repor
 
 SWIMBA_F32 = 0
 SWIMBA_BF16 = 1
-SWIMBA_OP_ROUTE, SWIMBA_OP_PROJ, SWIMBA_OP_SCAN, SWIMBA_OP_STEP, SWIMBA_OP_LAYER = range(5)
+(SWIMBA_OP_ROUTE, SWIMBA_OP_PROJ, SWIMBA_OP_SCAN, SWIMBA_OP_STEP, SWIMBA_OP_LAYER, SWIMBA_OP_SUMMARY,
+ SWIMBA_OP_SEPARATE) = range(7)
 
 STATUS = {
     0: "SWIMBA_OK",
@@ -44,7 +45,14 @@ EXPORTED = [
     "swimba_route",
     "swimba_mixed_proj",
     "swimba_scan_fwd",
+    "swimba_scan_fwd_zoh",
     "swimba_scan_fwd_noalloc",
+    "swimba_scan_fwd_noalloc_status",
+    "swimba_scan_fwd_noalloc_status_block",
+    "swimba_scan_summary",
+    "swimba_scan_chain",
+    "swimba_separate_proj",
+    "swimba_separate_scan",
     "swimba_step",
     "swimba_get_device_status",
     "swimba_check_wait_timeout",
@@ -96,9 +104,26 @@ _lib.swimba_mixed_proj.restype = ctypes.c_int
 _lib.swimba_scan_fwd.argtypes = [ctypes.POINTER(swimba_dims), _P, _P, _P, _P, _P, _P, _P,
                                  ctypes.POINTER(swimba_weights), _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.swimba_scan_fwd.restype = ctypes.c_int
+_lib.swimba_scan_fwd_zoh.argtypes = _lib.swimba_scan_fwd.argtypes
+_lib.swimba_scan_fwd_zoh.restype = ctypes.c_int
 _lib.swimba_scan_fwd_noalloc.argtypes = [ctypes.POINTER(swimba_dims), _P, _P, _P, _P, _P, _P, _P,
                                          ctypes.POINTER(swimba_weights), _P, _P, _P, _P, _P]
 _lib.swimba_scan_fwd_noalloc.restype = ctypes.c_int
+_lib.swimba_scan_fwd_noalloc_status.argtypes = [_P]
+_lib.swimba_scan_fwd_noalloc_status.restype = ctypes.c_int
+_lib.swimba_scan_fwd_noalloc_status_block.argtypes = []
+_lib.swimba_scan_fwd_noalloc_status_block.restype = ctypes.c_void_p
+_lib.swimba_scan_summary.argtypes = [ctypes.POINTER(swimba_dims), _P, _P, _P, _P, _P, ctypes.POINTER(swimba_weights),
+                                     _P, _P, _P, ctypes.c_size_t, _P]
+_lib.swimba_scan_summary.restype = ctypes.c_int
+_lib.swimba_scan_chain.argtypes = [ctypes.POINTER(swimba_dims), ctypes.c_int32, _P, _P, _P, _P, _P]
+_lib.swimba_scan_chain.restype = ctypes.c_int
+_lib.swimba_separate_proj.argtypes = [ctypes.POINTER(swimba_dims), _P, _P, _P, ctypes.POINTER(swimba_weights), _P,
+                                      _P, _P, _P]
+_lib.swimba_separate_proj.restype = ctypes.c_int
+_lib.swimba_separate_scan.argtypes = [ctypes.POINTER(swimba_dims), _P, _P, _P, _P, _P, _P, _P,
+                                      ctypes.POINTER(swimba_weights), _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.swimba_separate_scan.restype = ctypes.c_int
 _lib.swimba_step.argtypes = [ctypes.POINTER(swimba_dims), _P, _P, _P, _P, _P, _P, _P,
                              ctypes.POINTER(swimba_weights), _P, _P, _P]
 _lib.swimba_step.restype = ctypes.c_int
@@ -190,11 +215,50 @@ def swimba_scan_fwd(dims, x, z, delta, B_mix, C_mix, idx, gates, weights, h0, ou
                                 _ptr(y_pre), _ptr(ws), int(ws_bytes), _stream(stream))
 
 
+def swimba_scan_fwd_zoh(dims, x, z, delta, B_mix, C_mix, idx, gates, weights, h0, out, h_final, y_pre, ws, ws_bytes,
+                        stream=None) -> int:
+    return _lib.swimba_scan_fwd_zoh(ctypes.byref(dims), _ptr(x), _ptr(z), _ptr(delta), _ptr(B_mix), _ptr(C_mix),
+                                    _ptr(idx), _ptr(gates), ctypes.byref(weights), _ptr(h0), _ptr(out),
+                                    _ptr(h_final), _ptr(y_pre), _ptr(ws), int(ws_bytes), _stream(stream))
+
+
 def swimba_scan_fwd_noalloc(dims, x, z, delta, B_mix, C_mix, idx, gates, weights, h0, out, h_final, y_pre,
                             stream=None) -> int:
     return _lib.swimba_scan_fwd_noalloc(ctypes.byref(dims), _ptr(x), _ptr(z), _ptr(delta), _ptr(B_mix), _ptr(C_mix),
                                         _ptr(idx), _ptr(gates), ctypes.byref(weights), _ptr(h0), _ptr(out),
                                         _ptr(h_final), _ptr(y_pre), _stream(stream))
+
+
+def swimba_scan_fwd_noalloc_status(stream=None) -> int:
+    return _lib.swimba_scan_fwd_noalloc_status(_stream(stream))
+
+
+def swimba_scan_fwd_noalloc_status_block() -> int | None:
+    return _lib.swimba_scan_fwd_noalloc_status_block()
+
+
+def swimba_scan_summary(dims, x, delta, B_mix, idx, gates, weights, h_zero, log_decay, ws, ws_bytes,
+                        stream=None) -> int:
+    return _lib.swimba_scan_summary(ctypes.byref(dims), _ptr(x), _ptr(delta), _ptr(B_mix), _ptr(idx), _ptr(gates),
+                                    ctypes.byref(weights), _ptr(h_zero), _ptr(log_decay), _ptr(ws), int(ws_bytes),
+                                    _stream(stream))
+
+
+def swimba_scan_chain(dims, parts, h_zero, log_decay, h0, h_start, stream=None) -> int:
+    return _lib.swimba_scan_chain(ctypes.byref(dims), int(parts), _ptr(h_zero), _ptr(log_decay), _ptr(h0),
+                                  _ptr(h_start), _stream(stream))
+
+
+def swimba_separate_proj(dims, x, idx, gates, weights, delta_j, B_j, C_j, stream=None) -> int:
+    return _lib.swimba_separate_proj(ctypes.byref(dims), _ptr(x), _ptr(idx), _ptr(gates), ctypes.byref(weights),
+                                     _ptr(delta_j), _ptr(B_j), _ptr(C_j), _stream(stream))
+
+
+def swimba_separate_scan(dims, x, z, delta_j, B_j, C_j, idx, gates, weights, h0, out, h_final, y_pre, ws, ws_bytes,
+                         stream=None) -> int:
+    return _lib.swimba_separate_scan(ctypes.byref(dims), _ptr(x), _ptr(z), _ptr(delta_j), _ptr(B_j), _ptr(C_j),
+                                     _ptr(idx), _ptr(gates), ctypes.byref(weights), _ptr(h0), _ptr(out),
+                                     _ptr(h_final), _ptr(y_pre), _ptr(ws), int(ws_bytes), _stream(stream))
 
 
 def swimba_step(dims, x, z, delta, B_mix, C_mix, idx, gates, weights, h, out, stream=None) -> int:

@@ -63,6 +63,30 @@ def oracle_layer(case: Case, rows=None, channels=None) -> dict:
     return O.layer_forward(case.x64(rows), case.z64(rows), case.weights64(), case.cfg.top_k, h0=h0, channels=channels)
 
 
+def oracle_route_proj(case: Case, rows, chunk=8192) -> dict:
+    """The oracle's routing and mixed projections (idx, gates, dt_mix, B_mix, C_mix, delta) for
+    every token of the given batch rows, all channels. Tokens are processed in chunks so that the
+    fp64 temporaries stay bounded; each token's result depends only on that token."""
+    cfg = case.cfg
+    W = case.weights64()
+    R, N = cfg.dt_rank, cfg.d_state
+    parts = {k: [] for k in ("idx", "gates", "dt_mix", "B_mix", "C_mix")}
+    for b in rows:
+        xs = case.x[b]
+        for t0 in range(0, xs.shape[0], chunk):
+            x64 = synth.widen(xs[t0:t0 + chunk], cfg.io_dtype)
+            idx, gates, _ = O.route(x64, W["W_r"], cfg.top_k)
+            pr = O.expert_projections(x64, idx, gates, W["W_x"], W["W_dt"], W["b_dt"], R, N)
+            parts["idx"].append(idx)
+            parts["gates"].append(gates)
+            for k in ("dt_mix", "B_mix", "C_mix"):
+                parts[k].append(pr[k])
+    L = case.x.shape[1]
+    out = {k: np.concatenate(v).reshape(len(rows), L, *v[0].shape[1:]) for k, v in parts.items()}
+    out["delta"] = O.softplus(out["dt_mix"])
+    return out
+
+
 def scaled_err(got, ref):
     """max |got - ref| / (1 + |ref|)."""
     got = np.asarray(got, dtype=np.float64)

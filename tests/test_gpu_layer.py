@@ -12,7 +12,7 @@ from oracle import swimba_oracle as O
 from oracle.conditioning import condition_router_margin
 from parameter_space_moe_swimba_b200 import synth
 from parameter_space_moe_swimba_b200.configs import CONFIGS, LayerConfig, dense_variant
-from tests.swimba_cases import TOL_Y, make_case, oracle_layer, rel_rms_err, scaled_err
+from tests.swimba_cases import TOL_Y, make_case, oracle_layer, oracle_route_proj, rel_rms_err, scaled_err
 
 pytestmark = pytest.mark.gpu
 
@@ -109,36 +109,59 @@ def _sampled_channels(D, n, seed):
     return np.unique(np.concatenate([[0, 1, 31, 32, D - 1], rng.choice(D, n, replace=False)]))
 
 
-def test_mamba1p4b_like_full_size_sampled(S):
+def check_route_proj_all_tokens(case, got):
+    """Every token of every batch row: router indices bit-exact, gates, B_mix and C_mix, and Δ on
+    every channel, against the oracle's routing and mixed projections."""
+    cfg = case.cfg
+    worst = {"gates": 0.0, "B_mix": 0.0, "C_mix": 0.0, "delta": 0.0}
+    for b in range(cfg.batch):
+        ref = oracle_route_proj(case, [b])
+        np.testing.assert_array_equal(got["idx"][b:b + 1], ref["idx"], err_msg=f"batch row {b}")
+        worst["gates"] = max(worst["gates"], float(np.max(np.abs(got["gates"][b:b + 1] - ref["gates"]))))
+        for k in ("B_mix", "C_mix", "delta"):
+            worst[k] = max(worst[k], rel_rms_err(got[k][b:b + 1], ref[k]))
+    print(cfg.name, "all tokens", {k: f"{v:.2e}" for k, v in worst.items()})
+    assert worst["gates"] <= 1e-5
+    assert worst["B_mix"] <= 1e-4 and worst["C_mix"] <= 1e-4
+    assert worst["delta"] <= (1e-5 if cfg.io_dtype == "f32" else 1e-2)
+
+
+def test_mamba1p4b_like_full_size(S):
+    """Routing and projections on all 32768 tokens; the scan on every channel of batch row 0 and
+    on sampled channels of the last row."""
     cfg = CONFIGS["mamba1p4b_like"]
     case = make_case(cfg)
     got = run_gpu_layer(S, case)
-    rows = [0, cfg.batch - 1]
+    check_route_proj_all_tokens(case, got)
+    check_layer(case, got, oracle_layer(case, rows=[0]), rows=[0])
+    last = [cfg.batch - 1]
     ch = _sampled_channels(cfg.d_inner, 27, 11)
-    check_layer(case, got, oracle_layer(case, rows=rows, channels=ch), rows=rows, channels=ch)
+    check_layer(case, got, oracle_layer(case, rows=last, channels=ch), rows=last, channels=ch)
 
 
-def test_mamba1p4b_like_dense_e1_sampled(S):
+def test_mamba1p4b_like_dense_e1(S):
     cfg = dense_variant(CONFIGS["mamba1p4b_like"])
     case = make_case(cfg)
     got = run_gpu_layer(S, case)
     assert np.all(got["idx"] == 0) and np.all(got["gates"] == 1.0)
-    rows = [3]
-    ch = _sampled_channels(cfg.d_inner, 27, 12)
-    check_layer(case, got, oracle_layer(case, rows=rows, channels=ch), rows=rows, channels=ch)
+    check_route_proj_all_tokens(case, got)
+    check_layer(case, got, oracle_layer(case, rows=[3]), rows=[3])
 
 
-def test_long_seq_65536_sampled(S):
+def test_long_seq_65536_full(S):
+    """All 65536 tokens and all 2048 channels (the sequence is split into segments whose start
+    states are carried from one to the next)."""
     cfg = CONFIGS["long_seq_65536"]
     case = make_case(cfg)
     got = run_gpu_layer(S, case)
-    ch = _sampled_channels(cfg.d_inner, 11, 13)
-    check_layer(case, got, oracle_layer(case, channels=ch), channels=ch)
+    check_route_proj_all_tokens(case, got)
+    check_layer(case, got, oracle_layer(case))
 
 
 def test_decode_b256_1000_steps(S):
-    """1000 consecutive decode steps on the cached state; every step's output of the sampled
-    sequences and their final state are compared with the oracle's sequential run."""
+    """1000 consecutive decode steps on the cached state; every step's router indices and output of
+    32 sequences spread over the batch, and their final state, are compared with the oracle's
+    sequential run."""
     cfg = CONFIGS["decode_b256"]
     steps = cfg.decode_steps
     w = synth.draw_weights(cfg)
@@ -148,7 +171,8 @@ def test_decode_b256_1000_steps(S):
     buf = S.LayerBuffers(dims, torch.bfloat16)
     h0 = synth.draw_h0(cfg)
     h = torch.from_numpy(h0).cuda()
-    rows = [0, 77, 255]
+    rows = np.unique(np.linspace(0, cfg.batch - 1, 32).astype(int)).tolist()
+    assert len(rows) == 32
     W64 = {
         "W_r": w.W_r.astype(np.float64), "W_x": synth.widen(w.W_x, "bf16"), "W_dt": synth.widen(w.W_dt, "bf16"),
         "b_dt": w.b_dt.astype(np.float64), "A": w.A.astype(np.float64), "D_skip": w.D_skip.astype(np.float64),
@@ -203,6 +227,15 @@ EDGE = [
     # the one-CTA bucketing of the tensor-core projection covers up to 4096 tokens: both sides of it
     (2, 2048, 64, 16, 16, 4, 2, "bf16", "bf16"),
     (1, 4097, 64, 16, 16, 8, 1, "bf16", "bf16"),
+    # the fast scan (bf16, N = 16, k <= 2, D % 16 == 0): one token and one 16-channel warp tile;
+    # E = 16 (the widest TMEM window) with a 1-token last segment; hundreds of 16-token segments
+    # chained by the carry pass (ragged last segment); E = 1; many sequences, no segments, a
+    # ragged last chunk
+    (1, 1, 16, 16, 16, 2, 1, "bf16", "bf16"),
+    (2, 17, 48, 16, 16, 16, 2, "bf16", "bf16"),
+    (3, 4111, 32, 16, 16, 5, 2, "bf16", "bf16"),
+    (1, 5000, 16, 16, 16, 1, 1, "bf16", "bf16"),
+    (64, 40, 512, 16, 32, 8, 1, "bf16", "bf16"),
 ]
 
 
@@ -217,7 +250,8 @@ def test_edge_shapes(S, shape, with_h0):
 
 @pytest.mark.parametrize("name", ["mamba130m_like", "tiny_fp32"])
 def test_layer_is_deterministic(S, name):
-    """Token bucketing uses atomics, but every output row depends only on its own token."""
+    """Two runs give bitwise equal results: the token bucketing is a stable counting sort (the slot
+    order does not depend on scheduling) and every output row depends only on its own token."""
     cfg = CONFIGS[name]
     if cfg.batch * cfg.seqlen > 4096:
         cfg = cfg.with_(batch=2, seqlen=1024)
@@ -312,3 +346,44 @@ def test_bad_arguments_are_rejected_before_launch(S):
     bc = torch.empty((1, 128, 16), device="cuda")
     assert S.swimba_mixed_proj(dims, x, idx, g, W.struct(), d, bc, bc, ws, 16) == 4
     assert S.swimba_get_device_status(ws) == 0
+
+
+@pytest.mark.parametrize("shape", [
+    (2, 333, 1536, 16, 48, 8, 2, "bf16", "bf16"),  # fast path, several segments per sequence
+    (8, 300, 4096, 16, 128, 8, 2, "bf16", "bf16"),  # fast path, no segments
+    (2, 45, 40, 5, 3, 3, 3, "f32", "f32"),          # generic path
+], ids=lambda s: "B{}L{}D{}N{}R{}E{}k{}{}{}".format(*s))
+def test_zoh_scan_on_oracle_streams(S, shape):
+    """swimba_scan_fwd_zoh fed with the oracle's routing and mixed streams, against the oracle's
+    scan with the zero-order-hold injection; the Euler scan on the same streams differs from it."""
+    B, L, D, N, R, E, k, io, wd = shape
+    cfg = LayerConfig("zoh", B, L, D, N, R, E, k, io, wd, seed=17, cached_state=True)
+    case = make_case(cfg, a_mode="random", with_h0=True)
+    W = case.weights64()
+    ref = oracle_layer(case, channels=None)
+    y_z, out_z, h_z, _ = O.selective_scan(case.x64(), case.z64(), ref["dt_mix"], ref["B_mix"], ref["C_mix"],
+                                          ref["idx"], ref["gates"], W["A"], W["D_skip"], h0=case.h0,
+                                          injection="zoh")
+    dims = S.make_dims(cfg)
+    Wd = S.upload_weights(case.w)
+    f = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dt).cuda()
+    io_t = torch.bfloat16 if io == "bf16" else torch.float32
+    out = torch.empty((B, L, D), dtype=io_t, device="cuda")
+    y = torch.empty((B, L, D), dtype=torch.float32, device="cuda")
+    hf = torch.empty((B, D, N), dtype=torch.float32, device="cuda")
+    ws = S.new_workspace(dims)
+    S.check(S.swimba_scan_fwd_zoh(dims, S.to_device(case.x, io), S.to_device(case.z, io), f(ref["delta"]),
+                                  f(ref["B_mix"]), f(ref["C_mix"]), f(ref["idx"], torch.int32), f(ref["gates"]),
+                                  Wd.struct(), f(case.h0), out, hf, y, ws, ws.numel()), "scan_fwd_zoh")
+    torch.cuda.synchronize()
+    assert S.swimba_get_device_status(ws) == 0
+    tol = 1e-4
+    ey = scaled_err(y.cpu().numpy(), y_z)
+    ess = rel_rms_err(y.cpu().numpy() - W["D_skip"] * case.x64(), y_z - W["D_skip"] * case.x64())
+    eh = rel_rms_err(hf.cpu().numpy(), h_z)
+    eo = scaled_err(out.float().cpu().numpy(), out_z)
+    print(shape, {"y": ey, "y_ssm": ess, "h_final": eh, "out": eo})
+    assert ey <= tol and ess <= tol and eh <= tol
+    assert eo <= (1e-4 if io == "f32" else TOL_Y["bf16"])
+    # the two injections are different discretisations
+    assert rel_rms_err(ref["h_final"], h_z) > 10 * tol

@@ -52,17 +52,39 @@ def test_noalloc_scan_equals_workspace_scan_on_two_calls(S):
 
 
 def test_noalloc_scan_refuses_a_shape_whose_scratch_does_not_fit(S):
-    # one 27648-channel sequence: the scan splits it into segments whose carries need ~10.6 MB
-    cfg = LayerConfig("wide", 1, 64, 27648, 16, 16, 8, 2, "bf16", "bf16", seed=3)
+    # one wide sequence: when its channels alone cannot fill the GPU the scan splits it into
+    # segments, whose carries need 3 x S x D x 16 floats; the width that exceeds the 8 MiB array
+    # depends on the SM count, so it is searched for
+    L = 256
+    found = None
+    for D in (4096, 8192, 12288, 16384, 18432, 24576, 32768, 49152):
+        cfg = LayerConfig("wide", 1, L, D, 16, 16, 8, 2, "bf16", "bf16", seed=3)
+        if S.swimba_workspace_size(S.make_dims(cfg), S.SWIMBA_OP_SCAN) > (8 << 20):
+            found = cfg
+            break
+    if found is None:
+        pytest.skip("no single-sequence shape on this GPU needs more than the fixed scratch")
+    cfg, D = found, found.d_inner
     dims = S.make_dims(cfg)
-    assert S.swimba_workspace_size(dims, S.SWIMBA_OP_SCAN) > (8 << 20)
     dev = dict(device="cuda")
-    x = torch.zeros((1, 64, 27648), dtype=torch.bfloat16, **dev)
+    x = torch.zeros((1, L, D), dtype=torch.bfloat16, **dev)
     f = lambda *shape: torch.zeros(shape, dtype=torch.float32, **dev)
-    idx = torch.zeros((1, 64, 2), dtype=torch.int32, **dev)
+    idx = torch.zeros((1, L, 2), dtype=torch.int32, **dev)
     w = synth.draw_weights(cfg.with_(d_inner=64))  # tables are never read: the call stops first
     W = S.upload_weights(w)
-    st = S.swimba_scan_fwd_noalloc(dims, x, x, f(1, 64, 27648), f(1, 64, 16), f(1, 64, 16), idx, f(1, 64, 2),
+    st = S.swimba_scan_fwd_noalloc(dims, x, x, f(1, L, D), f(1, L, 16), f(1, L, 16), idx, f(1, L, 2),
                                    W.struct(), None, torch.empty_like(x), None, None)
     assert st == 4  # SWIMBA_ERR_WORKSPACE
     assert "fixed array holds" in S.swimba_last_error_string()
+
+
+def test_noalloc_status_reports_a_wait_that_gave_up(S):
+    """A bounded wait that runs out on the fixed array's status block is reported by
+    swimba_scan_fwd_noalloc_status (then cleared), and the next call works."""
+    block = S.swimba_scan_fwd_noalloc_status_block()
+    assert block
+    assert S.swimba_check_wait_timeout(block, 256, 20_000_000) == 0
+    assert S.swimba_scan_fwd_noalloc_status() == 6  # SWIMBA_ERR_TIMEOUT
+    assert S.swimba_scan_fwd_noalloc_status() == 0  # cleared
+    test_noalloc_scan_equals_workspace_scan_on_two_calls(S)
+    assert S.swimba_scan_fwd_noalloc_status() == 0
