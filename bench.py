@@ -53,6 +53,9 @@ def parse():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--report", action="store_true",
                     help="per-workload table (one JSON line each): every workload, decode steps, E sweep")
+    ap.add_argument("--report-ssd", action="store_true", help="only the SSD-form line")
+    ap.add_argument("--report-decode", action="store_true",
+                    help="only the decode line (--steps decode steps of the decode workload)")
     ap.add_argument("--report-separate", action="store_true",
                     help="only the separate-SSM comparison line (Teorema 2)")
     ap.add_argument("--report-block", action="store_true",
@@ -528,6 +531,49 @@ def report_separate(torch, S, cfg, peaks, flush, reps, warmup):
     }
 
 
+SSD_WORKLOAD = {"name": "swimba_ssd_nemotron_like", "batch": 8, "seqlen": 4096, "heads": 64, "head_dim": 64,
+                "d_state": 128}
+
+
+def report_ssd(torch, S, peaks, flush, reps, warmup, w=SSD_WORKLOAD):
+    """Swimba on the Mamba-2 SSD form (swimba_ssd_scan): B=8, L=4096, 64 heads of 64 channels,
+    state 128, one active expert per token. FLOPs counted as computed per (chunk of 128, head):
+    C Bᵀ (2 Q² N), W X (2 Q² P), C S_inᵀ (2 Q N P), Bᵀ X_w (2 N Q P)."""
+    B, L, H, P, N = w["batch"], w["seqlen"], w["heads"], w["head_dim"], w["d_state"]
+    inp = synth.draw_ssd_inputs(B, L, H, P, N, seed=9)
+    dims = S.swimba_ssd_dims(batch=B, seqlen=L, n_heads=H, head_dim=P, d_state=N, top_k=1)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to("cuda:0")
+    X, Bm, C = (S.to_device(a, "bf16", "cuda:0") for a in (inp.X, inp.B, inp.C_mix))
+    g, dl, A, Dk, S0 = t(inp.gates), t(inp.delta), t(inp.A), t(inp.D_skip), t(inp.S0)
+    y = torch.empty((B, L, H, P), dtype=torch.float32, device="cuda:0")
+    sf = torch.empty((B, H, P, N), dtype=torch.float32, device="cuda:0")
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda:0")
+    s = torch.cuda.current_stream()
+
+    def run(ev):
+        if ev is not None:
+            ev[0].record(s)
+        S.check(S.swimba_ssd_scan(dims, X, Bm, C, g, dl, A, Dk, S0, y, sf, ws, ws.numel(), s), "ssd_scan")
+        if ev is not None:
+            ev[1].record(s)
+
+    (ms,), _ = _median_kernel_ms(torch, run, reps, warmup, flush, 2)
+    S.check(S.swimba_get_device_status(ws, s), "device status")
+    Q = 128
+    chunks = -(-L // Q)
+    flops = B * H * chunks * (2 * Q * Q * N + 2 * Q * Q * P + 2 * Q * N * P + 2 * N * Q * P)
+    nbytes = B * L * (H * P * 2 + 2 * N * 2 + 4 + H * 4 + H * P * 4) + 2 * B * H * P * N * 4
+    sec = ms / 1e3
+    return {
+        "report": "ssd", "workload": w["name"], "batch": B, "seqlen": L, "heads": H, "head_dim": P, "d_state": N,
+        "top_k": 1, "tokens": B * L, "ssd_us": 1e3 * ms, "tokens_per_s": B * L / sec,
+        "tflops": flops / sec / 1e12, "frac_of_tc_peak": flops / sec / 1e12 / peaks["bf16_tflops"],
+        "gbs": nbytes / sec / 1e9, "frac_of_hbm": nbytes / sec / 1e9 / peaks["hbm_gbs"],
+        "flops_per_launch": flops, "bytes_per_launch": nbytes,
+        "median_of": reps, "l2": "flushed (256 MB write) before every run",
+    }
+
+
 def report_decode(torch, S, cfg, peaks, flush, steps):
     """``steps`` decode steps (route -> mixed_proj -> step) on one cached state, L2 flushed before
     every step; the same x, z every step (draws of step 0)."""
@@ -676,6 +722,8 @@ def run_report(args):
     print(json.dumps(report_block(torch, S, CONFIGS["mamba1p4b_like"], 2048, 4, peaks, flush, reps, args.warmup)),
           flush=True)
     print(json.dumps(report_block_decode(torch, S, CONFIGS["decode_b256"], 2048, 4, peaks, flush, 200)), flush=True)
+    # Swimba on the Mamba-2 SSD form
+    print(json.dumps(report_ssd(torch, S, peaks, flush, reps, args.warmup)), flush=True)
     # Theorem 2 against the design it is set against: one trajectory per expert
     print(json.dumps(report_separate(torch, S, CONFIGS["mamba1p4b_like"], peaks, flush, reps, args.warmup)),
           flush=True)
@@ -698,6 +746,23 @@ def main():
         return run_report(args)
     if args.report_block:
         return run_report_block(args)
+    if args.report_ssd:
+        import torch
+
+        from parameter_space_moe_swimba_b200 import swimba as S
+
+        torch.cuda.set_device(0)
+        print(json.dumps(report_ssd(torch, S, load_peaks(), L2Flush(torch, "cuda:0"), 20, args.warmup)), flush=True)
+        return 0
+    if args.report_decode:
+        import torch
+
+        from parameter_space_moe_swimba_b200 import swimba as S
+
+        torch.cuda.set_device(0)
+        print(json.dumps(report_decode(torch, S, CONFIGS["decode_b256"], load_peaks(), L2Flush(torch, "cuda:0"),
+                                       args.steps)), flush=True)
+        return 0
     if args.report_separate:
         import torch
 

@@ -232,6 +232,41 @@ swimba_status swimba_separate_scan(const swimba_dims *dims, const void *x, const
                                    const float *h0, void *out, float *h_final, float *y_pre, void *ws,
                                    size_t ws_bytes, void *stream);
 
+/* ---- Swimba on the Mamba-2 state-space-dual form ---------------------------------------------
+ * ("Swimba: Switch Mamba Model Scales State Space Models", Spanish summary §2 "Arquitectura de
+ * Swimba": built on Mamba-2 and its state space duality; expert-specific streams B^(e), C^(e),
+ * X^(e); the transition A shared by the experts and over time; Dutch summary §2 "Architectuur
+ * Implementatie": the SSD computation and chunked processing carry over.) Heads of P channels,
+ * one negative scalar A_h per head, one step delta_t[h] per token, the active expert's streams
+ * X_t [H, P] and B_t [N], gate g_t and the gate-mixed readout C_mix,t [N]:
+ *   S_t[h] = exp(delta_t[h] A_h) S_{t-1}[h] + delta_t[h] g_t X_t[h] (outer) B_t
+ *   y_t[h] = S_t[h] C_mix,t + D_skip[h] g_t X_t[h]
+ * evaluated in chunks of 128 tokens on the tensor cores (the decay-masked C B^T products, the
+ * carried state's readout and the state update are bf16 MMAs with fp32 accumulation; the state is
+ * carried in fp32). Supported: head_dim 64, d_state 128, top_k 1 (the pages' model routes each
+ * token to one expert); anything else returns SWIMBA_ERR_UNSUPPORTED. */
+typedef struct {
+  int64_t batch;    /* B */
+  int64_t seqlen;   /* L */
+  int32_t n_heads;  /* H */
+  int32_t head_dim; /* P */
+  int32_t d_state;  /* N */
+  int32_t top_k;    /* k (active experts per token) */
+} swimba_ssd_dims;
+
+/*   X       [B, L, k, H, P] bf16: the active expert's input stream X^(e_t)_t       (in)
+ *   B_j     [B, L, k, N] bf16: its state-input stream B^(e_t)_t                   (in)
+ *   C_mix   [B, L, N] bf16: the gate-mixed readout stream                         (in)
+ *   gates   [B, L, k] fp32; delta [B, L, H] fp32 (> 0); A [H] fp32 (< 0); D_skip [H] fp32
+ *   S0      [B, H, P, N] fp32 start state, or NULL for zeros                       (in)
+ *   y       [B, L, H, P] fp32                                                      (out)
+ *   S_final [B, H, P, N] fp32 state after the last token, or NULL                  (out)
+ *   ws: at least 256 bytes (the status block). One CTA per (sequence, head). */
+swimba_status swimba_ssd_scan(const swimba_ssd_dims *dims, const void *X, const void *B_j,
+                              const void *C_mix, const float *gates, const float *delta,
+                              const float *A, const float *D_skip, const float *S0, float *y,
+                              float *S_final, void *ws, size_t ws_bytes, void *stream);
+
 /* One decode step (dims->seqlen must be 1): the scan for a single token per sequence, continuing
  * from and overwriting the cached state h [B, D, N] fp32. Other arguments as swimba_scan_fwd. */
 swimba_status swimba_step(const swimba_dims *dims, const void *x, const void *z, const float *delta,

@@ -23,6 +23,10 @@ cudaError_t separate_scan_entry(const void* x, const void* z, const float* dj, c
                                 const int32_t* idx, const float* gates, const float* A, const float* D_skip,
                                 const float* h0, void* out, float* h_final, float* y_pre, void* status, int64_t L,
                                 int B, int D, int N, int E, int k, bool io_bf16, cudaStream_t s);
+bool ssd_supported(int P, int N, int k);
+cudaError_t run_ssd(const void* X, const void* Bm, const void* Cmix, const float* gates, const float* delta,
+                    const float* A, const float* D_skip, const float* S0, float* y, float* S_final, void* status,
+                    int64_t L, int B, int H, cudaStream_t s);
 }  // namespace swimba
 
 namespace swimba {
@@ -321,6 +325,24 @@ swimba_status swimba_separate_scan(const swimba_dims* dims, const void* x, const
                                          y_pre, ws, dims->seqlen, (int)dims->batch, dims->d_inner, dims->d_state,
                                          dims->n_experts, dims->top_k, dims->io_dtype == SWIMBA_BF16,
                                          static_cast<cudaStream_t>(stream)));
+}
+
+swimba_status swimba_ssd_scan(const swimba_ssd_dims* d, const void* X, const void* B_j, const void* C_mix,
+                              const float* gates, const float* delta, const float* A, const float* D_skip,
+                              const float* S0, float* y, float* S_final, void* ws, size_t ws_bytes, void* stream) {
+  if (d == nullptr || d->batch <= 0 || d->seqlen <= 0 || d->n_heads <= 0 || d->head_dim <= 0 || d->d_state <= 0 ||
+      d->top_k <= 0)
+    return SWIMBA_ERR_INVALID_ARG;
+  if (!X || !B_j || !C_mix || !gates || !delta || !A || !D_skip || !y) return SWIMBA_ERR_INVALID_ARG;
+  if (!ssd_supported(d->head_dim, d->d_state, d->top_k) || d->batch * d->n_heads > (int64_t(1) << 30) ||
+      d->batch * d->seqlen > (int64_t(1) << 31))
+    return SWIMBA_ERR_UNSUPPORTED;
+  if (ws == nullptr || ws_bytes < kStatusBytes) return SWIMBA_ERR_WORKSPACE;
+  if (!aligned16(ws) || !aligned16(X) || !aligned16(B_j) || !aligned16(C_mix) || !aligned16(y) ||
+      (S0 && !aligned16(S0)) || (S_final && !aligned16(S_final)))
+    return SWIMBA_ERR_ALIGN;
+  return cuda_status(run_ssd(X, B_j, C_mix, gates, delta, A, D_skip, S0, y, S_final, ws, d->seqlen, (int)d->batch,
+                             d->n_heads, static_cast<cudaStream_t>(stream)));
 }
 
 swimba_status swimba_step(const swimba_dims* dims, const void* x, const void* z, const float* delta,

@@ -60,6 +60,11 @@
 #ifndef SWIMBA_SCAN_NPOLY
 #define SWIMBA_SCAN_NPOLY 0
 #endif
+// 1: the chunk's per-token expert columns and gates reach the lanes by warp shuffles from the
+// lanes that hold them, instead of a broadcast shared-memory load per token.
+#ifndef SWIMBA_SCAN_META_SHFL
+#define SWIMBA_SCAN_META_SHFL 0
+#endif
 // 1: with E <= 8 experts, keep the transition rows in registers instead of tensor memory.
 #ifndef SWIMBA_SCAN_AREG
 #define SWIMBA_SCAN_AREG 0
@@ -97,7 +102,7 @@ struct Stage {
 // Per-warp area after the rings: partial readouts and two output tiles (the TMA store of one may
 // still be reading while the next is written).
 struct Epi {
-  static constexpr int P = 0;                        // f32 [LC][kPRow]: [token][state quarter][16 channels]
+  static constexpr int P = 0;                        // f32 [LC][kPRow]: [token][channel pair][state quarter][2]
   static constexpr int O = P + LC * kPRow * 4;       // bf16 [2][LC][16]
   static constexpr int BYTES = O + 2 * LC * kCPW * 2;
   static_assert(O % 128 == 0 && BYTES % 128 == 0, "readout area layout");
@@ -391,6 +396,14 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       phase_bits ^= 1u << sidx;
       const uint8_t* st = ring + sidx * St::BYTES;
       const int4* meta = reinterpret_cast<const int4*>(st + St::META);
+#if SWIMBA_SCAN_META_SHFL
+      // lane t < 16 holds token t's {columns packed, g0, g1}
+      int3 mreg = make_int3(0, 0, 0);
+      if (lane < LC) {
+        const int4 mm = meta[lane];
+        mreg = make_int3(mm.x | (mm.y << 16), mm.z, mm.w);
+      }
+#endif
       const uint32_t* xs2 = reinterpret_cast<const uint32_t*>(st + St::X);
       const float2* ds2 = reinterpret_cast<const float2*>(st + St::DL);
       const float4* bsm = reinterpret_cast<const float4*>(st + St::B);
@@ -399,7 +412,15 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
 
       // issue token t's loads (TMEM loads are waited for by the caller)
       auto load_tok = [&](TokIn& tk, int t) {
+#if SWIMBA_SCAN_META_SHFL
+        {
+          const int c01 = __shfl_sync(0xffffffffu, mreg.x, t);
+          tk.m = make_int4(c01 & 0xffff, c01 >> 16, __shfl_sync(0xffffffffu, mreg.y, t),
+                           __shfl_sync(0xffffffffu, mreg.z, t));
+        }
+#else
         tk.m = meta[t];
+#endif
         if (!AREG) {
           tmem_ld8_nowait(tbase + (uint32_t)tk.m.x, tk.ar[0]);
           if (K == 2) tmem_ld8_nowait(tbase + (uint32_t)tk.m.y, tk.ar[1]);
@@ -462,7 +483,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
           y = __ffma2_rn(f2(cur.cq.y), h[1], y);
           y = __ffma2_rn(f2(cur.cq.z), h[2], y);
           y = __ffma2_rn(f2(cur.cq.w), h[3], y);
-          *reinterpret_cast<float2*>(psm + t * kPRow + q * kCPW + 2 * cp) = y;
+          *reinterpret_cast<float2*>(psm + t * kPRow + cp * 8 + q * 2) = y;
         }
         if (t + 1 < LC) {
           if (!AREG) tmem_wait_ld();
@@ -476,18 +497,14 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
         __syncwarp();
         float2 yv[4];
         {
-          const float4* pr = reinterpret_cast<const float4*>(psm + rt * kPRow + rc);
-          float4 s0 = pr[0], s1 = pr[1];
+          // channel pair i of this lane's 8 channels: (c0, c1) partials of the four state quarters
+          const float4* pr = reinterpret_cast<const float4*>(psm + rt * kPRow + (rc / 2) * 8);
 #pragma unroll
-          for (int qq = 1; qq < 4; ++qq) {
-            const float4 v0 = pr[qq * (kCPW / 4)], v1 = pr[qq * (kCPW / 4) + 1];
-            s0 = make_float4(s0.x + v0.x, s0.y + v0.y, s0.z + v0.z, s0.w + v0.w);
-            s1 = make_float4(s1.x + v1.x, s1.y + v1.y, s1.z + v1.z, s1.w + v1.w);
+          for (int i = 0; i < 4; ++i) {
+            const float4 a = pr[2 * i], b = pr[2 * i + 1];
+            yv[i] = __fadd2_rn(__fadd2_rn(make_float2(a.x, a.y), make_float2(a.z, a.w)),
+                               __fadd2_rn(make_float2(b.x, b.y), make_float2(b.z, b.w)));
           }
-          yv[0] = make_float2(s0.x, s0.y);
-          yv[1] = make_float2(s0.z, s0.w);
-          yv[2] = make_float2(s1.x, s1.y);
-          yv[3] = make_float2(s1.z, s1.w);
         }
         float2 xf[4], zf[4];
         bf16x8_to_float2(*reinterpret_cast<const uint4*>(st + St::X + (rt * kCPW + rc) * 2), xf);

@@ -358,24 +358,20 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
         }
         // the next token may advance the same expert: its state must be back in TMEM first
         tmem_wait_st();
-        *reinterpret_cast<float2*>(psm + t * kPRow + q * kCPW + 2 * cp) = y;
+        *reinterpret_cast<float2*>(psm + t * kPRow + cp * 8 + q * 2) = y;
       }
       // readout pass: lane = (token rt, channels rc..rc+7)
       __syncwarp();
       float2 yv[4];
       {
-        const float4* pr = reinterpret_cast<const float4*>(psm + rt * kPRow + rc);
-        float4 s0 = pr[0], s1 = pr[1];
+        // channel pair i of this lane's 8 channels: (c0, c1) partials of the four state quarters
+        const float4* pr = reinterpret_cast<const float4*>(psm + rt * kPRow + (rc / 2) * 8);
 #pragma unroll
-        for (int qq = 1; qq < 4; ++qq) {
-          const float4 v0 = pr[qq * (kCPW / 4)], v1 = pr[qq * (kCPW / 4) + 1];
-          s0 = make_float4(s0.x + v0.x, s0.y + v0.y, s0.z + v0.z, s0.w + v0.w);
-          s1 = make_float4(s1.x + v1.x, s1.y + v1.y, s1.z + v1.z, s1.w + v1.w);
+        for (int i = 0; i < 4; ++i) {
+          const float4 a = pr[2 * i], b = pr[2 * i + 1];
+          yv[i] = __fadd2_rn(__fadd2_rn(make_float2(a.x, a.y), make_float2(a.z, a.w)),
+                             __fadd2_rn(make_float2(b.x, b.y), make_float2(b.z, b.w)));
         }
-        yv[0] = make_float2(s0.x, s0.y);
-        yv[1] = make_float2(s0.z, s0.w);
-        yv[2] = make_float2(s1.x, s1.y);
-        yv[3] = make_float2(s1.z, s1.w);
       }
       const uint4 xq = *reinterpret_cast<const uint4*>(st + St::X + (rt * kCPW + rc) * 2);
       const uint4 zq = *reinterpret_cast<const uint4*>(st + St::Z + (rt * kCPW + rc) * 2);

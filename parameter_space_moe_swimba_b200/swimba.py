@@ -51,6 +51,7 @@ EXPORTED = [
     "swimba_scan_fwd_noalloc_status_block",
     "swimba_scan_summary",
     "swimba_scan_chain",
+    "swimba_ssd_scan",
     "swimba_separate_proj",
     "swimba_separate_scan",
     "swimba_step",
@@ -78,6 +79,17 @@ class swimba_dims(ctypes.Structure):
         ("top_k", ctypes.c_int32),
         ("io_dtype", ctypes.c_int32),
         ("w_dtype", ctypes.c_int32),
+    ]
+
+
+class swimba_ssd_dims(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int64),
+        ("seqlen", ctypes.c_int64),
+        ("n_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("d_state", ctypes.c_int32),
+        ("top_k", ctypes.c_int32),
     ]
 
 
@@ -118,6 +130,8 @@ _lib.swimba_scan_summary.argtypes = [ctypes.POINTER(swimba_dims), _P, _P, _P, _P
 _lib.swimba_scan_summary.restype = ctypes.c_int
 _lib.swimba_scan_chain.argtypes = [ctypes.POINTER(swimba_dims), ctypes.c_int32, _P, _P, _P, _P, _P]
 _lib.swimba_scan_chain.restype = ctypes.c_int
+_lib.swimba_ssd_scan.argtypes = [ctypes.POINTER(swimba_ssd_dims)] + [_P] * 10 + [_P, ctypes.c_size_t, _P]
+_lib.swimba_ssd_scan.restype = ctypes.c_int
 _lib.swimba_separate_proj.argtypes = [ctypes.POINTER(swimba_dims), _P, _P, _P, ctypes.POINTER(swimba_weights), _P,
                                       _P, _P, _P]
 _lib.swimba_separate_proj.restype = ctypes.c_int
@@ -247,6 +261,12 @@ def swimba_scan_summary(dims, x, delta, B_mix, idx, gates, weights, h_zero, log_
 def swimba_scan_chain(dims, parts, h_zero, log_decay, h0, h_start, stream=None) -> int:
     return _lib.swimba_scan_chain(ctypes.byref(dims), int(parts), _ptr(h_zero), _ptr(log_decay), _ptr(h0),
                                   _ptr(h_start), _stream(stream))
+
+
+def swimba_ssd_scan(dims, X, B_j, C_mix, gates, delta, A, D_skip, S0, y, S_final, ws, ws_bytes, stream=None) -> int:
+    return _lib.swimba_ssd_scan(ctypes.byref(dims), _ptr(X), _ptr(B_j), _ptr(C_mix), _ptr(gates), _ptr(delta), _ptr(A),
+                                _ptr(D_skip), _ptr(S0), _ptr(y), _ptr(S_final), _ptr(ws), int(ws_bytes),
+                                _stream(stream))
 
 
 def swimba_separate_proj(dims, x, idx, gates, weights, delta_j, B_j, C_j, stream=None) -> int:

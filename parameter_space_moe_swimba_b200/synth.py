@@ -20,6 +20,11 @@ Initialisation recipe (shared by every workload):
   conv bias [D] ~ U(-1/sqrt(W), 1/sqrt(W)), fp32; a carried conv state [B, W-1, D] ~ N(0, 1) in
   the io dtype.
 
+* Swimba on the Mamba-2 SSD form (heads of P channels, state N, one active expert per token):
+  X [B, L, 1, H, P], B [B, L, 1, N] and the mixed readout C_mix [B, L, N] ~ N(0, 1) in bf16;
+  gates 1 (top-1); step delta [B, L, H] ~ logU(1e-3, 1e-1) per (token, head); A_h = -U(1, 16) per
+  head; D_skip [H] ~ N(0, 1); start state S0 [B, H, P, N] ~ N(0, 0.1), fp32.
+
 N(m, s2) names the variance. bf16 values are rounded to nearest-even directly from the fp64 draw.
 
 Random streams: every group of draws has its own PCG64 stream keyed by (seed, stream id, ...), so a
@@ -43,6 +48,7 @@ STREAM_BLOCK_WEIGHTS = 5
 STREAM_BLOCK_INPUT = 6
 STREAM_CONV_STATE = 7
 STREAM_BLOCK_REDRAW = 8
+STREAM_SSD = 9
 
 _BF16_MIN_NORMAL = 2.0 ** -126
 _BF16_MAX = float.fromhex("0x1.fep127")
@@ -229,3 +235,29 @@ def redraw_u_row(cfg: LayerConfig, d_model: int, b: int, t: int, attempt: int) -
     """A fresh block input row [d_model] for token (b, t), from stream (seed, 8, b, t, attempt)."""
     g = rng(cfg.seed, STREAM_BLOCK_REDRAW, b, t, attempt)
     return round_to(g.standard_normal(d_model), cfg.io_dtype)
+
+
+@dataclass
+class SsdInputs:
+    X: np.ndarray       # [B, L, 1, H, P] bf16 bits
+    B: np.ndarray       # [B, L, 1, N] bf16 bits
+    C_mix: np.ndarray   # [B, L, N] bf16 bits
+    gates: np.ndarray   # [B, L, 1] f32
+    delta: np.ndarray   # [B, L, H] f32
+    A: np.ndarray       # [H] f32
+    D_skip: np.ndarray  # [H] f32
+    S0: np.ndarray      # [B, H, P, N] f32
+
+
+def draw_ssd_inputs(batch: int, seqlen: int, heads: int, head_dim: int, d_state: int, seed: int) -> SsdInputs:
+    """The SSD-form workload's inputs (recipe in the module docstring), one stream per tensor."""
+    g = lambda i: rng(seed, STREAM_SSD, i)
+    B, L, H, P, N = batch, seqlen, heads, head_dim, d_state
+    X = round_to(g(0).standard_normal((B, L, 1, H, P)), "bf16")
+    Bm = round_to(g(1).standard_normal((B, L, 1, N)), "bf16")
+    C = round_to(g(2).standard_normal((B, L, N)), "bf16")
+    delta = np.exp(g(3).uniform(np.log(1e-3), np.log(1e-1), (B, L, H))).astype(np.float32)
+    A = (-g(4).uniform(1.0, 16.0, H)).astype(np.float32)
+    D_skip = g(5).standard_normal(H).astype(np.float32)
+    S0 = (g(6).standard_normal((B, H, P, N)) * np.sqrt(0.1)).astype(np.float32)
+    return SsdInputs(X, Bm, C, np.ones((B, L, 1), np.float32), delta, A, D_skip, S0)
