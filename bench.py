@@ -371,7 +371,9 @@ class OraclePool:
         import multiprocessing as mp
 
         self.cfg, self.tokens, self.rows = cfg, tokens, rows
-        self.cores = os.cpu_count() or 1
+        # every worker holds the fp64 weights and one row's projections (a few hundred MB on the
+        # bench workload), so the pool stops at 128 processes on hosts with more cores
+        self.cores = min(os.cpu_count() or 1, 128)
         blocks = max(1, min(cfg.d_inner // 64, -(-self.cores // len(rows))))
         edges = [round(i * cfg.d_inner / blocks) for i in range(blocks + 1)]
         self.tasks = [(b, edges[i], edges[i + 1]) for b in rows for i in range(blocks)]
@@ -652,12 +654,44 @@ def report_block(torch, S, cfg, d_model, d_conv, peaks, flush, reps, warmup):
 
     (b_ms, c_ms), _ = _median_kernel_ms(torch, run, reps, warmup, flush, 3)
     S.check(S.swimba_get_device_status(ws, s), "device status")
+
+    # the two projection GEMMs alone through swimba_block_gemm, and cuBLAS (torch.matmul) on the
+    # same operands beside them for comparison
+    W_in, W_out = keep["W_in"], keep["W_out"]
+    u2 = u.view(T, d_model)
+    xz = torch.empty(T, 2 * D, dtype=u.dtype, device="cuda:0")
+    yb = torch.randn(T, D, device="cuda:0").to(u.dtype)
+    o2 = torch.empty(T, d_model, dtype=u.dtype, device="cuda:0")
+    gws = torch.zeros(256, dtype=torch.uint8, device="cuda:0")
+    dt = S.dtype_code(cfg.io_dtype)
+
+    def run_gemm(ev):
+        ev[0].record(s)
+        S.check(S.swimba_block_gemm(dt, T, 2 * D, d_model, u2, d_model, W_in, 2 * D, xz, 2 * D, None, 0, 2 * D, None,
+                                    0, gws, 256, s), "block_gemm in")
+        ev[1].record(s)
+        S.check(S.swimba_block_gemm(dt, T, d_model, D, yb, D, W_out, d_model, o2, d_model, None, 0, d_model, u2,
+                                    d_model, gws, 256, s), "block_gemm out")
+        ev[2].record(s)
+        torch.matmul(u2, W_in, out=xz)
+        ev[3].record(s)
+        torch.addmm(u2, yb, W_out, out=o2)
+        ev[4].record(s)
+
+    (gi_ms, go_ms, ci_ms, co_ms), _ = _median_kernel_ms(torch, run_gemm, reps, warmup, flush, 5)
+    S.check(S.swimba_get_device_status(gws, s), "gemm device status")
     conv_bytes = 2 * T * D * 2
-    gemm_flops = 2 * T * d_model * 2 * D + 2 * T * D * d_model
+    in_flops, out_flops = 2 * T * d_model * 2 * D, 2 * T * D * d_model
+    tc_peak = peaks["bf16_tflops"]
     return {
         "report": "block", "workload": cfg.name, "d_model": d_model, "d_conv": d_conv, "tokens": T,
         "block_us": 1e3 * b_ms, "tokens_per_s": T / (b_ms / 1e3),
-        "projection_gemm_gflop": gemm_flops / 1e9,
+        "projection_gemm_gflop": (in_flops + out_flops) / 1e9,
+        "in_gemm_us": 1e3 * gi_ms, "in_gemm_tflops": in_flops / gi_ms / 1e9,
+        "in_gemm_frac_of_tc_peak": in_flops / gi_ms / 1e9 / tc_peak,
+        "out_gemm_us": 1e3 * go_ms, "out_gemm_tflops": out_flops / go_ms / 1e9,
+        "out_gemm_frac_of_tc_peak": out_flops / go_ms / 1e9 / tc_peak,
+        "cublas_in_gemm_us": 1e3 * ci_ms, "cublas_out_gemm_us": 1e3 * co_ms,
         "conv_us": 1e3 * c_ms, "conv_gbs": conv_bytes / (c_ms / 1e3) / 1e9,
         "conv_frac_of_hbm": conv_bytes / (c_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
         "median_of": reps, "l2": "flushed (256 MB write) before every run",

@@ -286,10 +286,31 @@ swimba_status swimba_step(const swimba_dims *dims, const void *x, const void *z,
  *   p = [conv_state_in ; x_pre] along time (the W-1 inputs before the first token, oldest first);
  *   the Swimba layer on (x, z) gives out_layer = y * SiLU(z);  o = out_layer W_out + u.
  *
- * The in- and out-projections are plain dense GEMMs run by cuBLAS (operands in io_dtype, fp32
- * accumulation); the first block call of a host thread on a device creates that thread's cuBLAS
- * handle for the device (cuBLAS allocates its own state then): make it before any stream capture.
- * With bf16 activations x_pre, z, x, the layer output and o are each rounded to bf16 once. */
+ * The in- and out-projections are dense GEMMs run by the library's own kernel (swimba_block_gemm
+ * below: tcgen05 tensor cores for bf16, fp32 accumulation; a SIMT kernel for fp32). The
+ * in-projection is one GEMM whose output columns are split between x_pre and z; the
+ * out-projection adds the residual u in its epilogue. With bf16 activations x_pre, z, x, the
+ * layer output and o are each rounded to bf16 once. Nothing allocates: every block call can be
+ * captured in a CUDA graph. */
+
+/* The block's projection GEMM on its own: C = A B (+ R), with the output columns [0, split)
+ * written to C0 and [split, N) to C1 (the in-projection's [x_pre | z] split; split = N writes
+ * everything to C0).
+ *   dtype  SWIMBA_BF16: tcgen05 tensor cores, fp32 accumulation in tensor memory, bf16 out;
+ *          SWIMBA_F32: fp32 SIMT kernel. A, B, R, C0, C1 all of that type.
+ *   A      [M, K] row-major, row stride lda >= K                                   (in)
+ *   B      [K, N] row-major, row stride ldb >= N                                   (in)
+ *   R      [M, N] row stride ldr >= N, or NULL: added to the product (a residual)  (in)
+ *   C0     [M, split] row stride ldc0 >= split; C1 [M, N - split] row stride ldc1  (out)
+ *   C0 or C1 may be R itself (each element is read and written by one thread); no other overlap.
+ * bf16 needs N, split and every row stride a multiple of 8 elements and 16-byte aligned
+ * pointers (SWIMBA_ERR_UNSUPPORTED / SWIMBA_ERR_ALIGN otherwise). M = 0 or N = 0 is a no-op;
+ * K must be at least 1. ws: at least 256 bytes (the status block; a tensor-core wait that
+ * runs out leaves SWIMBA_ERR_TIMEOUT there). */
+swimba_status swimba_block_gemm(int32_t dtype, int32_t M, int32_t N, int32_t K, const void *A,
+                                int32_t lda, const void *B, int32_t ldb, void *C0, int32_t ldc0,
+                                void *C1, int32_t ldc1, int32_t split, const void *R, int32_t ldr,
+                                void *ws, size_t ws_bytes, void *stream);
 
 typedef struct {
   swimba_dims layer; /* B, L, D, N, R, E, k and dtypes of the Swimba layer inside the block */

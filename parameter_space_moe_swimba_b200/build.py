@@ -19,9 +19,9 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libswimba.so")
 SOURCES = [
     "api.cu", "route.cu", "route_tc.cu", "proj_simt.cu", "proj_tc.cu", "scan.cu", "scan_fast.cu", "conv.cu",
-    "block.cu", "separate.cu", "ssd.cu",
+    "block.cu", "separate.cu", "ssd.cu", "gemm.cu",
 ]
-LIBS = ["-lcublas"]  # the block's in- and out-projection GEMMs
+LIBS: list = []
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr"]
 

@@ -5,16 +5,18 @@
 // Models", Dutch summary §2 "Architectuur Implementatie"):
 //   [x_pre | z] = u W_in;  x = SiLU(causal depthwise conv(x_pre));  the Swimba layer on (x, z);
 //   o = layer_out W_out + u.
-// The two projections are plain dense GEMMs and go to cuBLAS (bf16 or fp32 operands, fp32
-// accumulation); the residual is added by the out-projection GEMM (beta = 1 on a copy of u). The
-// convolution runs in conv.cu, the layer in the library's route / projection / scan kernels.
-#include <cublas_v2.h>
-
+// The two projections are dense GEMMs on the library's own kernel (gemm.cu: tcgen05 for bf16,
+// SIMT for fp32): the in-projection's epilogue splits its columns into x_pre and z, the
+// out-projection's adds the residual u. The convolution runs in conv.cu, the layer in the
+// library's route / projection / scan kernels.
 #include <cstdio>
 
 #include "conv.cuh"
 
 namespace swimba {
+cudaError_t run_block_gemm(bool bf16, int M, int N, int K, const void* A, int lda, const void* B, int ldb, void* C0,
+                           int ldc0, void* C1, int ldc1, int split, const void* R, int ldr, void* status,
+                           cudaStream_t s);
 swimba_status api_check_dims(const swimba_dims* d);
 swimba_status api_cuda_status(cudaError_t e);
 void api_set_error(const char* msg);
@@ -74,37 +76,6 @@ BlockLayout block_layout(const swimba_block_dims* bd) {
   return l;
 }
 
-cublasHandle_t cublas_handle() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  thread_local cublasHandle_t handles[64] = {};
-  if (handles[dev] == nullptr && cublasCreate(&handles[dev]) != CUBLAS_STATUS_SUCCESS) handles[dev] = nullptr;
-  return handles[dev];
-}
-
-// Row-major C[M, n] = A[M, kd] (row stride lda) * W[kd, n] (row stride ldw) + beta C, ldc the row
-// stride of C. cuBLAS is column-major: the same memory is C^T = W^T A^T with W^T as the first operand.
-swimba_status gemm_rm(cudaStream_t s, bool bf16, int M, int n, int kd, const void* A, int lda, const void* W, int ldw,
-                      void* C, int ldc, float beta) {
-  cublasHandle_t h = cublas_handle();
-  if (h == nullptr) {
-    api_set_error("cuBLAS handle could not be created");
-    return SWIMBA_ERR_CUDA;
-  }
-  if (cublasSetStream(h, s) != CUBLAS_STATUS_SUCCESS) return SWIMBA_ERR_CUDA;
-  const cudaDataType t = bf16 ? CUDA_R_16BF : CUDA_R_32F;
-  const float alpha = 1.0f;
-  const cublasStatus_t cs = cublasGemmEx(h, CUBLAS_OP_N, CUBLAS_OP_N, n, M, kd, &alpha, W, t, ldw, A, t, lda, &beta,
-                                         C, t, ldc, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
-  if (cs != CUBLAS_STATUS_SUCCESS) {
-    char msg[96];
-    snprintf(msg, sizeof(msg), "cublasGemmEx failed with status %d", (int)cs);
-    api_set_error(msg);
-    return SWIMBA_ERR_CUDA;
-  }
-  return SWIMBA_OK;
-}
-
 // Every argument a block call hands to the calls it makes, checked before the first launch (the
 // layer's own calls check them again, but by then the in-projection would be queued).
 swimba_status check_weights(const swimba_block_weights* w) {
@@ -127,29 +98,25 @@ swimba_status check_states(const swimba_block_dims* bd, const float* h0, const f
   return SWIMBA_OK;
 }
 
-// in-projection: x_pre = u W_in[:, :D], z = u W_in[:, D:]
+// in-projection: [x_pre | z] = u W_in, one GEMM whose epilogue writes columns [0, D) to x_pre and
+// [D, 2D) to z
 swimba_status in_proj(const swimba_block_dims* bd, const void* u, const swimba_block_weights* w, void* x_pre, void* z,
-                      cudaStream_t s) {
+                      void* status, cudaStream_t s) {
   const swimba_dims& d = bd->layer;
   const bool bf16 = d.io_dtype == SWIMBA_BF16;
   const int M = (int)(d.batch * d.seqlen), D = d.d_inner, dm = bd->d_model;
-  const char* W_z = static_cast<const char*>(w->W_in) + (size_t)D * io_bytes(d.w_dtype);
-  swimba_status st = gemm_rm(s, bf16, M, D, dm, u, dm, w->W_in, 2 * D, x_pre, D, 0.0f);
-  if (st != SWIMBA_OK) return st;
-  return gemm_rm(s, bf16, M, D, dm, u, dm, W_z, 2 * D, z, D, 0.0f);
+  return api_cuda_status(
+      run_block_gemm(bf16, M, 2 * D, dm, u, dm, w->W_in, 2 * D, x_pre, D, z, D, D, nullptr, 0, status, s));
 }
 
-// out-projection with the residual: out = u; out += y W_out
+// out-projection with the residual added in the GEMM's epilogue: out = y W_out + u (out may be u:
+// every element is read and written by the same thread)
 swimba_status out_proj(const swimba_block_dims* bd, const void* u, const swimba_block_weights* w, const void* y,
-                       void* out, cudaStream_t s) {
+                       void* out, void* status, cudaStream_t s) {
   const swimba_dims& d = bd->layer;
   const int M = (int)(d.batch * d.seqlen), D = d.d_inner, dm = bd->d_model;
-  const size_t bytes = (size_t)M * dm * io_bytes(d.io_dtype);
-  if (out != u) {
-    const swimba_status st = api_cuda_status(cudaMemcpyAsync(out, u, bytes, cudaMemcpyDeviceToDevice, s));
-    if (st != SWIMBA_OK) return st;
-  }
-  return gemm_rm(s, d.io_dtype == SWIMBA_BF16, M, dm, D, y, D, w->W_out, dm, out, dm, 1.0f);
+  return api_cuda_status(run_block_gemm(d.io_dtype == SWIMBA_BF16, M, dm, D, y, D, w->W_out, dm, out, dm, out, dm,
+                                        dm, u, dm, status, s));
 }
 
 }  // namespace
@@ -183,6 +150,31 @@ swimba_status swimba_conv1d_step(const swimba_dims* dims, int32_t d_conv, const 
   return api_cuda_status(run_conv1d(p, dims->io_dtype == SWIMBA_BF16, true, static_cast<cudaStream_t>(stream)));
 }
 
+swimba_status swimba_block_gemm(int32_t dtype, int32_t M, int32_t N, int32_t K, const void* A, int32_t lda,
+                                const void* B, int32_t ldb, void* C0, int32_t ldc0, void* C1, int32_t ldc1,
+                                int32_t split, const void* R, int32_t ldr, void* ws, size_t ws_bytes,
+                                void* stream) {
+  if (dtype != SWIMBA_BF16 && dtype != SWIMBA_F32) return SWIMBA_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 1 || split < 0 || split > N) return SWIMBA_ERR_INVALID_ARG;
+  if (ws == nullptr || ws_bytes < 256) return SWIMBA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SWIMBA_ERR_ALIGN;
+  if (M == 0 || N == 0) return SWIMBA_OK;
+  if (!A || !B || lda < K || ldb < N || (split > 0 && (!C0 || ldc0 < split)) ||
+      (split < N && (!C1 || ldc1 < N - split)) || (R && ldr < N))
+    return SWIMBA_ERR_INVALID_ARG;
+  const bool bf16 = dtype == SWIMBA_BF16;
+  if (bf16) {
+    if (N % 8 || split % 8 || lda % 8 || ldb % 8 || (split > 0 && ldc0 % 8) ||
+        (split < N && ldc1 % 8) || (R && ldr % 8))
+      return SWIMBA_ERR_UNSUPPORTED;
+    if (!aligned16(A) || !aligned16(B) || (C0 && !aligned16(C0)) || (C1 && !aligned16(C1)) ||
+        (R && !aligned16(R)))
+      return SWIMBA_ERR_ALIGN;
+  }
+  return api_cuda_status(run_block_gemm(bf16, M, N, K, A, lda, B, ldb, C0, ldc0, C1, ldc1, split, R, ldr, ws,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 size_t swimba_block_workspace_size(const swimba_block_dims* bd) {
   if (check_block(bd) != SWIMBA_OK) return 0;
   return block_layout(bd).total;
@@ -211,7 +203,7 @@ swimba_status swimba_block_fwd(const swimba_block_dims* bd, const void* u, const
   float* Cm = reinterpret_cast<float*>(base + l.Cm);
   const size_t layer_ws = swimba_workspace_size(d, SWIMBA_OP_LAYER);
 
-  if ((st = in_proj(bd, u, w, x_pre, z, s)) != SWIMBA_OK) return st;
+  if ((st = in_proj(bd, u, w, x_pre, z, ws, s)) != SWIMBA_OK) return st;
   if ((st = swimba_conv1d_fwd(d, bd->d_conv, x_pre, w->conv_w, w->conv_b, conv_state_in, x, conv_state_out,
                               stream)) != SWIMBA_OK)
     return st;
@@ -221,7 +213,7 @@ swimba_status swimba_block_fwd(const swimba_block_dims* bd, const void* u, const
   if ((st = swimba_scan_fwd(d, x, z, delta, Bm, Cm, idx, gates, &w->layer, h0, y, h_final, nullptr, ws, layer_ws,
                             stream)) != SWIMBA_OK)
     return st;
-  return out_proj(bd, u, w, y, out, s);
+  return out_proj(bd, u, w, y, out, ws, s);
 }
 
 swimba_status swimba_block_step(const swimba_block_dims* bd, const void* u, const swimba_block_weights* w, float* h,
@@ -246,14 +238,14 @@ swimba_status swimba_block_step(const swimba_block_dims* bd, const void* u, cons
   float* Cm = reinterpret_cast<float*>(base + l.Cm);
   const size_t layer_ws = swimba_workspace_size(d, SWIMBA_OP_LAYER);
 
-  if ((st = in_proj(bd, u, w, x_pre, z, s)) != SWIMBA_OK) return st;
+  if ((st = in_proj(bd, u, w, x_pre, z, ws, s)) != SWIMBA_OK) return st;
   if ((st = swimba_conv1d_step(d, bd->d_conv, x_pre, w->conv_w, w->conv_b, conv_state, x, stream)) != SWIMBA_OK)
     return st;
   if ((st = swimba_route(d, x, w->layer.W_r, idx, gates, stream)) != SWIMBA_OK) return st;
   if ((st = swimba_mixed_proj(d, x, idx, gates, &w->layer, delta, Bm, Cm, ws, layer_ws, stream)) != SWIMBA_OK)
     return st;
   if ((st = swimba_step(d, x, z, delta, Bm, Cm, idx, gates, &w->layer, h, y, stream)) != SWIMBA_OK) return st;
-  return out_proj(bd, u, w, y, out, s);
+  return out_proj(bd, u, w, y, out, ws, s);
 }
 
 }  // extern "C"

@@ -1,0 +1,341 @@
+// The surrounding block's two dense projections on the tcgen05 tensor cores.
+//
+// Source: "Mamba y las SSMs: el retorno del estado persistente", section "Mamba" (Figura 3: a linear
+// projection makes the SSM branch and the gate branch, a linear projection maps the gated output
+// back) and "Estado interno puramente lineal" (the output projection is followed by a residual
+// connection).
+//
+//   in-projection:   [x_pre | z] = u W_in        (the epilogue splits the columns into the x_pre
+//                                                 and z buffers)
+//   out-projection:  o = y W_out + u             (the residual is added in the epilogue)
+//
+// C[M, N] = A[M, K] B[K, N] (+ R[M, N]), bf16 operands as stored (A row-major with K contiguous,
+// B row-major with N contiguous), fp32 accumulation in tensor memory, bf16 out. Persistent,
+// warp-specialised: warp 0 streams A tiles [128 x 64] (K-major, 128-byte swizzle) and B tiles
+// [64 x 256] (four MN-major boxes) by TMA through a 4-stage ring; warp 1 issues tcgen05.mma
+// M=128, N=256, K=16 into one of two 256-column TMEM accumulators; warps 2-5 drain the other
+// accumulator (one TMEM lane = one output row) while the next tile accumulates. Tiles go in
+// M-fastest order, so consecutive CTAs share the weight columns they read from L2. Every wait is
+// bounded: a wait that runs out records SWIMBA_ERR_TIMEOUT in the status block, the CTA lets its
+// copies land, frees TMEM and exits. fp32 operands take a SIMT kernel (tiles of 64 x 64 in
+// shared memory).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace swimba {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int GBM = 128, GBN = 256, GBK = 64;
+constexpr int kGStages = 4;
+constexpr int kGA = GBM * GBK * 2;   // 16 KB
+constexpr int kGB = GBK * GBN * 2;   // 32 KB: four 64-column boxes of 8 KB
+constexpr int kGStage = kGA + kGB;
+
+__device__ __forceinline__ uint32_t bf16pair(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+struct GemmParams {
+  void* C0;           // columns [0, split) of the output
+  void* C1;           // columns [split, N) (split == N: unused)
+  const void* R;      // residual [M, N] or null
+  void* status;
+  int M, N, K, split, ldc0, ldc1, ldr;
+};
+
+}  // namespace
+
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                   const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGStages * kGStage);
+  uint64_t* empty = full + kGStages;
+  uint64_t* acc_full = empty + kGStages;   // [2]
+  uint64_t* acc_empty = acc_full + 2;      // [2]
+  uint64_t* done = acc_empty + 2;          // every MMA of the CTA has completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kGStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int mt = (p.M + GBM - 1) / GBM, nt = (p.N + GBN - 1) / GBN, kt = (p.K + GBK - 1) / GBK;
+  const int tiles = mt * nt;
+
+  if (warp == 0) {
+    // ---------------- producer ----------------
+    int stage = 0, issued = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+      const int m0 = (tile % mt) * GBM, n0 = (tile / mt) * GBN;
+      for (int k = 0; k < kt; ++k) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = smem + stage * kGStage;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[stage], (uint32_t)kGStage);
+          tma_load_2d(st, &tm_a, &full[stage], k * GBK, m0);
+          for (int i = 0; i < 4; ++i) tma_load_2d(st + kGA + i * 8192, &tm_b, &full[stage], n0 + 64 * i, k * GBK);
+        }
+        __syncwarp();
+        ++issued;
+        if (++stage == kGStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) record_device_error(p.status, SWIMBA_ERR_TIMEOUT, 61, blockIdx.x, 0);
+      // the copies of the last min(issued, stages) stages may still be landing
+      for (int i = 0; i < (issued < kGStages ? issued : kGStages); ++i) {
+        if (--stage < 0) {
+          stage = kGStages - 1;
+          phase ^= 1u;
+        }
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&full[stage], phase) && globaltimer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(GBM, GBN, /*b_mn_major=*/true);
+      const uint32_t base = smem_u32(smem);
+      int stage = 0, buf = 0;
+      uint32_t phase = 0;
+      uint32_t acc_phase[2] = {0, 0};
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(&acc_empty[buf], acc_phase[buf] ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        acc_phase[buf] ^= 1u;
+        tc_fence_after();
+        for (int k = 0; k < kt; ++k) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = base + stage * kGStage, sb = sa + kGA;
+#pragma unroll
+          for (int kk = 0; kk < GBK / 16; ++kk) {
+            mma_bf16(tmem + buf * GBN, smem_desc(sa + kk * 32, 16, 1024, kLayoutSW128),
+                     smem_desc(sb + kk * 16 * 128, 8192, 1024, kLayoutSW128), idesc, (k | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == kGStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[buf]);
+        buf ^= 1;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_device_error(p.status, SWIMBA_ERR_TIMEOUT, 62, blockIdx.x, 0);
+      }
+      // every MMA this thread issued has completed when `done` completes its first phase
+      mma_commit(done);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(done, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue: warps 2..5, TMEM lane quarter = warp % 4 ----------------
+    const int q = warp & 3;
+    const int row_in_tile = 32 * q + lane;
+    int buf = 0;
+    uint32_t acc_phase[2] = {0, 0};
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+      const int m0 = (tile % mt) * GBM, n0 = (tile / mt) * GBN;
+      if (!mbar_wait(&acc_full[buf], acc_phase[buf], abort_flag)) {
+        *abort_flag = 1;
+        if (lane == 0) record_device_error(p.status, SWIMBA_ERR_TIMEOUT, 63, blockIdx.x, tile);
+        break;
+      }
+      acc_phase[buf] ^= 1u;
+      tc_fence_after();
+      const int m = m0 + row_in_tile;
+      for (int cb = 0; cb < GBN / 32; ++cb) {
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + buf * GBN + cb * 32, v);
+        const int n = n0 + cb * 32;
+        if (m < p.M && n < p.N) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {  // groups of 8 columns (N and split are multiples of 8)
+            const int col = n + j;
+            if (col < p.N) {
+              float o[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) o[e] = v[j + e];
+              if (p.R != nullptr) {
+                const uint4 w = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.R) +
+                                                                (size_t)m * p.ldr + col);
+                o[0] += bf16lo(w.x);
+                o[1] += bf16hi(w.x);
+                o[2] += bf16lo(w.y);
+                o[3] += bf16hi(w.y);
+                o[4] += bf16lo(w.z);
+                o[5] += bf16hi(w.z);
+                o[6] += bf16lo(w.w);
+                o[7] += bf16hi(w.w);
+              }
+              __nv_bfloat16* out = col < p.split
+                                       ? reinterpret_cast<__nv_bfloat16*>(p.C0) + (size_t)m * p.ldc0 + col
+                                       : reinterpret_cast<__nv_bfloat16*>(p.C1) + (size_t)m * p.ldc1 + (col - p.split);
+              *reinterpret_cast<uint4*>(out) = make_uint4(bf16pair(o[0], o[1]), bf16pair(o[2], o[3]),
+                                                          bf16pair(o[4], o[5]), bf16pair(o[6], o[7]));
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      buf ^= 1;
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// fp32 operands: C[M, N] = A B (+ R), 64 x 64 tiles, 256 threads with 4 x 4 outputs each.
+__global__ void __launch_bounds__(256) gemm_simt_f32_kernel(const float* A, int lda, const float* B, int ldb,
+                                                            float* C0, int ldc0, float* C1, int ldc1, int split,
+                                                            const float* R, int ldr, int M, int N, int K) {
+  __shared__ float As[16][64 + 1];
+  __shared__ float Bs[16][64 + 1];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    for (int i = threadIdx.x; i < 16 * 64; i += 256) {
+      const int kk = i / 64, c = i % 64;
+      As[kk][c] = (m0 + c < M && k0 + kk < K) ? A[(size_t)(m0 + c) * lda + k0 + kk] : 0.f;
+      Bs[kk][c] = (n0 + c < N && k0 + kk < K) ? B[(size_t)(k0 + kk) * ldb + n0 + c] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(As[kk][ty + 16 * i], Bs[kk][tx + 16 * j], acc[i][j]);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int m = m0 + ty + 16 * i, n = n0 + tx + 16 * j;
+      if (m < M && n < N) {
+        const float v = acc[i][j] + (R != nullptr ? R[(size_t)m * ldr + n] : 0.f);
+        if (n < split) C0[(size_t)m * ldc0 + n] = v;
+        else C1[(size_t)m * ldc1 + n - split] = v;
+      }
+    }
+}
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 gemm_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+// 2-D bf16 map over a row-major [rows, cols] matrix with row stride ld (elements), box {64, box_rows}.
+bool gemm_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld, int box_rows) {
+  auto fn = gemm_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t str[1] = {(cuuint64_t)(ld * 2)};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, str, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+// C[M, N] = A[M, K] (row stride lda) B[K, N] (row stride ldb) (+ R, row stride ldr): columns below
+// `split` go to C0 (row stride ldc0), the others to C1 (ldc1). bf16 needs every row stride and
+// split a multiple of 8 elements and 16-byte aligned pointers.
+cudaError_t run_block_gemm(bool bf16, int M, int N, int K, const void* A, int lda, const void* B, int ldb, void* C0,
+                           int ldc0, void* C1, int ldc1, int split, const void* R, int ldr, void* status,
+                           cudaStream_t s) {
+  if (!bf16) {
+    dim3 grid((unsigned)((N + 63) / 64), (unsigned)((M + 63) / 64));
+    gemm_simt_f32_kernel<<<grid, 256, 0, s>>>(static_cast<const float*>(A), lda, static_cast<const float*>(B), ldb,
+                                              static_cast<float*>(C0), ldc0, static_cast<float*>(C1), ldc1, split,
+                                              static_cast<const float*>(R), ldr, M, N, K);
+    note_launch();
+    return cudaGetLastError();
+  }
+  CUtensorMap ta, tb;
+  if (!gemm_map(&ta, A, M, K, lda, GBM) || !gemm_map(&tb, B, K, N, ldb, GBK)) return cudaErrorInvalidValue;
+  GemmParams p{C0, C1, R, status, M, N, K, split, ldc0, ldc1, ldr};
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int tiles = ((M + GBM - 1) / GBM) * ((N + GBN - 1) / GBN);
+  const size_t smem = 1024 + (size_t)kGStages * kGStage + 256;  // ring, then barriers and the TMEM slot
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  gemm_tc_kernel<<<(unsigned)std::min(tiles, sms), 192, smem, s>>>(ta, tb, p);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace swimba

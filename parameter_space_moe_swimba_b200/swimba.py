@@ -62,6 +62,7 @@ EXPORTED = [
     "swimba_last_error_string",
     "swimba_conv1d_fwd",
     "swimba_conv1d_step",
+    "swimba_block_gemm",
     "swimba_block_workspace_size",
     "swimba_block_fwd",
     "swimba_block_step",
@@ -155,6 +156,9 @@ _lib.swimba_conv1d_fwd.argtypes = [ctypes.POINTER(swimba_dims), ctypes.c_int32, 
 _lib.swimba_conv1d_fwd.restype = ctypes.c_int
 _lib.swimba_conv1d_step.argtypes = [ctypes.POINTER(swimba_dims), ctypes.c_int32, _P, _P, _P, _P, _P, _P]
 _lib.swimba_conv1d_step.restype = ctypes.c_int
+_I = ctypes.c_int32
+_lib.swimba_block_gemm.argtypes = [_I, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P, _I, _I, _P, _I, _P, ctypes.c_size_t, _P]
+_lib.swimba_block_gemm.restype = ctypes.c_int
 _lib.swimba_block_workspace_size.argtypes = [ctypes.POINTER(swimba_block_dims)]
 _lib.swimba_block_workspace_size.restype = ctypes.c_size_t
 _lib.swimba_block_fwd.argtypes = [ctypes.POINTER(swimba_block_dims), _P, ctypes.POINTER(swimba_block_weights), _P, _P,
@@ -308,6 +312,13 @@ def swimba_block_workspace_size(bdims: swimba_block_dims) -> int:
     return int(_lib.swimba_block_workspace_size(ctypes.byref(bdims)))
 
 
+def swimba_block_gemm(dtype, M, N, K, A, lda, B, ldb, C0, ldc0, C1, ldc1, split, R, ldr, ws, ws_bytes,
+                      stream=None) -> int:
+    return _lib.swimba_block_gemm(int(dtype), int(M), int(N), int(K), _ptr(A), int(lda), _ptr(B), int(ldb), _ptr(C0),
+                                  int(ldc0), _ptr(C1), int(ldc1), int(split), _ptr(R), int(ldr), _ptr(ws),
+                                  int(ws_bytes), _stream(stream))
+
+
 def swimba_block_fwd(bdims, u, bweights, h0, conv_state_in, out, h_final, conv_state_out, ws, ws_bytes,
                      stream=None) -> int:
     return _lib.swimba_block_fwd(ctypes.byref(bdims), _ptr(u), ctypes.byref(bweights), _ptr(h0), _ptr(conv_state_in),
@@ -324,8 +335,11 @@ def swimba_block_step(bdims, u, bweights, h, conv_state, out, ws, ws_bytes, stre
 # marshalling helpers: shapes, host arrays -> device tensors, buffers of one layer call
 # ------------------------------------------------------------------------------------------------
 
-def _dtype_code(name: str) -> int:
+def dtype_code(name: str) -> int:
     return {"f32": SWIMBA_F32, "bf16": SWIMBA_BF16}[name]
+
+
+_dtype_code = dtype_code
 
 
 def make_dims(cfg, seqlen=None, batch=None, n_experts=None, top_k=None) -> swimba_dims:
