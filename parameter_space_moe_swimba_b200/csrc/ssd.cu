@@ -19,7 +19,10 @@
 //
 // One CTA of 4 warps per (sequence, head) walks the chunks in order, so the carried state never
 // leaves the SM: Sᵀ [N x P] is an fp32 accumulator in tensor memory, scaled by the chunk's decay
-// and accumulated by the state MMA; its bf16 copy in shared memory is the next chunk's operand.
+// and accumulated by the state MMA. The three operands the kernel makes itself -- the state's copy
+// for the readout, W and X_w -- enter the MMAs as two bf16 parts, hi = bf16(v) and
+// lo = bf16(v - hi) (about 16 significant bits, one more MMA each), so the state read out stays
+// fp32-accurate; a single bf16 copy of each moved y by up to 2e-2 (1 + |y|) on the test shapes.
 // Thread i owns row i of every [Q x *] accumulator (TMEM lane i): it builds row i of W, scales
 // row i of X, writes row i of y, and row i of Sᵀ. One thread issues the TMA loads (C_mix, B, X
 // tiles, 128-byte swizzled; the next chunk's as soon as the MMAs have read the current one) and
@@ -47,10 +50,10 @@ struct SsdSmem {
   static constexpr int C = 0;                 // C_mix  [128 tok][128 n]: 2 boxes (K-major A)
   static constexpr int B = C + 2 * kBox;      // B      [128 tok][128 n]: 2 boxes (K-major B; MN-major A)
   static constexpr int X = B + 2 * kBox;      // X      [128 tok][64 p]:  1 box (MN-major B)
-  static constexpr int XW = X + kBox;         // X_w    [128 tok][64 p]:  1 box (MN-major B)
-  static constexpr int W = XW + kBox;         // W      [128 i][128 s]:   2 boxes (K-major A)
-  static constexpr int S = W + 2 * kBox;      // S_inᵀ  [128 n][64 p]:    1 box (MN-major B)
-  static constexpr int CUM = S + kBox;        // f32 [128] cum
+  static constexpr int XW = X + kBox;         // X_w    [128 tok][64 p]:  hi, lo: 1 box each (MN-major B)
+  static constexpr int W = XW + 2 * kBox;     // W      [128 i][128 s]:   hi, lo: 2 boxes each (K-major A)
+  static constexpr int S = W + 4 * kBox;      // S_inᵀ  [128 n][64 p]:    hi, lo: 1 box each (MN-major B)
+  static constexpr int CUM = S + 2 * kBox;    // f32 [128] cum
   static constexpr int DG = CUM + SQ * 4;     // f32 [128] Δ g
   static constexpr int WSUM = DG + SQ * 4;    // f32 [4] warp totals of the scan
   static constexpr int BAR = WSUM + 64;       // 2 mbarriers
@@ -80,6 +83,12 @@ __device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * 12
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Two values as bf16 pairs hi = bf16(v), lo = bf16(v - hi).
+__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  hi = pack2(a, b);
+  lo = pack2(a - bf16lo(hi), b - bf16hi(hi));
 }
 
 }  // namespace
@@ -130,23 +139,26 @@ __global__ void __launch_bounds__(128, 1)
     tma_load_3d(sm + SsdSmem::X, &tm_x, bar_tma, h * SP, t0, b);
   };
 
-  // the carried state: Sᵀ[n][p] (thread n = TMEM lane n) into TMEM (fp32) and its bf16 copy
+  // the carried state: Sᵀ[n][p] (thread n = TMEM lane n) into TMEM (fp32) and its hi/lo copy
   {
     uint32_t r[32];
     for (int half = 0; half < 2; ++half) {
-      uint32_t w16[16];
+      uint32_t hi[16], lo[16];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const int pp = half * 32 + j;
         const float v = p.S0 != nullptr ? p.S0[(((size_t)b * p.H + h) * SP + pp) * SN + tid] : 0.f;
         r[j] = __float_as_uint(v);
-        if (j & 1) w16[j >> 1] = pack2(__uint_as_float(r[j - 1]), v);
+        if (j & 1) split2(__uint_as_float(r[j - 1]), v, hi[j >> 1], lo[j >> 1]);
       }
       tmem_st32(tlane + kColS + half * 32, r);
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 4; ++c) {
         *reinterpret_cast<uint4*>(sm + SsdSmem::S + swz(tid, half * 4 + c)) =
-            make_uint4(w16[4 * c], w16[4 * c + 1], w16[4 * c + 2], w16[4 * c + 3]);
+            make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+        *reinterpret_cast<uint4*>(sm + SsdSmem::S + kBox + swz(tid, half * 4 + c)) =
+            make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
+      }
     }
     tmem_wait_st();
     fence_proxy_async_smem();
@@ -201,6 +213,8 @@ __global__ void __launch_bounds__(128, 1)
                  smem_desc(sB + koff, 16, 1024, kLayoutSW128), id_qq, ks > 0 ? 1u : 0u);
         mma_bf16(tmem + kColY2, smem_desc(sC + koff, 16, 1024, kLayoutSW128),
                  smem_desc(sS + ks * 16 * 128, 8192, 1024, kLayoutSW128), id_qp, ks > 0 ? 1u : 0u);
+        mma_bf16(tmem + kColY2, smem_desc(sC + koff, 16, 1024, kLayoutSW128),
+                 smem_desc(sS + kBox + ks * 16 * 128, 8192, 1024, kLayoutSW128), id_qp, 1u);
       }
       mma_commit(bar_mma);
     }
@@ -214,8 +228,11 @@ __global__ void __launch_bounds__(128, 1)
         const uint32_t in[4] = {q.x, q.y, q.z, q.w};
         uint32_t o[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) o[e] = pack2(bf16lo(in[e]) * ws, bf16hi(in[e]) * ws);
+        uint32_t l[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) split2(bf16lo(in[e]) * ws, bf16hi(in[e]) * ws, o[e], l[e]);
         *reinterpret_cast<uint4*>(sm + SsdSmem::XW + swz(tid, cc)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(sm + SsdSmem::XW + kBox + swz(tid, cc)) = make_uint4(l[0], l[1], l[2], l[3]);
       }
     }
     // Sᵀ (thread n) decays by the chunk's total before the state MMA adds to it
@@ -243,19 +260,22 @@ __global__ void __launch_bounds__(128, 1)
       for (int blk = 0; blk < 4; ++blk) {  // 32 columns s at a time
         float gr[32];
         tmem_ld32(tlane + kColG + blk * 32, gr);
-        uint32_t w16[16];
+        uint32_t w16[16], l16[16];
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           const int s0 = blk * 32 + j;
           const float w0 = s0 <= tid ? __expf(ci - cum[s0]) * dg[s0] * gr[j] : 0.f;
           const float w1 = s0 + 1 <= tid ? __expf(ci - cum[s0 + 1]) * dg[s0 + 1] * gr[j + 1] : 0.f;
-          w16[j >> 1] = pack2(w0, w1);
+          split2(w0, w1, w16[j >> 1], l16[j >> 1]);
         }
-        // columns blk*32 .. +31: box blk/2, 16-byte chunks (blk&1)*4 .. +3 of row tid
+        // columns blk*32 .. +31: box blk/2 (hi), 2 + blk/2 (lo), 16-byte chunks (blk&1)*4 .. +3 of row tid
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
+        for (int cc = 0; cc < 4; ++cc) {
           *reinterpret_cast<uint4*>(sm + SsdSmem::W + (blk >> 1) * kBox + swz(tid, (blk & 1) * 4 + cc)) =
               make_uint4(w16[4 * cc], w16[4 * cc + 1], w16[4 * cc + 2], w16[4 * cc + 3]);
+          *reinterpret_cast<uint4*>(sm + SsdSmem::W + (2 + (blk >> 1)) * kBox + swz(tid, (blk & 1) * 4 + cc)) =
+              make_uint4(l16[4 * cc], l16[4 * cc + 1], l16[4 * cc + 2], l16[4 * cc + 3]);
+        }
       }
     }
     fence_proxy_async_smem();
@@ -269,8 +289,12 @@ __global__ void __launch_bounds__(128, 1)
         const uint32_t aoff = (uint32_t)((ks >> 2) * kBox + (ks & 3) * 32);
         mma_bf16(tmem + kColY1, smem_desc(sW + aoff, 16, 1024, kLayoutSW128),
                  smem_desc(sX + ks * 16 * 128, 8192, 1024, kLayoutSW128), id_qp, ks > 0 ? 1u : 0u);
+        mma_bf16(tmem + kColY1, smem_desc(sW + 2 * kBox + aoff, 16, 1024, kLayoutSW128),
+                 smem_desc(sX + ks * 16 * 128, 8192, 1024, kLayoutSW128), id_qp, 1u);
         mma_bf16(tmem + kColS, smem_desc(sB + ks * 16 * 128, kBox, 1024, kLayoutSW128),
                  smem_desc(sXW + ks * 16 * 128, 8192, 1024, kLayoutSW128), id_st, 1u);
+        mma_bf16(tmem + kColS, smem_desc(sB + ks * 16 * 128, kBox, 1024, kLayoutSW128),
+                 smem_desc(sXW + kBox + ks * 16 * 128, 8192, 1024, kLayoutSW128), id_st, 1u);
       }
       mma_commit(bar_mma);
     }
@@ -312,19 +336,20 @@ __global__ void __launch_bounds__(128, 1)
         }
       }
     }
-    // the new state's bf16 copy Sᵀ[n][p] (thread n), the next chunk's Y2 operand
-    {
-      uint32_t w16[32];
-      for (int half = 0; half < 2; ++half) {
-        float f[32];
-        tmem_ld32(tlane + kColS + half * 32, f);
+    // the new state's hi/lo copy Sᵀ[n][p] (thread n), the next chunk's Y2 operand
+    for (int half = 0; half < 2; ++half) {
+      float f[32];
+      tmem_ld32(tlane + kColS + half * 32, f);
+      uint32_t w16[16], l16[16];
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) w16[half * 16 + (j >> 1)] = pack2(f[j], f[j + 1]);
-      }
+      for (int j = 0; j < 32; j += 2) split2(f[j], f[j + 1], w16[j >> 1], l16[j >> 1]);
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc)
-        *reinterpret_cast<uint4*>(sm + SsdSmem::S + swz(tid, cc)) =
+      for (int cc = 0; cc < 4; ++cc) {
+        *reinterpret_cast<uint4*>(sm + SsdSmem::S + swz(tid, half * 4 + cc)) =
             make_uint4(w16[4 * cc], w16[4 * cc + 1], w16[4 * cc + 2], w16[4 * cc + 3]);
+        *reinterpret_cast<uint4*>(sm + SsdSmem::S + kBox + swz(tid, half * 4 + cc)) =
+            make_uint4(l16[4 * cc], l16[4 * cc + 1], l16[4 * cc + 2], l16[4 * cc + 3]);
+      }
     }
     fence_proxy_async_smem();
     tc_fence_before();

@@ -1,8 +1,11 @@
 """Swimba on the Mamba-2 SSD form through the C ABI (swimba_ssd_scan: chunks of 128 tokens on the
 tcgen05 tensor cores) against the fp64 oracle's sequential recurrence and its chunked (SSD) form
-on the same bf16 inputs: y within 2e-2 (1 + |y|) and its state-space part within 2e-2 of its own
-scale (bf16 MMA operands, fp32 accumulation and fp32 carried state), the final state within 1e-2 of
-its scale; ragged last chunks, one token, and a start state."""
+on the same bf16 inputs: y within the layer's bf16 bound 2e-2 (1 + |y|). The operands the kernel
+makes itself (the carried state's copy, W, X_w) enter the MMAs as bf16 hi + lo pairs (about 16
+significant bits) with fp32 accumulation, so the result is held to fp32-like bounds as well: y and
+its state-space part within 1e-3 of their scale and the final state within 1e-3 of its scale (a
+single bf16 copy of those operands gives about 2e-2 and 1e-2 here); ragged last chunks, one token,
+and a start state."""
 from __future__ import annotations
 
 import numpy as np
@@ -75,7 +78,7 @@ def test_ssd_scan_matches_sequential_and_chunked_oracle(S, shape):
         e = {"y": scaled_err(y, y_ref), "y_ssm": rel_rms_err(y - skip, y_ref - skip), "S_final": rel_rms_err(sf, s_ref)}
         print(shape, "chunked" if chunked else "sequential", {k: f"{v:.2e}" for k, v in e.items()})
         assert e["y"] <= 2e-2 and e["y_ssm"] <= 2e-2
-        assert e["S_final"] <= 1e-2
+        assert e["y"] <= 1e-3 and e["y_ssm"] <= 1e-3 and e["S_final"] <= 1e-3
 
 
 def test_ssd_scan_rejects_unsupported_and_bad_arguments(S):
