@@ -268,117 +268,104 @@ cudaError_t run_scan_chain(int64_t BDN, int P, const float* h_zero, const float*
   return cudaGetLastError();
 }
 
-// Decode step, N = 16, k <= 2: a CTA owns a tile of up to 256 channels of one sequence. Its 256
-// threads first put the whole tile's inputs in flight with cp.async 16-byte copies into shared memory
-// -- the state tile (16 KB), Δ, x, z, B_mix, C_mix -- then, once thread 0 has read the token's
-// experts, the two selected experts' A tiles (16 KB each, L2-resident tables). The copies need no
-// registers, so every SM keeps tens of KB of the state stream in flight (the per-thread loads of
-// step_kernel above kept a few KB). Then thread i computes 4 (channel, state quarter) items of the
-// tile from shared memory, the four quarters of a channel reduce the readout with two shuffles,
-// and the new state goes back to HBM with coalesced 16-byte stores. The waits are the hardware's
-// cp.async group waits (no spin).
-constexpr int kStepTile = 256;  // channels per CTA
-
-__device__ __forceinline__ void cp_async16_s(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
-               : "memory");
-}
+// Decode step, N = 16, k <= 2. The state stream (h read and written, 128 bytes per channel and
+// sequence) is the step's traffic; the A tables are small and shared by every sequence. So a CTA
+// owns a tile of 64 channels and a group of sequences: it stages the A rows of ALL E experts for
+// its channels in shared memory once (E x 4 KB, read from L2 once per CTA instead of once per
+// sequence), then streams its sequences past them. Thread i owns (channel i / 4, state quarter
+// i % 4); it puts four sequences' state quarters, Δ, x, z, B/C quarters and experts in flight
+// before it computes any of them, and the four quarters of a channel reduce the readout with two
+// shuffles. Groups are sized so that the grid is about three CTAs per SM (the resident limit at
+// 85 registers a thread).
+constexpr int kStepCh = 64;  // channels per CTA
+constexpr int kStepU = 4;    // sequences in flight per thread
 
 template <typename IO, int K>
-__global__ void __launch_bounds__(256) step_bulk_kernel(ScanParams p) {
-  extern __shared__ __align__(16) uint8_t ssm[];
-  float* hs = reinterpret_cast<float*>(ssm);             // [256][16]
-  float* a0s = hs + kStepTile * 16;                        // [256][16]
-  float* a1s = a0s + kStepTile * 16;                       // [256][16]
-  float* ds = a1s + kStepTile * 16;                        // [256]
-  float* bcs = ds + kStepTile;                             // [32]: B_mix, C_mix
-  IO* xs = reinterpret_cast<IO*>(bcs + 32);                // [256]
-  IO* zs = xs + kStepTile;                                 // [256]
-  __shared__ int sel[2];
-  __shared__ float gsel[2];
-  const int tid = threadIdx.x;
-  const int tiles = (p.D + kStepTile - 1) / kStepTile;
-  const int b = blockIdx.x / tiles;
-  const int d0 = (blockIdx.x % tiles) * kStepTile;
-  const int nc = min(kStepTile, p.D - d0);  // channels of this tile (a multiple of 8)
-  const size_t tok = (size_t)b;             // seqlen == 1
-  float* hg = p.h_final + ((size_t)b * p.D + d0) * 16;
-  // group 0: everything that does not depend on the token's experts
-  for (int i = tid; i < nc * 4; i += 256) cp_async16_s(hs + 4 * i, hg + 4 * i);
-  for (int i = tid; i < nc / 4; i += 256) cp_async16_s(ds + 4 * i, p.delta + tok * p.D + d0 + 4 * i);
-  constexpr int per16 = 16 / (int)sizeof(IO);
-  for (int i = tid; i < nc / per16; i += 256) {
-    cp_async16_s(xs + per16 * i, reinterpret_cast<const IO*>(p.x) + tok * p.D + d0 + per16 * i);
-    cp_async16_s(zs + per16 * i, reinterpret_cast<const IO*>(p.z) + tok * p.D + d0 + per16 * i);
-  }
-  if (tid < 4) cp_async16_s(bcs + 4 * tid, p.B_mix + tok * 16 + 4 * tid);
-  else if (tid < 8) cp_async16_s(bcs + 16 + 4 * (tid - 4), p.C_mix + tok * 16 + 4 * (tid - 4));
-  asm volatile("cp.async.commit_group;" ::: "memory");
-  if (tid < K) {
-    sel[tid] = min(max(__ldg(p.idx + tok * K + tid), 0), p.E - 1);  // indices outside [0, E) are clamped
-    gsel[tid] = __ldg(p.gates + tok * K + tid);
+__global__ void __launch_bounds__(256, 3) step_stream_kernel(ScanParams p, int seq_per_cta) {
+  extern __shared__ float4 a_rows[];  // [E][kStepCh][4] float4 = the E experts' A rows of the tile
+  const int tid = threadIdx.x, c = tid >> 2, q = tid & 3;
+  const int tiles = (p.D + kStepCh - 1) / kStepCh;
+  const int tile = blockIdx.x % tiles, grp = blockIdx.x / tiles;
+  const int d0 = tile * kStepCh, nc = min(kStepCh, p.D - d0);  // nc % 8 == 0
+  for (int i = tid; i < p.E * nc * 4; i += 256) {
+    const int e = i / (nc * 4), r = i - e * nc * 4;
+    a_rows[e * kStepCh * 4 + r] = __ldg(reinterpret_cast<const float4*>(p.A + ((size_t)e * p.D + d0) * 16) + r);
   }
   __syncthreads();
-  // group 1: the selected experts' A tiles
-  const float* A0 = p.A + ((size_t)sel[0] * p.D + d0) * 16;
-  for (int i = tid; i < nc * 4; i += 256) cp_async16_s(a0s + 4 * i, A0 + 4 * i);
-  if (K == 2) {
-    const float* A1 = p.A + ((size_t)sel[1] * p.D + d0) * 16;
-    for (int i = tid; i < nc * 4; i += 256) cp_async16_s(a1s + 4 * i, A1 + 4 * i);
-  }
-  asm volatile("cp.async.commit_group;" ::: "memory");
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-  __syncthreads();
-  const float g0 = gsel[0], g1 = K == 2 ? gsel[1] : 0.f;
-  const int q = tid & 3;
-  const float4 bq = reinterpret_cast<const float4*>(bcs)[q];
-  const float4 cq = reinterpret_cast<const float4*>(bcs + 16)[q];
-  const float bv[4] = {bq.x, bq.y, bq.z, bq.w}, cv[4] = {cq.x, cq.y, cq.z, cq.w};
+  if (c >= nc) return;  // whole warps (8 channels each) leave together; nothing below synchronises
+  const int d = d0 + c;
+  const float dsk = p.D_skip[d];
+  const int b_begin = grp * seq_per_cta, b_end = min(p.B, b_begin + seq_per_cta);
+  for (int bb = b_begin; bb < b_end; bb += kStepU) {
+    float4 h4[kStepU], bq[kStepU], cq[kStepU];
+    float dl[kStepU], xv[kStepU], zv[kStepU], g0[kStepU], g1[kStepU];
+    int e0[kStepU], e1[kStepU];
 #pragma unroll
-  for (int r = 0; r < kStepTile / 64; ++r) {
-    const int c = (tid >> 2) + 64 * r;  // channel within the tile
-    if (c >= nc) break;                  // nc % 8 == 0: whole quads leave together
-    const float4 h4 = reinterpret_cast<const float4*>(hs)[c * 4 + q];
-    const float4 x0 = reinterpret_cast<const float4*>(a0s)[c * 4 + q];
-    const float dlt = ds[c];
-    const float xv = to_f32(xs[c]);
-    const float c0 = dlt * g0 * kLog2e;
-    float arg[4] = {c0 * x0.x, c0 * x0.y, c0 * x0.z, c0 * x0.w};
-    if (K == 2) {
-      const float4 x1 = reinterpret_cast<const float4*>(a1s)[c * 4 + q];
-      const float c1 = dlt * g1 * kLog2e;
-      arg[0] = fmaf(c1, x1.x, arg[0]);
-      arg[1] = fmaf(c1, x1.y, arg[1]);
-      arg[2] = fmaf(c1, x1.z, arg[2]);
-      arg[3] = fmaf(c1, x1.w, arg[3]);
+    for (int u = 0; u < kStepU; ++u) {
+      const int b = min(bb + u, b_end - 1);  // past the group's end: a repeat of its last sequence, not stored
+      const size_t bd = (size_t)b * p.D + d;
+      h4[u] = reinterpret_cast<const float4*>(p.h_final)[bd * 4 + q];
+      dl[u] = p.delta[bd];
+      xv[u] = to_f32(reinterpret_cast<const IO*>(p.x)[bd]);
+      zv[u] = to_f32(reinterpret_cast<const IO*>(p.z)[bd]);
+      bq[u] = __ldg(reinterpret_cast<const float4*>(p.B_mix + (size_t)b * 16) + q);
+      cq[u] = __ldg(reinterpret_cast<const float4*>(p.C_mix + (size_t)b * 16) + q);
+      e0[u] = min(max(__ldg(p.idx + (size_t)b * K), 0), p.E - 1);  // indices outside [0, E) are clamped
+      g0[u] = __ldg(p.gates + (size_t)b * K);
+      if (K == 2) {
+        e1[u] = min(max(__ldg(p.idx + (size_t)b * K + 1), 0), p.E - 1);
+        g1[u] = __ldg(p.gates + (size_t)b * K + 1);
+      }
     }
-    float h[4] = {h4.x, h4.y, h4.z, h4.w};
-    const float dx = dlt * xv;
-    float y = 0.f;
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      h[s] = fmaf(ex2_approx(arg[s]), h[s], dx * bv[s]);
-      y = fmaf(cv[s], h[s], y);
-    }
-    y += __shfl_xor_sync(0xffffffffu, y, 1);
-    y += __shfl_xor_sync(0xffffffffu, y, 2);
-    reinterpret_cast<float4*>(hg)[c * 4 + q] = make_float4(h[0], h[1], h[2], h[3]);
-    if (q == 0) {
-      const int d = d0 + c;
-      y = fmaf(p.D_skip[d], xv, y);
-      if (p.y_pre != nullptr) p.y_pre[tok * p.D + d] = y;
-      from_f32(reinterpret_cast<IO*>(p.out)[tok * p.D + d], silu_gate(y, to_f32(zs[c])));
+    for (int u = 0; u < kStepU; ++u) {
+      if (bb + u >= b_end) break;
+      const size_t bd = (size_t)(bb + u) * p.D + d;
+      const float4 a0 = a_rows[(e0[u] * kStepCh + c) * 4 + q];
+      const float c0 = dl[u] * g0[u] * kLog2e;
+      float arg[4] = {c0 * a0.x, c0 * a0.y, c0 * a0.z, c0 * a0.w};
+      if (K == 2) {
+        const float4 a1 = a_rows[(e1[u] * kStepCh + c) * 4 + q];
+        const float c1 = dl[u] * g1[u] * kLog2e;
+        arg[0] = fmaf(c1, a1.x, arg[0]);
+        arg[1] = fmaf(c1, a1.y, arg[1]);
+        arg[2] = fmaf(c1, a1.z, arg[2]);
+        arg[3] = fmaf(c1, a1.w, arg[3]);
+      }
+      float h[4] = {h4[u].x, h4[u].y, h4[u].z, h4[u].w};
+      const float bv[4] = {bq[u].x, bq[u].y, bq[u].z, bq[u].w}, cv[4] = {cq[u].x, cq[u].y, cq[u].z, cq[u].w};
+      const float dx = dl[u] * xv[u];
+      float y = 0.f;
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        h[s] = fmaf(ex2_approx(arg[s]), h[s], dx * bv[s]);
+        y = fmaf(cv[s], h[s], y);
+      }
+      y += __shfl_xor_sync(0xffffffffu, y, 1);
+      y += __shfl_xor_sync(0xffffffffu, y, 2);
+      reinterpret_cast<float4*>(p.h_final)[bd * 4 + q] = make_float4(h[0], h[1], h[2], h[3]);
+      if (q == 0) {
+        y = fmaf(dsk, xv[u], y);
+        if (p.y_pre != nullptr) p.y_pre[bd] = y;
+        from_f32(reinterpret_cast<IO*>(p.out)[bd], silu_gate(y, zv[u]));
+      }
     }
   }
 }
 
 template <typename IO, int K>
-static cudaError_t launch_step_bulk(const ScanParams& p, cudaStream_t s) {
-  const size_t smem = sizeof(float) * (3 * kStepTile * 16 + kStepTile + 32) + 2 * kStepTile * sizeof(IO);
-  cudaError_t e = cudaFuncSetAttribute(step_bulk_kernel<IO, K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+static cudaError_t launch_step_stream(const ScanParams& p, cudaStream_t s) {
+  const size_t smem = sizeof(float4) * (size_t)p.E * kStepCh * 4;
+  cudaError_t e = cudaFuncSetAttribute(step_stream_kernel<IO, K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int tiles = (p.D + kStepTile - 1) / kStepTile;
-  step_bulk_kernel<IO, K><<<(unsigned)(p.B * tiles), 256, smem, s>>>(p);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int tiles = (p.D + kStepCh - 1) / kStepCh;
+  int groups = std::max(1, std::min(p.B, (3 * sms + tiles - 1) / tiles));
+  const int spc = (p.B + groups - 1) / groups;
+  groups = (p.B + spc - 1) / spc;
+  step_stream_kernel<IO, K><<<(unsigned)(tiles * groups), 256, smem, s>>>(p, spc);
   note_launch();
   return cudaGetLastError();
 }
@@ -387,7 +374,7 @@ template <typename IO, int K>
 static cudaError_t launch_scan(const ScanParams& p, bool step, cudaStream_t s) {
   const size_t smem = sizeof(float) * (size_t)p.E * kDT * kNMax;
   const unsigned gx = (unsigned)((p.D + kDT - 1) / kDT);
-  if (step && p.N == kNMax && (K == 1 || K == 2)) return launch_step_bulk<IO, (K == 2 ? 2 : 1)>(p, s);
+  if (step && p.N == kNMax && (K == 1 || K == 2)) return launch_step_stream<IO, (K == 2 ? 2 : 1)>(p, s);
   if (step) {
     const int64_t threads = (int64_t)p.B * p.D * kG;
     step_kernel<IO, K><<<(unsigned)((threads + 127) / 128), 128, 0, s>>>(p);
