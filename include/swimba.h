@@ -61,7 +61,10 @@ enum {
   SWIMBA_OP_STEP = 3,
   SWIMBA_OP_LAYER = 4,  /* large enough for every op of the layer */
   SWIMBA_OP_SUMMARY = 5, /* swimba_scan_summary */
-  SWIMBA_OP_SEPARATE = 6 /* swimba_separate_scan */
+  SWIMBA_OP_SEPARATE = 6, /* swimba_separate_scan */
+  SWIMBA_OP_SCAN_BWD = 7,  /* swimba_scan_bwd */
+  SWIMBA_OP_PROJ_BWD = 8,  /* swimba_proj_bwd */
+  SWIMBA_OP_ROUTE_BWD = 9  /* swimba_route_bwd */
 };
 
 typedef struct {
@@ -141,6 +144,67 @@ swimba_status swimba_scan_fwd_zoh(const swimba_dims *dims, const void *x, const 
                                   const int32_t *idx, const float *gates, const swimba_weights *w,
                                   const float *h0, void *out, float *h_final, float *y_pre, void *ws,
                                   size_t ws_bytes, void *stream);
+
+/* Backward pass of swimba_scan_fwd (Euler injection): the exact gradients of the scan's outputs
+ * with respect to its inputs, given g_out = dL/dout. The pages train Swimba-14B ("Swimba: Switch
+ * Mamba Model Scales State Space Models", Dutch summary, "Resultaten") but give no training
+ * details; this is reverse-mode differentiation of the forward above:
+ *   dy_t = g_out,t SiLU(z_t);  dz_t = g_out,t y_t SiLU'(z_t)
+ *   lambda_t = C_mix,t dy_t + exp(delta_{t+1} A_{t+1}) lambda_{t+1}      (per channel and state)
+ *   dx_t = D dy_t + delta_t sum_n lambda_t B_mix,t;  dB_t = sum_d lambda_t delta_t x_t;
+ *   dC_t = sum_d dy_t h_t;  ddelta_t = sum_n lambda_t (A_t a_t h_{t-1} + B_mix,t x_t);
+ *   dA^e += g_j lambda_t delta_t a_t h_{t-1} (e = idx_j);  dgates_j = sum_{d,n} of that times A^e;
+ *   dD = sum_t dy_t x_t;  dh0 = exp(delta_0 A_0) lambda_0.
+ * The forward states are recomputed (checkpoints every 16 tokens, kept in ws), not read from the
+ * forward call.
+ *   Inputs as swimba_scan_fwd (x, z, g_out in io_dtype; delta, B_mix, C_mix, gates, A, D_skip, h0
+ *   fp32); g_out [B, L, D] required.
+ *   Outputs, fp32, all required except dh0: dx, dz, ddelta [B, L, D]; dB, dC [B, L, N];
+ *   dgates [B, L, k]; dA [E, D, N] (w's A table shape); dD [D]; dh0 [B, D, N] or NULL.
+ *   The sums over channels, tokens and sequences are taken in a fixed order (deterministic).
+ *   ws: at least swimba_workspace_size(dims, SWIMBA_OP_SCAN_BWD) bytes (checkpoints and partial
+ *   sums: about B L D N / 4 + B L (2N + k) D / 16 floats). No pointer may alias another. */
+swimba_status swimba_scan_bwd(const swimba_dims *dims, const void *x, const void *z,
+                              const float *delta, const float *B_mix, const float *C_mix,
+                              const int32_t *idx, const float *gates, const swimba_weights *w,
+                              const float *h0, const void *g_out, float *dx, float *dz,
+                              float *ddelta, float *dB, float *dC, float *dgates, float *dA,
+                              float *dD, float *dh0, void *ws, size_t ws_bytes, void *stream);
+
+/* Backward pass of swimba_mixed_proj: given dL/ddelta (g_delta, e.g. swimba_scan_bwd's ddelta) and
+ * dL/dB_mix, dL/dC_mix, the gradients of the mixed projection's inputs and weights ("Swimba: Switch
+ * Mamba Model Scales State Space Models", §2 "Generación de Parámetros" / "Mezcla en el Espacio de
+ * Parámetros": v_j = x W_x^{e_j} = [dt_low | B | C], dt_j = dt_low W_dt^{e_j} + b_dt^{e_j},
+ * delta = softplus(sum_j g_j dt_j), B_mix = sum_j g_j B_j, C_mix = sum_j g_j C_j; the pages give no
+ * training details, this is the exact reverse-mode gradient). softplus' derivative is taken from
+ * delta itself: sigma(dt_mix) = 1 - exp(-delta).
+ *   x [B, L, D] bf16; idx, gates [B, L, k] (the router's); w: W_x, W_dt (bf16), b_dt (fp32);
+ *   delta [B, L, D] fp32 (the forward's output); g_delta [B, L, D], g_B, g_C [B, L, N] fp32.
+ *   Outputs fp32: dx [B, L, D] (overwritten, or added to when dx_accumulate != 0);
+ *   dgates [B, L, k] (this step's part of dL/dgates); dW_x [E, D, R+2N]; dW_dt [E, R, D];
+ *   db_dt [E, D] (every expert's, zeros for an expert no token chose).
+ * Products run on the tensor cores with bf16 operands (x, dL/d(dt_mix), and the per-token rows
+ * built from them are rounded to bf16 once) and fp32 accumulation. Needs io_dtype = w_dtype =
+ * bf16, R % 8 == 0, N % 4 == 0 (SWIMBA_ERR_UNSUPPORTED otherwise). The call reads the number of
+ * (token, slot) pairs per expert back to the host once, so it synchronises `stream` and cannot be
+ * captured in a CUDA graph. ws: swimba_workspace_size(dims, SWIMBA_OP_PROJ_BWD) bytes. */
+swimba_status swimba_proj_bwd(const swimba_dims *dims, const void *x, const int32_t *idx,
+                              const float *gates, const swimba_weights *w, const float *delta,
+                              const float *g_delta, const float *g_B, const float *g_C, float *dx,
+                              int32_t dx_accumulate, float *dgates, float *dW_x, float *dW_dt,
+                              float *db_dt, void *ws, size_t ws_bytes, void *stream);
+
+/* Backward pass of swimba_route: the gates are the softmax of the k selected logits of x W_r (the
+ * selection itself is piecewise constant and carries no gradient). With G = g_gates_a (+ g_gates_b
+ * when not NULL, e.g. the scan's and the projection's parts of dL/dgates):
+ *   dL/dlogit_{idx_j} = gates_j (G_j - sum_i gates_i G_i);  dx += dlogits W_r^T;  dW_r = x^T dlogits.
+ *   x [B, L, D] io_dtype; W_r [D, E] fp32; idx, gates, g_gates_* [B, L, k] fp32.
+ *   dx [B, L, D] fp32 (overwritten, or added to when dx_accumulate != 0); dW_r [D, E] fp32.
+ *   ws: swimba_workspace_size(dims, SWIMBA_OP_ROUTE_BWD) bytes. */
+swimba_status swimba_route_bwd(const swimba_dims *dims, const void *x, const float *W_r,
+                               const int32_t *idx, const float *gates, const float *g_gates_a,
+                               const float *g_gates_b, float *dx, int32_t dx_accumulate,
+                               float *dW_r, void *ws, size_t ws_bytes, void *stream);
 
 /* swimba_scan_fwd without a caller workspace, for callers that cannot allocate device memory: a
  * plugin inside a framework that owns all device memory and gives it no allocator, or a

@@ -19,7 +19,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libswimba.so")
 SOURCES = [
     "api.cu", "route.cu", "route_tc.cu", "proj_simt.cu", "proj_tc.cu", "scan.cu", "scan_fast.cu", "conv.cu",
-    "block.cu", "separate.cu", "ssd.cu", "gemm.cu",
+    "block.cu", "separate.cu", "ssd.cu", "gemm.cu", "scan_bwd.cu", "proj_bwd.cu",
 ]
 LIBS: list = []
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

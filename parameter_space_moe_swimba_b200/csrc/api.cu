@@ -23,6 +23,14 @@ cudaError_t separate_scan_entry(const void* x, const void* z, const float* dj, c
                                 const int32_t* idx, const float* gates, const float* A, const float* D_skip,
                                 const float* h0, void* out, float* h_final, float* y_pre, void* status, int64_t L,
                                 int B, int D, int N, int E, int k, bool io_bf16, cudaStream_t s);
+size_t proj_bwd_workspace(int64_t T, int D, int R, int N, int E, int k);
+cudaError_t run_proj_bwd(const void* x, const float* delta, const float* g_delta, const float* gB, const float* gC,
+                         const int32_t* idx, const float* gates, const void* W_x, const void* W_dt, const void* b_dt,
+                         bool b_bf16, float* dx, int accumulate, float* dgates, float* dW_x, float* dW_dt, float* db,
+                         int64_t T, int D, int R, int N, int E, int k, void* ws, void* status, cudaStream_t s);
+cudaError_t run_route_bwd(const void* x, bool io_bf16, const float* W_r, const int32_t* idx, const float* gates,
+                          const float* gg_a, const float* gg_b, float* dlogits, float* dx, int accumulate, float* dW_r,
+                          int64_t T, int D, int E, int k, cudaStream_t s);
 bool ssd_supported(int P, int N, int k);
 cudaError_t run_ssd(const void* X, const void* Bm, const void* Cmix, const float* gates, const float* delta,
                     const float* A, const float* D_skip, const float* S0, float* y, float* S_final, void* status,
@@ -145,6 +153,14 @@ size_t swimba_workspace_size(const swimba_dims* dims, int op) {
       return summary_workspace(dims);
     case SWIMBA_OP_SEPARATE:
       return kStatusBytes;
+    case SWIMBA_OP_PROJ_BWD:
+      return kStatusBytes + proj_bwd_workspace(dims->batch * dims->seqlen, dims->d_inner, dims->dt_rank,
+                                               dims->d_state, dims->n_experts, dims->top_k);
+    case SWIMBA_OP_ROUTE_BWD:
+      return kStatusBytes + (size_t)dims->batch * dims->seqlen * dims->n_experts * 4;
+    case SWIMBA_OP_SCAN_BWD:
+      return kStatusBytes + scan_bwd_workspace(dims->batch, dims->seqlen, dims->d_inner, dims->d_state,
+                                               dims->n_experts, dims->top_k);
     default:
       return 0;
   }
@@ -228,6 +244,87 @@ swimba_status swimba_scan_fwd_zoh(const swimba_dims* dims, const void* x, const 
   if (!aligned16(ws)) return SWIMBA_ERR_ALIGN;
   return scan_common(dims, x, z, delta, B_mix, C_mix, idx, gates, w, h0, out, h_final, y_pre, false, ws, stream,
                      true);
+}
+
+swimba_status swimba_scan_bwd(const swimba_dims* dims, const void* x, const void* z, const float* delta,
+                              const float* B_mix, const float* C_mix, const int32_t* idx, const float* gates,
+                              const swimba_weights* w, const float* h0, const void* g_out, float* dx, float* dz,
+                              float* ddelta, float* dB, float* dC, float* dgates, float* dA, float* dD, float* dh0,
+                              void* ws, size_t ws_bytes, void* stream) {
+  swimba_status st = check_dims(dims);
+  if (st != SWIMBA_OK) return st;
+  if (!x || !z || !delta || !B_mix || !C_mix || !idx || !gates || !w || !w->A || !w->D_skip || !g_out || !dx || !dz ||
+      !ddelta || !dB || !dC || !dgates || !dA || !dD)
+    return SWIMBA_ERR_INVALID_ARG;
+  if (!aligned16(w->A) || !aligned16(ws) || (h0 && !aligned16(h0)) || (dh0 && !aligned16(dh0)))
+    return SWIMBA_ERR_ALIGN;
+  if (ws == nullptr || ws_bytes < swimba_workspace_size(dims, SWIMBA_OP_SCAN_BWD)) return SWIMBA_ERR_WORKSPACE;
+  ScanBwdParams p{};
+  p.x = x;
+  p.z = z;
+  p.delta = delta;
+  p.B_mix = B_mix;
+  p.C_mix = C_mix;
+  p.idx = idx;
+  p.gates = gates;
+  p.A = w->A;
+  p.D_skip = w->D_skip;
+  p.h0 = h0;
+  p.g_out = g_out;
+  p.dx = dx;
+  p.dz = dz;
+  p.ddelta = ddelta;
+  p.dB = dB;
+  p.dC = dC;
+  p.dgates = dgates;
+  p.dA = dA;
+  p.dD = dD;
+  p.dh0 = dh0;
+  p.L = dims->seqlen;
+  p.B = (int)dims->batch;
+  p.D = dims->d_inner;
+  p.N = dims->d_state;
+  p.E = dims->n_experts;
+  p.k = dims->top_k;
+  return cuda_status(run_scan_bwd(p, dims->io_dtype == SWIMBA_BF16, static_cast<uint8_t*>(ws) + kStatusBytes,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+swimba_status swimba_proj_bwd(const swimba_dims* dims, const void* x, const int32_t* idx, const float* gates,
+                              const swimba_weights* w, const float* delta, const float* g_delta, const float* g_B,
+                              const float* g_C, float* dx, int32_t dx_accumulate, float* dgates, float* dW_x,
+                              float* dW_dt, float* db_dt, void* ws, size_t ws_bytes, void* stream) {
+  swimba_status st = check_dims(dims);
+  if (st != SWIMBA_OK) return st;
+  if (!x || !idx || !gates || !w || !w->W_x || !w->W_dt || !w->b_dt || !delta || !g_delta || !g_B || !g_C || !dx ||
+      !dgates || !dW_x || !dW_dt || !db_dt)
+    return SWIMBA_ERR_INVALID_ARG;
+  const int64_t T = dims->batch * dims->seqlen;
+  if (dims->io_dtype != SWIMBA_BF16 || dims->w_dtype != SWIMBA_BF16 || dims->dt_rank % 8 != 0 ||
+      dims->d_state % 4 != 0 || T * dims->top_k >= (int64_t(1) << 31))
+    return SWIMBA_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(delta) || !aligned16(g_delta) || !aligned16(dx) || !aligned16(dW_x) ||
+      !aligned16(dW_dt) || !aligned16(db_dt) || !aligned16(w->W_x) || !aligned16(w->W_dt) || !aligned16(ws))
+    return SWIMBA_ERR_ALIGN;
+  if (ws == nullptr || ws_bytes < swimba_workspace_size(dims, SWIMBA_OP_PROJ_BWD)) return SWIMBA_ERR_WORKSPACE;
+  return cuda_status(run_proj_bwd(x, delta, g_delta, g_B, g_C, idx, gates, w->W_x, w->W_dt, w->b_dt, false, dx,
+                                  dx_accumulate ? 1 : 0, dgates, dW_x, dW_dt, db_dt, T, dims->d_inner, dims->dt_rank,
+                                  dims->d_state, dims->n_experts, dims->top_k, static_cast<uint8_t*>(ws) + kStatusBytes,
+                                  ws, static_cast<cudaStream_t>(stream)));
+}
+
+swimba_status swimba_route_bwd(const swimba_dims* dims, const void* x, const float* W_r, const int32_t* idx,
+                               const float* gates, const float* g_gates_a, const float* g_gates_b, float* dx,
+                               int32_t dx_accumulate, float* dW_r, void* ws, size_t ws_bytes, void* stream) {
+  swimba_status st = check_dims(dims);
+  if (st != SWIMBA_OK) return st;
+  if (!x || !W_r || !idx || !gates || !g_gates_a || !dx || !dW_r) return SWIMBA_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return SWIMBA_ERR_ALIGN;
+  if (ws == nullptr || ws_bytes < swimba_workspace_size(dims, SWIMBA_OP_ROUTE_BWD)) return SWIMBA_ERR_WORKSPACE;
+  float* dlogits = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kStatusBytes);
+  return cuda_status(run_route_bwd(x, dims->io_dtype == SWIMBA_BF16, W_r, idx, gates, g_gates_a, g_gates_b, dlogits,
+                                   dx, dx_accumulate ? 1 : 0, dW_r, dims->batch * dims->seqlen, dims->d_inner,
+                                   dims->n_experts, dims->top_k, static_cast<cudaStream_t>(stream)));
 }
 
 swimba_status swimba_scan_fwd_noalloc(const swimba_dims* dims, const void* x, const void* z, const float* delta,

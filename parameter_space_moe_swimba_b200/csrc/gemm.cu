@@ -9,16 +9,18 @@
 //                                                 and z buffers)
 //   out-projection:  o = y W_out + u             (the residual is added in the epilogue)
 //
-// C[M, N] = A[M, K] B[K, N] (+ R[M, N]), bf16 operands as stored (A row-major with K contiguous,
-// B row-major with N contiguous), fp32 accumulation in tensor memory, bf16 out. Persistent,
-// warp-specialised: warp 0 streams A tiles [128 x 64] (K-major, 128-byte swizzle) and B tiles
-// [64 x 256] (four MN-major boxes) by TMA through a 4-stage ring; warp 1 issues tcgen05.mma
-// M=128, N=256, K=16 into one of two 256-column TMEM accumulators; warps 2-5 drain the other
-// accumulator (one TMEM lane = one output row) while the next tile accumulates. Tiles go in
-// M-fastest order, so consecutive CTAs share the weight columns they read from L2. Every wait is
-// bounded: a wait that runs out records SWIMBA_ERR_TIMEOUT in the status block, the CTA lets its
-// copies land, frees TMEM and exits. fp32 operands take a SIMT kernel (tiles of 64 x 64 in
-// shared memory).
+// C[M, N] = A[M, K] B[K, N] (+ R[M, N]), bf16 operands as stored, fp32 accumulation in tensor
+// memory, bf16 or fp32 out. A is stored either [M, K] (K contiguous, "K-major") or [K, M] (M
+// contiguous: the transpose of a stored matrix, as the weight gradients x^T dV need); B is stored
+// either [K, N] (N contiguous) or [N, K] (K contiguous: a stored weight used transposed, as the
+// input gradients dV W^T need). Persistent, warp-specialised: warp 0 streams the A tile [128 x 64]
+// and the B tile [64 x 256] of each k-step by TMA (128-byte swizzle; MN-major operands as 64-wide
+// boxes) through a 4-stage ring; warp 1 issues tcgen05.mma M=128, N=256, K=16 into one of two
+// 256-column TMEM accumulators; warps 2-5 drain the other accumulator (one TMEM lane = one output
+// row) while the next tile accumulates. Tiles go in M-fastest order, so consecutive CTAs share the
+// weight columns they read from L2. Every wait is bounded: a wait that runs out records
+// SWIMBA_ERR_TIMEOUT in the status block, the CTA lets its copies land, frees TMEM and exits. fp32
+// operands take a SIMT kernel (tiles of 64 x 64 in shared memory).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -54,6 +56,7 @@ struct GemmParams {
 
 }  // namespace
 
+template <bool A_MN, bool B_K, bool F32OUT>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                    const GemmParams p) {
@@ -107,8 +110,17 @@ __global__ void __launch_bounds__(192, 1)
         uint8_t* st = smem + stage * kGStage;
         if (lane == 0) {
           mbar_arrive_expect_tx(&full[stage], (uint32_t)kGStage);
-          tma_load_2d(st, &tm_a, &full[stage], k * GBK, m0);
-          for (int i = 0; i < 4; ++i) tma_load_2d(st + kGA + i * 8192, &tm_b, &full[stage], n0 + 64 * i, k * GBK);
+          if (A_MN) {  // two 64-column boxes of the stored [K, M]
+            tma_load_2d(st, &tm_a, &full[stage], m0, k * GBK);
+            tma_load_2d(st + 8192, &tm_a, &full[stage], m0 + 64, k * GBK);
+          } else {
+            tma_load_2d(st, &tm_a, &full[stage], k * GBK, m0);
+          }
+          if (B_K) {  // one box of 256 rows of the stored [N, K]
+            tma_load_2d(st + kGA, &tm_b, &full[stage], k * GBK, n0);
+          } else {
+            for (int i = 0; i < 4; ++i) tma_load_2d(st + kGA + i * 8192, &tm_b, &full[stage], n0 + 64 * i, k * GBK);
+          }
         }
         __syncwarp();
         ++issued;
@@ -135,7 +147,7 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(GBM, GBN, /*b_mn_major=*/true);
+      const uint32_t idesc = idesc_bf16(GBM, GBN, /*b_mn_major=*/!B_K, /*a_mn_major=*/A_MN);
       const uint32_t base = smem_u32(smem);
       int stage = 0, buf = 0;
       uint32_t phase = 0;
@@ -157,8 +169,11 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t sa = base + stage * kGStage, sb = sa + kGA;
 #pragma unroll
           for (int kk = 0; kk < GBK / 16; ++kk) {
-            mma_bf16(tmem + buf * GBN, smem_desc(sa + kk * 32, 16, 1024, kLayoutSW128),
-                     smem_desc(sb + kk * 16 * 128, 8192, 1024, kLayoutSW128), idesc, (k | kk) != 0 ? 1u : 0u);
+            const uint64_t adesc = A_MN ? smem_desc(sa + kk * 16 * 128, 8192, 1024, kLayoutSW128)
+                                        : smem_desc(sa + kk * 32, 16, 1024, kLayoutSW128);
+            const uint64_t bdesc = B_K ? smem_desc(sb + kk * 32, 16, 1024, kLayoutSW128)
+                                       : smem_desc(sb + kk * 16 * 128, 8192, 1024, kLayoutSW128);
+            mma_bf16(tmem + buf * GBN, adesc, bdesc, idesc, (k | kk) != 0 ? 1u : 0u);
           }
           mma_commit(&empty[stage]);
           if (++stage == kGStages) {
@@ -205,7 +220,28 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int j = 0; j < 32; j += 8) {  // groups of 8 columns (N and split are multiples of 8)
             const int col = n + j;
-            if (col < p.N) {
+            if (col < p.N && F32OUT) {
+              float o[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) o[e] = v[j + e];
+              if (p.R != nullptr) {
+                const float4* r4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.R) +
+                                                                   (size_t)m * p.ldr + col);
+                const float4 r0 = r4[0], r1 = r4[1];
+                o[0] += r0.x;
+                o[1] += r0.y;
+                o[2] += r0.z;
+                o[3] += r0.w;
+                o[4] += r1.x;
+                o[5] += r1.y;
+                o[6] += r1.z;
+                o[7] += r1.w;
+              }
+              float* out = col < p.split ? reinterpret_cast<float*>(p.C0) + (size_t)m * p.ldc0 + col
+                                         : reinterpret_cast<float*>(p.C1) + (size_t)m * p.ldc1 + (col - p.split);
+              reinterpret_cast<float4*>(out)[0] = make_float4(o[0], o[1], o[2], o[3]);
+              reinterpret_cast<float4*>(out)[1] = make_float4(o[4], o[5], o[6], o[7]);
+            } else if (col < p.N) {
               float o[8];
 #pragma unroll
               for (int e = 0; e < 8; ++e) o[e] = v[j + e];
@@ -309,6 +345,46 @@ bool gemm_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int6
 
 }  // namespace
 
+template <bool A_MN, bool B_K, bool F32OUT>
+cudaError_t launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, cudaStream_t s) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int tiles = ((p.M + GBM - 1) / GBM) * ((p.N + GBN - 1) / GBN);
+  const size_t smem = 1024 + (size_t)kGStages * kGStage + 256;  // ring, then barriers and the TMEM slot
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<A_MN, B_K, F32OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  gemm_tc_kernel<A_MN, B_K, F32OUT><<<(unsigned)std::min(tiles, sms), 192, smem, s>>>(ta, tb, p);
+  note_launch();
+  return cudaGetLastError();
+}
+
+// The tensor-core GEMM in its four operand layouts: A stored [M, K] (a_t = false, row stride lda)
+// or [K, M] (a_t = true); B stored [K, N] (b_t = false, row stride ldb) or [N, K] (b_t = true).
+// bf16 operands; out (C0 below column `split`, C1 from it) and the optional residual R are bf16 or,
+// with f32_out, fp32. Row strides must be multiples of 8 elements (bf16) and pointers 16-byte aligned.
+cudaError_t run_gemm_tc(bool a_t, bool b_t, bool f32_out, int M, int N, int K, const void* A, int lda, const void* B,
+                        int ldb, void* C0, int ldc0, void* C1, int ldc1, int split, const void* R, int ldr,
+                        void* status, cudaStream_t s) {
+  CUtensorMap ta, tb;
+  const bool ok_a = a_t ? gemm_map(&ta, A, K, M, lda, GBK) : gemm_map(&ta, A, M, K, lda, GBM);
+  const bool ok_b = b_t ? gemm_map(&tb, B, N, K, ldb, GBN) : gemm_map(&tb, B, K, N, ldb, GBK);
+  if (!ok_a || !ok_b) return cudaErrorInvalidValue;
+  GemmParams p{C0, C1, R, status, M, N, K, split, ldc0, ldc1, ldr};
+  const int sel = (a_t ? 4 : 0) | (b_t ? 2 : 0) | (f32_out ? 1 : 0);
+  switch (sel) {
+    case 0: return launch_gemm_tc<false, false, false>(ta, tb, p, s);
+    case 1: return launch_gemm_tc<false, false, true>(ta, tb, p, s);
+    case 2: return launch_gemm_tc<false, true, false>(ta, tb, p, s);
+    case 3: return launch_gemm_tc<false, true, true>(ta, tb, p, s);
+    case 4: return launch_gemm_tc<true, false, false>(ta, tb, p, s);
+    case 5: return launch_gemm_tc<true, false, true>(ta, tb, p, s);
+    case 6: return launch_gemm_tc<true, true, false>(ta, tb, p, s);
+    default: return launch_gemm_tc<true, true, true>(ta, tb, p, s);
+  }
+}
+
 // C[M, N] = A[M, K] (row stride lda) B[K, N] (row stride ldb) (+ R, row stride ldr): columns below
 // `split` go to C0 (row stride ldc0), the others to C1 (ldc1). bf16 needs every row stride and
 // split a multiple of 8 elements and 16-byte aligned pointers.
@@ -323,19 +399,7 @@ cudaError_t run_block_gemm(bool bf16, int M, int N, int K, const void* A, int ld
     note_launch();
     return cudaGetLastError();
   }
-  CUtensorMap ta, tb;
-  if (!gemm_map(&ta, A, M, K, lda, GBM) || !gemm_map(&tb, B, K, N, ldb, GBK)) return cudaErrorInvalidValue;
-  GemmParams p{C0, C1, R, status, M, N, K, split, ldc0, ldc1, ldr};
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int tiles = ((M + GBM - 1) / GBM) * ((N + GBN - 1) / GBN);
-  const size_t smem = 1024 + (size_t)kGStages * kGStage + 256;  // ring, then barriers and the TMEM slot
-  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  gemm_tc_kernel<<<(unsigned)std::min(tiles, sms), 192, smem, s>>>(ta, tb, p);
-  note_launch();
-  return cudaGetLastError();
+  return run_gemm_tc(false, false, false, M, N, K, A, lda, B, ldb, C0, ldc0, C1, ldc1, split, R, ldr, status, s);
 }
 
 }  // namespace swimba

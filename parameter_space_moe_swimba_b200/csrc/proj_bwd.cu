@@ -1,0 +1,430 @@
+// Backward pass of the mixed expert projection and of the router.
+//
+// Source of the forward: "Swimba: Switch Mamba Model Scales State Space Models", §2 "Generación de
+// Parámetros" / "Mezcla en el Espacio de Parámetros" (es), "Kernmechanisme van Swimba" (nl): per
+// active expert e_j of token t, v_j = x_t W_x^{e_j} = [dt_low_j | B_j | C_j],
+// dt_j = dt_low_j W_dt^{e_j} + b_dt^{e_j}; the streams mix with the gates g_j; Δ = softplus(Σ g_j dt_j).
+// The router's gates are the softmax of the k selected logits of x W_r. The pages give no training
+// details; these are the exact gradients of that forward (reverse mode), with bf16 MMA operands:
+//   g_dt      = ∂L/∂Δ σ(dt_mix) = ∂L/∂Δ (1 − e^{−Δ})               (Δ = softplus(dt_mix))
+//   q_j       = W_dt^{e_j} g_dt                                     [R]
+//   ∂L/∂g_j   = dt_low_j · q_j + b_dt^{e_j} · g_dt + B_j · ∂L/∂B_mix + C_j · ∂L/∂C_mix
+//   dV_j      = [g_j q_j | g_j ∂L/∂B_mix | g_j ∂L/∂C_mix]            [R + 2N]
+//   ∂L/∂x    += Σ_j W_x^{e_j} dV_j;   ∂L/∂W_x^e = Σ_{(t,j): e} x_tᵀ dV_j
+//   ∂L/∂W_dt^e = Σ_{(t,j): e} (g_j dt_low_j)ᵀ g_dt;   ∂L/∂b_dt^e = Σ_{(t,j): e} g_j g_dt
+//   router: ∂L/∂s_j = g_j (∂L/∂g_j − Σ_i g_i ∂L/∂g_i) on the selected logits s;
+//           ∂L/∂x += Σ_e ∂L/∂logit_e W_r[:, e];  ∂L/∂W_r = Σ_t x_tᵀ ∂L/∂logits_t.
+//
+// Layout of the work: the (token, slot) pairs are sorted by expert (a stable counting sort), so
+// every product above is a dense GEMM per expert on contiguous rows, run by the library's tcgen05
+// GEMM (gemm.cu) in its transposed-operand forms: the rows' x and g_dt are gathered once into bf16
+// matrices Xg and G; v (recomputed, fp32) = Xg W_x^e and q = G W_dt^eᵀ; then a per-pair kernel forms
+// dV, g_j dt_low (with g_j appended as an extra column, so that the W_dt GEMM also yields the bias
+// gradient) and the gate gradient; then Xgᵀ dV = ∂L/∂W_x^e, (g dt_low | g)ᵀ G = [∂L/∂W_dt^e ; ∂L/∂b_dt^e],
+// dV W_x^eᵀ = the pairs' input gradients, summed per token in slot order. The expert sizes are read
+// back to the host once per call (so the GEMM shapes are exact); that makes this entry point
+// synchronise its stream, unlike the forward ones.
+#include <vector>
+
+#include "common.cuh"
+
+namespace swimba {
+
+cudaError_t run_gemm_tc(bool a_t, bool b_t, bool f32_out, int M, int N, int K, const void* A, int lda, const void* B,
+                        int ldb, void* C0, int ldc0, void* C1, int ldc1, int split, const void* R, int ldr,
+                        void* status, cudaStream_t s);
+
+namespace {
+
+constexpr int kSortThreads = 1024;
+constexpr int kMaxE = 16;
+
+// Stable counting sort of the P = T k pairs by expert, one CTA: each thread counts a contiguous
+// run of pairs per expert, an exclusive scan over the threads (per expert) gives every thread's
+// first slot, and the run is scattered in order. perm[row] = pair, inv[pair] = row,
+// counts[e] = pairs of expert e, offsets[e] = first row of expert e.
+__global__ void __launch_bounds__(kSortThreads) pair_sort_kernel(const int32_t* idx, int64_t P, int E, int* counts,
+                                                                 int* offsets, int* perm, int* inv) {
+  extern __shared__ int cnt[];  // [E][kSortThreads]
+  const int tid = threadIdx.x;
+  const int64_t per = (P + kSortThreads - 1) / kSortThreads;
+  const int64_t p0 = min(P, per * tid), p1 = min(P, p0 + per);
+  int local[kMaxE];
+#pragma unroll
+  for (int e = 0; e < kMaxE; ++e) local[e] = 0;
+  for (int64_t p = p0; p < p1; ++p) {
+    const int e = min(max(idx[p], 0), E - 1);
+#pragma unroll
+    for (int ee = 0; ee < kMaxE; ++ee) local[ee] += (ee == e);
+  }
+  for (int e = 0; e < E; ++e) cnt[e * kSortThreads + tid] = local[e];
+  __syncthreads();
+  // exclusive scan per expert over the threads (thread e < E walks its row; E <= 16 rows)
+  __shared__ int base[kMaxE + 1];
+  if (tid < E) {
+    int run = 0;
+    for (int i = 0; i < kSortThreads; ++i) {
+      const int v = cnt[tid * kSortThreads + i];
+      cnt[tid * kSortThreads + i] = run;
+      run += v;
+    }
+    counts[tid] = run;
+    base[tid] = run;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int o = 0;
+    for (int e = 0; e < E; ++e) {
+      const int n = base[e];
+      base[e] = o;
+      offsets[e] = o;
+      o += n;
+    }
+    base[E] = o;
+    offsets[E] = o;
+  }
+  __syncthreads();
+  int next[kMaxE];
+#pragma unroll
+  for (int e = 0; e < kMaxE; ++e) next[e] = e < E ? base[e] + cnt[e * kSortThreads + tid] : 0;
+  for (int64_t p = p0; p < p1; ++p) {
+    const int e = min(max(idx[p], 0), E - 1);
+    int row = 0;
+#pragma unroll
+    for (int ee = 0; ee < kMaxE; ++ee)
+      if (ee == e) row = next[ee]++;
+    perm[row] = (int)p;
+    inv[p] = row;
+  }
+}
+
+// One CTA per sorted row: Xg[row] = x[t] (bf16), G[row] = bf16(g_dt[t]) with
+// g_dt = ∂L/∂Δ (1 − e^{−Δ}), and bg[row] = b_dt^e · g_dt (fp32).
+template <typename WT>
+__global__ void __launch_bounds__(256) proj_bwd_gather_kernel(const __nv_bfloat16* x, const float* delta,
+                                                              const float* g_delta, const int32_t* idx,
+                                                              const WT* b_dt, const int* perm, int k, int D, int E,
+                                                              __nv_bfloat16* Xg, __nv_bfloat16* G, float* bg) {
+  const int row = blockIdx.x;
+  const int p = perm[row];
+  const int64_t t = p / k;
+  const int e = min(max(idx[p], 0), E - 1);
+  const __nv_bfloat16* xr = x + t * D;
+  float part = 0.f;
+  for (int c = threadIdx.x * 8; c < D; c += 256 * 8) {  // D % 8 == 0
+    *reinterpret_cast<uint4*>(Xg + (size_t)row * D + c) = *reinterpret_cast<const uint4*>(xr + c);
+    const float4 d0 = *reinterpret_cast<const float4*>(delta + t * D + c);
+    const float4 d1 = *reinterpret_cast<const float4*>(delta + t * D + c + 4);
+    const float4 g0 = *reinterpret_cast<const float4*>(g_delta + t * D + c);
+    const float4 g1 = *reinterpret_cast<const float4*>(g_delta + t * D + c + 4);
+    const float dl[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+    const float gd[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+    float gdt[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      gdt[i] = -gd[i] * expm1f(-dl[i]);
+      part = fmaf(gdt[i], to_f32(b_dt[(size_t)e * D + c + i]), part);
+    }
+    __nv_bfloat162 h[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(gdt[2 * i], gdt[2 * i + 1]);
+    *reinterpret_cast<uint4*>(G + (size_t)row * D + c) = *reinterpret_cast<const uint4*>(h);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  __shared__ float wsum[8];
+  if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5] = part;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s = 0.f;
+    for (int w = 0; w < 8; ++w) s += wsum[w];
+    bg[row] = s;
+  }
+}
+
+// One CTA (128 threads) per sorted row, after v = Xg W_x^e (XD, fp32 [R + 2N]) and q = G W_dt^eᵀ
+// (Q, fp32 [R]): dV[row] = bf16[g q | g ∂L/∂B | g ∂L/∂C]; DTs[row] = bf16[g dt_low | g | 0 x 7];
+// the pair's gate gradient dt_low·q + bg + B·∂L/∂B + C·∂L/∂C.
+__global__ void __launch_bounds__(128) proj_bwd_pair_kernel(const float* XD, const float* Q, const float* bg,
+                                                            const float* gB, const float* gC, const float* gates,
+                                                            const int* perm, int k, int R, int N, __nv_bfloat16* dV,
+                                                            __nv_bfloat16* DTs, float* dgates) {
+  const int row = blockIdx.x;
+  const int p = perm[row];
+  const int64_t t = p / k;
+  const float g = gates[p];
+  const int W = R + 2 * N;
+  const float* xd = XD + (size_t)row * W;
+  const float* q = Q + (size_t)row * R;
+  float part = 0.f;
+  for (int i = threadIdx.x; i < W; i += 128) {
+    float dv;
+    if (i < R) {
+      dv = g * q[i];
+      part = fmaf(xd[i], q[i], part);
+    } else if (i < R + N) {
+      const float gb = gB[t * N + i - R];
+      dv = g * gb;
+      part = fmaf(xd[i], gb, part);
+    } else {
+      const float gc = gC[t * N + i - R - N];
+      dv = g * gc;
+      part = fmaf(xd[i], gc, part);
+    }
+    dV[(size_t)row * W + i] = __float2bfloat16_rn(dv);
+  }
+  for (int i = threadIdx.x; i < R + 8; i += 128)
+    DTs[(size_t)row * (R + 8) + i] = __float2bfloat16_rn(i < R ? g * xd[i] : (i == R ? g : 0.f));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  __shared__ float wsum[4];
+  if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5] = part;
+  __syncthreads();
+  if (threadIdx.x == 0) dgates[p] = wsum[0] + wsum[1] + wsum[2] + wsum[3] + bg[row];
+}
+
+// [∂L/∂W_dt^e ; ∂L/∂b_dt^e] (TMP rows 0..R-1 and R of expert e) -> the caller's arrays.
+__global__ void proj_bwd_split_kernel(const float* TMP, int E, int R, int D, float* dW_dt, float* db) {
+  const int64_t n = (int64_t)E * (R + 1) * D;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t e = i / ((int64_t)(R + 1) * D), r = (i / D) % (R + 1), d = i % D;
+    const float v = TMP[(e * (R + 8) + r) * D + d];
+    if (r < R) dW_dt[(e * R + r) * D + d] = v;
+    else db[e * D + d] = v;
+  }
+}
+
+// ∂L/∂x[t] (+)= Σ_j DXP[inv[t k + j]] in slot order.
+__global__ void proj_bwd_dx_kernel(const float* DXP, const int* inv, int64_t T, int k, int D, float* dx,
+                                   int accumulate) {
+  const int64_t n4 = T * (D / 4);
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / (D / 4);
+    const int c = (int)(i % (D / 4)) * 4;
+    float4 acc = accumulate ? *reinterpret_cast<const float4*>(dx + t * D + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+      const float4 v = *reinterpret_cast<const float4*>(DXP + (size_t)inv[t * k + j] * D + c);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    *reinterpret_cast<float4*>(dx + t * D + c) = acc;
+  }
+}
+
+// Router: per token, ∂L/∂logits from the gate gradients (the sum of up to two contributions), then
+// ∂L/∂x[t] (+)= Σ_e ∂L/∂logit_e W_r[:, e]. One warp per token.
+template <typename IO>
+__global__ void route_bwd_dx_kernel(const IO* x, const float* W_r, const int32_t* idx, const float* gates,
+                                    const float* gg_a, const float* gg_b, int64_t T, int D, int E, int k,
+                                    float* dlogits, float* dx, int accumulate) {
+  const int64_t t = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  float dl[kMaxE];
+  float mean = 0.f;
+  for (int j = 0; j < k; ++j) {
+    const float gg = gg_a[t * k + j] + (gg_b ? gg_b[t * k + j] : 0.f);
+    mean = fmaf(gates[t * k + j], gg, mean);
+  }
+#pragma unroll
+  for (int e = 0; e < kMaxE; ++e) dl[e] = 0.f;
+  for (int j = 0; j < k; ++j) {
+    const float gg = gg_a[t * k + j] + (gg_b ? gg_b[t * k + j] : 0.f);
+    const int e = min(max(idx[t * k + j], 0), E - 1);
+    const float v = gates[t * k + j] * (gg - mean);
+#pragma unroll
+    for (int ee = 0; ee < kMaxE; ++ee)
+      if (ee == e) dl[ee] += v;
+  }
+  if (lane < E) {
+    float v = 0.f;
+#pragma unroll
+    for (int ee = 0; ee < kMaxE; ++ee)
+      if (ee == lane) v = dl[ee];
+    dlogits[t * E + lane] = v;
+  }
+  for (int d = lane; d < D; d += 32) {
+    float s = accumulate ? dx[t * D + d] : 0.f;
+    for (int e = 0; e < E; ++e) s = fmaf(dl[e < kMaxE ? e : 0], W_r[(size_t)d * E + e], s);
+    dx[t * D + d] = s;
+  }
+  (void)x;
+}
+
+// ∂L/∂W_r[d, e] = Σ_t x[t, d] ∂L/∂logits[t, e]: a CTA owns 32 channels and all experts, threads
+// split the tokens into 8 runs, summed in a fixed order.
+template <typename IO>
+__global__ void __launch_bounds__(256) route_bwd_dw_kernel(const IO* x, const float* dlogits, int64_t T, int D, int E,
+                                                           float* dW_r) {
+  __shared__ float red[8][32][kMaxE];
+  const int c = threadIdx.x & 31, run = threadIdx.x >> 5;
+  const int d = blockIdx.x * 32 + c;
+  float acc[kMaxE];
+#pragma unroll
+  for (int e = 0; e < kMaxE; ++e) acc[e] = 0.f;
+  const int64_t per = (T + 7) / 8;
+  const int64_t t0 = run * per, t1 = min(T, t0 + per);
+  if (d < D) {
+    for (int64_t t = t0; t < t1; ++t) {
+      const float xv = to_f32(x[t * D + d]);
+#pragma unroll
+      for (int e = 0; e < kMaxE; ++e)
+        if (e < E) acc[e] = fmaf(xv, dlogits[t * E + e], acc[e]);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < kMaxE; ++e) red[run][c][e] = acc[e];
+  __syncthreads();
+  if (run == 0 && d < D) {
+    for (int e = 0; e < E; ++e) {
+      float s = 0.f;
+      for (int r = 0; r < 8; ++r) s += red[r][c][e];
+      dW_r[(size_t)d * E + e] = s;
+    }
+  }
+}
+
+size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
+
+struct ProjBwdLayout {
+  size_t counts, offsets, perm, inv, bg, Xg, G, XD, Q, dV, DTs, DXP, TMP, total;
+};
+
+ProjBwdLayout proj_bwd_layout(int64_t T, int D, int R, int N, int E, int k) {
+  ProjBwdLayout l{};
+  const size_t P = (size_t)T * k, W = (size_t)R + 2 * N;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = up256(o + bytes);
+    return at;
+  };
+  l.counts = take(4 * (kMaxE + 1));
+  l.offsets = take(4 * (kMaxE + 1));
+  l.perm = take(4 * P);
+  l.inv = take(4 * P);
+  l.bg = take(4 * P);
+  l.Xg = take(2 * P * D);
+  l.G = take(2 * P * D);
+  l.XD = take(4 * P * W);
+  l.Q = take(4 * P * R);
+  l.dV = take(2 * P * W);
+  l.DTs = take(2 * P * (R + 8));
+  l.DXP = take(4 * P * D);
+  l.TMP = take(4 * (size_t)E * (R + 8) * D);
+  l.total = o;
+  return l;
+}
+
+}  // namespace
+
+size_t proj_bwd_workspace(int64_t T, int D, int R, int N, int E, int k) { return proj_bwd_layout(T, D, R, N, E, k).total; }
+
+cudaError_t run_proj_bwd(const void* x, const float* delta, const float* g_delta, const float* gB, const float* gC,
+                         const int32_t* idx, const float* gates, const void* W_x, const void* W_dt, const void* b_dt,
+                         bool b_bf16, float* dx, int accumulate, float* dgates, float* dW_x, float* dW_dt, float* db,
+                         int64_t T, int D, int R, int N, int E, int k, void* ws, void* status, cudaStream_t s) {
+  const ProjBwdLayout l = proj_bwd_layout(T, D, R, N, E, k);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int* counts = reinterpret_cast<int*>(w + l.counts);
+  int* offsets = reinterpret_cast<int*>(w + l.offsets);
+  int* perm = reinterpret_cast<int*>(w + l.perm);
+  int* inv = reinterpret_cast<int*>(w + l.inv);
+  float* bg = reinterpret_cast<float*>(w + l.bg);
+  __nv_bfloat16* Xg = reinterpret_cast<__nv_bfloat16*>(w + l.Xg);
+  __nv_bfloat16* G = reinterpret_cast<__nv_bfloat16*>(w + l.G);
+  float* XD = reinterpret_cast<float*>(w + l.XD);
+  float* Q = reinterpret_cast<float*>(w + l.Q);
+  __nv_bfloat16* dV = reinterpret_cast<__nv_bfloat16*>(w + l.dV);
+  __nv_bfloat16* DTs = reinterpret_cast<__nv_bfloat16*>(w + l.DTs);
+  float* DXP = reinterpret_cast<float*>(w + l.DXP);
+  float* TMP = reinterpret_cast<float*>(w + l.TMP);
+  const int64_t P = T * k;
+  const int W = R + 2 * N;
+  cudaError_t e;
+  const size_t sort_smem = sizeof(int) * (size_t)E * kSortThreads;
+  if ((e = cudaFuncSetAttribute(pair_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sort_smem)) !=
+      cudaSuccess)
+    return e;
+  pair_sort_kernel<<<1, kSortThreads, sort_smem, s>>>(idx, P, E, counts, offsets, perm, inv);
+  if (b_bf16)
+    proj_bwd_gather_kernel<__nv_bfloat16><<<(unsigned)P, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), delta, g_delta, idx, static_cast<const __nv_bfloat16*>(b_dt), perm, k,
+        D, E, Xg, G, bg);
+  else
+    proj_bwd_gather_kernel<float><<<(unsigned)P, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), delta, g_delta,
+                                                              idx, static_cast<const float*>(b_dt), perm, k, D, E, Xg,
+                                                              G, bg);
+  note_launch(2);
+  int h_off[kMaxE + 1];
+  if ((e = cudaMemcpyAsync(h_off, offsets, sizeof(int) * (E + 1), cudaMemcpyDeviceToHost, s)) != cudaSuccess) return e;
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return e;
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const __nv_bfloat16* Wx = static_cast<const __nv_bfloat16*>(W_x);
+  const __nv_bfloat16* Wdt = static_cast<const __nv_bfloat16*>(W_dt);
+  // v = Xg W_x^e and q = G W_dt^eᵀ per expert
+  for (int ex = 0; ex < E; ++ex) {
+    const int o = h_off[ex], n = h_off[ex + 1] - h_off[ex];
+    if (n == 0) continue;
+    if ((e = run_gemm_tc(false, false, true, n, W, D, Xg + (size_t)o * D, D, Wx + (size_t)ex * D * W, W,
+                         XD + (size_t)o * W, W, nullptr, 0, W, nullptr, 0, status, s)) != cudaSuccess)
+      return e;
+    if ((e = run_gemm_tc(false, true, true, n, R, D, G + (size_t)o * D, D, Wdt + (size_t)ex * R * D, D,
+                         Q + (size_t)o * R, R, nullptr, 0, R, nullptr, 0, status, s)) != cudaSuccess)
+      return e;
+  }
+  proj_bwd_pair_kernel<<<(unsigned)P, 128, 0, s>>>(XD, Q, bg, gB, gC, gates, perm, k, R, N, dV, DTs, dgates);
+  note_launch();
+  for (int ex = 0; ex < E; ++ex) {
+    const int o = h_off[ex], n = h_off[ex + 1] - h_off[ex];
+    if (n == 0) continue;
+    // the pairs' input gradients dV W_x^eᵀ (W_x^e stored [D, R + 2N] = [N, K] of this product)
+    if ((e = run_gemm_tc(false, true, true, n, D, W, dV + (size_t)o * W, W, Wx + (size_t)ex * D * W, W,
+                         DXP + (size_t)o * D, D, nullptr, 0, D, nullptr, 0, status, s)) != cudaSuccess)
+      return e;
+    // ∂L/∂W_x^e = Xgᵀ dV (Xg stored [pairs, D] = [K, M])
+    if ((e = run_gemm_tc(true, false, true, D, W, n, Xg + (size_t)o * D, D, dV + (size_t)o * W, W,
+                         dW_x + (size_t)ex * D * W, W, nullptr, 0, W, nullptr, 0, status, s)) != cudaSuccess)
+      return e;
+    // [∂L/∂W_dt^e ; ∂L/∂b_dt^e] = [g dt_low | g]ᵀ G
+    if ((e = run_gemm_tc(true, false, true, R + 8, D, n, DTs + (size_t)o * (R + 8), R + 8, G + (size_t)o * D, D,
+                         TMP + (size_t)ex * (R + 8) * D, D, nullptr, 0, D, nullptr, 0, status, s)) != cudaSuccess)
+      return e;
+  }
+  // experts without pairs have zero weight gradients
+  for (int ex = 0; ex < E; ++ex) {
+    if (h_off[ex + 1] != h_off[ex]) continue;
+    if ((e = cudaMemsetAsync(dW_x + (size_t)ex * D * W, 0, sizeof(float) * (size_t)D * W, s)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(TMP + (size_t)ex * (R + 8) * D, 0, sizeof(float) * (size_t)(R + 8) * D, s)) !=
+        cudaSuccess)
+      return e;
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  proj_bwd_split_kernel<<<(unsigned)(2 * sms), 256, 0, s>>>(TMP, E, R, D, dW_dt, db);
+  proj_bwd_dx_kernel<<<(unsigned)(8 * sms), 256, 0, s>>>(DXP, inv, T, k, D, dx, accumulate);
+  note_launch(2);
+  return cudaGetLastError();
+}
+
+cudaError_t run_route_bwd(const void* x, bool io_bf16, const float* W_r, const int32_t* idx, const float* gates,
+                          const float* gg_a, const float* gg_b, float* dlogits, float* dx, int accumulate, float* dW_r,
+                          int64_t T, int D, int E, int k, cudaStream_t s) {
+  const unsigned g1 = (unsigned)((T * 32 + 255) / 256), g2 = (unsigned)((D + 31) / 32);
+  if (io_bf16) {
+    route_bwd_dx_kernel<__nv_bfloat16><<<g1, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), W_r, idx, gates, gg_a,
+                                                          gg_b, T, D, E, k, dlogits, dx, accumulate);
+    route_bwd_dw_kernel<__nv_bfloat16><<<g2, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), dlogits, T, D, E, dW_r);
+  } else {
+    route_bwd_dx_kernel<float><<<g1, 256, 0, s>>>(static_cast<const float*>(x), W_r, idx, gates, gg_a, gg_b, T, D, E,
+                                                  k, dlogits, dx, accumulate);
+    route_bwd_dw_kernel<float><<<g2, 256, 0, s>>>(static_cast<const float*>(x), dlogits, T, D, E, dW_r);
+  }
+  note_launch(2);
+  return cudaGetLastError();
+}
+
+}  // namespace swimba

@@ -275,8 +275,8 @@ cudaError_t run_scan_chain(int64_t BDN, int P, const float* h_zero, const float*
 // sequence), then streams its sequences past them. Thread i owns (channel i / 4, state quarter
 // i % 4); it puts four sequences' state quarters, Δ, x, z, B/C quarters and experts in flight
 // before it computes any of them, and the four quarters of a channel reduce the readout with two
-// shuffles. Groups are sized so that the grid is about three CTAs per SM (the resident limit at
-// 85 registers a thread).
+// shuffles. The grid is one wave: tiles x groups <= the CTAs the SMs hold at once (three per SM at
+// 80 registers a thread), so no CTA waits for a second wave.
 constexpr int kStepCh = 64;  // channels per CTA
 constexpr int kStepU = 4;    // sequences in flight per thread
 
@@ -358,11 +358,14 @@ static cudaError_t launch_step_stream(const ScanParams& p, cudaStream_t s) {
   const size_t smem = sizeof(float4) * (size_t)p.E * kStepCh * 4;
   cudaError_t e = cudaFuncSetAttribute(step_stream_kernel<IO, K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
+  int dev = 0, sms = 148, per_sm = 1;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, step_stream_kernel<IO, K>, 256, smem)) != cudaSuccess)
+    return e;
+  // every CTA resident at once (one wave): the groups of a tile split the sequences evenly
   const int tiles = (p.D + kStepCh - 1) / kStepCh;
-  int groups = std::max(1, std::min(p.B, (3 * sms + tiles - 1) / tiles));
+  int groups = std::max(1, std::min(p.B, std::max(1, per_sm) * sms / tiles));
   const int spc = (p.B + groups - 1) / groups;
   groups = (p.B + spc - 1) / spc;
   step_stream_kernel<IO, K><<<(unsigned)(tiles * groups), 256, smem, s>>>(p, spc);

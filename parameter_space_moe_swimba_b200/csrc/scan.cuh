@@ -54,4 +54,39 @@ cudaError_t run_scan_chain(int64_t BDN, int P, const float* h_zero, const float*
 constexpr size_t kScanNoAllocScratchBytes = size_t(8) << 20;
 cudaError_t scan_noalloc_scratch(void** addr);
 
+// Backward pass of the scan (Euler injection): inputs as ScanParams plus the incoming gradient of
+// out; gradients in fp32. ckpt, part, part_A, part_D and nck are set by run_scan_bwd inside `ws`.
+struct ScanBwdParams {
+  const void* x;         // [B, L, D] io
+  const void* z;         // [B, L, D] io
+  const float* delta;    // [B, L, D]
+  const float* B_mix;    // [B, L, N]
+  const float* C_mix;    // [B, L, N]
+  const int32_t* idx;    // [B, L, k]
+  const float* gates;    // [B, L, k]
+  const float* A;        // [E, D, N]
+  const float* D_skip;   // [D]
+  const float* h0;       // [B, D, N] or null
+  const void* g_out;     // [B, L, D] io: dL/dout
+  float* dx;             // [B, L, D]
+  float* dz;             // [B, L, D]
+  float* ddelta;         // [B, L, D]
+  float* dB;             // [B, L, N]
+  float* dC;             // [B, L, N]
+  float* dgates;         // [B, L, k]
+  float* dA;             // [E, D, N]
+  float* dD;             // [D]
+  float* dh0;            // [B, D, N] or null
+  float* ckpt;           // [B, nck, D, N]: the state at the start of every 16-token chunk
+  float* part;           // [tiles, B, L, 2N + k]: per channel tile, dB | dC | dgates
+  float* part_A;         // [B, E, D, N]
+  float* part_D;         // [B, D]
+  int64_t L;
+  int B, D, N, E, k;
+  int nck;
+};
+
+size_t scan_bwd_workspace(int64_t B, int64_t L, int D, int N, int E, int k);
+cudaError_t run_scan_bwd(ScanBwdParams p, bool io_bf16, void* ws, cudaStream_t s);
+
 }  // namespace swimba

@@ -27,7 +27,7 @@ import torch  # noqa: E402  (after the library check so a missing build is repor
 SWIMBA_F32 = 0
 SWIMBA_BF16 = 1
 (SWIMBA_OP_ROUTE, SWIMBA_OP_PROJ, SWIMBA_OP_SCAN, SWIMBA_OP_STEP, SWIMBA_OP_LAYER, SWIMBA_OP_SUMMARY,
- SWIMBA_OP_SEPARATE) = range(7)
+ SWIMBA_OP_SEPARATE, SWIMBA_OP_SCAN_BWD, SWIMBA_OP_PROJ_BWD, SWIMBA_OP_ROUTE_BWD) = range(10)
 
 STATUS = {
     0: "SWIMBA_OK",
@@ -51,6 +51,9 @@ EXPORTED = [
     "swimba_scan_fwd_noalloc_status_block",
     "swimba_scan_summary",
     "swimba_scan_chain",
+    "swimba_scan_bwd",
+    "swimba_proj_bwd",
+    "swimba_route_bwd",
     "swimba_ssd_scan",
     "swimba_separate_proj",
     "swimba_separate_scan",
@@ -131,6 +134,14 @@ _lib.swimba_scan_summary.argtypes = [ctypes.POINTER(swimba_dims), _P, _P, _P, _P
 _lib.swimba_scan_summary.restype = ctypes.c_int
 _lib.swimba_scan_chain.argtypes = [ctypes.POINTER(swimba_dims), ctypes.c_int32, _P, _P, _P, _P, _P]
 _lib.swimba_scan_chain.restype = ctypes.c_int
+_lib.swimba_scan_bwd.argtypes = [ctypes.POINTER(swimba_dims)] + [_P] * 7 + [ctypes.POINTER(swimba_weights)] + \
+    [_P] * 11 + [_P, ctypes.c_size_t, _P]
+_lib.swimba_scan_bwd.restype = ctypes.c_int
+_lib.swimba_proj_bwd.argtypes = [ctypes.POINTER(swimba_dims), _P, _P, _P, ctypes.POINTER(swimba_weights)] + \
+    [_P] * 5 + [ctypes.c_int32] + [_P] * 5 + [ctypes.c_size_t, _P]
+_lib.swimba_proj_bwd.restype = ctypes.c_int
+_lib.swimba_route_bwd.argtypes = [ctypes.POINTER(swimba_dims)] + [_P] * 7 + [ctypes.c_int32, _P, _P, ctypes.c_size_t, _P]
+_lib.swimba_route_bwd.restype = ctypes.c_int
 _lib.swimba_ssd_scan.argtypes = [ctypes.POINTER(swimba_ssd_dims)] + [_P] * 10 + [_P, ctypes.c_size_t, _P]
 _lib.swimba_ssd_scan.restype = ctypes.c_int
 _lib.swimba_separate_proj.argtypes = [ctypes.POINTER(swimba_dims), _P, _P, _P, ctypes.POINTER(swimba_weights), _P,
@@ -265,6 +276,28 @@ def swimba_scan_summary(dims, x, delta, B_mix, idx, gates, weights, h_zero, log_
 def swimba_scan_chain(dims, parts, h_zero, log_decay, h0, h_start, stream=None) -> int:
     return _lib.swimba_scan_chain(ctypes.byref(dims), int(parts), _ptr(h_zero), _ptr(log_decay), _ptr(h0),
                                   _ptr(h_start), _stream(stream))
+
+
+def swimba_scan_bwd(dims, x, z, delta, B_mix, C_mix, idx, gates, weights, h0, g_out, dx, dz, ddelta, dB, dC, dgates,
+                    dA, dD, dh0, ws, ws_bytes, stream=None) -> int:
+    return _lib.swimba_scan_bwd(ctypes.byref(dims), _ptr(x), _ptr(z), _ptr(delta), _ptr(B_mix), _ptr(C_mix), _ptr(idx),
+                                _ptr(gates), ctypes.byref(weights), _ptr(h0), _ptr(g_out), _ptr(dx), _ptr(dz),
+                                _ptr(ddelta), _ptr(dB), _ptr(dC), _ptr(dgates), _ptr(dA), _ptr(dD), _ptr(dh0), _ptr(ws),
+                                int(ws_bytes), _stream(stream))
+
+
+def swimba_proj_bwd(dims, x, idx, gates, weights, delta, g_delta, g_B, g_C, dx, dx_accumulate, dgates, dW_x, dW_dt,
+                    db_dt, ws, ws_bytes, stream=None) -> int:
+    return _lib.swimba_proj_bwd(ctypes.byref(dims), _ptr(x), _ptr(idx), _ptr(gates), ctypes.byref(weights), _ptr(delta),
+                                _ptr(g_delta), _ptr(g_B), _ptr(g_C), _ptr(dx), int(dx_accumulate), _ptr(dgates),
+                                _ptr(dW_x), _ptr(dW_dt), _ptr(db_dt), _ptr(ws), int(ws_bytes), _stream(stream))
+
+
+def swimba_route_bwd(dims, x, W_r, idx, gates, g_gates_a, g_gates_b, dx, dx_accumulate, dW_r, ws, ws_bytes,
+                     stream=None) -> int:
+    return _lib.swimba_route_bwd(ctypes.byref(dims), _ptr(x), _ptr(W_r), _ptr(idx), _ptr(gates), _ptr(g_gates_a),
+                                 _ptr(g_gates_b), _ptr(dx), int(dx_accumulate), _ptr(dW_r), _ptr(ws), int(ws_bytes),
+                                 _stream(stream))
 
 
 def swimba_ssd_scan(dims, X, B_j, C_mix, gates, delta, A, D_skip, S0, y, S_final, ws, ws_bytes, stream=None) -> int:

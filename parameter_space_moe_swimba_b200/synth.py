@@ -49,6 +49,7 @@ STREAM_BLOCK_INPUT = 6
 STREAM_CONV_STATE = 7
 STREAM_BLOCK_REDRAW = 8
 STREAM_SSD = 9
+STREAM_OUT_GRAD = 10
 
 _BF16_MIN_NORMAL = 2.0 ** -126
 _BF16_MAX = float.fromhex("0x1.fep127")
@@ -168,6 +169,13 @@ def draw_step_activations(cfg: LayerConfig, step: int) -> tuple[np.ndarray, np.n
     x = round_to(g.standard_normal(shape), cfg.io_dtype)
     z = round_to(g.standard_normal(shape), cfg.io_dtype)
     return x, z
+
+
+def draw_out_grad(cfg: LayerConfig) -> np.ndarray:
+    """The incoming gradient dL/dout [B, L, D] ~ N(0, 1) in the io dtype's storage form (a
+    backward pass's input; the loss itself is not modelled)."""
+    g = rng(cfg.seed, STREAM_OUT_GRAD)
+    return round_to(g.standard_normal((cfg.batch, cfg.seqlen, cfg.d_inner)), cfg.io_dtype)
 
 
 def draw_h0(cfg: LayerConfig) -> np.ndarray:

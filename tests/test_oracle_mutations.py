@@ -208,3 +208,69 @@ def test_ssd_pins_catch_planted_mistake(name, monkeypatch):
             failed.append(exc)
             break
     assert failed, f"no pin fails with the planted mistake: {name}"
+
+
+# ---- the backward pass (oracle/swimba_backward_oracle.py) --------------------------------------
+
+from oracle import swimba_backward_oracle as BO  # noqa: E402
+import tests.test_oracle_backward_pins as BWP  # noqa: E402
+
+BWD_PINS = [
+    lambda: BWP.test_scan_backward_matches_finite_differences(0),
+    BWP.test_scan_backward_one_token_closed_form,
+    lambda: BWP.test_projection_backward_matches_finite_differences(0),
+    BWP.test_softplus_backward_matches_finite_differences,
+    BWP.test_route_backward_matches_finite_differences,
+]
+
+BWD_MUTATIONS = {
+    "adjoint not carried back": ("scan_backward", "carry = a_ts[t] * lam", "carry = 0.0 * lam"),
+    "adjoint carried without the decay": ("scan_backward", "carry = a_ts[t] * lam", "carry = lam"),
+    "readout gradient from the previous state": ("scan_backward", 'dC[:, t, :] = np.einsum("bd,bdn->bn", dy[:, t, :], hs[t])',
+                                                 'dC[:, t, :] = np.einsum("bd,bdn->bn", dy[:, t, :], h_prev[t])'),
+    "step gradient without the decay term": ("scan_backward", 'np.einsum("bdn,bdn->bd", lam, A_ts[t] * a_ts[t] * h_prev[t]) + \\\n',
+                                             '0.0 * np.einsum("bdn,bdn->bd", lam, A_ts[t] * a_ts[t] * h_prev[t]) + \\\n'),
+    "step gradient without the injection term": ("scan_backward", 'np.einsum("bdn,bn->bd", lam, B_mix[:, t, :]) * x[:, t, :]\n',
+                                                 '0.0 * x[:, t, :]\n'),
+    "gate gradient through the wrong table": ("scan_backward", "dg[b, t, j] += np.sum(dA_t[b] * A[e[b]])",
+                                              "dg[b, t, j] += np.sum(dA_t[b] * A[0])"),
+    "A gradient ungated": ("scan_backward", "dA[e[b]] += gates[b, t, j] * dA_t[b]", "dA[e[b]] += dA_t[b]"),
+    "SiLU derivative as sigmoid": ("silu_grad", "return s * (1.0 + np.asarray(z, dtype=np.float64) * (1.0 - s))",
+                                   "return s"),
+    "input gradient without the skip": ("scan_backward", "dx[:, t, :] = D_skip[None, :] * dy[:, t, :] + ",
+                                        "dx[:, t, :] = "),
+    "projection: bias gradient ungated": ("projection_backward", "d_dtj = gates[:, j, None] * g_dtmix",
+                                          "d_dtj = g_dtmix"),
+    "projection: W_dt gradient transposed use": ("projection_backward", "dv_e[:, :R] = d_dtj[rows] @ W_dt[e].T",
+                                                 "dv_e[:, :R] = d_dtj[rows] @ W_dt[(e + 1) % W_x.shape[0]].T"),
+    "projection: gate gradient without B": ("projection_backward", "np.sum(g_B * xdbl[:, j, R:R + N], axis=1)",
+                                            "0.0"),
+    "softplus derivative as exp": ("softplus_backward", "* sigmoid(dt_mix)", "* np.exp(dt_mix)"),
+    "router: softmax Jacobian without the mean": ("route_backward",
+                                                  "d_sel = gates * (g_gates - np.sum(gates * g_gates, axis=1, keepdims=True))",
+                                                  "d_sel = gates * g_gates"),
+}
+
+
+def _bwd_mutant(fn_name, old, new):
+    src = textwrap.dedent(inspect.getsource(getattr(BO, fn_name)))
+    assert old in src, f"mutation target not found in {fn_name}: {old!r}"
+    src = src.replace(old, new, 1)
+    ns = dict(vars(BO))
+    exec(compile(src, f"<mutant {fn_name}>", "exec"), ns)
+    return ns[fn_name]
+
+
+@pytest.mark.parametrize("name", sorted(BWD_MUTATIONS))
+def test_backward_pins_catch_planted_mistake(name, monkeypatch):
+    fn_name, old, new = BWD_MUTATIONS[name]
+    mutant = _bwd_mutant(fn_name, old, new)
+    monkeypatch.setattr(BO, fn_name, mutant)
+    failed = []
+    for pin in BWD_PINS:
+        try:
+            pin()
+        except Exception as exc:
+            failed.append(exc)
+            break
+    assert failed, f"no pin fails with the planted mistake: {name}"
