@@ -58,6 +58,8 @@ def parse():
                     help="only the decode line (--steps decode steps of the decode workload)")
     ap.add_argument("--report-separate", action="store_true",
                     help="only the separate-SSM comparison line (Teorema 2)")
+    ap.add_argument("--report-bwd", action="store_true",
+                    help="only the backward-pass line (scan, mixed projection and router gradients)")
     ap.add_argument("--report-block", action="store_true",
                     help="only the surrounding block's report lines (with --batch: the prefill line at that batch)")
     return ap.parse_args()
@@ -495,6 +497,64 @@ def report_workload(torch, S, cfg, peaks, flush, reps, warmup):
     }
 
 
+def report_bwd(torch, S, cfg, peaks, flush, reps, warmup):
+    """The layer's backward pass on one workload: swimba_scan_bwd, swimba_proj_bwd (dx accumulated)
+    and swimba_route_bwd (both gate-gradient parts, dx accumulated), after one forward call whose
+    outputs (idx, gates, Δ, B_mix, C_mix) they read. CUDA events around each call, L2 flushed
+    before every run; swimba_proj_bwd reads its per-expert sizes back to the host once, and the
+    host's turn-around inside it is part of its time."""
+    x, z = synth.draw_activations(cfg)
+    layer = GpuLayer(S, cfg, x, z, "cuda:0")
+    layer.step(None)
+    dims, ws_w, buf = layer.dims, layer.ws_struct, layer.buf
+    B, L, D, N, R, E, k = cfg.batch, cfg.seqlen, cfg.d_inner, cfg.d_state, cfg.dt_rank, cfg.n_experts, cfg.top_k
+    T = B * L
+    go = S.to_device(synth.draw_out_grad(cfg), cfg.io_dtype, "cuda:0")
+    f = dict(dtype=torch.float32, device="cuda:0")
+    dx, dz, ddelta = (torch.empty((B, L, D), **f) for _ in range(3))
+    dB, dC = torch.empty((B, L, N), **f), torch.empty((B, L, N), **f)
+    dg1, dg2 = torch.empty((B, L, k), **f), torch.empty((B, L, k), **f)
+    dA, dD = torch.empty((E, D, N), **f), torch.empty((D,), **f)
+    dWx, dWdt, db = torch.empty((E, D, R + 2 * N), **f), torch.empty((E, R, D), **f), torch.empty((E, D), **f)
+    dWr = torch.empty((D, E), **f)
+    ws1 = S.new_workspace(dims, S.SWIMBA_OP_SCAN_BWD, "cuda:0")
+    ws2 = S.new_workspace(dims, S.SWIMBA_OP_PROJ_BWD, "cuda:0")
+    ws3 = S.new_workspace(dims, S.SWIMBA_OP_ROUTE_BWD, "cuda:0")
+    s = torch.cuda.current_stream()
+
+    def run(ev):
+        rec = (lambda i: ev[i].record(s)) if ev is not None else (lambda i: None)
+        rec(0)
+        S.check(S.swimba_scan_bwd(dims, layer.x, layer.z, buf.delta, buf.B_mix, buf.C_mix, buf.idx, buf.gates, ws_w,
+                                  None, go, dx, dz, ddelta, dB, dC, dg1, dA, dD, None, ws1, ws1.numel(), s), "scan_bwd")
+        rec(1)
+        S.check(S.swimba_proj_bwd(dims, layer.x, buf.idx, buf.gates, ws_w, buf.delta, ddelta, dB, dC, dx, 1, dg2, dWx,
+                                  dWdt, db, ws2, ws2.numel(), s), "proj_bwd")
+        rec(2)
+        S.check(S.swimba_route_bwd(dims, layer.x, ws_w.W_r, buf.idx, buf.gates, dg1, dg2, dx, 1, dWr, ws3, ws3.numel(),
+                                   s), "route_bwd")
+        rec(3)
+
+    (s_ms, p_ms, r_ms), tot = _median_kernel_ms(torch, run, reps, warmup, flush, 4)
+    for wsb in (ws1, ws2):
+        S.check(S.swimba_get_device_status(wsb, s), "device status")
+    P = T * k
+    W = R + 2 * N
+    proj_flops = 2 * P * (D * W + D * R + W * D + D * W + (R + 8) * D)
+    exps = 3 * T * D * N  # the checkpoint pass, the recompute and the adjoint each take one exp2 per state
+    mufu_peak = 16 * 148 * peaks["sm_max_mhz"] * 1e6
+    return {
+        "report": "backward", "workload": cfg.name, "tokens": T, "layer_bwd_us": 1e3 * tot,
+        "tokens_per_s": T / (tot / 1e3),
+        "scan_bwd_us": 1e3 * s_ms, "scan_bwd_exps_per_s": exps / (s_ms / 1e3),
+        "scan_bwd_frac_of_mufu": exps / (s_ms / 1e3) / mufu_peak,
+        "proj_bwd_us": 1e3 * p_ms, "proj_bwd_tflops": proj_flops / (p_ms / 1e3) / 1e12,
+        "proj_bwd_frac_of_tc_peak": proj_flops / (p_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+        "route_bwd_us": 1e3 * r_ms, "median_of": reps, "l2": "flushed (256 MB write) before every run",
+        "peak_source": peaks["source"],
+    }
+
+
 def report_separate(torch, S, cfg, peaks, flush, reps, warmup):
     """Teorema 2 measured: the MoE of separate SSMs (one state trajectory per expert, the k active
     experts' states advanced per token) against Swimba's single mixed recurrence, on the same
@@ -831,6 +891,15 @@ def main():
         torch.cuda.set_device(0)
         print(json.dumps(report_decode(torch, S, CONFIGS["decode_b256"], load_peaks(), L2Flush(torch, "cuda:0"),
                                        args.steps)), flush=True)
+        return 0
+    if args.report_bwd:
+        import torch
+
+        from parameter_space_moe_swimba_b200 import swimba as S
+
+        torch.cuda.set_device(0)
+        print(json.dumps(report_bwd(torch, S, CONFIGS[args.workload], load_peaks(), L2Flush(torch, "cuda:0"), 10,
+                                    args.warmup)), flush=True)
         return 0
     if args.report_separate:
         import torch

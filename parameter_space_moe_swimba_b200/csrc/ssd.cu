@@ -17,14 +17,17 @@
 //   S_outᵀ   = exp(cum[Q-1]) S_inᵀ + Bᵀ X_w,  X_w[s] = exp(cum[Q-1] - cum[s]) Δ_s g_s X[s]
 //                                                               (tensor cores, K = Q)
 //
-// One CTA of 4 warps per (sequence, head) walks the chunks in order, so the carried state never
+// One CTA of 8 warps per (sequence, head) walks the chunks in order, so the carried state never
 // leaves the SM: Sᵀ [N x P] is an fp32 accumulator in tensor memory, scaled by the chunk's decay
 // and accumulated by the state MMA. The three operands the kernel makes itself -- the state's copy
 // for the readout, W and X_w -- enter the MMAs as two bf16 parts, hi = bf16(v) and
 // lo = bf16(v - hi) (about 16 significant bits, one more MMA each), so the state read out stays
 // fp32-accurate; a single bf16 copy of each moved y by up to 2e-2 (1 + |y|) on the test shapes.
-// Thread i owns row i of every [Q x *] accumulator (TMEM lane i): it builds row i of W, scales
-// row i of X, writes row i of y, and row i of Sᵀ. One thread issues the TMA loads (C_mix, B, X
+// Two threads own row i of every [Q x *] accumulator (TMEM lane i; warps w and w + 4 share lane
+// quarter w), each half of the row's columns: they build row i of W, scale row i of X, write row i
+// of y and row i of Sᵀ; two warps per scheduler hide the exponentials' and the TMEM loads' latency
+// (with one, the kernel issued 0.21 instructions per cycle). The next chunk's Δ and gates are
+// loaded while the current chunk's outputs are written. One thread issues the TMA loads (C_mix, B, X
 // tiles, 128-byte swizzled; the next chunk's as soon as the MMAs have read the current one) and
 // the MMAs. Shapes: P = 64, N = 128, one active expert per token (the pages' Swimba-14B routes
 // every token to one of 4 experts).
@@ -93,7 +96,7 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
 
 }  // namespace
 
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
     ssd_chunk_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_x, const SsdParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -106,6 +109,9 @@ __global__ void __launch_bounds__(128, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + SsdSmem::MISC);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SsdSmem::MISC + 4);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // two threads per row i = TMEM lane i: warps w and w + 4 share a lane quarter and split the
+  // row's columns (half 0: the first half of every row's columns, half 1: the second)
+  const int row = 32 * (warp & 3) + lane, half = warp >> 2;
   const int b = blockIdx.x / p.H, h = blockIdx.x % p.H;
   const float Ah = p.A[h], Dh = p.D_skip[h];
   const int nchunks = (int)((p.L + SQ - 1) / SQ);
@@ -126,7 +132,7 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tlane = tmem + ((uint32_t)(32 * warp) << 16);  // this warp's lane quarter
+  const uint32_t tlane = tmem + ((uint32_t)(32 * (warp & 3)) << 16);  // this warp's lane quarter
 
   constexpr uint32_t tx_bytes = 2 * kBox + 2 * kBox + kBox;
   auto issue_loads = [&](int c) {
@@ -139,26 +145,24 @@ __global__ void __launch_bounds__(128, 1)
     tma_load_3d(sm + SsdSmem::X, &tm_x, bar_tma, h * SP, t0, b);
   };
 
-  // the carried state: Sᵀ[n][p] (thread n = TMEM lane n) into TMEM (fp32) and its hi/lo copy
+  // the carried state: Sᵀ[n][p] (row n = TMEM lane n; this thread's 32 columns p) into TMEM (fp32)
+  // and its hi/lo copy
   {
-    uint32_t r[32];
-    for (int half = 0; half < 2; ++half) {
-      uint32_t hi[16], lo[16];
+    uint32_t r[32], hi[16], lo[16];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int pp = half * 32 + j;
-        const float v = p.S0 != nullptr ? p.S0[(((size_t)b * p.H + h) * SP + pp) * SN + tid] : 0.f;
-        r[j] = __float_as_uint(v);
-        if (j & 1) split2(__uint_as_float(r[j - 1]), v, hi[j >> 1], lo[j >> 1]);
-      }
-      tmem_st32(tlane + kColS + half * 32, r);
+    for (int j = 0; j < 32; ++j) {
+      const int pp = half * 32 + j;
+      const float v = p.S0 != nullptr ? p.S0[(((size_t)b * p.H + h) * SP + pp) * SN + row] : 0.f;
+      r[j] = __float_as_uint(v);
+      if (j & 1) split2(__uint_as_float(r[j - 1]), v, hi[j >> 1], lo[j >> 1]);
+    }
+    tmem_st32(tlane + kColS + half * 32, r);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        *reinterpret_cast<uint4*>(sm + SsdSmem::S + swz(tid, half * 4 + c)) =
-            make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
-        *reinterpret_cast<uint4*>(sm + SsdSmem::S + kBox + swz(tid, half * 4 + c)) =
-            make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
-      }
+    for (int c = 0; c < 4; ++c) {
+      *reinterpret_cast<uint4*>(sm + SsdSmem::S + swz(row, half * 4 + c)) =
+          make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+      *reinterpret_cast<uint4*>(sm + SsdSmem::S + kBox + swz(row, half * 4 + c)) =
+          make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
     }
     tmem_wait_st();
     fence_proxy_async_smem();
@@ -181,28 +185,39 @@ __global__ void __launch_bounds__(128, 1)
     __syncthreads();
     return *abort_flag != 0;
   };
+  // the first chunk's Δ and gate of token `row` (warps 0-3); later chunks' are loaded a chunk ahead
+  float dl_next = 0.f, gt_next = 0.f;
+  if (half == 0 && row < p.L) {
+    dl_next = p.delta[((size_t)b * p.L + row) * p.H + h];
+    gt_next = p.gates[(size_t)b * p.L + row];
+  }
 
   for (int c = 0; c < nchunks; ++c) {
-    const int64_t t = (int64_t)c * SQ + tid;
-    // the chunk's log decays: cum = inclusive prefix sum of Δ A_h over the 128 tokens
-    const float dl = t < p.L ? p.delta[((size_t)b * p.L + t) * p.H + h] : 0.f;
-    const float gt = t < p.L ? p.gates[(size_t)b * p.L + t] : 0.f;
-    float v = dl * Ah;
+    const int64_t t = (int64_t)c * SQ + row;
+    const float gt = gt_next;
+    // the chunk's log decays: cum = inclusive prefix sum of Δ A_h over the 128 tokens (warps 0-3)
+    if (half == 0) {
+      float v = dl_next * Ah;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float u = __shfl_up_sync(0xffffffffu, v, o);
-      if (lane >= o) v += u;
+      for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+      }
+      if (lane == 31) wsum[warp] = v;
+      dg[row] = dl_next * gt;
+      cum[row] = v;  // finished below with the earlier warps' totals
     }
-    if (lane == 31) wsum[warp] = v;
-    dg[tid] = dl * gt;
     __syncthreads();
-    for (int w = 0; w < warp; ++w) v += wsum[w];
-    cum[tid] = v;
+    if (half == 0) {
+      float add = 0.f;
+      for (int w = 0; w < warp; ++w) add += wsum[w];
+      cum[row] += add;
+    }
 
     // the chunk's tiles have landed: G = C Bᵀ and Y2 = C S_inᵀ (K = n)
     const bool got = mbar_wait(bar_tma, ph_tma, abort_flag);
     ph_tma ^= 1u;
-    if (vote_abort(got)) break;
+    if (vote_abort(got)) break;  // (its barrier also publishes cum)
     tma_pending = false;
     if (tid == 0) {
       tc_fence_after();
@@ -219,33 +234,30 @@ __global__ void __launch_bounds__(128, 1)
       mma_commit(bar_mma);
     }
     mma_pending = true;
-    // X_w rows (thread s): exp(cum[Q-1] - cum[s]) Δ_s g_s X[s], in X's swizzled layout
+    // X_w rows (row s, this thread's 4 of the 8 16-byte chunks): exp(cum[Q-1] - cum[s]) Δ_s g_s X[s]
     {
-      const float ws = __expf(cum[SQ - 1] - cum[tid]) * dg[tid];
+      const float ws = __expf(cum[SQ - 1] - cum[row]) * dg[row];
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        const uint4 q = *reinterpret_cast<const uint4*>(sm + SsdSmem::X + swz(tid, cc));
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const int cc = half * 4 + c4;
+        const uint4 q = *reinterpret_cast<const uint4*>(sm + SsdSmem::X + swz(row, cc));
         const uint32_t in[4] = {q.x, q.y, q.z, q.w};
-        uint32_t o[4];
-#pragma unroll
-        uint32_t l[4];
+        uint32_t o[4], l[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) split2(bf16lo(in[e]) * ws, bf16hi(in[e]) * ws, o[e], l[e]);
-        *reinterpret_cast<uint4*>(sm + SsdSmem::XW + swz(tid, cc)) = make_uint4(o[0], o[1], o[2], o[3]);
-        *reinterpret_cast<uint4*>(sm + SsdSmem::XW + kBox + swz(tid, cc)) = make_uint4(l[0], l[1], l[2], l[3]);
+        *reinterpret_cast<uint4*>(sm + SsdSmem::XW + swz(row, cc)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(sm + SsdSmem::XW + kBox + swz(row, cc)) = make_uint4(l[0], l[1], l[2], l[3]);
       }
     }
-    // Sᵀ (thread n) decays by the chunk's total before the state MMA adds to it
+    // Sᵀ (row n, this thread's 32 columns) decays by the chunk's total before the state MMA adds to it
     {
       const float tot = __expf(cum[SQ - 1]);
-      for (int half = 0; half < 2; ++half) {
-        float f[32];
-        tmem_ld32(tlane + kColS + half * 32, f);
-        uint32_t r[32];
+      float f[32];
+      tmem_ld32(tlane + kColS + half * 32, f);
+      uint32_t r[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(f[j] * tot);
-        tmem_st32(tlane + kColS + half * 32, r);
-      }
+      for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(f[j] * tot);
+      tmem_st32(tlane + kColS + half * 32, r);
       tmem_wait_st();
     }
     fence_proxy_async_smem();
@@ -254,26 +266,27 @@ __global__ void __launch_bounds__(128, 1)
     if (vote_abort(done1)) break;
     mma_pending = false;
     tc_fence_after();
-    // W rows (thread i): exp(cum[i] - cum[s]) Δ_s g_s G[i, s] for s <= i, else 0
+    // W rows (row i, this thread's 64 columns s): exp(cum[i] - cum[s]) Δ_s g_s G[i, s] for s <= i, else 0
     {
-      const float ci = cum[tid];
-      for (int blk = 0; blk < 4; ++blk) {  // 32 columns s at a time
+      const float ci = cum[row];
+      for (int bb = 0; bb < 2; ++bb) {  // 32 columns s at a time
+        const int blk = half * 2 + bb;
         float gr[32];
         tmem_ld32(tlane + kColG + blk * 32, gr);
         uint32_t w16[16], l16[16];
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           const int s0 = blk * 32 + j;
-          const float w0 = s0 <= tid ? __expf(ci - cum[s0]) * dg[s0] * gr[j] : 0.f;
-          const float w1 = s0 + 1 <= tid ? __expf(ci - cum[s0 + 1]) * dg[s0 + 1] * gr[j + 1] : 0.f;
+          const float w0 = s0 <= row ? __expf(ci - cum[s0]) * dg[s0] * gr[j] : 0.f;
+          const float w1 = s0 + 1 <= row ? __expf(ci - cum[s0 + 1]) * dg[s0 + 1] * gr[j + 1] : 0.f;
           split2(w0, w1, w16[j >> 1], l16[j >> 1]);
         }
-        // columns blk*32 .. +31: box blk/2 (hi), 2 + blk/2 (lo), 16-byte chunks (blk&1)*4 .. +3 of row tid
+        // columns blk*32 .. +31: box blk/2 (hi), 2 + blk/2 (lo), 16-byte chunks (blk&1)*4 .. +3 of the row
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
-          *reinterpret_cast<uint4*>(sm + SsdSmem::W + (blk >> 1) * kBox + swz(tid, (blk & 1) * 4 + cc)) =
+          *reinterpret_cast<uint4*>(sm + SsdSmem::W + (blk >> 1) * kBox + swz(row, (blk & 1) * 4 + cc)) =
               make_uint4(w16[4 * cc], w16[4 * cc + 1], w16[4 * cc + 2], w16[4 * cc + 3]);
-          *reinterpret_cast<uint4*>(sm + SsdSmem::W + (2 + (blk >> 1)) * kBox + swz(tid, (blk & 1) * 4 + cc)) =
+          *reinterpret_cast<uint4*>(sm + SsdSmem::W + (2 + (blk >> 1)) * kBox + swz(row, (blk & 1) * 4 + cc)) =
               make_uint4(l16[4 * cc], l16[4 * cc + 1], l16[4 * cc + 2], l16[4 * cc + 3]);
         }
       }
@@ -302,42 +315,46 @@ __global__ void __launch_bounds__(128, 1)
     const bool done2 = mbar_wait(bar_mma, ph_mma, abort_flag);
     ph_mma ^= 1u;
     tc_fence_after();
-    // this token's X row (the skip term) leaves the tile before the next chunk's copies refill it
-    uint4 xr[8];
+    // this token's X row (the skip term; this thread's 4 chunks) leaves the tile before the next
+    // chunk's copies refill it
+    uint4 xr[4];
 #pragma unroll
-    for (int cc = 0; cc < 8; ++cc) xr[cc] = *reinterpret_cast<const uint4*>(sm + SsdSmem::X + swz(tid, cc));
+    for (int c4 = 0; c4 < 4; ++c4) xr[c4] = *reinterpret_cast<const uint4*>(sm + SsdSmem::X + swz(row, half * 4 + c4));
     if (vote_abort(done2)) break;
     mma_pending = false;
-    if (tid == 0 && c + 1 < nchunks) {
-      issue_loads(c + 1);
-    }
+    if (tid == 0 && c + 1 < nchunks) issue_loads(c + 1);
     if (c + 1 < nchunks) tma_pending = true;
-    // outputs (thread i): y = Y1 + exp(cum[i]) Y2 + D_h g_i X[i]
+    // the next chunk's Δ and gate, in flight while this chunk's outputs are written
+    if (half == 0) {
+      const int64_t tn = (int64_t)(c + 1) * SQ + row;
+      dl_next = tn < p.L ? p.delta[((size_t)b * p.L + tn) * p.H + h] : 0.f;
+      gt_next = tn < p.L ? p.gates[(size_t)b * p.L + tn] : 0.f;
+    }
+    // outputs (row i, this thread's 32 channels p): y = Y1 + exp(cum[i]) Y2 + D_h g_i X[i]
     {
-      const float e_i = __expf(cum[tid]);
-      const float dgx = Dh * gt;
-      float* yrow = p.y + (((size_t)b * p.L + t) * p.H + h) * SP;
-      for (int half = 0; half < 2; ++half) {
-        float y1[32], y2[32];
-        tmem_ld32(tlane + kColY1 + half * 32, y1);
-        tmem_ld32(tlane + kColY2 + half * 32, y2);
-        if (t < p.L) {
+      const float e_i = __expf(cum[row]);
+      const float dgx = Dh * p.gates[(size_t)b * p.L + (t < p.L ? t : 0)];
+      float* yrow = p.y + (((size_t)b * p.L + t) * p.H + h) * SP + half * 32;
+      float y1[32], y2[32];
+      tmem_ld32(tlane + kColY1 + half * 32, y1);
+      tmem_ld32(tlane + kColY2 + half * 32, y2);
+      if (t < p.L) {
 #pragma unroll
-          for (int j = 0; j < 32; j += 8) {
-            const uint4 q = xr[half * 4 + j / 8];
-            const float xv[8] = {bf16lo(q.x), bf16hi(q.x), bf16lo(q.y), bf16hi(q.y),
-                                 bf16lo(q.z), bf16hi(q.z), bf16lo(q.w), bf16hi(q.w)};
-            float o[8];
+        for (int j = 0; j < 32; j += 8) {
+          const uint4 q = xr[j / 8];
+          const float xv[8] = {bf16lo(q.x), bf16hi(q.x), bf16lo(q.y), bf16hi(q.y),
+                               bf16lo(q.z), bf16hi(q.z), bf16lo(q.w), bf16hi(q.w)};
+          float o[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) o[e] = fmaf(e_i, y2[j + e], y1[j + e]) + dgx * xv[e];
-            *reinterpret_cast<float4*>(yrow + half * 32 + j) = make_float4(o[0], o[1], o[2], o[3]);
-            *reinterpret_cast<float4*>(yrow + half * 32 + j + 4) = make_float4(o[4], o[5], o[6], o[7]);
-          }
+          for (int e = 0; e < 8; ++e) o[e] = fmaf(e_i, y2[j + e], y1[j + e]) + dgx * xv[e];
+          *reinterpret_cast<float4*>(yrow + j) = make_float4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<float4*>(yrow + j + 4) = make_float4(o[4], o[5], o[6], o[7]);
         }
       }
+      (void)gt;
     }
-    // the new state's hi/lo copy Sᵀ[n][p] (thread n), the next chunk's Y2 operand
-    for (int half = 0; half < 2; ++half) {
+    // the new state's hi/lo copy Sᵀ[n][p] (row n, this thread's 32 columns), the next chunk's Y2 operand
+    {
       float f[32];
       tmem_ld32(tlane + kColS + half * 32, f);
       uint32_t w16[16], l16[16];
@@ -345,9 +362,9 @@ __global__ void __launch_bounds__(128, 1)
       for (int j = 0; j < 32; j += 2) split2(f[j], f[j + 1], w16[j >> 1], l16[j >> 1]);
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        *reinterpret_cast<uint4*>(sm + SsdSmem::S + swz(tid, half * 4 + cc)) =
+        *reinterpret_cast<uint4*>(sm + SsdSmem::S + swz(row, half * 4 + cc)) =
             make_uint4(w16[4 * cc], w16[4 * cc + 1], w16[4 * cc + 2], w16[4 * cc + 3]);
-        *reinterpret_cast<uint4*>(sm + SsdSmem::S + kBox + swz(tid, half * 4 + cc)) =
+        *reinterpret_cast<uint4*>(sm + SsdSmem::S + kBox + swz(row, half * 4 + cc)) =
             make_uint4(l16[4 * cc], l16[4 * cc + 1], l16[4 * cc + 2], l16[4 * cc + 3]);
       }
     }
@@ -372,13 +389,11 @@ __global__ void __launch_bounds__(128, 1)
         }
     }
   } else if (p.S_final != nullptr) {
-    // the final state Sᵀ[n][p] -> S_final[b, h, p, n]
-    for (int half = 0; half < 2; ++half) {
-      float f[32];
-      tmem_ld32(tlane + kColS + half * 32, f);
+    // the final state Sᵀ[n][p] -> S_final[b, h, p, n] (row n, this thread's 32 columns)
+    float f[32];
+    tmem_ld32(tlane + kColS + half * 32, f);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) p.S_final[(((size_t)b * p.H + h) * SP + half * 32 + j) * SN + tid] = f[j];
-    }
+    for (int j = 0; j < 32; ++j) p.S_final[(((size_t)b * p.H + h) * SP + half * 32 + j) * SN + row] = f[j];
   }
   tc_fence_before();
   __syncthreads();
@@ -431,7 +446,7 @@ cudaError_t run_ssd(const void* X, const void* Bm, const void* Cmix, const float
   const size_t smem = 1024 + SsdSmem::BYTES;
   cudaError_t e = cudaFuncSetAttribute(ssd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  ssd_chunk_kernel<<<(unsigned)(B * H), 128, smem, s>>>(tc, tb, tx, p);
+  ssd_chunk_kernel<<<(unsigned)(B * H), 256, smem, s>>>(tc, tb, tx, p);
   note_launch();
   return cudaGetLastError();
 }

@@ -5,11 +5,15 @@ pinned by finite differences of the forward oracle).
 
 Tolerance, from the arithmetic: the projection's products run on the tensor cores with bf16
 operands (x exactly; dL/d(dt_mix), g_j q_j, g_j dL/dB, g_j dL/dC and g_j dt_low rounded once, each
-to 2^-9 relative) and fp32 accumulation, so every product term carries at most about 2^-8 relative
-error and a sum of n terms of random sign an error near 2^-8 sqrt(n) |term| against a scale near
-sqrt(n) |term|: 4e-3 of the field's scale, and the worst element of a field a few times that. The
-fields are held to 2e-2 of their scale (max |err| / (rms + |ref|)), the layer's bf16 bound. The
-router's backward is fp32 SIMT on stored inputs: 1e-4."""
+by at most 2^-9 relative) and fp32 accumulation: mixed-precision gradients as training uses them.
+A product of two rounded operands carries up to 2^-8 relative error per term; in a sum whose terms
+cancel, the worst element of a field lands at several times that against the field's scale
+(measured up to 2.2e-2 for ∂L/∂W_dt, whose both operands are rounded). The fields are held to
+5e-2 of their scale (max |err| / (rms + |ref|)) against the exact oracle, AND the weight
+gradients are checked at 2e-3 against the same products formed in the test from the oracle's
+intermediates with the operands rounded to bf16 where the kernel rounds them -- which pins that
+the gap to the exact oracle is that rounding and nothing else. The router's backward is fp32 SIMT
+on stored inputs: 1e-4."""
 from __future__ import annotations
 
 import numpy as np
@@ -25,7 +29,8 @@ pytestmark = pytest.mark.gpu
 
 torch = pytest.importorskip("torch")
 
-TOL_BF16_GRAD = 2e-2
+TOL_BF16_GRAD = 5e-2
+TOL_ROUNDED = 2e-3
 
 
 @pytest.fixture(scope="module")
@@ -100,9 +105,26 @@ def test_proj_and_route_backward_match_the_oracle(S, shape):
     torch.cuda.synchronize()
     errs["route_dx"] = rel_rms_err(rdx.cpu().numpy(), rref["dx"])
     errs["dW_r"] = rel_rms_err(dWr.cpu().numpy(), rref["dW_r"])
+    # the weight gradients from operands rounded where the kernel rounds them (bf16, nearest even)
+    bf = lambda a: synth.widen(synth.round_to(a, "bf16"), "bf16")
+    pr = O.expert_projections(x64, idx, gates, W["W_x"], W["W_dt"], W["b_dt"], R, N)
+    G = bf(g_dtmix)
+    emu_dWdt = np.zeros((E, R, D))
+    emu_db = np.zeros((E, D))
+    for j in range(k):
+        g = gates[:, j].astype(np.float64)
+        dts = bf(g[:, None] * pr["xdbl"][:, j, :R])
+        gb = bf(g)
+        for e in range(E):
+            rows = np.nonzero(idx[:, j] == e)[0]
+            emu_dWdt[e] += dts[rows].T @ G[rows]
+            emu_db[e] += gb[rows] @ G[rows]
+    errs["dW_dt_rounded"] = rel_rms_err(dWdt.cpu().numpy(), emu_dWdt)
+    errs["db_dt_rounded"] = rel_rms_err(db.cpu().numpy(), emu_db)
     print(shape, {kk: f"{v:.2e}" for kk, v in errs.items()})
     for name in ("dx", "dgates", "dW_x", "dW_dt", "db_dt"):
         assert errs[name] <= TOL_BF16_GRAD, (name, errs[name])
+    assert errs["dW_dt_rounded"] <= TOL_ROUNDED and errs["db_dt_rounded"] <= TOL_ROUNDED
     assert errs["route_dx"] <= 1e-4 and errs["dW_r"] <= 1e-4
 
 
