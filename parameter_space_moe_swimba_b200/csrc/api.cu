@@ -28,8 +28,9 @@ cudaError_t run_proj_bwd(const void* x, const float* delta, const float* g_delta
                          const int32_t* idx, const float* gates, const void* W_x, const void* W_dt, const void* b_dt,
                          bool b_bf16, float* dx, int accumulate, float* dgates, float* dW_x, float* dW_dt, float* db,
                          int64_t T, int D, int R, int N, int E, int k, void* ws, void* status, cudaStream_t s);
+size_t route_bwd_workspace(int64_t T, int D, int E);
 cudaError_t run_route_bwd(const void* x, bool io_bf16, const float* W_r, const int32_t* idx, const float* gates,
-                          const float* gg_a, const float* gg_b, float* dlogits, float* dx, int accumulate, float* dW_r,
+                          const float* gg_a, const float* gg_b, void* ws, float* dx, int accumulate, float* dW_r,
                           int64_t T, int D, int E, int k, cudaStream_t s);
 bool ssd_supported(int P, int N, int k);
 cudaError_t run_ssd(const void* X, const void* Bm, const void* Cmix, const float* gates, const float* delta,
@@ -157,7 +158,7 @@ size_t swimba_workspace_size(const swimba_dims* dims, int op) {
       return kStatusBytes + proj_bwd_workspace(dims->batch * dims->seqlen, dims->d_inner, dims->dt_rank,
                                                dims->d_state, dims->n_experts, dims->top_k);
     case SWIMBA_OP_ROUTE_BWD:
-      return kStatusBytes + (size_t)dims->batch * dims->seqlen * dims->n_experts * 4;
+      return kStatusBytes + route_bwd_workspace(dims->batch * dims->seqlen, dims->d_inner, dims->n_experts);
     case SWIMBA_OP_SCAN_BWD:
       return kStatusBytes + scan_bwd_workspace(dims->batch, dims->seqlen, dims->d_inner, dims->d_state,
                                                dims->n_experts, dims->top_k);
@@ -321,10 +322,11 @@ swimba_status swimba_route_bwd(const swimba_dims* dims, const void* x, const flo
   if (!x || !W_r || !idx || !gates || !g_gates_a || !dx || !dW_r) return SWIMBA_ERR_INVALID_ARG;
   if (!aligned16(ws)) return SWIMBA_ERR_ALIGN;
   if (ws == nullptr || ws_bytes < swimba_workspace_size(dims, SWIMBA_OP_ROUTE_BWD)) return SWIMBA_ERR_WORKSPACE;
-  float* dlogits = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kStatusBytes);
-  return cuda_status(run_route_bwd(x, dims->io_dtype == SWIMBA_BF16, W_r, idx, gates, g_gates_a, g_gates_b, dlogits,
-                                   dx, dx_accumulate ? 1 : 0, dW_r, dims->batch * dims->seqlen, dims->d_inner,
-                                   dims->n_experts, dims->top_k, static_cast<cudaStream_t>(stream)));
+  if (!aligned16(dx) || !aligned16(W_r)) return SWIMBA_ERR_ALIGN;
+  return cuda_status(run_route_bwd(x, dims->io_dtype == SWIMBA_BF16, W_r, idx, gates, g_gates_a, g_gates_b,
+                                   static_cast<uint8_t*>(ws) + kStatusBytes, dx, dx_accumulate ? 1 : 0, dW_r,
+                                   dims->batch * dims->seqlen, dims->d_inner, dims->n_experts, dims->top_k,
+                                   static_cast<cudaStream_t>(stream)));
 }
 
 swimba_status swimba_scan_fwd_noalloc(const swimba_dims* dims, const void* x, const void* z, const float* delta,

@@ -21,10 +21,11 @@
 // matrices Xg and G; v (recomputed, fp32) = Xg W_x^e and q = G W_dt^eᵀ; then a per-pair kernel forms
 // dV, g_j dt_low (with g_j appended as an extra column, so that the W_dt GEMM also yields the bias
 // gradient) and the gate gradient; then Xgᵀ dV = ∂L/∂W_x^e, (g dt_low | g)ᵀ G = [∂L/∂W_dt^e ; ∂L/∂b_dt^e],
-// dV W_x^eᵀ = the pairs' input gradients, summed per token in slot order. The expert sizes are read
-// back to the host once per call (so the GEMM shapes are exact); that makes this entry point
-// synchronise its stream, unlike the forward ones.
-#include <vector>
+// dV W_x^eᵀ = the pairs' input gradients, scattered straight into ∂L/∂x rows by the GEMM's epilogue
+// (expert after expert: deterministic). The experts' independent GEMMs run side by side on a few
+// internal streams. The expert sizes are read back to the host once per call (so the GEMM shapes
+// are exact); that makes this entry point synchronise its stream, unlike the forward ones.
+#include <mutex>
 
 #include "common.cuh"
 
@@ -32,7 +33,7 @@ namespace swimba {
 
 cudaError_t run_gemm_tc(bool a_t, bool b_t, bool f32_out, int M, int N, int K, const void* A, int lda, const void* B,
                         int ldb, void* C0, int ldc0, void* C1, int ldc1, int split, const void* R, int ldr,
-                        void* status, cudaStream_t s);
+                        void* status, cudaStream_t s, const int* rows, int rows_div);
 
 namespace {
 
@@ -98,21 +99,21 @@ __global__ void __launch_bounds__(kSortThreads) pair_sort_kernel(const int32_t* 
   }
 }
 
-// One CTA per sorted row: Xg[row] = x[t] (bf16), G[row] = bf16(g_dt[t]) with
-// g_dt = ∂L/∂Δ (1 − e^{−Δ}), and bg[row] = b_dt^e · g_dt (fp32).
+// One CTA per token: g_dt = ∂L/∂Δ (1 − e^{−Δ}) is formed once, and each of the token's k pairs gets
+// its sorted row: Xg[row] = x[t] (bf16), G[row] = bf16(g_dt), bg[row] = b_dt^e · g_dt (fp32).
+constexpr int kMaxK = 16;
 template <typename WT>
 __global__ void __launch_bounds__(256) proj_bwd_gather_kernel(const __nv_bfloat16* x, const float* delta,
                                                               const float* g_delta, const int32_t* idx,
-                                                              const WT* b_dt, const int* perm, int k, int D, int E,
+                                                              const WT* b_dt, const int* inv, int k, int D, int E,
                                                               __nv_bfloat16* Xg, __nv_bfloat16* G, float* bg) {
-  const int row = blockIdx.x;
-  const int p = perm[row];
-  const int64_t t = p / k;
-  const int e = min(max(idx[p], 0), E - 1);
+  const int64_t t = blockIdx.x;
   const __nv_bfloat16* xr = x + t * D;
-  float part = 0.f;
+  float part[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) part[j] = 0.f;
   for (int c = threadIdx.x * 8; c < D; c += 256 * 8) {  // D % 8 == 0
-    *reinterpret_cast<uint4*>(Xg + (size_t)row * D + c) = *reinterpret_cast<const uint4*>(xr + c);
+    const uint4 xv = *reinterpret_cast<const uint4*>(xr + c);
     const float4 d0 = *reinterpret_cast<const float4*>(delta + t * D + c);
     const float4 d1 = *reinterpret_cast<const float4*>(delta + t * D + c + 4);
     const float4 g0 = *reinterpret_cast<const float4*>(g_delta + t * D + c);
@@ -121,24 +122,38 @@ __global__ void __launch_bounds__(256) proj_bwd_gather_kernel(const __nv_bfloat1
     const float gd[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
     float gdt[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      gdt[i] = -gd[i] * expm1f(-dl[i]);
-      part = fmaf(gdt[i], to_f32(b_dt[(size_t)e * D + c + i]), part);
+    for (int i = 0; i < 8; ++i) gdt[i] = -gd[i] * expm1f(-dl[i]);
+    __nv_bfloat162 hb[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) hb[i] = __floats2bfloat162_rn(gdt[2 * i], gdt[2 * i + 1]);
+    const uint4 gv = *reinterpret_cast<const uint4*>(hb);
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (j < k) {
+        const int row = inv[t * k + j];
+        const int e = min(max(idx[t * k + j], 0), E - 1);
+        *reinterpret_cast<uint4*>(Xg + (size_t)row * D + c) = xv;
+        *reinterpret_cast<uint4*>(G + (size_t)row * D + c) = gv;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) part[j] = fmaf(gdt[i], to_f32(b_dt[(size_t)e * D + c + i]), part[j]);
+      }
     }
-    __nv_bfloat162 h[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(gdt[2 * i], gdt[2 * i + 1]);
-    *reinterpret_cast<uint4*>(G + (size_t)row * D + c) = *reinterpret_cast<const uint4*>(h);
   }
+  __shared__ float wsum[8][kMaxK];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-  __shared__ float wsum[8];
-  if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5] = part;
+  for (int j = 0; j < kMaxK; ++j) {
+    if (j < k) {
+      float v = part[j];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5][j] = v;
+    }
+  }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    float s = 0.f;
-    for (int w = 0; w < 8; ++w) s += wsum[w];
-    bg[row] = s;
+  if (threadIdx.x < k) {
+    float v = 0.f;
+    for (int w = 0; w < 8; ++w) v += wsum[w][threadIdx.x];
+    bg[inv[t * k + threadIdx.x]] = v;
   }
 }
 
@@ -194,102 +209,96 @@ __global__ void proj_bwd_split_kernel(const float* TMP, int E, int R, int D, flo
   }
 }
 
-// ∂L/∂x[t] (+)= Σ_j DXP[inv[t k + j]] in slot order.
-__global__ void proj_bwd_dx_kernel(const float* DXP, const int* inv, int64_t T, int k, int D, float* dx,
-                                   int accumulate) {
-  const int64_t n4 = T * (D / 4);
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t t = i / (D / 4);
-    const int c = (int)(i % (D / 4)) * 4;
-    float4 acc = accumulate ? *reinterpret_cast<const float4*>(dx + t * D + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-      const float4 v = *reinterpret_cast<const float4*>(DXP + (size_t)inv[t * k + j] * D + c);
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
-    }
-    *reinterpret_cast<float4*>(dx + t * D + c) = acc;
-  }
-}
-
-// Router: per token, ∂L/∂logits from the gate gradients (the sum of up to two contributions), then
-// ∂L/∂x[t] (+)= Σ_e ∂L/∂logit_e W_r[:, e]. One warp per token.
-template <typename IO>
-__global__ void route_bwd_dx_kernel(const IO* x, const float* W_r, const int32_t* idx, const float* gates,
-                                    const float* gg_a, const float* gg_b, int64_t T, int D, int E, int k,
-                                    float* dlogits, float* dx, int accumulate) {
-  const int64_t t = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
+// Router: ∂L/∂logits per token from the gate gradients (the sum of up to two contributions):
+// ∂L/∂s_j = g_j (G_j − Σ_i g_i G_i) on the selected logits, zero elsewhere. One thread per token.
+__global__ void route_bwd_logits_kernel(const int32_t* idx, const float* gates, const float* gg_a, const float* gg_b,
+                                        int64_t T, int E, int k, float* dlogits) {
+  const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (t >= T) return;
-  float dl[kMaxE];
   float mean = 0.f;
-  for (int j = 0; j < k; ++j) {
-    const float gg = gg_a[t * k + j] + (gg_b ? gg_b[t * k + j] : 0.f);
-    mean = fmaf(gates[t * k + j], gg, mean);
-  }
-#pragma unroll
-  for (int e = 0; e < kMaxE; ++e) dl[e] = 0.f;
+  for (int j = 0; j < k; ++j) mean = fmaf(gates[t * k + j], gg_a[t * k + j] + (gg_b ? gg_b[t * k + j] : 0.f), mean);
+  for (int e = 0; e < E; ++e) dlogits[t * E + e] = 0.f;
   for (int j = 0; j < k; ++j) {
     const float gg = gg_a[t * k + j] + (gg_b ? gg_b[t * k + j] : 0.f);
     const int e = min(max(idx[t * k + j], 0), E - 1);
-    const float v = gates[t * k + j] * (gg - mean);
-#pragma unroll
-    for (int ee = 0; ee < kMaxE; ++ee)
-      if (ee == e) dl[ee] += v;
+    dlogits[t * E + e] += gates[t * k + j] * (gg - mean);
   }
-  if (lane < E) {
-    float v = 0.f;
-#pragma unroll
-    for (int ee = 0; ee < kMaxE; ++ee)
-      if (ee == lane) v = dl[ee];
-    dlogits[t * E + lane] = v;
-  }
-  for (int d = lane; d < D; d += 32) {
-    float s = accumulate ? dx[t * D + d] : 0.f;
-    for (int e = 0; e < E; ++e) s = fmaf(dl[e < kMaxE ? e : 0], W_r[(size_t)d * E + e], s);
-    dx[t * D + d] = s;
-  }
-  (void)x;
 }
 
-// ∂L/∂W_r[d, e] = Σ_t x[t, d] ∂L/∂logits[t, e]: a CTA owns 32 channels and all experts, threads
-// split the tokens into 8 runs, summed in a fixed order.
+// ∂L/∂x[t, d] (+)= Σ_e ∂L/∂logits[t, e] W_r[d, e]: a CTA owns 256 channels (a thread each, its
+// W_r row in registers) and a run of 64 tokens, whose ∂L/∂logits rows it stages in shared memory;
+// every dx access is a coalesced row segment.
+constexpr int kDxTok = 64;
+__global__ void __launch_bounds__(256) route_bwd_dx_kernel(const float* W_r, const float* dlogits, int64_t T, int D,
+                                                           int E, float* dx, int accumulate) {
+  __shared__ float dl[kDxTok][kMaxE];
+  const int d = blockIdx.x * 256 + threadIdx.x;
+  const int64_t t0 = (int64_t)blockIdx.y * kDxTok;
+  const int nt = (int)(T - t0 < kDxTok ? T - t0 : kDxTok);
+  for (int i = threadIdx.x; i < nt * kMaxE; i += 256) {
+    const int r = i / kMaxE, e = i % kMaxE;
+    dl[r][e] = e < E ? dlogits[(t0 + r) * E + e] : 0.f;
+  }
+  float w[kMaxE];
+#pragma unroll
+  for (int e = 0; e < kMaxE; ++e) w[e] = (d < D && e < E) ? W_r[(size_t)d * E + e] : 0.f;
+  __syncthreads();
+  if (d >= D) return;
+  for (int r = 0; r < nt; ++r) {
+    float acc = accumulate ? dx[(t0 + r) * D + d] : 0.f;
+#pragma unroll
+    for (int e = 0; e < kMaxE; ++e) acc = fmaf(dl[r][e], w[e], acc);
+    dx[(t0 + r) * D + d] = acc;
+  }
+}
+
+constexpr int kDwTok = 256;  // tokens per partial of ∂L/∂W_r
+
+// Partial ∂L/∂W_r over a block of 256 tokens: a CTA owns 64 channels x 4 token runs of 64; the
+// runs are summed in shared memory and the block's partial written [block][d][e].
 template <typename IO>
 __global__ void __launch_bounds__(256) route_bwd_dw_kernel(const IO* x, const float* dlogits, int64_t T, int D, int E,
-                                                           float* dW_r) {
-  __shared__ float red[8][32][kMaxE];
-  const int c = threadIdx.x & 31, run = threadIdx.x >> 5;
-  const int d = blockIdx.x * 32 + c;
+                                                           float* part) {
+  __shared__ float red[4][64][kMaxE + 1];
+  const int c = threadIdx.x & 63, run = threadIdx.x >> 6;
+  const int d = blockIdx.x * 64 + c;
+  const int64_t tb = blockIdx.y;
   float acc[kMaxE];
 #pragma unroll
   for (int e = 0; e < kMaxE; ++e) acc[e] = 0.f;
-  const int64_t per = (T + 7) / 8;
-  const int64_t t0 = run * per, t1 = min(T, t0 + per);
+  const int64_t t0 = tb * kDwTok + run * (kDwTok / 4), t1 = min(T, t0 + kDwTok / 4);
   if (d < D) {
+#pragma unroll 4
     for (int64_t t = t0; t < t1; ++t) {
       const float xv = to_f32(x[t * D + d]);
 #pragma unroll
       for (int e = 0; e < kMaxE; ++e)
-        if (e < E) acc[e] = fmaf(xv, dlogits[t * E + e], acc[e]);
+        if (e < E) acc[e] = fmaf(xv, __ldg(dlogits + t * E + e), acc[e]);
     }
   }
 #pragma unroll
   for (int e = 0; e < kMaxE; ++e) red[run][c][e] = acc[e];
   __syncthreads();
   if (run == 0 && d < D) {
-    for (int e = 0; e < E; ++e) {
-      float s = 0.f;
-      for (int r = 0; r < 8; ++r) s += red[r][c][e];
-      dW_r[(size_t)d * E + e] = s;
-    }
+    for (int e = 0; e < E; ++e)
+      part[(tb * D + d) * E + e] = red[0][c][e] + red[1][c][e] + red[2][c][e] + red[3][c][e];
+  }
+}
+
+// ∂L/∂W_r = Σ over the token blocks' partials, in block order.
+__global__ void route_bwd_dw_reduce_kernel(const float* part, int64_t nblk, int D, int E, float* dW_r) {
+  const int64_t n = (int64_t)D * E;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    float s = 0.f;
+    for (int64_t b = 0; b < nblk; ++b) s += part[b * n + i];
+    dW_r[i] = s;
   }
 }
 
 size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct ProjBwdLayout {
-  size_t counts, offsets, perm, inv, bg, Xg, G, XD, Q, dV, DTs, DXP, TMP, total;
+  size_t counts, offsets, perm, inv, bg, Xg, G, XD, Q, dV, DTs, TMP, total;
 };
 
 ProjBwdLayout proj_bwd_layout(int64_t T, int D, int R, int N, int E, int k) {
@@ -312,10 +321,51 @@ ProjBwdLayout proj_bwd_layout(int64_t T, int D, int R, int N, int E, int k) {
   l.Q = take(4 * P * R);
   l.dV = take(2 * P * W);
   l.DTs = take(2 * P * (R + 8));
-  l.DXP = take(4 * P * D);
   l.TMP = take(4 * (size_t)E * (R + 8) * D);
   l.total = o;
   return l;
+}
+
+
+// Side streams (per device, created once) on which the experts' independent GEMMs run side by
+// side: one expert's product fills only part of the GPU when its K or N is small.
+constexpr int kSideStreams = 4;
+struct SideStreams {
+  cudaStream_t s[kSideStreams];
+  cudaEvent_t fork, join[kSideStreams];
+  bool ok = false;
+};
+SideStreams* side_streams() {
+  static std::mutex mu;
+  static SideStreams per_dev[16];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  SideStreams& ss = per_dev[dev];
+  if (!ss.ok) {
+    bool good = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < kSideStreams && good; ++i)
+      good = cudaStreamCreateWithFlags(&ss.s[i], cudaStreamNonBlocking) == cudaSuccess &&
+             cudaEventCreateWithFlags(&ss.join[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!good) return nullptr;
+    ss.ok = true;
+  }
+  return &ss;
+}
+
+cudaError_t fork_to(SideStreams* ss, cudaStream_t s) {
+  cudaError_t e = cudaEventRecord(ss->fork, s);
+  for (int i = 0; i < kSideStreams && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(ss->s[i], ss->fork, 0);
+  return e;
+}
+
+cudaError_t join_from(SideStreams* ss, cudaStream_t s) {
+  cudaError_t e = cudaSuccess;
+  for (int i = 0; i < kSideStreams && e == cudaSuccess; ++i) {
+    e = cudaEventRecord(ss->join[i], ss->s[i]);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join[i], 0);
+  }
+  return e;
 }
 
 }  // namespace
@@ -339,10 +389,11 @@ cudaError_t run_proj_bwd(const void* x, const float* delta, const float* g_delta
   float* Q = reinterpret_cast<float*>(w + l.Q);
   __nv_bfloat16* dV = reinterpret_cast<__nv_bfloat16*>(w + l.dV);
   __nv_bfloat16* DTs = reinterpret_cast<__nv_bfloat16*>(w + l.DTs);
-  float* DXP = reinterpret_cast<float*>(w + l.DXP);
   float* TMP = reinterpret_cast<float*>(w + l.TMP);
   const int64_t P = T * k;
   const int W = R + 2 * N;
+  SideStreams* ss = side_streams();
+  if (ss == nullptr) return cudaErrorNotReady;
   cudaError_t e;
   const size_t sort_smem = sizeof(int) * (size_t)E * kSortThreads;
   if ((e = cudaFuncSetAttribute(pair_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sort_smem)) !=
@@ -350,80 +401,102 @@ cudaError_t run_proj_bwd(const void* x, const float* delta, const float* g_delta
     return e;
   pair_sort_kernel<<<1, kSortThreads, sort_smem, s>>>(idx, P, E, counts, offsets, perm, inv);
   if (b_bf16)
-    proj_bwd_gather_kernel<__nv_bfloat16><<<(unsigned)P, 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), delta, g_delta, idx, static_cast<const __nv_bfloat16*>(b_dt), perm, k,
+    proj_bwd_gather_kernel<__nv_bfloat16><<<(unsigned)T, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), delta, g_delta, idx, static_cast<const __nv_bfloat16*>(b_dt), inv, k,
         D, E, Xg, G, bg);
   else
-    proj_bwd_gather_kernel<float><<<(unsigned)P, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), delta, g_delta,
-                                                              idx, static_cast<const float*>(b_dt), perm, k, D, E, Xg,
+    proj_bwd_gather_kernel<float><<<(unsigned)T, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), delta, g_delta,
+                                                              idx, static_cast<const float*>(b_dt), inv, k, D, E, Xg,
                                                               G, bg);
   note_launch(2);
+  if (!accumulate && (e = cudaMemsetAsync(dx, 0, sizeof(float) * (size_t)T * D, s)) != cudaSuccess) return e;
   int h_off[kMaxE + 1];
   if ((e = cudaMemcpyAsync(h_off, offsets, sizeof(int) * (E + 1), cudaMemcpyDeviceToHost, s)) != cudaSuccess) return e;
   if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return e;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const __nv_bfloat16* Wx = static_cast<const __nv_bfloat16*>(W_x);
   const __nv_bfloat16* Wdt = static_cast<const __nv_bfloat16*>(W_dt);
-  // v = Xg W_x^e and q = G W_dt^eᵀ per expert
+  // v = Xg W_x^e and q = G W_dt^eᵀ per expert, the experts side by side
+  if ((e = fork_to(ss, s)) != cudaSuccess) return e;
   for (int ex = 0; ex < E; ++ex) {
     const int o = h_off[ex], n = h_off[ex + 1] - h_off[ex];
     if (n == 0) continue;
+    cudaStream_t se = ss->s[ex % kSideStreams];
     if ((e = run_gemm_tc(false, false, true, n, W, D, Xg + (size_t)o * D, D, Wx + (size_t)ex * D * W, W,
-                         XD + (size_t)o * W, W, nullptr, 0, W, nullptr, 0, status, s)) != cudaSuccess)
+                         XD + (size_t)o * W, W, nullptr, 0, W, nullptr, 0, status, se, nullptr, 1)) != cudaSuccess)
       return e;
     if ((e = run_gemm_tc(false, true, true, n, R, D, G + (size_t)o * D, D, Wdt + (size_t)ex * R * D, D,
-                         Q + (size_t)o * R, R, nullptr, 0, R, nullptr, 0, status, s)) != cudaSuccess)
+                         Q + (size_t)o * R, R, nullptr, 0, R, nullptr, 0, status, se, nullptr, 1)) != cudaSuccess)
       return e;
   }
+  if ((e = join_from(ss, s)) != cudaSuccess) return e;
   proj_bwd_pair_kernel<<<(unsigned)P, 128, 0, s>>>(XD, Q, bg, gB, gC, gates, perm, k, R, N, dV, DTs, dgates);
   note_launch();
+  // the weight gradients, the experts side by side: ∂L/∂W_x^e = Xgᵀ dV (Xg stored [pairs, D] = [K, M]);
+  // [∂L/∂W_dt^e ; ∂L/∂b_dt^e] = [g dt_low | g]ᵀ G
+  if ((e = fork_to(ss, s)) != cudaSuccess) return e;
   for (int ex = 0; ex < E; ++ex) {
     const int o = h_off[ex], n = h_off[ex + 1] - h_off[ex];
-    if (n == 0) continue;
-    // the pairs' input gradients dV W_x^eᵀ (W_x^e stored [D, R + 2N] = [N, K] of this product)
-    if ((e = run_gemm_tc(false, true, true, n, D, W, dV + (size_t)o * W, W, Wx + (size_t)ex * D * W, W,
-                         DXP + (size_t)o * D, D, nullptr, 0, D, nullptr, 0, status, s)) != cudaSuccess)
-      return e;
-    // ∂L/∂W_x^e = Xgᵀ dV (Xg stored [pairs, D] = [K, M])
+    cudaStream_t se = ss->s[ex % kSideStreams];
+    if (n == 0) {  // an expert no token chose has zero weight gradients
+      if ((e = cudaMemsetAsync(dW_x + (size_t)ex * D * W, 0, sizeof(float) * (size_t)D * W, se)) != cudaSuccess) return e;
+      if ((e = cudaMemsetAsync(TMP + (size_t)ex * (R + 8) * D, 0, sizeof(float) * (size_t)(R + 8) * D, se)) !=
+          cudaSuccess)
+        return e;
+      continue;
+    }
     if ((e = run_gemm_tc(true, false, true, D, W, n, Xg + (size_t)o * D, D, dV + (size_t)o * W, W,
-                         dW_x + (size_t)ex * D * W, W, nullptr, 0, W, nullptr, 0, status, s)) != cudaSuccess)
+                         dW_x + (size_t)ex * D * W, W, nullptr, 0, W, nullptr, 0, status, se, nullptr, 1)) !=
+        cudaSuccess)
       return e;
-    // [∂L/∂W_dt^e ; ∂L/∂b_dt^e] = [g dt_low | g]ᵀ G
     if ((e = run_gemm_tc(true, false, true, R + 8, D, n, DTs + (size_t)o * (R + 8), R + 8, G + (size_t)o * D, D,
-                         TMP + (size_t)ex * (R + 8) * D, D, nullptr, 0, D, nullptr, 0, status, s)) != cudaSuccess)
-      return e;
-  }
-  // experts without pairs have zero weight gradients
-  for (int ex = 0; ex < E; ++ex) {
-    if (h_off[ex + 1] != h_off[ex]) continue;
-    if ((e = cudaMemsetAsync(dW_x + (size_t)ex * D * W, 0, sizeof(float) * (size_t)D * W, s)) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(TMP + (size_t)ex * (R + 8) * D, 0, sizeof(float) * (size_t)(R + 8) * D, s)) !=
+                         TMP + (size_t)ex * (R + 8) * D, D, nullptr, 0, D, nullptr, 0, status, se, nullptr, 1)) !=
         cudaSuccess)
       return e;
   }
+  // meanwhile, on the caller's stream, the input gradients dV W_x^eᵀ (W_x^e stored [D, R + 2N] = [N, K]),
+  // added straight into dx rows (a token's pairs belong to distinct experts, so one expert's rows
+  // never repeat a token; the experts go one after another, in expert order)
+  for (int ex = 0; ex < E; ++ex) {
+    const int o = h_off[ex], n = h_off[ex + 1] - h_off[ex];
+    if (n == 0) continue;
+    if ((e = run_gemm_tc(false, true, true, n, D, W, dV + (size_t)o * W, W, Wx + (size_t)ex * D * W, W, dx, D, nullptr,
+                         0, D, dx, D, status, s, perm + o, k)) != cudaSuccess)
+      return e;
+  }
+  if ((e = join_from(ss, s)) != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   proj_bwd_split_kernel<<<(unsigned)(2 * sms), 256, 0, s>>>(TMP, E, R, D, dW_dt, db);
-  proj_bwd_dx_kernel<<<(unsigned)(8 * sms), 256, 0, s>>>(DXP, inv, T, k, D, dx, accumulate);
-  note_launch(2);
+  note_launch();
   return cudaGetLastError();
 }
 
+size_t route_bwd_workspace(int64_t T, int D, int E) {
+  const int64_t nblk = (T + kDwTok - 1) / kDwTok;
+  return up256((size_t)T * E * 4) + (size_t)nblk * D * E * 4;
+}
+
 cudaError_t run_route_bwd(const void* x, bool io_bf16, const float* W_r, const int32_t* idx, const float* gates,
-                          const float* gg_a, const float* gg_b, float* dlogits, float* dx, int accumulate, float* dW_r,
+                          const float* gg_a, const float* gg_b, void* ws, float* dx, int accumulate, float* dW_r,
                           int64_t T, int D, int E, int k, cudaStream_t s) {
-  const unsigned g1 = (unsigned)((T * 32 + 255) / 256), g2 = (unsigned)((D + 31) / 32);
-  if (io_bf16) {
-    route_bwd_dx_kernel<__nv_bfloat16><<<g1, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), W_r, idx, gates, gg_a,
-                                                          gg_b, T, D, E, k, dlogits, dx, accumulate);
-    route_bwd_dw_kernel<__nv_bfloat16><<<g2, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), dlogits, T, D, E, dW_r);
-  } else {
-    route_bwd_dx_kernel<float><<<g1, 256, 0, s>>>(static_cast<const float*>(x), W_r, idx, gates, gg_a, gg_b, T, D, E,
-                                                  k, dlogits, dx, accumulate);
-    route_bwd_dw_kernel<float><<<g2, 256, 0, s>>>(static_cast<const float*>(x), dlogits, T, D, E, dW_r);
-  }
-  note_launch(2);
+  float* dlogits = static_cast<float*>(ws);
+  float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + up256((size_t)T * E * 4));
+  const int64_t nblk = (T + kDwTok - 1) / kDwTok;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  route_bwd_logits_kernel<<<(unsigned)((T + 255) / 256), 256, 0, s>>>(idx, gates, gg_a, gg_b, T, E, k, dlogits);
+  route_bwd_dx_kernel<<<dim3((unsigned)((D + 255) / 256), (unsigned)((T + kDxTok - 1) / kDxTok)), 256, 0, s>>>(
+      W_r, dlogits, T, D, E, dx, accumulate);
+  const dim3 g((unsigned)((D + 63) / 64), (unsigned)nblk);
+  if (io_bf16)
+    route_bwd_dw_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), dlogits, T, D, E, part);
+  else
+    route_bwd_dw_kernel<float><<<g, 256, 0, s>>>(static_cast<const float*>(x), dlogits, T, D, E, part);
+  route_bwd_dw_reduce_kernel<<<(unsigned)(2 * sms), 256, 0, s>>>(part, nblk, D, E, dW_r);
+  note_launch(4);
   return cudaGetLastError();
 }
 
