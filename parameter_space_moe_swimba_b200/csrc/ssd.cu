@@ -23,14 +23,16 @@
 // for the readout, W and X_w -- enter the MMAs as two bf16 parts, hi = bf16(v) and
 // lo = bf16(v - hi) (about 16 significant bits, one more MMA each), so the state read out stays
 // fp32-accurate; a single bf16 copy of each moved y by up to 2e-2 (1 + |y|) on the test shapes.
+// W goes to tensor memory (tcgen05.st), where the Y1 product reads it as its A operand, which
+// leaves shared memory for two sets of the chunk tiles: the copies for chunk c + 1 are issued when
+// chunk c starts.
 // Two threads own row i of every [Q x *] accumulator (TMEM lane i; warps w and w + 4 share lane
 // quarter w), each half of the row's columns: they build row i of W, scale row i of X, write row i
-// of y and row i of Sᵀ; two warps per scheduler hide the exponentials' and the TMEM loads' latency
-// (with one, the kernel issued 0.21 instructions per cycle). The next chunk's Δ and gates are
-// loaded while the current chunk's outputs are written. One thread issues the TMA loads (C_mix, B, X
-// tiles, 128-byte swizzled; the next chunk's as soon as the MMAs have read the current one) and
-// the MMAs. Shapes: P = 64, N = 128, one active expert per token (the pages' Swimba-14B routes
-// every token to one of 4 experts).
+// of y and row i of Sᵀ; two warps per scheduler hide the exponentials' and the TMEM loads' latency.
+// The next chunk's Δ and gates are loaded while the current chunk's outputs are written. One
+// thread issues the TMA loads (C_mix, B, X tiles, 128-byte swizzled) and the MMAs. Shapes: P = 64,
+// N = 128, one active expert per token (the pages' Swimba-14B routes every token to one of 4
+// experts).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -48,24 +50,26 @@ constexpr int SP = 64;   // channels per head
 constexpr int SN = 128;  // state size
 constexpr int kBox = SQ * 128;  // one 128-row x 128-byte swizzled box: 16 KB
 
-// Shared memory (1024-byte aligned boxes for the 128-byte swizzle).
+// Shared memory (1024-byte aligned boxes for the 128-byte swizzle). A chunk's tiles (C_mix, B, X)
+// are double-buffered: the copies for chunk c + 1 are issued when chunk c starts.
 struct SsdSmem {
-  static constexpr int C = 0;                 // C_mix  [128 tok][128 n]: 2 boxes (K-major A)
-  static constexpr int B = C + 2 * kBox;      // B      [128 tok][128 n]: 2 boxes (K-major B; MN-major A)
-  static constexpr int X = B + 2 * kBox;      // X      [128 tok][64 p]:  1 box (MN-major B)
-  static constexpr int XW = X + kBox;         // X_w    [128 tok][64 p]:  hi, lo: 1 box each (MN-major B)
-  static constexpr int W = XW + 2 * kBox;     // W      [128 i][128 s]:   hi, lo: 2 boxes each (K-major A)
-  static constexpr int S = W + 4 * kBox;      // S_inᵀ  [128 n][64 p]:    hi, lo: 1 box each (MN-major B)
+  static constexpr int TILE = 5 * kBox;       // one chunk: C_mix [128 tok][128 n] (2 boxes, K-major A),
+                                              // B [128 tok][128 n] (2 boxes, K-major B / MN-major A),
+                                              // X [128 tok][64 p] (1 box, MN-major B)
+  static constexpr int TC = 0, TB = 2 * kBox, TX = 4 * kBox;  // offsets inside a tile buffer
+  static constexpr int XW = 2 * TILE;         // X_w    [128 tok][64 p]:  hi, lo: 1 box each (MN-major B)
+  static constexpr int S = XW + 2 * kBox;     // S_inᵀ  [128 n][64 p]:    hi, lo: 1 box each (MN-major B)
   static constexpr int CUM = S + 2 * kBox;    // f32 [128] cum
   static constexpr int DG = CUM + SQ * 4;     // f32 [128] Δ g
   static constexpr int WSUM = DG + SQ * 4;    // f32 [4] warp totals of the scan
-  static constexpr int BAR = WSUM + 64;       // 2 mbarriers
-  static constexpr int MISC = BAR + 16;       // abort flag, TMEM base
+  static constexpr int BAR = WSUM + 64;       // 3 mbarriers: copies into buffer 0, 1; MMAs
+  static constexpr int MISC = BAR + 32;       // abort flag, TMEM base
   static constexpr int BYTES = MISC + 16;
 };
 
-// TMEM columns of the accumulators.
-constexpr uint32_t kColG = 0, kColY1 = 128, kColY2 = 192, kColS = 256;
+// TMEM columns: fp32 accumulators G, Y1, Y2, Sᵀ; then W (the Y1 product's A operand, bf16 pairs):
+// hi in [kColW, kColW + 64), lo in [kColW + 64, kColW + 128).
+constexpr uint32_t kColG = 0, kColY1 = 128, kColY2 = 192, kColS = 256, kColW = 320;
 
 struct SsdParams {
   const float* gates;  // [B, L, 1]
@@ -104,8 +108,8 @@ __global__ void __launch_bounds__(256, 1)
   float* cum = reinterpret_cast<float*>(sm + SsdSmem::CUM);
   float* dg = reinterpret_cast<float*>(sm + SsdSmem::DG);
   float* wsum = reinterpret_cast<float*>(sm + SsdSmem::WSUM);
-  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + SsdSmem::BAR);
-  uint64_t* bar_mma = bar_tma + 1;
+  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + SsdSmem::BAR);  // [2]: copies into buffer 0, 1
+  uint64_t* bar_mma = bar_tma + 2;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + SsdSmem::MISC);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SsdSmem::MISC + 4);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -117,7 +121,8 @@ __global__ void __launch_bounds__(256, 1)
   const int nchunks = (int)((p.L + SQ - 1) / SQ);
 
   if (tid == 0) {
-    mbar_init(bar_tma, 1);
+    mbar_init(&bar_tma[0], 1);
+    mbar_init(&bar_tma[1], 1);
     mbar_init(bar_mma, 1);
     fence_mbar_init();
     *abort_flag = 0;
@@ -135,14 +140,16 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t tlane = tmem + ((uint32_t)(32 * (warp & 3)) << 16);  // this warp's lane quarter
 
   constexpr uint32_t tx_bytes = 2 * kBox + 2 * kBox + kBox;
-  auto issue_loads = [&](int c) {
-    mbar_arrive_expect_tx(bar_tma, tx_bytes);
+  auto issue_loads = [&](int c) {  // chunk c into buffer c & 1
+    uint64_t* bar = &bar_tma[c & 1];
+    uint8_t* tile = sm + (c & 1) * SsdSmem::TILE;
+    mbar_arrive_expect_tx(bar, tx_bytes);
     const int t0 = c * SQ;
-    tma_load_3d(sm + SsdSmem::C, &tm_c, bar_tma, 0, t0, b);
-    tma_load_3d(sm + SsdSmem::C + kBox, &tm_c, bar_tma, 64, t0, b);
-    tma_load_3d(sm + SsdSmem::B, &tm_b, bar_tma, 0, t0, b);
-    tma_load_3d(sm + SsdSmem::B + kBox, &tm_b, bar_tma, 64, t0, b);
-    tma_load_3d(sm + SsdSmem::X, &tm_x, bar_tma, h * SP, t0, b);
+    tma_load_3d(tile + SsdSmem::TC, &tm_c, bar, 0, t0, b);
+    tma_load_3d(tile + SsdSmem::TC + kBox, &tm_c, bar, 64, t0, b);
+    tma_load_3d(tile + SsdSmem::TB, &tm_b, bar, 0, t0, b);
+    tma_load_3d(tile + SsdSmem::TB + kBox, &tm_b, bar, 64, t0, b);
+    tma_load_3d(tile + SsdSmem::TX, &tm_x, bar, h * SP, t0, b);
   };
 
   // the carried state: Sᵀ[n][p] (row n = TMEM lane n; this thread's 32 columns p) into TMEM (fp32)
@@ -172,13 +179,12 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   tc_fence_after();
 
-  uint32_t ph_tma = 0, ph_mma = 0;
-  bool tma_pending = true, mma_pending = false;  // copies / MMAs issued and not yet waited for
+  uint32_t ph_tma[2] = {0, 0}, ph_mma = 0;
+  bool tma_pending[2] = {true, false}, mma_pending = false;  // copies / MMAs issued and not yet waited for
   const uint32_t id_qq = idesc_bf16(SQ, SQ, /*b_mn_major=*/false);        // G = C Bᵀ
   const uint32_t id_qp = idesc_bf16(SQ, SP, /*b_mn_major=*/true);         // Y1 = W X, Y2 = C Sᵀ
   const uint32_t id_st = idesc_bf16(SN, SP, /*b_mn_major=*/true, true);   // Sᵀ += Bᵀ X_w
-  const uint32_t sC = smem_u32(sm + SsdSmem::C), sB = smem_u32(sm + SsdSmem::B), sX = smem_u32(sm + SsdSmem::X);
-  const uint32_t sXW = smem_u32(sm + SsdSmem::XW), sW = smem_u32(sm + SsdSmem::W), sS = smem_u32(sm + SsdSmem::S);
+  const uint32_t sXW = smem_u32(sm + SsdSmem::XW), sS = smem_u32(sm + SsdSmem::S);
   // every wait ends in a CTA-wide vote, so that all threads leave the loop together
   auto vote_abort = [&](bool ok_here) -> bool {
     if (!ok_here) *abort_flag = 1;
@@ -195,6 +201,15 @@ __global__ void __launch_bounds__(256, 1)
   for (int c = 0; c < nchunks; ++c) {
     const int64_t t = (int64_t)c * SQ + row;
     const float gt = gt_next;
+    const int buf = c & 1;
+    uint8_t* tile = sm + buf * SsdSmem::TILE;
+    const uint32_t sC = smem_u32(tile + SsdSmem::TC), sB = smem_u32(tile + SsdSmem::TB),
+                   sX = smem_u32(tile + SsdSmem::TX);
+    // the next chunk's tiles into the other buffer (chunk c - 1, its last reader, is finished)
+    if (c + 1 < nchunks) {
+      if (tid == 0) issue_loads(c + 1);
+      tma_pending[buf ^ 1] = true;
+    }
     // the chunk's log decays: cum = inclusive prefix sum of Δ A_h over the 128 tokens (warps 0-3)
     if (half == 0) {
       float v = dl_next * Ah;
@@ -215,10 +230,10 @@ __global__ void __launch_bounds__(256, 1)
     }
 
     // the chunk's tiles have landed: G = C Bᵀ and Y2 = C S_inᵀ (K = n)
-    const bool got = mbar_wait(bar_tma, ph_tma, abort_flag);
-    ph_tma ^= 1u;
+    const bool got = mbar_wait(&bar_tma[buf], ph_tma[buf], abort_flag);
+    ph_tma[buf] ^= 1u;
     if (vote_abort(got)) break;  // (its barrier also publishes cum)
-    tma_pending = false;
+    tma_pending[buf] = false;
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
@@ -240,7 +255,7 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
         const int cc = half * 4 + c4;
-        const uint4 q = *reinterpret_cast<const uint4*>(sm + SsdSmem::X + swz(row, cc));
+        const uint4 q = *reinterpret_cast<const uint4*>(tile + SsdSmem::TX + swz(row, cc));
         const uint32_t in[4] = {q.x, q.y, q.z, q.w};
         uint32_t o[4], l[4];
 #pragma unroll
@@ -281,29 +296,23 @@ __global__ void __launch_bounds__(256, 1)
           const float w1 = s0 + 1 <= row ? __expf(ci - cum[s0 + 1]) * dg[s0 + 1] * gr[j + 1] : 0.f;
           split2(w0, w1, w16[j >> 1], l16[j >> 1]);
         }
-        // columns blk*32 .. +31: box blk/2 (hi), 2 + blk/2 (lo), 16-byte chunks (blk&1)*4 .. +3 of the row
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          *reinterpret_cast<uint4*>(sm + SsdSmem::W + (blk >> 1) * kBox + swz(row, (blk & 1) * 4 + cc)) =
-              make_uint4(w16[4 * cc], w16[4 * cc + 1], w16[4 * cc + 2], w16[4 * cc + 3]);
-          *reinterpret_cast<uint4*>(sm + SsdSmem::W + (2 + (blk >> 1)) * kBox + swz(row, (blk & 1) * 4 + cc)) =
-              make_uint4(l16[4 * cc], l16[4 * cc + 1], l16[4 * cc + 2], l16[4 * cc + 3]);
-        }
+        // columns s = blk*32 .. +31 of row i: 16 packed bf16 pairs of hi and of lo
+        tmem_st16(tlane + kColW + blk * 16, w16);
+        tmem_st16(tlane + kColW + 64 + blk * 16, l16);
       }
+      tmem_wait_st();
     }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    // Y1 = W X and Sᵀ += Bᵀ X_w (K = s)
+    // Y1 = W X (W from tensor memory) and Sᵀ += Bᵀ X_w (K = s)
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
       for (int ks = 0; ks < SQ / 16; ++ks) {
-        const uint32_t aoff = (uint32_t)((ks >> 2) * kBox + (ks & 3) * 32);
-        mma_bf16(tmem + kColY1, smem_desc(sW + aoff, 16, 1024, kLayoutSW128),
-                 smem_desc(sX + ks * 16 * 128, 8192, 1024, kLayoutSW128), id_qp, ks > 0 ? 1u : 0u);
-        mma_bf16(tmem + kColY1, smem_desc(sW + 2 * kBox + aoff, 16, 1024, kLayoutSW128),
-                 smem_desc(sX + ks * 16 * 128, 8192, 1024, kLayoutSW128), id_qp, 1u);
+        mma_bf16_ts(tmem + kColY1, tmem + kColW + ks * 8, smem_desc(sX + ks * 16 * 128, 8192, 1024, kLayoutSW128),
+                    id_qp, ks > 0 ? 1u : 0u);
+        mma_bf16_ts(tmem + kColY1, tmem + kColW + 64 + ks * 8,
+                    smem_desc(sX + ks * 16 * 128, 8192, 1024, kLayoutSW128), id_qp, 1u);
         mma_bf16(tmem + kColS, smem_desc(sB + ks * 16 * 128, kBox, 1024, kLayoutSW128),
                  smem_desc(sXW + ks * 16 * 128, 8192, 1024, kLayoutSW128), id_st, 1u);
         mma_bf16(tmem + kColS, smem_desc(sB + ks * 16 * 128, kBox, 1024, kLayoutSW128),
@@ -319,11 +328,9 @@ __global__ void __launch_bounds__(256, 1)
     // chunk's copies refill it
     uint4 xr[4];
 #pragma unroll
-    for (int c4 = 0; c4 < 4; ++c4) xr[c4] = *reinterpret_cast<const uint4*>(sm + SsdSmem::X + swz(row, half * 4 + c4));
+    for (int c4 = 0; c4 < 4; ++c4) xr[c4] = *reinterpret_cast<const uint4*>(tile + SsdSmem::TX + swz(row, half * 4 + c4));
     if (vote_abort(done2)) break;
     mma_pending = false;
-    if (tid == 0 && c + 1 < nchunks) issue_loads(c + 1);
-    if (c + 1 < nchunks) tma_pending = true;
     // the next chunk's Δ and gate, in flight while this chunk's outputs are written
     if (half == 0) {
       const int64_t tn = (int64_t)(c + 1) * SQ + row;
@@ -379,10 +386,12 @@ __global__ void __launch_bounds__(256, 1)
       record_device_error(p.status, SWIMBA_ERR_TIMEOUT, 51, blockIdx.x, 0);
       // let the copies and MMAs still in flight finish before TMEM and shared memory go away
       // (bounded; the flag is ignored here)
-      const uint64_t w0 = globaltimer_ns();
-      if (tma_pending)
-        while (!mbar_try_wait(bar_tma, ph_tma) && globaltimer_ns() - w0 < kWaitLimitNs) {
-        }
+      for (int bb = 0; bb < 2; ++bb) {
+        const uint64_t w0 = globaltimer_ns();
+        if (tma_pending[bb])
+          while (!mbar_try_wait(&bar_tma[bb], ph_tma[bb]) && globaltimer_ns() - w0 < kWaitLimitNs) {
+          }
+      }
       const uint64_t w1 = globaltimer_ns();
       if (mma_pending)
         while (!mbar_try_wait(bar_mma, ph_mma) && globaltimer_ns() - w1 < kWaitLimitNs) {
