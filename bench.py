@@ -898,8 +898,11 @@ def main():
         from parameter_space_moe_swimba_b200 import swimba as S
 
         torch.cuda.set_device(0)
-        print(json.dumps(report_bwd(torch, S, CONFIGS[args.workload], load_peaks(), L2Flush(torch, "cuda:0"), 10,
-                                    args.warmup)), flush=True)
+        cfg = CONFIGS[args.workload]
+        cfg = cfg.with_(batch=args.batch) if args.batch > 0 else cfg
+        cfg = cfg.with_(seqlen=args.seqlen) if args.seqlen > 0 else cfg
+        print(json.dumps(report_bwd(torch, S, cfg, load_peaks(), L2Flush(torch, "cuda:0"), 10, args.warmup)),
+              flush=True)
         return 0
     if args.report_separate:
         import torch

@@ -351,6 +351,7 @@ __global__ void __launch_bounds__(kSmallBucketThreads) group_bucket_small_kernel
 struct Stage1Params {
   int D, W, R, N, R_pad, K2, nbw;  // nbw: 64-column W_x boxes per expert
   int split, kper;                 // K split (1: the epilogue finishes the tile) and slices per split
+  int xshift;                      // x row of slot token v: v >> xshift (1: slots are (token, slot) pairs)
   const __nv_bfloat16* x;          // [T, D]
   float* partial;                  // split > 1: [tile * split + s][k * W + c][128 rows] fp32
   const int* num_tiles;
@@ -462,7 +463,8 @@ __global__ void __launch_bounds__(224, 1)
       const TileInfo ti = p.tiles[tile];
       int tokrow[32];  // token of tile row 4i + lane/8
 #pragma unroll
-      for (int i = 0; i < 32; ++i) tokrow[i] = p.slot_tok[ti.row_begin + min(4 * i + (lane >> 3), ti.rows - 1)];
+      for (int i = 0; i < 32; ++i)
+        tokrow[i] = p.slot_tok[ti.row_begin + min(4 * i + (lane >> 3), ti.rows - 1)] >> p.xshift;
       for (int ks = kb; ks < ke; ++ks) {
         if (!mbar_wait(&empty_a[stage], phase ^ 1u, abort_flag)) {
           ok = false;
@@ -687,7 +689,8 @@ struct Stage2Params {
   const int* slot_tok;
   const float* slot_gate;
   const float* b_dt;  // [E, D]
-  float* delta;
+  float* delta;       // softplus of the tile rows' sums; raw != 0: the sums themselves
+  int raw;
   void* status;
 };
 
@@ -1043,8 +1046,9 @@ __global__ void __launch_bounds__(576, 1)
                 bmix.y = fmaf(g[dh][r][j], bias[j].y, bmix.y);
               }
               if (valid[dh][r]) {
-                const float2 o = make_float2(softplus_fast(__uint_as_float(v[4 * k + 2 * r]) + bmix.x),
-                                             softplus_fast(__uint_as_float(v[4 * k + 2 * r + 1]) + bmix.y));
+                const float a0 = __uint_as_float(v[4 * k + 2 * r]) + bmix.x;
+                const float a1 = __uint_as_float(v[4 * k + 2 * r + 1]) + bmix.y;
+                const float2 o = p.raw ? make_float2(a0, a1) : make_float2(softplus_fast(a0), softplus_fast(a1));
                 *reinterpret_cast<float2*>(p.delta + (size_t)tok[dh][r] * p.D + d) = o;
               }
             }
@@ -1092,8 +1096,10 @@ int num_sms() {
   return n;
 }
 
+// The projection over "slots" p.T x k: tokens (xshift 0), or (token, slot) pairs run with k = 1
+// (xshift 1, raw 1: per-pair sums out, no softplus; see run_proj_pairs).
 template <int K>
-cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s) {
+cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s, int xshift = 0, int raw = 0) {
   const TcLayout L = tc_layout(p.T, p.E, K, p.R, p.D);
   int* group_of = reinterpret_cast<int*>(ws + L.group_of);
   int* blockhist = reinterpret_cast<int*>(ws + L.blockhist);
@@ -1144,7 +1150,7 @@ cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s) {
 
   const int sms = num_sms();
   Stage1Params s1{p.D,     W,       p.R,    p.N,      L.R_pad, L.K2,      nbw,       L.split,
-                  L.kper,  reinterpret_cast<const __nv_bfloat16*>(p.x), reinterpret_cast<float*>(ws + L.partial),
+                  L.kper,  xshift,  reinterpret_cast<const __nv_bfloat16*>(p.x), reinterpret_cast<float*>(ws + L.partial),
                   num_tiles, tiles, slot_tok, slot_gate, aprime, p.B_mix, p.C_mix, ws};
   const size_t smem1 = 1024 + (size_t)kStagesA * kSlotA + (size_t)kStagesW * kSlotW + 256;
   e = cudaFuncSetAttribute(proj_stage1_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
@@ -1158,7 +1164,7 @@ cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
 
-  Stage2Params s2{p.D, p.R, L.R_pad, L.K2, RS, num_tiles, tiles, slot_tok, slot_gate, p.b_dt, p.delta, ws};
+  Stage2Params s2{p.D, p.R, L.R_pad, L.K2, RS, num_tiles, tiles, slot_tok, slot_gate, p.b_dt, p.delta, raw, ws};
   const size_t smem2 = 1024 + (size_t)(L.K2 / 64) * kApBox + (size_t)kStages2 * kSlot2 + 16 * kBiasW + 256;
   e = cudaFuncSetAttribute(proj_stage2_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
   if (e != cudaSuccess) return e;
@@ -1166,6 +1172,75 @@ cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s) {
   note_launch();
   return cudaGetLastError();
 }
+
+// ---- few tokens, k = 2: the (token, slot) pairs bucketed by single expert ----------------------------
+// Bucketing tokens by expert PAIR leaves a decode step's 256 tokens spread over up to E(E-1)/2
+// groups of a few rows, each tile reading two experts' tables. For few tokens the projection runs
+// instead on the T k (token, slot) pairs v = k t + j as k = 1 slots (their expert idx[t][j], gate
+// g[t][j], x row t): every expert's tables are read by about (T k / 128 + 1) tiles, and the tiles
+// are fuller. The per-pair results -- g_j (dt_low_j W_dt^{e_j} + b_dt^{e_j}), g_j B^j, g_j C^j --
+// are summed per token in slot order by pair_combine_kernel, which also takes the softplus.
+constexpr int64_t kPairMaxT = 1024;  // tokens up to which k = 2 runs on expanded pairs
+
+struct PairLayout {
+  TcLayout inner;
+  size_t raw, bv, cv, total;
+};
+
+PairLayout pair_layout(int64_t T, int E, int R, int D) {
+  PairLayout L{};
+  L.inner = tc_layout(2 * T, E, 1, R, D);
+  size_t o = L.inner.total;
+  L.raw = o; o = align_up(o + 4 * (size_t)2 * T * D, 256);
+  L.bv = o; o = align_up(o + 4 * (size_t)2 * T * 16, 256);
+  L.cv = o; o = align_up(o + 4 * (size_t)2 * T * 16, 256);
+  L.total = o;
+  return L;
+}
+
+__global__ void __launch_bounds__(256) pair_combine_kernel(const float* raw, const float* bv, const float* cv,
+                                                           int64_t T, int D, float* delta, float* B_mix,
+                                                           float* C_mix) {
+  const int64_t nd = T * (D / 4), total = nd + T * 8;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    if (i < nd) {
+      const int64_t t = i / (D / 4);
+      const int c4 = (int)(i - t * (D / 4));
+      const float4 a = reinterpret_cast<const float4*>(raw + (size_t)(2 * t) * D)[c4];
+      const float4 b = reinterpret_cast<const float4*>(raw + (size_t)(2 * t + 1) * D)[c4];
+      reinterpret_cast<float4*>(delta + (size_t)t * D)[c4] =
+          make_float4(softplus_fast(a.x + b.x), softplus_fast(a.y + b.y), softplus_fast(a.z + b.z),
+                      softplus_fast(a.w + b.w));
+    } else {
+      const int64_t r = i - nd, t = r / 8;
+      const int q = (int)(r - t * 8);  // 0..3: B_mix float4 q; 4..7: C_mix float4 q - 4
+      const float* src = q < 4 ? bv : cv;
+      const float4 a = reinterpret_cast<const float4*>(src + (size_t)(2 * t) * 16)[q & 3];
+      const float4 b = reinterpret_cast<const float4*>(src + (size_t)(2 * t + 1) * 16)[q & 3];
+      reinterpret_cast<float4*>((q < 4 ? B_mix : C_mix) + (size_t)t * 16)[q & 3] =
+          make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+    }
+  }
+}
+
+cudaError_t run_proj_pairs(const ProjParams& p, uint8_t* ws, cudaStream_t s) {
+  const PairLayout L = pair_layout(p.T, p.E, p.R, p.D);
+  ProjParams q = p;
+  q.T = 2 * p.T;  // idx and gates [T, 2] are the pairs' [2T, 1]
+  q.k = 1;
+  q.delta = reinterpret_cast<float*>(ws + L.raw);
+  q.B_mix = reinterpret_cast<float*>(ws + L.bv);
+  q.C_mix = reinterpret_cast<float*>(ws + L.cv);
+  cudaError_t e = run_tc<1>(q, ws, s, 1, 1);
+  if (e != cudaSuccess) return e;
+  const int64_t total = p.T * (p.D / 4 + 8);
+  const unsigned grid = (unsigned)std::min<int64_t>((total + 255) / 256, 4 * (int64_t)num_sms());
+  pair_combine_kernel<<<grid, 256, 0, s>>>(q.delta, q.B_mix, q.C_mix, p.T, p.D, p.delta, p.B_mix, p.C_mix);
+  note_launch();
+  return cudaGetLastError();
+}
+
+bool use_pairs(int64_t T, int k) { return k == 2 && T <= kPairMaxT; }
 
 }  // namespace
 
@@ -1181,10 +1256,13 @@ bool proj_tc_supported(const ProjParams& p, bool io_bf16, bool w_bf16) {
   return true;
 }
 
-size_t proj_tc_workspace(int64_t T, int E, int k, int R, int D) { return tc_layout(T, E, k, R, D).total; }
+size_t proj_tc_workspace(int64_t T, int E, int k, int R, int D) {
+  return use_pairs(T, k) ? pair_layout(T, E, R, D).total : tc_layout(T, E, k, R, D).total;
+}
 
 cudaError_t run_proj_tc(const ProjParams& p, void* ws, cudaStream_t s) {
   uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+  if (use_pairs(p.T, p.k)) return run_proj_pairs(p, w, s);
   return p.k == 1 ? run_tc<1>(p, w, s) : run_tc<2>(p, w, s);
 }
 

@@ -25,7 +25,8 @@
 //           dA accumulates per thread in shared memory, dD in a register;
 //   reduce  sums the partials over channel tiles (dB, dC, dgates) and sequences (dA, dD) in a fixed
 //           order, so the result does not depend on scheduling.
-// Shapes: N <= 16, any k <= E <= 16, io fp32 or bf16.
+// Shapes: N <= 16, any k <= E <= 16, io fp32 or bf16. For N = 16, k <= 2 and D % 16 == 0 the bwd
+// kernel runs in a packed layout (two channels per lane, f32x2 arithmetic; scan_bwd_pk_kernel).
 #include "common.cuh"
 #include "scan.cuh"
 
@@ -49,8 +50,8 @@ __device__ __forceinline__ void load_a_rows(float* As, const float* A, int E, in
 
 }  // namespace
 
-// A chunk of up to 16 tokens of the CTA's 64 channels, staged in shared memory by all 256 threads
-// with 16-byte loads (the inner loops then read on-chip memory, not a chain of global loads).
+// A chunk of up to 16 tokens of the CTA's 64 channels, staged in shared memory by all the CTA's
+// threads with 16-byte loads (the inner loops then read on-chip memory, not a chain of global loads).
 template <typename IO>
 struct ChunkTile {
   float dl[kBwdLc][kBwdCh];
@@ -69,12 +70,12 @@ __device__ __forceinline__ void load_chunk(ChunkTile<IO>& ct, const ScanBwdParam
   const int tid = threadIdx.x;
   constexpr int per16 = 16 / (int)sizeof(IO);
   const int v4 = nc / 4, vio = nc / per16;  // nc % 8 == 0
-  for (int i = tid; i < nt * v4; i += 256) {
+  for (int i = tid; i < nt * v4; i += blockDim.x) {
     const int r = i / v4, c = (i % v4) * 4;
     *reinterpret_cast<float4*>(&ct.dl[r][c]) =
         *reinterpret_cast<const float4*>(p.delta + ((size_t)b * p.L + t0 + r) * p.D + d0 + c);
   }
-  for (int i = tid; i < nt * vio; i += 256) {
+  for (int i = tid; i < nt * vio; i += blockDim.x) {
     const int r = i / vio, c = (i % vio) * per16;
     const size_t g = ((size_t)b * p.L + t0 + r) * p.D + d0 + c;
     *reinterpret_cast<uint4*>(&ct.x[r][c]) = *reinterpret_cast<const uint4*>(reinterpret_cast<const IO*>(p.x) + g);
@@ -84,7 +85,7 @@ __device__ __forceinline__ void load_chunk(ChunkTile<IO>& ct, const ScanBwdParam
           *reinterpret_cast<const uint4*>(reinterpret_cast<const IO*>(p.g_out) + g);
     }
   }
-  for (int i = tid; i < nt * 16; i += 256) {
+  for (int i = tid; i < nt * 16; i += blockDim.x) {
     const int r = i / 16, n = i % 16;
     const size_t bt = (size_t)b * p.L + t0 + r;
     ct.B[r][n] = n < p.N ? p.B_mix[bt * p.N + n] : 0.f;
@@ -357,6 +358,362 @@ __global__ void __launch_bounds__(256, 2) scan_bwd_kernel(ScanBwdParams p) {
   }
 }
 
+// ---- packed layout for N = 16, k <= 2, D % 16 == 0 ---------------------------------------------
+// A CTA of 4 warps owns 64 channels; lane l of warp w holds the channel pair c0 = 16 w + 2 (l >> 2),
+// c1 = c0 + 1 and the state quarter q = l & 3 (states 4q .. 4q + 3), every per-state value a
+// float2 over the two channels (packed f32x2 arithmetic, as in the forward scan). Against the
+// one-channel layout above it halves the arithmetic and the per-channel loads per state element,
+// and the per-token sums over channels (dB, dC, the gate gradients) leave each lane with one value
+// of a reduce-scatter instead of every lane with every value.
+constexpr int kPkThreads = 128;
+constexpr int kPkWarps = 4;
+
+__device__ __forceinline__ float2 f2s(float v) { return make_float2(v, v); }
+
+// The A rows (4 states) of token r's expert slots for the lane's two channels. Lanes of odd channel
+// pairs read their second channel first, so every 8-lane phase of the 16-byte loads touches 8
+// distinct bank groups.
+template <int K, typename IO>
+__device__ __forceinline__ void load_a2(const ChunkTile<IO>& ct, const float* As, int r, int c0, int q,
+                                       float4 (&a0)[K], float4 (&a1)[K]) {
+  const bool sw = (c0 >> 1) & 1;
+#pragma unroll
+  for (int j = 0; j < K; ++j) {
+    const float4* row = reinterpret_cast<const float4*>(As) + (ct.e[r][j] * kBwdCh + c0) * 4 + q;
+    const float4 f = row[sw ? 4 : 0], t = row[sw ? 0 : 4];
+    a0[j] = sw ? t : f;
+    a1[j] = sw ? f : t;
+  }
+}
+
+// The mixed transition rows A_t = Σ_j g_j A^{e_j} (4 states, both channels) of staged token r.
+template <int K, typename IO>
+__device__ __forceinline__ void mix_a2(const ChunkTile<IO>& ct, const float4 (&a0)[K], const float4 (&a1)[K], int r,
+                                      float2 (&at)[4]) {
+#pragma unroll
+  for (int s = 0; s < 4; ++s) at[s] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < K; ++j) {
+    const float2 g = f2s(ct.g[r][j]);
+    at[0] = __ffma2_rn(g, make_float2(a0[j].x, a1[j].x), at[0]);
+    at[1] = __ffma2_rn(g, make_float2(a0[j].y, a1[j].y), at[1]);
+    at[2] = __ffma2_rn(g, make_float2(a0[j].z, a1[j].z), at[2]);
+    at[3] = __ffma2_rn(g, make_float2(a0[j].w, a1[j].w), at[3]);
+  }
+}
+
+template <int K, typename IO>
+__device__ __forceinline__ void mix_a2(const ChunkTile<IO>& ct, const float* As, int r, int c0, int q,
+                                      float2 (&at)[4]) {
+  float4 a0[K], a1[K];
+  load_a2<K>(ct, As, r, c0, q, a0, a1);
+  mix_a2<K>(ct, a0, a1, r, at);
+}
+
+__device__ __forceinline__ float2 ld2(const float (&row)[kBwdCh], int c0) {
+  return *reinterpret_cast<const float2*>(&row[c0]);
+}
+__device__ __forceinline__ float2 ld2(const __nv_bfloat16 (&row)[kBwdCh], int c0) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&row[c0]));
+}
+
+// One exp2 per component (the special-function unit has no packed form).
+__device__ __forceinline__ float2 ex2_2(float2 v) { return make_float2(ex2_approx(v.x), ex2_approx(v.y)); }
+
+template <typename IO, int K>
+__global__ void __launch_bounds__(kPkThreads) scan_bwd_ckpt_pk_kernel(ScanBwdParams p) {
+  extern __shared__ __align__(16) float smem_pk[];
+  float* As = smem_pk;  // [E][64][16]
+  ChunkTile<IO>& ct = *reinterpret_cast<ChunkTile<IO>*>(As + p.E * kBwdCh * 16);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q = lane & 3;
+  const int c0 = 16 * warp + 2 * (lane >> 2);
+  const int tiles = (p.D + kBwdCh - 1) / kBwdCh;
+  const int tile = blockIdx.x % tiles, b = blockIdx.x / tiles;
+  const int d0 = tile * kBwdCh, nc = min(kBwdCh, p.D - d0);  // nc % 16 == 0
+  const bool valid = 16 * warp < nc;                         // whole warps
+  load_a_rows(As, p.A, p.E, p.D, p.N, d0, nc);
+  float2 h[4];
+  {
+    float4 u0 = make_float4(0.f, 0.f, 0.f, 0.f), u1 = u0;
+    if (valid && p.h0 != nullptr) {
+      u0 = *reinterpret_cast<const float4*>(p.h0 + ((size_t)b * p.D + d0 + c0) * 16 + 4 * q);
+      u1 = *reinterpret_cast<const float4*>(p.h0 + ((size_t)b * p.D + d0 + c0 + 1) * 16 + 4 * q);
+    }
+    h[0] = make_float2(u0.x, u1.x);
+    h[1] = make_float2(u0.y, u1.y);
+    h[2] = make_float2(u0.z, u1.z);
+    h[3] = make_float2(u0.w, u1.w);
+  }
+  for (int ck = 0; ck < p.nck; ++ck) {
+    const int64_t t0 = (int64_t)ck * kBwdLc;
+    const int nt = (int)(p.L - t0 < kBwdLc ? p.L - t0 : kBwdLc);
+    if (valid) {
+      float* dst = p.ckpt + (((size_t)b * p.nck + ck) * p.D + d0 + c0) * 16 + 4 * q;
+      *reinterpret_cast<float4*>(dst) = make_float4(h[0].x, h[1].x, h[2].x, h[3].x);
+      *reinterpret_cast<float4*>(dst + 16) = make_float4(h[0].y, h[1].y, h[2].y, h[3].y);
+    }
+    __syncthreads();  // the previous chunk's tile is no longer read
+    load_chunk(ct, p, b, t0, nt, d0, nc, false);
+    __syncthreads();
+    for (int i = 0; i < nt; ++i) {
+      float2 at[4];
+      mix_a2<K>(ct, As, i, c0, q, at);
+      const float2 dl = ld2(ct.dl[i], c0);
+      const float2 c2 = __fmul2_rn(dl, f2s(kLog2e)), dx = __fmul2_rn(dl, ld2(ct.x[i], c0));
+#pragma unroll
+      for (int s = 0; s < 4; ++s)
+        h[s] = __ffma2_rn(ex2_2(__fmul2_rn(c2, at[s])), h[s], __fmul2_rn(dx, f2s(ct.B[i][4 * q + s])));
+    }
+  }
+}
+
+// The adjoint back through tokens [i0, i0 + ni) of the staged chunk (ni <= 4), packed layout: the
+// sub-block's states, transitions and dy are recomputed into registers from h_in (the state
+// before token i0), then walked backwards, updating `carry` (a_{t+1} λ_{t+1}).
+template <int K, typename IO>
+__device__ __forceinline__ void adjoint_sub_pk(const ScanBwdParams& p, const ChunkTile<IO>& ct, const float* As,
+                                               float* dAacc, float* red, int rw, int i0, int ni,
+                                               const float2 (&h_in)[4], int64_t t0, int b, int d0, int c0,
+                                               bool valid, float2 dsk, int tid, int warp, int lane, int q,
+                                               float2 (&carry)[4], float2& dD) {
+  float2 H[kBwdSub][4], AB[kBwdSub][4], DY[kBwdSub];
+  {
+    float2 h[4] = {h_in[0], h_in[1], h_in[2], h_in[3]};
+#pragma unroll
+    for (int u = 0; u < kBwdSub; ++u) {
+      if (u < ni) {
+        const int i = i0 + u;
+        float2 at[4];
+        mix_a2<K>(ct, As, i, c0, q, at);
+        const float2 dl = ld2(ct.dl[i], c0), xv = ld2(ct.x[i], c0);
+        const float2 c2 = __fmul2_rn(dl, f2s(kLog2e)), dx = __fmul2_rn(dl, xv);
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          AB[u][s] = ex2_2(__fmul2_rn(c2, at[s]));
+          h[s] = __ffma2_rn(AB[u][s], h[s], __fmul2_rn(dx, f2s(ct.B[i][4 * q + s])));
+          H[u][s] = h[s];
+        }
+        const float2 zv = ld2(ct.z[i], c0), go = ld2(ct.go[i], c0);
+        DY[u] = __fmul2_rn(__fmul2_rn(go, zv), make_float2(sigmoid_f(zv.x), sigmoid_f(zv.y)));
+      }
+    }
+  }
+#pragma unroll
+  for (int u = kBwdSub - 1; u >= 0; --u) {
+    if (u < ni) {
+      const int i = i0 + u;
+      float4 a0[K], a1[K];
+      load_a2<K>(ct, As, i, c0, q, a0, a1);
+      float2 at[4];
+      mix_a2<K>(ct, a0, a1, i, at);
+      const float2 dl = ld2(ct.dl[i], c0), xv = ld2(ct.x[i], c0);
+      const float2 dlx = __fmul2_rn(dl, xv);
+      float2 dA[4], sum_b = make_float2(0.f, 0.f), sum_d = make_float2(0.f, 0.f);
+      float vB[4], vC[4];
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const float2 hp = u > 0 ? H[u > 0 ? u - 1 : 0][s] : h_in[s];
+        const float2 lam = __ffma2_rn(f2s(ct.C[i][4 * q + s]), DY[u], carry[s]);
+        const float2 ahp = __fmul2_rn(AB[u][s], hp);
+        dA[s] = __fmul2_rn(__fmul2_rn(lam, dl), ahp);
+        sum_b = __ffma2_rn(lam, f2s(ct.B[i][4 * q + s]), sum_b);
+        sum_d = __ffma2_rn(__fmul2_rn(lam, at[s]), ahp, sum_d);
+        vB[s] = fmaf(lam.x, dlx.x, lam.y * dlx.y);               // this lane's 2 channels
+        vC[s] = fmaf(DY[u].x, H[u][s].x, DY[u].y * H[u][s].y);
+        carry[s] = __fmul2_rn(AB[u][s], lam);
+      }
+      // dx, dΔ: sums over the channel's 4 state quarters
+#pragma unroll
+      for (int o = 1; o < 4; o <<= 1) {
+        sum_b.x += __shfl_xor_sync(0xffffffffu, sum_b.x, o);
+        sum_b.y += __shfl_xor_sync(0xffffffffu, sum_b.y, o);
+        sum_d.x += __shfl_xor_sync(0xffffffffu, sum_d.x, o);
+        sum_d.y += __shfl_xor_sync(0xffffffffu, sum_d.y, o);
+      }
+      if (valid && q == 0) {
+        const size_t g = ((size_t)b * p.L + t0 + i) * p.D + d0 + c0;
+        *reinterpret_cast<float2*>(p.dx + g) = __ffma2_rn(dsk, DY[u], __fmul2_rn(dl, sum_b));
+        *reinterpret_cast<float2*>(p.ddelta + g) = __ffma2_rn(sum_b, xv, sum_d);
+        dD = __ffma2_rn(DY[u], xv, dD);
+      }
+      // dB, dC: the 8 values (vB[0..3], vC[0..3]) summed over the warp's 8 channel pairs (lane
+      // bits 2-4) by recursive halving; lane l ends with the value of type (l >> 4) & 1 (B, C) and
+      // state 4q + 2((l >> 3) & 1) + ((l >> 2) & 1)
+      float v4[4], v2[2], v1;
+      {
+        const bool hi = lane & 16;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const float keep = hi ? vC[m] : vB[m], send = hi ? vB[m] : vC[m];
+          v4[m] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+        }
+      }
+      {
+        const bool hi = lane & 8;
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          const float keep = hi ? v4[m + 2] : v4[m], send = hi ? v4[m] : v4[m + 2];
+          v2[m] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+        }
+      }
+      {
+        const bool hi = lane & 4;
+        const float keep = hi ? v2[1] : v2[0], send = hi ? v2[0] : v2[1];
+        v1 = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+      }
+      float* rrow = red + ((size_t)warp * kBwdLc + i) * rw;
+      rrow[((lane >> 4) & 1) * 16 + 4 * q + 2 * ((lane >> 3) & 1) + ((lane >> 2) & 1)] = v1;
+      // dA per expert slot, and the slots' gate gradients (sums over the warp's channels and states)
+      float pj[K];
+#pragma unroll
+      for (int j = 0; j < K; ++j) {
+        const int e = ct.e[i][j];
+        const float2 g = f2s(ct.g[i][j]);
+        float4* acc = reinterpret_cast<float4*>(dAacc) + (size_t)e * 2 * kPkThreads + tid;
+        float4 w0 = acc[0], w1 = acc[kPkThreads];
+        w0.x = fmaf(g.x, dA[0].x, w0.x);
+        w0.y = fmaf(g.x, dA[1].x, w0.y);
+        w0.z = fmaf(g.x, dA[2].x, w0.z);
+        w0.w = fmaf(g.x, dA[3].x, w0.w);
+        w1.x = fmaf(g.x, dA[0].y, w1.x);
+        w1.y = fmaf(g.x, dA[1].y, w1.y);
+        w1.z = fmaf(g.x, dA[2].y, w1.z);
+        w1.w = fmaf(g.x, dA[3].y, w1.w);
+        acc[0] = w0;
+        acc[kPkThreads] = w1;
+        pj[j] = dA[0].x * a0[j].x + dA[1].x * a0[j].y + dA[2].x * a0[j].z + dA[3].x * a0[j].w + dA[0].y * a1[j].x +
+                dA[1].y * a1[j].y + dA[2].y * a1[j].z + dA[3].y * a1[j].w;
+      }
+      float gsum;
+      if (K == 2) {  // first level of a reduce-scatter: lanes with bit 4 set carry slot 1
+        const bool hi = lane & 16;
+        gsum = (hi ? pj[K - 1] : pj[0]) + __shfl_xor_sync(0xffffffffu, hi ? pj[0] : pj[K - 1], 16);
+      } else {
+        gsum = pj[0] + __shfl_xor_sync(0xffffffffu, pj[0], 16);
+      }
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) gsum += __shfl_xor_sync(0xffffffffu, gsum, o);
+      if (lane == 0) rrow[32] = gsum;
+      if (K == 2 && lane == 16) rrow[33] = gsum;
+    }
+  }
+}
+
+// The chunk walk of the packed layout (same order as scan_bwd_kernel: the forward through each chunk
+// from its checkpoint, then the adjoint one sub-block at a time). Shared memory:
+// As[E][64][16] | dAacc[E][2][128 threads] float4 | sub[4][2][128 threads] float4 | red[4 warps][16][rw] |
+// tile (thread-fastest layouts: the 16-byte accesses are free of bank conflicts).
+template <typename IO, int K>
+__global__ void __launch_bounds__(kPkThreads) scan_bwd_pk_kernel(ScanBwdParams p) {
+  extern __shared__ __align__(16) float smem_pk[];
+  float* As = smem_pk;
+  float* dAacc = As + p.E * kBwdCh * 16;
+  float4* sub = reinterpret_cast<float4*>(dAacc + p.E * kPkThreads * 8);
+  float* red = reinterpret_cast<float*>(sub + (kBwdLc / kBwdSub) * kPkThreads * 2);
+  const int rw = 2 * 16 + K;  // per token: dB[16], dC[16], dgates[K]
+  ChunkTile<IO>& ct = *reinterpret_cast<ChunkTile<IO>*>(red + kPkWarps * kBwdLc * rw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q = lane & 3;
+  const int c0 = 16 * warp + 2 * (lane >> 2);
+  const int tiles = (p.D + kBwdCh - 1) / kBwdCh;
+  const int tile = blockIdx.x % tiles, b = blockIdx.x / tiles;
+  const int d0 = tile * kBwdCh, nc = min(kBwdCh, p.D - d0);  // nc % 16 == 0
+  const bool valid = 16 * warp < nc;                         // whole warps
+  load_a_rows(As, p.A, p.E, p.D, p.N, d0, nc);
+  for (int i = tid; i < p.E * kPkThreads * 8; i += kPkThreads) dAacc[i] = 0.f;
+  const float2 dsk = valid ? *reinterpret_cast<const float2*>(p.D_skip + d0 + c0) : make_float2(0.f, 0.f);
+  float2 carry[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float2 dD = make_float2(0.f, 0.f);
+
+  for (int ck = p.nck - 1; ck >= 0; --ck) {
+    const int64_t t0 = (int64_t)ck * kBwdLc;
+    const int nt = (int)(p.L - t0 < kBwdLc ? p.L - t0 : kBwdLc);
+    __syncthreads();  // the previous chunk's tile and partial sums are no longer read
+    load_chunk(ct, p, b, t0, nt, d0, nc, true);
+    float2 h[4];
+    {
+      float4 u0 = make_float4(0.f, 0.f, 0.f, 0.f), u1 = u0;
+      if (valid) {
+        const float* src = p.ckpt + (((size_t)b * p.nck + ck) * p.D + d0 + c0) * 16 + 4 * q;
+        u0 = *reinterpret_cast<const float4*>(src);
+        u1 = *reinterpret_cast<const float4*>(src + 16);
+      }
+      h[0] = make_float2(u0.x, u1.x);
+      h[1] = make_float2(u0.y, u1.y);
+      h[2] = make_float2(u0.z, u1.z);
+      h[3] = make_float2(u0.w, u1.w);
+    }
+    __syncthreads();
+    if (valid) {
+      // ---- forward through the chunk: the state before every sub-block, and dz ----
+      for (int i = 0; i < nt; ++i) {
+        if ((i & (kBwdSub - 1)) == 0) {
+          float4* sv = sub + (i / kBwdSub) * 2 * kPkThreads + tid;
+          sv[0] = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
+          sv[kPkThreads] = make_float4(h[2].x, h[2].y, h[3].x, h[3].y);
+        }
+        float2 at[4];
+        mix_a2<K>(ct, As, i, c0, q, at);
+        const float2 dl = ld2(ct.dl[i], c0), xv = ld2(ct.x[i], c0);
+        const float2 c2 = __fmul2_rn(dl, f2s(kLog2e)), dx = __fmul2_rn(dl, xv);
+        float2 y = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          h[s] = __ffma2_rn(ex2_2(__fmul2_rn(c2, at[s])), h[s], __fmul2_rn(dx, f2s(ct.B[i][4 * q + s])));
+          y = __ffma2_rn(f2s(ct.C[i][4 * q + s]), h[s], y);
+        }
+        y.x += __shfl_xor_sync(0xffffffffu, y.x, 1);
+        y.y += __shfl_xor_sync(0xffffffffu, y.y, 1);
+        y.x += __shfl_xor_sync(0xffffffffu, y.x, 2);
+        y.y += __shfl_xor_sync(0xffffffffu, y.y, 2);
+        if (q == 0) {
+          const float2 zv = ld2(ct.z[i], c0), go = ld2(ct.go[i], c0);
+          const float2 yy = __ffma2_rn(dsk, xv, y);
+          const float s0 = sigmoid_f(zv.x), s1 = sigmoid_f(zv.y);
+          *reinterpret_cast<float2*>(p.dz + ((size_t)b * p.L + t0 + i) * p.D + d0 + c0) =
+              make_float2(go.x * yy.x * s0 * fmaf(zv.x, 1.f - s0, 1.f), go.y * yy.y * s1 * fmaf(zv.y, 1.f - s1, 1.f));
+        }
+      }
+      // ---- the adjoint back through the chunk, one sub-block at a time ----
+      for (int sb = (nt - 1) / kBwdSub; sb >= 0; --sb) {
+        const int i0 = sb * kBwdSub;
+        const int ni = nt - i0 < kBwdSub ? nt - i0 : kBwdSub;
+        const float4* sv = sub + sb * 2 * kPkThreads + tid;
+        const float4 v0 = sv[0], v1 = sv[kPkThreads];
+        const float2 h_in[4] = {make_float2(v0.x, v0.y), make_float2(v0.z, v0.w), make_float2(v1.x, v1.y),
+                                make_float2(v1.z, v1.w)};
+        adjoint_sub_pk<K>(p, ct, As, dAacc, red, rw, i0, ni, h_in, t0, b, d0, c0, valid, dsk, tid, warp, lane, q,
+                          carry, dD);
+      }
+    } else {
+      for (int v = lane; v < nt * rw; v += 32) red[(size_t)warp * kBwdLc * rw + v] = 0.f;
+    }
+    __syncthreads();
+    // the chunk's per-token sums over the CTA's warps -> this tile's partial
+    for (int v = tid; v < nt * rw; v += kPkThreads) {
+      const int i = v / rw, w = v % rw;
+      float sum = 0.f;
+#pragma unroll
+      for (int wp = 0; wp < kPkWarps; ++wp) sum += red[((size_t)wp * kBwdLc + i) * rw + w];
+      const size_t tok = (size_t)b * p.L + t0 + i;
+      p.part[((size_t)tile * p.B * p.L + tok) * rw + w] = sum;
+    }
+  }
+  if (valid) {
+    if (p.dh0 != nullptr) {
+      float* dst = p.dh0 + ((size_t)b * p.D + d0 + c0) * 16 + 4 * q;
+      *reinterpret_cast<float4*>(dst) = make_float4(carry[0].x, carry[1].x, carry[2].x, carry[3].x);
+      *reinterpret_cast<float4*>(dst + 16) = make_float4(carry[0].y, carry[1].y, carry[2].y, carry[3].y);
+    }
+    for (int e = 0; e < p.E; ++e) {
+      const float4* acc = reinterpret_cast<const float4*>(dAacc) + (size_t)e * 2 * kPkThreads + tid;
+      float* dst = p.part_A + (((size_t)b * p.E + e) * p.D + d0 + c0) * 16 + 4 * q;
+      *reinterpret_cast<float4*>(dst) = acc[0];
+      *reinterpret_cast<float4*>(dst + 16) = acc[kPkThreads];
+    }
+    if (q == 0) *reinterpret_cast<float2*>(p.part_D + (size_t)b * p.D + d0 + c0) = dD;
+  }
+}
+
 // Sums of the partials in a fixed order: dB, dC, dgates over channel tiles; dA, dD over sequences.
 __global__ void scan_bwd_reduce_kernel(ScanBwdParams p, int tiles) {
   const int rw = 2 * p.N + p.k;
@@ -400,6 +757,20 @@ cudaError_t launch_bwd_pair(const ScanBwdParams& p, unsigned grid, size_t smem_c
   return cudaGetLastError();
 }
 
+template <typename IO, int K>
+cudaError_t launch_bwd_pk(const ScanBwdParams& p, unsigned grid, size_t smem_ck, size_t smem_bw, cudaStream_t s) {
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(scan_bwd_ckpt_pk_kernel<IO, K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem_ck)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(scan_bwd_pk_kernel<IO, K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem_bw)) != cudaSuccess)
+    return e;
+  scan_bwd_ckpt_pk_kernel<IO, K><<<grid, kPkThreads, smem_ck, s>>>(p);
+  scan_bwd_pk_kernel<IO, K><<<grid, kPkThreads, smem_bw, s>>>(p);
+  return cudaGetLastError();
+}
+
 size_t scan_bwd_workspace(int64_t B, int64_t L, int D, int N, int E, int k) {
   const int64_t tiles = (D + kBwdCh - 1) / kBwdCh;
   const int64_t nck = (L + kBwdLc - 1) / kBwdLc;
@@ -427,7 +798,20 @@ cudaError_t run_scan_bwd(ScanBwdParams p, bool io_bf16, void* ws, cudaStream_t s
   const size_t smem_bw = a_bytes + sizeof(float) * ((size_t)p.E * 256 * 4 + (size_t)kBwdWarps * kBwdLc * (2 * p.N + p.k)) +
                          sizeof(float4) * (kBwdLc / kBwdSub) * 256 + tile_bytes;
   cudaError_t e;
-  if (io_bf16) {
+  // packed layout: N = 16, k <= 2, whole 16-channel warps
+  const bool packed = p.N == 16 && (p.k == 1 || p.k == 2) && p.D % 16 == 0;
+  const size_t smem_pk = a_bytes +
+                         sizeof(float) * ((size_t)p.E * kPkThreads * 8 + (size_t)kPkWarps * kBwdLc * (32 + p.k)) +
+                         sizeof(float4) * (kBwdLc / kBwdSub) * kPkThreads * 2 + tile_bytes;
+  if (packed) {
+    if (io_bf16) {
+      e = p.k == 1 ? launch_bwd_pk<__nv_bfloat16, 1>(p, grid, smem_ck, smem_pk, s)
+                   : launch_bwd_pk<__nv_bfloat16, 2>(p, grid, smem_ck, smem_pk, s);
+    } else {
+      e = p.k == 1 ? launch_bwd_pk<float, 1>(p, grid, smem_ck, smem_pk, s)
+                   : launch_bwd_pk<float, 2>(p, grid, smem_ck, smem_pk, s);
+    }
+  } else if (io_bf16) {
     if (p.k == 1) e = launch_bwd_pair<__nv_bfloat16, 1>(p, grid, smem_ck, smem_bw, s);
     else if (p.k == 2) e = launch_bwd_pair<__nv_bfloat16, 2>(p, grid, smem_ck, smem_bw, s);
     else e = launch_bwd_pair<__nv_bfloat16, 0>(p, grid, smem_ck, smem_bw, s);

@@ -39,6 +39,8 @@ SHAPES = [
     (2, 40, 72, 5, 3, 6, 3, "f32", True),      # N = 5 < 16, k = 3
     (3, 1, 16, 16, 4, 4, 2, "bf16", True),     # one token
     (2, 300, 256, 16, 16, 8, 2, "bf16", True),  # several chunks and tiles
+    (1, 45, 208, 16, 8, 4, 1, "f32", True),    # packed layout, last tile one warp wide (208 = 3 x 64 + 16)
+    (2, 50, 72, 16, 8, 8, 2, "bf16", False),   # N = 16, k = 2 but D % 16 != 0: the one-channel layout
 ]
 
 
@@ -114,3 +116,4 @@ def test_scan_backward_rejects_bad_arguments(S):
     assert S.swimba_scan_bwd(dims, *full, W, None, None, *outs, None, ws, ws.numel()) == 1  # g_out missing
     assert S.swimba_scan_bwd(dims, *full, W, None, t, *outs, None, ws, 16) == 4
     assert S.swimba_scan_bwd(dims, *full, W, None, t, *outs, t.data_ptr() + 4, ws, ws.numel()) == 3
+    assert S.swimba_scan_bwd(dims, *full, W, None, t, t.data_ptr() + 8, *outs[1:], None, ws, ws.numel()) == 3
