@@ -176,20 +176,37 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(RouteParams 
   for (int c = threadIdx.x; c < p.D / V; c += kSmallThreads) {
     float xf[V];
     Vec16<IO>::unpack(__ldg(reinterpret_cast<const uint4*>(x) + c), xf);
+    if (vec) {
+      // every W_r load of the chunk is issued before the first multiply-add, so the V rows (from
+      // L2) arrive in one round trip rather than one after another
+      // (in groups of VG rows, at most 16 float4 registers)
+      constexpr int VG = V * (EP / 4) <= 16 ? V : 16 / (EP / 4);
+#pragma unroll
+      for (int v0 = 0; v0 < V; v0 += VG) {
+        float4 w4[VG][EP / 4];
+#pragma unroll
+        for (int v = 0; v < VG; ++v)
+#pragma unroll
+          for (int q = 0; q < EP / 4; ++q)
+            w4[v][q] = 4 * q < p.E
+                           ? __ldg(reinterpret_cast<const float4*>(p.W_r + (size_t)(c * V + v0 + v) * p.E) + q)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int v = 0; v < VG; ++v)
+#pragma unroll
+          for (int q = 0; q < EP / 4; ++q) {
+            acc[4 * q] = fmaf(xf[v0 + v], w4[v][q].x, acc[4 * q]);
+            acc[4 * q + 1] = fmaf(xf[v0 + v], w4[v][q].y, acc[4 * q + 1]);
+            acc[4 * q + 2] = fmaf(xf[v0 + v], w4[v][q].z, acc[4 * q + 2]);
+            acc[4 * q + 3] = fmaf(xf[v0 + v], w4[v][q].w, acc[4 * q + 3]);
+          }
+      }
+      continue;
+    }
 #pragma unroll
     for (int v = 0; v < V; ++v) {
       const float* w = p.W_r + (size_t)(c * V + v) * p.E;
-      if (vec) {
-#pragma unroll
-        for (int q = 0; q < EP / 4; ++q)
-          if (4 * q < p.E) {
-            const float4 w4 = __ldg(reinterpret_cast<const float4*>(w) + q);
-            acc[4 * q] = fmaf(xf[v], w4.x, acc[4 * q]);
-            acc[4 * q + 1] = fmaf(xf[v], w4.y, acc[4 * q + 1]);
-            acc[4 * q + 2] = fmaf(xf[v], w4.z, acc[4 * q + 2]);
-            acc[4 * q + 3] = fmaf(xf[v], w4.w, acc[4 * q + 3]);
-          }
-      } else {
+      {
 #pragma unroll
         for (int e = 0; e < EP; ++e)
           if (e < p.E) acc[e] = fmaf(xf[v], __ldg(w + e), acc[e]);
