@@ -32,6 +32,33 @@ __device__ __forceinline__ void record_device_error(void* ws, int code, int wher
 // Counts every kernel launch of the library (read through swimba_kernel_launches).
 void note_launch(int n = 1);
 
+// ---- programmatic dependent launch ---------------------------------------------------------------
+// The kernels of a chain (a decode step: router, bucketing, the projection's stages, the state
+// step) are launched with programmatic stream serialisation: a kernel may be scheduled while its
+// predecessor in the stream still runs, does its set-up (barriers, tensor memory, weight rows) and
+// then waits in pdl_wait() -- a hardware dependency, not a spin -- until the predecessor grid has
+// completed and its writes are visible. Nothing before pdl_wait() reads what an earlier kernel of
+// the stream writes or writes what it reads. pdl_trigger() lets the successor be scheduled early.
+// Launched without the attribute (or after a host-side dependency) both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 constexpr float kLog2e = 1.4426950408889634f;  // log2(e)
 
 // 2^x with the MUFU ex2 instruction (flush-to-zero; relative error about 2^-22).

@@ -264,6 +264,8 @@ __global__ void __launch_bounds__(kSmallBucketThreads) group_bucket_small_kernel
   __shared__ int s_run[kMaxGroups];
   __shared__ int warpcnt[kWarps][kMaxGroups];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_trigger();
+  pdl_wait();  // the router has completed
   for (int g = tid; g < G; g += kSmallBucketThreads) s_cnt[g] = 0;
   __syncthreads();
   int gs[kChunks];
@@ -441,6 +443,8 @@ __global__ void __launch_bounds__(224, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();  // the bucketing (or the previous stage) has completed
   const int num_tiles = *p.num_tiles;
   const int ksteps = p.D / BK1;
   const uint32_t w_bytes = (uint32_t)(K * p.nbw) * 8192u;
@@ -703,6 +707,8 @@ struct Stage2Params {
 template <int K>
 __global__ void __launch_bounds__(128) stage1_finish_kernel(const Stage1Params p) {
   const int tile = blockIdx.x;
+  pdl_trigger();
+  pdl_wait();
   if (tile >= *p.num_tiles) return;
   const int row = threadIdx.x;
   const TileInfo ti = p.tiles[tile];
@@ -825,6 +831,8 @@ __global__ void __launch_bounds__(576, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();  // the bucketing (or the previous stage) has completed
   const int num_tiles = *p.num_tiles;
   const int nchunks = (p.D + NC - 1) / NC;
   const long long total = (long long)num_tiles * nchunks;
@@ -1113,8 +1121,9 @@ cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s, int xshift 
 
   cudaError_t e;
   if (p.T <= kSmallBucketT) {
-    group_bucket_small_kernel<K><<<1, kSmallBucketThreads, 0, s>>>(p.idx, p.gates, (int)p.T, p.E, L.G, offsets,
-                                                                    num_tiles, tiles, slot_tok, slot_gate);
+    if ((e = launch_pdl(group_bucket_small_kernel<K>, dim3(1), dim3(kSmallBucketThreads), 0, s, p.idx, p.gates, (int)p.T,
+                        p.E, L.G, offsets, num_tiles, tiles, slot_tok, slot_gate)) != cudaSuccess)
+      return e;
     note_launch();
   } else {
     group_count_kernel<K><<<(unsigned)L.nb, kBucketBlock, 0, s>>>(p.idx, p.T, p.E, L.G, group_of, blockhist);
@@ -1155,11 +1164,15 @@ cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s, int xshift 
   const size_t smem1 = 1024 + (size_t)kStagesA * kSlotA + (size_t)kStagesW * kSlotW + 256;
   e = cudaFuncSetAttribute(proj_stage1_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
   if (e != cudaSuccess) return e;
-  proj_stage1_kernel<K><<<(unsigned)std::min(L.max_tiles * L.split, sms), 224, smem1, s>>>(tm_wx, s1);
+  if ((e = launch_pdl(proj_stage1_kernel<K>, dim3((unsigned)std::min(L.max_tiles * L.split, sms)), dim3(224), smem1, s,
+                      tm_wx, s1)) != cudaSuccess)
+    return e;
   note_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (L.split > 1) {
-    stage1_finish_kernel<K><<<dim3((unsigned)L.max_tiles, (unsigned)(K * p.R / 8 + 4)), 128, 0, s>>>(s1);
+    if ((e = launch_pdl(stage1_finish_kernel<K>, dim3((unsigned)L.max_tiles, (unsigned)(K * p.R / 8 + 4)), dim3(128), 0,
+                        s, s1)) != cudaSuccess)
+      return e;
     note_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -1168,7 +1181,8 @@ cudaError_t run_tc(const ProjParams& p, uint8_t* ws, cudaStream_t s, int xshift 
   const size_t smem2 = 1024 + (size_t)(L.K2 / 64) * kApBox + (size_t)kStages2 * kSlot2 + 16 * kBiasW + 256;
   e = cudaFuncSetAttribute(proj_stage2_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
   if (e != cudaSuccess) return e;
-  proj_stage2_kernel<K><<<(unsigned)sms, 576, smem2, s>>>(tm_ap, tm_wdt, s2);
+  if ((e = launch_pdl(proj_stage2_kernel<K>, dim3((unsigned)sms), dim3(576), smem2, s, tm_ap, tm_wdt, s2)) != cudaSuccess)
+    return e;
   note_launch();
   return cudaGetLastError();
 }
@@ -1201,6 +1215,8 @@ PairLayout pair_layout(int64_t T, int E, int R, int D) {
 __global__ void __launch_bounds__(256) pair_combine_kernel(const float* raw, const float* bv, const float* cv,
                                                            int64_t T, int D, float* delta, float* B_mix,
                                                            float* C_mix) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t nd = T * (D / 4), total = nd + T * 8;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
     if (i < nd) {
@@ -1235,7 +1251,9 @@ cudaError_t run_proj_pairs(const ProjParams& p, uint8_t* ws, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int64_t total = p.T * (p.D / 4 + 8);
   const unsigned grid = (unsigned)std::min<int64_t>((total + 255) / 256, 4 * (int64_t)num_sms());
-  pair_combine_kernel<<<grid, 256, 0, s>>>(q.delta, q.B_mix, q.C_mix, p.T, p.D, p.delta, p.B_mix, p.C_mix);
+  if ((e = launch_pdl(pair_combine_kernel, dim3(grid), dim3(256), 0, s, q.delta, q.B_mix, q.C_mix, p.T, p.D, p.delta,
+                      p.B_mix, p.C_mix)) != cudaSuccess)
+    return e;
   note_launch();
   return cudaGetLastError();
 }

@@ -167,6 +167,8 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(RouteParams 
   constexpr int kWarps = kSmallThreads / 32;
   __shared__ float part[kWarps][EP];
   const int64_t t = blockIdx.x;
+  pdl_trigger();
+  pdl_wait();  // x may come from the kernel before
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const IO* x = reinterpret_cast<const IO*>(p.x) + t * p.D;
   float acc[EP];
@@ -238,7 +240,8 @@ static cudaError_t launch_route(const RouteParams& p, cudaStream_t s) {
   const size_t smem = sizeof(float2) * (EP / 2) * (size_t)p.D;
   (void)V;
   if (p.T <= kSmallT) {
-    route_small_kernel<IO, EP><<<(unsigned)p.T, kSmallThreads, 0, s>>>(p);
+    const cudaError_t e = launch_pdl(route_small_kernel<IO, EP>, dim3((unsigned)p.T), dim3(kSmallThreads), 0, s, p);
+    if (e != cudaSuccess) return e;
   } else if (smem <= 160 * 1024) {
     cudaError_t e =
         cudaFuncSetAttribute(route_smem_kernel<IO, EP, TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

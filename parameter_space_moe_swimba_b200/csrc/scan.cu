@@ -292,6 +292,8 @@ __global__ void __launch_bounds__(256, 3) step_stream_kernel(ScanParams p, int s
     a_rows[e * kStepCh * 4 + r] = __ldg(reinterpret_cast<const float4*>(p.A + ((size_t)e * p.D + d0) * 16) + r);
   }
   __syncthreads();
+  pdl_trigger();
+  pdl_wait();  // Δ, B_mix, C_mix, the experts and gates of this step have been written
   if (c >= nc) return;  // whole warps (8 channels each) leave together; nothing below synchronises
   const int d = d0 + c;
   const float dsk = p.D_skip[d];
@@ -368,7 +370,9 @@ static cudaError_t launch_step_stream(const ScanParams& p, cudaStream_t s) {
   int groups = std::max(1, std::min(p.B, std::max(1, per_sm) * sms / tiles));
   const int spc = (p.B + groups - 1) / groups;
   groups = (p.B + spc - 1) / spc;
-  step_stream_kernel<IO, K><<<(unsigned)(tiles * groups), 256, smem, s>>>(p, spc);
+  if ((e = launch_pdl(step_stream_kernel<IO, K>, dim3((unsigned)(tiles * groups)), dim3(256), smem, s, p, spc)) !=
+      cudaSuccess)
+    return e;
   note_launch();
   return cudaGetLastError();
 }
