@@ -154,35 +154,42 @@ __global__ void __launch_bounds__(512, 1) route_smem_kernel(RouteParams p) {
   }
 }
 
-// Few tokens (decode steps, short prompts): one CTA of 512 threads per token, so every SM works
-// even when T is a few hundred. The threads split the channels in 16-byte chunks of x (one chunk
-// each at D = 4096 bf16, so a thread's x and W_r loads are all in flight at once), each
-// accumulates the E partial logits of its chunks (W_r rows from L2), a shuffle butterfly and a
-// shared-memory pass reduce them, and thread 0 selects and normalises the token's experts.
+// Few tokens (decode steps, short prompts): one CTA of 512 threads per TB tokens (TB = 4, 2 for
+// E > 8), so every SM works even when T is a few hundred while each W_r row read from L2 serves TB
+// tokens. The threads split the channels in 16-byte chunks of x (one chunk each at D = 4096
+// bf16); for each chunk a thread loads the TB tokens' x, then the chunk's W_r rows in groups (all
+// loads of a group issued before its multiply-adds), and accumulates the E partial logits of every
+// token; per token a shuffle butterfly and a shared-memory pass over the warps reduce them (in the
+// same order for every TB, so the logits do not depend on it), and one thread per token selects and
+// normalises its experts.
 constexpr int kSmallThreads = 512;  // one 16-byte chunk of x per thread at D = 4096 (bf16)
 
-template <typename IO, int EP>
-__global__ void __launch_bounds__(kSmallThreads) route_small_kernel(RouteParams p) {
+template <typename IO, int EP, int TB>
+__global__ void __launch_bounds__(kSmallThreads, 1) route_small_kernel(RouteParams p) {
   constexpr int V = Vec16<IO>::n;
   constexpr int kWarps = kSmallThreads / 32;
-  __shared__ float part[kWarps][EP];
-  const int64_t t = blockIdx.x;
+  constexpr int VG = 32 / EP < V ? 32 / EP : V;  // W_r rows per load group: at most 32 registers
+  __shared__ float part[kWarps][TB][EP];
+  __shared__ float logit[TB][EP];
+  const int64_t t0 = (int64_t)blockIdx.x * TB;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   pdl_trigger();
   pdl_wait();  // x may come from the kernel before
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const IO* x = reinterpret_cast<const IO*>(p.x) + t * p.D;
-  float acc[EP];
+  float acc[TB][EP];
 #pragma unroll
-  for (int e = 0; e < EP; ++e) acc[e] = 0.f;
+  for (int tb = 0; tb < TB; ++tb)
+#pragma unroll
+    for (int e = 0; e < EP; ++e) acc[tb][e] = 0.f;
   const bool vec = (p.E & 3) == 0;  // W_r rows of 16-byte multiples: float4 loads
   for (int c = threadIdx.x; c < p.D / V; c += kSmallThreads) {
-    float xf[V];
-    Vec16<IO>::unpack(__ldg(reinterpret_cast<const uint4*>(x) + c), xf);
+    float xf[TB][V];
+#pragma unroll
+    for (int tb = 0; tb < TB; ++tb) {
+      const int64_t t = t0 + tb < p.T ? t0 + tb : p.T - 1;  // past the end: a repeat, not stored
+      Vec16<IO>::unpack(__ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const IO*>(p.x) + t * p.D) + c),
+                        xf[tb]);
+    }
     if (vec) {
-      // every W_r load of the chunk is issued before the first multiply-add, so the V rows (from
-      // L2) arrive in one round trip rather than one after another
-      // (in groups of VG rows, at most 16 float4 registers)
-      constexpr int VG = V * (EP / 4) <= 16 ? V : 16 / (EP / 4);
 #pragma unroll
       for (int v0 = 0; v0 < V; v0 += VG) {
         float4 w4[VG][EP / 4];
@@ -194,42 +201,54 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(RouteParams 
                            ? __ldg(reinterpret_cast<const float4*>(p.W_r + (size_t)(c * V + v0 + v) * p.E) + q)
                            : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int v = 0; v < VG; ++v)
+        for (int tb = 0; tb < TB; ++tb)
 #pragma unroll
-          for (int q = 0; q < EP / 4; ++q) {
-            acc[4 * q] = fmaf(xf[v0 + v], w4[v][q].x, acc[4 * q]);
-            acc[4 * q + 1] = fmaf(xf[v0 + v], w4[v][q].y, acc[4 * q + 1]);
-            acc[4 * q + 2] = fmaf(xf[v0 + v], w4[v][q].z, acc[4 * q + 2]);
-            acc[4 * q + 3] = fmaf(xf[v0 + v], w4[v][q].w, acc[4 * q + 3]);
-          }
+          for (int v = 0; v < VG; ++v)
+#pragma unroll
+            for (int q = 0; q < EP / 4; ++q) {
+              acc[tb][4 * q] = fmaf(xf[tb][v0 + v], w4[v][q].x, acc[tb][4 * q]);
+              acc[tb][4 * q + 1] = fmaf(xf[tb][v0 + v], w4[v][q].y, acc[tb][4 * q + 1]);
+              acc[tb][4 * q + 2] = fmaf(xf[tb][v0 + v], w4[v][q].z, acc[tb][4 * q + 2]);
+              acc[tb][4 * q + 3] = fmaf(xf[tb][v0 + v], w4[v][q].w, acc[tb][4 * q + 3]);
+            }
       }
-      continue;
-    }
+    } else {
 #pragma unroll
-    for (int v = 0; v < V; ++v) {
-      const float* w = p.W_r + (size_t)(c * V + v) * p.E;
-      {
+      for (int v = 0; v < V; ++v) {
+        const float* w = p.W_r + (size_t)(c * V + v) * p.E;
 #pragma unroll
         for (int e = 0; e < EP; ++e)
-          if (e < p.E) acc[e] = fmaf(xf[v], __ldg(w + e), acc[e]);
+          if (e < p.E) {
+            const float we = __ldg(w + e);
+#pragma unroll
+            for (int tb = 0; tb < TB; ++tb) acc[tb][e] = fmaf(xf[tb][v], we, acc[tb][e]);
+          }
       }
     }
   }
 #pragma unroll
-  for (int e = 0; e < EP; ++e) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
-    if (lane == 0) part[warp][e] = acc[e];
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float l[EP];
+  for (int tb = 0; tb < TB; ++tb)
 #pragma unroll
     for (int e = 0; e < EP; ++e) {
-      float a = 0.f;
-      for (int w = 0; w < kWarps; ++w) a += part[w][e];
-      l[e] = a;
+      float a = acc[tb][e];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+      if (lane == 0) part[warp][tb][e] = a;
     }
+  __syncthreads();
+  if (threadIdx.x < TB * EP) {
+    const int tb = threadIdx.x / EP, e = threadIdx.x % EP;
+    float a = 0.f;
+    for (int w = 0; w < kWarps; ++w) a += part[w][tb][e];
+    logit[tb][e] = a;
+  }
+  __syncthreads();
+  if (threadIdx.x < TB && t0 + threadIdx.x < p.T) {
+    const int tb = threadIdx.x;
+    float l[EP];
+#pragma unroll
+    for (int e = 0; e < EP; ++e) l[e] = logit[tb][e];
+    const int64_t t = t0 + tb;
     select_topk<EP>(l, p.E, p.k, p.idx + t * p.k, p.gates + t * p.k);
   }
 }
@@ -240,7 +259,9 @@ static cudaError_t launch_route(const RouteParams& p, cudaStream_t s) {
   const size_t smem = sizeof(float2) * (EP / 2) * (size_t)p.D;
   (void)V;
   if (p.T <= kSmallT) {
-    const cudaError_t e = launch_pdl(route_small_kernel<IO, EP>, dim3((unsigned)p.T), dim3(kSmallThreads), 0, s, p);
+    constexpr int TB = EP <= 8 ? 4 : 2;
+    const cudaError_t e =
+        launch_pdl(route_small_kernel<IO, EP, TB>, dim3((unsigned)((p.T + TB - 1) / TB)), dim3(kSmallThreads), 0, s, p);
     if (e != cudaSuccess) return e;
   } else if (smem <= 160 * 1024) {
     cudaError_t e =

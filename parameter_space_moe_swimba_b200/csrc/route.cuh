@@ -47,8 +47,8 @@ __device__ __forceinline__ void select_topk(const float (&l)[EP], int E, int k, 
     if (j < k) gates[j] = wsel[j] / sum;
 }
 
-// Up to this many tokens the router runs one CTA per token (route_small_kernel): enough CTAs to
-// fill the GPU when T is small, where the tile-streaming kernels would leave most SMs idle.
+// Up to this many tokens the router runs one CTA per 2-4 tokens (route_small_kernel): enough CTAs
+// to fill the GPU when T is small, where the tile-streaming kernels would leave most SMs idle.
 constexpr int64_t kSmallT = 2048;
 
 // Tensor-core router (route_tc.cu): bf16 x, D a multiple of 64, E <= 16.
