@@ -26,9 +26,11 @@
 //   reduce  sums the partials over channel tiles (dB, dC, dgates) and sequences (dA, dD) in a fixed
 //           order, so the result does not depend on scheduling.
 // Shapes: N <= 16, any k <= E <= 16, io fp32 or bf16. For N = 16, k <= 2 and D % 16 == 0 the bwd
-// kernel runs in a packed layout (two channels per lane, f32x2 arithmetic; scan_bwd_pk_kernel).
+// kernel runs in a packed layout (two channels per lane, f32x2 arithmetic, the A rows in tensor
+// memory; scan_bwd_pk_kernel).
 #include "common.cuh"
 #include "scan.cuh"
+#include "sm100.cuh"
 
 namespace swimba {
 
@@ -38,7 +40,7 @@ constexpr int kBwdCh = 64;    // channels per CTA
 constexpr int kBwdLc = 16;    // tokens per checkpoint chunk
 constexpr int kBwdWarps = 8;  // 256 threads
 
-__device__ __forceinline__ float sigmoid_f(float v) { return 1.f / (1.f + ex2_approx(-v * kLog2e)); }
+__device__ __forceinline__ float sigmoid_f(float v) { return __fdividef(1.f, 1.f + ex2_approx(-v * kLog2e)); }
 
 // The A rows of every expert for the CTA's channels: As[e][c][16], zero beyond N.
 __device__ __forceinline__ void load_a_rows(float* As, const float* A, int E, int D, int N, int d0, int nc) {
@@ -410,6 +412,25 @@ __device__ __forceinline__ void mix_a2(const ChunkTile<IO>& ct, const float* As,
   mix_a2<K>(ct, a0, a1, r, at);
 }
 
+// The same rows from tensor memory: in the warp's lane quarter (tm_lane = its address), column 8e of
+// lane l holds (A[e][c0][4q .. 4q+3], A[e][c0+1][4q .. 4q+3]) for the lane's channels and quarter.
+// The expert of a token is uniform over the warp, so the load is one warp-wide tcgen05.ld per slot.
+template <int K, typename IO>
+__device__ __forceinline__ void load_a2_tm(const ChunkTile<IO>& ct, uint32_t tm_lane, int r, float4 (&a0)[K],
+                                          float4 (&a1)[K]) {
+  uint32_t v[K][8];
+#pragma unroll
+  for (int j = 0; j < K; ++j) sm100::tmem_ld8_nowait(tm_lane + (uint32_t)ct.e[r][j] * 8u, v[j]);
+  sm100::tmem_wait_ld();
+#pragma unroll
+  for (int j = 0; j < K; ++j) {
+    a0[j] = make_float4(__uint_as_float(v[j][0]), __uint_as_float(v[j][1]), __uint_as_float(v[j][2]),
+                        __uint_as_float(v[j][3]));
+    a1[j] = make_float4(__uint_as_float(v[j][4]), __uint_as_float(v[j][5]), __uint_as_float(v[j][6]),
+                        __uint_as_float(v[j][7]));
+  }
+}
+
 __device__ __forceinline__ float2 ld2(const float (&row)[kBwdCh], int c0) {
   return *reinterpret_cast<const float2*>(&row[c0]);
 }
@@ -471,7 +492,7 @@ __global__ void __launch_bounds__(kPkThreads) scan_bwd_ckpt_pk_kernel(ScanBwdPar
 // sub-block's states, transitions and dy are recomputed into registers from h_in (the state
 // before token i0), then walked backwards, updating `carry` (a_{t+1} λ_{t+1}).
 template <int K, typename IO>
-__device__ __forceinline__ void adjoint_sub_pk(const ScanBwdParams& p, const ChunkTile<IO>& ct, const float* As,
+__device__ __forceinline__ void adjoint_sub_pk(const ScanBwdParams& p, const ChunkTile<IO>& ct, uint32_t tm_lane,
                                                float* dAacc, float* red, int rw, int i0, int ni,
                                                const float2 (&h_in)[4], int64_t t0, int b, int d0, int c0,
                                                bool valid, float2 dsk, int tid, int warp, int lane, int q,
@@ -483,8 +504,10 @@ __device__ __forceinline__ void adjoint_sub_pk(const ScanBwdParams& p, const Chu
     for (int u = 0; u < kBwdSub; ++u) {
       if (u < ni) {
         const int i = i0 + u;
+        float4 a0[K], a1[K];
+        load_a2_tm<K>(ct, tm_lane, i, a0, a1);
         float2 at[4];
-        mix_a2<K>(ct, As, i, c0, q, at);
+        mix_a2<K>(ct, a0, a1, i, at);
         const float2 dl = ld2(ct.dl[i], c0), xv = ld2(ct.x[i], c0);
         const float2 c2 = __fmul2_rn(dl, f2s(kLog2e)), dx = __fmul2_rn(dl, xv);
 #pragma unroll
@@ -503,7 +526,7 @@ __device__ __forceinline__ void adjoint_sub_pk(const ScanBwdParams& p, const Chu
     if (u < ni) {
       const int i = i0 + u;
       float4 a0[K], a1[K];
-      load_a2<K>(ct, As, i, c0, q, a0, a1);
+      load_a2_tm<K>(ct, tm_lane, i, a0, a1);
       float2 at[4];
       mix_a2<K>(ct, a0, a1, i, at);
       const float2 dl = ld2(ct.dl[i], c0), xv = ld2(ct.x[i], c0);
@@ -599,15 +622,20 @@ __device__ __forceinline__ void adjoint_sub_pk(const ScanBwdParams& p, const Chu
   }
 }
 
+// Tensor-memory columns for the packed kernel's A rows: 8 per expert, rounded up to a power of two
+// of at least 32 (the allocation unit).
+__host__ __device__ constexpr uint32_t pk_tmem_cols(int E) { return E * 8 <= 32 ? 32u : (E * 8 <= 64 ? 64u : 128u); }
+
 // The chunk walk of the packed layout (same order as scan_bwd_kernel: the forward through each chunk
 // from its checkpoint, then the adjoint one sub-block at a time). Shared memory:
-// As[E][64][16] | dAacc[E][2][128 threads] float4 | sub[4][2][128 threads] float4 | red[4 warps][16][rw] |
-// tile (thread-fastest layouts: the 16-byte accesses are free of bank conflicts).
+// dAacc[E][2][128 threads] float4 | sub[4][2][128 threads] float4 | red[4 warps][16][rw] | tile
+// (thread-fastest layouts: the 16-byte accesses are free of bank conflicts); the A rows live in
+// tensor memory (load_a2_tm), so three CTAs fit on an SM.
 template <typename IO, int K>
-__global__ void __launch_bounds__(kPkThreads) scan_bwd_pk_kernel(ScanBwdParams p) {
+__global__ void __launch_bounds__(kPkThreads, 3) scan_bwd_pk_kernel(ScanBwdParams p) {
   extern __shared__ __align__(16) float smem_pk[];
-  float* As = smem_pk;
-  float* dAacc = As + p.E * kBwdCh * 16;
+  __shared__ uint32_t tm_slot;
+  float* dAacc = smem_pk;
   float4* sub = reinterpret_cast<float4*>(dAacc + p.E * kPkThreads * 8);
   float* red = reinterpret_cast<float*>(sub + (kBwdLc / kBwdSub) * kPkThreads * 2);
   const int rw = 2 * 16 + K;  // per token: dB[16], dC[16], dgates[K]
@@ -618,8 +646,30 @@ __global__ void __launch_bounds__(kPkThreads) scan_bwd_pk_kernel(ScanBwdParams p
   const int tile = blockIdx.x % tiles, b = blockIdx.x / tiles;
   const int d0 = tile * kBwdCh, nc = min(kBwdCh, p.D - d0);  // nc % 16 == 0
   const bool valid = 16 * warp < nc;                         // whole warps
-  load_a_rows(As, p.A, p.E, p.D, p.N, d0, nc);
+  // the A rows of every expert for the lane's channels and quarter in tensor memory (8 columns per
+  // expert), which keeps the shared memory of a CTA small enough for three CTAs per SM
+  const uint32_t tm_cols = pk_tmem_cols(p.E);
+  if (warp == 0) {
+    sm100::tmem_alloc(&tm_slot, tm_cols);
+    sm100::tmem_relinquish();
+  }
   for (int i = tid; i < p.E * kPkThreads * 8; i += kPkThreads) dAacc[i] = 0.f;
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tm_lane = tm_slot + ((uint32_t)(32 * warp) << 16);
+  for (int e = 0; e < p.E; ++e) {
+    float4 u0 = make_float4(0.f, 0.f, 0.f, 0.f), u1 = u0;
+    if (valid) {
+      const float* src = p.A + ((size_t)e * p.D + d0 + c0) * 16 + 4 * q;
+      u0 = __ldg(reinterpret_cast<const float4*>(src));
+      u1 = __ldg(reinterpret_cast<const float4*>(src + 16));
+    }
+    const uint32_t r[8] = {__float_as_uint(u0.x), __float_as_uint(u0.y), __float_as_uint(u0.z), __float_as_uint(u0.w),
+                           __float_as_uint(u1.x), __float_as_uint(u1.y), __float_as_uint(u1.z), __float_as_uint(u1.w)};
+    sm100::tmem_st8(tm_lane + (uint32_t)e * 8u, r);
+  }
+  sm100::tmem_wait_st();  // each warp reads back only what its own lanes wrote
   const float2 dsk = valid ? *reinterpret_cast<const float2*>(p.D_skip + d0 + c0) : make_float2(0.f, 0.f);
   float2 carry[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
   float2 dD = make_float2(0.f, 0.f);
@@ -651,8 +701,10 @@ __global__ void __launch_bounds__(kPkThreads) scan_bwd_pk_kernel(ScanBwdParams p
           sv[0] = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
           sv[kPkThreads] = make_float4(h[2].x, h[2].y, h[3].x, h[3].y);
         }
+        float4 a0[K], a1[K];
+        load_a2_tm<K>(ct, tm_lane, i, a0, a1);
         float2 at[4];
-        mix_a2<K>(ct, As, i, c0, q, at);
+        mix_a2<K>(ct, a0, a1, i, at);
         const float2 dl = ld2(ct.dl[i], c0), xv = ld2(ct.x[i], c0);
         const float2 c2 = __fmul2_rn(dl, f2s(kLog2e)), dx = __fmul2_rn(dl, xv);
         float2 y = make_float2(0.f, 0.f);
@@ -681,7 +733,7 @@ __global__ void __launch_bounds__(kPkThreads) scan_bwd_pk_kernel(ScanBwdParams p
         const float4 v0 = sv[0], v1 = sv[kPkThreads];
         const float2 h_in[4] = {make_float2(v0.x, v0.y), make_float2(v0.z, v0.w), make_float2(v1.x, v1.y),
                                 make_float2(v1.z, v1.w)};
-        adjoint_sub_pk<K>(p, ct, As, dAacc, red, rw, i0, ni, h_in, t0, b, d0, c0, valid, dsk, tid, warp, lane, q,
+        adjoint_sub_pk<K>(p, ct, tm_lane, dAacc, red, rw, i0, ni, h_in, t0, b, d0, c0, valid, dsk, tid, warp, lane, q,
                           carry, dD);
       }
     } else {
@@ -711,6 +763,12 @@ __global__ void __launch_bounds__(kPkThreads) scan_bwd_pk_kernel(ScanBwdParams p
       *reinterpret_cast<float4*>(dst + 16) = acc[kPkThreads];
     }
     if (q == 0) *reinterpret_cast<float2*>(p.part_D + (size_t)b * p.D + d0 + c0) = dD;
+  }
+  sm100::tc_fence_before();
+  __syncthreads();  // every warp's tensor-memory loads have completed (each waited for its own)
+  if (warp == 0) {
+    sm100::tc_fence_after();
+    sm100::tmem_dealloc(tm_slot, tm_cols);
   }
 }
 
@@ -800,8 +858,7 @@ cudaError_t run_scan_bwd(ScanBwdParams p, bool io_bf16, void* ws, cudaStream_t s
   cudaError_t e;
   // packed layout: N = 16, k <= 2, whole 16-channel warps
   const bool packed = p.N == 16 && (p.k == 1 || p.k == 2) && p.D % 16 == 0;
-  const size_t smem_pk = a_bytes +
-                         sizeof(float) * ((size_t)p.E * kPkThreads * 8 + (size_t)kPkWarps * kBwdLc * (32 + p.k)) +
+  const size_t smem_pk = sizeof(float) * ((size_t)p.E * kPkThreads * 8 + (size_t)kPkWarps * kBwdLc * (32 + p.k)) +
                          sizeof(float4) * (kBwdLc / kBwdSub) * kPkThreads * 2 + tile_bytes;
   if (packed) {
     if (io_bf16) {
