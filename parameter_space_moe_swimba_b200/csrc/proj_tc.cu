@@ -722,6 +722,7 @@ __global__ void __launch_bounds__(128) stage1_finish_kernel(const Stage1Params p
   auto sum8 = [&](int j, int c, float (&v)[8]) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = 0.f;
+#pragma unroll 8  // the splits' loads in flight together (split <= 8)
     for (int sp = 0; sp < p.split; ++sp) {
       const float* q = base + sp * item_stride + (size_t)(j * p.W + c) * BM;
 #pragma unroll
@@ -1249,8 +1250,8 @@ cudaError_t run_proj_pairs(const ProjParams& p, uint8_t* ws, cudaStream_t s) {
   q.C_mix = reinterpret_cast<float*>(ws + L.cv);
   cudaError_t e = run_tc<1>(q, ws, s, 1, 1);
   if (e != cudaSuccess) return e;
-  const int64_t total = p.T * (p.D / 4 + 8);
-  const unsigned grid = (unsigned)std::min<int64_t>((total + 255) / 256, 4 * (int64_t)num_sms());
+  const int64_t total = p.T * (p.D / 4 + 8);  // one item per thread: a single round of loads
+  const unsigned grid = (unsigned)std::min<int64_t>((total + 255) / 256, 1 << 20);
   if ((e = launch_pdl(pair_combine_kernel, dim3(grid), dim3(256), 0, s, q.delta, q.B_mix, q.C_mix, p.T, p.D, p.delta,
                       p.B_mix, p.C_mix)) != cudaSuccess)
     return e;
