@@ -289,6 +289,7 @@ swimba_status swimba_scan_bwd(const swimba_dims* dims, const void* x, const void
   p.N = dims->d_state;
   p.E = dims->n_experts;
   p.k = dims->top_k;
+  p.status = ws;
   return cuda_status(run_scan_bwd(p, dims->io_dtype == SWIMBA_BF16, static_cast<uint8_t*>(ws) + kStatusBytes,
                                   static_cast<cudaStream_t>(stream)));
 }

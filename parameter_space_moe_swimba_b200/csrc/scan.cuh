@@ -36,6 +36,9 @@ struct ScanPlan {
 };
 ScanPlan scan_fast_plan(int64_t B, int64_t L, int D, int N, int E, int k, bool io_bf16);
 cudaError_t run_scan_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s);
+// The recurrence alone over whole sequences from h0 (bf16 x, N = 16, k <= 2: the fast-path shapes),
+// writing the state at the start of every 16-token chunk into ckpt [B, nck, D, 16].
+cudaError_t run_scan_fast_ckpt(const ScanParams& sp, float* ckpt, int nck, void* status, cudaStream_t s);
 
 // Summary of a whole sequence (the hand-off of one piece of a longer one): h_zero [B, D, N] = the
 // end state from zero, log_decay [B, D, N] = Σ_t Δ_t A_t. The fast path stages per-segment
@@ -81,6 +84,7 @@ struct ScanBwdParams {
   float* part;           // [tiles, B, L, 2N + k]: per channel tile, dB | dC | dgates
   float* part_A;         // [B, E, D, N]
   float* part_D;         // [B, D]
+  void* status;          // the workspace's device status block (bounded waits that gave up)
   int64_t L;
   int B, D, N, E, k;
   int nck;

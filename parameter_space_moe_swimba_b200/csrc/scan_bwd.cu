@@ -815,16 +815,41 @@ cudaError_t launch_bwd_pair(const ScanBwdParams& p, unsigned grid, size_t smem_c
   return cudaGetLastError();
 }
 
+// The packed pair; fast_ckpt: the checkpoints come from the forward's fast scan (bf16 x), whose
+// chunk walk (TMA ring, A rows in tensor memory, one warp per 16 channels) runs the recurrence in
+// about half the time of scan_bwd_ckpt_pk_kernel.
 template <typename IO, int K>
-cudaError_t launch_bwd_pk(const ScanBwdParams& p, unsigned grid, size_t smem_ck, size_t smem_bw, cudaStream_t s) {
+cudaError_t launch_bwd_pk(const ScanBwdParams& p, unsigned grid, size_t smem_ck, size_t smem_bw, bool fast_ckpt,
+                          cudaStream_t s) {
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(scan_bwd_ckpt_pk_kernel<IO, K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem_ck)) != cudaSuccess)
-    return e;
+  if (fast_ckpt) {
+    ScanParams sp{};
+    sp.x = p.x;
+    sp.z = p.z;
+    sp.delta = p.delta;
+    sp.B_mix = p.B_mix;
+    sp.C_mix = p.C_mix;
+    sp.idx = p.idx;
+    sp.gates = p.gates;
+    sp.A = p.A;
+    sp.D_skip = p.D_skip;
+    sp.h0 = p.h0;
+    sp.L = p.L;
+    sp.B = p.B;
+    sp.D = p.D;
+    sp.N = p.N;
+    sp.E = p.E;
+    sp.k = p.k;
+    if ((e = run_scan_fast_ckpt(sp, p.ckpt, p.nck, p.status, s)) != cudaSuccess) return e;
+  } else {
+    if ((e = cudaFuncSetAttribute(scan_bwd_ckpt_pk_kernel<IO, K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem_ck)) != cudaSuccess)
+      return e;
+    scan_bwd_ckpt_pk_kernel<IO, K><<<grid, kPkThreads, smem_ck, s>>>(p);
+  }
   if ((e = cudaFuncSetAttribute(scan_bwd_pk_kernel<IO, K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)smem_bw)) != cudaSuccess)
     return e;
-  scan_bwd_ckpt_pk_kernel<IO, K><<<grid, kPkThreads, smem_ck, s>>>(p);
   scan_bwd_pk_kernel<IO, K><<<grid, kPkThreads, smem_bw, s>>>(p);
   return cudaGetLastError();
 }
@@ -860,13 +885,14 @@ cudaError_t run_scan_bwd(ScanBwdParams p, bool io_bf16, void* ws, cudaStream_t s
   const bool packed = p.N == 16 && (p.k == 1 || p.k == 2) && p.D % 16 == 0;
   const size_t smem_pk = sizeof(float) * ((size_t)p.E * kPkThreads * 8 + (size_t)kPkWarps * kBwdLc * (32 + p.k)) +
                          sizeof(float4) * (kBwdLc / kBwdSub) * kPkThreads * 2 + tile_bytes;
+  const bool fast_ckpt = packed && io_bf16 && scan_fast_plan(p.B, p.L, p.D, p.N, p.E, p.k, true).fast;
   if (packed) {
     if (io_bf16) {
-      e = p.k == 1 ? launch_bwd_pk<__nv_bfloat16, 1>(p, grid, smem_ck, smem_pk, s)
-                   : launch_bwd_pk<__nv_bfloat16, 2>(p, grid, smem_ck, smem_pk, s);
+      e = p.k == 1 ? launch_bwd_pk<__nv_bfloat16, 1>(p, grid, smem_ck, smem_pk, fast_ckpt, s)
+                   : launch_bwd_pk<__nv_bfloat16, 2>(p, grid, smem_ck, smem_pk, fast_ckpt, s);
     } else {
-      e = p.k == 1 ? launch_bwd_pk<float, 1>(p, grid, smem_ck, smem_pk, s)
-                   : launch_bwd_pk<float, 2>(p, grid, smem_ck, smem_pk, s);
+      e = p.k == 1 ? launch_bwd_pk<float, 1>(p, grid, smem_ck, smem_pk, false, s)
+                   : launch_bwd_pk<float, 2>(p, grid, smem_ck, smem_pk, false, s);
     }
   } else if (io_bf16) {
     if (p.k == 1) e = launch_bwd_pair<__nv_bfloat16, 1>(p, grid, smem_ck, smem_bw, s);
@@ -882,7 +908,7 @@ cudaError_t run_scan_bwd(ScanBwdParams p, bool io_bf16, void* ws, cudaStream_t s
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   scan_bwd_reduce_kernel<<<(unsigned)(4 * sms), 256, 0, s>>>(p, tiles);
-  note_launch(3);
+  note_launch(fast_ckpt ? 2 : 3);  // (the fast scan's checkpoint pass counts itself)
   return cudaGetLastError();
 }
 

@@ -200,6 +200,9 @@ struct FastParams {
   float* h_final;       // [B, D, 16] or null
   float* agg_h;         // pass 1: [B, S, D, 16] end state from zero
   float* agg_logp;      // pass 1: [B, S, D, 16] log2 of the decay product
+  float* ckpt;          // checkpoint pass (AGG kernel, one segment from h0): [B, nck, D, 16] the state at
+                        // the start of every 16-token chunk, or null
+  int nck;
   void* status;
   int64_t L, Lseg;
   int B, D, E, S;
@@ -320,7 +323,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
     float2 h[kSPL];
     {
       const float* hs = nullptr;
-      if (!AGG) {
+      if (!AGG || p.ckpt != nullptr) {
         if (p.h_seg != nullptr) hs = p.h_seg + (((size_t)b * p.S + seg) * p.D + dA) * 16;
         else if (p.h0 != nullptr && seg == 0) hs = p.h0 + ((size_t)b * p.D + dA) * 16;
       }
@@ -409,6 +412,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       const float4* bsm = reinterpret_cast<const float4*>(st + St::B);
       const float4* csm = reinterpret_cast<const float4*>(st + St::C);
       const int64_t t0 = t_begin + (int64_t)c * LC;
+      if (AGG && p.ckpt != nullptr) {  // the state before this chunk
+        float* ck = p.ckpt + (((size_t)b * p.nck + t0 / LC) * p.D + dA) * 16 + 4 * q;
+        *reinterpret_cast<float4*>(ck) = make_float4(h[0].x, h[1].x, h[2].x, h[3].x);
+        *reinterpret_cast<float4*>(ck + 16) = make_float4(h[0].y, h[1].y, h[2].y, h[3].y);
+      }
 
       // issue token t's loads (TMEM loads are waited for by the caller)
       auto load_tok = [&](TokIn& tk, int t) {
@@ -561,7 +569,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
     // end state (segment aggregates in pass 1, h_final after the last segment)
     float* hout = nullptr;
     float* lout = nullptr;
-    if (AGG) {
+    if (AGG && p.ckpt == nullptr) {
       hout = p.agg_h + (((size_t)b * p.S + seg) * p.D + dA) * 16;
       lout = p.agg_logp + (((size_t)b * p.S + seg) * p.D + dA) * 16;
     } else if (p.h_final != nullptr && seg == p.S - 1) {
@@ -822,6 +830,33 @@ static cudaError_t launch_summary(const ScanParams& sp, const ScanPlan& pl, void
                                                                        sp.D);
   note_launch();
   return cudaGetLastError();
+}
+
+// The checkpoint pass of the scan backward: the recurrence alone (no readout) over each whole
+// sequence from h0, writing the state at the start of every 16-token chunk into ckpt [B, nck, D, 16].
+template <int K>
+static cudaError_t launch_ckpt(const ScanParams& sp, float* ckpt, int nck, void* status, cudaStream_t s) {
+  const ScanPlan pl{true, 1, sp.L, 0};
+  FastLaunch f;
+  if (!fast_setup(sp, pl, status, f)) return cudaErrorInvalidValue;
+  FastParams a = f.p;
+  a.ckpt = ckpt;
+  a.nck = nck;
+  a.h_seg = nullptr;
+  auto kagg = pick_kernel<K, true>(a.E, f.zoh);
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(kagg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fast_smem(kMaxWarps))) !=
+      cudaSuccess)
+    return e;
+  int ctas, warps;
+  if ((e = fast_shape((const void*)kagg, a.units, f.sms, f.win, ctas, warps, a.tmem_cols)) != cudaSuccess) return e;
+  kagg<<<ctas, warps * 32, fast_smem(warps), s>>>(f.tx, f.tz, f.td, f.tb, f.tc, f.to, a);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t run_scan_fast_ckpt(const ScanParams& sp, float* ckpt, int nck, void* status, cudaStream_t s) {
+  return sp.k == 1 ? launch_ckpt<1>(sp, ckpt, nck, status, s) : launch_ckpt<2>(sp, ckpt, nck, status, s);
 }
 
 cudaError_t run_scan_fast(const ScanParams& sp, const ScanPlan& pl, void* seg_ws, void* status, cudaStream_t s) {
