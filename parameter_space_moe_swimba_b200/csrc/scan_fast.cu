@@ -48,26 +48,13 @@
 #include "scan.cuh"
 #include "sm100.cuh"
 
-// Tuning knobs, fixed at build time: the warps per SM the segment plan aims at, the warp count per
-// SM below which a sequence is split into segments, and how many of a lane's 8 exponentials per
-// token run as a polynomial on the FMA pipe instead of the special-function unit.
+// Tuning knobs, fixed at build time: the warps per SM the segment plan aims at, and the warp count
+// per SM below which a sequence is split into segments.
 #ifndef SWIMBA_SCAN_TARGET_WARPS
 #define SWIMBA_SCAN_TARGET_WARPS 14
 #endif
 #ifndef SWIMBA_SCAN_MIN_WARPS
 #define SWIMBA_SCAN_MIN_WARPS 8
-#endif
-#ifndef SWIMBA_SCAN_NPOLY
-#define SWIMBA_SCAN_NPOLY 0
-#endif
-// 1: the chunk's per-token expert columns and gates reach the lanes by warp shuffles from the
-// lanes that hold them, instead of a broadcast shared-memory load per token.
-#ifndef SWIMBA_SCAN_META_SHFL
-#define SWIMBA_SCAN_META_SHFL 0
-#endif
-// 1: with E <= 8 experts, keep the transition rows in registers instead of tensor memory.
-#ifndef SWIMBA_SCAN_AREG
-#define SWIMBA_SCAN_AREG 0
 #endif
 
 namespace swimba {
@@ -82,8 +69,6 @@ constexpr int kCPW = 16;          // channels per warp
 constexpr int kSPL = 4;           // states per lane and channel
 constexpr int kMaxWarps = 16;     // warps per CTA (128 registers per thread)
 constexpr int kPRow = 4 * kCPW + 4;  // floats per token row of the partial-readout buffer (padded)
-constexpr int kNPoly = SWIMBA_SCAN_NPOLY;
-static_assert(kNPoly >= 0 && kNPoly <= 8, "exponentials per lane and token");
 
 // Byte offsets inside one ring stage of one warp (TMA destinations, 128-byte aligned).
 struct Stage {
@@ -113,25 +98,6 @@ constexpr int kWarpBytes = kStages * Stage::BYTES + Epi::BYTES;
 // TMEM columns one warp needs (8 per expert, rounded up to the 32-column allocation granule).
 __host__ __device__ constexpr int tmem_cols_per_warp(int E) { return ((E * 8 + 31) / 32) * 32; }
 
-// 2^x on the FMA pipe for x <= 0: x = j + f with j = round(x) (the 1.5*2^23 shifter), f in
-// [-1/2, 1/2]; 2^f by a degree-5 polynomial fitted for minimax relative error on that interval
-// (fit_exp2_poly.py beside this file: float32 Horner error 2.4e-7, the size of ex2.approx's);
-// the exponent j is added to the result's exponent field. Inputs below -125 are clamped (result
-// 2^-125 instead of a flushed 0, which no decay product here can tell apart).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = __fadd_rn(x, 12582912.f);
-  const float j = __fadd_rn(t, -12582912.f);
-  const float f = __fadd_rn(x, -j);
-  float p = 0x1.5c08e6p-10f;
-  p = __fmaf_rn(p, f, 0x1.3d0c52p-7f);
-  p = __fmaf_rn(p, f, 0x1.c6b6e4p-5f);
-  p = __fmaf_rn(p, f, 0x1.ebf918p-3f);
-  p = __fmaf_rn(p, f, 0x1.62e428p-1f);
-  p = __fmaf_rn(p, f, 0x1.000002p+0f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -152,30 +118,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float2 v) {
 }
 
 __device__ __forceinline__ float2 f2(float v) { return make_float2(v, v); }
-
-// arg[s] (+)= dg * A^e[s] for the lane's 4 state pairs, with the E <= 8 experts' rows held in
-// registers: the expert is warp-uniform, so the switch is one uniform indexed branch, and every case
-// reads its own registers (a dynamically indexed register array would live in local memory).
-template <bool ACC>
-__device__ __forceinline__ void mix_areg(const float2 (&ar)[8][4], int e, float2 dg, float2 (&arg)[4]) {
-#define SWIMBA_MIX_CASE(c)                                                                   \
-  case c:                                                                                    \
-    _Pragma("unroll") for (int s = 0; s < 4; ++s) arg[s] =                                    \
-        ACC ? __ffma2_rn(dg, ar[c][s], arg[s]) : __fmul2_rn(dg, ar[c][s]);                     \
-    break;
-  switch (e) {
-    SWIMBA_MIX_CASE(0)
-    SWIMBA_MIX_CASE(1)
-    SWIMBA_MIX_CASE(2)
-    SWIMBA_MIX_CASE(3)
-    SWIMBA_MIX_CASE(4)
-    SWIMBA_MIX_CASE(5)
-    SWIMBA_MIX_CASE(6)
-    default:
-      SWIMBA_MIX_CASE(7)
-  }
-#undef SWIMBA_MIX_CASE
-}
 
 // One token's scan inputs as the recurrence pass holds them (lane view: channels c0, c1 as the two
 // halves of every float2; states 4q .. 4q+3).
@@ -211,10 +153,10 @@ struct FastParams {
   int tmem_cols;        // TMEM columns the CTA allocates
 };
 
-// AGG = true: pass 1 (segments 0 .. S-2 only; no readout, no output). AREG = true: the experts'
-// transition rows in registers (E <= 8) instead of tensor memory. ZOH = true: zero-order-hold
-// injection (φ Δ B x, φ = (ā - 1) / (Δ A_t)) instead of Euler's Δ B x.
-template <int K, int NPOLY, bool AGG, bool AREG, bool ZOH>
+// AGG = true: pass 1 (segments 0 .. S-2 only; no readout, no output), or the checkpoint pass of the
+// backward (p.ckpt set). ZOH = true: zero-order-hold injection (φ Δ B x, φ = (ā - 1) / (Δ A_t))
+// instead of Euler's Δ B x.
+template <int K, bool AGG, bool ZOH>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1)
     scan_fast_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
                      const __grid_constant__ CUtensorMap tm_dl, const __grid_constant__ CUtensorMap tm_b,
@@ -248,22 +190,26 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       }
     }
   }
-  if (!AREG && warp == 0) {
+  if (warp == 0) {
     tmem_alloc(tmem_slot, (uint32_t)p.tmem_cols);
     tmem_relinquish();
   }
   __syncthreads();
   tc_fence_after();
   // this warp's TMEM window: its lane quarter, tmem_cols_per_warp(E) columns
-  const uint32_t tbase = AREG ? 0u
-                              : *tmem_slot + ((uint32_t)(32 * (warp & 3)) << 16) +
-                                    (uint32_t)(warp >> 2) * (uint32_t)tmem_cols_per_warp(p.E);
-  float2 areg[8][4];  // AREG: the experts' rows (x log2 e), (c0, c1) per state
+  const uint32_t tbase =
+      *tmem_slot + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(warp >> 2) * (uint32_t)tmem_cols_per_warp(p.E);
 
   const int cp = lane >> 2;        // recurrence pass: channel pair 2cp, 2cp+1 of the warp's 16
   const int q = lane & 3;          //                  state quarter: states 4q .. 4q+3
-  const int rt = lane >> 1;        // readout pass: token rt of the chunk,
-  const int rc = (lane & 1) * 8;   //               channels rc .. rc+7 of the warp's 16
+  // readout pass: lane = (token rt of the chunk, channels rc .. rc+7 of the warp's 16); the eight
+  // lanes of a 16-byte load phase take eight consecutive tokens of one channel half, so their reads
+  // of the partial-readout rows (stride 68 floats) fall in eight distinct bank groups (with the two
+  // halves of one token in a phase they collided two by two: 10 % of the kernel's shared-memory
+  // wavefronts); the x, z and output tile rows (32 bytes) then conflict two ways instead, for a
+  // quarter of those wavefronts
+  const int rt = lane & 15;
+  const int rc = (lane >> 4) * 8;
   const int ntiles = p.D / kCPW;
   const int u_begin = (int)((int64_t)p.units * blockIdx.x / gridDim.x);
   const int u_end = (int)((int64_t)p.units * (blockIdx.x + 1) / gridDim.x);
@@ -284,22 +230,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
     const int nchunks = (int)((t_end - t_begin + LC - 1) / LC);
 
     // per-expert transition rows of this lane's 2 channels x 4 states, times log2(e), into TMEM
-    // columns 8e + 2s + channel (or into registers)
-    if (AREG) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
-        if (e < p.E) {
-          a0 = __ldg(reinterpret_cast<const float4*>(p.A + ((size_t)e * p.D + dA) * 16 + 4 * q));
-          a1 = __ldg(reinterpret_cast<const float4*>(p.A + ((size_t)e * p.D + dA + 1) * 16 + 4 * q));
-        }
-        areg[e][0] = make_float2(a0.x * kLog2e, a1.x * kLog2e);
-        areg[e][1] = make_float2(a0.y * kLog2e, a1.y * kLog2e);
-        areg[e][2] = make_float2(a0.z * kLog2e, a1.z * kLog2e);
-        areg[e][3] = make_float2(a0.w * kLog2e, a1.w * kLog2e);
-      }
-    }
-    for (int e = 0; e < (AREG ? 0 : p.E); ++e) {
+    // columns 8e + 2s + channel (a copy of the rows in registers behind a warp-uniform switch ran
+    // the Mamba-1.4B-like scan in 1627 against 961 µs: spills and branches)
+    for (int e = 0; e < p.E; ++e) {
       const float4 a0 = __ldg(reinterpret_cast<const float4*>(p.A + ((size_t)e * p.D + dA) * 16 + 4 * q));
       const float4 a1 = __ldg(reinterpret_cast<const float4*>(p.A + ((size_t)e * p.D + dA + 1) * 16 + 4 * q));
       const uint32_t r[8] = {__float_as_uint(a0.x * kLog2e), __float_as_uint(a1.x * kLog2e),
@@ -308,7 +241,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
                              __float_as_uint(a0.w * kLog2e), __float_as_uint(a1.w * kLog2e)};
       tmem_st8(tbase + (uint32_t)(e * 8), r);
     }
-    if (!AREG) tmem_wait_st();
+    tmem_wait_st();
     float2 dsk[4];  // readout pass: D_skip of channels rc .. rc+7
     if (!AGG) {
       const float4 d0 = __ldg(reinterpret_cast<const float4*>(p.D_skip + tile * kCPW + rc));
@@ -350,10 +283,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       const int64_t t = t_begin + (int64_t)c * LC + lane;
       if (lane < LC && c < nchunks && t < t_end) {
         const size_t tok = (size_t)b * p.L + t;
-        m.x = (int)(min((uint32_t)__ldg(p.idx + tok * K), emax) * (AREG ? 1u : 8u));
+        m.x = (int)(min((uint32_t)__ldg(p.idx + tok * K), emax) * 8u);
         m.z = __float_as_int(__ldg(p.gates + tok * K));
         if (K == 2) {
-          m.y = (int)(min((uint32_t)__ldg(p.idx + tok * K + 1), emax) * (AREG ? 1u : 8u));
+          m.y = (int)(min((uint32_t)__ldg(p.idx + tok * K + 1), emax) * 8u);
           m.w = __float_as_int(__ldg(p.gates + tok * K + 1));
         }
       }
@@ -399,14 +332,6 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       phase_bits ^= 1u << sidx;
       const uint8_t* st = ring + sidx * St::BYTES;
       const int4* meta = reinterpret_cast<const int4*>(st + St::META);
-#if SWIMBA_SCAN_META_SHFL
-      // lane t < 16 holds token t's {columns packed, g0, g1}
-      int3 mreg = make_int3(0, 0, 0);
-      if (lane < LC) {
-        const int4 mm = meta[lane];
-        mreg = make_int3(mm.x | (mm.y << 16), mm.z, mm.w);
-      }
-#endif
       const uint32_t* xs2 = reinterpret_cast<const uint32_t*>(st + St::X);
       const float2* ds2 = reinterpret_cast<const float2*>(st + St::DL);
       const float4* bsm = reinterpret_cast<const float4*>(st + St::B);
@@ -420,19 +345,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
 
       // issue token t's loads (TMEM loads are waited for by the caller)
       auto load_tok = [&](TokIn& tk, int t) {
-#if SWIMBA_SCAN_META_SHFL
-        {
-          const int c01 = __shfl_sync(0xffffffffu, mreg.x, t);
-          tk.m = make_int4(c01 & 0xffff, c01 >> 16, __shfl_sync(0xffffffffu, mreg.y, t),
-                           __shfl_sync(0xffffffffu, mreg.z, t));
-        }
-#else
-        tk.m = meta[t];
-#endif
-        if (!AREG) {
-          tmem_ld8_nowait(tbase + (uint32_t)tk.m.x, tk.ar[0]);
-          if (K == 2) tmem_ld8_nowait(tbase + (uint32_t)tk.m.y, tk.ar[1]);
-        }
+        tk.m = meta[t];  // (handing it over by warp shuffles from the lanes that load it ran slower)
+        tmem_ld8_nowait(tbase + (uint32_t)tk.m.x, tk.ar[0]);
+        if (K == 2) tmem_ld8_nowait(tbase + (uint32_t)tk.m.y, tk.ar[1]);
         tk.dl = ds2[t * (kCPW / 2) + cp];
         const uint32_t xw = xs2[t * (kCPW / 2) + cp];
         tk.xv = make_float2(bf16lo(xw), bf16hi(xw));
@@ -444,26 +359,18 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
         tk.dx = __fmul2_rn(tk.dl, tk.xv);
         const float2 dg0 = __fmul2_rn(tk.dl, f2(__int_as_float(tk.m.z)));
         const float2 dg1 = __fmul2_rn(tk.dl, f2(__int_as_float(tk.m.w)));
-        float2 args[kSPL];
-        if (AREG) {
-          mix_areg<false>(areg, tk.m.x, dg0, args);
-          if (K == 2) mix_areg<true>(areg, tk.m.y, dg1, args);
-        }
 #pragma unroll
         for (int s = 0; s < kSPL; ++s) {
-          float2 arg;
-          if (AREG) {
-            arg = args[s];
-          } else {
-            arg = __fmul2_rn(dg0, make_float2(__uint_as_float(tk.ar[0][2 * s]), __uint_as_float(tk.ar[0][2 * s + 1])));
-            if (K == 2)
-              arg = __ffma2_rn(dg1, make_float2(__uint_as_float(tk.ar[1][2 * s]), __uint_as_float(tk.ar[1][2 * s + 1])),
-                               arg);
-          }
+          float2 arg =
+              __fmul2_rn(dg0, make_float2(__uint_as_float(tk.ar[0][2 * s]), __uint_as_float(tk.ar[0][2 * s + 1])));
+          if (K == 2)
+            arg = __ffma2_rn(dg1, make_float2(__uint_as_float(tk.ar[1][2 * s]), __uint_as_float(tk.ar[1][2 * s + 1])),
+                             arg);
           if (AGG) lsum[s] = __fadd2_rn(lsum[s], arg);  // Σ_t log2 ā_t
-          // elements 2s, 2s+1 of the lane's 8; the last NPOLY of them go to the FMA pipe
-          const float ax = (2 * s >= 8 - NPOLY) ? exp2_poly(arg.x) : ex2_approx(arg.x);
-          const float ay = (2 * s + 1 >= 8 - NPOLY) ? exp2_poly(arg.y) : ex2_approx(arg.y);
+          // every exponential on the special-function unit (moving one per lane and token to a
+          // polynomial on the FMA pipe ran slower: 1029 against 961 µs)
+          const float ax = ex2_approx(arg.x);
+          const float ay = ex2_approx(arg.y);
           tk.a[s] = make_float2(ax, ay);
           if (ZOH) tk.phi[s] = make_float2(zoh_phi(arg.x, ax), zoh_phi(arg.y, ay));
         }
@@ -474,7 +381,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       // loaded (its A rows from TMEM, Δ, x, B, C from the ring) and its decay factors computed.
       TokIn cur, nxt;
       load_tok(cur, 0);
-      if (!AREG) tmem_wait_ld();
+      tmem_wait_ld();
       decay(cur);
 #pragma unroll
       for (int t = 0; t < LC; ++t) {
@@ -494,7 +401,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
           *reinterpret_cast<float2*>(psm + t * kPRow + cp * 8 + q * 2) = y;
         }
         if (t + 1 < LC) {
-          if (!AREG) tmem_wait_ld();
+          tmem_wait_ld();
           decay(nxt);
           cur = nxt;
         }
@@ -588,7 +495,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
   // the output stores must have read their shared-memory tiles before the CTA's memory goes away
   if (!AGG && lane == 0) bulk_wait<0>();
   __syncthreads();
-  if (!AREG && warp == 0) {
+  if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(*tmem_slot, (uint32_t)p.tmem_cols);
   }
@@ -697,11 +604,8 @@ using FastKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensor
 
 template <int K, bool AGG>
 static FastKernel pick_kernel(int E, bool zoh) {
-#if SWIMBA_SCAN_AREG
-  if (E <= 8) return zoh ? scan_fast_kernel<K, kNPoly, AGG, true, true> : scan_fast_kernel<K, kNPoly, AGG, true, false>;
-#endif
   (void)E;
-  return zoh ? scan_fast_kernel<K, kNPoly, AGG, false, true> : scan_fast_kernel<K, kNPoly, AGG, false, false>;
+  return zoh ? scan_fast_kernel<K, AGG, true> : scan_fast_kernel<K, AGG, false>;
 }
 
 struct FastLaunch {
