@@ -27,7 +27,8 @@
 //           order, so the result does not depend on scheduling.
 // Shapes: N <= 16, any k <= E <= 16, io fp32 or bf16. For N = 16, k <= 2 and D % 16 == 0 the bwd
 // kernel runs in a packed layout (two channels per lane, f32x2 arithmetic, the A rows in tensor
-// memory; scan_bwd_pk_kernel).
+// memory; scan_bwd_pk_kernel), and with bf16 io the checkpoints come from the forward's fast scan
+// (its recurrence-only pass in checkpoint mode, run_scan_fast_ckpt) instead of the ckpt kernel.
 #include "common.cuh"
 #include "scan.cuh"
 #include "sm100.cuh"
