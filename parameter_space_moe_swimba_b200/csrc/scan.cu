@@ -273,15 +273,17 @@ cudaError_t run_scan_chain(int64_t BDN, int P, const float* h_zero, const float*
 // owns a tile of 64 channels and a group of sequences: it stages the A rows of ALL E experts for
 // its channels in shared memory once (E x 4 KB, read from L2 once per CTA instead of once per
 // sequence), then streams its sequences past them. Thread i owns (channel i / 4, state quarter
-// i % 4); it puts four sequences' state quarters, Δ, x, z, B/C quarters and experts in flight
+// i % 4); it puts two sequences' state quarters, Δ, x, z, B/C quarters and experts in flight
 // before it computes any of them, and the four quarters of a channel reduce the readout with two
-// shuffles. The grid is one wave: tiles x groups <= the CTAs the SMs hold at once (three per SM at
-// 80 registers a thread), so no CTA waits for a second wave.
+// shuffles. Two sequences per thread at four CTAs per SM (60 registers) keep more warps in flight
+// than four sequences at three CTAs (80 registers): 35.5 against 40.8 µs for 256 sequences in a
+// timing probe of the same loop. The grid is one wave: tiles x groups <= the CTAs the SMs hold
+// at once, so no CTA waits for a second wave.
 constexpr int kStepCh = 64;  // channels per CTA
-constexpr int kStepU = 4;    // sequences in flight per thread
+constexpr int kStepU = 2;    // sequences in flight per thread
 
 template <typename IO, int K>
-__global__ void __launch_bounds__(256, 3) step_stream_kernel(ScanParams p, int seq_per_cta) {
+__global__ void __launch_bounds__(256, 4) step_stream_kernel(ScanParams p, int seq_per_cta) {
   extern __shared__ float4 a_rows[];  // [E][kStepCh][4] float4 = the E experts' A rows of the tile
   const int tid = threadIdx.x, c = tid >> 2, q = tid & 3;
   const int tiles = (p.D + kStepCh - 1) / kStepCh;
