@@ -224,6 +224,10 @@ EDGE = [
     # the SIMT tile router for more than 2048 tokens (E % 4 != 0; fp32 x)
     (1, 2100, 96, 16, 8, 6, 3, "bf16", "f32"),
     (1, 2100, 40, 5, 3, 3, 3, "f32", "f32"),
+    # k = 2 with at most 1024 tokens runs the projection on (token, slot) pairs bucketed by single
+    # expert: both sides of that limit
+    (1, 1024, 64, 16, 16, 4, 2, "bf16", "bf16"),
+    (1, 1025, 64, 16, 16, 4, 2, "bf16", "bf16"),
     # the one-CTA bucketing of the tensor-core projection covers up to 4096 tokens: both sides of it
     (2, 2048, 64, 16, 16, 4, 2, "bf16", "bf16"),
     (1, 4097, 64, 16, 16, 8, 1, "bf16", "bf16"),
