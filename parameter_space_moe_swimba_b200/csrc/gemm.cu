@@ -240,26 +240,52 @@ __global__ void __launch_bounds__(192, 1)
         const int n = n0 + cb * 32;
         if (m < p.M && n < p.N) {
           const int mo = (F32OUT && p.rows != nullptr) ? p.rows[m] / p.rows_div : m;
+          // the residual's 32 values of this slice are loaded before any of the slice is stored:
+          // the residual may be the output itself (an in-place accumulation), so the compiler may
+          // not move a load above an earlier store, and loads interleaved with stores would make
+          // one memory round trip per 8 columns
+          float rr[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) rr[e] = 0.f;
+          if (p.R != nullptr) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              const int col = n + j;
+              if (col < p.N) {
+                if (F32OUT) {
+                  const float4* r4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.R) +
+                                                                     (size_t)mo * p.ldr + col);
+                  const float4 r0 = r4[0], r1 = r4[1];
+                  rr[j] = r0.x;
+                  rr[j + 1] = r0.y;
+                  rr[j + 2] = r0.z;
+                  rr[j + 3] = r0.w;
+                  rr[j + 4] = r1.x;
+                  rr[j + 5] = r1.y;
+                  rr[j + 6] = r1.z;
+                  rr[j + 7] = r1.w;
+                } else {
+                  const uint4 w = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.R) +
+                                                                  (size_t)m * p.ldr + col);
+                  rr[j] = bf16lo(w.x);
+                  rr[j + 1] = bf16hi(w.x);
+                  rr[j + 2] = bf16lo(w.y);
+                  rr[j + 3] = bf16hi(w.y);
+                  rr[j + 4] = bf16lo(w.z);
+                  rr[j + 5] = bf16hi(w.z);
+                  rr[j + 6] = bf16lo(w.w);
+                  rr[j + 7] = bf16hi(w.w);
+                }
+              }
+            }
+          }
 #pragma unroll
           for (int j = 0; j < 32; j += 8) {  // groups of 8 columns (N and split are multiples of 8)
             const int col = n + j;
             if (col < p.N && F32OUT) {
               float o[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) o[e] = v[j + e];
-              if (p.R != nullptr) {
-                const float4* r4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.R) +
-                                                                   (size_t)mo * p.ldr + col);
-                const float4 r0 = r4[0], r1 = r4[1];
-                o[0] += r0.x;
-                o[1] += r0.y;
-                o[2] += r0.z;
-                o[3] += r0.w;
-                o[4] += r1.x;
-                o[5] += r1.y;
-                o[6] += r1.z;
-                o[7] += r1.w;
-              }
+              for (int e = 0; e < 8; ++e) o[e] = p.R != nullptr ? v[j + e] + rr[j + e] : v[j + e];
               float* out = col < p.split ? reinterpret_cast<float*>(p.C0) + (size_t)mo * p.ldc0 + col
                                          : reinterpret_cast<float*>(p.C1) + (size_t)mo * p.ldc1 + (col - p.split);
               reinterpret_cast<float4*>(out)[0] = make_float4(o[0], o[1], o[2], o[3]);
@@ -267,19 +293,7 @@ __global__ void __launch_bounds__(192, 1)
             } else if (col < p.N) {
               float o[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) o[e] = v[j + e];
-              if (p.R != nullptr) {
-                const uint4 w = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.R) +
-                                                                (size_t)m * p.ldr + col);
-                o[0] += bf16lo(w.x);
-                o[1] += bf16hi(w.x);
-                o[2] += bf16lo(w.y);
-                o[3] += bf16hi(w.y);
-                o[4] += bf16lo(w.z);
-                o[5] += bf16hi(w.z);
-                o[6] += bf16lo(w.w);
-                o[7] += bf16hi(w.w);
-              }
+              for (int e = 0; e < 8; ++e) o[e] = p.R != nullptr ? v[j + e] + rr[j + e] : v[j + e];
               __nv_bfloat16* out = col < p.split
                                        ? reinterpret_cast<__nv_bfloat16*>(p.C0) + (size_t)m * p.ldc0 + col
                                        : reinterpret_cast<__nv_bfloat16*>(p.C1) + (size_t)m * p.ldc1 + (col - p.split);
