@@ -234,51 +234,56 @@ __global__ void __launch_bounds__(192, 1)
       // that a warp instruction covers one row was timed slower: 987 against 500 µs for the
       // out-projection with its residual, 9.8 against 2.8 ms for the projection backward.)
       const int m = m0 + 32 * q + lane;
+      const int mo = (F32OUT && p.rows != nullptr && m < p.M) ? p.rows[m] / p.rows_div : m;
+      // The residual's 32 values of a slice are loaded one slice ahead, before the current slice is
+      // stored: the residual may be the output itself (an in-place accumulation), so the compiler
+      // may not move a load above an earlier store, and loads interleaved with the stores made one
+      // memory round trip per 8 columns.
+      auto load_r = [&](int cb, float (&r)[32]) {
+        const int n = n0 + cb * 32;
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+          const int col = n + j;
+          if (p.R != nullptr && m < p.M && col < p.N) {
+            if (F32OUT) {
+              const float4* r4 =
+                  reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.R) + (size_t)mo * p.ldr + col);
+              const float4 r0 = r4[0], r1 = r4[1];
+              r[j] = r0.x;
+              r[j + 1] = r0.y;
+              r[j + 2] = r0.z;
+              r[j + 3] = r0.w;
+              r[j + 4] = r1.x;
+              r[j + 5] = r1.y;
+              r[j + 6] = r1.z;
+              r[j + 7] = r1.w;
+            } else {
+              const uint4 w = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.R) +
+                                                              (size_t)m * p.ldr + col);
+              r[j] = bf16lo(w.x);
+              r[j + 1] = bf16hi(w.x);
+              r[j + 2] = bf16lo(w.y);
+              r[j + 3] = bf16hi(w.y);
+              r[j + 4] = bf16lo(w.z);
+              r[j + 5] = bf16hi(w.z);
+              r[j + 6] = bf16lo(w.w);
+              r[j + 7] = bf16hi(w.w);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) r[j + e] = 0.f;
+          }
+        }
+      };
+      float rr[32], rn[32];
+      load_r(0, rr);
+#pragma unroll
       for (int cb = 0; cb < GBN / 32; ++cb) {
+        if (cb + 1 < GBN / 32) load_r(cb + 1, rn);
         float v[32];
         tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + buf * GBN + cb * 32, v);
         const int n = n0 + cb * 32;
         if (m < p.M && n < p.N) {
-          const int mo = (F32OUT && p.rows != nullptr) ? p.rows[m] / p.rows_div : m;
-          // the residual's 32 values of this slice are loaded before any of the slice is stored:
-          // the residual may be the output itself (an in-place accumulation), so the compiler may
-          // not move a load above an earlier store, and loads interleaved with stores would make
-          // one memory round trip per 8 columns
-          float rr[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) rr[e] = 0.f;
-          if (p.R != nullptr) {
-#pragma unroll
-            for (int j = 0; j < 32; j += 8) {
-              const int col = n + j;
-              if (col < p.N) {
-                if (F32OUT) {
-                  const float4* r4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.R) +
-                                                                     (size_t)mo * p.ldr + col);
-                  const float4 r0 = r4[0], r1 = r4[1];
-                  rr[j] = r0.x;
-                  rr[j + 1] = r0.y;
-                  rr[j + 2] = r0.z;
-                  rr[j + 3] = r0.w;
-                  rr[j + 4] = r1.x;
-                  rr[j + 5] = r1.y;
-                  rr[j + 6] = r1.z;
-                  rr[j + 7] = r1.w;
-                } else {
-                  const uint4 w = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.R) +
-                                                                  (size_t)m * p.ldr + col);
-                  rr[j] = bf16lo(w.x);
-                  rr[j + 1] = bf16hi(w.x);
-                  rr[j + 2] = bf16lo(w.y);
-                  rr[j + 3] = bf16hi(w.y);
-                  rr[j + 4] = bf16lo(w.z);
-                  rr[j + 5] = bf16hi(w.z);
-                  rr[j + 6] = bf16lo(w.w);
-                  rr[j + 7] = bf16hi(w.w);
-                }
-              }
-            }
-          }
 #pragma unroll
           for (int j = 0; j < 32; j += 8) {  // groups of 8 columns (N and split are multiples of 8)
             const int col = n + j;
@@ -302,6 +307,8 @@ __global__ void __launch_bounds__(192, 1)
             }
           }
         }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) rr[e] = rn[e];
       }
       tc_fence_before();
       __syncwarp();
