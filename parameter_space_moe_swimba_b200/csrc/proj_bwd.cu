@@ -244,11 +244,31 @@ __global__ void __launch_bounds__(256) route_bwd_dx_kernel(const float* W_r, con
   for (int e = 0; e < kMaxE; ++e) w[e] = (d < D && e < E) ? W_r[(size_t)d * E + e] : 0.f;
   __syncthreads();
   if (d >= D) return;
-  for (int r = 0; r < nt; ++r) {
-    float acc = accumulate ? dx[(t0 + r) * D + d] : 0.f;
+  // dx is read and written in place, so the compiler may not move a load above an earlier store
+  // (one memory round trip per row otherwise): rows go in batches of 8, the next batch's values
+  // loaded before the current one is stored
+  constexpr int kB = 8;
+  float a[kB], an[kB];
 #pragma unroll
-    for (int e = 0; e < kMaxE; ++e) acc = fmaf(dl[r][e], w[e], acc);
-    dx[(t0 + r) * D + d] = acc;
+  for (int i = 0; i < kB; ++i) a[i] = (accumulate && i < nt) ? dx[(t0 + i) * D + d] : 0.f;
+  for (int r0 = 0; r0 < nt; r0 += kB) {
+#pragma unroll
+    for (int i = 0; i < kB; ++i) {
+      const int r = r0 + kB + i;
+      an[i] = (accumulate && r < nt) ? dx[(t0 + r) * D + d] : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < kB; ++i) {
+      const int r = r0 + i;
+      if (r < nt) {
+        float acc = a[i];
+#pragma unroll
+        for (int e = 0; e < kMaxE; ++e) acc = fmaf(dl[r][e], w[e], acc);
+        dx[(t0 + r) * D + d] = acc;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kB; ++i) a[i] = an[i];
   }
 }
 
