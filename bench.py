@@ -580,7 +580,9 @@ def report_bwd(torch, S, cfg, peaks, flush, reps, warmup):
     P = T * k
     W = R + 2 * N
     proj_flops = 2 * P * (D * W + D * R + W * D + D * W + (R + 8) * D)
-    exps = 3 * T * D * N  # the checkpoint pass, the recompute and the adjoint each take one exp2 per state
+    # one exp2 per state element in each of: the checkpoint pass, the forward through each chunk, the
+    # sub-block recompute and the adjoint
+    exps = 4 * T * D * N
     mufu_peak = 16 * 148 * peaks["sm_max_mhz"] * 1e6
     return {
         "report": "backward", "workload": cfg.name, "tokens": T, "layer_bwd_us": 1e3 * tot,

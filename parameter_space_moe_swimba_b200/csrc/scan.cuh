@@ -84,6 +84,7 @@ struct ScanBwdParams {
   float* part;           // [tiles, B, L, 2N + k]: per channel tile, dB | dC | dgates
   float* part_A;         // [B, E, D, N]
   float* part_D;         // [B, D]
+  float* sub;            // [tiles * B, 4, 2, 128] float4: the packed kernel's sub-block states
   void* status;          // the workspace's device status block (bounded waits that gave up)
   int64_t L;
   int B, D, N, E, k;

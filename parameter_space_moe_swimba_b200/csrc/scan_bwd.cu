@@ -27,8 +27,10 @@
 //           order, so the result does not depend on scheduling.
 // Shapes: N <= 16, any k <= E <= 16, io fp32 or bf16. For N = 16, k <= 2 and D % 16 == 0 the bwd
 // kernel runs in a packed layout (two channels per lane, f32x2 arithmetic, the A rows in tensor
-// memory; scan_bwd_pk_kernel), and with bf16 io the checkpoints come from the forward's fast scan
-// (its recurrence-only pass in checkpoint mode, run_scan_fast_ckpt) instead of the ckpt kernel.
+// memory, the sub-block states in an L2-resident global scratch and the adjoint's exponentials
+// recomputed rather than kept, so four CTAs fit on an SM; scan_bwd_pk_kernel), and with bf16 io the
+// checkpoints come from the forward's fast scan (its recurrence-only pass in checkpoint mode,
+// run_scan_fast_ckpt) instead of the ckpt kernel.
 #include "common.cuh"
 #include "scan.cuh"
 #include "sm100.cuh"
@@ -498,7 +500,7 @@ __device__ __forceinline__ void adjoint_sub_pk(const ScanBwdParams& p, const Chu
                                                const float2 (&h_in)[4], int64_t t0, int b, int d0, int c0,
                                                bool valid, float2 dsk, int tid, int warp, int lane, int q,
                                                float2 (&carry)[4], float2& dD) {
-  float2 H[kBwdSub][4], AB[kBwdSub][4], DY[kBwdSub];
+  float2 H[kBwdSub][4], DY[kBwdSub];
   {
     float2 h[4] = {h_in[0], h_in[1], h_in[2], h_in[3]};
 #pragma unroll
@@ -513,8 +515,7 @@ __device__ __forceinline__ void adjoint_sub_pk(const ScanBwdParams& p, const Chu
         const float2 c2 = __fmul2_rn(dl, f2s(kLog2e)), dx = __fmul2_rn(dl, xv);
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
-          AB[u][s] = ex2_2(__fmul2_rn(c2, at[s]));
-          h[s] = __ffma2_rn(AB[u][s], h[s], __fmul2_rn(dx, f2s(ct.B[i][4 * q + s])));
+          h[s] = __ffma2_rn(ex2_2(__fmul2_rn(c2, at[s])), h[s], __fmul2_rn(dx, f2s(ct.B[i][4 * q + s])));
           H[u][s] = h[s];
         }
         const float2 zv = ld2(ct.z[i], c0), go = ld2(ct.go[i], c0);
@@ -531,20 +532,21 @@ __device__ __forceinline__ void adjoint_sub_pk(const ScanBwdParams& p, const Chu
       float2 at[4];
       mix_a2<K>(ct, a0, a1, i, at);
       const float2 dl = ld2(ct.dl[i], c0), xv = ld2(ct.x[i], c0);
-      const float2 dlx = __fmul2_rn(dl, xv);
+      const float2 dlx = __fmul2_rn(dl, xv), c2 = __fmul2_rn(dl, f2s(kLog2e));
       float2 dA[4], sum_b = make_float2(0.f, 0.f), sum_d = make_float2(0.f, 0.f);
       float vB[4], vC[4];
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
         const float2 hp = u > 0 ? H[u > 0 ? u - 1 : 0][s] : h_in[s];
         const float2 lam = __ffma2_rn(f2s(ct.C[i][4 * q + s]), DY[u], carry[s]);
-        const float2 ahp = __fmul2_rn(AB[u][s], hp);
+        const float2 ab = ex2_2(__fmul2_rn(c2, at[s]));  // recomputed: not kept from the forward above
+        const float2 ahp = __fmul2_rn(ab, hp);
         dA[s] = __fmul2_rn(__fmul2_rn(lam, dl), ahp);
         sum_b = __ffma2_rn(lam, f2s(ct.B[i][4 * q + s]), sum_b);
         sum_d = __ffma2_rn(__fmul2_rn(lam, at[s]), ahp, sum_d);
         vB[s] = fmaf(lam.x, dlx.x, lam.y * dlx.y);               // this lane's 2 channels
         vC[s] = fmaf(DY[u].x, H[u][s].x, DY[u].y * H[u][s].y);
-        carry[s] = __fmul2_rn(AB[u][s], lam);
+        carry[s] = __fmul2_rn(ab, lam);
       }
       // dx, dΔ: sums over the channel's 4 state quarters
 #pragma unroll
@@ -629,16 +631,21 @@ __host__ __device__ constexpr uint32_t pk_tmem_cols(int E) { return E * 8 <= 32 
 
 // The chunk walk of the packed layout (same order as scan_bwd_kernel: the forward through each chunk
 // from its checkpoint, then the adjoint one sub-block at a time). Shared memory:
-// dAacc[E][2][128 threads] float4 | sub[4][2][128 threads] float4 | red[4 warps][16][rw] | tile
-// (thread-fastest layouts: the 16-byte accesses are free of bank conflicts); the A rows live in
-// tensor memory (load_a2_tm), so three CTAs fit on an SM.
+// dAacc[E][2][128 threads] float4 | red[4 warps][16][rw] | tile (thread-fastest layouts: the
+// 16-byte accesses are free of bank conflicts), 55 KB at E = 8 with bf16 io; the A rows live in
+// tensor memory (load_a2_tm) and the state before each sub-block in a per-CTA global scratch
+// (p.sub, [4][2][128 threads] float4, written and read back by the same thread; 16 KB per CTA, so
+// it stays in L2). The adjoint recomputes each token's exp(Δ A) instead of keeping the sub-block's
+// 16 float2 of them: 127 registers. Four CTAs per SM (16 warps) against three with the sub-block
+// states in shared memory and the exponentials kept (156 registers): 10.4 -> 8.3 ms on the
+// Mamba-1.4B-like shape, for one more exponential per state element.
 template <typename IO, int K>
-__global__ void __launch_bounds__(kPkThreads, 3) scan_bwd_pk_kernel(ScanBwdParams p) {
+__global__ void __launch_bounds__(kPkThreads, 4) scan_bwd_pk_kernel(ScanBwdParams p) {
   extern __shared__ __align__(16) float smem_pk[];
   __shared__ uint32_t tm_slot;
   float* dAacc = smem_pk;
-  float4* sub = reinterpret_cast<float4*>(dAacc + p.E * kPkThreads * 8);
-  float* red = reinterpret_cast<float*>(sub + (kBwdLc / kBwdSub) * kPkThreads * 2);
+  float* red = dAacc + p.E * kPkThreads * 8;
+  float4* sub = reinterpret_cast<float4*>(p.sub) + (size_t)blockIdx.x * (kBwdLc / kBwdSub) * kPkThreads * 2;
   const int rw = 2 * 16 + K;  // per token: dB[16], dC[16], dgates[K]
   ChunkTile<IO>& ct = *reinterpret_cast<ChunkTile<IO>*>(red + kPkWarps * kBwdLc * rw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q = lane & 3;
@@ -648,7 +655,7 @@ __global__ void __launch_bounds__(kPkThreads, 3) scan_bwd_pk_kernel(ScanBwdParam
   const int d0 = tile * kBwdCh, nc = min(kBwdCh, p.D - d0);  // nc % 16 == 0
   const bool valid = 16 * warp < nc;                         // whole warps
   // the A rows of every expert for the lane's channels and quarter in tensor memory (8 columns per
-  // expert), which keeps the shared memory of a CTA small enough for three CTAs per SM
+  // expert), which keeps the shared memory of a CTA small enough for four CTAs per SM
   const uint32_t tm_cols = pk_tmem_cols(p.E);
   if (warp == 0) {
     sm100::tmem_alloc(&tm_slot, tm_cols);
@@ -855,12 +862,17 @@ cudaError_t launch_bwd_pk(const ScanBwdParams& p, unsigned grid, size_t smem_ck,
   return cudaGetLastError();
 }
 
+// The packed kernel's per-CTA scratch: the state before each 4-token sub-block of the current chunk
+// (written by the forward through the chunk, read back by the same thread in the adjoint; it stays in
+// L2).
+static size_t sub_bytes(int64_t ctas) { return (size_t)ctas * (kBwdLc / kBwdSub) * kPkThreads * 2 * sizeof(float4); }
+
 size_t scan_bwd_workspace(int64_t B, int64_t L, int D, int N, int E, int k) {
   const int64_t tiles = (D + kBwdCh - 1) / kBwdCh;
   const int64_t nck = (L + kBwdLc - 1) / kBwdLc;
   auto up = [](size_t v) { return (v + 255) & ~size_t(255); };
   return up((size_t)B * nck * D * N * 4) + up((size_t)tiles * B * L * (2 * N + k) * 4) +
-         up((size_t)B * E * D * N * 4) + up((size_t)B * D * 4);
+         up((size_t)B * E * D * N * 4) + up((size_t)B * D * 4) + up(sub_bytes(tiles * B));
 }
 
 cudaError_t run_scan_bwd(ScanBwdParams p, bool io_bf16, void* ws, cudaStream_t s) {
@@ -875,6 +887,8 @@ cudaError_t run_scan_bwd(ScanBwdParams p, bool io_bf16, void* ws, cudaStream_t s
   p.part_A = reinterpret_cast<float*>(w);
   w += up((size_t)p.B * p.E * p.D * p.N * 4);
   p.part_D = reinterpret_cast<float*>(w);
+  w += up((size_t)p.B * p.D * 4);
+  p.sub = reinterpret_cast<float*>(w);
   const unsigned grid = (unsigned)(tiles * p.B);
   const size_t a_bytes = sizeof(float) * (size_t)p.E * kBwdCh * 16;
   const size_t tile_bytes = io_bf16 ? sizeof(ChunkTile<__nv_bfloat16>) : sizeof(ChunkTile<float>);
@@ -885,7 +899,7 @@ cudaError_t run_scan_bwd(ScanBwdParams p, bool io_bf16, void* ws, cudaStream_t s
   // packed layout: N = 16, k <= 2, whole 16-channel warps
   const bool packed = p.N == 16 && (p.k == 1 || p.k == 2) && p.D % 16 == 0;
   const size_t smem_pk = sizeof(float) * ((size_t)p.E * kPkThreads * 8 + (size_t)kPkWarps * kBwdLc * (32 + p.k)) +
-                         sizeof(float4) * (kBwdLc / kBwdSub) * kPkThreads * 2 + tile_bytes;
+                         tile_bytes;
   const bool fast_ckpt = packed && io_bf16 && scan_fast_plan(p.B, p.L, p.D, p.N, p.E, p.k, true).fast;
   if (packed) {
     if (io_bf16) {
