@@ -494,7 +494,9 @@ __global__ void __launch_bounds__(kPkThreads) scan_bwd_ckpt_pk_kernel(ScanBwdPar
 // The adjoint back through tokens [i0, i0 + ni) of the staged chunk (ni <= 4), packed layout: the
 // sub-block's states, transitions and dy are recomputed into registers from h_in (the state
 // before token i0), then walked backwards, updating `carry` (a_{t+1} λ_{t+1}).
-template <int K, typename IO>
+// FULL: the sub-block holds kBwdSub tokens (every sub-block but a ragged tail), so its token loops
+// carry no bounds test and the compiler may interleave the tokens' independent work.
+template <int K, bool FULL, typename IO>
 __device__ __forceinline__ void adjoint_sub_pk(const ScanBwdParams& p, const ChunkTile<IO>& ct, uint32_t tm_lane,
                                                float* dAacc, float* red, int rw, int i0, int ni,
                                                const float2 (&h_in)[4], int64_t t0, int b, int d0, int c0,
@@ -505,7 +507,7 @@ __device__ __forceinline__ void adjoint_sub_pk(const ScanBwdParams& p, const Chu
     float2 h[4] = {h_in[0], h_in[1], h_in[2], h_in[3]};
 #pragma unroll
     for (int u = 0; u < kBwdSub; ++u) {
-      if (u < ni) {
+      if (FULL || u < ni) {
         const int i = i0 + u;
         float4 a0[K], a1[K];
         load_a2_tm<K>(ct, tm_lane, i, a0, a1);
@@ -525,7 +527,7 @@ __device__ __forceinline__ void adjoint_sub_pk(const ScanBwdParams& p, const Chu
   }
 #pragma unroll
   for (int u = kBwdSub - 1; u >= 0; --u) {
-    if (u < ni) {
+    if (FULL || u < ni) {
       const int i = i0 + u;
       float4 a0[K], a1[K];
       load_a2_tm<K>(ct, tm_lane, i, a0, a1);
@@ -703,12 +705,9 @@ __global__ void __launch_bounds__(kPkThreads, 4) scan_bwd_pk_kernel(ScanBwdParam
     __syncthreads();
     if (valid) {
       // ---- forward through the chunk: the state before every sub-block, and dz ----
-      for (int i = 0; i < nt; ++i) {
-        if ((i & (kBwdSub - 1)) == 0) {
-          float4* sv = sub + (i / kBwdSub) * 2 * kPkThreads + tid;
-          sv[0] = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
-          sv[kPkThreads] = make_float4(h[2].x, h[2].y, h[3].x, h[3].y);
-        }
+      // (one token; lanes q = 0, 1 write dz of channel c0 + q, lanes 2, 3 compute the same and skip
+      // the store, so the body has no branch)
+      auto fwd_token = [&](int i) {
         float4 a0[K], a1[K];
         load_a2_tm<K>(ct, tm_lane, i, a0, a1);
         float2 at[4];
@@ -725,12 +724,21 @@ __global__ void __launch_bounds__(kPkThreads, 4) scan_bwd_pk_kernel(ScanBwdParam
         y.y += __shfl_xor_sync(0xffffffffu, y.y, 1);
         y.x += __shfl_xor_sync(0xffffffffu, y.x, 2);
         y.y += __shfl_xor_sync(0xffffffffu, y.y, 2);
-        if (q == 0) {
-          const float2 zv = ld2(ct.z[i], c0), go = ld2(ct.go[i], c0);
-          const float2 yy = __ffma2_rn(dsk, xv, y);
-          const float s0 = sigmoid_f(zv.x), s1 = sigmoid_f(zv.y);
-          *reinterpret_cast<float2*>(p.dz + ((size_t)b * p.L + t0 + i) * p.D + d0 + c0) =
-              make_float2(go.x * yy.x * s0 * fmaf(zv.x, 1.f - s0, 1.f), go.y * yy.y * s1 * fmaf(zv.y, 1.f - s1, 1.f));
+        const int ch = c0 + (q & 1);
+        const float zv = to_f32(ct.z[i][ch]), go = to_f32(ct.go[i][ch]);
+        const float yy = fmaf(q & 1 ? dsk.y : dsk.x, q & 1 ? xv.y : xv.x, q & 1 ? y.y : y.x);
+        const float sg = sigmoid_f(zv);
+        if (q < 2) p.dz[((size_t)b * p.L + t0 + i) * p.D + d0 + ch] = go * yy * sg * fmaf(zv, 1.f - sg, 1.f);
+      };
+      for (int i0 = 0; i0 < nt; i0 += kBwdSub) {
+        float4* sv = sub + (i0 / kBwdSub) * 2 * kPkThreads + tid;
+        sv[0] = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
+        sv[kPkThreads] = make_float4(h[2].x, h[2].y, h[3].x, h[3].y);
+        if (nt - i0 >= kBwdSub) {
+#pragma unroll
+          for (int u = 0; u < kBwdSub; ++u) fwd_token(i0 + u);
+        } else {
+          for (int i = i0; i < nt; ++i) fwd_token(i);
         }
       }
       // ---- the adjoint back through the chunk, one sub-block at a time ----
@@ -741,8 +749,12 @@ __global__ void __launch_bounds__(kPkThreads, 4) scan_bwd_pk_kernel(ScanBwdParam
         const float4 v0 = sv[0], v1 = sv[kPkThreads];
         const float2 h_in[4] = {make_float2(v0.x, v0.y), make_float2(v0.z, v0.w), make_float2(v1.x, v1.y),
                                 make_float2(v1.z, v1.w)};
-        adjoint_sub_pk<K>(p, ct, tm_lane, dAacc, red, rw, i0, ni, h_in, t0, b, d0, c0, valid, dsk, tid, warp, lane, q,
-                          carry, dD);
+        if (ni == kBwdSub)
+          adjoint_sub_pk<K, true>(p, ct, tm_lane, dAacc, red, rw, i0, ni, h_in, t0, b, d0, c0, valid, dsk, tid, warp,
+                                  lane, q, carry, dD);
+        else
+          adjoint_sub_pk<K, false>(p, ct, tm_lane, dAacc, red, rw, i0, ni, h_in, t0, b, d0, c0, valid, dsk, tid, warp,
+                                   lane, q, carry, dD);
       }
     } else {
       for (int v = lane; v < nt * rw; v += 32) red[(size_t)warp * kBwdLc * rw + v] = 0.f;
