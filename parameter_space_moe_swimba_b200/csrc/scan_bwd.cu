@@ -558,11 +558,16 @@ __device__ __forceinline__ void adjoint_sub_pk(const ScanBwdParams& p, const Chu
         sum_d.x += __shfl_xor_sync(0xffffffffu, sum_d.x, o);
         sum_d.y += __shfl_xor_sync(0xffffffffu, sum_d.y, o);
       }
-      if (valid && q == 0) {
-        const size_t g = ((size_t)b * p.L + t0 + i) * p.D + d0 + c0;
-        *reinterpret_cast<float2*>(p.dx + g) = __ffma2_rn(dsk, DY[u], __fmul2_rn(dl, sum_b));
-        *reinterpret_cast<float2*>(p.ddelta + g) = __ffma2_rn(sum_b, xv, sum_d);
-        dD = __ffma2_rn(DY[u], xv, dD);
+      // every lane of a quarter group now holds both channels' sums: lane q writes one of the four
+      // values (dx of c0, c0 + 1; dΔ of c0, c0 + 1), so no branch
+      {
+        const bool odd = q & 1;
+        const float sb = odd ? sum_b.y : sum_b.x;
+        const float vdx = fmaf(odd ? dsk.y : dsk.x, odd ? DY[u].y : DY[u].x, (odd ? dl.y : dl.x) * sb);
+        const float vdd = fmaf(sb, odd ? xv.y : xv.x, odd ? sum_d.y : sum_d.x);
+        const size_t g = ((size_t)b * p.L + t0 + i) * p.D + d0 + c0 + (odd ? 1 : 0);
+        if (valid) (q < 2 ? p.dx : p.ddelta)[g] = q < 2 ? vdx : vdd;
+        dD = __ffma2_rn(DY[u], xv, dD);  // every lane alike; the q == 0 lanes' sums are written
       }
       // dB, dC: the 8 values (vB[0..3], vC[0..3]) summed over the warp's 8 channel pairs (lane
       // bits 2-4) by recursive halving; lane l ends with the value of type (l >> 4) & 1 (B, C) and
