@@ -258,8 +258,8 @@ swimba_status swimba_scan_bwd(const swimba_dims* dims, const void* x, const void
       !ddelta || !dB || !dC || !dgates || !dA || !dD)
     return SWIMBA_ERR_INVALID_ARG;
   if (!aligned16(w->A) || !aligned16(w->D_skip) || !aligned16(ws) || !aligned16(x) || !aligned16(z) ||
-      !aligned16(delta) || !aligned16(g_out) || !aligned16(dx) || !aligned16(dz) || !aligned16(ddelta) ||
-      (h0 && !aligned16(h0)) || (dh0 && !aligned16(dh0)))
+      !aligned16(delta) || !aligned16(B_mix) || !aligned16(C_mix) || !aligned16(g_out) || !aligned16(dx) ||
+      !aligned16(dz) || !aligned16(ddelta) || (h0 && !aligned16(h0)) || (dh0 && !aligned16(dh0)))
     return SWIMBA_ERR_ALIGN;
   if (ws == nullptr || ws_bytes < swimba_workspace_size(dims, SWIMBA_OP_SCAN_BWD)) return SWIMBA_ERR_WORKSPACE;
   ScanBwdParams p{};

@@ -632,6 +632,58 @@ __device__ __forceinline__ void adjoint_sub_pk(const ScanBwdParams& p, const Chu
   }
 }
 
+// The packed kernel's chunk load for a full chunk (16 tokens) of a full tile (64 channels), k == K:
+// every thread issues all of its global loads (Δ 2 x 16 B; x, z, g_out 16 B each; a quarter row of
+// B_mix or C_mix; one expert index and gate for threads < 16K) before its first shared-memory store,
+// so the chunk costs one memory round trip instead of one per loop trip of load_chunk. Only the
+// first K expert slots of each token are written; the packed kernel reads no other.
+template <int K, typename IO>
+__device__ __forceinline__ void load_chunk_pk_full(ChunkTile<IO>& ct, const ScanBwdParams& p, int b, int64_t t0,
+                                                   int d0) {
+  static_assert(kPkThreads == 128 && kBwdLc == 16 && kBwdCh == 64, "thread-to-item map below");
+  const int tid = threadIdx.x;
+  const size_t row0 = (size_t)b * p.L + t0;
+  const int r0 = tid >> 4, cd = (tid & 15) * 4;  // Δ: items tid and tid + 128 of 16 x 16 float4
+  const float4 dl0 = *reinterpret_cast<const float4*>(p.delta + (row0 + r0) * p.D + d0 + cd);
+  const float4 dl1 = *reinterpret_cast<const float4*>(p.delta + (row0 + r0 + 8) * p.D + d0 + cd);
+  constexpr int per16 = 16 / (int)sizeof(IO), vio = kBwdCh / per16;  // 16-byte items per row
+  uint4 xv[2], zv[2], gv[2];
+  int rio[2], cio[2];
+  constexpr int nio = (kBwdLc * vio + kPkThreads - 1) / kPkThreads;  // 1 (bf16) or 2 (fp32)
+#pragma unroll
+  for (int a = 0; a < nio; ++a) {
+    const int it = tid + a * kPkThreads;
+    rio[a] = it / vio;
+    cio[a] = (it % vio) * per16;
+    const size_t g = (row0 + rio[a]) * p.D + d0 + cio[a];
+    xv[a] = *reinterpret_cast<const uint4*>(reinterpret_cast<const IO*>(p.x) + g);
+    zv[a] = *reinterpret_cast<const uint4*>(reinterpret_cast<const IO*>(p.z) + g);
+    gv[a] = *reinterpret_cast<const uint4*>(reinterpret_cast<const IO*>(p.g_out) + g);
+  }
+  // B_mix / C_mix rows of the chunk's 16 tokens are 256 contiguous floats each (N = 16)
+  const int bc = tid & 63;
+  const float4 bcv = *reinterpret_cast<const float4*>((tid < 64 ? p.B_mix : p.C_mix) + row0 * 16 + 4 * bc);
+  int ev = 0;
+  float gw = 0.f;
+  if (tid < kBwdLc * K) {
+    ev = min(max(p.idx[row0 * K + tid], 0), p.E - 1);
+    gw = p.gates[row0 * K + tid];
+  }
+  *reinterpret_cast<float4*>(&ct.dl[r0][cd]) = dl0;
+  *reinterpret_cast<float4*>(&ct.dl[r0 + 8][cd]) = dl1;
+#pragma unroll
+  for (int a = 0; a < nio; ++a) {
+    *reinterpret_cast<uint4*>(&ct.x[rio[a]][cio[a]]) = xv[a];
+    *reinterpret_cast<uint4*>(&ct.z[rio[a]][cio[a]]) = zv[a];
+    *reinterpret_cast<uint4*>(&ct.go[rio[a]][cio[a]]) = gv[a];
+  }
+  *reinterpret_cast<float4*>(tid < 64 ? &ct.B[bc >> 2][4 * (bc & 3)] : &ct.C[bc >> 2][4 * (bc & 3)]) = bcv;
+  if (tid < kBwdLc * K) {
+    ct.e[tid / K][tid % K] = ev;
+    ct.g[tid / K][tid % K] = gw;
+  }
+}
+
 // Tensor-memory columns for the packed kernel's A rows: 8 per expert, rounded up to a power of two
 // of at least 32 (the allocation unit).
 __host__ __device__ constexpr uint32_t pk_tmem_cols(int E) { return E * 8 <= 32 ? 32u : (E * 8 <= 64 ? 64u : 128u); }
@@ -693,7 +745,8 @@ __global__ void __launch_bounds__(kPkThreads, 4) scan_bwd_pk_kernel(ScanBwdParam
     const int64_t t0 = (int64_t)ck * kBwdLc;
     const int nt = (int)(p.L - t0 < kBwdLc ? p.L - t0 : kBwdLc);
     __syncthreads();  // the previous chunk's tile and partial sums are no longer read
-    load_chunk(ct, p, b, t0, nt, d0, nc, true);
+    if (nt == kBwdLc && nc == kBwdCh && p.k == K) load_chunk_pk_full<K>(ct, p, b, t0, d0);
+    else load_chunk(ct, p, b, t0, nt, d0, nc, true);
     float2 h[4];
     {
       float4 u0 = make_float4(0.f, 0.f, 0.f, 0.f), u1 = u0;

@@ -117,3 +117,5 @@ def test_scan_backward_rejects_bad_arguments(S):
     assert S.swimba_scan_bwd(dims, *full, W, None, t, *outs, None, ws, 16) == 4
     assert S.swimba_scan_bwd(dims, *full, W, None, t, *outs, t.data_ptr() + 4, ws, ws.numel()) == 3
     assert S.swimba_scan_bwd(dims, *full, W, None, t, t.data_ptr() + 8, *outs[1:], None, ws, ws.numel()) == 3
+    bad_b = [t, t, t, t.data_ptr() + 4, t, t, t]  # B_mix off its 16-byte boundary
+    assert S.swimba_scan_bwd(dims, *bad_b, W, None, t, *outs, None, ws, ws.numel()) == 3
