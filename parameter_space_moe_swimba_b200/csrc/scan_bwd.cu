@@ -695,7 +695,7 @@ __host__ __device__ constexpr uint32_t pk_tmem_cols(int E) { return E * 8 <= 32 
 // tensor memory (load_a2_tm) and the state before each sub-block in a per-CTA global scratch
 // (p.sub, [4][2][128 threads] float4, written and read back by the same thread; 16 KB per CTA, so
 // it stays in L2). The adjoint recomputes each token's exp(Δ A) instead of keeping the sub-block's
-// 16 float2 of them: 127 registers. Four CTAs per SM (16 warps) against three with the sub-block
+// 16 float2 of them: at most 128 registers. Four CTAs per SM (16 warps) against three with the sub-block
 // states in shared memory and the exponentials kept (156 registers): 10.4 -> 8.3 ms on the
 // Mamba-1.4B-like shape, for one more exponential per state element.
 template <typename IO, int K>
