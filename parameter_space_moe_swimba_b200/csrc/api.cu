@@ -308,7 +308,8 @@ swimba_status swimba_proj_bwd(const swimba_dims* dims, const void* x, const int3
       dims->d_state % 4 != 0 || T * dims->top_k >= (int64_t(1) << 31))
     return SWIMBA_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(delta) || !aligned16(g_delta) || !aligned16(dx) || !aligned16(dW_x) ||
-      !aligned16(dW_dt) || !aligned16(db_dt) || !aligned16(w->W_x) || !aligned16(w->W_dt) || !aligned16(ws))
+      !aligned16(dW_dt) || !aligned16(db_dt) || !aligned16(w->W_x) || !aligned16(w->W_dt) ||
+      !aligned16(w->b_dt) || !aligned16(ws))
     return SWIMBA_ERR_ALIGN;
   if (ws == nullptr || ws_bytes < swimba_workspace_size(dims, SWIMBA_OP_PROJ_BWD)) return SWIMBA_ERR_WORKSPACE;
   return cuda_status(run_proj_bwd(x, delta, g_delta, g_B, g_C, idx, gates, w->W_x, w->W_dt, w->b_dt, false, dx,

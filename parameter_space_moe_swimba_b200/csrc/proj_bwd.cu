@@ -37,71 +37,107 @@ cudaError_t run_gemm_tc(bool a_t, bool b_t, bool f32_out, int M, int N, int K, c
 
 namespace {
 
-constexpr int kSortThreads = 1024;
 constexpr int kMaxE = 16;
 
-// Stable counting sort of the P = T k pairs by expert, one CTA: each thread counts a contiguous
-// run of pairs per expert, an exclusive scan over the threads (per expert) gives every thread's
-// first slot, and the run is scattered in order. perm[row] = pair, inv[pair] = row,
-// counts[e] = pairs of expert e, offsets[e] = first row of expert e.
-__global__ void __launch_bounds__(kSortThreads) pair_sort_kernel(const int32_t* idx, int64_t P, int E, int* counts,
-                                                                 int* offsets, int* perm, int* inv) {
-  extern __shared__ int cnt[];  // [E][kSortThreads]
-  const int tid = threadIdx.x;
-  const int64_t per = (P + kSortThreads - 1) / kSortThreads;
-  const int64_t p0 = min(P, per * tid), p1 = min(P, p0 + per);
-  int local[kMaxE];
-#pragma unroll
-  for (int e = 0; e < kMaxE; ++e) local[e] = 0;
-  for (int64_t p = p0; p < p1; ++p) {
-    const int e = min(max(idx[p], 0), E - 1);
-#pragma unroll
-    for (int ee = 0; ee < kMaxE; ++ee) local[ee] += (ee == e);
-  }
-  for (int e = 0; e < E; ++e) cnt[e * kSortThreads + tid] = local[e];
+// Stable counting sort of the P = T k pairs by expert over blocks of kPairBlock pairs, three
+// kernels: per-block counts per expert; one CTA turning them into the experts' sizes and offsets and
+// every block's first row per expert; each block placing its pairs at that row plus their rank
+// among the block's earlier pairs of the expert (warp match + per-warp counts). perm[row] = pair,
+// inv[pair] = row, counts[e] = pairs of expert e, offsets[e] = first row of expert e; inside an
+// expert the rows keep ascending pair order, whatever the scheduling.
+constexpr int kPairBlock = 1024;
+
+__global__ void __launch_bounds__(kPairBlock) pair_count_kernel(const int32_t* idx, int64_t P, int E, int* bhist) {
+  __shared__ int hist[kMaxE];
+  if (threadIdx.x < kMaxE) hist[threadIdx.x] = 0;
   __syncthreads();
-  // exclusive scan per expert over the threads (thread e < E walks its row; E <= 16 rows)
-  __shared__ int base[kMaxE + 1];
-  if (tid < E) {
-    int run = 0;
-    for (int i = 0; i < kSortThreads; ++i) {
-      const int v = cnt[tid * kSortThreads + i];
-      cnt[tid * kSortThreads + i] = run;
-      run += v;
-    }
-    counts[tid] = run;
-    base[tid] = run;
+  const int64_t p = (int64_t)blockIdx.x * kPairBlock + threadIdx.x;
+  if (p < P) atomicAdd(&hist[min(max(idx[p], 0), E - 1)], 1);
+  __syncthreads();
+  if (threadIdx.x < E) bhist[(size_t)blockIdx.x * E + threadIdx.x] = hist[threadIdx.x];
+}
+
+// One CTA, a warp per expert: the expert's total over the blocks, then (after the offsets) an
+// exclusive scan of its per-block counts, 32 blocks at a time.
+__global__ void __launch_bounds__(32 * kMaxE) pair_scan_kernel(const int* bhist, int nb, int E, int* counts,
+                                                              int* offsets, int* bbase) {
+  __shared__ int s_cnt[kMaxE], s_off[kMaxE];
+  const int lane = threadIdx.x & 31, e = threadIdx.x >> 5;
+  if (e < E) {
+    int c = 0;
+    for (int bb = lane; bb < nb; bb += 32) c += bhist[(size_t)bb * E + e];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    if (lane == 0) s_cnt[e] = c;
   }
   __syncthreads();
-  if (tid == 0) {
+  if (threadIdx.x == 0) {
     int o = 0;
-    for (int e = 0; e < E; ++e) {
-      const int n = base[e];
-      base[e] = o;
-      offsets[e] = o;
-      o += n;
+    for (int x = 0; x < E; ++x) {
+      s_off[x] = o;
+      counts[x] = s_cnt[x];
+      offsets[x] = o;
+      o += s_cnt[x];
     }
-    base[E] = o;
     offsets[E] = o;
   }
   __syncthreads();
-  int next[kMaxE];
+  if (e < E) {
+    int carry = s_off[e];
+    for (int b0 = 0; b0 < nb; b0 += 32) {
+      const int bb = b0 + lane;
+      const int v = bb < nb ? bhist[(size_t)bb * E + e] : 0;
+      int incl = v;
 #pragma unroll
-  for (int e = 0; e < kMaxE; ++e) next[e] = e < E ? base[e] + cnt[e * kSortThreads + tid] : 0;
-  for (int64_t p = p0; p < p1; ++p) {
-    const int e = min(max(idx[p], 0), E - 1);
-    int row = 0;
-#pragma unroll
-    for (int ee = 0; ee < kMaxE; ++ee)
-      if (ee == e) row = next[ee]++;
-    perm[row] = (int)p;
-    inv[p] = row;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      if (bb < nb) bbase[(size_t)bb * E + e] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
   }
+}
+
+__global__ void __launch_bounds__(kPairBlock) pair_scatter_kernel(const int32_t* idx, int64_t P, int E,
+                                                                 const int* bbase, int* perm, int* inv) {
+  __shared__ int warpcnt[kPairBlock / 32][kMaxE];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < (kPairBlock / 32) * kMaxE; i += kPairBlock) (&warpcnt[0][0])[i] = 0;
+  __syncthreads();
+  const int64_t p = (int64_t)blockIdx.x * kPairBlock + threadIdx.x;
+  const bool valid = p < P;
+  const int e = valid ? min(max(idx[p], 0), E - 1) : -1;
+  const unsigned same = __match_any_sync(0xffffffffu, e);
+  const int lane_rank = __popc(same & ((1u << lane) - 1u));
+  if (valid && lane_rank == 0) warpcnt[warp][e] = __popc(same);
+  __syncthreads();
+  if (!valid) return;
+  int row = bbase[(size_t)blockIdx.x * E + e] + lane_rank;
+  for (int w = 0; w < warp; ++w) row += warpcnt[w][e];
+  perm[row] = (int)p;
+  inv[p] = row;
 }
 
 // One CTA per token: g_dt = ∂L/∂Δ (1 − e^{−Δ}) is formed once, and each of the token's k pairs gets
 // its sorted row: Xg[row] = x[t] (bf16), G[row] = bf16(g_dt), bg[row] = b_dt^e · g_dt (fp32).
 constexpr int kMaxK = 16;
+// 8 consecutive weights as floats, in one 16-byte load (bf16) or two (fp32); 16-byte aligned.
+__device__ __forceinline__ void load8(const __nv_bfloat16* src, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(src);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void load8(const float* src, float (&v)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(src), b = *reinterpret_cast<const float4*>(src + 4);
+  v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w, v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+}
+
 template <typename WT>
 __global__ void __launch_bounds__(256) proj_bwd_gather_kernel(const __nv_bfloat16* x, const float* delta,
                                                               const float* g_delta, const int32_t* idx,
@@ -134,8 +170,10 @@ __global__ void __launch_bounds__(256) proj_bwd_gather_kernel(const __nv_bfloat1
         const int e = min(max(idx[t * k + j], 0), E - 1);
         *reinterpret_cast<uint4*>(Xg + (size_t)row * D + c) = xv;
         *reinterpret_cast<uint4*>(G + (size_t)row * D + c) = gv;
+        float bv[8];
+        load8(b_dt + (size_t)e * D + c, bv);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) part[j] = fmaf(gdt[i], to_f32(b_dt[(size_t)e * D + c + i]), part[j]);
+        for (int i = 0; i < 8; ++i) part[j] = fmaf(gdt[i], bv[i], part[j]);
       }
     }
   }
@@ -318,7 +356,7 @@ __global__ void route_bwd_dw_reduce_kernel(const float* part, int64_t nblk, int 
 size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct ProjBwdLayout {
-  size_t counts, offsets, perm, inv, bg, Xg, G, XD, Q, dV, DTs, TMP, total;
+  size_t counts, offsets, perm, inv, bhist, bbase, bg, Xg, G, XD, Q, dV, DTs, TMP, total;
 };
 
 ProjBwdLayout proj_bwd_layout(int64_t T, int D, int R, int N, int E, int k) {
@@ -334,6 +372,9 @@ ProjBwdLayout proj_bwd_layout(int64_t T, int D, int R, int N, int E, int k) {
   l.offsets = take(4 * (kMaxE + 1));
   l.perm = take(4 * P);
   l.inv = take(4 * P);
+  const size_t nb = (P + kPairBlock - 1) / kPairBlock;
+  l.bhist = take(4 * nb * E);
+  l.bbase = take(4 * nb * E);
   l.bg = take(4 * P);
   l.Xg = take(2 * P * D);
   l.G = take(2 * P * D);
@@ -415,11 +456,12 @@ cudaError_t run_proj_bwd(const void* x, const float* delta, const float* g_delta
   SideStreams* ss = side_streams();
   if (ss == nullptr) return cudaErrorNotReady;
   cudaError_t e;
-  const size_t sort_smem = sizeof(int) * (size_t)E * kSortThreads;
-  if ((e = cudaFuncSetAttribute(pair_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sort_smem)) !=
-      cudaSuccess)
-    return e;
-  pair_sort_kernel<<<1, kSortThreads, sort_smem, s>>>(idx, P, E, counts, offsets, perm, inv);
+  const int nb = (int)((P + kPairBlock - 1) / kPairBlock);
+  int* bhist = reinterpret_cast<int*>(w + l.bhist);
+  int* bbase = reinterpret_cast<int*>(w + l.bbase);
+  pair_count_kernel<<<(unsigned)nb, kPairBlock, 0, s>>>(idx, P, E, bhist);
+  pair_scan_kernel<<<1, 32 * kMaxE, 0, s>>>(bhist, nb, E, counts, offsets, bbase);
+  pair_scatter_kernel<<<(unsigned)nb, kPairBlock, 0, s>>>(idx, P, E, bbase, perm, inv);
   if (b_bf16)
     proj_bwd_gather_kernel<__nv_bfloat16><<<(unsigned)T, 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(x), delta, g_delta, idx, static_cast<const __nv_bfloat16*>(b_dt), inv, k,
@@ -428,7 +470,7 @@ cudaError_t run_proj_bwd(const void* x, const float* delta, const float* g_delta
     proj_bwd_gather_kernel<float><<<(unsigned)T, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), delta, g_delta,
                                                               idx, static_cast<const float*>(b_dt), inv, k, D, E, Xg,
                                                               G, bg);
-  note_launch(2);
+  note_launch(4);  // the three sorting kernels and the gather
   if (!accumulate && (e = cudaMemsetAsync(dx, 0, sizeof(float) * (size_t)T * D, s)) != cudaSuccess) return e;
   int h_off[kMaxE + 1];
   if ((e = cudaMemcpyAsync(h_off, offsets, sizeof(int) * (E + 1), cudaMemcpyDeviceToHost, s)) != cudaSuccess) return e;
