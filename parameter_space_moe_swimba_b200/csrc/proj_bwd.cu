@@ -27,6 +27,8 @@
 // are exact); that makes this entry point synchronise its stream, unlike the forward ones.
 #include <mutex>
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace swimba {
@@ -264,22 +266,24 @@ __global__ void route_bwd_logits_kernel(const int32_t* idx, const float* gates, 
 }
 
 // ∂L/∂x[t, d] (+)= Σ_e ∂L/∂logits[t, e] W_r[d, e]: a CTA owns 256 channels (a thread each, its
-// W_r row in registers) and a run of 64 tokens, whose ∂L/∂logits rows it stages in shared memory;
-// every dx access is a coalesced row segment.
+// W_r row in registers) and a run of 64 tokens, whose ∂L/∂logits rows it stages in shared memory
+// (EP = E rounded up to 4 columns, zero-padded, read back as float4 broadcasts); every dx access
+// is a coalesced row segment.
 constexpr int kDxTok = 64;
+template <int EP>
 __global__ void __launch_bounds__(256) route_bwd_dx_kernel(const float* W_r, const float* dlogits, int64_t T, int D,
                                                            int E, float* dx, int accumulate) {
-  __shared__ float dl[kDxTok][kMaxE];
+  __shared__ __align__(16) float dl[kDxTok][EP];
   const int d = blockIdx.x * 256 + threadIdx.x;
   const int64_t t0 = (int64_t)blockIdx.y * kDxTok;
   const int nt = (int)(T - t0 < kDxTok ? T - t0 : kDxTok);
-  for (int i = threadIdx.x; i < nt * kMaxE; i += 256) {
-    const int r = i / kMaxE, e = i % kMaxE;
-    dl[r][e] = e < E ? dlogits[(t0 + r) * E + e] : 0.f;
+  for (int i = threadIdx.x; i < kDxTok * EP; i += 256) {
+    const int r = i / EP, e = i % EP;
+    dl[r][e] = (r < nt && e < E) ? dlogits[(t0 + r) * E + e] : 0.f;
   }
-  float w[kMaxE];
+  float w[EP];
 #pragma unroll
-  for (int e = 0; e < kMaxE; ++e) w[e] = (d < D && e < E) ? W_r[(size_t)d * E + e] : 0.f;
+  for (int e = 0; e < EP; ++e) w[e] = (d < D && e < E) ? W_r[(size_t)d * E + e] : 0.f;
   __syncthreads();
   if (d >= D) return;
   // dx is read and written in place, so the compiler may not move a load above an earlier store
@@ -301,7 +305,13 @@ __global__ void __launch_bounds__(256) route_bwd_dx_kernel(const float* W_r, con
       if (r < nt) {
         float acc = a[i];
 #pragma unroll
-        for (int e = 0; e < kMaxE; ++e) acc = fmaf(dl[r][e], w[e], acc);
+        for (int e4 = 0; e4 < EP; e4 += 4) {
+          const float4 g = *reinterpret_cast<const float4*>(&dl[r][e4]);
+          acc = fmaf(g.x, w[e4], acc);
+          acc = fmaf(g.y, w[e4 + 1], acc);
+          acc = fmaf(g.z, w[e4 + 2], acc);
+          acc = fmaf(g.w, w[e4 + 3], acc);
+        }
         dx[(t0 + r) * D + d] = acc;
       }
     }
@@ -312,35 +322,59 @@ __global__ void __launch_bounds__(256) route_bwd_dx_kernel(const float* W_r, con
 
 constexpr int kDwTok = 256;  // tokens per partial of ∂L/∂W_r
 
-// Partial ∂L/∂W_r over a block of 256 tokens: a CTA owns 64 channels x 4 token runs of 64; the
-// runs are summed in shared memory and the block's partial written [block][d][e].
-template <typename IO>
+__device__ __forceinline__ float2 ld2f(const __nv_bfloat16* p) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+__device__ __forceinline__ float2 ld2f(const float* p) { return *reinterpret_cast<const float2*>(p); }
+
+// Partial ∂L/∂W_r over a block of 256 tokens: a CTA owns 512 channels (two per thread, one 2-element
+// load per token) and the block's tokens, whose ∂L/∂logits rows it stages in shared memory (EP
+// columns, zero-padded, read back as float4 broadcasts); eight tokens' x loads are issued before
+// their multiply-adds. The partial goes to part[block][d][e].
+template <typename IO, int EP>
 __global__ void __launch_bounds__(256) route_bwd_dw_kernel(const IO* x, const float* dlogits, int64_t T, int D, int E,
                                                            float* part) {
-  __shared__ float red[4][64][kMaxE + 1];
-  const int c = threadIdx.x & 63, run = threadIdx.x >> 6;
-  const int d = blockIdx.x * 64 + c;
-  const int64_t tb = blockIdx.y;
-  float acc[kMaxE];
+  __shared__ __align__(16) float dls[kDwTok][EP];
+  const int64_t tb = blockIdx.y, t0 = tb * kDwTok;
+  const int nt = (int)(T - t0 < kDwTok ? T - t0 : kDwTok);
+  for (int i = threadIdx.x; i < kDwTok * EP; i += 256) {
+    const int r = i / EP, e = i % EP;
+    dls[r][e] = (r < nt && e < E) ? dlogits[(t0 + r) * E + e] : 0.f;
+  }
+  __syncthreads();
+  const int d = (blockIdx.x * 256 + threadIdx.x) * 2;  // D % 8 == 0: d < D means d + 1 < D
+  if (d >= D) return;
+  float a0[EP], a1[EP];
 #pragma unroll
-  for (int e = 0; e < kMaxE; ++e) acc[e] = 0.f;
-  const int64_t t0 = tb * kDwTok + run * (kDwTok / 4), t1 = min(T, t0 + kDwTok / 4);
-  if (d < D) {
-#pragma unroll 4
-    for (int64_t t = t0; t < t1; ++t) {
-      const float xv = to_f32(x[t * D + d]);
+  for (int e = 0; e < EP; ++e) a0[e] = a1[e] = 0.f;
+  constexpr int U = 8;  // divides kDwTok, so rows r0 .. r0 + 7 stay inside dls
+  for (int r0 = 0; r0 < nt; r0 += U) {
+    float2 xv[U];
 #pragma unroll
-      for (int e = 0; e < kMaxE; ++e)
-        if (e < E) acc[e] = fmaf(xv, __ldg(dlogits + t * E + e), acc[e]);
+    for (int u = 0; u < U; ++u) xv[u] = r0 + u < nt ? ld2f(x + (t0 + r0 + u) * D + d) : make_float2(0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+#pragma unroll
+      for (int e4 = 0; e4 < EP; e4 += 4) {
+        const float4 g = *reinterpret_cast<const float4*>(&dls[r0 + u][e4]);
+        a0[e4] = fmaf(xv[u].x, g.x, a0[e4]);
+        a0[e4 + 1] = fmaf(xv[u].x, g.y, a0[e4 + 1]);
+        a0[e4 + 2] = fmaf(xv[u].x, g.z, a0[e4 + 2]);
+        a0[e4 + 3] = fmaf(xv[u].x, g.w, a0[e4 + 3]);
+        a1[e4] = fmaf(xv[u].y, g.x, a1[e4]);
+        a1[e4 + 1] = fmaf(xv[u].y, g.y, a1[e4 + 1]);
+        a1[e4 + 2] = fmaf(xv[u].y, g.z, a1[e4 + 2]);
+        a1[e4 + 3] = fmaf(xv[u].y, g.w, a1[e4 + 3]);
+      }
     }
   }
+  float* dst = part + (tb * D + d) * E;
 #pragma unroll
-  for (int e = 0; e < kMaxE; ++e) red[run][c][e] = acc[e];
-  __syncthreads();
-  if (run == 0 && d < D) {
-    for (int e = 0; e < E; ++e)
-      part[(tb * D + d) * E + e] = red[0][c][e] + red[1][c][e] + red[2][c][e] + red[3][c][e];
-  }
+  for (int e = 0; e < EP; ++e)
+    if (e < E) {
+      dst[e] = a0[e];
+      dst[E + e] = a1[e];
+    }
 }
 
 // ∂L/∂W_r = Σ over the token blocks' partials, in block order.
@@ -550,13 +584,21 @@ cudaError_t run_route_bwd(const void* x, bool io_bf16, const float* W_r, const i
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   route_bwd_logits_kernel<<<(unsigned)((T + 255) / 256), 256, 0, s>>>(idx, gates, gg_a, gg_b, T, E, k, dlogits);
-  route_bwd_dx_kernel<<<dim3((unsigned)((D + 255) / 256), (unsigned)((T + kDxTok - 1) / kDxTok)), 256, 0, s>>>(
-      W_r, dlogits, T, D, E, dx, accumulate);
-  const dim3 g((unsigned)((D + 63) / 64), (unsigned)nblk);
-  if (io_bf16)
-    route_bwd_dw_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), dlogits, T, D, E, part);
-  else
-    route_bwd_dw_kernel<float><<<g, 256, 0, s>>>(static_cast<const float*>(x), dlogits, T, D, E, part);
+  const dim3 gx((unsigned)((D + 255) / 256), (unsigned)((T + kDxTok - 1) / kDxTok));
+  const dim3 gw((unsigned)((D + 511) / 512), (unsigned)nblk);
+  auto both = [&](auto ep) {
+    constexpr int EP = decltype(ep)::value;
+    route_bwd_dx_kernel<EP><<<gx, 256, 0, s>>>(W_r, dlogits, T, D, E, dx, accumulate);
+    if (io_bf16)
+      route_bwd_dw_kernel<__nv_bfloat16, EP><<<gw, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), dlogits, T, D,
+                                                                 E, part);
+    else
+      route_bwd_dw_kernel<float, EP><<<gw, 256, 0, s>>>(static_cast<const float*>(x), dlogits, T, D, E, part);
+  };
+  if (E <= 4) both(std::integral_constant<int, 4>{});
+  else if (E <= 8) both(std::integral_constant<int, 8>{});
+  else if (E <= 12) both(std::integral_constant<int, 12>{});
+  else both(std::integral_constant<int, 16>{});
   route_bwd_dw_reduce_kernel<<<(unsigned)(2 * sms), 256, 0, s>>>(part, nblk, D, E, dW_r);
   note_launch(4);
   return cudaGetLastError();
