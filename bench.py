@@ -897,6 +897,8 @@ def run_report(args):
     # Theorem 2 against the design it is set against: one trajectory per expert
     print(json.dumps(report_separate(torch, S, CONFIGS["mamba1p4b_like"], peaks, flush, reps, args.warmup)),
           flush=True)
+    # the layer's backward pass (scan, projection and router gradients)
+    print(json.dumps(report_bwd(torch, S, CONFIGS["mamba1p4b_like"], peaks, flush, 10, args.warmup)), flush=True)
     # Theorem 2: the recurrence's cost does not grow with E (k = 2 fixed; E = 1 forces k = 1)
     base = CONFIGS["mamba1p4b_like"]
     for E in (1, 4, 8, 16):
