@@ -164,7 +164,7 @@ swimba_status swimba_scan_fwd_zoh(const swimba_dims *dims, const void *x, const 
  *   The sums over channels, tokens and sequences are taken in a fixed order (deterministic).
  *   ws: at least swimba_workspace_size(dims, SWIMBA_OP_SCAN_BWD) bytes (checkpoints, partial
  *   sums and a per-block scratch of the sub-block states: about B L D N / 4 + B L (2N + k) D / 16
- *   + 64 B D floats). No pointer may alias another. */
+ *   + 256 B D bytes). No pointer may alias another. */
 swimba_status swimba_scan_bwd(const swimba_dims *dims, const void *x, const void *z,
                               const float *delta, const float *B_mix, const float *C_mix,
                               const int32_t *idx, const float *gates, const swimba_weights *w,
