@@ -55,6 +55,25 @@ def test_workspace_sizes(S):
     assert S.swimba_workspace_size(bad, 4) == 0
 
 
+def test_scan_backward_workspace_holds_its_buffers(S):
+    """The scan backward's workspace: the status block, the state at every 16-token chunk start
+    (B x ceil(L/16) x D x N fp32), the per-64-channel-tile partial rows (dB | dC | dgates), the
+    per-sequence dA and dD partials and the packed kernel's per-CTA sub-block state scratch
+    (16 KB per CTA of 64 channels), each rounded up to 256 bytes."""
+    from parameter_space_moe_swimba_b200.configs import CONFIGS
+
+    up = lambda v: (v + 255) // 256 * 256
+    for name in ("tiny_fp32", "mamba130m_like", "mamba1p4b_like", "long_seq_65536"):
+        cfg = CONFIGS[name]
+        dims = S.make_dims(cfg)
+        B, L, D, N, E, k = cfg.batch, cfg.seqlen, cfg.d_inner, cfg.d_state, cfg.n_experts, cfg.top_k
+        tiles, nck = -(-D // 64), -(-L // 16)
+        need = (up(B * nck * D * N * 4) + up(tiles * B * L * (2 * N + k) * 4) + up(B * E * D * N * 4) +
+                up(B * D * 4) + up(tiles * B * 4 * 2 * 128 * 16))
+        got = S.swimba_workspace_size(dims, S.SWIMBA_OP_SCAN_BWD)
+        assert need <= got <= need + 4096, (name, need, got)
+
+
 def test_invalid_arguments_return_before_any_launch(S):
     from parameter_space_moe_swimba_b200.configs import CONFIGS
 
